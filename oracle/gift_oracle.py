@@ -222,7 +222,8 @@ def jacobi_eigh(B, sweeps: int = 60, tol: float = 1e-15):
                 bpq = B[p, q]
                 if bpq == 0.0:
                     continue
-                theta = (B[q, q] - B[p, p]) / (2.0 * bpq)
+                with np.errstate(over="ignore"):
+                    theta = (B[q, q] - B[p, p]) / (2.0 * bpq)
                 if abs(theta) > 1e150:          # theta^2 would overflow: t ~ 1/(2 theta)
                     t = 0.5 / theta
                 else:
