@@ -314,21 +314,23 @@ def quantize_e4m3_blocks(W, block: int = BLOCK_E4M3):
     """Per-row, per-`block` E4M3 quantisation of W (d_out x d_in).
 
     For each block: amax = max|W| (fp32); scale s = amax/448 (fp32);
-    codes = E4M3_RNE_satfinite(W * fp32(448/amax)).  A block whose amax is 0
-    gets s = 0 and all codes 0x00.
+    codes = E4M3_RNE_satfinite(W * fp32(448/amax)).  A block whose amax is 0,
+    or so small that fp32(448/amax) overflows, is flushed: s = 0 and all
+    codes 0x00.
     """
     W32 = np.asarray(W, dtype=np.float64).astype(_F32)
     d_out, d_in = W32.shape
     nb = d_in // block
     Wb = W32.reshape(d_out, nb, block)
     amax = np.max(np.abs(Wb), axis=2)                       # exact in fp32
-    with np.errstate(divide="ignore"):
-        inv = np.where(amax > 0, _F32(E4M3_MAX) / np.where(amax > 0, amax, _F32(1)), _F32(0))
-    inv = inv.astype(_F32)
-    scales = (amax / _F32(E4M3_MAX)).astype(_F32)
+    with np.errstate(divide="ignore", over="ignore"):
+        inv = (_F32(E4M3_MAX) / np.where(amax > 0, amax, _F32(1))).astype(_F32)
+    live = (amax > 0) & np.isfinite(inv)
+    inv = np.where(live, inv, _F32(0)).astype(_F32)
+    scales = np.where(live, amax / _F32(E4M3_MAX), _F32(0)).astype(_F32)
     y = (Wb * inv[:, :, None]).astype(_F32)
     codes = e4m3_encode(y)
-    codes = np.where((amax > 0)[:, :, None], codes, np.uint8(0)).astype(np.uint8)
+    codes = np.where(live[:, :, None], codes, np.uint8(0)).astype(np.uint8)
     return codes.reshape(d_out, d_in), scales
 
 
@@ -371,7 +373,8 @@ def quantize_nvfp4(W, block: int = BLOCK_NVFP4):
 
     S_t = amax(W) / (6*448); per block b: s_b = E4M3(amax_b / (6*S_t));
     element codes E2M1(W * fp32(1 / (value(s_b) * S_t))); a block whose
-    scale code is zero (or a zero tensor) gets all-zero codes.
+    scale code is zero, or whose reciprocal overflows fp32, gets scale code 0
+    and all-zero element codes.
     Returns (codes packed two per byte, low nibble = even column;
     block scale codes uint8 [d_out, d_in/16]; tensor scale float32).
     """
@@ -390,11 +393,14 @@ def quantize_nvfp4(W, block: int = BLOCK_NVFP4):
     sb = e4m3_encode(ratio)
     sbv = e4m3_decode(sb).astype(_F32)
     dq = (sbv * S_t).astype(_F32)
-    with np.errstate(divide="ignore"):
-        inv = np.where(dq > 0, _F32(1.0) / np.where(dq > 0, dq, _F32(1)), _F32(0)).astype(_F32)
+    with np.errstate(divide="ignore", over="ignore"):
+        inv = (_F32(1.0) / np.where(dq > 0, dq, _F32(1))).astype(_F32)
+    live = (dq > 0) & np.isfinite(inv)
+    inv = np.where(live, inv, _F32(0)).astype(_F32)
+    sb = np.where(live, sb, np.uint8(0)).astype(np.uint8)
     y = (Wb * inv[:, :, None]).astype(_F32)
     q = e2m1_encode(y)
-    q = np.where((dq > 0)[:, :, None], q, np.uint8(0)).reshape(d_out, d_in)
+    q = np.where(live[:, :, None], q, np.uint8(0)).reshape(d_out, d_in)
     packed = (q[:, 0::2] | (q[:, 1::2] << 4)).astype(np.uint8)
     return packed, sb.astype(np.uint8), S_t
 

@@ -176,3 +176,13 @@ def test_fidelity_report_whitened_norm():
     gift_w = O.whitened_error(G, Gh, M)
     eucl_w = O.whitened_error(G, Ge, M)
     assert gift_w < eucl_w
+
+
+def test_block_too_small_for_the_fp32_reciprocal_is_flushed():
+    # 448/amax overflows fp32 for amax below ~1.3e-36: such a block is flushed
+    W = np.zeros((1, 256))
+    W[0, 5] = -2.5e-38          # 448/2.5e-38 = 1.8e40 > FLT_MAX
+    W[0, 130] = 1e-30           # 448/1e-30 = 4.5e32 is representable
+    codes, scales = O.quantize_e4m3_blocks(W)
+    assert scales[0, 0] == 0 and np.all(codes[0, :128] == 0)
+    assert scales[0, 1] == np.float32(1e-30) / np.float32(448) and codes[0, 130] == 0x7E
