@@ -1,0 +1,407 @@
+#!/usr/bin/env python
+"""Benchmark of the GIFT whitened-FP8 gradient codec on B200.
+
+Workload (one step): the Llama-600M-sized stand-in stack of 24 layers x
+{qkv 1536->4608, o 1536->1536, up 1536->4096, down 4096->1536} bf16
+gradients (528.5 M elements, 1.06 GB).  Selective deployment: o and down
+are whitened at rank 32, qkv and up take the Euclidean per-block E4M3
+codec.  A step runs the whole per-step hot path of the paper:
+  * factor refresh of one whitened layer (A = X^T X / N on 8192 tokens,
+    subspace iteration, Rayleigh-Ritz) -- 48 whitened layers refreshed every
+    K = 50 steps (section V.E, Algorithm 1) is ~one refresh per step;
+  * encode of all 96 gradients, then decode of all 96;
+  * the one-step round-trip error of the refreshed layer.
+value = gradient bytes of the stack / step time (GB/s).
+
+Multi-GPU (`--gpus N` under torchrun): replicas only -- the codec has no
+exchange step, so every rank runs its own copy of the stack (weak scaling);
+the timed region is bracketed by barriers and the reported time is the max
+over ranks.
+
+`--impl reference` times the CPU oracle (oracle/gift_oracle.py) on a
+bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "whitened FP8 encode+decode GB/s of gradient and % of B200 HBM roofline"
+UNIT = "GB/s"
+WORKLOAD = ("llama600m-standin stack: 24 x {qkv 4608x1536, o 1536x1536, up 4096x1536, down 1536x4096} "
+            "bf16 gradients; o/down whitened rank 32 (refresh N=8192), qkv/up Euclidean; E4M3 block 128")
+REFRESH_N = 8192
+RANK, OVERSAMPLE, ITERS = 32, 16, 4
+HBM_FALLBACK = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="gift", choices=["gift", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--depth", type=int, default=24, help="layers in the stack (24 = the full stand-in)")
+    return ap.parse_args()
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d.get("hbm_gbs", HBM_FALLBACK), "measured"
+    return HBM_FALLBACK, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        out = {"sm_mhz": None, "sm_max_mhz": None, "reasons": []}
+        if self.proc is None:
+            return out
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        os.unlink(self.path)
+        if sm:
+            out = {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                   "samples": len(sm)}
+        return out
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+def build_workload(torch, ops, synth, dev, depth, seed):
+    """Device-resident stack: G, codes, scales, G_hat in single buffers; per whitened layer X and factors."""
+    shapes = synth.stack_shapes(depth)
+    n_el = sum(d_out * d_in for _, _, d_out, d_in, _ in shapes)
+    G_all = torch.empty((n_el,), device=dev, dtype=torch.bfloat16)
+    Gh_all = torch.empty((n_el,), device=dev, dtype=torch.bfloat16)
+    C_all = torch.empty((n_el,), device=dev, dtype=torch.uint8)
+    S_all = torch.empty((n_el // 128,), device=dev, dtype=torch.float32)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(seed)
+    Qs = {}
+    for d in (1536, 4096):
+        Qs[d] = torch.from_numpy(synth.haar_orthogonal(d, 3000 + d).astype(np.float32)).to(dev)
+    layers, whitened = [], []
+    off = 0
+    for (l, name, d_out, d_in, wh) in shapes:
+        n = d_out * d_in
+        G = G_all[off:off + n].view(d_out, d_in)
+        G.copy_(synth.device_gradient(d_out, d_in, 1.0, Qs[d_in], gen, torch.bfloat16))
+        L = ops.LayerArgs(d_out=d_out, d_in=d_in, rank=RANK if wh else 0, dtype=torch.bfloat16, G=G,
+                          G_hat=Gh_all[off:off + n].view(d_out, d_in), codes=C_all[off:off + n].view(d_out, d_in),
+                          scales=S_all[off // 128:(off + n) // 128].view(d_out, d_in // 128))
+        if wh:
+            sigma = torch.arange(1, d_in + 1, device=dev, dtype=torch.float32) ** -1.0
+            X = synth.device_activations(REFRESH_N, sigma, Qs[d_in], gen, torch.bfloat16)
+            L.U = torch.empty((d_in, RANK), device=dev, dtype=torch.float32)
+            L.lam = torch.empty((RANK,), device=dev, dtype=torch.float32)
+            L.rho = torch.empty((1,), device=dev, dtype=torch.float32)
+            ws = torch.empty((ops.refresh_workspace_size(REFRESH_N, d_in, RANK, OVERSAMPLE),), device=dev,
+                             dtype=torch.uint8)
+            st = torch.zeros((1,), device=dev, dtype=torch.int32)
+            whitened.append(dict(layer=L, X=X, ws=ws, st=st, seed=7000 + len(whitened)))
+        layers.append(L)
+        off += n
+    ews = torch.empty((max(ops.error_workspace_size(4096, 4096), 16),), device=dev, dtype=torch.uint8)
+    err = torch.empty((3,), device=dev, dtype=torch.float64)
+    return dict(layers=layers, whitened=whitened, G_all=G_all, Gh_all=Gh_all, C_all=C_all, S_all=S_all,
+                n_el=n_el, packed=ops.make_layers(layers), ews=ews, err=err)
+
+
+def refresh(ops, w, stream=None):
+    L = w["layer"]
+    ops.factor_refresh(w["X"], RANK, OVERSAMPLE, ITERS, w["seed"], ws=w["ws"], dev_status=w["st"],
+                       out=(L.U, L.lam, L.rho), stream=stream)
+
+
+def step(ops, W, k, ev=None):
+    """One step; if `ev` (list of 5 events) is given, phase boundaries are recorded."""
+    w = W["whitened"][k % len(W["whitened"])]
+    if ev:
+        ev[0].record()
+    refresh(ops, w)
+    if ev:
+        ev[1].record()
+    ops.encode_many(W["packed"], len(W["layers"]))
+    if ev:
+        ev[2].record()
+    ops.decode_many(W["packed"], len(W["layers"]))
+    if ev:
+        ev[3].record()
+    L = w["layer"]
+    ops.roundtrip_error(L.G, L.G_hat, out=W["err"], ws=W["ews"])
+    if ev:
+        ev[4].record()
+
+
+def algorithmic_bytes(W):
+    """Per step: encode reads G (2 B) and writes codes (1 B) + scales (4/128 B); decode the reverse."""
+    n = W["n_el"]
+    return n * (2 + 1 + 4 / 128), n * (1 + 4 / 128 + 2)
+
+
+def count_launches(torch, ops, W):
+    """Kernels of libgift launched by one step, counted with the CUDA profiler (untimed pass)."""
+    try:
+        from torch.profiler import ProfilerActivity, profile
+        with profile(activities=[ProfilerActivity.CUDA]) as prof:
+            step(ops, W, 0)
+            torch.cuda.synchronize()
+        names = [e.name for e in prof.events() if e.device_type.name == "CUDA"]
+        return sum(1 for n in names if "gift" in n), sorted(set(n for n in names if "gift" in n))
+    except Exception as e:  # pragma: no cover
+        return None, [f"profiler unavailable: {e}"]
+
+
+def cpu_baseline(sample_seconds=12.0):
+    """The oracle as it stands on the host cores: bounded sample of the same workload."""
+    from oracle import gift_oracle as O
+    from geometry_aware_fp8_b200 import synth
+    t_end = time.time() + sample_seconds
+    nbytes, t_used, reps = 0, 0.0, 0
+    Q = synth.haar_orthogonal(1536, 11)
+    X = synth.to_storage(synth.activations(REFRESH_N, Q, synth.column_power(1536, 1.0), 12), "bf16")
+    Go = synth.to_storage(synth.gradient(1536, Q, 1.0, 13), "bf16")
+    Gq = synth.to_storage(synth.gradient(4608, Q, 1.0, 14), "bf16")
+    while time.time() < t_end or reps == 0:
+        t0 = time.perf_counter()
+        A = O.input_factor(X)
+        U, lam, rho, _ = O.factor_refresh(A, RANK, OVERSAMPLE, ITERS, seed=reps)
+        c, s = O.encode_e4m3(Go, U, lam, rho)
+        Gh = O.bf16_round(O.decode_e4m3(c, s, U, lam, rho))
+        O.roundtrip_error(Go, Gh)
+        c2, s2 = O.quantize_e4m3_blocks(Gq)
+        O.bf16_round(O.dequantize_e4m3_blocks(c2, s2))
+        t_used += time.perf_counter() - t0
+        nbytes += 2 * (Go.size + Gq.size)
+        reps += 1
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count()
+    return {"value": nbytes / t_used / 1e9, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": (f"{reps} x [o-projection 1536x1536 bf16: refresh from X 8192x1536 + whitened encode + "
+                       f"decode + error; qkv 4608x1536 Euclidean encode + decode], {t_used:.1f} s"),
+            "host_cpus": os.cpu_count()}
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+    from geometry_aware_fp8_b200 import ops, synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.warmup < 3:
+        args.warmup = 3
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    W = build_workload(torch, ops, synth, dev, args.depth, seed=1234 + rank)
+    for w in W["whitened"]:
+        refresh(ops, w)
+    torch.cuda.synchronize()
+
+    for k in range(args.warmup):
+        step(ops, W, k)
+    torch.cuda.synchronize()
+
+    # ---- timed region: device resident inputs (1.06 GB of G > 126 MB L2) ----
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+    clocks = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for k in range(K):
+        step(ops, W, k, evs[k])
+    t1.record()
+    torch.cuda.synchronize()
+    barrier()
+    clock_info = clocks.stop()
+    ms_total = t0.elapsed_time(t1)
+    phase = np.array([[e[i].elapsed_time(e[i + 1]) for i in range(4)] for e in evs])  # refresh, enc, dec, err
+    if world > 1:
+        t = torch.tensor([ms_total], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = t.item()
+    ms_step = ms_total / K
+    g_bytes = W["n_el"] * 2
+    value = world * g_bytes / (ms_step * 1e-3) / 1e9
+
+    enc_b, dec_b = algorithmic_bytes(W)
+    enc_ms, dec_ms = phase[:, 1].mean(), phase[:, 2].mean()
+    peak, peak_kind = measured_peaks()
+    dom = "encode" if enc_ms >= dec_ms else "decode"
+    dom_ms = max(enc_ms, dec_ms)
+    dom_b = enc_b if dom == "encode" else dec_b
+    achieved = dom_b / (dom_ms * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "kernel": f"grouped {dom} over the 96-tensor stack", "achieved": achieved,
+                "peak": peak, "peak_source": peak_kind, "unit": "GB/s", "frac": achieved / peak, "traffic": None}
+    codec_ms = enc_ms + dec_ms
+    codec = {"encode_ms": enc_ms, "decode_ms": dec_ms, "refresh_ms": phase[:, 0].mean(),
+             "error_ms": phase[:, 3].mean(),
+             "codec_gradient_gbs": g_bytes / (codec_ms * 1e-3) / 1e9,
+             "codec_roofline_frac": (enc_b + dec_b) / (codec_ms * 1e-3) / 1e9 / peak}
+
+    launches, names = count_launches(torch, ops, W)
+
+    # ---- end to end through host buffers ----
+    e2e = None
+    if not args.no_e2e:
+        G_host = torch.empty((W["n_el"],), dtype=torch.bfloat16, pin_memory=True)
+        G_host.copy_(W["G_all"].cpu())
+        Gh_host = torch.empty_like(G_host, pin_memory=True)
+        X_host = {id(w): w["X"].cpu().pin_memory() for w in W["whitened"][:2]}
+        err_host = torch.empty((3,), dtype=torch.float64, pin_memory=True)
+        Ke = max(3, min(K, 10))
+
+        def e2e_step(k):
+            w = W["whitened"][k % 2]
+            W["G_all"].copy_(G_host, non_blocking=True)
+            w["X"].copy_(X_host[id(w)], non_blocking=True)
+            step(ops, W, k % 2)
+            Gh_host.copy_(W["Gh_all"], non_blocking=True)
+            err_host.copy_(W["err"], non_blocking=True)
+
+        e2e_step(0)
+        torch.cuda.synchronize()
+        barrier()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        for k in range(Ke):
+            e2e_step(k)
+        b.record()
+        torch.cuda.synchronize()
+        ms_e = a.elapsed_time(b)
+        if world > 1:
+            t = torch.tensor([ms_e], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms_e = t.item()
+        x_bytes = sum(W["whitened"][k % 2]["X"].numel() * 2 for k in range(Ke)) / Ke
+        e2e = {"value": world * g_bytes / (ms_e / Ke * 1e-3) / 1e9, "unit": UNIT,
+               "h2d_bytes_per_step": int(g_bytes + x_bytes), "d2h_bytes_per_step": int(g_bytes + 24),
+               "ms_per_step": ms_e / Ke}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline()
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+                "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "f32", "data": "synthetic",
+                "config": {"workload": WORKLOAD, "depth": args.depth, "gradient_elements": W["n_el"],
+                           "gradient_bytes": g_bytes, "storage": "bf16 G / e4m3 codes / fp32 scales",
+                           "l2": "inputs larger than L2 (1.06 GB of gradients streamed per step)",
+                           "parallelism": f"replicas x{world}"},
+                "roofline": roofline, "codec": codec, "e2e": e2e, "cpu_baseline": cpu,
+                "gpu_launches": launches, "kernels": names, "clocks": clock_info}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the CPU oracle on the host cores
+# ---------------------------------------------------------------------------
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    warm = max(args.warmup, 0)
+    for _ in range(min(warm, 2)):
+        cpu_baseline(sample_seconds=0.0)
+    vals = []
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        r = cpu_baseline(sample_seconds=0.0)
+        vals.append(r["value"])
+    wall = time.perf_counter() - t0
+    v = float(statistics.mean(vals))
+    cpu = dict(r, value=v)
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": 0, "steps": args.steps,
+            "warmup": warm, "ms_per_step": wall / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "sample": cpu["sample"]},
+            "cpu_baseline": cpu, "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    a = parse()
+    if a.impl == "reference":
+        run_reference(a)
+    else:
+        run_gpu(a)

@@ -1,0 +1,220 @@
+// C-ABI entry points of libgift (declared in include/gift.h).
+//
+// Each entry point validates every argument on the host first and returns a
+// status before touching CUDA, so argument errors are reported identically
+// with or without a GPU.  Only then does it check the device (sm_100) and
+// enqueue kernels on the caller's stream.  Nothing here allocates device
+// memory; scratch space comes from the caller's workspace.
+#include <cstdio>
+#include <mutex>
+#include <vector>
+
+#include "common.cuh"
+#include "internal.h"
+
+using namespace gift;
+
+namespace {
+
+inline bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+inline bool aligned(const void* p, size_t a) { return ((uintptr_t)p & (a - 1)) == 0; }
+inline bool dtype_ok(int d) { return d == GIFT_F32 || d == GIFT_BF16; }
+
+constexpr int kMaxDevices = 64;
+
+// sm_100 check, cached per device (the only state the library keeps).
+gift_status device_ok() {
+  static int major_cache[kMaxDevices];
+  static std::once_flag once;
+  std::call_once(once, [] {
+    for (int i = 0; i < kMaxDevices; ++i) major_cache[i] = -1;
+  });
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return GIFT_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return GIFT_ERR_UNSUPPORTED;
+  int major = major_cache[dev];
+  if (major < 0) {
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return GIFT_ERR_CUDA;
+    major_cache[dev] = major;
+  }
+  return major == 10 ? GIFT_OK : GIFT_ERR_UNSUPPORTED;
+}
+
+inline gift_status cuda_status(cudaError_t e) { return e == cudaSuccess ? GIFT_OK : GIFT_ERR_CUDA; }
+
+gift_status check_codec_args(const void* G, int gdt, int64_t d_out, int64_t d_in, const float* U,
+                             const float* lambda, const float* rho, int rank, const void* codes, const float* scales) {
+  if (!G || !codes || !scales) return GIFT_ERR_INVALID_ARG;
+  if (!dtype_ok(gdt)) return GIFT_ERR_INVALID_ARG;
+  if (d_out < 0 || d_in <= 0) return GIFT_ERR_INVALID_ARG;
+  if (d_in % GIFT_E4M3_BLOCK != 0) return GIFT_ERR_SHAPE;
+  if (d_in > (1 << 20) || d_out > ((int64_t)1 << 31)) return GIFT_ERR_SHAPE;
+  if (rank < 0 || rank > GIFT_MAX_RANK) return GIFT_ERR_SHAPE;
+  if (rank > 0 && (!U || !lambda || !rho)) return GIFT_ERR_INVALID_ARG;
+  if (!aligned16(G) || !aligned16(codes) || !aligned16(scales)) return GIFT_ERR_ALIGN;
+  if (rank > 0 && (!aligned16(U) || !aligned(lambda, 4) || !aligned(rho, 4))) return GIFT_ERR_ALIGN;
+  return GIFT_OK;
+}
+
+// Whitened bf16 layers with rank 32 go to the tensor-core kernels when they
+// are built in; everything else runs on the CUDA-core kernels.
+inline bool use_tc(int dt, int rank, int64_t d_in) {
+  return dt == GIFT_BF16 && rank > 0 && tc_codec_available() && d_in <= 8192;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* gift_status_string(gift_status s) {
+  switch (s) {
+    case GIFT_OK: return "GIFT_OK";
+    case GIFT_ERR_INVALID_ARG: return "GIFT_ERR_INVALID_ARG: null pointer, bad enum or bad size";
+    case GIFT_ERR_SHAPE: return "GIFT_ERR_SHAPE: unsupported shape or rank";
+    case GIFT_ERR_ALIGN: return "GIFT_ERR_ALIGN: pointer not 16-byte aligned";
+    case GIFT_ERR_WORKSPACE: return "GIFT_ERR_WORKSPACE: workspace missing or too small";
+    case GIFT_ERR_CUDA: return "GIFT_ERR_CUDA: CUDA runtime or launch failure";
+    case GIFT_ERR_UNSUPPORTED: return "GIFT_ERR_UNSUPPORTED: device is not sm_100";
+  }
+  return "GIFT_ERR_UNKNOWN";
+}
+
+int gift_version(void) { return 100; }
+
+// ---------------------------------------------------------------------------
+gift_status gift_refresh_workspace_size(int64_t N, int64_t d_in, int rank, int oversample, int a_out_given,
+                                        size_t* bytes) {
+  if (!bytes) return GIFT_ERR_INVALID_ARG;
+  if (N < 1 || d_in <= 0 || rank < 1 || oversample < 0) return GIFT_ERR_INVALID_ARG;
+  if (d_in % GIFT_E4M3_BLOCK != 0 || d_in > 32768) return GIFT_ERR_SHAPE;
+  if (rank + oversample > GIFT_MAX_SUBSPACE || rank + oversample > d_in) return GIFT_ERR_SHAPE;
+  RefreshPlan p;
+  refresh_plan(N, d_in, rank, oversample, a_out_given != 0, &p);
+  *bytes = p.total;
+  return GIFT_OK;
+}
+
+gift_status gift_factor_refresh(const void* X, gift_dtype xdt, int64_t N, int64_t d_in, int rank, int oversample,
+                                int iters, uint64_t seed, float* U, float* lambda, float* rho, float* A_out,
+                                void* ws, size_t ws_bytes, uint32_t* dev_status, gift_stream_t stream) {
+  if (!X || !U || !lambda || !rho) return GIFT_ERR_INVALID_ARG;
+  if (!dtype_ok(xdt)) return GIFT_ERR_INVALID_ARG;
+  if (iters < 0 || iters > 1000) return GIFT_ERR_INVALID_ARG;
+  size_t need = 0;
+  gift_status st = gift_refresh_workspace_size(N, d_in, rank, oversample, A_out != nullptr, &need);
+  if (st != GIFT_OK) return st;
+  if (need > 0 && (!ws || ws_bytes < need)) return GIFT_ERR_WORKSPACE;
+  if (!aligned16(X) || !aligned16(U) || !aligned(lambda, 4) || !aligned(rho, 4)) return GIFT_ERR_ALIGN;
+  if ((A_out && !aligned16(A_out)) || (ws && !aligned16(ws)) || (dev_status && !aligned(dev_status, 4)))
+    return GIFT_ERR_ALIGN;
+  if ((st = device_ok()) != GIFT_OK) return st;
+  RefreshPlan p;
+  refresh_plan(N, d_in, rank, oversample, A_out != nullptr, &p);
+  p.iters = iters;
+  p.seed = seed;
+  return cuda_status(launch_refresh(p, X, xdt, U, lambda, rho, A_out, ws, dev_status, (cudaStream_t)stream));
+}
+
+// ---------------------------------------------------------------------------
+gift_status gift_encode(const void* G, gift_dtype gdt, int64_t d_out, int64_t d_in, const float* U,
+                        const float* lambda, const float* rho, int rank, uint8_t* codes, float* scales,
+                        gift_stream_t stream) {
+  gift_status st = check_codec_args(G, gdt, d_out, d_in, U, lambda, rho, rank, codes, scales);
+  if (st != GIFT_OK) return st;
+  if (d_out == 0) return GIFT_OK;
+  if ((st = device_ok()) != GIFT_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (rank == 0) return cuda_status(launch_euclid_encode(G, gdt, d_out * (d_in / GIFT_E4M3_BLOCK), codes, scales, s));
+  if (use_tc(gdt, rank, d_in)) {
+    TcLayer L{G, nullptr, codes, scales, U, lambda, rho, (int)d_out, (int)d_in, rank};
+    return cuda_status(launch_whiten_encode_tc(&L, 1, s));
+  }
+  return cuda_status(launch_whiten_encode_simt(G, gdt, d_out, d_in, U, lambda, rho, rank, codes, scales, s));
+}
+
+gift_status gift_decode(const uint8_t* codes, const float* scales, int64_t d_out, int64_t d_in, const float* U,
+                        const float* lambda, const float* rho, int rank, void* G_hat, gift_dtype out_dt,
+                        gift_stream_t stream) {
+  gift_status st = check_codec_args(G_hat, out_dt, d_out, d_in, U, lambda, rho, rank, codes, scales);
+  if (st != GIFT_OK) return st;
+  if (d_out == 0) return GIFT_OK;
+  if ((st = device_ok()) != GIFT_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (rank == 0)
+    return cuda_status(launch_euclid_decode(codes, scales, d_out * (d_in / GIFT_E4M3_BLOCK), G_hat, out_dt, s));
+  if (use_tc(out_dt, rank, d_in)) {
+    TcLayer L{nullptr, G_hat, (uint8_t*)codes, (float*)scales, U, lambda, rho, (int)d_out, (int)d_in, rank};
+    return cuda_status(launch_whiten_decode_tc(&L, 1, s));
+  }
+  return cuda_status(launch_whiten_decode_simt(codes, scales, d_out, d_in, U, lambda, rho, rank, G_hat, out_dt, s));
+}
+
+// ---------------------------------------------------------------------------
+static gift_status run_many(const gift_layer* layers, int n, gift_stream_t stream, bool encode) {
+  if (n < 0 || (n > 0 && !layers)) return GIFT_ERR_INVALID_ARG;
+  for (int i = 0; i < n; ++i) {
+    const gift_layer& L = layers[i];
+    const void* g = encode ? L.G : (const void*)L.G_hat;
+    gift_status st = check_codec_args(g, L.dtype, L.d_out, L.d_in, L.U, L.lambda, L.rho, L.rank, L.codes, L.scales);
+    if (st != GIFT_OK) return st;
+  }
+  if (n == 0) return GIFT_OK;
+  gift_status st = device_ok();
+  if (st != GIFT_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  std::vector<TcLayer> tc;
+  for (int i = 0; i < n; ++i) {
+    const gift_layer& L = layers[i];
+    if (L.d_out == 0) continue;
+    cudaError_t e = cudaSuccess;
+    const int64_t nb = L.d_out * (L.d_in / GIFT_E4M3_BLOCK);
+    if (L.rank == 0) {
+      e = encode ? launch_euclid_encode(L.G, (gift_dtype)L.dtype, nb, L.codes, L.scales, s)
+                 : launch_euclid_decode(L.codes, L.scales, nb, L.G_hat, (gift_dtype)L.dtype, s);
+    } else if (use_tc(L.dtype, L.rank, L.d_in)) {
+      tc.push_back(TcLayer{L.G, L.G_hat, L.codes, L.scales, L.U, L.lambda, L.rho, (int)L.d_out, (int)L.d_in, L.rank});
+    } else {
+      e = encode ? launch_whiten_encode_simt(L.G, (gift_dtype)L.dtype, L.d_out, L.d_in, L.U, L.lambda, L.rho, L.rank,
+                                             L.codes, L.scales, s)
+                 : launch_whiten_decode_simt(L.codes, L.scales, L.d_out, L.d_in, L.U, L.lambda, L.rho, L.rank,
+                                             L.G_hat, (gift_dtype)L.dtype, s);
+    }
+    if (e != cudaSuccess) return GIFT_ERR_CUDA;
+  }
+  if (!tc.empty()) {
+    cudaError_t e = encode ? launch_whiten_encode_tc(tc.data(), (int)tc.size(), s)
+                           : launch_whiten_decode_tc(tc.data(), (int)tc.size(), s);
+    if (e != cudaSuccess) return GIFT_ERR_CUDA;
+  }
+  return GIFT_OK;
+}
+
+gift_status gift_encode_many(const gift_layer* layers, int n, gift_stream_t stream) {
+  return run_many(layers, n, stream, true);
+}
+gift_status gift_decode_many(const gift_layer* layers, int n, gift_stream_t stream) {
+  return run_many(layers, n, stream, false);
+}
+
+// ---------------------------------------------------------------------------
+gift_status gift_error_workspace_size(int64_t d_out, int64_t d_in, size_t* bytes) {
+  if (!bytes || d_out < 1 || d_in < 1) return GIFT_ERR_INVALID_ARG;
+  if (d_in % GIFT_E4M3_BLOCK != 0) return GIFT_ERR_SHAPE;
+  *bytes = error_ws_bytes(d_out * d_in);
+  return GIFT_OK;
+}
+
+gift_status gift_roundtrip_error(const void* G, const void* G_hat, gift_dtype dt, int64_t d_out, int64_t d_in,
+                                 double* out, void* ws, size_t ws_bytes, gift_stream_t stream) {
+  if (!G || !G_hat || !out) return GIFT_ERR_INVALID_ARG;
+  if (!dtype_ok(dt)) return GIFT_ERR_INVALID_ARG;
+  size_t need = 0;
+  gift_status st = gift_error_workspace_size(d_out, d_in, &need);
+  if (st != GIFT_OK) return st;
+  if (!ws || ws_bytes < need) return GIFT_ERR_WORKSPACE;
+  if (!aligned16(G) || !aligned16(G_hat) || !aligned(out, 8) || !aligned16(ws)) return GIFT_ERR_ALIGN;
+  if ((st = device_ok()) != GIFT_OK) return st;
+  return cuda_status(launch_roundtrip_error(G, G_hat, dt, d_out * d_in, out, ws, (cudaStream_t)stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,158 @@
+// Euclidean per-block E4M3 codec (M = I): the comparison arm of the GIFT
+// round-trip study (Tables I-II) and the path of every layer that the
+// selective deployment leaves unwhitened (section V.C, Fig. 4).
+//
+// Pure streaming work, bound by HBM: 2 (bf16) or 4 (fp32) bytes in, 1 byte
+// plus 4/128 bytes out per element.  Eight threads own one 128-element block
+// (16 elements each, 16-byte vector loads and one 16-byte code store), the
+// block maximum is three xor-shuffles, and the grid is a multiple of the SM
+// count that strides over all blocks.
+#include "common.cuh"
+#include "internal.h"
+
+namespace gift {
+namespace {
+
+template <typename T>
+struct Vec16;  // 16 consecutive elements loaded with 16-byte loads
+
+template <>
+struct Vec16<__nv_bfloat16> {
+  static GIFT_DEV void load(const __nv_bfloat16* p, float (&v)[16]) {
+    const uint4* q = reinterpret_cast<const uint4*>(p);
+    uint4 a = __ldcs(q), b = __ldcs(q + 1);
+    uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      v[2 * i] = bf16lo(w[i]);
+      v[2 * i + 1] = bf16hi(w[i]);
+    }
+  }
+  static GIFT_DEV void store(__nv_bfloat16* p, const float (&v)[16]) {
+    uint32_t w[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) w[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+    uint4* q = reinterpret_cast<uint4*>(p);
+    __stcs(q, make_uint4(w[0], w[1], w[2], w[3]));
+    __stcs(q + 1, make_uint4(w[4], w[5], w[6], w[7]));
+  }
+};
+
+template <>
+struct Vec16<float> {
+  static GIFT_DEV void load(const float* p, float (&v)[16]) {
+    const float4* q = reinterpret_cast<const float4*>(p);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float4 f = __ldcs(q + i);
+      v[4 * i] = f.x;
+      v[4 * i + 1] = f.y;
+      v[4 * i + 2] = f.z;
+      v[4 * i + 3] = f.w;
+    }
+  }
+  static GIFT_DEV void store(float* p, const float (&v)[16]) {
+    float4* q = reinterpret_cast<float4*>(p);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) __stcs(q + i, make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]));
+  }
+};
+
+// Quantise 16 values of one block given its reciprocal scale; returns the codes packed in a uint4.
+GIFT_DEV uint4 quantize16(const float (&v)[16], float inv) {
+  uint32_t w[4];
+  if (inv > 0.0f) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      uint32_t lo = f32x2_to_e4m3x2(__fmul_rn(v[4 * i], inv), __fmul_rn(v[4 * i + 1], inv));
+      uint32_t hi = f32x2_to_e4m3x2(__fmul_rn(v[4 * i + 2], inv), __fmul_rn(v[4 * i + 3], inv));
+      w[i] = lo | (hi << 16);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) w[i] = 0u;
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) euclid_encode_kernel(const T* __restrict__ G, uint8_t* __restrict__ codes,
+                                                            float* __restrict__ scales, int64_t n_blocks) {
+  const int sub = threadIdx.x & 7;
+  const int64_t groups_per_grid = (int64_t)gridDim.x * (blockDim.x >> 3);
+  for (int64_t b = (int64_t)blockIdx.x * (blockDim.x >> 3) + (threadIdx.x >> 3); b < n_blocks;
+       b += groups_per_grid) {
+    const int64_t e0 = b * kBlock + sub * 16;
+    float v[16];
+    Vec16<T>::load(G + e0, v);
+    float m = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[i]));
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+    const float inv = e4m3_inv_scale(m);
+    __stcs(reinterpret_cast<uint4*>(codes + e0), quantize16(v, inv));
+    if (sub == 0) scales[b] = e4m3_scale(m, inv);
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) euclid_decode_kernel(const uint8_t* __restrict__ codes,
+                                                            const float* __restrict__ scales, T* __restrict__ out,
+                                                            int64_t n_blocks) {
+  const int sub = threadIdx.x & 7;
+  const int64_t groups_per_grid = (int64_t)gridDim.x * (blockDim.x >> 3);
+  for (int64_t b = (int64_t)blockIdx.x * (blockDim.x >> 3) + (threadIdx.x >> 3); b < n_blocks;
+       b += groups_per_grid) {
+    const int64_t e0 = b * kBlock + sub * 16;
+    const uint4 q = __ldcs(reinterpret_cast<const uint4*>(codes + e0));
+    const float s = __ldg(scales + b);
+    uint32_t w[4] = {q.x, q.y, q.z, q.w};
+    float v[16];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float2 a = e4m3x2_to_f32x2((uint16_t)(w[i] & 0xFFFF));
+      float2 c = e4m3x2_to_f32x2((uint16_t)(w[i] >> 16));
+      v[4 * i] = a.x * s;
+      v[4 * i + 1] = a.y * s;
+      v[4 * i + 2] = c.x * s;
+      v[4 * i + 3] = c.y * s;
+    }
+    Vec16<T>::store(out + e0, v);
+  }
+}
+
+inline int grid_for(int64_t n_blocks) {
+  // 8 blocks per 256-thread CTA; up to 8 resident CTAs per SM.
+  int64_t need = (n_blocks + 31) / 32;  // four blocks of work per group
+  int64_t cap = (int64_t)kNumSMs * 8;
+  if (need < 1) need = 1;
+  return (int)(need < cap ? need : cap);
+}
+
+}  // namespace
+
+cudaError_t launch_euclid_encode(const void* G, gift_dtype dt, int64_t n_blocks, uint8_t* codes, float* scales,
+                                 cudaStream_t s) {
+  if (n_blocks == 0) return cudaSuccess;
+  const int grid = grid_for(n_blocks);
+  if (dt == GIFT_BF16)
+    euclid_encode_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>((const __nv_bfloat16*)G, codes, scales, n_blocks);
+  else
+    euclid_encode_kernel<float><<<grid, 256, 0, s>>>((const float*)G, codes, scales, n_blocks);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_euclid_decode(const uint8_t* codes, const float* scales, int64_t n_blocks, void* G_hat,
+                                 gift_dtype dt, cudaStream_t s) {
+  if (n_blocks == 0) return cudaSuccess;
+  const int grid = grid_for(n_blocks);
+  if (dt == GIFT_BF16)
+    euclid_decode_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(codes, scales, (__nv_bfloat16*)G_hat, n_blocks);
+  else
+    euclid_decode_kernel<float><<<grid, 256, 0, s>>>(codes, scales, (float*)G_hat, n_blocks);
+  return cudaGetLastError();
+}
+
+}  // namespace gift

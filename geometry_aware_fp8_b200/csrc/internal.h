@@ -1,0 +1,64 @@
+// Internal launch interface between the C-ABI layer (abi.cu) and the kernel
+// files.  Every launcher enqueues work on `stream` and returns the launch
+// error (cudaSuccess when the launch was accepted).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/gift.h"
+
+namespace gift {
+
+// ---- Euclidean per-block E4M3 codec (rank 0): flat arrays of n_blocks*128 ----
+cudaError_t launch_euclid_encode(const void* G, gift_dtype dt, int64_t n_blocks, uint8_t* codes,
+                                 float* scales, cudaStream_t s);
+cudaError_t launch_euclid_decode(const uint8_t* codes, const float* scales, int64_t n_blocks, void* G_hat,
+                                 gift_dtype dt, cudaStream_t s);
+
+// ---- Whitened codec on CUDA cores (any rank <= 32, fp32 or bf16) ----
+cudaError_t launch_whiten_encode_simt(const void* G, gift_dtype dt, int64_t d_out, int64_t d_in, const float* U,
+                                      const float* lambda, const float* rho, int rank, uint8_t* codes,
+                                      float* scales, cudaStream_t s);
+cudaError_t launch_whiten_decode_simt(const uint8_t* codes, const float* scales, int64_t d_out, int64_t d_in,
+                                      const float* U, const float* lambda, const float* rho, int rank,
+                                      void* G_hat, gift_dtype dt, cudaStream_t s);
+
+// ---- Whitened codec on the tensor cores (bf16 G, tcgen05 + TMA) ----
+struct TcLayer {
+  const void* G;      // bf16 d_out x d_in (encode input)
+  void* G_hat;        // bf16 d_out x d_in (decode output)
+  uint8_t* codes;
+  float* scales;
+  const float* U;
+  const float* lambda;
+  const float* rho;
+  int d_out;
+  int d_in;
+  int rank;
+};
+bool tc_codec_available();
+cudaError_t launch_whiten_encode_tc(const TcLayer* layers, int n, cudaStream_t s);
+cudaError_t launch_whiten_decode_tc(const TcLayer* layers, int n, cudaStream_t s);
+
+// ---- Round-trip error ----
+size_t error_ws_bytes(int64_t n_elems);
+cudaError_t launch_roundtrip_error(const void* G, const void* G_hat, gift_dtype dt, int64_t n_elems,
+                                   double* out, void* ws, cudaStream_t s);
+
+// ---- Factor refresh ----
+struct RefreshPlan {
+  int64_t N, d;
+  int rank, m;          // m = rank + oversample
+  int iters;
+  uint64_t seed;
+  int gram_parts;       // partial Gram blocks
+  int syrk_splits;      // split-K partial sums of A
+  // workspace carve-up (byte offsets from ws)
+  size_t off_A, off_Q, off_Y, off_gram, off_small, off_syrk, total;
+};
+void refresh_plan(int64_t N, int64_t d, int rank, int oversample, bool a_out_given, RefreshPlan* p);
+cudaError_t launch_refresh(const RefreshPlan& p, const void* X, gift_dtype xdt, float* U, float* lambda,
+                           float* rho, float* A_out, void* ws, uint32_t* dev_status, cudaStream_t s);
+
+}  // namespace gift

@@ -1,0 +1,224 @@
+"""ctypes binding of libgift (include/gift.h): argument marshalling only.
+
+Every function here checks tensor placement/dtype, allocates missing outputs
+with torch (device memory is torch's job), passes raw pointers and the
+current CUDA stream to the C ABI, and raises GiftError on a non-OK status.
+No step of the codec is computed here; if libgift.so is missing every call
+raises instead of falling back to anything else.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional, Sequence
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgift.so")
+
+GIFT_F32, GIFT_BF16 = 0, 1
+E4M3_BLOCK = 128
+DEV_RHO_FLOORED, DEV_RANK_DEFICIENT, DEV_NONFINITE = 0x1, 0x2, 0x4
+STATUS = {0: "GIFT_OK", 1: "GIFT_ERR_INVALID_ARG", 2: "GIFT_ERR_SHAPE", 3: "GIFT_ERR_ALIGN",
+          4: "GIFT_ERR_WORKSPACE", 5: "GIFT_ERR_CUDA", 6: "GIFT_ERR_UNSUPPORTED"}
+
+EXPORTED = ("gift_status_string", "gift_version", "gift_refresh_workspace_size", "gift_factor_refresh",
+            "gift_encode", "gift_decode", "gift_encode_many", "gift_decode_many",
+            "gift_error_workspace_size", "gift_roundtrip_error")
+
+
+class GiftError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)}")
+
+
+class Layer(ctypes.Structure):
+    """Mirror of gift_layer."""
+    _fields_ = [("G", ctypes.c_void_p), ("G_hat", ctypes.c_void_p), ("codes", ctypes.c_void_p),
+                ("scales", ctypes.c_void_p), ("U", ctypes.c_void_p), ("lambda_", ctypes.c_void_p),
+                ("rho", ctypes.c_void_p), ("d_out", ctypes.c_int64), ("d_in", ctypes.c_int64),
+                ("rank", ctypes.c_int32), ("dtype", ctypes.c_int32)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Open libgift.so once; raise if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m geometry_aware_fp8_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+        L.gift_status_string.restype = ctypes.c_char_p
+        L.gift_status_string.argtypes = [i32]
+        L.gift_version.restype = i32
+        L.gift_refresh_workspace_size.argtypes = [i64, i64, i32, i32, i32, ctypes.POINTER(sz)]
+        L.gift_factor_refresh.argtypes = [vp, i32, i64, i64, i32, i32, i32, ctypes.c_uint64, vp, vp, vp, vp,
+                                          vp, sz, vp, vp]
+        L.gift_encode.argtypes = [vp, i32, i64, i64, vp, vp, vp, i32, vp, vp, vp]
+        L.gift_decode.argtypes = [vp, vp, i64, i64, vp, vp, vp, i32, vp, i32, vp]
+        L.gift_encode_many.argtypes = [ctypes.POINTER(Layer), i32, vp]
+        L.gift_decode_many.argtypes = [ctypes.POINTER(Layer), i32, vp]
+        L.gift_error_workspace_size.argtypes = [i64, i64, ctypes.POINTER(sz)]
+        L.gift_roundtrip_error.argtypes = [vp, vp, i32, i64, i64, vp, vp, sz, vp]
+        for name in EXPORTED:
+            if name not in ("gift_status_string", "gift_version"):
+                getattr(L, name).restype = i32
+        _lib = L
+    return _lib
+
+
+def _check(st: int, where: str):
+    if st != 0:
+        raise GiftError(st, where)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return GIFT_BF16
+    if t.dtype == torch.float32:
+        return GIFT_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _cuda(*ts):
+    for t in ts:
+        if t is not None:
+            if not t.is_cuda:
+                raise ValueError("tensor must live on a CUDA device")
+            if not t.is_contiguous():
+                raise ValueError("tensor must be contiguous")
+
+
+# ---------------------------------------------------------------------------
+def refresh_workspace_size(N: int, d_in: int, rank: int = 32, oversample: int = 16,
+                           a_out_given: bool = False) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().gift_refresh_workspace_size(N, d_in, rank, oversample, int(a_out_given), ctypes.byref(n)),
+           "gift_refresh_workspace_size")
+    return n.value
+
+
+def factor_refresh(X: torch.Tensor, rank: int = 32, oversample: int = 16, iters: int = 4, seed: int = 0,
+                   A_out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+                   dev_status: Optional[torch.Tensor] = None, stream=None, out=None):
+    """(U, lambda, rho, dev_status) of the input factor A = X^T X / N (see gift_factor_refresh)."""
+    _cuda(X, A_out, ws, dev_status)
+    N, d = X.shape
+    dev = X.device
+    if out is None:
+        U = torch.empty((d, rank), device=dev, dtype=torch.float32)
+        lam = torch.empty((rank,), device=dev, dtype=torch.float32)
+        rho = torch.empty((1,), device=dev, dtype=torch.float32)
+    else:
+        U, lam, rho = out
+    need = refresh_workspace_size(N, d, rank, oversample, A_out is not None)
+    if ws is None:
+        ws = torch.empty((max(need, 16),), device=dev, dtype=torch.uint8)
+    if dev_status is None:
+        dev_status = torch.zeros((1,), device=dev, dtype=torch.int32)
+    _check(lib().gift_factor_refresh(_ptr(X), _dt(X), N, d, rank, oversample, iters, seed & (2**64 - 1),
+                                     _ptr(U), _ptr(lam), _ptr(rho), _ptr(A_out), _ptr(ws), ws.numel(),
+                                     _ptr(dev_status), _stream(stream)), "gift_factor_refresh")
+    return U, lam, rho, dev_status
+
+
+def encode(G: torch.Tensor, U=None, lam=None, rho=None, rank: Optional[int] = None,
+           codes: Optional[torch.Tensor] = None, scales: Optional[torch.Tensor] = None, stream=None):
+    """(codes uint8 [d_out, d_in], scales fp32 [d_out, d_in/128]); rank 0 / U None = Euclidean."""
+    _cuda(G, U, lam, rho, codes, scales)
+    d_out, d_in = G.shape
+    if rank is None:
+        rank = 0 if U is None else U.shape[1]
+    if codes is None:
+        codes = torch.empty((d_out, d_in), device=G.device, dtype=torch.uint8)
+    if scales is None:
+        scales = torch.empty((d_out, max(d_in // E4M3_BLOCK, 1)), device=G.device, dtype=torch.float32)
+    _check(lib().gift_encode(_ptr(G), _dt(G), d_out, d_in, _ptr(U), _ptr(lam), _ptr(rho), rank,
+                             _ptr(codes), _ptr(scales), _stream(stream)), "gift_encode")
+    return codes, scales
+
+
+def decode(codes: torch.Tensor, scales: torch.Tensor, U=None, lam=None, rho=None, rank: Optional[int] = None,
+           out_dtype=torch.bfloat16, out: Optional[torch.Tensor] = None, stream=None):
+    """G_hat [d_out, d_in] in out_dtype (bf16 or fp32)."""
+    _cuda(codes, scales, U, lam, rho, out)
+    d_out, d_in = codes.shape
+    if rank is None:
+        rank = 0 if U is None else U.shape[1]
+    if out is None:
+        out = torch.empty((d_out, d_in), device=codes.device, dtype=out_dtype)
+    _check(lib().gift_decode(_ptr(codes), _ptr(scales), d_out, d_in, _ptr(U), _ptr(lam), _ptr(rho), rank,
+                             _ptr(out), _dt(out), _stream(stream)), "gift_decode")
+    return out
+
+
+@dataclass
+class LayerArgs:
+    d_out: int
+    d_in: int
+    rank: int
+    dtype: torch.dtype
+    G: Optional[torch.Tensor] = None
+    G_hat: Optional[torch.Tensor] = None
+    codes: Optional[torch.Tensor] = None
+    scales: Optional[torch.Tensor] = None
+    U: Optional[torch.Tensor] = None
+    lam: Optional[torch.Tensor] = None
+    rho: Optional[torch.Tensor] = None
+
+
+def make_layers(layers: Sequence[LayerArgs]):
+    """Pack a list of LayerArgs into a ctypes gift_layer array (kept alive by the caller)."""
+    arr = (Layer * max(len(layers), 1))()
+    for i, L in enumerate(layers):
+        arr[i] = Layer(_ptr(L.G), _ptr(L.G_hat), _ptr(L.codes), _ptr(L.scales), _ptr(L.U), _ptr(L.lam),
+                       _ptr(L.rho), L.d_out, L.d_in, L.rank,
+                       GIFT_BF16 if L.dtype == torch.bfloat16 else GIFT_F32)
+    return arr
+
+
+def encode_many(packed, n: int, stream=None):
+    _check(lib().gift_encode_many(packed, n, _stream(stream)), "gift_encode_many")
+
+
+def decode_many(packed, n: int, stream=None):
+    _check(lib().gift_decode_many(packed, n, _stream(stream)), "gift_decode_many")
+
+
+def error_workspace_size(d_out: int, d_in: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().gift_error_workspace_size(d_out, d_in, ctypes.byref(n)), "gift_error_workspace_size")
+    return n.value
+
+
+def roundtrip_error(G: torch.Tensor, G_hat: torch.Tensor, out: Optional[torch.Tensor] = None,
+                    ws: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Device tensor [rel_err, ||G_hat-G||^2, ||G||^2] (fp64)."""
+    _cuda(G, G_hat, out, ws)
+    if G.dtype != G_hat.dtype or G.shape != G_hat.shape:
+        raise ValueError("G and G_hat must match in shape and dtype")
+    d_out, d_in = G.shape
+    if out is None:
+        out = torch.empty((3,), device=G.device, dtype=torch.float64)
+    if ws is None:
+        ws = torch.empty((error_workspace_size(d_out, d_in),), device=G.device, dtype=torch.uint8)
+    _check(lib().gift_roundtrip_error(_ptr(G), _ptr(G_hat), _dt(G), d_out, d_in, _ptr(out), _ptr(ws),
+                                      ws.numel(), _stream(stream)), "gift_roundtrip_error")
+    return out

@@ -1,0 +1,174 @@
+/*
+ * gift.h — C ABI of the B200 (sm_100a) GIFT gradient codec.
+ *
+ * GIFT: Geometry-Informed Low-precision Gradient Communication for LLM
+ * Pretraining (arXiv 2607.07494).  Per linear layer, the gradient G
+ * (d_out x d_in) is moved into coordinates whitened on its input side by a
+ * rank-r approximation of the K-FAC input factor A = X^T X / N, quantised
+ * (FP8 E4M3 with one fp32 scale per 128 contiguous elements of a row, or
+ * NVFP4), dequantised on the far side and mapped back (review page, "What
+ * carries the argument"; abstract).  The rank is 32 (section V.B, Table II);
+ * the factor is refreshed every K = 50 steps (section V.E, Algorithm 1).
+ *
+ * The pages do not print the transform.  This library uses
+ *     M      = rho^{-1/2} I + U diag(c)  U^T,  c_k  = (lambda_k+rho)^{-1/2} - rho^{-1/2}
+ *     M^{-1} = rho^{+1/2} I + U diag(c') U^T,  c'_k = (lambda_k+rho)^{+1/2} - rho^{+1/2}
+ * with (U, lambda) the top-r eigenpairs of A and rho the mean of A's other
+ * eigenvalues, i.e. M = (U diag(lambda) U^T + rho I)^{-1/2} for orthonormal U.
+ * Encode: W = G M, per-block E4M3.  Decode: G_hat = W_hat M^{-1}.
+ *
+ * Conventions for every entry point:
+ *  - All array pointers are DEVICE pointers owned by the caller, except where
+ *    a comment says "host".  The library never allocates device memory:
+ *    scratch space is the caller's `ws`, sized by the *_workspace_size calls.
+ *  - Layouts are row-major and dense: G, G_hat, codes are d_out x d_in (row
+ *    stride d_in elements); scales are d_out x (d_in/128); X is N x d_in;
+ *    U is d_in x rank fp32 (row stride rank); A_out is d_in x d_in fp32.
+ *  - Every call is asynchronous on `stream` (NULL = legacy default stream)
+ *    and runs entirely on the current device; there is no host round trip,
+ *    so refresh -> encode -> decode chains need no synchronisation.
+ *  - Host-detectable errors (null pointers, bad enums, shapes, alignment,
+ *    workspace too small) return a status before anything is launched and
+ *    before any CUDA call, so they can be checked without a GPU.  Launch
+ *    failures return GIFT_ERR_CUDA.  Numerical conditions found on the
+ *    device are OR-ed into the caller's `dev_status` word (GIFT_DEV_* bits);
+ *    no kernel traps.
+ *  - rank == 0 selects the Euclidean codec (M = I): U, lambda, rho ignored.
+ *  - The library keeps no state between calls except a per-process cache of
+ *    device properties; calls are re-entrant.
+ */
+#ifndef GIFT_H_
+#define GIFT_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t; declared here so the header needs no CUDA headers. */
+typedef struct CUstream_st* gift_stream_t;
+
+typedef enum {
+  GIFT_OK = 0,
+  GIFT_ERR_INVALID_ARG = 1, /* null pointer, bad enum, negative or zero size */
+  GIFT_ERR_SHAPE = 2,       /* d_in not a multiple of the block, rank too large, ... */
+  GIFT_ERR_ALIGN = 3,       /* a pointer is not 16-byte aligned */
+  GIFT_ERR_WORKSPACE = 4,   /* ws == NULL or ws_bytes below the required size */
+  GIFT_ERR_CUDA = 5,        /* a CUDA runtime call or a launch failed */
+  GIFT_ERR_UNSUPPORTED = 6  /* the current device is not sm_100 */
+} gift_status;
+
+typedef enum { GIFT_F32 = 0, GIFT_BF16 = 1 } gift_dtype;
+
+/* Bits OR-ed into *dev_status by the factor refresh. */
+#define GIFT_DEV_RHO_FLOORED 0x1u    /* rho <= 2^-24 lambda_1: floored to that value */
+#define GIFT_DEV_RANK_DEFICIENT 0x2u /* a Cholesky-QR pivot vanished: the sampled
+                                        subspace has lower rank; that column is zeroed */
+#define GIFT_DEV_NONFINITE 0x4u      /* a non-finite value reached A, lambda or rho */
+
+#define GIFT_E4M3_BLOCK 128
+#define GIFT_NVFP4_BLOCK 16
+#define GIFT_MAX_RANK 32             /* encode/decode: 0 <= rank <= 32 */
+#define GIFT_MAX_SUBSPACE 64         /* refresh: rank + oversample <= 64 */
+
+const char* gift_status_string(gift_status s);
+
+/* Library version, e.g. 100 for 0.1.0. */
+int gift_version(void);
+
+/* ------------------------------------------------------------------------
+ * Factor refresh (section V.E, Algorithm 1: the input-side factor is
+ * recomputed every K steps; rank 32 from section V.B).
+ *
+ *   A = X^T X / N                       (bf16 or fp32 X, fp32 accumulation)
+ *   Omega[i][j] = +-1 from SplitMix64(seed ^ (i*m + j)), m = rank+oversample
+ *   Q = orth(Omega); repeat `iters` times: Q = orth(A Q)   (Cholesky-QR2)
+ *   B = Q^T A Q; (theta, V) = eig(B) descending; lambda = theta[0:rank];
+ *   U = Q V[:, 0:rank]; rho = (trace A - sum lambda) / (d_in - rank),
+ *   floored at 2^-24 lambda_1 (GIFT_DEV_RHO_FLOORED).
+ *
+ * X: N x d_in, dtype xdt, 16-byte aligned.  Requires N >= 1,
+ * d_in % 128 == 0, 1 <= rank, rank + oversample <= 64 and <= d_in.
+ * Outputs: U (d_in x rank fp32), lambda (rank fp32, descending), rho (1 fp32);
+ * A_out (d_in x d_in fp32, full symmetric) if non-NULL, else A lives in ws.
+ * dev_status may be NULL; bits are OR-ed in (the caller zeroes it).
+ * ------------------------------------------------------------------------ */
+gift_status gift_refresh_workspace_size(int64_t N, int64_t d_in, int rank, int oversample,
+                                        int a_out_given, size_t* bytes /* host */);
+
+gift_status gift_factor_refresh(const void* X, gift_dtype xdt, int64_t N, int64_t d_in, int rank,
+                                int oversample, int iters, uint64_t seed, float* U, float* lambda,
+                                float* rho, float* A_out, void* ws, size_t ws_bytes,
+                                uint32_t* dev_status, gift_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Encode (review page, "What carries the argument": whiten with the
+ * input-side factor before FP8 quantisation and communication).
+ *
+ *   W = G M  (fp32),  per row and per block b of 128 columns:
+ *   amax = max |W|;  scales[b] = amax / 448;
+ *   codes = E4M3_RNE_satfinite(W * (448 / amax))   (all 0x00 when amax == 0)
+ *
+ * G: d_out x d_in (GIFT_BF16 or GIFT_F32).  codes: d_out x d_in bytes.
+ * scales: d_out x (d_in/128) fp32.  U/lambda/rho as produced by the refresh
+ * (rho > 0 and finite); 0 <= rank <= 32.  d_in % 128 == 0, d_out >= 1.
+ * ------------------------------------------------------------------------ */
+gift_status gift_encode(const void* G, gift_dtype gdt, int64_t d_out, int64_t d_in, const float* U,
+                        const float* lambda, const float* rho, int rank, uint8_t* codes,
+                        float* scales, gift_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Decode ("applies the inverse transform afterward").
+ *
+ *   W_hat = E4M3_value(codes) * scales (per block);  G_hat = W_hat M^{-1},
+ *   written as out_dt (bf16 by round-to-nearest-even, or fp32).
+ * ------------------------------------------------------------------------ */
+gift_status gift_decode(const uint8_t* codes, const float* scales, int64_t d_out, int64_t d_in,
+                        const float* U, const float* lambda, const float* rho, int rank,
+                        void* G_hat, gift_dtype out_dt, gift_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Grouped encode / decode over many layers in as few launches as possible
+ * (selective deployment: whitened layers have rank 32, the others rank 0;
+ * section V.C, Fig. 3 / Fig. 4).  `layers` is a HOST array of n entries;
+ * each entry follows the rules of gift_encode / gift_decode.  Encode reads
+ * G and writes codes/scales; decode reads codes/scales and writes G_hat.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+  const void* G;       /* encode input */
+  void* G_hat;         /* decode output */
+  uint8_t* codes;      /* encode output / decode input */
+  float* scales;       /* encode output / decode input */
+  const float* U;      /* d_in x rank, ignored when rank == 0 */
+  const float* lambda; /* rank */
+  const float* rho;    /* 1 */
+  int64_t d_out;
+  int64_t d_in;
+  int32_t rank;        /* 0 (Euclidean) or 1..32 */
+  int32_t dtype;       /* gift_dtype of G and G_hat */
+} gift_layer;
+
+gift_status gift_encode_many(const gift_layer* layers /* host */, int n, gift_stream_t stream);
+gift_status gift_decode_many(const gift_layer* layers /* host */, int n, gift_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * One-step round-trip error (Tables I-II: relative reconstruction error of
+ * the FP8 round trip against the full-precision gradient).
+ *
+ *   out[0] = ||G_hat - G||_F / ||G||_F,  out[1] = ||G_hat - G||_F^2,
+ *   out[2] = ||G||_F^2, all accumulated in fp64 in a fixed order
+ *   (deterministic).  out: 3 doubles on the device.
+ * ------------------------------------------------------------------------ */
+gift_status gift_error_workspace_size(int64_t d_out, int64_t d_in, size_t* bytes /* host */);
+
+gift_status gift_roundtrip_error(const void* G, const void* G_hat, gift_dtype dt, int64_t d_out,
+                                 int64_t d_in, double* out, void* ws, size_t ws_bytes,
+                                 gift_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GIFT_H_ */

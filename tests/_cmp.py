@@ -1,0 +1,57 @@
+"""Comparison helpers for GPU-vs-oracle parity (test code only).
+
+Match criteria for the codec (written here once, used by every parity test):
+  * E4M3 codes: bit-exact on >= 99.9 % of elements; every other element
+    one code step away (adjacent representable values; +0 and -0 count as
+    the same value).  The kernels form W in fp32 with a different summation
+    order than the fp64 oracle, so a value within ~1e-6 of a rounding
+    boundary may land on the neighbouring code.
+  * scales: relative error <= 1e-3 (they are amax/448 of the same W).
+  * G_hat (decoder fed the oracle's codes): fp32 output within 1e-3 of the
+    oracle relative to the row's largest magnitude; bf16 output within one
+    bf16 rounding (2^-8 relative) of the same reference plus that 1e-3.
+"""
+import numpy as np
+
+CODE_EXACT_FRAC = 0.999
+SCALE_RTOL = 1e-3
+GHAT_RTOL = 1e-3
+
+
+def e4m3_position(codes):
+    c = np.asarray(codes, dtype=np.int64)
+    mag = c & 0x7F
+    return np.where(c & 0x80, -mag, mag)
+
+
+def check_codes(got, want, frac=CODE_EXACT_FRAC):
+    got = np.asarray(got)
+    want = np.asarray(want)
+    assert got.shape == want.shape
+    exact = got == want
+    pos_diff = np.abs(e4m3_position(got) - e4m3_position(want))
+    same_value = pos_diff == 0  # +0 / -0
+    ok = exact | same_value
+    rate = ok.mean() if ok.size else 1.0
+    assert rate >= frac, f"bit-exact rate {rate:.6f} < {frac}"
+    assert pos_diff.max(initial=0) <= 1, f"max code distance {pos_diff.max()}"
+    return rate
+
+
+def check_scales(got, want, rtol=SCALE_RTOL):
+    got = np.asarray(got, dtype=np.float64)
+    want = np.asarray(want, dtype=np.float64)
+    err = np.abs(got - want) / np.maximum(np.abs(want), 1e-300)
+    err = np.where(want == 0, np.abs(got), err)
+    assert err.max(initial=0) <= rtol, f"scale rel err {err.max()}"
+
+
+def check_rows(got, want, rtol=GHAT_RTOL, bf16=False):
+    got = np.asarray(got, dtype=np.float64)
+    want = np.asarray(want, dtype=np.float64)
+    rowmax = np.max(np.abs(want), axis=1, keepdims=True)
+    tol = rtol * rowmax
+    if bf16:
+        tol = tol + 2.0 ** -8 * np.abs(want)
+    bad = np.abs(got - want) > tol + 1e-30
+    assert not bad.any(), f"{bad.sum()} elements off; worst {(np.abs(got - want) / np.maximum(rowmax, 1e-30)).max()}"

@@ -1,0 +1,130 @@
+"""CPU-only checks of the C ABI: the library loads without a GPU, exports
+every function include/gift.h declares, and rejects bad arguments on the
+host before any CUDA call (the status codes gift.h documents).
+
+Only argument combinations that fail host validation are passed here; the
+fake addresses below are never dereferenced because validation returns
+first.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from geometry_aware_fp8_b200 import ops
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+OK, INVALID, SHAPE, ALIGN, WORKSPACE = 0, 1, 2, 3, 4
+A16 = 0x10000          # aligned fake address (never dereferenced)
+A_ODD = 0x10004        # 4-byte but not 16-byte aligned
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "gift.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(gift_[a-z0-9_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    try:
+        return ops.lib()
+    except RuntimeError as e:
+        pytest.fail(str(e))
+
+
+def test_library_exports_every_declared_symbol(L):
+    names = declared_functions()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(ops.EXPORTED)
+
+
+def test_version_and_status_strings(L):
+    assert L.gift_version() >= 100
+    for s in range(7):
+        assert L.gift_status_string(s).startswith(b"GIFT_")
+
+
+def test_encode_rejects_bad_arguments(L):
+    s = None
+    # null pointers
+    assert L.gift_encode(None, 1, 4, 128, None, None, None, 0, A16, A16, s) == INVALID
+    # bad dtype
+    assert L.gift_encode(A16, 7, 4, 128, None, None, None, 0, A16, A16, s) == INVALID
+    # d_in not a multiple of 128
+    assert L.gift_encode(A16, 1, 4, 100, None, None, None, 0, A16, A16, s) == SHAPE
+    # rank above 32
+    assert L.gift_encode(A16, 1, 4, 128, A16, A16, A16, 33, A16, A16, s) == SHAPE
+    # whitened without factors
+    assert L.gift_encode(A16, 1, 4, 128, None, None, None, 32, A16, A16, s) == INVALID
+    # misaligned gradient / codes
+    assert L.gift_encode(A_ODD, 1, 4, 128, None, None, None, 0, A16, A16, s) == ALIGN
+    assert L.gift_encode(A16, 1, 4, 128, None, None, None, 0, A_ODD, A16, s) == ALIGN
+    # negative sizes
+    assert L.gift_encode(A16, 1, -1, 128, None, None, None, 0, A16, A16, s) == INVALID
+
+
+def test_decode_rejects_bad_arguments(L):
+    s = None
+    assert L.gift_decode(None, A16, 4, 128, None, None, None, 0, A16, 1, s) == INVALID
+    assert L.gift_decode(A16, A16, 4, 256 + 64, None, None, None, 0, A16, 1, s) == SHAPE
+    assert L.gift_decode(A16, A16, 4, 128, None, None, None, 0, A16, 3, s) == INVALID
+    assert L.gift_decode(A16, A16, 4, 128, None, None, None, 0, A_ODD, 1, s) == ALIGN
+
+
+def test_refresh_rejects_bad_arguments(L):
+    s = None
+    n = ctypes.c_size_t(0)
+    assert L.gift_refresh_workspace_size(1024, 512, 32, 16, 0, ctypes.byref(n)) == OK
+    need = n.value
+    assert need >= 512 * 512 * 4  # A lives in the workspace when A_out is not given
+    assert L.gift_refresh_workspace_size(1024, 512, 32, 16, 1, ctypes.byref(n)) == OK
+    assert n.value < need
+    assert L.gift_refresh_workspace_size(1024, 500, 32, 16, 0, ctypes.byref(n)) == SHAPE
+    assert L.gift_refresh_workspace_size(1024, 512, 48, 17, 0, ctypes.byref(n)) == SHAPE
+    assert L.gift_refresh_workspace_size(0, 512, 32, 16, 0, ctypes.byref(n)) == INVALID
+    args = dict(X=A16, xdt=1, N=1024, d=512, r=32, p=16, it=4, seed=0, U=A16, lam=A16, rho=A16, A=None)
+
+    def call(ws, ws_bytes, **kw):
+        a = dict(args, **kw)
+        return L.gift_factor_refresh(a["X"], a["xdt"], a["N"], a["d"], a["r"], a["p"], a["it"], a["seed"], a["U"],
+                                     a["lam"], a["rho"], a["A"], ws, ws_bytes, None, s)
+
+    assert call(None, 0) == WORKSPACE
+    assert call(A16, need - 1) == WORKSPACE
+    assert call(A16, need, X=None) == INVALID
+    assert call(A16, need, xdt=5) == INVALID
+    assert call(A16, need, X=A_ODD) == ALIGN
+    assert call(A16, need, it=-1) == INVALID
+    assert call(A16, need, r=0) == INVALID
+
+
+def test_error_rejects_bad_arguments(L):
+    n = ctypes.c_size_t(0)
+    assert L.gift_error_workspace_size(16, 256, ctypes.byref(n)) == OK and n.value >= 16
+    assert L.gift_roundtrip_error(A16, A16, 1, 16, 256, A16, None, 0, None) == WORKSPACE
+    assert L.gift_roundtrip_error(A16, None, 1, 16, 256, A16, A16, n.value, None) == INVALID
+    assert L.gift_roundtrip_error(A16, A_ODD, 1, 16, 256, A16, A16, n.value, None) == ALIGN
+
+
+def test_many_rejects_a_bad_layer_before_launching(L):
+    good = ops.Layer(A16, A16, A16, A16, None, None, None, 8, 256, 0, 1)
+    bad = ops.Layer(A16, A16, A16, A16, None, None, None, 8, 200, 0, 1)
+    arr = (ops.Layer * 2)(good, bad)
+    assert L.gift_encode_many(arr, 2, None) == SHAPE
+    assert L.gift_encode_many(None, 3, None) == INVALID
+    assert L.gift_encode_many(arr, 0, None) == OK
+
+
+def test_product_path_has_no_oracle_import():
+    pkg = os.path.join(ROOT, "geometry_aware_fp8_b200")
+    pat = re.compile(r"^\s*(from|import)\s+oracle\b|gift_oracle|#include\s+\"[^\"]*oracle", re.M)
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                txt = open(os.path.join(dirpath, f)).read()
+                assert not pat.search(txt), f

@@ -1,0 +1,102 @@
+"""GPU parity of the factor refresh against the CPU oracle, through the C ABI.
+
+Criteria: A entries within 1e-5 of max|A| (fp32 accumulation of exact bf16/fp32
+products); the top-32 Ritz values within 1e-4 relative (same algorithm, same
+SplitMix64 start block); rho within 1e-4 relative; U orthonormal to 1e-5;
+the Ritz property U^T A U = diag(lambda) on the oracle's fp64 A.  The
+transform M is compared in relative Frobenius norm within 1e-2: after four
+iterations the Ritz vectors next to the rank cut (lambda_32 vs lambda_33)
+rotate by about |dB| / (theta_32 - theta_33), which for fp32 arithmetic and
+the i^-2 spectra here is ~1e-3 of M's norm.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import gift_oracle as O
+from geometry_aware_fp8_b200 import ops, synth
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+
+def _refresh_both(X, rank=32, over=16, iters=4, seed=7, dtype="f32"):
+    Xs = synth.to_storage(X, dtype)
+    Xd = torch.from_numpy(Xs).to(DEV)
+    if dtype == "bf16":
+        Xd = Xd.to(torch.bfloat16)
+    d = X.shape[1]
+    A_out = torch.empty((d, d), device=DEV, dtype=torch.float32)
+    U, lam, rho, st = ops.factor_refresh(Xd, rank, over, iters, seed, A_out=A_out)
+    torch.cuda.synchronize()
+    A = O.input_factor(Xs)
+    Uo, lo, ro, fo = O.factor_refresh(A, rank, over, iters, seed=seed)
+    return (A_out.cpu().numpy().astype(np.float64), U.cpu().numpy().astype(np.float64),
+            lam.cpu().numpy().astype(np.float64), float(rho.item()), int(st.item())), (A, Uo, lo, ro, fo)
+
+
+def _check(gpu, orc, m_tol=1e-2):
+    Ag, Ug, lg, rg, sg = gpu
+    A, Uo, lo, ro, fo = orc
+    assert np.max(np.abs(Ag - A)) <= 1e-5 * np.max(np.abs(A))
+    assert np.allclose(lg, lo, rtol=1e-4, atol=0)
+    assert rg == pytest.approx(ro, rel=1e-4)
+    assert (sg & ops.DEV_RHO_FLOORED) == (fo & 1)
+    r = Ug.shape[1]
+    assert np.max(np.abs(Ug.T @ Ug - np.eye(r))) < 1e-5
+    R = Ug.T @ A @ Ug
+    assert np.max(np.abs(R - np.diag(lg))) < 1e-4 * lg[0]
+    Mg = O.transform_matrix(Ug, lg, rg)
+    Mo = O.transform_matrix(Uo, lo, ro)
+    assert np.linalg.norm(Mg - Mo) / np.linalg.norm(Mo) < m_tol
+
+
+def test_refresh_config1_fp32():
+    """One 512-wide layer: X 2048 x 512 fp32, sigma_i = i^-1."""
+    Q = synth.haar_orthogonal(512, 1003)
+    X = synth.activations(2048, Q, synth.column_power(512, 1.0), 1001)
+    g, o = _refresh_both(X, dtype="f32", seed=1004)
+    _check(g, o)
+
+
+def test_refresh_bf16_spiked_spectrum():
+    """bf16 X with the config-4 spectrum shape (i^-1.2, five spikes of 100x), scaled down."""
+    d = 1024
+    Q = synth.haar_orthogonal(d, 11)
+    X = synth.activations(4096, Q, synth.spectrum_power(d, 1.2, 5, 100.0), 12)
+    g, o = _refresh_both(X, dtype="bf16", seed=13)
+    _check(g, o)
+
+
+@pytest.mark.parametrize("rank,over,iters", [(8, 8, 2), (32, 0, 3), (16, 17, 1)])
+def test_refresh_rank_and_oversample_variants(rank, over, iters):
+    d = 256
+    Q = synth.haar_orthogonal(d, 21)
+    X = synth.activations(1024, Q, synth.spectrum_power(d, 2.0), 22)
+    g, o = _refresh_both(X, rank, over, iters, seed=23)
+    _check(g, o, m_tol=5e-2)
+
+
+def test_refresh_rank_deficient_input_sets_status():
+    """N = 20 tokens < rank + oversample: A has rank 20, the sampled subspace
+    loses columns (status bit), the nonzero Ritz values still match."""
+    d = 128
+    Q = synth.haar_orthogonal(d, 31)
+    X = synth.activations(20, Q, synth.column_power(d, 0.5), 32)
+    g, o = _refresh_both(X, 32, 16, 2, seed=33)
+    Ag, Ug, lg, rg, sg = g
+    A, Uo, lo, ro, fo = o
+    assert sg & ops.DEV_RANK_DEFICIENT
+    assert sg & ops.DEV_RHO_FLOORED and fo & 1
+    assert np.allclose(lg[:20], lo[:20], rtol=1e-4)
+    assert np.all(np.isfinite(Ug)) and np.isfinite(rg) and rg > 0
+
+
+def test_refresh_is_deterministic():
+    d = 512
+    Q = synth.haar_orthogonal(d, 41)
+    X = torch.from_numpy(synth.activations(2048, Q, synth.column_power(d, 1.0), 42).astype(np.float32)).to(DEV)
+    a = ops.factor_refresh(X, 32, 16, 4, 5)
+    b = ops.factor_refresh(X, 32, 16, 4, 5)
+    for x, y in zip(a[:3], b[:3]):
+        assert torch.equal(x, y)
