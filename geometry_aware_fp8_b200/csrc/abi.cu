@@ -44,12 +44,13 @@ inline gift_status cuda_status(cudaError_t e) { return e == cudaSuccess ? GIFT_O
 
 gift_status check_codec_args(const void* G, int gdt, int64_t d_out, int64_t d_in, const float* U,
                              const float* lambda, const float* rho, int rank, const void* codes, const float* scales) {
-  if (!G || !codes || !scales) return GIFT_ERR_INVALID_ARG;
   if (!dtype_ok(gdt)) return GIFT_ERR_INVALID_ARG;
   if (d_out < 0 || d_in <= 0) return GIFT_ERR_INVALID_ARG;
   if (d_in % GIFT_E4M3_BLOCK != 0) return GIFT_ERR_SHAPE;
   if (d_in > (1 << 20) || d_out > ((int64_t)1 << 31)) return GIFT_ERR_SHAPE;
   if (rank < 0 || rank > GIFT_MAX_RANK) return GIFT_ERR_SHAPE;
+  if (d_out == 0) return GIFT_OK;  // empty gradient: nothing is read or written
+  if (!G || !codes || !scales) return GIFT_ERR_INVALID_ARG;
   if (rank > 0 && (!U || !lambda || !rho)) return GIFT_ERR_INVALID_ARG;
   if (!aligned16(G) || !aligned16(codes) || !aligned16(scales)) return GIFT_ERR_ALIGN;
   if (rank > 0 && (!aligned16(U) || !aligned(lambda, 4) || !aligned(rho, 4))) return GIFT_ERR_ALIGN;

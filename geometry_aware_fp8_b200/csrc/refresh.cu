@@ -12,6 +12,8 @@
 // dense steps (m x m Cholesky, Jacobi, sort) run in one CTA in fp64 shared
 // memory; Gram matrices are reduced in fp64 with a fixed order so results
 // are bit-identical from run to run.
+#include <atomic>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -503,11 +505,17 @@ static cudaError_t orth_cholqr2(float* Yb, float* tmp, int d, int m, int parts, 
 
 cudaError_t launch_refresh(const RefreshPlan& p, const void* X, gift_dtype xdt, float* U, float* lambda, float* rho,
                            float* A_out, void* ws, uint32_t* dev_status, cudaStream_t s) {
-  static bool attr_done = false;
-  if (!attr_done) {
-    cudaFuncSetAttribute(chol_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmallSmem);
-    cudaFuncSetAttribute(rr_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmallSmem);
-    attr_done = true;
+  // the two single-CTA fp64 kernels need 65 KB of dynamic shared memory
+  static std::atomic<uint64_t> attr_done{0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const uint64_t bit = 1ull << (dev & 63);
+  if (!(attr_done.load() & bit)) {
+    cudaError_t e1 = cudaFuncSetAttribute(chol_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmallSmem);
+    cudaError_t e2 = cudaFuncSetAttribute(rr_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmallSmem);
+    if (e1 != cudaSuccess) return e1;
+    if (e2 != cudaSuccess) return e2;
+    attr_done.fetch_or(bit);
   }
   char* w = (char*)ws;
   const int d = (int)p.d, m = p.m, r = p.rank;

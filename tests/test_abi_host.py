@@ -51,8 +51,9 @@ def test_version_and_status_strings(L):
 
 def test_encode_rejects_bad_arguments(L):
     s = None
-    # null pointers
+    # null pointers (an empty gradient, d_out == 0, may pass nulls)
     assert L.gift_encode(None, 1, 4, 128, None, None, None, 0, A16, A16, s) == INVALID
+    assert L.gift_encode(None, 1, 0, 128, None, None, None, 0, None, None, s) == OK
     # bad dtype
     assert L.gift_encode(A16, 7, 4, 128, None, None, None, 0, A16, A16, s) == INVALID
     # d_in not a multiple of 128
