@@ -20,7 +20,8 @@
 namespace gift {
 
 cudaError_t launch_syrk_tc(const void* X, gift_dtype xdt, int64_t N, int d, float* A, float* part, int splits,
-                           cudaStream_t s, bool* used);
+                           uint32_t* err, cudaStream_t s, bool* used);
+int syrk_tc_tiles(int d);
 
 namespace {
 
@@ -115,18 +116,18 @@ __global__ void __launch_bounds__(kRT) syrk_simt_kernel(const T* __restrict__ X,
     }
 }
 
-// Sum of split-K partials (upper tiles only) into the full symmetric A.
+// Sum of split-K partials (entries j >= i) into the full symmetric A.
 __global__ void syrk_reduce_kernel(const float* __restrict__ part, int splits, int d, float* __restrict__ A,
                                    float scale) {
   const int64_t dd = (int64_t)d * d;
   for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < dd; e += (int64_t)gridDim.x * blockDim.x) {
     const int i = (int)(e / d), j = (int)(e % d);
-    if (i / 128 > j / 128) continue;  // lower tiles are written as mirrors
+    if (j < i) continue;  // the lower triangle is written as the mirror
     float v = 0.0f;
     for (int s = 0; s < splits; ++s) v += part[s * dd + e];
     v *= scale;
     A[e] = v;
-    if (i / 128 != j / 128) A[(int64_t)j * d + i] = v;
+    if (j != i) A[(int64_t)j * d + i] = v;
   }
 }
 
@@ -468,9 +469,9 @@ void refresh_plan(int64_t N, int64_t d, int rank, int oversample, bool a_out_giv
   p->seed = 0;
   p->gram_parts = (int)((d + 63) / 64);
   // split-K over tokens so that the triangle of 128 x 256 tiles fills the SMs
-  const int64_t tiles = (d / 128) * (d / 128 + 1) / 2;
+  const int64_t tiles = syrk_tc_tiles((int)d);
   int splits = 1;
-  while (splits < 16 && tiles * splits < 2 * kNumSMs && N / (splits * 2) >= 1024) splits *= 2;
+  while (splits < 16 && tiles * splits < kNumSMs && N / (splits * 2) >= 1024) splits *= 2;
   p->syrk_splits = splits;
   size_t off = 0;
   p->off_A = off;
@@ -529,7 +530,8 @@ cudaError_t launch_refresh(const RefreshPlan& p, const void* X, gift_dtype xdt, 
 
   // R1: A = X^T X / N
   bool used_tc = false;
-  cudaError_t e = launch_syrk_tc(X, xdt, p.N, d, A, (float*)(w + p.off_syrk), p.syrk_splits, s, &used_tc);
+  cudaError_t e = launch_syrk_tc(X, xdt, p.N, d, A, (float*)(w + p.off_syrk), p.syrk_splits, dev_status, s,
+                                 &used_tc);
   if (e != cudaSuccess) return e;
   if (!used_tc) {
     const int nt = d / 64;

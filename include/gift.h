@@ -67,6 +67,8 @@ typedef enum { GIFT_F32 = 0, GIFT_BF16 = 1 } gift_dtype;
 #define GIFT_DEV_RANK_DEFICIENT 0x2u /* a Cholesky-QR pivot vanished: the sampled
                                         subspace has lower rank; that column is zeroed */
 #define GIFT_DEV_NONFINITE 0x4u      /* a non-finite value reached A, lambda or rho */
+#define GIFT_DEV_TIMEOUT 0x8u        /* a pipeline wait inside a kernel gave up after its
+                                        iteration bound; the outputs of that call are undefined */
 
 #define GIFT_E4M3_BLOCK 128
 #define GIFT_NVFP4_BLOCK 16

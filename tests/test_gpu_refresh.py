@@ -100,3 +100,59 @@ def test_refresh_is_deterministic():
     b = ops.factor_refresh(X, 32, 16, 4, 5)
     for x, y in zip(a[:3], b[:3]):
         assert torch.equal(x, y)
+
+
+def test_refresh_config2_bf16_split_k():
+    """MLP up-projection stand-in: X 8192 x 1536 bf16 (sigma_i = i^-1); the
+    tensor-core syrk splits the token range four ways here."""
+    Q = synth.haar_orthogonal(1536, 2003)
+    X = synth.activations(8192, Q, synth.column_power(1536, 1.0), 2001)
+    g, o = _refresh_both(X, dtype="bf16", seed=2004)
+    _check(g, o)
+
+
+def test_refresh_config4_full_size_properties():
+    """Factor refresh at scale: X 65536 x 4096 bf16, eigenvalues i^-1.2 with
+    five 100x spikes, 4 iterations, oversample 16.  The oracle cannot form
+    A at this size in seconds, so it checks what holds at any size:
+    sampled entries of A (exact fp64 dot products of bf16 columns), the
+    Rayleigh-Ritz property (XU)^T (XU) / N = diag(lambda) in fp64, and rho
+    against the trace identity on the GPU's own U."""
+    N, d = 65536, 4096
+    gen = torch.Generator(device=DEV)
+    gen.manual_seed(4001)
+    Qd = torch.from_numpy(synth.haar_orthogonal(d, 4003).astype(np.float32)).to(DEV)
+    sig = torch.from_numpy(synth.spectrum_power(d, 1.2, 5, 100.0).astype(np.float32)).to(DEV)
+    X = synth.device_activations(N, sig, Qd, gen, torch.bfloat16)
+    A_out = torch.empty((d, d), device=DEV, dtype=torch.float32)
+    U, lam, rho, st = ops.factor_refresh(X, 32, 16, 4, 4004, A_out=A_out)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    Xh = X.float().cpu().numpy()
+    rng = np.random.default_rng(0)
+    idx = rng.integers(0, d, size=(200, 2))
+    idx[:20, 1] = idx[:20, 0]                       # include diagonal entries
+    Ah = A_out.cpu().numpy()
+    want = np.array([np.dot(Xh[:, i].astype(np.float64), Xh[:, j].astype(np.float64)) / N for i, j in idx])
+    got = Ah[idx[:, 0], idx[:, 1]]
+    scale = np.sqrt(Ah[idx[:, 0], idx[:, 0]].astype(np.float64) * Ah[idx[:, 1], idx[:, 1]])
+    assert np.max(np.abs(got - want) / scale) < 1e-5
+    assert np.array_equal(Ah, Ah.T)
+    Ug = U.cpu().numpy().astype(np.float64)
+    lg = lam.cpu().numpy().astype(np.float64)
+    XU = np.zeros((32, 32))
+    fro = 0.0
+    for r0 in range(0, N, 8192):
+        blk = Xh[r0:r0 + 8192].astype(np.float64)
+        P = blk @ Ug
+        XU += P.T @ P
+        fro += np.sum(blk * blk)
+    R = XU / N
+    assert np.allclose(np.diag(R), lg, rtol=1e-4)
+    assert np.max(np.abs(R - np.diag(np.diag(R)))) < 1e-4 * lg[0]
+    rho_ref = (fro / N - np.trace(R)) / (d - 32)
+    rel = abs(rho.item() - rho_ref) / rho_ref
+    print(f"config4 rho {rho.item():.6e} vs trace identity {rho_ref:.6e} (rel {rel:.2e}); lambda_1 {lg[0]:.4f}")
+    # rho is a difference of two ~500-sized sums that leaves ~1.5: the fp32
+    # accumulation of A's diagonal (~1e-6 relative) is amplified ~300x.
+    assert rel < 1e-3
