@@ -1,14 +1,486 @@
 // Whitened E4M3 codec on the tcgen05 tensor cores (bf16 gradients).
-// Not yet enabled: the C-ABI routes every layer to the CUDA-core kernels
-// while tc_codec_available() returns false.
+//
+// GIFT review page, "What carries the argument": the gradient G of a linear
+// layer is whitened on its input side before FP8 quantisation,
+//   W = G M,  M = a I + U diag(c) U^T,  a = rho^{-1/2},
+//   c_k = (lambda_k + rho)^{-1/2} - a,
+// and mapped back with M^{-1} after dequantisation.  Per 128-row panel:
+//   E1  P = G U            (M=128, N=64, K=d_in)  tensor cores
+//   E2  W = a G + (P o c) U^T  (M=128, N=128 per chunk, K=32)
+//   E3  amax per 128-column block, E4M3 codes, fp32 scales
+// U is fp32; it is split into bf16 hi + lo parts so that every product is
+// exact to ~2^-17 (G is exact in bf16, so E1 needs G.U_hi + G.U_lo; E2 needs
+// Pc_hi.U_hi + Pc_lo.U_hi + Pc_hi.U_lo).  Accumulation is fp32 in TMEM.
+//
+// Data flow (one persistent CTA per SM, 288 threads, warp-specialised):
+//   warp 4 lane 0   TMA loads of 128x128 G chunks (two 64-column SW128 boxes)
+//   warps 4-7       convert the matching 128 rows of U into one bf16 tile
+//                   [128 rows][hi 32 | lo 32] with the 128-byte swizzle; the
+//                   tile is the MN-major B operand of E1 and the K-major B
+//                   operand of E2
+//   warp 8          TMEM allocation; one thread issues every MMA
+//   warps 0-3       epilogue, thread = row: forms the bf16 hi/lo tile of P o c
+//                   (the A operand of E2), then per chunk reads W from TMEM and
+//                   G from shared memory, finds the block maximum and stores
+//                   128 codes (8 x 16-byte stores) and one scale.
+// E1 streams G forward from HBM; E2 walks the same chunks backwards so the
+// most recently loaded ones are re-read while still in L2.  Panels of all
+// layers of one launch are assigned to CTAs on the host by longest-first
+// greedy scheduling (a panel costs d_in/128 chunks).
+#include <algorithm>
+#include <queue>
+#include <vector>
+
 #include "common.cuh"
 #include "internal.h"
+#include "tma_host.h"
 
 namespace gift {
+namespace {
 
-bool tc_codec_available() { return false; }
+constexpr int kPanel = 128;                 // rows per panel = UMMA M
+constexpr int kChunk = 128;                 // columns per step = one scale block
+constexpr int kStages = 4;
+constexpr int kGBytes = kPanel * kChunk * 2;   // 32 KB: two [128][64] bf16 boxes
+constexpr int kGHalf = kGBytes / 2;
+constexpr int kUBytes = kChunk * 128;          // 16 KB: [128 rows][64 bf16]
+constexpr int kStageBytes = kGBytes + kUBytes;
+constexpr int kPcBytes = kPanel * 128;         // 16 KB: [128 rows][64 bf16]
+constexpr int kSmemBytes = kStages * kStageBytes + kPcBytes + 1024 + 512;
+constexpr int kThreads = 288;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColW0 = 0, kColW1 = 128, kColP = 256;
+constexpr uint32_t kIdescE1 = umma_idesc_bf16(128, 64, 0, 1);   // A K-major, B MN-major
+constexpr uint32_t kIdescE2 = umma_idesc_bf16(128, 128, 0, 0);  // both K-major
+constexpr uint32_t kWaitLimit = 1u << 22;
+constexpr int kMaxJobs = 48;
+constexpr int kMaxPanels = 1536;
 
-cudaError_t launch_whiten_encode_tc(const TcLayer*, int, cudaStream_t) { return cudaErrorNotSupported; }
+struct alignas(64) EncJob {
+  CUtensorMap tmG;  // bf16 [d_out][d_in], box [128][64], 128-byte swizzle
+  const float* U;
+  const float* lambda;
+  const float* rho;
+  uint8_t* codes;
+  float* scales;
+  int d_out, d_in, rank, pad;
+};
+
+struct EncParams {
+  EncJob jobs[kMaxJobs];
+  uint16_t sched_off[kNumSMs + 1];  // CTA b runs sched_ids[sched_off[b] .. sched_off[b+1])
+  uint16_t sched_ids[kMaxPanels];   // job << 8 | panel
+};
+
+// 16-byte chunk q of row r of a [rows][128 B] tile with the 128-byte swizzle
+GIFT_DEV uint32_t sw128(uint32_t r, uint32_t q) { return r * 128u + ((q ^ (r & 7u)) << 4); }
+
+GIFT_DEV void named_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
+
+// Named barrier that also ORs a predicate over the group: every member gets
+// the same answer, so a group can agree to stop without a shared flag.
+GIFT_DEV bool named_sync_or(int id, int n, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %3, 0;\n\t"
+      "barrier.red.or.pred p, %1, %2, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"(id), "r"(n), "r"((uint32_t)v)
+      : "memory");
+  return r != 0;
+}
+
+GIFT_DEV void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+GIFT_DEV uint4 ld_shared_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+
+// Split fp32 into bf16 hi (RNE) and bf16 lo = RNE(x - hi).
+GIFT_DEV void split_bf16(float x, float& hi, float& lo) {
+  hi = __bfloat162float(__float2bfloat16_rn(x));
+  lo = x - hi;
+}
+
+// Convert rows [j0, j0+128) of U (d_in x rank fp32) into the swizzled
+// [128][hi 32 | lo 32] bf16 tile; thread t of the 128 converter threads owns row t.
+GIFT_DEV void convert_u_tile(const float* __restrict__ U, int rank, int j0, uint32_t tile, int t) {
+  float u[32];
+  const float* src = U + (int64_t)(j0 + t) * rank;
+  if (rank == 32) {
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      float4 v = __ldg(reinterpret_cast<const float4*>(src) + q);
+      u[4 * q] = v.x; u[4 * q + 1] = v.y; u[4 * q + 2] = v.z; u[4 * q + 3] = v.w;
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < 32; ++k) u[k] = k < rank ? __ldg(src + k) : 0.0f;
+  }
+  uint32_t hi[16], lo[16];
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    float h0, l0, h1, l1;
+    split_bf16(u[2 * k], h0, l0);
+    split_bf16(u[2 * k + 1], h1, l1);
+    hi[k] = pack_bf16x2(h0, h1);
+    lo[k] = pack_bf16x2(l0, l1);
+  }
+#pragma unroll
+  for (int q = 0; q < 4; ++q) st_shared_v4(tile + sw128(t, q), hi[4 * q], hi[4 * q + 1], hi[4 * q + 2], hi[4 * q + 3]);
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    st_shared_v4(tile + sw128(t, 4 + q), lo[4 * q], lo[4 * q + 1], lo[4 * q + 2], lo[4 * q + 3]);
+}
+
+__global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __grid_constant__ EncParams p,
+                                                                     uint32_t* err) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t pc_tile = sbase + kStages * kStageBytes;
+  uint64_t* bars = (uint64_t*)(smem + kStages * kStageBytes + kPcBytes);
+  uint64_t* full = bars;                  // [kStages] count 2: TMA tx + converter
+  uint64_t* empty = bars + kStages;       // [kStages] count 1
+  uint64_t* p_full = bars + 2 * kStages;  // count 1 (MMA commit)
+  uint64_t* pc_full = p_full + 1;         // count 128 (epilogue)
+  uint64_t* w_full = p_full + 2;          // [2] count 1
+  uint64_t* w_empty = p_full + 4;         // [2] count 128
+  uint32_t* tmem_slot = (uint32_t*)(p_full + 6);
+  __shared__ int failed;  // any role gave up (reported at exit)
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int beg = p.sched_off[blockIdx.x], end = p.sched_off[blockIdx.x + 1];
+
+  if (threadIdx.x == 0) {
+    failed = 0;
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 2);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(p_full, 1);
+    mbar_init(pc_full, 128);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&w_full[b], 1);
+      mbar_init(&w_empty[b], 128);
+    }
+    fence_mbar_init();
+  }
+  if (warp == 8) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+
+  if (warp >= 4 && warp < 8) {
+    // ---------------- producer: TMA for G + U conversion ----------------
+    // Exit decisions are taken on the group-local flag right after a named
+    // barrier, so all 128 threads leave at the same step.
+    const int t = threadIdx.x - 128;
+    uint32_t step = 0;
+    bool stop = false;  // group vote: set for all 128 threads at the same barrier
+    for (int it = beg; it < end && !stop; ++it) {
+      const int jb = p.sched_ids[it] >> 8, panel = p.sched_ids[it] & 255;
+      const EncJob& J = p.jobs[jb];
+      const int nc = J.d_in / kChunk;
+      for (int pass = 0; pass < 2 && !stop; ++pass) {
+        for (int i = 0; i < nc; ++i, ++step) {
+          const int c = pass == 0 ? i : nc - 1 - i;
+          const int s = step % kStages;
+          const uint32_t use = step / kStages;
+          const bool ok = step < kStages || mbar_wait(&empty[s], (use - 1) & 1u, kWaitLimit);
+          stop = named_sync_or(1, 128, !ok);
+          if (stop) {
+            failed = 1;
+            break;
+          }
+          const uint32_t g_tile = sbase + s * kStageBytes;
+          if (t == 0) {
+            mbar_arrive_expect_tx(&full[s], kGBytes);
+            tma_load_2d(smem + s * kStageBytes, &J.tmG, &full[s], c * kChunk, panel * kPanel);
+            tma_load_2d(smem + s * kStageBytes + kGHalf, &J.tmG, &full[s], c * kChunk + 64, panel * kPanel);
+          }
+          convert_u_tile(J.U, J.rank, c * kChunk, g_tile + kGBytes, t);
+          fence_async_shared();
+          named_sync(1, 128);
+          if (t == 0) mbar_arrive(&full[s]);
+        }
+      }
+    }
+  } else if (warp == 8) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      uint32_t step = 0, e2 = 0, np = 0;
+      for (int it = beg; it < end && !failed; ++it, ++np) {
+        const EncJob& J = p.jobs[p.sched_ids[it] >> 8];
+        const int nc = J.d_in / kChunk;
+        // E1: P2[128 x 64] = G . [U_hi | U_lo]
+        for (int c = 0; c < nc; ++c, ++step) {
+          const int s = step % kStages;
+          if (!mbar_wait(&full[s], (step / kStages) & 1u, kWaitLimit)) { failed = 1; break; }
+          tc_fence_after();
+          const uint32_t g_tile = sbase + s * kStageBytes, u_tile = g_tile + kGBytes;
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t ad = umma_desc_sw128(g_tile + h * kGHalf + kk * 32, 16, 1024);
+              const uint64_t bd = umma_desc_sw128(u_tile + (h * 64 + kk * 16) * 128, 16, 1024);
+              umma_bf16(tbase + kColP, ad, bd, kIdescE1, (c | h | kk) ? 1u : 0u);
+            }
+          umma_commit(&empty[s]);
+        }
+        umma_commit(p_full);
+        if (failed || !mbar_wait(pc_full, np & 1u, kWaitLimit)) { failed = 1; break; }
+        tc_fence_after();
+        // E2: W[128 x 128] = Pc_hi U_hi^T + Pc_lo U_hi^T + Pc_hi U_lo^T
+        for (int i = 0; i < nc; ++i, ++step, ++e2) {
+          const int s = step % kStages;
+          const int b = e2 & 1;
+          if (!mbar_wait(&full[s], (step / kStages) & 1u, kWaitLimit)) { failed = 1; break; }
+          if (e2 >= 2 && !mbar_wait(&w_empty[b], ((e2 >> 1) - 1) & 1u, kWaitLimit)) { failed = 1; break; }
+          tc_fence_after();
+          const uint32_t u_tile = sbase + s * kStageBytes + kGBytes;
+          const uint32_t d = tbase + (b ? kColW1 : kColW0);
+          const int ak[6] = {0, 16, 32, 48, 0, 16};   // Pc: hi = k 0..31, lo = k 32..63
+          const int bk[6] = {0, 16, 0, 16, 32, 48};   // U : hi = k 0..31, lo = k 32..63
+#pragma unroll
+          for (int q = 0; q < 6; ++q) {
+            const uint64_t ad = umma_desc_sw128(pc_tile + ak[q] * 2, 16, 1024);
+            const uint64_t bd = umma_desc_sw128(u_tile + bk[q] * 2, 16, 1024);
+            umma_bf16(d, ad, bd, kIdescE2, q ? 1u : 0u);
+          }
+          umma_commit(&w_full[b]);
+        }
+      }
+    }
+  } else {
+    // ---------------- epilogue: warps 0-3, thread = row ----------------
+    const int r = threadIdx.x;                 // 0..127
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    uint32_t step = 0, e2 = 0, np = 0;
+    bool stop = false;  // group vote: set for all 128 threads at the same barrier
+    for (int it = beg; it < end && !stop; ++it, ++np) {
+      const int jb = p.sched_ids[it] >> 8, panel = p.sched_ids[it] & 255;
+      const EncJob& J = p.jobs[jb];
+      const int nc = J.d_in / kChunk;
+      // transform coefficients of this layer (fp64, rounded once)
+      float cf[32];
+      const double rho = (double)__ldg(J.rho);
+      const double a64 = 1.0 / sqrt(rho);
+      const float a = (float)a64;
+#pragma unroll
+      for (int k = 0; k < 32; ++k)
+        cf[k] = k < J.rank ? (float)(1.0 / sqrt((double)__ldg(J.lambda + k) + rho) - a64) : 0.0f;
+      // P o c, split into the bf16 A operand of E2
+      stop = named_sync_or(2, 128, !mbar_wait(p_full, np & 1u, kWaitLimit));
+      if (stop) {
+        failed = 1;
+        break;
+      }
+      tc_fence_after();
+      uint32_t pr[64];
+      tmem_ld32(tbase + lane_off + kColP, pr);
+      tmem_ld32(tbase + lane_off + kColP + 32, pr + 32);
+      tmem_wait_ld();
+      uint32_t hi[16], lo[16];
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        const float v0 = (__uint_as_float(pr[2 * k]) + __uint_as_float(pr[32 + 2 * k])) * cf[2 * k];
+        const float v1 = (__uint_as_float(pr[2 * k + 1]) + __uint_as_float(pr[33 + 2 * k])) * cf[2 * k + 1];
+        float h0, l0, h1, l1;
+        split_bf16(v0, h0, l0);
+        split_bf16(v1, h1, l1);
+        hi[k] = pack_bf16x2(h0, h1);
+        lo[k] = pack_bf16x2(l0, l1);
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        st_shared_v4(pc_tile + sw128(r, q), hi[4 * q], hi[4 * q + 1], hi[4 * q + 2], hi[4 * q + 3]);
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        st_shared_v4(pc_tile + sw128(r, 4 + q), lo[4 * q], lo[4 * q + 1], lo[4 * q + 2], lo[4 * q + 3]);
+      fence_async_shared();
+      tc_fence_before();
+      mbar_arrive(pc_full);
+      step += nc;  // the E1 steps
+      const int64_t row = (int64_t)panel * kPanel + r;
+      const bool live = row < J.d_out;
+      for (int i = 0; i < nc; ++i, ++step, ++e2) {
+        const int c = nc - 1 - i;
+        const int s = step % kStages;
+        const int b = e2 & 1;
+        stop = named_sync_or(2, 128, !mbar_wait(&w_full[b], (e2 >> 1) & 1u, kWaitLimit));
+        if (stop) {
+          failed = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t wcol = tbase + lane_off + (b ? kColW1 : kColW0);
+        const uint32_t g_tile = sbase + s * kStageBytes;
+        // pass 1: block maximum of w = a g + acc
+        float amax = 0.0f;
+#pragma unroll
+        for (int g4 = 0; g4 < 4; ++g4) {
+          uint32_t acc[32];
+          tmem_ld32(wcol + g4 * 32, acc);
+          tmem_wait_ld();
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int qq = g4 * 4 + q;                       // 16-byte chunk of the 256-byte row
+            const uint4 gv = ld_shared_v4(g_tile + (qq >> 3) * kGHalf + sw128(r, qq & 7));
+            const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float w0 = fmaf(a, bf16lo(gw[e]), __uint_as_float(acc[q * 8 + 2 * e]));
+              const float w1 = fmaf(a, bf16hi(gw[e]), __uint_as_float(acc[q * 8 + 2 * e + 1]));
+              amax = fmaxf(amax, fmaxf(fabsf(w0), fabsf(w1)));
+            }
+          }
+        }
+        const float inv = e4m3_inv_scale(amax);
+        // pass 2: codes
+        uint8_t* dst = J.codes + row * J.d_in + c * kChunk;
+#pragma unroll
+        for (int g4 = 0; g4 < 4; ++g4) {
+          uint32_t acc[32];
+          tmem_ld32(wcol + g4 * 32, acc);
+          tmem_wait_ld();
+          uint32_t cw[8];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int qq = g4 * 4 + q;
+            const uint4 gv = ld_shared_v4(g_tile + (qq >> 3) * kGHalf + sw128(r, qq & 7));
+            const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const float w0 = fmaf(a, bf16lo(gw[2 * e]), __uint_as_float(acc[q * 8 + 4 * e]));
+              const float w1 = fmaf(a, bf16hi(gw[2 * e]), __uint_as_float(acc[q * 8 + 4 * e + 1]));
+              const float w2 = fmaf(a, bf16lo(gw[2 * e + 1]), __uint_as_float(acc[q * 8 + 4 * e + 2]));
+              const float w3 = fmaf(a, bf16hi(gw[2 * e + 1]), __uint_as_float(acc[q * 8 + 4 * e + 3]));
+              const uint32_t c01 = f32x2_to_e4m3x2(__fmul_rn(w0, inv), __fmul_rn(w1, inv));
+              const uint32_t c23 = f32x2_to_e4m3x2(__fmul_rn(w2, inv), __fmul_rn(w3, inv));
+              cw[q * 2 + e] = inv > 0.0f ? (c01 | (c23 << 16)) : 0u;
+            }
+          }
+          if (live) {
+            *reinterpret_cast<uint4*>(dst + g4 * 32) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+            *reinterpret_cast<uint4*>(dst + g4 * 32 + 16) = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+          }
+        }
+        if (live) J.scales[row * (J.d_in / kChunk) + c] = e4m3_scale(amax, inv);
+        tc_fence_before();
+        mbar_arrive(&w_empty[b]);
+        named_sync(2, 128);
+        if (r == 0) mbar_arrive(&empty[s]);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) tmem_dealloc(tbase, kTmemCols);
+  if (threadIdx.x == 0 && failed && err) atomicOr(err, GIFT_DEV_TIMEOUT);
+}
+
+unsigned long long g_enc_attr = 0;
+
+// Longest-processing-time-first assignment of panels to CTAs.
+int schedule(const TcLayer* layers, int n, uint16_t* off, uint16_t* ids, int max_ids) {
+  struct Item {
+    int cost;
+    uint16_t id;
+  };
+  std::vector<Item> items;
+  for (int l = 0; l < n; ++l) {
+    const int np = (layers[l].d_out + kPanel - 1) / kPanel;
+    for (int q = 0; q < np; ++q) items.push_back({layers[l].d_in / kChunk, (uint16_t)((l << 8) | q)});
+  }
+  if ((int)items.size() > max_ids) return -1;
+  std::stable_sort(items.begin(), items.end(), [](const Item& x, const Item& y) { return x.cost > y.cost; });
+  const int grid = std::min<int>(kNumSMs, (int)items.size());
+  std::vector<std::vector<uint16_t>> per(grid);
+  using E = std::pair<long, int>;
+  std::priority_queue<E, std::vector<E>, std::greater<E>> heap;
+  for (int b = 0; b < grid; ++b) heap.push({0, b});
+  for (const Item& it : items) {
+    E e = heap.top();
+    heap.pop();
+    per[e.second].push_back(it.id);
+    heap.push({e.first + it.cost, e.second});
+  }
+  int k = 0;
+  for (int b = 0; b < grid; ++b) {
+    off[b] = (uint16_t)k;
+    for (uint16_t id : per[b]) ids[k++] = id;
+  }
+  off[grid] = (uint16_t)k;
+  return grid;
+}
+
+}  // namespace
+
+bool tc_codec_available() { return tmap_encoder() != nullptr; }
+
+cudaError_t launch_whiten_encode_tc(const TcLayer* layers, int n, cudaStream_t s) {
+  cudaError_t e = ensure_smem_attr(whiten_encode_tc_kernel, kSmemBytes, &g_enc_attr);
+  if (e != cudaSuccess) return e;
+  for (int base = 0; base < n;) {
+    // pack as many layers as fit one launch
+    int cnt = 0, panels = 0;
+    while (base + cnt < n && cnt < kMaxJobs) {
+      const int np = (layers[base + cnt].d_out + kPanel - 1) / kPanel;
+      if (np > 256 || panels + np > kMaxPanels) break;
+      panels += np;
+      ++cnt;
+    }
+    if (cnt == 0) {
+      // a single layer with more than 256 panels: split it by rows
+      const TcLayer& L = layers[base];
+      const int rows = 256 * kPanel;
+      for (int r0 = 0; r0 < L.d_out; r0 += rows) {
+        TcLayer part = L;
+        part.d_out = std::min(rows, L.d_out - r0);
+        part.G = (const __nv_bfloat16*)L.G + (int64_t)r0 * L.d_in;
+        part.codes = L.codes + (int64_t)r0 * L.d_in;
+        part.scales = L.scales + (int64_t)r0 * (L.d_in / kChunk);
+        if ((e = launch_whiten_encode_tc(&part, 1, s)) != cudaSuccess) return e;
+      }
+      ++base;
+      continue;
+    }
+    static thread_local EncParams P;
+    for (int l = 0; l < cnt; ++l) {
+      const TcLayer& L = layers[base + l];
+      EncJob& J = P.jobs[l];
+      if (!make_tmap_2d(&J.tmG, L.G, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)L.d_out, (uint64_t)L.d_in,
+                        kPanel, 64))
+        return cudaErrorInvalidValue;
+      J.U = L.U;
+      J.lambda = L.lambda;
+      J.rho = L.rho;
+      J.codes = L.codes;
+      J.scales = L.scales;
+      J.d_out = L.d_out;
+      J.d_in = L.d_in;
+      J.rank = L.rank;
+    }
+    const int grid = schedule(layers + base, cnt, P.sched_off, P.sched_ids, kMaxPanels);
+    if (grid <= 0) return cudaErrorInvalidValue;
+    whiten_encode_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(P, nullptr);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    base += cnt;
+  }
+  return cudaSuccess;
+}
+
 cudaError_t launch_whiten_decode_tc(const TcLayer*, int, cudaStream_t) { return cudaErrorNotSupported; }
 
 }  // namespace gift

@@ -2,7 +2,11 @@
 
 Criteria: A entries within 1e-5 of max|A| (fp32 accumulation of exact bf16/fp32
 products); the top-32 Ritz values within 1e-4 relative (same algorithm, same
-SplitMix64 start block); rho within 1e-4 relative; U orthonormal to 1e-5;
+SplitMix64 start block); U orthonormal to 1e-5; rho within 1e-4 relative or
+within the fp32-accumulation bound of its numerator: rho = (tr A - sum
+lambda)/(d - r) is a small difference of two sums of size tr A, and A's
+diagonal carries the rounding of an fp32 sum over N tokens, about
+2^-24 sqrt(N) relative, so |d rho| <= 2^-24 sqrt(N) tr(A) / (d - r);
 the Ritz property U^T A U = diag(lambda) on the oracle's fp64 A.  The
 transform M is compared in relative Frobenius norm within 1e-2: after four
 iterations the Ritz vectors next to the rank cut (lambda_32 vs lambda_33)
@@ -35,12 +39,16 @@ def _refresh_both(X, rank=32, over=16, iters=4, seed=7, dtype="f32"):
             lam.cpu().numpy().astype(np.float64), float(rho.item()), int(st.item())), (A, Uo, lo, ro, fo)
 
 
-def _check(gpu, orc, m_tol=1e-2):
+def rho_tol(rho, trace, N, d, r):
+    return max(1e-4 * rho, 2.0 ** -24 * np.sqrt(N) * trace / (d - r))
+
+
+def _check(gpu, orc, N, m_tol=1e-2):
     Ag, Ug, lg, rg, sg = gpu
     A, Uo, lo, ro, fo = orc
     assert np.max(np.abs(Ag - A)) <= 1e-5 * np.max(np.abs(A))
     assert np.allclose(lg, lo, rtol=1e-4, atol=0)
-    assert rg == pytest.approx(ro, rel=1e-4)
+    assert abs(rg - ro) <= rho_tol(ro, np.trace(A), N, A.shape[0], Ug.shape[1]), (rg, ro)
     assert (sg & ops.DEV_RHO_FLOORED) == (fo & 1)
     r = Ug.shape[1]
     assert np.max(np.abs(Ug.T @ Ug - np.eye(r))) < 1e-5
@@ -56,7 +64,7 @@ def test_refresh_config1_fp32():
     Q = synth.haar_orthogonal(512, 1003)
     X = synth.activations(2048, Q, synth.column_power(512, 1.0), 1001)
     g, o = _refresh_both(X, dtype="f32", seed=1004)
-    _check(g, o)
+    _check(g, o, 2048)
 
 
 def test_refresh_bf16_spiked_spectrum():
@@ -65,7 +73,7 @@ def test_refresh_bf16_spiked_spectrum():
     Q = synth.haar_orthogonal(d, 11)
     X = synth.activations(4096, Q, synth.spectrum_power(d, 1.2, 5, 100.0), 12)
     g, o = _refresh_both(X, dtype="bf16", seed=13)
-    _check(g, o)
+    _check(g, o, 4096)
 
 
 @pytest.mark.parametrize("rank,over,iters", [(8, 8, 2), (32, 0, 3), (16, 17, 1)])
@@ -74,7 +82,7 @@ def test_refresh_rank_and_oversample_variants(rank, over, iters):
     Q = synth.haar_orthogonal(d, 21)
     X = synth.activations(1024, Q, synth.spectrum_power(d, 2.0), 22)
     g, o = _refresh_both(X, rank, over, iters, seed=23)
-    _check(g, o, m_tol=5e-2)
+    _check(g, o, 1024, m_tol=5e-2)
 
 
 def test_refresh_rank_deficient_input_sets_status():
@@ -108,7 +116,7 @@ def test_refresh_config2_bf16_split_k():
     Q = synth.haar_orthogonal(1536, 2003)
     X = synth.activations(8192, Q, synth.column_power(1536, 1.0), 2001)
     g, o = _refresh_both(X, dtype="bf16", seed=2004)
-    _check(g, o)
+    _check(g, o, 8192)
 
 
 def test_refresh_config4_full_size_properties():
@@ -153,6 +161,4 @@ def test_refresh_config4_full_size_properties():
     rho_ref = (fro / N - np.trace(R)) / (d - 32)
     rel = abs(rho.item() - rho_ref) / rho_ref
     print(f"config4 rho {rho.item():.6e} vs trace identity {rho_ref:.6e} (rel {rel:.2e}); lambda_1 {lg[0]:.4f}")
-    # rho is a difference of two ~500-sized sums that leaves ~1.5: the fp32
-    # accumulation of A's diagonal (~1e-6 relative) is amplified ~300x.
-    assert rel < 1e-3
+    assert abs(rho.item() - rho_ref) <= rho_tol(rho_ref, fro / N, N, d, 32)
