@@ -162,8 +162,13 @@ def build_workload(torch, ops, synth, dev, depth, seed):
         off += n
     ews = torch.empty((max(ops.error_workspace_size(4096, 4096), 16),), device=dev, dtype=torch.uint8)
     err = torch.empty((3,), device=dev, dtype=torch.float64)
+    wl = [L for L in layers if L.rank > 0]
+    el = [L for L in layers if L.rank == 0]
     return dict(layers=layers, whitened=whitened, G_all=G_all, Gh_all=Gh_all, C_all=C_all, S_all=S_all,
-                n_el=n_el, packed=ops.make_layers(layers), ews=ews, err=err)
+                n_el=n_el, ews=ews, err=err,
+                n_wh=sum(L.d_out * L.d_in for L in wl), n_eu=sum(L.d_out * L.d_in for L in el),
+                packed_wh=ops.make_layers(wl), n_packed_wh=len(wl),
+                packed_eu=ops.make_layers(el), n_packed_eu=len(el))
 
 
 def refresh(ops, w, stream=None):
@@ -172,30 +177,39 @@ def refresh(ops, w, stream=None):
                        out=(L.U, L.lam, L.rho), stream=stream)
 
 
+PHASES = ("refresh", "encode_euclid", "encode_whitened", "decode_euclid", "decode_whitened", "error")
+
+
 def step(ops, W, k, ev=None):
-    """One step; if `ev` (list of 5 events) is given, phase boundaries are recorded."""
+    """One step: refresh one whitened layer, encode and decode all 96 gradients
+    (each codec phase is one grouped launch), round-trip error of that layer.
+    If `ev` (len(PHASES)+1 events) is given, phase boundaries are recorded."""
     w = W["whitened"][k % len(W["whitened"])]
-    if ev:
-        ev[0].record()
+    rec = (lambda i: ev[i].record()) if ev else (lambda i: None)
+    rec(0)
     refresh(ops, w)
-    if ev:
-        ev[1].record()
-    ops.encode_many(W["packed"], len(W["layers"]))
-    if ev:
-        ev[2].record()
-    ops.decode_many(W["packed"], len(W["layers"]))
-    if ev:
-        ev[3].record()
+    rec(1)
+    ops.encode_many(W["packed_eu"], W["n_packed_eu"])
+    rec(2)
+    ops.encode_many(W["packed_wh"], W["n_packed_wh"])
+    rec(3)
+    ops.decode_many(W["packed_eu"], W["n_packed_eu"])
+    rec(4)
+    ops.decode_many(W["packed_wh"], W["n_packed_wh"])
+    rec(5)
     L = w["layer"]
     ops.roundtrip_error(L.G, L.G_hat, out=W["err"], ws=W["ews"])
-    if ev:
-        ev[4].record()
+    rec(6)
 
 
-def algorithmic_bytes(W):
-    """Per step: encode reads G (2 B) and writes codes (1 B) + scales (4/128 B); decode the reverse."""
-    n = W["n_el"]
-    return n * (2 + 1 + 4 / 128), n * (1 + 4 / 128 + 2)
+def phase_bytes(W):
+    """Algorithmic bytes of each codec launch: encode reads G (2 B/element) and
+    writes codes (1 B) + scales (4/128 B); decode the reverse; plus U per layer."""
+    enc = 2 + 1 + 4 / 128
+    dec = 1 + 4 / 128 + 2
+    u_bytes = sum(w["layer"].d_in * RANK * 4 for w in W["whitened"])
+    return {"encode_euclid": W["n_eu"] * enc, "encode_whitened": W["n_wh"] * enc + u_bytes,
+            "decode_euclid": W["n_eu"] * dec, "decode_whitened": W["n_wh"] * dec + u_bytes}
 
 
 def count_launches(torch, ops, W):
@@ -274,7 +288,7 @@ def run_gpu(args):
 
     # ---- timed region: device resident inputs (1.06 GB of G > 126 MB L2) ----
     K = args.steps
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(PHASES) + 1)] for _ in range(K)]
     clocks = ClockSampler(local)
     barrier()
     torch.cuda.synchronize()
@@ -289,7 +303,8 @@ def run_gpu(args):
     barrier()
     clock_info = clocks.stop()
     ms_total = t0.elapsed_time(t1)
-    phase = np.array([[e[i].elapsed_time(e[i + 1]) for i in range(4)] for e in evs])  # refresh, enc, dec, err
+    phase = np.array([[e[i].elapsed_time(e[i + 1]) for i in range(len(PHASES))] for e in evs])
+    pm = {n: float(phase[:, i].mean()) for i, n in enumerate(PHASES)}
     if world > 1:
         t = torch.tensor([ms_total], device=dev, dtype=torch.float64)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -298,20 +313,19 @@ def run_gpu(args):
     g_bytes = W["n_el"] * 2
     value = world * g_bytes / (ms_step * 1e-3) / 1e9
 
-    enc_b, dec_b = algorithmic_bytes(W)
-    enc_ms, dec_ms = phase[:, 1].mean(), phase[:, 2].mean()
+    pb = phase_bytes(W)
     peak, peak_kind = measured_peaks()
-    dom = "encode" if enc_ms >= dec_ms else "decode"
-    dom_ms = max(enc_ms, dec_ms)
-    dom_b = enc_b if dom == "encode" else dec_b
-    achieved = dom_b / (dom_ms * 1e-3) / 1e9
-    roofline = {"bound": "hbm", "kernel": f"grouped {dom} over the 96-tensor stack", "achieved": achieved,
-                "peak": peak, "peak_source": peak_kind, "unit": "GB/s", "frac": achieved / peak, "traffic": None}
-    codec_ms = enc_ms + dec_ms
-    codec = {"encode_ms": enc_ms, "decode_ms": dec_ms, "refresh_ms": phase[:, 0].mean(),
-             "error_ms": phase[:, 3].mean(),
+    dom = max(pb, key=lambda n: pm[n])
+    achieved = pb[dom] / (pm[dom] * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "kernel": f"{dom} (one grouped launch over its layers of the stack)",
+                "achieved": achieved, "peak": peak, "peak_source": peak_kind, "unit": "GB/s",
+                "frac": achieved / peak, "traffic": None}
+    codec_ms = sum(pm[n] for n in pb)
+    codec = {"phase_ms": pm,
+             "phase_gbs": {n: pb[n] / (pm[n] * 1e-3) / 1e9 for n in pb},
+             "phase_roofline_frac": {n: pb[n] / (pm[n] * 1e-3) / 1e9 / peak for n in pb},
              "codec_gradient_gbs": g_bytes / (codec_ms * 1e-3) / 1e9,
-             "codec_roofline_frac": (enc_b + dec_b) / (codec_ms * 1e-3) / 1e9 / peak}
+             "codec_roofline_frac": sum(pb.values()) / (codec_ms * 1e-3) / 1e9 / peak}
 
     launches, names = count_launches(torch, ops, W)
 

@@ -164,14 +164,15 @@ static gift_status run_many(const gift_layer* layers, int n, gift_stream_t strea
   if (st != GIFT_OK) return st;
   cudaStream_t s = (cudaStream_t)stream;
   std::vector<TcLayer> tc;
+  std::vector<EuclidLayer> eu[2];  // by dtype
   for (int i = 0; i < n; ++i) {
     const gift_layer& L = layers[i];
     if (L.d_out == 0) continue;
     cudaError_t e = cudaSuccess;
     const int64_t nb = L.d_out * (L.d_in / GIFT_E4M3_BLOCK);
     if (L.rank == 0) {
-      e = encode ? launch_euclid_encode(L.G, (gift_dtype)L.dtype, nb, L.codes, L.scales, s)
-                 : launch_euclid_decode(L.codes, L.scales, nb, L.G_hat, (gift_dtype)L.dtype, s);
+      eu[L.dtype].push_back(encode ? EuclidLayer{L.G, L.codes, L.scales, nb}
+                                   : EuclidLayer{L.codes, L.G_hat, L.scales, nb});
     } else if (use_tc(L.dtype, L.rank, L.d_in)) {
       tc.push_back(TcLayer{L.G, L.G_hat, L.codes, L.scales, L.U, L.lambda, L.rho, (int)L.d_out, (int)L.d_in, L.rank});
     } else {
@@ -182,6 +183,10 @@ static gift_status run_many(const gift_layer* layers, int n, gift_stream_t strea
     }
     if (e != cudaSuccess) return GIFT_ERR_CUDA;
   }
+  for (int dt = 0; dt < 2; ++dt)
+    if (!eu[dt].empty() &&
+        launch_euclid_group(eu[dt].data(), (int)eu[dt].size(), (gift_dtype)dt, encode, s) != cudaSuccess)
+      return GIFT_ERR_CUDA;
   if (!tc.empty()) {
     cudaError_t e = encode ? launch_whiten_encode_tc(tc.data(), (int)tc.size(), s)
                            : launch_whiten_decode_tc(tc.data(), (int)tc.size(), s);

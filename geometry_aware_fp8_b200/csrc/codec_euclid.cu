@@ -123,6 +123,83 @@ __global__ void __launch_bounds__(256) euclid_decode_kernel(const uint8_t* __res
   }
 }
 
+// Grouped form: many layers in one launch.  A block index b of the
+// concatenated layers is mapped to its layer by a search over the prefix
+// sums of the layers' block counts (kept in shared memory).
+constexpr int kGroupMax = 64;
+
+struct EuclidGroup {
+  const void* src[kGroupMax];   // encode: G; decode: codes
+  void* dst[kGroupMax];         // encode: codes; decode: G_hat
+  float* scales[kGroupMax];
+  int64_t prefix[kGroupMax + 1];  // prefix[i] = first block of layer i
+  int n;
+};
+
+GIFT_DEV int find_layer(const int64_t* pre, int n, int64_t b) {
+  int lo = 0, hi = n - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (pre[mid] <= b) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) euclid_encode_group_kernel(const __grid_constant__ EuclidGroup g) {
+  __shared__ int64_t pre[kGroupMax + 1];
+  for (int i = threadIdx.x; i <= g.n; i += blockDim.x) pre[i] = g.prefix[i];
+  __syncthreads();
+  const int sub = threadIdx.x & 7;
+  const int64_t total = pre[g.n];
+  const int64_t groups_per_grid = (int64_t)gridDim.x * (blockDim.x >> 3);
+  for (int64_t b = (int64_t)blockIdx.x * (blockDim.x >> 3) + (threadIdx.x >> 3); b < total; b += groups_per_grid) {
+    const int l = find_layer(pre, g.n, b);
+    const int64_t lb = b - pre[l];
+    const int64_t e0 = lb * kBlock + sub * 16;
+    float v[16];
+    Vec16<T>::load((const T*)g.src[l] + e0, v);
+    float m = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[i]));
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+    const float inv = e4m3_inv_scale(m);
+    __stcs(reinterpret_cast<uint4*>((uint8_t*)g.dst[l] + e0), quantize16(v, inv));
+    if (sub == 0) g.scales[l][lb] = e4m3_scale(m, inv);
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) euclid_decode_group_kernel(const __grid_constant__ EuclidGroup g) {
+  __shared__ int64_t pre[kGroupMax + 1];
+  for (int i = threadIdx.x; i <= g.n; i += blockDim.x) pre[i] = g.prefix[i];
+  __syncthreads();
+  const int sub = threadIdx.x & 7;
+  const int64_t total = pre[g.n];
+  const int64_t groups_per_grid = (int64_t)gridDim.x * (blockDim.x >> 3);
+  for (int64_t b = (int64_t)blockIdx.x * (blockDim.x >> 3) + (threadIdx.x >> 3); b < total; b += groups_per_grid) {
+    const int l = find_layer(pre, g.n, b);
+    const int64_t lb = b - pre[l];
+    const int64_t e0 = lb * kBlock + sub * 16;
+    const uint4 q = __ldcs(reinterpret_cast<const uint4*>((const uint8_t*)g.src[l] + e0));
+    const float s = __ldg(g.scales[l] + lb);
+    uint32_t w[4] = {q.x, q.y, q.z, q.w};
+    float v[16];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float2 a = e4m3x2_to_f32x2((uint16_t)(w[i] & 0xFFFF));
+      float2 c = e4m3x2_to_f32x2((uint16_t)(w[i] >> 16));
+      v[4 * i] = a.x * s;
+      v[4 * i + 1] = a.y * s;
+      v[4 * i + 2] = c.x * s;
+      v[4 * i + 3] = c.y * s;
+    }
+    Vec16<T>::store((T*)g.dst[l] + e0, v);
+  }
+}
+
 inline int grid_for(int64_t n_blocks) {
   // 8 blocks per 256-thread CTA; up to 8 resident CTAs per SM.
   int64_t need = (n_blocks + 31) / 32;  // four blocks of work per group
@@ -153,6 +230,36 @@ cudaError_t launch_euclid_decode(const uint8_t* codes, const float* scales, int6
   else
     euclid_decode_kernel<float><<<grid, 256, 0, s>>>(codes, scales, (float*)G_hat, n_blocks);
   return cudaGetLastError();
+}
+
+cudaError_t launch_euclid_group(const EuclidLayer* layers, int n, gift_dtype dt, bool encode, cudaStream_t s) {
+  for (int base = 0; base < n; base += kGroupMax) {
+    const int cnt = n - base < kGroupMax ? n - base : kGroupMax;
+    EuclidGroup g;
+    g.n = cnt;
+    int64_t tot = 0;
+    for (int i = 0; i < cnt; ++i) {
+      const EuclidLayer& L = layers[base + i];
+      g.src[i] = L.src;
+      g.dst[i] = L.dst;
+      g.scales[i] = L.scales;
+      g.prefix[i] = tot;
+      tot += L.n_blocks;
+    }
+    g.prefix[cnt] = tot;
+    if (tot == 0) continue;
+    const int grid = grid_for(tot);
+    if (encode) {
+      if (dt == GIFT_BF16) euclid_encode_group_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(g);
+      else euclid_encode_group_kernel<float><<<grid, 256, 0, s>>>(g);
+    } else {
+      if (dt == GIFT_BF16) euclid_decode_group_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(g);
+      else euclid_decode_group_kernel<float><<<grid, 256, 0, s>>>(g);
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 }  // namespace gift

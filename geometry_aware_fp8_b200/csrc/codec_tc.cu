@@ -390,6 +390,320 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
   if (threadIdx.x == 0 && failed && err) atomicOr(err, GIFT_DEV_TIMEOUT);
 }
 
+// ===========================================================================
+// Decode: G_hat = W_hat M^{-1},  W_hat = value(codes) * scale (per block),
+//   M^{-1} = a I + U diag(c) U^T,  a = rho^{1/2},  c_k = (lambda_k+rho)^{1/2} - a.
+//   D2  P = W_hat U = sum_c s_c (q_c U_c): the codes q are exact in bf16, so
+//       each chunk's product T_c = q_c [U_hi | U_lo] (M=128, N=64, K=128) is
+//       scaled by its block scale in the epilogue and summed in fp32.
+//   D3  G_hat = a W_hat + (P o c) U^T   (M=128, N=128 per chunk, K=32, split
+//       as in the encoder), bf16 output with round-to-nearest-even.
+// Stage = codes tile (TMA, [128][128 B], 128-byte swizzle) + bf16 copy of the
+// codes (the D2 A operand, written by the converter warps) + U tile.
+// ===========================================================================
+constexpr int kDStages = 3;
+constexpr int kDCodes = kPanel * kChunk;            // 16 KB
+constexpr int kDQ = kPanel * kChunk * 2;            // 32 KB: two [128][64] bf16 tiles
+constexpr int kDStageBytes = kDCodes + kDQ + kUBytes;
+constexpr int kDSmemBytes = kDStages * kDStageBytes + kPcBytes + 1024 + 512;
+static_assert(kDSmemBytes <= 232448, "decode shared memory");
+static_assert(kSmemBytes <= 232448, "encode shared memory");
+constexpr uint32_t kColT0 = 256, kColT1 = 320;
+constexpr uint32_t kIdescD2 = umma_idesc_bf16(128, 64, 0, 1);
+
+struct alignas(64) DecJob {
+  CUtensorMap tmC;  // uint8 codes [d_out][d_in], box [128][128], 128-byte swizzle
+  const float* U;
+  const float* lambda;
+  const float* rho;
+  const float* scales;
+  __nv_bfloat16* out;
+  int d_out, d_in, rank, pad;
+};
+
+struct DecParams {
+  DecJob jobs[kMaxJobs];
+  uint16_t sched_off[kNumSMs + 1];
+  uint16_t sched_ids[kMaxPanels];
+};
+
+// E4M3 pair -> bf16 pair (exact: every E4M3 value is a bf16 value)
+GIFT_DEV uint32_t e4m3x2_to_bf16x2(uint16_t v) {
+  const float2 f = e4m3x2_to_f32x2(v);
+  return pack_bf16x2(f.x, f.y);
+}
+
+__global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __grid_constant__ DecParams p,
+                                                                     uint32_t* err) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t pc_tile = sbase + kDStages * kDStageBytes;
+  uint64_t* bars = (uint64_t*)(smem + kDStages * kDStageBytes + kPcBytes);
+  uint64_t* full = bars;                   // [kDStages] count 1: converter (U tile, bf16 codes)
+  uint64_t* cfull = bars + kDStages;       // [kDStages] count 1 + tx: codes TMA
+  uint64_t* empty = bars + 2 * kDStages;   // [kDStages] count 1
+  uint64_t* t_full = bars + 3 * kDStages;  // [2] count 1
+  uint64_t* t_empty = t_full + 2;          // [2] count 128
+  uint64_t* pc_full = t_full + 4;          // count 128
+  uint64_t* w_full = t_full + 5;           // [2] count 1
+  uint64_t* w_empty = t_full + 7;          // [2] count 128
+  uint32_t* tmem_slot = (uint32_t*)(t_full + 9);
+  __shared__ int failed;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int beg = p.sched_off[blockIdx.x], end = p.sched_off[blockIdx.x + 1];
+  if (threadIdx.x == 0) {
+    failed = 0;
+    for (int s = 0; s < kDStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&cfull[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&t_full[b], 1);
+      mbar_init(&t_empty[b], 128);
+      mbar_init(&w_full[b], 1);
+      mbar_init(&w_empty[b], 128);
+    }
+    mbar_init(pc_full, 128);
+    fence_mbar_init();
+  }
+  if (warp == 8) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+
+  if (warp >= 4 && warp < 8) {
+    // ---------------- producer: TMA for codes, U tile, bf16 codes tile ----------------
+    const int t = threadIdx.x - 128;
+    uint32_t step = 0;
+    bool stop = false;
+    for (int it = beg; it < end && !stop; ++it) {
+      const int jb = p.sched_ids[it] >> 8, panel = p.sched_ids[it] & 255;
+      const DecJob& J = p.jobs[jb];
+      const int nc = J.d_in / kChunk;
+      for (int pass = 0; pass < 2 && !stop; ++pass) {
+        for (int i = 0; i < nc; ++i, ++step) {
+          const int c = pass == 0 ? i : nc - 1 - i;
+          const int s = step % kDStages;
+          const uint32_t use = step / kDStages;
+          const bool ok = step < kDStages || mbar_wait(&empty[s], (use - 1) & 1u, kWaitLimit);
+          stop = named_sync_or(1, 128, !ok);
+          if (stop) {
+            failed = 1;
+            break;
+          }
+          const uint32_t c_tile = sbase + s * kDStageBytes;
+          const uint32_t q_tile = c_tile + kDCodes;
+          const uint32_t u_tile = q_tile + kDQ;
+          if (t == 0) {
+            mbar_arrive_expect_tx(&cfull[s], kDCodes);
+            tma_load_2d(smem + s * kDStageBytes, &J.tmC, &cfull[s], c * kChunk, panel * kPanel);
+          }
+          convert_u_tile(J.U, J.rank, c * kChunk, u_tile, t);
+          if (pass == 0) {
+            // the codes of row t: wait for the TMA, then widen to bf16
+            if (!mbar_wait(&cfull[s], use & 1u, kWaitLimit)) failed = 1;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const uint4 v = ld_shared_v4(c_tile + sw128(t, q));
+              const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+              uint32_t o[8];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                o[2 * e] = e4m3x2_to_bf16x2((uint16_t)(w[e] & 0xFFFFu));
+                o[2 * e + 1] = e4m3x2_to_bf16x2((uint16_t)(w[e] >> 16));
+              }
+              // 16 codes -> 32 bytes of bf16 = chunks 2q, 2q+1 of the 256-byte row
+              const int c0 = 2 * q, c1 = 2 * q + 1;
+              st_shared_v4(q_tile + (c0 >> 3) * kGHalf + sw128(t, c0 & 7), o[0], o[1], o[2], o[3]);
+              st_shared_v4(q_tile + (c1 >> 3) * kGHalf + sw128(t, c1 & 7), o[4], o[5], o[6], o[7]);
+            }
+          }
+          fence_async_shared();
+          named_sync(1, 128);
+          if (t == 0) mbar_arrive(&full[s]);
+        }
+      }
+    }
+  } else if (warp == 8) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      uint32_t step = 0, e2 = 0, d2 = 0, np = 0;
+      for (int it = beg; it < end && !failed; ++it, ++np) {
+        const DecJob& J = p.jobs[p.sched_ids[it] >> 8];
+        const int nc = J.d_in / kChunk;
+        // D2: T_c[128 x 64] = q_c . [U_hi | U_lo]
+        for (int c = 0; c < nc; ++c, ++step, ++d2) {
+          const int s = step % kDStages;
+          const int b = d2 & 1;
+          if (!mbar_wait(&full[s], (step / kDStages) & 1u, kWaitLimit)) { failed = 1; break; }
+          if (d2 >= 2 && !mbar_wait(&t_empty[b], ((d2 >> 1) - 1) & 1u, kWaitLimit)) { failed = 1; break; }
+          tc_fence_after();
+          const uint32_t q_tile = sbase + s * kDStageBytes + kDCodes, u_tile = q_tile + kDQ;
+          const uint32_t d = tbase + (b ? kColT1 : kColT0);
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t ad = umma_desc_sw128(q_tile + h * kGHalf + kk * 32, 16, 1024);
+              const uint64_t bd = umma_desc_sw128(u_tile + (h * 64 + kk * 16) * 128, 16, 1024);
+              umma_bf16(d, ad, bd, kIdescD2, (h | kk) ? 1u : 0u);
+            }
+          umma_commit(&empty[s]);
+          umma_commit(&t_full[b]);
+        }
+        if (failed || !mbar_wait(pc_full, np & 1u, kWaitLimit)) { failed = 1; break; }
+        tc_fence_after();
+        // D3: W[128 x 128] = Pc . U^T (three split products)
+        for (int i = 0; i < nc; ++i, ++step, ++e2) {
+          const int s = step % kDStages;
+          const int b = e2 & 1;
+          if (!mbar_wait(&full[s], (step / kDStages) & 1u, kWaitLimit)) { failed = 1; break; }
+          if (e2 >= 2 && !mbar_wait(&w_empty[b], ((e2 >> 1) - 1) & 1u, kWaitLimit)) { failed = 1; break; }
+          tc_fence_after();
+          const uint32_t u_tile = sbase + s * kDStageBytes + kDCodes + kDQ;
+          const uint32_t d = tbase + (b ? kColW1 : kColW0);
+          const int ak[6] = {0, 16, 32, 48, 0, 16};
+          const int bk[6] = {0, 16, 0, 16, 32, 48};
+#pragma unroll
+          for (int q = 0; q < 6; ++q) {
+            const uint64_t ad = umma_desc_sw128(pc_tile + ak[q] * 2, 16, 1024);
+            const uint64_t bd = umma_desc_sw128(u_tile + bk[q] * 2, 16, 1024);
+            umma_bf16(d, ad, bd, kIdescE2, q ? 1u : 0u);
+          }
+          umma_commit(&w_full[b]);
+        }
+      }
+    }
+  } else {
+    // ---------------- epilogue: warps 0-3, thread = row ----------------
+    const int r = threadIdx.x;
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    uint32_t step = 0, e2 = 0, d2 = 0, np = 0;
+    bool stop = false;
+    for (int it = beg; it < end && !stop; ++it, ++np) {
+      const int jb = p.sched_ids[it] >> 8, panel = p.sched_ids[it] & 255;
+      const DecJob& J = p.jobs[jb];
+      const int nc = J.d_in / kChunk;
+      const int64_t row = (int64_t)panel * kPanel + r;
+      const bool live = row < J.d_out;
+      const float* srow = J.scales + (live ? row : 0) * nc;
+      float cf[32];
+      const double rho = (double)__ldg(J.rho);
+      const double a64 = sqrt(rho);
+      const float a = (float)a64;
+#pragma unroll
+      for (int k = 0; k < 32; ++k)
+        cf[k] = k < J.rank ? (float)(sqrt((double)__ldg(J.lambda + k) + rho) - a64) : 0.0f;
+      // D2 epilogue: P += s_c (T_hi + T_lo)
+      float P[32];
+#pragma unroll
+      for (int k = 0; k < 32; ++k) P[k] = 0.0f;
+      for (int c = 0; c < nc; ++c, ++step, ++d2) {
+        const int b = d2 & 1;
+        stop = named_sync_or(2, 128, !mbar_wait(&t_full[b], (d2 >> 1) & 1u, kWaitLimit));
+        if (stop) {
+          failed = 1;
+          break;
+        }
+        tc_fence_after();
+        uint32_t tr[64];
+        const uint32_t tcol = tbase + lane_off + (b ? kColT1 : kColT0);
+        tmem_ld32(tcol, tr);
+        tmem_ld32(tcol + 32, tr + 32);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(&t_empty[b]);
+        const float sc = live ? __ldg(srow + c) : 0.0f;
+#pragma unroll
+        for (int k = 0; k < 32; ++k) P[k] = fmaf(sc, __uint_as_float(tr[k]) + __uint_as_float(tr[32 + k]), P[k]);
+      }
+      if (stop) break;
+      // P o c -> bf16 hi/lo A operand of D3
+      uint32_t hi[16], lo[16];
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        float h0, l0, h1, l1;
+        split_bf16(P[2 * k] * cf[2 * k], h0, l0);
+        split_bf16(P[2 * k + 1] * cf[2 * k + 1], h1, l1);
+        hi[k] = pack_bf16x2(h0, h1);
+        lo[k] = pack_bf16x2(l0, l1);
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        st_shared_v4(pc_tile + sw128(r, q), hi[4 * q], hi[4 * q + 1], hi[4 * q + 2], hi[4 * q + 3]);
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        st_shared_v4(pc_tile + sw128(r, 4 + q), lo[4 * q], lo[4 * q + 1], lo[4 * q + 2], lo[4 * q + 3]);
+      fence_async_shared();
+      mbar_arrive(pc_full);
+      // D3 epilogue: G_hat = a s q + acc
+      for (int i = 0; i < nc; ++i, ++step, ++e2) {
+        const int c = nc - 1 - i;
+        const int s = step % kDStages;
+        const int b = e2 & 1;
+        const bool ok = mbar_wait(&w_full[b], (e2 >> 1) & 1u, kWaitLimit) &&
+                        mbar_wait(&cfull[s], (step / kDStages) & 1u, kWaitLimit);
+        stop = named_sync_or(2, 128, !ok);
+        if (stop) {
+          failed = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t wcol = tbase + lane_off + (b ? kColW1 : kColW0);
+        const uint32_t c_tile = sbase + s * kDStageBytes;
+        const float as = a * (live ? __ldg(srow + c) : 0.0f);
+        __nv_bfloat16* dst = J.out + row * J.d_in + c * kChunk;
+#pragma unroll
+        for (int g4 = 0; g4 < 4; ++g4) {
+          uint32_t acc[32];
+          tmem_ld32(wcol + g4 * 32, acc);
+          tmem_wait_ld();
+          // codes 32*g4 .. 32*g4+31 of this row: two 16-byte chunks
+          uint32_t o[16];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const uint4 v = ld_shared_v4(c_tile + sw128(r, 2 * g4 + h));
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f0 = e4m3x2_to_f32x2((uint16_t)(w[e] & 0xFFFFu));
+              const float2 f1 = e4m3x2_to_f32x2((uint16_t)(w[e] >> 16));
+              const int k = h * 16 + e * 4;
+              o[h * 8 + 2 * e] = pack_bf16x2(fmaf(as, f0.x, __uint_as_float(acc[k])),
+                                             fmaf(as, f0.y, __uint_as_float(acc[k + 1])));
+              o[h * 8 + 2 * e + 1] = pack_bf16x2(fmaf(as, f1.x, __uint_as_float(acc[k + 2])),
+                                                 fmaf(as, f1.y, __uint_as_float(acc[k + 3])));
+            }
+          }
+          if (live) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst + g4 * 32);
+            d4[0] = make_uint4(o[0], o[1], o[2], o[3]);
+            d4[1] = make_uint4(o[4], o[5], o[6], o[7]);
+            d4[2] = make_uint4(o[8], o[9], o[10], o[11]);
+            d4[3] = make_uint4(o[12], o[13], o[14], o[15]);
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&w_empty[b]);
+        named_sync(2, 128);
+        if (r == 0) mbar_arrive(&empty[s]);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) tmem_dealloc(tbase, kTmemCols);
+  if (threadIdx.x == 0 && failed && err) atomicOr(err, GIFT_DEV_TIMEOUT);
+}
+
+unsigned long long g_dec_attr = 0;
 unsigned long long g_enc_attr = 0;
 
 // Longest-processing-time-first assignment of panels to CTAs.
@@ -481,6 +795,56 @@ cudaError_t launch_whiten_encode_tc(const TcLayer* layers, int n, cudaStream_t s
   return cudaSuccess;
 }
 
-cudaError_t launch_whiten_decode_tc(const TcLayer*, int, cudaStream_t) { return cudaErrorNotSupported; }
+
+
+cudaError_t launch_whiten_decode_tc(const TcLayer* layers, int n, cudaStream_t s) {
+  cudaError_t e = ensure_smem_attr(whiten_decode_tc_kernel, kDSmemBytes, &g_dec_attr);
+  if (e != cudaSuccess) return e;
+  for (int base = 0; base < n;) {
+    int cnt = 0, panels = 0;
+    while (base + cnt < n && cnt < kMaxJobs) {
+      const int np = (layers[base + cnt].d_out + kPanel - 1) / kPanel;
+      if (np > 256 || panels + np > kMaxPanels) break;
+      panels += np;
+      ++cnt;
+    }
+    if (cnt == 0) {
+      const TcLayer& L = layers[base];
+      const int rows = 256 * kPanel;
+      for (int r0 = 0; r0 < L.d_out; r0 += rows) {
+        TcLayer part = L;
+        part.d_out = std::min(rows, L.d_out - r0);
+        part.G_hat = (__nv_bfloat16*)L.G_hat + (int64_t)r0 * L.d_in;
+        part.codes = L.codes + (int64_t)r0 * L.d_in;
+        part.scales = L.scales + (int64_t)r0 * (L.d_in / kChunk);
+        if ((e = launch_whiten_decode_tc(&part, 1, s)) != cudaSuccess) return e;
+      }
+      ++base;
+      continue;
+    }
+    static thread_local DecParams P;
+    for (int l = 0; l < cnt; ++l) {
+      const TcLayer& L = layers[base + l];
+      DecJob& J = P.jobs[l];
+      if (!make_tmap_2d(&J.tmC, L.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)L.d_out, (uint64_t)L.d_in,
+                        kPanel, kChunk))
+        return cudaErrorInvalidValue;
+      J.U = L.U;
+      J.lambda = L.lambda;
+      J.rho = L.rho;
+      J.scales = L.scales;
+      J.out = (__nv_bfloat16*)L.G_hat;
+      J.d_out = L.d_out;
+      J.d_in = L.d_in;
+      J.rank = L.rank;
+    }
+    const int grid = schedule(layers + base, cnt, P.sched_off, P.sched_ids, kMaxPanels);
+    if (grid <= 0) return cudaErrorInvalidValue;
+    whiten_decode_tc_kernel<<<grid, kThreads, kDSmemBytes, s>>>(P, nullptr);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    base += cnt;
+  }
+  return cudaSuccess;
+}
 
 }  // namespace gift

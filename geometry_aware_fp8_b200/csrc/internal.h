@@ -16,6 +16,15 @@ cudaError_t launch_euclid_encode(const void* G, gift_dtype dt, int64_t n_blocks,
 cudaError_t launch_euclid_decode(const uint8_t* codes, const float* scales, int64_t n_blocks, void* G_hat,
                                  gift_dtype dt, cudaStream_t s);
 
+// Grouped Euclidean codec: one launch for many rank-0 layers of one dtype.
+struct EuclidLayer {
+  const void* src;   // encode: G;     decode: codes
+  void* dst;         // encode: codes; decode: G_hat
+  float* scales;
+  int64_t n_blocks;  // d_out * d_in / 128
+};
+cudaError_t launch_euclid_group(const EuclidLayer* layers, int n, gift_dtype dt, bool encode, cudaStream_t s);
+
 // ---- Whitened codec on CUDA cores (any rank <= 32, fp32 or bf16) ----
 cudaError_t launch_whiten_encode_simt(const void* G, gift_dtype dt, int64_t d_out, int64_t d_in, const float* U,
                                       const float* lambda, const float* rho, int rank, uint8_t* codes,

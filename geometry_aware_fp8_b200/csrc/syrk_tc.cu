@@ -11,10 +11,14 @@
 // from X's rows: X[n][i] has i contiguous, so A-operand (M = i) and
 // B-operand (N = j) are MN-major 128-byte-swizzled tiles, one 64-column box
 // per 64 features.  One CTA per (tile, token split):
-//   warp 4     TMA producer (4-stage ring, 48 KB per stage)
-//   warp 5     TMEM allocation and the single-thread MMA issue
-//   warps 0-3  epilogue: TMEM -> registers -> A (j >= i only, mirrored),
+//   warp 8     TMA producer (4-stage ring, 48 KB per stage)
+//   warp 9     TMEM allocation and the single-thread MMA issue
+//   warps 0-7  epilogue: TMEM -> registers -> A (j >= i only, mirrored),
 //              or raw partial sums when the token range is split.
+// The tensor core's fp32 accumulation drifts low over long chains (measured
+// ~3e-4 relative after 65536 tokens in one accumulator), so each TMEM
+// accumulator only sums 2048 tokens; two accumulators alternate and the
+// epilogue adds the blocks in fp32 registers with round-to-nearest.
 #include "common.cuh"
 #include "internal.h"
 #include "tma_host.h"
@@ -31,7 +35,9 @@ constexpr int B_BYTES = BN * BK * 2;             // four 64-feature boxes
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;   // 48 KB
 constexpr int BOX_BYTES = 64 * BK * 2;           // 8 KB: 64 tokens x 128 B
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
-constexpr uint32_t TMEM_COLS = 256;
+constexpr uint32_t TMEM_COLS = 512;   // two 256-column accumulators
+constexpr int KB = 32;                // 64-token chunks per TMEM accumulation block (2048 tokens)
+constexpr int THREADS = 320;
 constexpr uint32_t IDESC = umma_idesc_bf16(BM, BN, /*a MN-major*/ 1, /*b MN-major*/ 1);
 constexpr uint32_t kWaitLimit = 1u << 22;
 
@@ -57,13 +63,14 @@ __device__ void tile_of(int t, int d, int* I, int* J2) {
   *J2 = i / 2 + t;
 }
 
-__global__ void __launch_bounds__(192, 1) syrk_tc_kernel(const __grid_constant__ CUtensorMap tmX, SyrkArgs a) {
+__global__ void __launch_bounds__(THREADS, 1) syrk_tc_kernel(const __grid_constant__ CUtensorMap tmX, SyrkArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint64_t* full = (uint64_t*)(smem + STAGES * STAGE_BYTES);
   uint64_t* empty = full + STAGES;
-  uint64_t* acc_full = empty + STAGES;
-  uint32_t* tmem_slot = (uint32_t*)(acc_full + 1);
+  uint64_t* acc_full = empty + STAGES;   // [2] count 1
+  uint64_t* acc_empty = acc_full + 2;    // [2] count 256
+  uint32_t* tmem_slot = (uint32_t*)(acc_full + 4);
   __shared__ int failed;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -81,10 +88,13 @@ __global__ void __launch_bounds__(192, 1) syrk_tc_kernel(const __grid_constant__
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(acc_full, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 256);
+    }
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(tmem_slot, TMEM_COLS);
     tmem_relinquish();
   }
@@ -93,7 +103,7 @@ __global__ void __launch_bounds__(192, 1) syrk_tc_kernel(const __grid_constant__
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
 
-  if (warp == 4) {
+  if (warp == 8) {
     if (lane == 0) {
       tma_prefetch_desc(&tmX);
       for (int k = 0; k < nk; ++k) {
@@ -113,12 +123,17 @@ __global__ void __launch_bounds__(192, 1) syrk_tc_kernel(const __grid_constant__
         for (int b = 0; b < 4; ++b) tma_load_2d(sb + b * BOX_BYTES, &tmX, &full[s], J2 * BN + b * 64, y);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     if (lane == 0) {
       for (int k = 0; k < nk; ++k) {
         const int s = k % STAGES;
         const uint32_t ph = (uint32_t)(k / STAGES) & 1u;
+        const int bk = k / KB, b = bk & 1;
         if (!mbar_wait(&full[s], ph, kWaitLimit)) {
+          failed = 1;
+          break;
+        }
+        if (k % KB == 0 && bk >= 2 && !mbar_wait(&acc_empty[b], ((bk >> 1) - 1) & 1u, kWaitLimit)) {
           failed = 1;
           break;
         }
@@ -130,33 +145,46 @@ __global__ void __launch_bounds__(192, 1) syrk_tc_kernel(const __grid_constant__
           // 16 tokens = 16 rows of 128 B; MN groups (64 features) one box apart
           const uint64_t ad = umma_desc_sw128(a0 + kk * 2048, BOX_BYTES, 1024);
           const uint64_t bd = umma_desc_sw128(b0 + kk * 2048, BOX_BYTES, 1024);
-          umma_bf16(tbase, ad, bd, IDESC, (k > 0 || kk > 0) ? 1u : 0u);
+          umma_bf16(tbase + b * BN, ad, bd, IDESC, (k % KB > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(&empty[s]);
+        if (k % KB == KB - 1 || k == nk - 1) umma_commit(&acc_full[b]);
       }
-      umma_commit(acc_full);
     }
   } else {
-    // epilogue: thread = output row i, 32 columns per TMEM load
-    const bool ok = (nk == 0) || mbar_wait(acc_full, 0, kWaitLimit);
-    if (!ok) failed = 1;
-    tc_fence_after();
-    const int i = I * BM + warp * 32 + lane;
-    const uint32_t trow = tbase + ((uint32_t)(warp * 32) << 16);
-    for (int cc = 0; cc < BN / 32; ++cc) {
-      uint32_t r[32];
-      if (nk > 0) {
-        tmem_ld32(trow + cc * 32, r);
-        tmem_wait_ld();
-      } else {
+    // epilogue: warp w owns rows 32*(w%4).. (its TMEM lane quarter) and
+    // columns 128*(w/4)..+128 of the tile; blocks are summed in registers
+    const int wq = warp & 3, wh = warp >> 2;
+    float sum[128];
 #pragma unroll
-        for (int t = 0; t < 32; ++t) r[t] = 0u;
+    for (int t = 0; t < 128; ++t) sum[t] = 0.0f;
+    const int nblk = (nk + KB - 1) / KB;
+    const uint32_t trow = tbase + ((uint32_t)(wq * 32) << 16) + wh * 128;
+    for (int bk = 0; bk < nblk; ++bk) {
+      const int b = bk & 1;
+      if (!mbar_wait(&acc_full[b], (bk >> 1) & 1u, kWaitLimit)) {
+        failed = 1;
+        break;
       }
+      tc_fence_after();
 #pragma unroll
-      for (int t = 0; t < 32; ++t) {
-        const int j = J2 * BN + cc * 32 + t;
+      for (int g = 0; g < 4; ++g) {
+        uint32_t r[32];
+        tmem_ld32(trow + b * BN + g * 32, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int t = 0; t < 32; ++t) sum[g * 32 + t] += __uint_as_float(r[t]);
+      }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[b]);
+    }
+    const int i = I * BM + wq * 32 + lane;
+#pragma unroll
+    for (int t = 0; t < 128; ++t) {
+      {
+        const int j = J2 * BN + wh * 128 + t;
         if (j < i || j >= a.d) continue;
-        const float v = __uint_as_float(r[t]);
+        const float v = sum[t];
         if (a.splits == 1) {
           a.A[(int64_t)i * a.d + j] = v * a.scale;
           if (j != i) a.A[(int64_t)j * a.d + i] = v * a.scale;
@@ -168,7 +196,7 @@ __global__ void __launch_bounds__(192, 1) syrk_tc_kernel(const __grid_constant__
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) tmem_dealloc(tbase, TMEM_COLS);
+  if (warp == 9) tmem_dealloc(tbase, TMEM_COLS);
   if (threadIdx.x == 0 && failed && a.err) atomicOr(a.err, GIFT_DEV_TIMEOUT);
 }
 
@@ -202,7 +230,7 @@ cudaError_t launch_syrk_tc(const void* X, gift_dtype xdt, int64_t N, int d, floa
   a.part = part;
   a.err = err;
   const int items = syrk_tc_tiles(d) * a.splits;
-  syrk_tc_kernel<<<items, 192, SMEM_BYTES, s>>>(tm, a);
+  syrk_tc_kernel<<<items, THREADS, SMEM_BYTES, s>>>(tm, a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (a.splits > 1) e = launch_syrk_reduce(part, a.splits, d, A, a.scale, s);
