@@ -124,6 +124,25 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------
+# rank plumbing (replicas only: the one collective is the timing reduction)
+# ---------------------------------------------------------------------------
+def max_over_ranks(ms: float, device=None) -> float:
+    """Max of a per-rank device time over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return ms
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(world: int, bytes_per_rank: float, ms_per_step: float) -> float:
+    """Whole-job throughput in GB/s: every rank processes its own replica (weak scaling)."""
+    return world * bytes_per_rank / (ms_per_step * 1e-3) / 1e9
+
+
+# ---------------------------------------------------------------------------
 # GPU arm
 # ---------------------------------------------------------------------------
 def build_workload(torch, ops, synth, dev, depth, seed):
@@ -305,13 +324,10 @@ def run_gpu(args):
     ms_total = t0.elapsed_time(t1)
     phase = np.array([[e[i].elapsed_time(e[i + 1]) for i in range(len(PHASES))] for e in evs])
     pm = {n: float(phase[:, i].mean()) for i, n in enumerate(PHASES)}
-    if world > 1:
-        t = torch.tensor([ms_total], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = t.item()
+    ms_total = max_over_ranks(ms_total, dev)
     ms_step = ms_total / K
     g_bytes = W["n_el"] * 2
-    value = world * g_bytes / (ms_step * 1e-3) / 1e9
+    value = job_value(world, g_bytes, ms_step)
 
     pb = phase_bytes(W)
     peak, peak_kind = measured_peaks()
@@ -357,11 +373,7 @@ def run_gpu(args):
             e2e_step(k)
         b.record()
         torch.cuda.synchronize()
-        ms_e = a.elapsed_time(b)
-        if world > 1:
-            t = torch.tensor([ms_e], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms_e = t.item()
+        ms_e = max_over_ranks(a.elapsed_time(b), dev)
         x_bytes = sum(W["whitened"][k % 2]["X"].numel() * 2 for k in range(Ke)) / Ke
         e2e = {"value": world * g_bytes / (ms_e / Ke * 1e-3) / 1e9, "unit": UNIT,
                "h2d_bytes_per_step": int(g_bytes + x_bytes), "d2h_bytes_per_step": int(g_bytes + 24),
