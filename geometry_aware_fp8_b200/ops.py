@@ -25,7 +25,7 @@ STATUS = {0: "GIFT_OK", 1: "GIFT_ERR_INVALID_ARG", 2: "GIFT_ERR_SHAPE", 3: "GIFT
           4: "GIFT_ERR_WORKSPACE", 5: "GIFT_ERR_CUDA", 6: "GIFT_ERR_UNSUPPORTED"}
 
 EXPORTED = ("gift_status_string", "gift_version", "gift_refresh_workspace_size", "gift_factor_refresh",
-            "gift_encode", "gift_decode", "gift_encode_many", "gift_decode_many",
+            "gift_factor_refresh_noalloc", "gift_encode", "gift_decode", "gift_encode_many", "gift_decode_many",
             "gift_error_workspace_size", "gift_roundtrip_error")
 
 
@@ -61,6 +61,8 @@ def lib() -> ctypes.CDLL:
         L.gift_refresh_workspace_size.argtypes = [i64, i64, i32, i32, i32, ctypes.POINTER(sz)]
         L.gift_factor_refresh.argtypes = [vp, i32, i64, i64, i32, i32, i32, ctypes.c_uint64, vp, vp, vp, vp,
                                           vp, sz, vp, vp]
+        L.gift_factor_refresh_noalloc.argtypes = [vp, i32, i64, i64, i32, i32, i32, ctypes.c_uint64, vp, vp, vp,
+                                                  vp, vp, vp]
         L.gift_encode.argtypes = [vp, i32, i64, i64, vp, vp, vp, i32, vp, vp, vp]
         L.gift_decode.argtypes = [vp, vp, i64, i64, vp, vp, vp, i32, vp, i32, vp]
         L.gift_encode_many.argtypes = [ctypes.POINTER(Layer), i32, vp]
@@ -136,6 +138,34 @@ def factor_refresh(X: torch.Tensor, rank: int = 32, oversample: int = 16, iters:
     _check(lib().gift_factor_refresh(_ptr(X), _dt(X), N, d, rank, oversample, iters, seed & (2**64 - 1),
                                      _ptr(U), _ptr(lam), _ptr(rho), _ptr(A_out), _ptr(ws), ws.numel(),
                                      _ptr(dev_status), _stream(stream)), "gift_factor_refresh")
+    return U, lam, rho, dev_status
+
+
+def factor_refresh_noalloc(X: torch.Tensor, A_out: torch.Tensor, rank: int = 32, oversample: int = 16,
+                           iters: int = 4, seed: int = 0, dev_status: Optional[torch.Tensor] = None,
+                           stream=None, out=None):
+    """Same result as factor_refresh, for callers that cannot supply a workspace.
+
+    The library keeps the scratch in a fixed array on each GPU, so this call
+    allocates nothing on the device besides the outputs created here when
+    `out` / `dev_status` are not passed.  A_out (d_in x d_in fp32) is
+    required; d_in <= 4096 and rank + oversample <= 64.  Calls must not
+    overlap on the GPU.
+    """
+    _cuda(X, A_out, dev_status)
+    N, d = X.shape
+    dev = X.device
+    if out is None:
+        U = torch.empty((d, rank), device=dev, dtype=torch.float32)
+        lam = torch.empty((rank,), device=dev, dtype=torch.float32)
+        rho = torch.empty((1,), device=dev, dtype=torch.float32)
+    else:
+        U, lam, rho = out
+    if dev_status is None:
+        dev_status = torch.zeros((1,), device=dev, dtype=torch.int32)
+    _check(lib().gift_factor_refresh_noalloc(_ptr(X), _dt(X), N, d, rank, oversample, iters, seed & (2**64 - 1),
+                                             _ptr(U), _ptr(lam), _ptr(rho), _ptr(A_out), _ptr(dev_status),
+                                             _stream(stream)), "gift_factor_refresh_noalloc")
     return U, lam, rho, dev_status
 
 

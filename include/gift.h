@@ -106,6 +106,31 @@ gift_status gift_factor_refresh(const void* X, gift_dtype xdt, int64_t N, int64_
                                 uint32_t* dev_status, gift_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * Factor refresh without any allocation.  The paper has no counterpart: this
+ * entry point exists for callers that cannot hand the library a workspace,
+ * e.g. code whose device memory is entirely owned by another allocator, or
+ * a step that must not call cudaMalloc because it can synchronise the
+ * device.  It computes exactly what gift_factor_refresh computes, with its
+ * scratch in a fixed array inside the library (present on every GPU that
+ * loads libgift, until the process exits; nothing is allocated per call).
+ *
+ * Same arguments as gift_factor_refresh without ws/ws_bytes, except that
+ * A_out is REQUIRED (d_in x d_in fp32, written in full).  Limits:
+ * d_in <= 4096 and rank + oversample <= 64 (GIFT_ERR_SHAPE beyond them);
+ * the token range is never split, so small layers use fewer SMs than
+ * gift_factor_refresh would.
+ * Set-up: the first call on each device looks up the array's device address
+ * with that device current; make that first call before any stream capture.
+ * Every call on a device shares the one array and leaves its contents
+ * behind; no value in it needs to start at zero.  Calls whose executions
+ * overlap on the GPU (different streams, or different host threads) race
+ * on the array and produce undefined results: serialise them.
+ * ------------------------------------------------------------------------ */
+gift_status gift_factor_refresh_noalloc(const void* X, gift_dtype xdt, int64_t N, int64_t d_in, int rank,
+                                        int oversample, int iters, uint64_t seed, float* U, float* lambda,
+                                        float* rho, float* A_out, uint32_t* dev_status, gift_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * Encode (review page, "What carries the argument": whiten with the
  * input-side factor before FP8 quantisation and communication).
  *

@@ -1,0 +1,77 @@
+"""The allocation-free factor refresh against the regular one (GPU).
+
+gift_factor_refresh_noalloc serves callers that cannot give the library a
+workspace (their device memory belongs to another allocator, or they may
+not call cudaMalloc in that step).  It must return what gift_factor_refresh
+returns, within the refresh tolerances: top-32 eigenvalues within 1e-4
+relative, rho within the fp32-accumulation bound of its numerator, A within
+1e-5 of max|A|, and the transform within 1e-2 in relative Frobenius norm.
+Two calls in a row check that the shared scratch array is reused cleanly.
+This file is collected last on purpose.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import gift_oracle as O
+from geometry_aware_fp8_b200 import ops, synth
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+
+def _rho_tol(rho, trace, N, d, r):
+    return max(1e-4 * rho, 2.0 ** -24 * np.sqrt(N) * trace / (d - r))
+
+
+def _compare(ref, got, A_ref, A_got, N):
+    U0, l0, r0, _ = [t.cpu().numpy().astype(np.float64) for t in ref]
+    U1, l1, r1, s1 = [t.cpu().numpy().astype(np.float64) for t in got]
+    A0 = A_ref.cpu().numpy().astype(np.float64)
+    A1 = A_got.cpu().numpy().astype(np.float64)
+    d, r = U0.shape
+    assert np.max(np.abs(A1 - A0)) <= 1e-5 * np.max(np.abs(A0))
+    assert np.allclose(l1, l0, rtol=1e-4, atol=0)
+    assert abs(r1[0] - r0[0]) <= _rho_tol(r0[0], np.trace(A0), N, d, r)
+    M0 = O.transform_matrix(U0, l0, r0[0])
+    M1 = O.transform_matrix(U1, l1, r1[0])
+    assert np.linalg.norm(M1 - M0) / np.linalg.norm(M0) < 1e-2
+
+
+@pytest.mark.parametrize("N,d,dtype", [(8192, 1536, "bf16"), (4096, 4096, "bf16"), (2048, 512, "f32")])
+def test_noalloc_refresh_matches_regular_refresh_twice(N, d, dtype):
+    Q = synth.haar_orthogonal(d, 77 + d)
+    X = synth.to_storage(synth.activations(N, Q, synth.column_power(d, 1.0), 78), dtype)
+    Xd = torch.from_numpy(X).to(DEV)
+    if dtype == "bf16":
+        Xd = Xd.to(torch.bfloat16)
+    A_ref = torch.empty((d, d), device=DEV, dtype=torch.float32)
+    ref = ops.factor_refresh(Xd, 32, 16, 4, 9, A_out=A_ref)
+    first = None
+    for call in range(2):
+        A_got = torch.empty((d, d), device=DEV, dtype=torch.float32)
+        got = ops.factor_refresh_noalloc(Xd, A_got, 32, 16, 4, 9)
+        torch.cuda.synchronize()
+        _compare(ref, got, A_ref, A_got, N)
+        if first is None:
+            first = [t.clone() for t in got[:3]]
+        else:
+            for a, b in zip(first, got[:3]):
+                assert torch.equal(a, b)
+
+
+def test_noalloc_refresh_rejects_what_it_cannot_hold():
+    X = torch.zeros((256, 4224), device=DEV, dtype=torch.bfloat16)
+    A = torch.empty((4224, 4224), device=DEV, dtype=torch.float32)
+    with pytest.raises(ops.GiftError) as e:
+        ops.factor_refresh_noalloc(X, A, 32, 16, 4, 0)
+    assert e.value.status == 2  # GIFT_ERR_SHAPE: d_in above 4096
+    X = torch.zeros((256, 512), device=DEV, dtype=torch.bfloat16)
+    A = torch.empty((512, 512), device=DEV, dtype=torch.float32)
+    with pytest.raises(ops.GiftError) as e:
+        ops.factor_refresh_noalloc(X, A, 48, 17, 4, 0)
+    assert e.value.status == 2  # rank + oversample above 64
+    L = ops.lib()
+    st = L.gift_factor_refresh_noalloc(X.data_ptr(), 1, 256, 512, 32, 16, 4, 0, A.data_ptr(), A.data_ptr(),
+                                       A.data_ptr(), None, None, None)
+    assert st == 1  # GIFT_ERR_INVALID_ARG: A_out is required
