@@ -63,10 +63,13 @@ struct RefreshPlan {
   uint64_t seed;
   int gram_parts;       // partial Gram blocks
   int syrk_splits;      // split-K partial sums of A
+  int skinny_slices;    // k-slices of the A Q product
   // workspace carve-up (byte offsets from ws)
-  size_t off_A, off_Q, off_Y, off_gram, off_small, off_syrk, total;
+  size_t off_A, off_Q, off_Y, off_T, off_gram, off_small, off_syrk, total;
 };
-void refresh_plan(int64_t N, int64_t d, int rank, int oversample, bool a_out_given, RefreshPlan* p);
+// no_split: one token range for A and one k-slice for A Q (smallest workspace)
+void refresh_plan(int64_t N, int64_t d, int rank, int oversample, bool a_out_given, RefreshPlan* p,
+                  bool no_split = false);
 cudaError_t launch_refresh(const RefreshPlan& p, const void* X, gift_dtype xdt, float* U, float* lambda,
                            float* rho, float* A_out, void* ws, uint32_t* dev_status, cudaStream_t s);
 

@@ -10,8 +10,8 @@
 // anything.
 //
 // Limits: d_in <= 4096 and rank + oversample <= 64, which bounds the scratch
-// (sampled subspace, its image, fp64 Gram partials and the small factors)
-// at 4,259,840 bytes.  A must be given by the caller as an output buffer,
+// (sampled subspace, its image, a Cholesky-QR temporary, fp64 Gram partials
+// and the small factors) at 4,259,840 bytes.  A must be given by the caller as an output buffer,
 // and the token range is not split, so the whole scratch need is known.
 #include <mutex>
 
@@ -72,9 +72,8 @@ extern "C" gift_status gift_factor_refresh_noalloc(const void* X, gift_dtype xdt
       (dev_status && !al(dev_status, 4)))
     return GIFT_ERR_ALIGN;
   RefreshPlan p;
-  refresh_plan(N, d_in, rank, oversample, /*a_out_given=*/true, &p);
-  p.syrk_splits = 1;      // no split-K partial sums: A_out is written directly
-  p.total = p.off_syrk;   // the split-K region is never touched
+  // one token range and one k-slice: A_out is written directly, nothing is split
+  refresh_plan(N, d_in, rank, oversample, /*a_out_given=*/true, &p, /*no_split=*/true);
   if (p.total > kNoAllocScratchBytes) return GIFT_ERR_SHAPE;
   p.iters = iters;
   p.seed = seed;

@@ -12,10 +12,9 @@
 // dense steps (m x m Cholesky, Jacobi, sort) run in one CTA in fp64 shared
 // memory; Gram matrices are reduced in fp64 with a fixed order so results
 // are bit-identical from run to run.
-#include <atomic>
-
 #include "common.cuh"
 #include "internal.h"
+#include "tma_host.h"
 
 namespace gift {
 
@@ -27,7 +26,7 @@ namespace {
 
 constexpr int kRT = 256;
 constexpr double kCholTol = 1e-10;     // pivot / max diagonal below this: column dropped
-constexpr double kJacobiTol = 1e-15;   // off(B) / ||B||_F at convergence
+constexpr double kJacobiTol = 1e-14;   // off(B) / ||B||_F at convergence
 constexpr int kJacobiMaxSweeps = 40;
 
 GIFT_DEV uint64_t splitmix64(uint64_t x) {
@@ -140,112 +139,179 @@ __global__ void omega_kernel(float* __restrict__ Y, int d, int m, uint64_t seed)
   }
 }
 
-// Y = A Q (d x d times d x m, m <= 64), 32 rows of Y per CTA, fp32 in a fixed order.
+// Y = A Q (d x d times d x m, m <= 64).  64 x 64 output tiles (columns >= m
+// idle), 4 x 4 outputs per thread from float4 shared-memory loads; the k
+// range is split into `ns` slices written to Yp[slice] (fp32, fixed order);
+// consumers add the slices in index order.
+constexpr int kSkK = 32;
+
 __global__ void __launch_bounds__(kRT) skinny_kernel(const float* __restrict__ A, const float* __restrict__ Q,
-                                                     float* __restrict__ Y, int d, int m) {
-  __shared__ float As[32][64 + 4];
-  __shared__ float Qs[64][64];
-  const int r = threadIdx.x >> 3, cg = (threadIdx.x & 7) * 8;
-  const int64_t row0 = (int64_t)blockIdx.x * 32;
-  float acc[8];
+                                                     float* __restrict__ Yp, int d, int m, int kslice) {
+  __shared__ __align__(16) float As[kSkK][64 + 4];  // As[k][row]
+  __shared__ __align__(16) float Qs[kSkK][64];
+  const int row0 = blockIdx.x * 64;
+  const int k_begin = blockIdx.y * kslice;
+  const int k_end = min(d, k_begin + kslice);
+  const int ti = threadIdx.x >> 4, tj = threadIdx.x & 15;
+  float acc[4][4];
 #pragma unroll
-  for (int c = 0; c < 8; ++c) acc[c] = 0.0f;
-  for (int k0 = 0; k0 < d; k0 += 64) {
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b = 0; b < 4; ++b) acc[a][b] = 0.0f;
+  const int lr = threadIdx.x & 63, lk = (threadIdx.x >> 6) * 8;  // A loader: row lr, k lk..lk+7
+  const int qk = threadIdx.x >> 3, qc = (threadIdx.x & 7) * 8;   // Q loader: k qk, cols qc..qc+7
+  for (int k0 = k_begin; k0 < k_end; k0 += kSkK) {
     {
-      const float* src = A + (row0 + r) * d + k0 + cg;
-      float4 a = __ldg(reinterpret_cast<const float4*>(src)), b = __ldg(reinterpret_cast<const float4*>(src) + 1);
-      As[r][cg + 0] = a.x; As[r][cg + 1] = a.y; As[r][cg + 2] = a.z; As[r][cg + 3] = a.w;
-      As[r][cg + 4] = b.x; As[r][cg + 5] = b.y; As[r][cg + 6] = b.z; As[r][cg + 7] = b.w;
-    }
-    for (int e = threadIdx.x; e < 64 * 64; e += kRT) {
-      const int kk = e >> 6, c = e & 63;
-      Qs[kk][c] = (c < m) ? __ldg(Q + (int64_t)(k0 + kk) * m + c) : 0.0f;
+      const float* src = A + (int64_t)(row0 + lr) * d + k0 + lk;
+      const float4 x = __ldg(reinterpret_cast<const float4*>(src));
+      const float4 y = __ldg(reinterpret_cast<const float4*>(src) + 1);
+      As[lk + 0][lr] = x.x; As[lk + 1][lr] = x.y; As[lk + 2][lr] = x.z; As[lk + 3][lr] = x.w;
+      As[lk + 4][lr] = y.x; As[lk + 5][lr] = y.y; As[lk + 6][lr] = y.z; As[lk + 7][lr] = y.w;
+      const float* qs = Q + (int64_t)(k0 + qk) * m;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) Qs[qk][qc + e] = (qc + e < m) ? __ldg(qs + qc + e) : 0.0f;
     }
     __syncthreads();
 #pragma unroll 8
-    for (int kk = 0; kk < 64; ++kk) {
-      const float a = As[r][kk];
+    for (int kk = 0; kk < kSkK; ++kk) {
+      const float4 a4 = *reinterpret_cast<const float4*>(&As[kk][ti * 4]);
+      const float4 q4 = *reinterpret_cast<const float4*>(&Qs[kk][tj * 4]);
+      const float av[4] = {a4.x, a4.y, a4.z, a4.w}, qv[4] = {q4.x, q4.y, q4.z, q4.w};
 #pragma unroll
-      for (int c = 0; c < 8; ++c) acc[c] = fmaf(a, Qs[kk][cg + c], acc[c]);
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) acc[a][b] = fmaf(av[a], qv[b], acc[a][b]);
     }
     __syncthreads();
   }
+  float* out = Yp + (int64_t)blockIdx.y * d * m;
 #pragma unroll
-  for (int c = 0; c < 8; ++c)
-    if (cg + c < m) Y[(row0 + r) * m + cg + c] = acc[c];
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const int c = tj * 4 + b;
+      if (c < m) out[(int64_t)(row0 + ti * 4 + a) * m + c] = acc[a][b];
+    }
 }
 
-// part[p] = Ya[rows of p]^T Yb[rows of p] (m x m, fp64), 64 rows per part.
-__global__ void __launch_bounds__(kRT) gram_partial_kernel(const float* __restrict__ Ya,
-                                                           const float* __restrict__ Yb, int d, int m,
+// Element (row, c) of a matrix stored as `ns` slices to be added (stride d*m).
+GIFT_DEV float sliced(const float* __restrict__ Y, int ns, int64_t stride, int64_t idx) {
+  float v = Y[idx];
+  for (int s = 1; s < ns; ++s) v += Y[s * stride + idx];
+  return v;
+}
+
+// part[p] = Ya[rows of p]^T Yb[rows of p] (m x m, fp64), kGramRows rows per
+// part, staged through shared memory 64 rows at a time.  Thread (ti, tj) of
+// a 16 x 16 grid owns the 4 x 4 block of entries (4 ti.., 4 tj..).  Ya and Yb
+// may be split into na / nb slices that are added on load.
+constexpr int kGramRows = 128;
+
+__global__ void __launch_bounds__(kRT) gram_partial_kernel(const float* __restrict__ Ya, int na,
+                                                           const float* __restrict__ Yb, int nb, int d, int m,
                                                            double* __restrict__ part) {
-  __shared__ float Sa[64][64];
-  __shared__ float Sb[64][64];
+  __shared__ __align__(16) float Sa[64][64];
+  __shared__ __align__(16) float Sb[64][64];
   const int p = blockIdx.x;
-  const int r0 = p * 64;
-  const int rows = min(64, d - r0);
-  for (int e = threadIdx.x; e < 64 * m; e += kRT) {
-    const int rr = e / m, c = e % m;
-    Sa[rr][c] = rr < rows ? Ya[(int64_t)(r0 + rr) * m + c] : 0.0f;
-    Sb[rr][c] = rr < rows ? Yb[(int64_t)(r0 + rr) * m + c] : 0.0f;
+  const int ti = threadIdx.x >> 4, tj = threadIdx.x & 15;
+  const int64_t stride = (int64_t)d * m;
+  double acc[4][4];
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b = 0; b < 4; ++b) acc[a][b] = 0.0;
+  for (int r0 = p * kGramRows; r0 < min(d, (p + 1) * kGramRows); r0 += 64) {
+    const int rows = min(64, d - r0);
+    __syncthreads();
+    for (int e = threadIdx.x; e < 64 * 64; e += kRT) {
+      const int rr = e >> 6, c = e & 63;
+      const bool in = rr < rows && c < m;
+      const int64_t idx = (int64_t)(r0 + rr) * m + c;
+      Sa[rr][c] = in ? sliced(Ya, na, stride, idx) : 0.0f;
+      Sb[rr][c] = in ? sliced(Yb, nb, stride, idx) : 0.0f;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int rr = 0; rr < 64; ++rr) {
+      const float4 va = *reinterpret_cast<const float4*>(&Sa[rr][ti * 4]);
+      const float4 vb = *reinterpret_cast<const float4*>(&Sb[rr][tj * 4]);
+      const double a4[4] = {va.x, va.y, va.z, va.w};
+      const double b4[4] = {vb.x, vb.y, vb.z, vb.w};
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) acc[a][b] = fma(a4[a], b4[b], acc[a][b]);
+    }
   }
-  __syncthreads();
-  for (int e = threadIdx.x; e < m * m; e += kRT) {
-    const int i = e / m, j = e % m;
-    double acc = 0.0;
-    for (int rr = 0; rr < 64; ++rr) acc = fma((double)Sa[rr][i], (double)Sb[rr][j], acc);
-    part[(int64_t)p * m * m + e] = acc;
-  }
+  const int mm = m * m;
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const int i = ti * 4 + a, j = tj * 4 + b;
+      if (i < m && j < m) part[(int64_t)p * mm + i * m + j] = acc[a][b];
+    }
 }
 
-// Sum the Gram partials, Cholesky-factor in fp64 (dropping columns whose
-// pivot vanishes), and write R^{-1} (m x m, upper) with dropped columns zeroed.
-__global__ void __launch_bounds__(kRT) chol_kernel(const double* __restrict__ part, int nparts, int m,
+// Fixed-order sum of the Gram partials of entry e (loads issued ahead).
+GIFT_DEV double sum_parts(const double* __restrict__ part, int nparts, int mm, int e) {
+  double g = 0.0;
+#pragma unroll 8
+  for (int p = 0; p < nparts; ++p) g += __ldg(part + (int64_t)p * mm + e);
+  return g;
+}
+
+constexpr int kST = 1024;  // threads of the single-CTA small-matrix kernels
+
+// Sum the Gram partials (all threads), Cholesky-factor in fp64 (one warp;
+// a column whose pivot falls below kCholTol of the largest diagonal entry
+// is dropped), and write R^{-1} (m x m, upper) with dropped columns zeroed.
+__global__ void __launch_bounds__(kST) chol_kernel(const double* __restrict__ part, int nparts, int m,
                                                    double* __restrict__ Rinv, uint32_t* __restrict__ dev_status) {
   extern __shared__ double sm[];
-  double* Gs = sm;                  // m x m (lower Cholesky factor in place)
-  double* Li = sm + 64 * 65;        // m x m, L^{-1}
-  __shared__ int defic[64];
-  __shared__ double maxdiag;
-  __shared__ int bad;
   const int ld = 65;
+  double* Gs = sm;            // m x m (lower Cholesky factor in place)
+  double* Li = sm + 64 * ld;  // m x m, L^{-1}
+  __shared__ int defic[64];
+  __shared__ int bad;
   if (threadIdx.x == 0) bad = 0;
   __syncthreads();
-  for (int e = threadIdx.x; e < m * m; e += kRT) {
-    double g = 0.0;
-    for (int p = 0; p < nparts; ++p) g += part[(int64_t)p * m * m + e];
+  for (int e = threadIdx.x; e < m * m; e += kST) {
+    const double g = sum_parts(part, nparts, m * m, e);
     if (!isfinite(g)) bad = 1;
     Gs[(e / m) * ld + e % m] = g;
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
     double mx = 0.0;
-    for (int i = 0; i < m; ++i) mx = fmax(mx, Gs[i * ld + i]);
-    maxdiag = mx;
+    for (int i = lane; i < m; i += 32) mx = fmax(mx, Gs[i * ld + i]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    for (int j = 0; j < m; ++j) {
+      const double piv = Gs[j * ld + j];
+      const bool ok = piv > kCholTol * mx;
+      const double Ljj = ok ? sqrt(piv) : 1.0;
+      __syncwarp();
+      if (lane == 0) {
+        Gs[j * ld + j] = Ljj;
+        defic[j] = ok ? 0 : 1;
+      }
+      for (int i = j + 1 + lane; i < m; i += 32) Gs[i * ld + j] = ok ? Gs[i * ld + j] / Ljj : 0.0;
+      __syncwarp();
+      const int rem = m - j - 1;
+      for (int e = lane; e < rem * rem; e += 32) {
+        const int i = j + 1 + e / rem, k = j + 1 + e % rem;
+        if (k <= i) Gs[i * ld + k] -= Gs[i * ld + j] * Gs[k * ld + j];
+      }
+      __syncwarp();
+    }
   }
   __syncthreads();
-  for (int j = 0; j < m; ++j) {
-    if (threadIdx.x == 0) {
-      const double piv = Gs[j * ld + j];
-      const bool ok = piv > kCholTol * maxdiag;
-      defic[j] = ok ? 0 : 1;
-      Gs[j * ld + j] = ok ? sqrt(piv) : 1.0;
-    }
-    __syncthreads();
-    const double Ljj = Gs[j * ld + j];
-    for (int i = j + 1 + threadIdx.x; i < m; i += kRT) Gs[i * ld + j] = defic[j] ? 0.0 : Gs[i * ld + j] / Ljj;
-    __syncthreads();
-    const int rem = m - j - 1;
-    for (int e = threadIdx.x; e < rem * rem; e += kRT) {
-      const int i = j + 1 + e / rem, k = j + 1 + e % rem;
-      if (k <= i) Gs[i * ld + k] -= Gs[i * ld + j] * Gs[k * ld + j];
-    }
-    __syncthreads();
-  }
   // L^{-1} column by column (forward substitution), one thread per column
   if (threadIdx.x < m) {
     const int c = threadIdx.x;
-    for (int i = 0; i < m; ++i) Li[i * ld + c] = 0.0;
+    for (int i = 0; i < c; ++i) Li[i * ld + c] = 0.0;
     for (int i = c; i < m; ++i) {
       double x = (i == c) ? 1.0 : 0.0;
       for (int k = c; k < i; ++k) x -= Gs[i * ld + k] * Li[k * ld + c];
@@ -254,7 +320,7 @@ __global__ void __launch_bounds__(kRT) chol_kernel(const double* __restrict__ pa
   }
   __syncthreads();
   // R = L^T, so R^{-1} = (L^{-1})^T; zero dropped columns so those Q columns are 0
-  for (int e = threadIdx.x; e < m * m; e += kRT) {
+  for (int e = threadIdx.x; e < m * m; e += kST) {
     const int k = e / m, c = e % m;
     Rinv[e] = defic[c] ? 0.0 : Li[c * ld + k];
   }
@@ -267,15 +333,17 @@ __global__ void __launch_bounds__(kRT) chol_kernel(const double* __restrict__ pa
   }
 }
 
-// Qo = Yi R^{-1} (row by row, fp64 accumulation), 4 rows per CTA.
-__global__ void __launch_bounds__(kRT) qr_apply_kernel(const float* __restrict__ Yi, const double* __restrict__ Rinv,
-                                                       float* __restrict__ Qo, int d, int m) {
+// Qo = Yi R^{-1} (row by row, fp64 accumulation), 4 rows per CTA; Yi may be
+// split into ns slices.
+__global__ void __launch_bounds__(kRT) qr_apply_kernel(const float* __restrict__ Yi, int ns,
+                                                       const double* __restrict__ Rinv, float* __restrict__ Qo,
+                                                       int d, int m) {
   __shared__ double Rs[64 * 64];
   __shared__ double Ys[4][64];
   for (int e = threadIdx.x; e < m * m; e += kRT) Rs[e] = Rinv[e];
   const int rr = threadIdx.x >> 6, c = threadIdx.x & 63;
   const int64_t row = (int64_t)blockIdx.x * 4 + rr;
-  if (row < d && c < m) Ys[rr][c] = (double)Yi[row * m + c];
+  if (row < d && c < m) Ys[rr][c] = (double)sliced(Yi, ns, (int64_t)d * m, row * m + c);
   __syncthreads();
   if (row < d && c < m) {
     double acc = 0.0;
@@ -284,65 +352,74 @@ __global__ void __launch_bounds__(kRT) qr_apply_kernel(const float* __restrict__
   }
 }
 
-// Rayleigh-Ritz on B = Q^T (A Q): fp64 Jacobi (parallel round-robin order),
-// eigenvalues sorted descending, lambda/rho written, sorted vectors to Vs.
-__global__ void __launch_bounds__(kRT) rr_kernel(const double* __restrict__ part, int nparts, int m, int r,
+// Rayleigh-Ritz on B = Q^T (A Q): fp64 Jacobi in parallel round-robin order.
+// Each round: the 2x2 rotations of the disjoint pairs are computed, then the
+// whole of B' = J^T B J and V' = V J is written to the other buffer from the
+// coefficient form (every entry depends on its own and its partner's row and
+// column only).  Eigenvalues are sorted descending; lambda, rho and the
+// sorted eigenvectors (Vs, m x r) are written.
+__global__ void __launch_bounds__(kST) rr_kernel(const double* __restrict__ part, int nparts, int m, int r,
                                                  const float* __restrict__ A, int d, double* __restrict__ Vs,
                                                  float* __restrict__ lambda, float* __restrict__ rho,
                                                  uint32_t* __restrict__ dev_status) {
   extern __shared__ double sm[];
   const int ld = 65;
-  double* B = sm;              // m x m
-  double* V = sm + 64 * ld;    // m x m
-  __shared__ double rc[32], rs[32];
-  __shared__ int rp[32], rq[32];
-  __shared__ double red[kRT];
+  double* Bb[2] = {sm, sm + 64 * ld};
+  double* Vb[2] = {sm + 2 * 64 * ld, sm + 3 * 64 * ld};
+  __shared__ double cself[64], cpart[64];
+  __shared__ int partner[64];
+  __shared__ double red[kST / 32];
   __shared__ int order[64];
   __shared__ int stop;
-  for (int e = threadIdx.x; e < m * m; e += kRT) {
-    double g = 0.0;
-    for (int p = 0; p < nparts; ++p) g += part[(int64_t)p * m * m + e];
-    B[(e / m) * ld + e % m] = g;
-    V[(e / m) * ld + e % m] = (e / m == e % m) ? 1.0 : 0.0;
+  for (int e = threadIdx.x; e < m * m; e += kST) {
+    Bb[0][(e / m) * ld + e % m] = sum_parts(part, nparts, m * m, e);
+    Vb[0][(e / m) * ld + e % m] = (e / m == e % m) ? 1.0 : 0.0;
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < m * m; e += kRT) {
+  for (int e = threadIdx.x; e < m * m; e += kST) {  // symmetrise
     const int i = e / m, j = e % m;
     if (i < j) {
-      const double s = 0.5 * (B[i * ld + j] + B[j * ld + i]);
-      B[i * ld + j] = s;
-      B[j * ld + i] = s;
+      const double v = 0.5 * (Bb[0][i * ld + j] + Bb[0][j * ld + i]);
+      Bb[0][i * ld + j] = v;
+      Bb[0][j * ld + i] = v;
     }
   }
   __syncthreads();
+  int cur = 0;
   const int mp = m + (m & 1);  // even count for the round-robin tournament
   const int npairs = mp / 2;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int sweep = 0; sweep < kJacobiMaxSweeps; ++sweep) {
     // convergence: off(B)^2 <= tol^2 ||B||_F^2
     double off = 0.0, tot = 0.0;
-    for (int e = threadIdx.x; e < m * m; e += kRT) {
-      const double b = B[(e / m) * ld + e % m];
+    for (int e = threadIdx.x; e < m * m; e += kST) {
+      const double b = Bb[cur][(e / m) * ld + e % m];
       tot += b * b;
       if (e / m != e % m) off += b * b;
     }
-    red[threadIdx.x] = off;
+    off = warp_sum(off);
+    tot = warp_sum(tot);
+    if (lane == 0) red[warp] = off;
     __syncthreads();
-    for (int o = kRT / 2; o > 0; o >>= 1) {
-      if (threadIdx.x < o) red[threadIdx.x] += red[threadIdx.x + o];
-      __syncthreads();
+    if (threadIdx.x == 0) {
+      double o = 0.0;
+      for (int w = 0; w < kST / 32; ++w) o += red[w];
+      red[0] = o;
     }
+    __syncthreads();
     const double off_all = red[0];
     __syncthreads();
-    red[threadIdx.x] = tot;
+    if (lane == 0) red[warp] = tot;
     __syncthreads();
-    for (int o = kRT / 2; o > 0; o >>= 1) {
-      if (threadIdx.x < o) red[threadIdx.x] += red[threadIdx.x + o];
-      __syncthreads();
+    if (threadIdx.x == 0) {
+      double t = 0.0;
+      for (int w = 0; w < kST / 32; ++w) t += red[w];
+      stop = (off_all <= kJacobiTol * kJacobiTol * t) ? 1 : 0;
     }
-    if (threadIdx.x == 0) stop = (off_all <= kJacobiTol * kJacobiTol * red[0]) ? 1 : 0;
     __syncthreads();
     if (stop) break;
     for (int round = 0; round < mp - 1; ++round) {
+      const double* B = Bb[cur];
       if (threadIdx.x < npairs) {
         const int i = threadIdx.x;
         auto pos = [&](int k) { return k == 0 ? 0 : 1 + (k - 1 + round) % (mp - 1); };
@@ -365,40 +442,31 @@ __global__ void __launch_bounds__(kRT) rr_kernel(const double* __restrict__ part
             c = 1.0 / sqrt(t * t + 1.0);
             s = t * c;
           }
+          // new p = c p - s q ; new q = s p + c q
+          cself[p] = c; cpart[p] = -s; partner[p] = q;
+          cself[q] = c; cpart[q] = s;  partner[q] = p;
+        } else if (p < m) {
+          cself[p] = 1.0; cpart[p] = 0.0; partner[p] = p;
         }
-        rc[i] = c;
-        rs[i] = s;
-        rp[i] = p;
-        rq[i] = q;
       }
       __syncthreads();
-      // rows: B[p,:], B[q,:]
-      for (int e = threadIdx.x; e < npairs * m; e += kRT) {
-        const int i = e / m, k = e % m;
-        const int p = rp[i], q = rq[i];
-        if (q >= m) continue;
-        const double c = rc[i], s = rs[i];
-        const double bp = B[p * ld + k], bq = B[q * ld + k];
-        B[p * ld + k] = c * bp - s * bq;
-        B[q * ld + k] = s * bp + c * bq;
+      double* Bn = Bb[cur ^ 1];
+      const double* V = Vb[cur];
+      double* Vn = Vb[cur ^ 1];
+      for (int e = threadIdx.x; e < m * m; e += kST) {
+        const int i = e / m, j = e % m;
+        const int pi = partner[i], pj = partner[j];
+        const double si = cself[i], ti = cpart[i], sj = cself[j], tj = cpart[j];
+        Bn[i * ld + j] = si * (sj * B[i * ld + j] + tj * B[i * ld + pj]) +
+                         ti * (sj * B[pi * ld + j] + tj * B[pi * ld + pj]);
+        Vn[i * ld + j] = sj * V[i * ld + j] + tj * V[i * ld + pj];
       }
       __syncthreads();
-      // columns: B[:,p], B[:,q] and V[:,p], V[:,q]
-      for (int e = threadIdx.x; e < npairs * m; e += kRT) {
-        const int i = e / m, k = e % m;
-        const int p = rp[i], q = rq[i];
-        if (q >= m) continue;
-        const double c = rc[i], s = rs[i];
-        const double bp = B[k * ld + p], bq = B[k * ld + q];
-        B[k * ld + p] = c * bp - s * bq;
-        B[k * ld + q] = s * bp + c * bq;
-        const double vp = V[k * ld + p], vq = V[k * ld + q];
-        V[k * ld + p] = c * vp - s * vq;
-        V[k * ld + q] = s * vp + c * vq;
-      }
-      __syncthreads();
+      cur ^= 1;
     }
   }
+  const double* B = Bb[cur];
+  const double* V = Vb[cur];
   // sort eigenvalues descending (ties by index)
   if (threadIdx.x < m) {
     const int i = threadIdx.x;
@@ -412,22 +480,22 @@ __global__ void __launch_bounds__(kRT) rr_kernel(const double* __restrict__ part
   }
   // trace(A) in a fixed order
   double tr = 0.0;
-  for (int i = threadIdx.x; i < d; i += kRT) tr += (double)A[(int64_t)i * d + i];
-  red[threadIdx.x] = tr;
+  for (int i = threadIdx.x; i < d; i += kST) tr += (double)A[(int64_t)i * d + i];
+  tr = warp_sum(tr);
   __syncthreads();
-  for (int o = kRT / 2; o > 0; o >>= 1) {
-    if (threadIdx.x < o) red[threadIdx.x] += red[threadIdx.x + o];
-    __syncthreads();
-  }
-  for (int e = threadIdx.x; e < m * r; e += kRT) {
+  if (lane == 0) red[warp] = tr;
+  __syncthreads();
+  for (int e = threadIdx.x; e < m * r; e += kST) {
     const int j = e / r, k = e % r;
     Vs[e] = V[j * ld + order[k]];
   }
   if (threadIdx.x == 0) {
+    double trace = 0.0;
+    for (int w = 0; w < kST / 32; ++w) trace += red[w];
     double sum = 0.0;
     for (int k = 0; k < r; ++k) sum += B[order[k] * ld + order[k]];
     const double l1 = B[order[0] * ld + order[0]];
-    double rh = (red[0] - sum) / (double)(d - r);
+    double rh = (trace - sum) / (double)(d - r);
     uint32_t f = 0;
     const double floor = ldexp(l1, -24);
     if (!(rh > floor)) {
@@ -438,7 +506,7 @@ __global__ void __launch_bounds__(kRT) rr_kernel(const double* __restrict__ part
     *rho = (float)rh;
     if (f && dev_status) atomicOr(dev_status, f);
   }
-  for (int k = threadIdx.x; k < r; k += kRT) lambda[k] = (float)B[order[k] * ld + order[k]];
+  for (int k = threadIdx.x; k < r; k += kST) lambda[k] = (float)B[order[k] * ld + order[k]];
 }
 
 // U = Q Vs (d x m times m x r), fp64 accumulation.
@@ -454,32 +522,47 @@ __global__ void form_u_kernel(const float* __restrict__ Q, const double* __restr
   }
 }
 
-constexpr size_t kSmallSmem = 2 * 64 * 65 * sizeof(double);
+constexpr size_t kCholSmem = 2 * 64 * 65 * sizeof(double);
+constexpr size_t kRRSmem = 4 * 64 * 65 * sizeof(double);
+
+// k-slices of the skinny product: enough CTAs to cover the SMs twice
+inline int skinny_slices(int d) {
+  const int tiles = d / 64;
+  int ns = (2 * kNumSMs + tiles - 1) / tiles;
+  const int max_ns = d / (4 * kSkK);
+  if (ns > max_ns) ns = max_ns;
+  return ns < 1 ? 1 : ns;
+}
 
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 }  // namespace
 
-void refresh_plan(int64_t N, int64_t d, int rank, int oversample, bool a_out_given, RefreshPlan* p) {
+void refresh_plan(int64_t N, int64_t d, int rank, int oversample, bool a_out_given, RefreshPlan* p,
+                  bool no_split) {
   p->N = N;
   p->d = d;
   p->rank = rank;
   p->m = rank + oversample;
   p->iters = 0;
   p->seed = 0;
-  p->gram_parts = (int)((d + 63) / 64);
+  p->gram_parts = (int)((d + kGramRows - 1) / kGramRows);
+  p->skinny_slices = no_split ? 1 : skinny_slices((int)d);
   // split-K over tokens so that the triangle of 128 x 256 tiles fills the SMs
   const int64_t tiles = syrk_tc_tiles((int)d);
   int splits = 1;
-  while (splits < 16 && tiles * splits < kNumSMs && N / (splits * 2) >= 1024) splits *= 2;
+  while (!no_split && splits < 16 && tiles * splits < kNumSMs && N / (splits * 2) >= 1024) splits *= 2;
   p->syrk_splits = splits;
+  const size_t dm = (size_t)d * p->m * sizeof(float);
   size_t off = 0;
   p->off_A = off;
   if (!a_out_given) off += align256((size_t)d * d * sizeof(float));
   p->off_Q = off;
-  off += align256((size_t)d * p->m * sizeof(float));
+  off += align256(dm);
   p->off_Y = off;
-  off += align256((size_t)d * p->m * sizeof(float));
+  off += align256(dm * p->skinny_slices);
+  p->off_T = off;
+  off += align256(dm);
   p->off_gram = off;
   off += align256((size_t)p->gram_parts * p->m * p->m * sizeof(double));
   p->off_small = off;
@@ -489,49 +572,36 @@ void refresh_plan(int64_t N, int64_t d, int rank, int oversample, bool a_out_giv
   p->total = off;
 }
 
-static cudaError_t orth_cholqr2(float* Yb, float* tmp, int d, int m, int parts, double* gram, double* Rinv,
-                                uint32_t* dev_status, cudaStream_t s) {
-  float* in = Yb;
-  float* out = tmp;
-  for (int pass = 0; pass < 2; ++pass) {
-    gram_partial_kernel<<<parts, kRT, 0, s>>>(in, in, d, m, gram);
-    chol_kernel<<<1, kRT, kSmallSmem, s>>>(gram, parts, m, Rinv, dev_status);
-    qr_apply_kernel<<<(d + 3) / 4, kRT, 0, s>>>(in, Rinv, out, d, m);
-    float* t = in;
-    in = out;
-    out = t;
-  }
-  return cudaGetLastError();
+// One Cholesky-QR pass: Qo = Yi R^{-1} with Yi^T Yi = R^T R (Yi in ns slices).
+static void cholqr_pass(const float* Yi, int ns, float* Qo, int d, int m, int parts, double* gram, double* Rinv,
+                        uint32_t* dev_status, cudaStream_t s) {
+  gram_partial_kernel<<<parts, kRT, 0, s>>>(Yi, ns, Yi, ns, d, m, gram);
+  chol_kernel<<<1, kST, kCholSmem, s>>>(gram, parts, m, Rinv, dev_status);
+  qr_apply_kernel<<<(d + 3) / 4, kRT, 0, s>>>(Yi, ns, Rinv, Qo, d, m);
 }
 
 cudaError_t launch_refresh(const RefreshPlan& p, const void* X, gift_dtype xdt, float* U, float* lambda, float* rho,
                            float* A_out, void* ws, uint32_t* dev_status, cudaStream_t s) {
-  // the two single-CTA fp64 kernels need 65 KB of dynamic shared memory
-  static std::atomic<uint64_t> attr_done{0};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  const uint64_t bit = 1ull << (dev & 63);
-  if (!(attr_done.load() & bit)) {
-    cudaError_t e1 = cudaFuncSetAttribute(chol_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmallSmem);
-    cudaError_t e2 = cudaFuncSetAttribute(rr_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmallSmem);
-    if (e1 != cudaSuccess) return e1;
-    if (e2 != cudaSuccess) return e2;
-    attr_done.fetch_or(bit);
-  }
+  static unsigned long long chol_attr = 0, rr_attr = 0;
+  cudaError_t e = ensure_smem_attr(chol_kernel, (int)kCholSmem, &chol_attr);
+  if (e != cudaSuccess) return e;
+  if ((e = ensure_smem_attr(rr_kernel, (int)kRRSmem, &rr_attr)) != cudaSuccess) return e;
   char* w = (char*)ws;
-  const int d = (int)p.d, m = p.m, r = p.rank;
+  const int d = (int)p.d, m = p.m, r = p.rank, ns = p.skinny_slices;
   float* A = A_out ? A_out : (float*)(w + p.off_A);
-  float* B1 = (float*)(w + p.off_Q);
-  float* B2 = (float*)(w + p.off_Y);
+  float* Q = (float*)(w + p.off_Q);
+  float* Y = (float*)(w + p.off_Y);
+  float* T = (float*)(w + p.off_T);
   double* gram = (double*)(w + p.off_gram);
   double* Rinv = (double*)(w + p.off_small);
   double* Vs = Rinv + 64 * 64;
   const float scale = (float)(1.0 / (double)p.N);
+  const dim3 skinny_grid(d / 64, ns);
+  const int kslice = (d / ns + kSkK - 1) / kSkK * kSkK;
 
   // R1: A = X^T X / N
   bool used_tc = false;
-  cudaError_t e = launch_syrk_tc(X, xdt, p.N, d, A, (float*)(w + p.off_syrk), p.syrk_splits, dev_status, s,
-                                 &used_tc);
+  e = launch_syrk_tc(X, xdt, p.N, d, A, (float*)(w + p.off_syrk), p.syrk_splits, dev_status, s, &used_tc);
   if (e != cudaSuccess) return e;
   if (!used_tc) {
     const int nt = d / 64;
@@ -541,21 +611,24 @@ cudaError_t launch_refresh(const RefreshPlan& p, const void* X, gift_dtype xdt, 
     else
       syrk_simt_kernel<float><<<tiles, kRT, 0, s>>>((const float*)X, p.N, d, A, scale);
   }
-  // R2: randomised subspace iteration
-  omega_kernel<<<(d * m + kRT - 1) / kRT, kRT, 0, s>>>(B1, d, m, p.seed);
-  if ((e = orth_cholqr2(B1, B2, d, m, p.gram_parts, gram, Rinv, dev_status, s)) != cudaSuccess) return e;
+  // R2: randomised subspace iteration.  span(A Omega) = span(A orth(Omega)), so
+  // the +-1 start block (exact) is multiplied by A directly; with no iterations
+  // it is orthonormalised for the Rayleigh-Ritz step instead.
+  omega_kernel<<<(d * m + kRT - 1) / kRT, kRT, 0, s>>>(Q, d, m, p.seed);
+  if (p.iters == 0) {
+    cholqr_pass(Q, 1, T, d, m, p.gram_parts, gram, Rinv, dev_status, s);
+    cholqr_pass(T, 1, Q, d, m, p.gram_parts, gram, Rinv, dev_status, s);
+  }
   for (int it = 0; it < p.iters; ++it) {
-    skinny_kernel<<<d / 32, kRT, 0, s>>>(A, B1, B2, d, m);
-    if ((e = orth_cholqr2(B2, B1, d, m, p.gram_parts, gram, Rinv, dev_status, s)) != cudaSuccess) return e;
-    float* t = B1;
-    B1 = B2;
-    B2 = t;
+    skinny_kernel<<<skinny_grid, kRT, 0, s>>>(A, Q, Y, d, m, kslice);
+    cholqr_pass(Y, ns, T, d, m, p.gram_parts, gram, Rinv, dev_status, s);  // Cholesky-QR2:
+    cholqr_pass(T, 1, Q, d, m, p.gram_parts, gram, Rinv, dev_status, s);   // two passes
   }
   // R3/R4: Rayleigh-Ritz, lambda, rho, U
-  skinny_kernel<<<d / 32, kRT, 0, s>>>(A, B1, B2, d, m);
-  gram_partial_kernel<<<p.gram_parts, kRT, 0, s>>>(B1, B2, d, m, gram);
-  rr_kernel<<<1, kRT, kSmallSmem, s>>>(gram, p.gram_parts, m, r, A, d, Vs, lambda, rho, dev_status);
-  form_u_kernel<<<(d * r + kRT - 1) / kRT, kRT, 0, s>>>(B1, Vs, d, m, r, U);
+  skinny_kernel<<<skinny_grid, kRT, 0, s>>>(A, Q, Y, d, m, kslice);
+  gram_partial_kernel<<<p.gram_parts, kRT, 0, s>>>(Q, 1, Y, ns, d, m, gram);
+  rr_kernel<<<1, kST, kRRSmem, s>>>(gram, p.gram_parts, m, r, A, d, Vs, lambda, rho, dev_status);
+  form_u_kernel<<<(d * r + kRT - 1) / kRT, kRT, 0, s>>>(Q, Vs, d, m, r, U);
   return cudaGetLastError();
 }
 
