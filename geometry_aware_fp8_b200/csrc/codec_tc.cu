@@ -47,7 +47,7 @@ constexpr int kUBytes = kChunk * 128;          // 16 KB: [128 rows][64 bf16]
 constexpr int kStageBytes = kGBytes + kUBytes;
 constexpr int kPcBytes = kPanel * 128;         // 16 KB: [128 rows][64 bf16]
 constexpr int kSmemBytes = kStages * kStageBytes + kPcBytes + 1024 + 512;
-constexpr int kThreads = 288;
+constexpr int kThreads = 320;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColW0 = 0, kColW1 = 128, kColP = 256;
 constexpr uint32_t kIdescE1 = umma_idesc_bf16(128, 64, 0, 1);   // A K-major, B MN-major
@@ -76,6 +76,49 @@ struct EncParams {
 GIFT_DEV uint32_t sw128(uint32_t r, uint32_t q) { return r * 128u + ((q ^ (r & 7u)) << 4); }
 
 GIFT_DEV void named_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
+
+// L2 eviction policies for TMA loads: the first pass over a panel keeps its
+// chunks (they are read again by the second pass), the second pass lets them go.
+GIFT_DEV uint64_t policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+GIFT_DEV uint64_t policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+GIFT_DEV void tma_load_2d_hint(uint32_t dst, const void* tmap, uint64_t* bar, int x, int y, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(dst),
+      "l"(tmap), "r"(smem_u32(bar)), "r"(x), "r"(y), "l"(policy)
+      : "memory");
+}
+
+// Walks the (panel, pass, chunk) steps of one CTA in the order every role
+// uses: for each scheduled panel, the first pass over chunks 0..nc-1, then
+// the second pass over nc-1..0.
+template <class P>
+struct Steps {
+  const P& p;
+  int it, end, pass, i, nc;
+  GIFT_DEV Steps(const P& p_, int beg, int end_) : p(p_), it(beg), end(end_), pass(0), i(0), nc(0) {
+    if (it < end) nc = p.jobs[job()].d_in / kChunk;
+  }
+  GIFT_DEV bool valid() const { return it < end; }
+  GIFT_DEV int job() const { return p.sched_ids[it] >> 8; }
+  GIFT_DEV int panel() const { return p.sched_ids[it] & 255; }
+  GIFT_DEV int chunk() const { return pass == 0 ? i : nc - 1 - i; }
+  GIFT_DEV void next() {
+    if (++i < nc) return;
+    i = 0;
+    if (++pass < 2) return;
+    pass = 0;
+    if (++it < end) nc = p.jobs[job()].d_in / kChunk;
+  }
+};
 
 // Named barrier that also ORs a predicate over the group: every member gets
 // the same answer, so a group can agree to stop without a shared flag.
@@ -107,11 +150,9 @@ GIFT_DEV void split_bf16(float x, float& hi, float& lo) {
   lo = x - hi;
 }
 
-// Convert rows [j0, j0+128) of U (d_in x rank fp32) into the swizzled
-// [128][hi 32 | lo 32] bf16 tile; thread t of the 128 converter threads owns row t.
-GIFT_DEV void convert_u_tile(const float* __restrict__ U, int rank, int j0, uint32_t tile, int t) {
-  float u[32];
-  const float* src = U + (int64_t)(j0 + t) * rank;
+// Row j of U (d_in x rank fp32) into registers, zero-padded to 32 values.
+GIFT_DEV void load_u_row(const float* __restrict__ U, int rank, int j, float (&u)[32]) {
+  const float* src = U + (int64_t)j * rank;
   if (rank == 32) {
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
@@ -122,6 +163,10 @@ GIFT_DEV void convert_u_tile(const float* __restrict__ U, int rank, int j0, uint
 #pragma unroll
     for (int k = 0; k < 32; ++k) u[k] = k < rank ? __ldg(src + k) : 0.0f;
   }
+}
+
+// Row t of the swizzled [128][hi 32 | lo 32] bf16 U tile from its fp32 values.
+GIFT_DEV void store_u_row(const float (&u)[32], uint32_t tile, int t) {
   uint32_t hi[16], lo[16];
 #pragma unroll
   for (int k = 0; k < 16; ++k) {
@@ -180,40 +225,54 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
 
-  if (warp >= 4 && warp < 8) {
-    // ---------------- producer: TMA for G + U conversion ----------------
-    // Exit decisions are taken on the group-local flag right after a named
-    // barrier, so all 128 threads leave at the same step.
+  if (warp == 9) {
+    // ---------------- TMA producer: G chunks, running ahead of the ring ----------------
+    if (lane == 0) {
+      const uint64_t keep = policy_evict_last(), drop = policy_evict_first();
+      uint32_t step = 0;
+      for (Steps<EncParams> st(p, beg, end); st.valid() && !failed; st.next(), ++step) {
+        const int s = step % kStages;
+        const uint32_t use = step / kStages;
+        if (step >= kStages && !mbar_wait(&empty[s], (use - 1) & 1u, kWaitLimit)) {
+          failed = 1;
+          break;
+        }
+        const EncJob& J = p.jobs[st.job()];
+        const uint64_t pol = st.pass == 0 ? keep : drop;
+        const uint32_t dst = sbase + s * kStageBytes;
+        mbar_arrive_expect_tx(&full[s], kGBytes);
+        tma_load_2d_hint(dst, &J.tmG, &full[s], st.chunk() * kChunk, st.panel() * kPanel, pol);
+        tma_load_2d_hint(dst + kGHalf, &J.tmG, &full[s], st.chunk() * kChunk + 64, st.panel() * kPanel, pol);
+      }
+    }
+  } else if (warp >= 4 && warp < 8) {
+    // ---------------- converters: U rows -> bf16 hi/lo tile, one row each ----------------
+    // The next step's U row is loaded before waiting for this step's stage.
+    // Exit decisions are voted at a named barrier so all 128 threads leave
+    // at the same step.
     const int t = threadIdx.x - 128;
     uint32_t step = 0;
-    bool stop = false;  // group vote: set for all 128 threads at the same barrier
-    for (int it = beg; it < end && !stop; ++it) {
-      const int jb = p.sched_ids[it] >> 8, panel = p.sched_ids[it] & 255;
-      const EncJob& J = p.jobs[jb];
-      const int nc = J.d_in / kChunk;
-      for (int pass = 0; pass < 2 && !stop; ++pass) {
-        for (int i = 0; i < nc; ++i, ++step) {
-          const int c = pass == 0 ? i : nc - 1 - i;
-          const int s = step % kStages;
-          const uint32_t use = step / kStages;
-          const bool ok = step < kStages || mbar_wait(&empty[s], (use - 1) & 1u, kWaitLimit);
-          stop = named_sync_or(1, 128, !ok);
-          if (stop) {
-            failed = 1;
-            break;
-          }
-          const uint32_t g_tile = sbase + s * kStageBytes;
-          if (t == 0) {
-            mbar_arrive_expect_tx(&full[s], kGBytes);
-            tma_load_2d(smem + s * kStageBytes, &J.tmG, &full[s], c * kChunk, panel * kPanel);
-            tma_load_2d(smem + s * kStageBytes + kGHalf, &J.tmG, &full[s], c * kChunk + 64, panel * kPanel);
-          }
-          convert_u_tile(J.U, J.rank, c * kChunk, g_tile + kGBytes, t);
-          fence_async_shared();
-          named_sync(1, 128);
-          if (t == 0) mbar_arrive(&full[s]);
-        }
+    Steps<EncParams> st(p, beg, end);
+    float u_next[32];
+    if (st.valid()) load_u_row(p.jobs[st.job()].U, p.jobs[st.job()].rank, st.chunk() * kChunk + t, u_next);
+    while (st.valid()) {
+      float u[32];
+#pragma unroll
+      for (int k = 0; k < 32; ++k) u[k] = u_next[k];
+      const int s = step % kStages;
+      const uint32_t use = step / kStages;
+      st.next();
+      if (st.valid()) load_u_row(p.jobs[st.job()].U, p.jobs[st.job()].rank, st.chunk() * kChunk + t, u_next);
+      const bool ok = step < kStages || mbar_wait(&empty[s], (use - 1) & 1u, kWaitLimit);
+      if (named_sync_or(1, 128, !ok)) {
+        failed = 1;
+        break;
       }
+      store_u_row(u, sbase + s * kStageBytes + kGBytes, t);
+      fence_async_shared();
+      named_sync(1, 128);
+      if (t == 0) mbar_arrive(&full[s]);
+      ++step;
     }
   } else if (warp == 8) {
     // ---------------- MMA issuer ----------------
@@ -372,8 +431,8 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
             }
           }
           if (live) {
-            *reinterpret_cast<uint4*>(dst + g4 * 32) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-            *reinterpret_cast<uint4*>(dst + g4 * 32 + 16) = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+            __stcs(reinterpret_cast<uint4*>(dst + g4 * 32), make_uint4(cw[0], cw[1], cw[2], cw[3]));
+            __stcs(reinterpret_cast<uint4*>(dst + g4 * 32 + 16), make_uint4(cw[4], cw[5], cw[6], cw[7]));
           }
         }
         if (live) J.scales[row * (J.d_in / kChunk) + c] = e4m3_scale(amax, inv);
@@ -478,58 +537,71 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
 
-  if (warp >= 4 && warp < 8) {
-    // ---------------- producer: TMA for codes, U tile, bf16 codes tile ----------------
+  if (warp == 9) {
+    // ---------------- TMA producer: codes chunks, running ahead of the ring ----------------
+    if (lane == 0) {
+      const uint64_t keep = policy_evict_last(), drop = policy_evict_first();
+      uint32_t step = 0;
+      for (Steps<DecParams> st(p, beg, end); st.valid() && !failed; st.next(), ++step) {
+        const int s = step % kDStages;
+        const uint32_t use = step / kDStages;
+        if (step >= kDStages && !mbar_wait(&empty[s], (use - 1) & 1u, kWaitLimit)) {
+          failed = 1;
+          break;
+        }
+        const DecJob& J = p.jobs[st.job()];
+        mbar_arrive_expect_tx(&cfull[s], kDCodes);
+        tma_load_2d_hint(sbase + s * kDStageBytes, &J.tmC, &cfull[s], st.chunk() * kChunk, st.panel() * kPanel,
+                         st.pass == 0 ? keep : drop);
+      }
+    }
+  } else if (warp >= 4 && warp < 8) {
+    // ---------------- converters: U tile, and in the first pass the bf16 codes ----------------
     const int t = threadIdx.x - 128;
     uint32_t step = 0;
-    bool stop = false;
-    for (int it = beg; it < end && !stop; ++it) {
-      const int jb = p.sched_ids[it] >> 8, panel = p.sched_ids[it] & 255;
-      const DecJob& J = p.jobs[jb];
-      const int nc = J.d_in / kChunk;
-      for (int pass = 0; pass < 2 && !stop; ++pass) {
-        for (int i = 0; i < nc; ++i, ++step) {
-          const int c = pass == 0 ? i : nc - 1 - i;
-          const int s = step % kDStages;
-          const uint32_t use = step / kDStages;
-          const bool ok = step < kDStages || mbar_wait(&empty[s], (use - 1) & 1u, kWaitLimit);
-          stop = named_sync_or(1, 128, !ok);
-          if (stop) {
-            failed = 1;
-            break;
-          }
-          const uint32_t c_tile = sbase + s * kDStageBytes;
-          const uint32_t q_tile = c_tile + kDCodes;
-          const uint32_t u_tile = q_tile + kDQ;
-          if (t == 0) {
-            mbar_arrive_expect_tx(&cfull[s], kDCodes);
-            tma_load_2d(smem + s * kDStageBytes, &J.tmC, &cfull[s], c * kChunk, panel * kPanel);
-          }
-          convert_u_tile(J.U, J.rank, c * kChunk, u_tile, t);
-          if (pass == 0) {
-            // the codes of row t: wait for the TMA, then widen to bf16
-            if (!mbar_wait(&cfull[s], use & 1u, kWaitLimit)) failed = 1;
+    Steps<DecParams> st(p, beg, end);
+    float u_next[32];
+    if (st.valid()) load_u_row(p.jobs[st.job()].U, p.jobs[st.job()].rank, st.chunk() * kChunk + t, u_next);
+    while (st.valid()) {
+      float u[32];
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              const uint4 v = ld_shared_v4(c_tile + sw128(t, q));
-              const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-              uint32_t o[8];
+      for (int k = 0; k < 32; ++k) u[k] = u_next[k];
+      const int s = step % kDStages;
+      const uint32_t use = step / kDStages;
+      const int pass = st.pass;
+      st.next();
+      if (st.valid()) load_u_row(p.jobs[st.job()].U, p.jobs[st.job()].rank, st.chunk() * kChunk + t, u_next);
+      const bool ok = step < kDStages || mbar_wait(&empty[s], (use - 1) & 1u, kWaitLimit);
+      if (named_sync_or(1, 128, !ok)) {
+        failed = 1;
+        break;
+      }
+      const uint32_t c_tile = sbase + s * kDStageBytes;
+      const uint32_t q_tile = c_tile + kDCodes;
+      store_u_row(u, q_tile + kDQ, t);
+      if (pass == 0) {
+        // the codes of row t: wait for the TMA, then widen to bf16
+        if (!mbar_wait(&cfull[s], use & 1u, kWaitLimit)) failed = 1;
 #pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                o[2 * e] = e4m3x2_to_bf16x2((uint16_t)(w[e] & 0xFFFFu));
-                o[2 * e + 1] = e4m3x2_to_bf16x2((uint16_t)(w[e] >> 16));
-              }
-              // 16 codes -> 32 bytes of bf16 = chunks 2q, 2q+1 of the 256-byte row
-              const int c0 = 2 * q, c1 = 2 * q + 1;
-              st_shared_v4(q_tile + (c0 >> 3) * kGHalf + sw128(t, c0 & 7), o[0], o[1], o[2], o[3]);
-              st_shared_v4(q_tile + (c1 >> 3) * kGHalf + sw128(t, c1 & 7), o[4], o[5], o[6], o[7]);
-            }
+        for (int q = 0; q < 8; ++q) {
+          const uint4 v = ld_shared_v4(c_tile + sw128(t, q));
+          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+          uint32_t o[8];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            o[2 * e] = e4m3x2_to_bf16x2((uint16_t)(w[e] & 0xFFFFu));
+            o[2 * e + 1] = e4m3x2_to_bf16x2((uint16_t)(w[e] >> 16));
           }
-          fence_async_shared();
-          named_sync(1, 128);
-          if (t == 0) mbar_arrive(&full[s]);
+          // 16 codes -> 32 bytes of bf16 = chunks 2q, 2q+1 of the 256-byte row
+          const int c0 = 2 * q, c1 = 2 * q + 1;
+          st_shared_v4(q_tile + (c0 >> 3) * kGHalf + sw128(t, c0 & 7), o[0], o[1], o[2], o[3]);
+          st_shared_v4(q_tile + (c1 >> 3) * kGHalf + sw128(t, c1 & 7), o[4], o[5], o[6], o[7]);
         }
       }
+      fence_async_shared();
+      named_sync(1, 128);
+      if (t == 0) mbar_arrive(&full[s]);
+      ++step;
     }
   } else if (warp == 8) {
     // ---------------- MMA issuer ----------------
@@ -605,7 +677,10 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
       float P[32];
 #pragma unroll
       for (int k = 0; k < 32; ++k) P[k] = 0.0f;
+      float sc_next = live ? __ldg(srow) : 0.0f;  // scale of the next chunk, loaded one chunk ahead
       for (int c = 0; c < nc; ++c, ++step, ++d2) {
+        const float sc = sc_next;
+        if (live && c + 1 < nc) sc_next = __ldg(srow + c + 1);
         const int b = d2 & 1;
         stop = named_sync_or(2, 128, !mbar_wait(&t_full[b], (d2 >> 1) & 1u, kWaitLimit));
         if (stop) {
@@ -620,7 +695,6 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(&t_empty[b]);
-        const float sc = live ? __ldg(srow + c) : 0.0f;
 #pragma unroll
         for (int k = 0; k < 32; ++k) P[k] = fmaf(sc, __uint_as_float(tr[k]) + __uint_as_float(tr[32 + k]), P[k]);
       }
@@ -644,8 +718,11 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
       fence_async_shared();
       mbar_arrive(pc_full);
       // D3 epilogue: G_hat = a s q + acc
+      sc_next = live ? __ldg(srow + nc - 1) : 0.0f;
       for (int i = 0; i < nc; ++i, ++step, ++e2) {
         const int c = nc - 1 - i;
+        const float sc3 = sc_next;
+        if (live && c > 0) sc_next = __ldg(srow + c - 1);
         const int s = step % kDStages;
         const int b = e2 & 1;
         const bool ok = mbar_wait(&w_full[b], (e2 >> 1) & 1u, kWaitLimit) &&
@@ -658,7 +735,7 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
         tc_fence_after();
         const uint32_t wcol = tbase + lane_off + (b ? kColW1 : kColW0);
         const uint32_t c_tile = sbase + s * kDStageBytes;
-        const float as = a * (live ? __ldg(srow + c) : 0.0f);
+        const float as = a * sc3;
         __nv_bfloat16* dst = J.out + row * J.d_in + c * kChunk;
 #pragma unroll
         for (int g4 = 0; g4 < 4; ++g4) {
@@ -684,10 +761,10 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
           }
           if (live) {
             uint4* d4 = reinterpret_cast<uint4*>(dst + g4 * 32);
-            d4[0] = make_uint4(o[0], o[1], o[2], o[3]);
-            d4[1] = make_uint4(o[4], o[5], o[6], o[7]);
-            d4[2] = make_uint4(o[8], o[9], o[10], o[11]);
-            d4[3] = make_uint4(o[12], o[13], o[14], o[15]);
+            __stcs(d4 + 0, make_uint4(o[0], o[1], o[2], o[3]));
+            __stcs(d4 + 1, make_uint4(o[4], o[5], o[6], o[7]));
+            __stcs(d4 + 2, make_uint4(o[8], o[9], o[10], o[11]));
+            __stcs(d4 + 3, make_uint4(o[12], o[13], o[14], o[15]));
           }
         }
         tc_fence_before();

@@ -11,7 +11,7 @@
 //
 // Limits: d_in <= 4096 and rank + oversample <= 64, which bounds the scratch
 // (sampled subspace, its image, a Cholesky-QR temporary, fp64 Gram partials
-// and the small factors) at 4,259,840 bytes.  A must be given by the caller as an output buffer,
+// and the small factors) at 5,308,416 bytes.  A must be given by the caller as an output buffer,
 // and the token range is not split, so the whole scratch need is known.
 #include <mutex>
 
@@ -23,7 +23,7 @@ namespace {
 
 constexpr int64_t kNoAllocMaxDin = 4096;
 constexpr int kNoAllocMaxSubspace = 64;
-constexpr size_t kNoAllocScratchBytes = 4259840;
+constexpr size_t kNoAllocScratchBytes = 5308416;
 
 // Scratch shared by every call on a device.  Host code cannot use this name
 // as a device address: it only names the host-side shadow of the symbol, so

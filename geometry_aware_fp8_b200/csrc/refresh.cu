@@ -194,54 +194,51 @@ __global__ void __launch_bounds__(kRT) skinny_kernel(const float* __restrict__ A
     }
 }
 
-// Element (row, c) of a matrix stored as `ns` slices to be added (stride d*m).
-GIFT_DEV float sliced(const float* __restrict__ Y, int ns, int64_t stride, int64_t idx) {
-  float v = Y[idx];
-  for (int s = 1; s < ns; ++s) v += Y[s * stride + idx];
-  return v;
+// Y[0..n) += Y[s n .. (s+1) n) for s = 1..ns-1, in slice order.
+__global__ void fold_slices_kernel(float* __restrict__ Y, int ns, int64_t n) {
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
+    float v = Y[e];
+    for (int s = 1; s < ns; ++s) v += Y[s * n + e];
+    Y[e] = v;
+  }
 }
 
-// part[p] = Ya[rows of p]^T Yb[rows of p] (m x m, fp64), kGramRows rows per
-// part, staged through shared memory 64 rows at a time.  Thread (ti, tj) of
-// a 16 x 16 grid owns the 4 x 4 block of entries (4 ti.., 4 tj..).  Ya and Yb
-// may be split into na / nb slices that are added on load.
-constexpr int kGramRows = 128;
+// part[p] = Ya[rows of p]^T Yb[rows of p] (m x m, fp64), 64 rows per part
+// staged in shared memory; thread (ti, tj) of a 16 x 16 grid owns the 4 x 4
+// block of entries (4 ti.., 4 tj..).
+constexpr int kGramRows = 64;
 
-__global__ void __launch_bounds__(kRT) gram_partial_kernel(const float* __restrict__ Ya, int na,
-                                                           const float* __restrict__ Yb, int nb, int d, int m,
+__global__ void __launch_bounds__(kRT) gram_partial_kernel(const float* __restrict__ Ya,
+                                                           const float* __restrict__ Yb, int d, int m,
                                                            double* __restrict__ part) {
   __shared__ __align__(16) float Sa[64][64];
   __shared__ __align__(16) float Sb[64][64];
   const int p = blockIdx.x;
+  const int r0 = p * kGramRows;
+  const int rows = min(kGramRows, d - r0);
   const int ti = threadIdx.x >> 4, tj = threadIdx.x & 15;
-  const int64_t stride = (int64_t)d * m;
+  for (int e = threadIdx.x; e < 64 * 64; e += kRT) {
+    const int rr = e >> 6, c = e & 63;
+    const bool in = rr < rows && c < m;
+    Sa[rr][c] = in ? Ya[(int64_t)(r0 + rr) * m + c] : 0.0f;
+    Sb[rr][c] = in ? Yb[(int64_t)(r0 + rr) * m + c] : 0.0f;
+  }
+  __syncthreads();
   double acc[4][4];
 #pragma unroll
   for (int a = 0; a < 4; ++a)
 #pragma unroll
     for (int b = 0; b < 4; ++b) acc[a][b] = 0.0;
-  for (int r0 = p * kGramRows; r0 < min(d, (p + 1) * kGramRows); r0 += 64) {
-    const int rows = min(64, d - r0);
-    __syncthreads();
-    for (int e = threadIdx.x; e < 64 * 64; e += kRT) {
-      const int rr = e >> 6, c = e & 63;
-      const bool in = rr < rows && c < m;
-      const int64_t idx = (int64_t)(r0 + rr) * m + c;
-      Sa[rr][c] = in ? sliced(Ya, na, stride, idx) : 0.0f;
-      Sb[rr][c] = in ? sliced(Yb, nb, stride, idx) : 0.0f;
-    }
-    __syncthreads();
 #pragma unroll 4
-    for (int rr = 0; rr < 64; ++rr) {
-      const float4 va = *reinterpret_cast<const float4*>(&Sa[rr][ti * 4]);
-      const float4 vb = *reinterpret_cast<const float4*>(&Sb[rr][tj * 4]);
-      const double a4[4] = {va.x, va.y, va.z, va.w};
-      const double b4[4] = {vb.x, vb.y, vb.z, vb.w};
+  for (int rr = 0; rr < 64; ++rr) {
+    const float4 va = *reinterpret_cast<const float4*>(&Sa[rr][ti * 4]);
+    const float4 vb = *reinterpret_cast<const float4*>(&Sb[rr][tj * 4]);
+    const double a4[4] = {va.x, va.y, va.z, va.w};
+    const double b4[4] = {vb.x, vb.y, vb.z, vb.w};
 #pragma unroll
-      for (int a = 0; a < 4; ++a)
+    for (int a = 0; a < 4; ++a)
 #pragma unroll
-        for (int b = 0; b < 4; ++b) acc[a][b] = fma(a4[a], b4[b], acc[a][b]);
-    }
+      for (int b = 0; b < 4; ++b) acc[a][b] = fma(a4[a], b4[b], acc[a][b]);
   }
   const int mm = m * m;
 #pragma unroll
@@ -263,129 +260,160 @@ GIFT_DEV double sum_parts(const double* __restrict__ part, int nparts, int mm, i
 
 constexpr int kST = 1024;  // threads of the single-CTA small-matrix kernels
 
-// Sum the Gram partials (all threads), Cholesky-factor in fp64 (one warp;
-// a column whose pivot falls below kCholTol of the largest diagonal entry
-// is dropped), and write R^{-1} (m x m, upper) with dropped columns zeroed.
+// Cholesky factor L of the summed Gram matrix (fp64, outer-product form):
+// at step j every thread updates its fixed lower-triangle entries (i, k),
+// k > j, by G[i][k] -= G[i][j] G[k][j] / G[j][j]; one barrier per column.
+// A pivot below kCholTol of the largest diagonal entry drops column j
+// (L[:, j] = e_j, flagged), so that column of Q comes out zero.
+// Output: Lout (m x m, row-major, lower part + diagonal), inv[j] = 1/L[j][j]
+// (0 for dropped columns).
 __global__ void __launch_bounds__(kST) chol_kernel(const double* __restrict__ part, int nparts, int m,
-                                                   double* __restrict__ Rinv, uint32_t* __restrict__ dev_status) {
+                                                   double* __restrict__ Lout, uint32_t* __restrict__ dev_status) {
   extern __shared__ double sm[];
   const int ld = 65;
-  double* Gs = sm;            // m x m (lower Cholesky factor in place)
-  double* Li = sm + 64 * ld;  // m x m, L^{-1}
-  __shared__ int defic[64];
+  double* G = sm;  // m x m
+  __shared__ double piv[64];
+  __shared__ double mxd;
   __shared__ int bad;
   if (threadIdx.x == 0) bad = 0;
   __syncthreads();
   for (int e = threadIdx.x; e < m * m; e += kST) {
     const double g = sum_parts(part, nparts, m * m, e);
     if (!isfinite(g)) bad = 1;
-    Gs[(e / m) * ld + e % m] = g;
+    G[(e / m) * ld + e % m] = g;
   }
   __syncthreads();
   if (threadIdx.x < 32) {
-    const int lane = threadIdx.x;
     double mx = 0.0;
-    for (int i = lane; i < m; i += 32) mx = fmax(mx, Gs[i * ld + i]);
+    for (int i = threadIdx.x; i < m; i += 32) mx = fmax(mx, G[i * ld + i]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    for (int j = 0; j < m; ++j) {
-      const double piv = Gs[j * ld + j];
-      const bool ok = piv > kCholTol * mx;
-      const double Ljj = ok ? sqrt(piv) : 1.0;
-      __syncwarp();
-      if (lane == 0) {
-        Gs[j * ld + j] = Ljj;
-        defic[j] = ok ? 0 : 1;
+    if (threadIdx.x == 0) mxd = mx;
+  }
+  // this thread's lower-triangle entries (i, k), k <= i (at most 3 for m <= 64)
+  int ei[3], ek[3], ne = 0;
+  {
+    int e = threadIdx.x, i = 0;
+    for (int q = 0; q < 3; ++q, e += kST) {
+      while (i < m && e >= (i + 1) * (i + 2) / 2) ++i;
+      if (i < m) {
+        ei[ne] = i;
+        ek[ne] = e - i * (i + 1) / 2;
+        ++ne;
       }
-      for (int i = j + 1 + lane; i < m; i += 32) Gs[i * ld + j] = ok ? Gs[i * ld + j] / Ljj : 0.0;
-      __syncwarp();
-      const int rem = m - j - 1;
-      for (int e = lane; e < rem * rem; e += 32) {
-        const int i = j + 1 + e / rem, k = j + 1 + e % rem;
-        if (k <= i) Gs[i * ld + k] -= Gs[i * ld + j] * Gs[k * ld + j];
-      }
-      __syncwarp();
     }
   }
   __syncthreads();
-  // L^{-1} column by column (forward substitution), one thread per column
-  if (threadIdx.x < m) {
-    const int c = threadIdx.x;
-    for (int i = 0; i < c; ++i) Li[i * ld + c] = 0.0;
-    for (int i = c; i < m; ++i) {
-      double x = (i == c) ? 1.0 : 0.0;
-      for (int k = c; k < i; ++k) x -= Gs[i * ld + k] * Li[k * ld + c];
-      Li[i * ld + c] = x / Gs[i * ld + i];
+  const double tol = kCholTol * mxd;
+  for (int j = 0; j < m; ++j) {
+    const double pj = G[j * ld + j];
+    const bool ok = pj > tol;
+    if (threadIdx.x == 0) piv[j] = ok ? pj : 0.0;
+    if (ok) {
+      const double inv = 1.0 / pj;
+      for (int q = 0; q < ne; ++q) {
+        const int i = ei[q], k = ek[q];
+        if (k > j) G[i * ld + k] -= G[i * ld + j] * G[k * ld + j] * inv;
+      }
     }
+    __syncthreads();
   }
-  __syncthreads();
-  // R = L^T, so R^{-1} = (L^{-1})^T; zero dropped columns so those Q columns are 0
+  // L[i][j] = G[i][j] / sqrt(piv_j) below the diagonal, sqrt(piv_j) on it
   for (int e = threadIdx.x; e < m * m; e += kST) {
-    const int k = e / m, c = e % m;
-    Rinv[e] = defic[c] ? 0.0 : Li[c * ld + k];
+    const int i = e / m, j = e % m;
+    const double pj = piv[j];
+    double v = 0.0;
+    if (pj > 0.0) {
+      if (i == j) v = sqrt(pj);
+      else if (i > j) v = G[i * ld + j] / sqrt(pj);
+    } else if (i == j) {
+      v = 1.0;
+    }
+    Lout[e] = v;
   }
+  if (threadIdx.x < m) Lout[m * m + threadIdx.x] = piv[threadIdx.x] > 0.0 ? 1.0 / sqrt(piv[threadIdx.x]) : 0.0;
   if (threadIdx.x == 0 && dev_status) {
     uint32_t f = 0;
     for (int j = 0; j < m; ++j)
-      if (defic[j]) f |= GIFT_DEV_RANK_DEFICIENT;
+      if (!(piv[j] > 0.0)) f |= GIFT_DEV_RANK_DEFICIENT;
     if (bad) f |= GIFT_DEV_NONFINITE;
     if (f) atomicOr(dev_status, f);
   }
 }
 
-// Qo = Yi R^{-1} (row by row, fp64 accumulation), 4 rows per CTA; Yi may be
-// split into ns slices.
-__global__ void __launch_bounds__(kRT) qr_apply_kernel(const float* __restrict__ Yi, int ns,
-                                                       const double* __restrict__ Rinv, float* __restrict__ Qo,
-                                                       int d, int m) {
-  __shared__ double Rs[64 * 64];
-  __shared__ double Ys[4][64];
-  for (int e = threadIdx.x; e < m * m; e += kRT) Rs[e] = Rinv[e];
-  const int rr = threadIdx.x >> 6, c = threadIdx.x & 63;
-  const int64_t row = (int64_t)blockIdx.x * 4 + rr;
-  if (row < d && c < m) Ys[rr][c] = (double)sliced(Yi, ns, (int64_t)d * m, row * m + c);
+// Qo = Yi R^{-1} with R = L^T: for each row, the forward substitution
+// q_c = (y_c - sum_{k<c} q_k L[c][k]) / L[c][c] (fp64), q_c = 0 for dropped
+// columns.  One warp per row: lane l owns columns l and l+32, the owner of
+// column c finishes q_c and broadcasts it.
+__global__ void __launch_bounds__(kRT) qr_apply_kernel(const float* __restrict__ Yi, const double* __restrict__ L,
+                                                       float* __restrict__ Qo, int d, int m) {
+  __shared__ double Ls[64 * 65];
+  __shared__ double inv[64];
+  for (int e = threadIdx.x; e < m * m; e += kRT) Ls[(e / m) * 65 + e % m] = L[e];
+  if (threadIdx.x < m) inv[threadIdx.x] = L[m * m + threadIdx.x];
   __syncthreads();
-  if (row < d && c < m) {
-    double acc = 0.0;
-    for (int k = 0; k <= c; ++k) acc = fma(Ys[rr][k], Rs[k * m + c], acc);
-    Qo[row * m + c] = (float)acc;
+  const int lane = threadIdx.x & 31;
+  for (int64_t row = (int64_t)blockIdx.x * (kRT / 32) + (threadIdx.x >> 5); row < d;
+       row += (int64_t)gridDim.x * (kRT / 32)) {
+    double acc0 = lane < m ? (double)Yi[row * m + lane] : 0.0;
+    double acc1 = lane + 32 < m ? (double)Yi[row * m + lane + 32] : 0.0;
+    double q0 = 0.0, q1 = 0.0;
+    for (int c = 0; c < m; ++c) {
+      double qc;
+      if (c < 32) {
+        qc = __shfl_sync(0xffffffffu, acc0 * inv[c], c);
+        if (lane == c) q0 = qc;
+      } else {
+        qc = __shfl_sync(0xffffffffu, acc1 * inv[c], c - 32);
+        if (lane == c - 32) q1 = qc;
+      }
+      if (lane > c) acc0 -= qc * Ls[lane * 65 + c];
+      if (lane + 32 > c && lane + 32 < m) acc1 -= qc * Ls[(lane + 32) * 65 + c];
+    }
+    if (lane < m) Qo[row * m + lane] = (float)q0;
+    if (lane + 32 < m) Qo[row * m + lane + 32] = (float)q1;
   }
 }
 
 // Rayleigh-Ritz on B = Q^T (A Q): fp64 Jacobi in parallel round-robin order.
-// Each round: the 2x2 rotations of the disjoint pairs are computed, then the
-// whole of B' = J^T B J and V' = V J is written to the other buffer from the
-// coefficient form (every entry depends on its own and its partner's row and
-// column only).  Eigenvalues are sorted descending; lambda, rho and the
-// sorted eigenvectors (Vs, m x r) are written.
+// Each round computes the rotations of the disjoint pairs, then every thread
+// updates whole 2x2 blocks: block (a, b) of B' = J^T B J needs only the four
+// entries of pairs a and b, and V' = V J is updated two entries at a time.
+// Eigenvalues are sorted descending; lambda, rho and the sorted eigenvectors
+// (Vs, m x r) are written.
 __global__ void __launch_bounds__(kST) rr_kernel(const double* __restrict__ part, int nparts, int m, int r,
                                                  const float* __restrict__ A, int d, double* __restrict__ Vs,
                                                  float* __restrict__ lambda, float* __restrict__ rho,
                                                  uint32_t* __restrict__ dev_status) {
   extern __shared__ double sm[];
   const int ld = 65;
-  double* Bb[2] = {sm, sm + 64 * ld};
-  double* Vb[2] = {sm + 2 * 64 * ld, sm + 3 * 64 * ld};
-  __shared__ double cself[64], cpart[64];
-  __shared__ int partner[64];
+  double* Bb0 = sm;
+  double* Bb1 = sm + 64 * ld;
+  double* Vb0 = sm + 2 * 64 * ld;
+  double* Vb1 = sm + 3 * 64 * ld;
+  __shared__ int pp[32], pq[32];
+  __shared__ double pc[32], ps[32];
   __shared__ double red[kST / 32];
   __shared__ int order[64];
   __shared__ int stop;
   for (int e = threadIdx.x; e < m * m; e += kST) {
-    Bb[0][(e / m) * ld + e % m] = sum_parts(part, nparts, m * m, e);
-    Vb[0][(e / m) * ld + e % m] = (e / m == e % m) ? 1.0 : 0.0;
+    Bb0[(e / m) * ld + e % m] = sum_parts(part, nparts, m * m, e);
+    Vb0[(e / m) * ld + e % m] = (e / m == e % m) ? 1.0 : 0.0;
   }
   __syncthreads();
   for (int e = threadIdx.x; e < m * m; e += kST) {  // symmetrise
     const int i = e / m, j = e % m;
     if (i < j) {
-      const double v = 0.5 * (Bb[0][i * ld + j] + Bb[0][j * ld + i]);
-      Bb[0][i * ld + j] = v;
-      Bb[0][j * ld + i] = v;
+      const double v = 0.5 * (Bb0[i * ld + j] + Bb0[j * ld + i]);
+      Bb0[i * ld + j] = v;
+      Bb0[j * ld + i] = v;
     }
   }
   __syncthreads();
-  int cur = 0;
+  double* B = Bb0;
+  double* Bn = Bb1;
+  double* V = Vb0;
+  double* Vn = Vb1;
   const int mp = m + (m & 1);  // even count for the round-robin tournament
   const int npairs = mp / 2;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -393,7 +421,7 @@ __global__ void __launch_bounds__(kST) rr_kernel(const double* __restrict__ part
     // convergence: off(B)^2 <= tol^2 ||B||_F^2
     double off = 0.0, tot = 0.0;
     for (int e = threadIdx.x; e < m * m; e += kST) {
-      const double b = Bb[cur][(e / m) * ld + e % m];
+      const double b = B[(e / m) * ld + e % m];
       tot += b * b;
       if (e / m != e % m) off += b * b;
     }
@@ -419,11 +447,10 @@ __global__ void __launch_bounds__(kST) rr_kernel(const double* __restrict__ part
     __syncthreads();
     if (stop) break;
     for (int round = 0; round < mp - 1; ++round) {
-      const double* B = Bb[cur];
       if (threadIdx.x < npairs) {
-        const int i = threadIdx.x;
+        const int a = threadIdx.x;
         auto pos = [&](int k) { return k == 0 ? 0 : 1 + (k - 1 + round) % (mp - 1); };
-        int p = pos(i), q = pos(mp - 1 - i);
+        int p = pos(a), q = pos(mp - 1 - a);
         if (p > q) {
           const int t = p;
           p = q;
@@ -439,34 +466,57 @@ __global__ void __launch_bounds__(kST) rr_kernel(const double* __restrict__ part
               t = 0.5 / theta;
             else
               t = copysign(1.0, theta) / (fabs(theta) + sqrt(theta * theta + 1.0));
-            c = 1.0 / sqrt(t * t + 1.0);
+            c = rsqrt(t * t + 1.0);
             s = t * c;
           }
-          // new p = c p - s q ; new q = s p + c q
-          cself[p] = c; cpart[p] = -s; partner[p] = q;
-          cself[q] = c; cpart[q] = s;  partner[q] = p;
-        } else if (p < m) {
-          cself[p] = 1.0; cpart[p] = 0.0; partner[p] = p;
+        }
+        pp[a] = p;
+        pq[a] = q;  // q == m marks the dummy partner of an odd m
+        pc[a] = c;
+        ps[a] = s;
+      }
+      __syncthreads();
+      // new row/column p = c p - s q, q = s p + c q
+      const int nb = npairs * npairs;
+      for (int w = threadIdx.x; w < nb + m * npairs; w += kST) {
+        if (w < nb) {
+          const int a = w / npairs, b = w % npairs;
+          const int pa = pp[a], qa = pq[a], pb = pp[b], qb = pq[b];
+          const double ca = pc[a], sa = ps[a], cb = pc[b], sb = ps[b];
+          const bool ha = qa < m, hb = qb < m;
+          const double b00 = B[pa * ld + pb];
+          const double b01 = hb ? B[pa * ld + qb] : 0.0;
+          const double b10 = ha ? B[qa * ld + pb] : 0.0;
+          const double b11 = (ha && hb) ? B[qa * ld + qb] : 0.0;
+          const double r00 = ca * b00 - sa * b10, r01 = ca * b01 - sa * b11;
+          const double r10 = sa * b00 + ca * b10, r11 = sa * b01 + ca * b11;
+          Bn[pa * ld + pb] = cb * r00 - sb * r01;
+          if (hb) Bn[pa * ld + qb] = sb * r00 + cb * r01;
+          if (ha) Bn[qa * ld + pb] = cb * r10 - sb * r11;
+          if (ha && hb) Bn[qa * ld + qb] = sb * r10 + cb * r11;
+        } else {
+          const int k = (w - nb) / npairs, b = (w - nb) % npairs;
+          const int pb = pp[b], qb = pq[b];
+          const double cb = pc[b], sb = ps[b];
+          const double v0 = V[k * ld + pb];
+          if (qb < m) {
+            const double v1 = V[k * ld + qb];
+            Vn[k * ld + pb] = cb * v0 - sb * v1;
+            Vn[k * ld + qb] = sb * v0 + cb * v1;
+          } else {
+            Vn[k * ld + pb] = v0;
+          }
         }
       }
       __syncthreads();
-      double* Bn = Bb[cur ^ 1];
-      const double* V = Vb[cur];
-      double* Vn = Vb[cur ^ 1];
-      for (int e = threadIdx.x; e < m * m; e += kST) {
-        const int i = e / m, j = e % m;
-        const int pi = partner[i], pj = partner[j];
-        const double si = cself[i], ti = cpart[i], sj = cself[j], tj = cpart[j];
-        Bn[i * ld + j] = si * (sj * B[i * ld + j] + tj * B[i * ld + pj]) +
-                         ti * (sj * B[pi * ld + j] + tj * B[pi * ld + pj]);
-        Vn[i * ld + j] = sj * V[i * ld + j] + tj * V[i * ld + pj];
-      }
-      __syncthreads();
-      cur ^= 1;
+      double* t = B;
+      B = Bn;
+      Bn = t;
+      t = V;
+      V = Vn;
+      Vn = t;
     }
   }
-  const double* B = Bb[cur];
-  const double* V = Vb[cur];
   // sort eigenvalues descending (ties by index)
   if (threadIdx.x < m) {
     const int i = threadIdx.x;
@@ -522,7 +572,7 @@ __global__ void form_u_kernel(const float* __restrict__ Q, const double* __restr
   }
 }
 
-constexpr size_t kCholSmem = 2 * 64 * 65 * sizeof(double);
+constexpr size_t kCholSmem = 64 * 65 * sizeof(double);
 constexpr size_t kRRSmem = 4 * 64 * 65 * sizeof(double);
 
 // k-slices of the skinny product: enough CTAs to cover the SMs twice
@@ -572,12 +622,26 @@ void refresh_plan(int64_t N, int64_t d, int rank, int oversample, bool a_out_giv
   p->total = off;
 }
 
-// One Cholesky-QR pass: Qo = Yi R^{-1} with Yi^T Yi = R^T R (Yi in ns slices).
-static void cholqr_pass(const float* Yi, int ns, float* Qo, int d, int m, int parts, double* gram, double* Rinv,
+// One Cholesky-QR pass: Qo = Yi R^{-1} with Yi^T Yi = R^T R.
+static void cholqr_pass(const float* Yi, float* Qo, int d, int m, int parts, double* gram, double* L,
                         uint32_t* dev_status, cudaStream_t s) {
-  gram_partial_kernel<<<parts, kRT, 0, s>>>(Yi, ns, Yi, ns, d, m, gram);
-  chol_kernel<<<1, kST, kCholSmem, s>>>(gram, parts, m, Rinv, dev_status);
-  qr_apply_kernel<<<(d + 3) / 4, kRT, 0, s>>>(Yi, ns, Rinv, Qo, d, m);
+  gram_partial_kernel<<<parts, kRT, 0, s>>>(Yi, Yi, d, m, gram);
+  chol_kernel<<<1, kST, kCholSmem, s>>>(gram, parts, m, L, dev_status);
+  int blocks = (d + 7) / 8;
+  if (blocks > 4 * kNumSMs) blocks = 4 * kNumSMs;
+  qr_apply_kernel<<<blocks, kRT, 0, s>>>(Yi, L, Qo, d, m);
+}
+
+// A Q into Y (k-slices folded into slice 0).
+static void skinny_product(const float* A, const float* Q, float* Y, int d, int m, int ns, cudaStream_t s) {
+  const int kslice = (d / ns + kSkK - 1) / kSkK * kSkK;
+  skinny_kernel<<<dim3(d / 64, ns), kRT, 0, s>>>(A, Q, Y, d, m, kslice);
+  if (ns > 1) {
+    const int64_t n = (int64_t)d * m;
+    int blocks = (int)((n + kRT - 1) / kRT);
+    if (blocks > 2 * kNumSMs) blocks = 2 * kNumSMs;
+    fold_slices_kernel<<<blocks, kRT, 0, s>>>(Y, ns, n);
+  }
 }
 
 cudaError_t launch_refresh(const RefreshPlan& p, const void* X, gift_dtype xdt, float* U, float* lambda, float* rho,
@@ -593,11 +657,9 @@ cudaError_t launch_refresh(const RefreshPlan& p, const void* X, gift_dtype xdt, 
   float* Y = (float*)(w + p.off_Y);
   float* T = (float*)(w + p.off_T);
   double* gram = (double*)(w + p.off_gram);
-  double* Rinv = (double*)(w + p.off_small);
-  double* Vs = Rinv + 64 * 64;
+  double* Lf = (double*)(w + p.off_small);   // Cholesky factor + reciprocal diagonal
+  double* Vs = Lf + 64 * 64 + 64;            // after m*m + m doubles (m <= 64)
   const float scale = (float)(1.0 / (double)p.N);
-  const dim3 skinny_grid(d / 64, ns);
-  const int kslice = (d / ns + kSkK - 1) / kSkK * kSkK;
 
   // R1: A = X^T X / N
   bool used_tc = false;
@@ -616,17 +678,17 @@ cudaError_t launch_refresh(const RefreshPlan& p, const void* X, gift_dtype xdt, 
   // it is orthonormalised for the Rayleigh-Ritz step instead.
   omega_kernel<<<(d * m + kRT - 1) / kRT, kRT, 0, s>>>(Q, d, m, p.seed);
   if (p.iters == 0) {
-    cholqr_pass(Q, 1, T, d, m, p.gram_parts, gram, Rinv, dev_status, s);
-    cholqr_pass(T, 1, Q, d, m, p.gram_parts, gram, Rinv, dev_status, s);
+    cholqr_pass(Q, T, d, m, p.gram_parts, gram, Lf, dev_status, s);
+    cholqr_pass(T, Q, d, m, p.gram_parts, gram, Lf, dev_status, s);
   }
   for (int it = 0; it < p.iters; ++it) {
-    skinny_kernel<<<skinny_grid, kRT, 0, s>>>(A, Q, Y, d, m, kslice);
-    cholqr_pass(Y, ns, T, d, m, p.gram_parts, gram, Rinv, dev_status, s);  // Cholesky-QR2:
-    cholqr_pass(T, 1, Q, d, m, p.gram_parts, gram, Rinv, dev_status, s);   // two passes
+    skinny_product(A, Q, Y, d, m, ns, s);
+    cholqr_pass(Y, T, d, m, p.gram_parts, gram, Lf, dev_status, s);  // Cholesky-QR2:
+    cholqr_pass(T, Q, d, m, p.gram_parts, gram, Lf, dev_status, s);  // two passes
   }
   // R3/R4: Rayleigh-Ritz, lambda, rho, U
-  skinny_kernel<<<skinny_grid, kRT, 0, s>>>(A, Q, Y, d, m, kslice);
-  gram_partial_kernel<<<p.gram_parts, kRT, 0, s>>>(Q, 1, Y, ns, d, m, gram);
+  skinny_product(A, Q, Y, d, m, ns, s);
+  gram_partial_kernel<<<p.gram_parts, kRT, 0, s>>>(Q, Y, d, m, gram);
   rr_kernel<<<1, kST, kRRSmem, s>>>(gram, p.gram_parts, m, r, A, d, Vs, lambda, rho, dev_status);
   form_u_kernel<<<(d * r + kRT - 1) / kRT, kRT, 0, s>>>(Q, Vs, d, m, r, U);
   return cudaGetLastError();

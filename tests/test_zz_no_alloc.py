@@ -38,19 +38,20 @@ def _compare(ref, got, A_ref, A_got, N):
     assert np.linalg.norm(M1 - M0) / np.linalg.norm(M0) < 1e-2
 
 
-@pytest.mark.parametrize("N,d,dtype", [(8192, 1536, "bf16"), (4096, 4096, "bf16"), (2048, 512, "f32")])
-def test_noalloc_refresh_matches_regular_refresh_twice(N, d, dtype):
+@pytest.mark.parametrize("N,d,dtype,rank,over", [(8192, 1536, "bf16", 32, 16), (4096, 4096, "bf16", 32, 16),
+                                                 (2048, 512, "f32", 32, 16), (4096, 4096, "bf16", 48, 16)])
+def test_noalloc_refresh_matches_regular_refresh_twice(N, d, dtype, rank, over):
     Q = synth.haar_orthogonal(d, 77 + d)
     X = synth.to_storage(synth.activations(N, Q, synth.column_power(d, 1.0), 78), dtype)
     Xd = torch.from_numpy(X).to(DEV)
     if dtype == "bf16":
         Xd = Xd.to(torch.bfloat16)
     A_ref = torch.empty((d, d), device=DEV, dtype=torch.float32)
-    ref = ops.factor_refresh(Xd, 32, 16, 4, 9, A_out=A_ref)
+    ref = ops.factor_refresh(Xd, rank, over, 4, 9, A_out=A_ref)
     first = None
     for call in range(2):
         A_got = torch.empty((d, d), device=DEV, dtype=torch.float32)
-        got = ops.factor_refresh_noalloc(Xd, A_got, 32, 16, 4, 9)
+        got = ops.factor_refresh_noalloc(Xd, A_got, rank, over, 4, 9)
         torch.cuda.synchronize()
         _compare(ref, got, A_ref, A_got, N)
         if first is None:
