@@ -6,11 +6,12 @@ Workload (one step): the Llama-600M-sized stand-in stack of 24 layers x
 gradients (528.5 M elements, 1.06 GB).  Selective deployment: o and down
 are whitened at rank 32, qkv and up take the Euclidean per-block E4M3
 codec.  A step runs the whole per-step hot path of the paper:
-  * factor refresh of one whitened layer (A = X^T X / N on 8192 tokens,
-    subspace iteration, Rayleigh-Ritz) -- 48 whitened layers refreshed every
-    K = 50 steps (section V.E, Algorithm 1) is ~one refresh per step;
+  * every K_REFRESH = 50 steps (section V.E, Algorithm 1), the factor
+    refresh of all 48 whitened layers (A = X^T X / N on 8192 tokens each,
+    subspace iteration, Rayleigh-Ritz) in one batched call; timed steps
+    0, 50, 100, ... carry it, so the default 50 timed steps hold exactly one;
   * encode of all 96 gradients, then decode of all 96;
-  * the one-step round-trip error of the refreshed layer.
+  * the one-step round-trip error of one whitened layer.
 value = gradient bytes of the stack / step time (GB/s).
 
 Multi-GPU (`--gpus N` under torchrun): replicas only -- the codec has no
@@ -44,13 +45,14 @@ WORKLOAD = ("llama600m-standin stack: 24 x {qkv 4608x1536, o 1536x1536, up 4096x
             "bf16 gradients; o/down whitened rank 32 (refresh N=8192), qkv/up Euclidean; E4M3 block 128")
 REFRESH_N = 8192
 RANK, OVERSAMPLE, ITERS = 32, 16, 4
+K_REFRESH = 50
 HBM_FALLBACK = 6650.0
 
 
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=K_REFRESH)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="gift", choices=["gift", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
@@ -183,30 +185,33 @@ def build_workload(torch, ops, synth, dev, depth, seed):
     err = torch.empty((3,), device=dev, dtype=torch.float64)
     wl = [L for L in layers if L.rank > 0]
     el = [L for L in layers if L.rank == 0]
+    jobs = ops.make_refresh_jobs([(w["X"], w["layer"].U, w["layer"].lam, w["layer"].rho, w["ws"], w["st"],
+                                   w["seed"], None) for w in whitened])
     return dict(layers=layers, whitened=whitened, G_all=G_all, Gh_all=Gh_all, C_all=C_all, S_all=S_all,
-                n_el=n_el, ews=ews, err=err,
+                n_el=n_el, ews=ews, err=err, jobs=jobs,
                 n_wh=sum(L.d_out * L.d_in for L in wl), n_eu=sum(L.d_out * L.d_in for L in el),
                 packed_wh=ops.make_layers(wl), n_packed_wh=len(wl),
                 packed_eu=ops.make_layers(el), n_packed_eu=len(el))
 
 
-def refresh(ops, w, stream=None):
-    L = w["layer"]
-    ops.factor_refresh(w["X"], RANK, OVERSAMPLE, ITERS, w["seed"], ws=w["ws"], dev_status=w["st"],
-                       out=(L.U, L.lam, L.rho), stream=stream)
+def refresh_all(ops, W):
+    """Factor refresh of every whitened layer in one batched call."""
+    ops.factor_refresh_many(W["jobs"], len(W["whitened"]), RANK, OVERSAMPLE, ITERS)
 
 
 PHASES = ("refresh", "encode_euclid", "encode_whitened", "decode_euclid", "decode_whitened", "error")
 
 
 def step(ops, W, k, ev=None):
-    """One step: refresh one whitened layer, encode and decode all 96 gradients
-    (each codec phase is one grouped launch), round-trip error of that layer.
+    """Step k: on every K_REFRESH-th step the batched refresh of all whitened
+    layers; then encode and decode all 96 gradients (each codec phase is one
+    grouped launch) and the round-trip error of one whitened layer.
     If `ev` (len(PHASES)+1 events) is given, phase boundaries are recorded."""
     w = W["whitened"][k % len(W["whitened"])]
     rec = (lambda i: ev[i].record()) if ev else (lambda i: None)
     rec(0)
-    refresh(ops, w)
+    if k % K_REFRESH == 0:
+        refresh_all(ops, W)
     rec(1)
     ops.encode_many(W["packed_eu"], W["n_packed_eu"])
     rec(2)
@@ -231,15 +236,23 @@ def phase_bytes(W):
             "decode_euclid": W["n_eu"] * dec, "decode_whitened": W["n_wh"] * dec + u_bytes}
 
 
-def count_launches(torch, ops, W):
-    """Kernels of libgift launched by one step, counted with the CUDA profiler (untimed pass)."""
+def count_launches(torch, ops, W, K):
+    """libgift kernels launched inside a timed region of K steps, counted with
+    the CUDA profiler on an untimed refresh step and an untimed codec step."""
     try:
         from torch.profiler import ProfilerActivity, profile
-        with profile(activities=[ProfilerActivity.CUDA]) as prof:
-            step(ops, W, 0)
-            torch.cuda.synchronize()
-        names = [e.name for e in prof.events() if e.device_type.name == "CUDA"]
-        return sum(1 for n in names if "gift" in n), sorted(set(n for n in names if "gift" in n))
+
+        def run(k):
+            with profile(activities=[ProfilerActivity.CUDA]) as prof:
+                step(ops, W, k)
+                torch.cuda.synchronize()
+            names = [e.name for e in prof.events() if e.device_type.name == "CUDA"]
+            return [n for n in names if "gift" in n]
+
+        with_refresh, plain = run(0), run(1)
+        n_ref = (K + K_REFRESH - 1) // K_REFRESH
+        total = n_ref * len(with_refresh) + (K - n_ref) * len(plain)
+        return total, sorted(set(with_refresh))
     except Exception as e:  # pragma: no cover
         return None, [f"profiler unavailable: {e}"]
 
@@ -297,12 +310,11 @@ def run_gpu(args):
             dist.barrier()
 
     W = build_workload(torch, ops, synth, dev, args.depth, seed=1234 + rank)
-    for w in W["whitened"]:
-        refresh(ops, w)
+    refresh_all(ops, W)
     torch.cuda.synchronize()
 
     for k in range(args.warmup):
-        step(ops, W, k)
+        step(ops, W, k)  # step 0 includes a batched refresh
     torch.cuda.synchronize()
 
     # ---- timed region: device resident inputs (1.06 GB of G > 126 MB L2) ----
@@ -337,47 +349,53 @@ def run_gpu(args):
                 "achieved": achieved, "peak": peak, "peak_source": peak_kind, "unit": "GB/s",
                 "frac": achieved / peak, "traffic": None}
     codec_ms = sum(pm[n] for n in pb)
+    ref_steps = [k for k in range(K) if k % K_REFRESH == 0]
     codec = {"phase_ms": pm,
+             "refresh_batched_ms": float(np.mean([phase[k, 0] for k in ref_steps])) if ref_steps else None,
+             "refresh_layers": len(W["whitened"]),
              "phase_gbs": {n: pb[n] / (pm[n] * 1e-3) / 1e9 for n in pb},
              "phase_roofline_frac": {n: pb[n] / (pm[n] * 1e-3) / 1e9 / peak for n in pb},
              "codec_gradient_gbs": g_bytes / (codec_ms * 1e-3) / 1e9,
              "codec_roofline_frac": sum(pb.values()) / (codec_ms * 1e-3) / 1e9 / peak}
 
-    launches, names = count_launches(torch, ops, W)
+    launches, names = count_launches(torch, ops, W, K)
 
-    # ---- end to end through host buffers ----
+    # ---- end to end through host buffers: the same schedule, with every
+    # step's gradients copied in from pinned host memory, the activations of
+    # all whitened layers copied in on refresh steps, and G_hat copied back ----
     e2e = None
     if not args.no_e2e:
         G_host = torch.empty((W["n_el"],), dtype=torch.bfloat16, pin_memory=True)
         G_host.copy_(W["G_all"].cpu())
         Gh_host = torch.empty_like(G_host, pin_memory=True)
-        X_host = {id(w): w["X"].cpu().pin_memory() for w in W["whitened"][:2]}
+        X_host = [w["X"].cpu().pin_memory() for w in W["whitened"]]
         err_host = torch.empty((3,), dtype=torch.float64, pin_memory=True)
-        Ke = max(3, min(K, 10))
+        x_bytes = sum(x.numel() * 2 for x in X_host)
 
         def e2e_step(k):
-            w = W["whitened"][k % 2]
             W["G_all"].copy_(G_host, non_blocking=True)
-            w["X"].copy_(X_host[id(w)], non_blocking=True)
-            step(ops, W, k % 2)
+            if k % K_REFRESH == 0:
+                for w, xh in zip(W["whitened"], X_host):
+                    w["X"].copy_(xh, non_blocking=True)
+            step(ops, W, k)
             Gh_host.copy_(W["Gh_all"], non_blocking=True)
             err_host.copy_(W["err"], non_blocking=True)
 
-        e2e_step(0)
+        e2e_step(1)
         torch.cuda.synchronize()
         barrier()
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
         a.record()
-        for k in range(Ke):
+        for k in range(K):
             e2e_step(k)
         b.record()
         torch.cuda.synchronize()
         ms_e = max_over_ranks(a.elapsed_time(b), dev)
-        x_bytes = sum(W["whitened"][k % 2]["X"].numel() * 2 for k in range(Ke)) / Ke
-        e2e = {"value": world * g_bytes / (ms_e / Ke * 1e-3) / 1e9, "unit": UNIT,
-               "h2d_bytes_per_step": int(g_bytes + x_bytes), "d2h_bytes_per_step": int(g_bytes + 24),
-               "ms_per_step": ms_e / Ke}
+        n_ref = (K + K_REFRESH - 1) // K_REFRESH
+        e2e = {"value": job_value(world, g_bytes, ms_e / K), "unit": UNIT,
+               "h2d_bytes_per_step": int(g_bytes + n_ref * x_bytes / K), "d2h_bytes_per_step": int(g_bytes + 24),
+               "ms_per_step": ms_e / K}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -116,6 +116,38 @@ gift_status gift_factor_refresh(const void* X, gift_dtype xdt, int64_t N, int64_
   return cuda_status(launch_refresh(p, X, xdt, U, lambda, rho, A_out, ws, dev_status, (cudaStream_t)stream));
 }
 
+gift_status gift_factor_refresh_many(const gift_refresh_job* jobs, int n, int rank, int oversample, int iters,
+                                     gift_stream_t stream) {
+  if (n < 0 || (n > 0 && !jobs)) return GIFT_ERR_INVALID_ARG;
+  if (iters < 0 || iters > 1000) return GIFT_ERR_INVALID_ARG;
+  for (int i = 0; i < n; ++i) {
+    const gift_refresh_job& J = jobs[i];
+    if (!J.X || !J.U || !J.lambda || !J.rho) return GIFT_ERR_INVALID_ARG;
+    if (!dtype_ok(J.xdt)) return GIFT_ERR_INVALID_ARG;
+    size_t need = 0;
+    gift_status st = gift_refresh_workspace_size(J.N, J.d_in, rank, oversample, J.A_out != nullptr, &need);
+    if (st != GIFT_OK) return st;
+    if (need > 0 && (!J.ws || J.ws_bytes < need)) return GIFT_ERR_WORKSPACE;
+    if (!aligned16(J.X) || !aligned16(J.U) || !aligned(J.lambda, 4) || !aligned(J.rho, 4)) return GIFT_ERR_ALIGN;
+    if ((J.A_out && !aligned16(J.A_out)) || (J.ws && !aligned16(J.ws)) ||
+        (J.dev_status && !aligned(J.dev_status, 4)))
+      return GIFT_ERR_ALIGN;
+  }
+  if (n == 0) return GIFT_OK;
+  gift_status st = device_ok();
+  if (st != GIFT_OK) return st;
+  std::vector<RefreshPlan> plans(n);
+  std::vector<RefreshIO> io(n);
+  for (int i = 0; i < n; ++i) {
+    const gift_refresh_job& J = jobs[i];
+    refresh_plan(J.N, J.d_in, rank, oversample, J.A_out != nullptr, &plans[i]);
+    plans[i].iters = iters;
+    plans[i].seed = J.seed;
+    io[i] = RefreshIO{J.X, (gift_dtype)J.xdt, J.U, J.lambda, J.rho, J.A_out, J.ws, J.dev_status};
+  }
+  return cuda_status(launch_refresh_batch(plans.data(), io.data(), n, (cudaStream_t)stream));
+}
+
 // ---------------------------------------------------------------------------
 gift_status gift_encode(const void* G, gift_dtype gdt, int64_t d_out, int64_t d_in, const float* U,
                         const float* lambda, const float* rho, int rank, uint8_t* codes, float* scales,

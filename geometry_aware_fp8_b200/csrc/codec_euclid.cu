@@ -145,6 +145,8 @@ GIFT_DEV int find_layer(const int64_t* pre, int n, int64_t b) {
   return lo;
 }
 
+// Two blocks per thread group per iteration: both blocks' loads are issued
+// before either is used, doubling the bytes in flight per thread.
 template <typename T>
 __global__ void __launch_bounds__(256) euclid_encode_group_kernel(const __grid_constant__ EuclidGroup g) {
   __shared__ int64_t pre[kGroupMax + 1];
@@ -152,22 +154,49 @@ __global__ void __launch_bounds__(256) euclid_encode_group_kernel(const __grid_c
   __syncthreads();
   const int sub = threadIdx.x & 7;
   const int64_t total = pre[g.n];
-  const int64_t groups_per_grid = (int64_t)gridDim.x * (blockDim.x >> 3);
-  for (int64_t b = (int64_t)blockIdx.x * (blockDim.x >> 3) + (threadIdx.x >> 3); b < total; b += groups_per_grid) {
-    const int l = find_layer(pre, g.n, b);
-    const int64_t lb = b - pre[l];
-    const int64_t e0 = lb * kBlock + sub * 16;
-    float v[16];
-    Vec16<T>::load((const T*)g.src[l] + e0, v);
-    float m = 0.0f;
+  const int64_t G = (int64_t)gridDim.x * (blockDim.x >> 3);
+  for (int64_t b0 = (int64_t)blockIdx.x * (blockDim.x >> 3) + (threadIdx.x >> 3); b0 < total; b0 += 2 * G) {
+    const int64_t b1 = b0 + G;
+    const bool has1 = b1 < total;
+    const int l0 = find_layer(pre, g.n, b0);
+    const int l1 = has1 ? find_layer(pre, g.n, b1) : l0;
+    const int64_t e0 = (b0 - pre[l0]) * kBlock + sub * 16;
+    const int64_t e1 = has1 ? (b1 - pre[l1]) * kBlock + sub * 16 : e0;
+    float v0[16], v1[16];
+    Vec16<T>::load((const T*)g.src[l0] + e0, v0);
+    if (has1) Vec16<T>::load((const T*)g.src[l1] + e1, v1);
+    float m0 = 0.0f, m1 = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[i]));
-    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
-    const float inv = e4m3_inv_scale(m);
-    __stcs(reinterpret_cast<uint4*>((uint8_t*)g.dst[l] + e0), quantize16(v, inv));
-    if (sub == 0) g.scales[l][lb] = e4m3_scale(m, inv);
+    for (int i = 0; i < 16; ++i) {
+      m0 = fmaxf(m0, fabsf(v0[i]));
+      m1 = fmaxf(m1, fabsf(v1[i]));
+    }
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) {
+      m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, o));
+      m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, o));
+    }
+    const float i0 = e4m3_inv_scale(m0);
+    __stcs(reinterpret_cast<uint4*>((uint8_t*)g.dst[l0] + e0), quantize16(v0, i0));
+    if (sub == 0) g.scales[l0][b0 - pre[l0]] = e4m3_scale(m0, i0);
+    if (has1) {
+      const float i1 = e4m3_inv_scale(m1);
+      __stcs(reinterpret_cast<uint4*>((uint8_t*)g.dst[l1] + e1), quantize16(v1, i1));
+      if (sub == 0) g.scales[l1][b1 - pre[l1]] = e4m3_scale(m1, i1);
+    }
+  }
+}
+
+GIFT_DEV void dequant16(uint4 q, float s, float (&v)[16]) {
+  const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 a = e4m3x2_to_f32x2((uint16_t)(w[i] & 0xFFFF));
+    const float2 c = e4m3x2_to_f32x2((uint16_t)(w[i] >> 16));
+    v[4 * i] = a.x * s;
+    v[4 * i + 1] = a.y * s;
+    v[4 * i + 2] = c.x * s;
+    v[4 * i + 3] = c.y * s;
   }
 }
 
@@ -178,25 +207,29 @@ __global__ void __launch_bounds__(256) euclid_decode_group_kernel(const __grid_c
   __syncthreads();
   const int sub = threadIdx.x & 7;
   const int64_t total = pre[g.n];
-  const int64_t groups_per_grid = (int64_t)gridDim.x * (blockDim.x >> 3);
-  for (int64_t b = (int64_t)blockIdx.x * (blockDim.x >> 3) + (threadIdx.x >> 3); b < total; b += groups_per_grid) {
-    const int l = find_layer(pre, g.n, b);
-    const int64_t lb = b - pre[l];
-    const int64_t e0 = lb * kBlock + sub * 16;
-    const uint4 q = __ldcs(reinterpret_cast<const uint4*>((const uint8_t*)g.src[l] + e0));
-    const float s = __ldg(g.scales[l] + lb);
-    uint32_t w[4] = {q.x, q.y, q.z, q.w};
-    float v[16];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      float2 a = e4m3x2_to_f32x2((uint16_t)(w[i] & 0xFFFF));
-      float2 c = e4m3x2_to_f32x2((uint16_t)(w[i] >> 16));
-      v[4 * i] = a.x * s;
-      v[4 * i + 1] = a.y * s;
-      v[4 * i + 2] = c.x * s;
-      v[4 * i + 3] = c.y * s;
+  const int64_t G = (int64_t)gridDim.x * (blockDim.x >> 3);
+  for (int64_t b0 = (int64_t)blockIdx.x * (blockDim.x >> 3) + (threadIdx.x >> 3); b0 < total; b0 += 2 * G) {
+    const int64_t b1 = b0 + G;
+    const bool has1 = b1 < total;
+    const int l0 = find_layer(pre, g.n, b0);
+    const int l1 = has1 ? find_layer(pre, g.n, b1) : l0;
+    const int64_t lb0 = b0 - pre[l0], lb1 = has1 ? b1 - pre[l1] : lb0;
+    const int64_t e0 = lb0 * kBlock + sub * 16, e1 = lb1 * kBlock + sub * 16;
+    const uint4 q0 = __ldcs(reinterpret_cast<const uint4*>((const uint8_t*)g.src[l0] + e0));
+    const float s0 = __ldg(g.scales[l0] + lb0);
+    uint4 q1 = make_uint4(0, 0, 0, 0);
+    float s1 = 0.0f;
+    if (has1) {
+      q1 = __ldcs(reinterpret_cast<const uint4*>((const uint8_t*)g.src[l1] + e1));
+      s1 = __ldg(g.scales[l1] + lb1);
     }
-    Vec16<T>::store((T*)g.dst[l] + e0, v);
+    float v[16];
+    dequant16(q0, s0, v);
+    Vec16<T>::store((T*)g.dst[l0] + e0, v);
+    if (has1) {
+      dequant16(q1, s1, v);
+      Vec16<T>::store((T*)g.dst[l1] + e1, v);
+    }
   }
 }
 

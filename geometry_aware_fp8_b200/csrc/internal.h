@@ -72,5 +72,17 @@ void refresh_plan(int64_t N, int64_t d, int rank, int oversample, bool a_out_giv
                   bool no_split = false);
 cudaError_t launch_refresh(const RefreshPlan& p, const void* X, gift_dtype xdt, float* U, float* lambda,
                            float* rho, float* A_out, void* ws, uint32_t* dev_status, cudaStream_t s);
+// Many refreshes in one sequence of launches (same rank, oversample, iters).
+struct RefreshIO {
+  const void* X;
+  gift_dtype xdt;
+  float* U;
+  float* lambda;
+  float* rho;
+  float* A_out;
+  void* ws;
+  uint32_t* dev_status;
+};
+cudaError_t launch_refresh_batch(const RefreshPlan* plans, const RefreshIO* io, int n, cudaStream_t s);
 
 }  // namespace gift

@@ -29,6 +29,29 @@ constexpr double kCholTol = 1e-10;     // pivot / max diagonal below this: colum
 constexpr double kJacobiTol = 1e-14;   // off(B) / ||B||_F at convergence
 constexpr int kJacobiMaxSweeps = 40;
 
+// Per-layer view of one refresh problem; the small-matrix kernels take a
+// batch of these and pick their layer with blockIdx.z, so the refreshes of
+// many layers run side by side (one CTA per layer for the fp64 steps).
+constexpr int kMaxBatch = 64;
+struct RefLayer {
+  const float* A;   // d x d
+  float* buf[3];    // [0] Q (d x m), [1] Y (ns k-slices of d x m), [2] T (d x m)
+  double* gram;     // parts x m x m fp64 partial Gram matrices
+  double* Lf;       // Cholesky factor (m x m) + reciprocal diagonal (m)
+  double* Vs;       // m x r sorted Ritz vectors
+  float* U;
+  float* lambda;
+  float* rho;
+  uint32_t* st;
+  uint64_t seed;
+  int d, ns, parts, kslice;
+};
+struct RefBatch {
+  RefLayer L[kMaxBatch];
+  int n, m, r;
+};
+enum { kBufQ = 0, kBufY = 1, kBufT = 2 };
+
 GIFT_DEV uint64_t splitmix64(uint64_t x) {
   uint64_t z = x + 0x9E3779B97F4A7C15ull;
   z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
@@ -131,10 +154,12 @@ __global__ void syrk_reduce_kernel(const float* __restrict__ part, int splits, i
 }
 
 // Omega[i][j] = +1 if the top bit of splitmix64(seed ^ (i*m + j)) is 0, else -1.
-__global__ void omega_kernel(float* __restrict__ Y, int d, int m, uint64_t seed) {
-  const int64_t n = (int64_t)d * m;
+__global__ void omega_kernel(const __grid_constant__ RefBatch b) {
+  const RefLayer& L = b.L[blockIdx.z];
+  float* Y = L.buf[kBufQ];
+  const int64_t n = (int64_t)L.d * b.m;
   for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
-    const uint64_t h = splitmix64(seed ^ (uint64_t)e);
+    const uint64_t h = splitmix64(L.seed ^ (uint64_t)e);
     Y[e] = (h >> 63) ? -1.0f : 1.0f;
   }
 }
@@ -145,8 +170,13 @@ __global__ void omega_kernel(float* __restrict__ Y, int d, int m, uint64_t seed)
 // consumers add the slices in index order.
 constexpr int kSkK = 32;
 
-__global__ void __launch_bounds__(kRT) skinny_kernel(const float* __restrict__ A, const float* __restrict__ Q,
-                                                     float* __restrict__ Yp, int d, int m, int kslice) {
+__global__ void __launch_bounds__(kRT) skinny_kernel(const __grid_constant__ RefBatch b, int src, int dst) {
+  const RefLayer& Lr = b.L[blockIdx.z];
+  const int d = Lr.d, m = b.m, kslice = Lr.kslice;
+  if ((int)blockIdx.x >= d / 64 || (int)blockIdx.y >= Lr.ns) return;
+  const float* __restrict__ A = Lr.A;
+  const float* __restrict__ Q = Lr.buf[src];
+  float* __restrict__ Yp = Lr.buf[dst];
   __shared__ __align__(16) float As[kSkK][64 + 4];  // As[k][row]
   __shared__ __align__(16) float Qs[kSkK][64];
   const int row0 = blockIdx.x * 64;
@@ -195,7 +225,12 @@ __global__ void __launch_bounds__(kRT) skinny_kernel(const float* __restrict__ A
 }
 
 // Y[0..n) += Y[s n .. (s+1) n) for s = 1..ns-1, in slice order.
-__global__ void fold_slices_kernel(float* __restrict__ Y, int ns, int64_t n) {
+__global__ void fold_slices_kernel(const __grid_constant__ RefBatch b, int which) {
+  const RefLayer& L = b.L[blockIdx.z];
+  const int ns = L.ns;
+  if (ns < 2) return;
+  float* __restrict__ Y = L.buf[which];
+  const int64_t n = (int64_t)L.d * b.m;
   for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
     float v = Y[e];
     for (int s = 1; s < ns; ++s) v += Y[s * n + e];
@@ -208,9 +243,13 @@ __global__ void fold_slices_kernel(float* __restrict__ Y, int ns, int64_t n) {
 // block of entries (4 ti.., 4 tj..).
 constexpr int kGramRows = 64;
 
-__global__ void __launch_bounds__(kRT) gram_partial_kernel(const float* __restrict__ Ya,
-                                                           const float* __restrict__ Yb, int d, int m,
-                                                           double* __restrict__ part) {
+__global__ void __launch_bounds__(kRT) gram_partial_kernel(const __grid_constant__ RefBatch bt, int wa, int wb) {
+  const RefLayer& Lr = bt.L[blockIdx.z];
+  const int d = Lr.d, m = bt.m;
+  if ((int)blockIdx.x >= Lr.parts) return;
+  const float* __restrict__ Ya = Lr.buf[wa];
+  const float* __restrict__ Yb = Lr.buf[wb];
+  double* __restrict__ part = Lr.gram;
   __shared__ __align__(16) float Sa[64][64];
   __shared__ __align__(16) float Sb[64][64];
   const int p = blockIdx.x;
@@ -267,8 +306,12 @@ constexpr int kST = 1024;  // threads of the single-CTA small-matrix kernels
 // (L[:, j] = e_j, flagged), so that column of Q comes out zero.
 // Output: Lout (m x m, row-major, lower part + diagonal), inv[j] = 1/L[j][j]
 // (0 for dropped columns).
-__global__ void __launch_bounds__(kST) chol_kernel(const double* __restrict__ part, int nparts, int m,
-                                                   double* __restrict__ Lout, uint32_t* __restrict__ dev_status) {
+__global__ void __launch_bounds__(kST) chol_kernel(const __grid_constant__ RefBatch bt) {
+  const RefLayer& Lr = bt.L[blockIdx.z];
+  const double* __restrict__ part = Lr.gram;
+  const int nparts = Lr.parts, m = bt.m;
+  double* __restrict__ Lout = Lr.Lf;
+  uint32_t* __restrict__ dev_status = Lr.st;
   extern __shared__ double sm[];
   const int ld = 65;
   double* G = sm;  // m x m
@@ -345,8 +388,12 @@ __global__ void __launch_bounds__(kST) chol_kernel(const double* __restrict__ pa
 // q_c = (y_c - sum_{k<c} q_k L[c][k]) / L[c][c] (fp64), q_c = 0 for dropped
 // columns.  One warp per row: lane l owns columns l and l+32, the owner of
 // column c finishes q_c and broadcasts it.
-__global__ void __launch_bounds__(kRT) qr_apply_kernel(const float* __restrict__ Yi, const double* __restrict__ L,
-                                                       float* __restrict__ Qo, int d, int m) {
+__global__ void __launch_bounds__(kRT) qr_apply_kernel(const __grid_constant__ RefBatch bt, int src, int dst) {
+  const RefLayer& Lr = bt.L[blockIdx.z];
+  const int d = Lr.d, m = bt.m;
+  const float* __restrict__ Yi = Lr.buf[src];
+  const double* __restrict__ L = Lr.Lf;
+  float* __restrict__ Qo = Lr.buf[dst];
   __shared__ double Ls[64 * 65];
   __shared__ double inv[64];
   for (int e = threadIdx.x; e < m * m; e += kRT) Ls[(e / m) * 65 + e % m] = L[e];
@@ -381,10 +428,15 @@ __global__ void __launch_bounds__(kRT) qr_apply_kernel(const float* __restrict__
 // entries of pairs a and b, and V' = V J is updated two entries at a time.
 // Eigenvalues are sorted descending; lambda, rho and the sorted eigenvectors
 // (Vs, m x r) are written.
-__global__ void __launch_bounds__(kST) rr_kernel(const double* __restrict__ part, int nparts, int m, int r,
-                                                 const float* __restrict__ A, int d, double* __restrict__ Vs,
-                                                 float* __restrict__ lambda, float* __restrict__ rho,
-                                                 uint32_t* __restrict__ dev_status) {
+__global__ void __launch_bounds__(kST) rr_kernel(const __grid_constant__ RefBatch bt) {
+  const RefLayer& Lr = bt.L[blockIdx.z];
+  const double* __restrict__ part = Lr.gram;
+  const int nparts = Lr.parts, m = bt.m, r = bt.r, d = Lr.d;
+  const float* __restrict__ A = Lr.A;
+  double* __restrict__ Vs = Lr.Vs;
+  float* __restrict__ lambda = Lr.lambda;
+  float* __restrict__ rho = Lr.rho;
+  uint32_t* __restrict__ dev_status = Lr.st;
   extern __shared__ double sm[];
   const int ld = 65;
   double* Bb0 = sm;
@@ -560,9 +612,13 @@ __global__ void __launch_bounds__(kST) rr_kernel(const double* __restrict__ part
 }
 
 // U = Q Vs (d x m times m x r), fp64 accumulation.
-__global__ void form_u_kernel(const float* __restrict__ Q, const double* __restrict__ Vs, int d, int m, int r,
-                              float* __restrict__ U) {
-  const int64_t n = (int64_t)d * r;
+__global__ void form_u_kernel(const __grid_constant__ RefBatch bt) {
+  const RefLayer& Lr = bt.L[blockIdx.z];
+  const float* __restrict__ Q = Lr.buf[kBufQ];
+  const double* __restrict__ Vs = Lr.Vs;
+  float* __restrict__ U = Lr.U;
+  const int m = bt.m, r = bt.r;
+  const int64_t n = (int64_t)Lr.d * r;
   for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
     const int64_t row = e / r;
     const int k = (int)(e % r);
@@ -622,76 +678,104 @@ void refresh_plan(int64_t N, int64_t d, int rank, int oversample, bool a_out_giv
   p->total = off;
 }
 
-// One Cholesky-QR pass: Qo = Yi R^{-1} with Yi^T Yi = R^T R.
-static void cholqr_pass(const float* Yi, float* Qo, int d, int m, int parts, double* gram, double* L,
-                        uint32_t* dev_status, cudaStream_t s) {
-  gram_partial_kernel<<<parts, kRT, 0, s>>>(Yi, Yi, d, m, gram);
-  chol_kernel<<<1, kST, kCholSmem, s>>>(gram, parts, m, L, dev_status);
-  int blocks = (d + 7) / 8;
-  if (blocks > 4 * kNumSMs) blocks = 4 * kNumSMs;
-  qr_apply_kernel<<<blocks, kRT, 0, s>>>(Yi, L, Qo, d, m);
-}
-
-// A Q into Y (k-slices folded into slice 0).
-static void skinny_product(const float* A, const float* Q, float* Y, int d, int m, int ns, cudaStream_t s) {
-  const int kslice = (d / ns + kSkK - 1) / kSkK * kSkK;
-  skinny_kernel<<<dim3(d / 64, ns), kRT, 0, s>>>(A, Q, Y, d, m, kslice);
-  if (ns > 1) {
-    const int64_t n = (int64_t)d * m;
-    int blocks = (int)((n + kRT - 1) / kRT);
-    if (blocks > 2 * kNumSMs) blocks = 2 * kNumSMs;
-    fold_slices_kernel<<<blocks, kRT, 0, s>>>(Y, ns, n);
-  }
-}
-
-cudaError_t launch_refresh(const RefreshPlan& p, const void* X, gift_dtype xdt, float* U, float* lambda, float* rho,
-                           float* A_out, void* ws, uint32_t* dev_status, cudaStream_t s) {
+cudaError_t launch_refresh_batch(const RefreshPlan* plans, const RefreshIO* io, int n, cudaStream_t s) {
   static unsigned long long chol_attr = 0, rr_attr = 0;
   cudaError_t e = ensure_smem_attr(chol_kernel, (int)kCholSmem, &chol_attr);
   if (e != cudaSuccess) return e;
   if ((e = ensure_smem_attr(rr_kernel, (int)kRRSmem, &rr_attr)) != cudaSuccess) return e;
-  char* w = (char*)ws;
-  const int d = (int)p.d, m = p.m, r = p.rank, ns = p.skinny_slices;
-  float* A = A_out ? A_out : (float*)(w + p.off_A);
-  float* Q = (float*)(w + p.off_Q);
-  float* Y = (float*)(w + p.off_Y);
-  float* T = (float*)(w + p.off_T);
-  double* gram = (double*)(w + p.off_gram);
-  double* Lf = (double*)(w + p.off_small);   // Cholesky factor + reciprocal diagonal
-  double* Vs = Lf + 64 * 64 + 64;            // after m*m + m doubles (m <= 64)
-  const float scale = (float)(1.0 / (double)p.N);
+  if (n <= 0) return cudaSuccess;
+  const int m = plans[0].m, r = plans[0].rank, iters = plans[0].iters;
+  for (int base = 0; base < n; base += kMaxBatch) {
+    const int cnt = n - base < kMaxBatch ? n - base : kMaxBatch;
+    static thread_local RefBatch B;
+    B.n = cnt;
+    B.m = m;
+    B.r = r;
+    int dmax = 0, nsmax = 1, pmax = 1;
+    for (int l = 0; l < cnt; ++l) {
+      const RefreshPlan& p = plans[base + l];
+      const RefreshIO& o = io[base + l];
+      char* w = (char*)o.ws;
+      const int d = (int)p.d;
+      float* A = o.A_out ? o.A_out : (float*)(w + p.off_A);
+      // R1: A = X^T X / N (one launch per layer; each fills the GPU)
+      bool used_tc = false;
+      e = launch_syrk_tc(o.X, o.xdt, p.N, d, A, (float*)(w + p.off_syrk), p.syrk_splits, o.dev_status, s,
+                         &used_tc);
+      if (e != cudaSuccess) return e;
+      if (!used_tc) {
+        const int nt = d / 64;
+        const int tiles = nt * (nt + 1) / 2;
+        const float scale = (float)(1.0 / (double)p.N);
+        if (o.xdt == GIFT_BF16)
+          syrk_simt_kernel<__nv_bfloat16><<<tiles, kRT, 0, s>>>((const __nv_bfloat16*)o.X, p.N, d, A, scale);
+        else
+          syrk_simt_kernel<float><<<tiles, kRT, 0, s>>>((const float*)o.X, p.N, d, A, scale);
+      }
+      RefLayer& L = B.L[l];
+      L.A = A;
+      L.buf[kBufQ] = (float*)(w + p.off_Q);
+      L.buf[kBufY] = (float*)(w + p.off_Y);
+      L.buf[kBufT] = (float*)(w + p.off_T);
+      L.gram = (double*)(w + p.off_gram);
+      L.Lf = (double*)(w + p.off_small);
+      L.Vs = L.Lf + 64 * 64 + 64;  // after m*m + m doubles (m <= 64)
+      L.U = o.U;
+      L.lambda = o.lambda;
+      L.rho = o.rho;
+      L.st = o.dev_status;
+      L.seed = p.seed;
+      L.d = d;
+      L.ns = p.skinny_slices;
+      L.parts = p.gram_parts;
+      L.kslice = (d / L.ns + kSkK - 1) / kSkK * kSkK;
+      dmax = d > dmax ? d : dmax;
+      nsmax = L.ns > nsmax ? L.ns : nsmax;
+      pmax = L.parts > pmax ? L.parts : pmax;
+    }
+    const int64_t dm = (int64_t)dmax * m;
+    const int ew_blocks = (int)((dm + kRT - 1) / kRT < 2 * kNumSMs ? (dm + kRT - 1) / kRT : 2 * kNumSMs);
+    const int qr_blocks = (dmax + 7) / 8 < 4 * kNumSMs ? (dmax + 7) / 8 : 4 * kNumSMs;
+    const dim3 g_ew(ew_blocks, 1, cnt), g_skinny(dmax / 64, nsmax, cnt), g_gram(pmax, 1, cnt), g_one(1, 1, cnt),
+        g_qr(qr_blocks, 1, cnt);
+    // one Cholesky-QR pass: dst = src R^{-1} with src^T src = R^T R
+    auto cholqr_pass = [&](int src, int dst) {
+      gram_partial_kernel<<<g_gram, kRT, 0, s>>>(B, src, src);
+      chol_kernel<<<g_one, kST, kCholSmem, s>>>(B);
+      qr_apply_kernel<<<g_qr, kRT, 0, s>>>(B, src, dst);
+    };
+    // A Q into Y, k-slices folded into slice 0
+    auto skinny_product = [&]() {
+      skinny_kernel<<<g_skinny, kRT, 0, s>>>(B, kBufQ, kBufY);
+      if (nsmax > 1) fold_slices_kernel<<<g_ew, kRT, 0, s>>>(B, kBufY);
+    };
+    // R2: randomised subspace iteration.  span(A Omega) = span(A orth(Omega)),
+    // so the +-1 start block (exact) is multiplied by A directly; with no
+    // iterations it is orthonormalised for the Rayleigh-Ritz step instead.
+    omega_kernel<<<g_ew, kRT, 0, s>>>(B);
+    if (iters == 0) {
+      cholqr_pass(kBufQ, kBufT);
+      cholqr_pass(kBufT, kBufQ);
+    }
+    for (int it = 0; it < iters; ++it) {
+      skinny_product();
+      cholqr_pass(kBufY, kBufT);  // Cholesky-QR2:
+      cholqr_pass(kBufT, kBufQ);  // two passes
+    }
+    // R3/R4: Rayleigh-Ritz, lambda, rho, U
+    skinny_product();
+    gram_partial_kernel<<<g_gram, kRT, 0, s>>>(B, kBufQ, kBufY);
+    rr_kernel<<<g_one, kST, kRRSmem, s>>>(B);
+    form_u_kernel<<<g_ew, kRT, 0, s>>>(B);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
 
-  // R1: A = X^T X / N
-  bool used_tc = false;
-  e = launch_syrk_tc(X, xdt, p.N, d, A, (float*)(w + p.off_syrk), p.syrk_splits, dev_status, s, &used_tc);
-  if (e != cudaSuccess) return e;
-  if (!used_tc) {
-    const int nt = d / 64;
-    const int tiles = nt * (nt + 1) / 2;
-    if (xdt == GIFT_BF16)
-      syrk_simt_kernel<__nv_bfloat16><<<tiles, kRT, 0, s>>>((const __nv_bfloat16*)X, p.N, d, A, scale);
-    else
-      syrk_simt_kernel<float><<<tiles, kRT, 0, s>>>((const float*)X, p.N, d, A, scale);
-  }
-  // R2: randomised subspace iteration.  span(A Omega) = span(A orth(Omega)), so
-  // the +-1 start block (exact) is multiplied by A directly; with no iterations
-  // it is orthonormalised for the Rayleigh-Ritz step instead.
-  omega_kernel<<<(d * m + kRT - 1) / kRT, kRT, 0, s>>>(Q, d, m, p.seed);
-  if (p.iters == 0) {
-    cholqr_pass(Q, T, d, m, p.gram_parts, gram, Lf, dev_status, s);
-    cholqr_pass(T, Q, d, m, p.gram_parts, gram, Lf, dev_status, s);
-  }
-  for (int it = 0; it < p.iters; ++it) {
-    skinny_product(A, Q, Y, d, m, ns, s);
-    cholqr_pass(Y, T, d, m, p.gram_parts, gram, Lf, dev_status, s);  // Cholesky-QR2:
-    cholqr_pass(T, Q, d, m, p.gram_parts, gram, Lf, dev_status, s);  // two passes
-  }
-  // R3/R4: Rayleigh-Ritz, lambda, rho, U
-  skinny_product(A, Q, Y, d, m, ns, s);
-  gram_partial_kernel<<<p.gram_parts, kRT, 0, s>>>(Q, Y, d, m, gram);
-  rr_kernel<<<1, kST, kRRSmem, s>>>(gram, p.gram_parts, m, r, A, d, Vs, lambda, rho, dev_status);
-  form_u_kernel<<<(d * r + kRT - 1) / kRT, kRT, 0, s>>>(Q, Vs, d, m, r, U);
-  return cudaGetLastError();
+cudaError_t launch_refresh(const RefreshPlan& p, const void* X, gift_dtype xdt, float* U, float* lambda, float* rho,
+                           float* A_out, void* ws, uint32_t* dev_status, cudaStream_t s) {
+  const RefreshIO io{X, xdt, U, lambda, rho, A_out, ws, dev_status};
+  return launch_refresh_batch(&p, &io, 1, s);
 }
 
 // Split-K reduction used by the tensor-core syrk.

@@ -25,7 +25,7 @@ STATUS = {0: "GIFT_OK", 1: "GIFT_ERR_INVALID_ARG", 2: "GIFT_ERR_SHAPE", 3: "GIFT
           4: "GIFT_ERR_WORKSPACE", 5: "GIFT_ERR_CUDA", 6: "GIFT_ERR_UNSUPPORTED"}
 
 EXPORTED = ("gift_status_string", "gift_version", "gift_refresh_workspace_size", "gift_factor_refresh",
-            "gift_factor_refresh_noalloc", "gift_encode", "gift_decode", "gift_encode_many", "gift_decode_many",
+            "gift_factor_refresh_noalloc", "gift_factor_refresh_many", "gift_encode", "gift_decode", "gift_encode_many", "gift_decode_many",
             "gift_error_workspace_size", "gift_roundtrip_error")
 
 
@@ -33,6 +33,15 @@ class GiftError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
         super().__init__(f"{where}: {STATUS.get(status, status)}")
+
+
+class RefreshJob(ctypes.Structure):
+    """Mirror of gift_refresh_job."""
+    _fields_ = [("X", ctypes.c_void_p), ("xdt", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("N", ctypes.c_int64), ("d_in", ctypes.c_int64), ("seed", ctypes.c_uint64),
+                ("U", ctypes.c_void_p), ("lambda_", ctypes.c_void_p), ("rho", ctypes.c_void_p),
+                ("A_out", ctypes.c_void_p), ("ws", ctypes.c_void_p), ("ws_bytes", ctypes.c_size_t),
+                ("dev_status", ctypes.c_void_p)]
 
 
 class Layer(ctypes.Structure):
@@ -63,6 +72,7 @@ def lib() -> ctypes.CDLL:
                                           vp, sz, vp, vp]
         L.gift_factor_refresh_noalloc.argtypes = [vp, i32, i64, i64, i32, i32, i32, ctypes.c_uint64, vp, vp, vp,
                                                   vp, vp, vp]
+        L.gift_factor_refresh_many.argtypes = [ctypes.POINTER(RefreshJob), i32, i32, i32, i32, vp]
         L.gift_encode.argtypes = [vp, i32, i64, i64, vp, vp, vp, i32, vp, vp, vp]
         L.gift_decode.argtypes = [vp, vp, i64, i64, vp, vp, vp, i32, vp, i32, vp]
         L.gift_encode_many.argtypes = [ctypes.POINTER(Layer), i32, vp]
@@ -167,6 +177,22 @@ def factor_refresh_noalloc(X: torch.Tensor, A_out: torch.Tensor, rank: int = 32,
                                              _ptr(U), _ptr(lam), _ptr(rho), _ptr(A_out), _ptr(dev_status),
                                              _stream(stream)), "gift_factor_refresh_noalloc")
     return U, lam, rho, dev_status
+
+
+def make_refresh_jobs(items):
+    """Pack [(X, U, lam, rho, ws, dev_status, seed, A_out or None), ...] into a gift_refresh_job array."""
+    arr = (RefreshJob * max(len(items), 1))()
+    for i, (X, U, lam, rho, ws, st, seed, A_out) in enumerate(items):
+        _cuda(X, U, lam, rho, ws, st, A_out)
+        arr[i] = RefreshJob(_ptr(X), _dt(X), 0, X.shape[0], X.shape[1], seed & (2**64 - 1), _ptr(U), _ptr(lam),
+                            _ptr(rho), _ptr(A_out), _ptr(ws), 0 if ws is None else ws.numel(), _ptr(st))
+    return arr
+
+
+def factor_refresh_many(jobs, n: int, rank: int = 32, oversample: int = 16, iters: int = 4, stream=None):
+    """Refresh n layers' factors in one batched sequence (see gift_factor_refresh_many)."""
+    _check(lib().gift_factor_refresh_many(jobs, n, rank, oversample, iters, _stream(stream)),
+           "gift_factor_refresh_many")
 
 
 def encode(G: torch.Tensor, U=None, lam=None, rho=None, rank: Optional[int] = None,

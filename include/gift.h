@@ -106,6 +106,35 @@ gift_status gift_factor_refresh(const void* X, gift_dtype xdt, int64_t N, int64_
                                 uint32_t* dev_status, gift_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * Refresh of many layers at once (section V.E, Algorithm 1 refreshes the
+ * factors of all whitened layers every K steps).  Same computation per job
+ * as gift_factor_refresh; the A = X^T X / N contraction runs per layer and
+ * all small fp64 steps of all layers run side by side (one CTA per layer),
+ * so the latency of n refreshes is close to that of one.
+ * `jobs` is a HOST array of n entries; every job has its own workspace of
+ * gift_refresh_workspace_size(N, d_in, rank, oversample, A_out != NULL)
+ * bytes.  rank, oversample and iters are shared by all jobs.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+  const void* X;          /* N x d_in, dtype xdt */
+  int32_t xdt;            /* gift_dtype */
+  int32_t reserved;       /* 0 */
+  int64_t N;
+  int64_t d_in;
+  uint64_t seed;
+  float* U;               /* d_in x rank */
+  float* lambda;          /* rank */
+  float* rho;             /* 1 */
+  float* A_out;           /* nullable, d_in x d_in */
+  void* ws;
+  size_t ws_bytes;
+  uint32_t* dev_status;   /* nullable */
+} gift_refresh_job;
+
+gift_status gift_factor_refresh_many(const gift_refresh_job* jobs /* host */, int n, int rank, int oversample,
+                                     int iters, gift_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * Factor refresh without any allocation.  The paper has no counterpart: this
  * entry point exists for callers that cannot hand the library a workspace,
  * e.g. code whose device memory is entirely owned by another allocator, or

@@ -162,3 +162,30 @@ def test_refresh_config4_full_size_properties():
     rel = abs(rho.item() - rho_ref) / rho_ref
     print(f"config4 rho {rho.item():.6e} vs trace identity {rho_ref:.6e} (rel {rel:.2e}); lambda_1 {lg[0]:.4f}")
     assert abs(rho.item() - rho_ref) <= rho_tol(rho_ref, fro / N, N, d, 32)
+
+
+def test_refresh_many_matches_single_refreshes_bitwise():
+    """The batched refresh runs the same arithmetic per layer, side by side:
+    each layer's result must equal its single refresh bit for bit (mixed
+    widths and dtypes in one batch)."""
+    specs = [(2048, 512, "f32", 3), (4096, 1536, "bf16", 4), (1024, 256, "bf16", 5), (8192, 1536, "bf16", 6)]
+    items, singles = [], []
+    for N, d, dtype, seed in specs:
+        Q = synth.haar_orthogonal(d, 100 + seed)
+        X = synth.to_storage(synth.activations(N, Q, synth.column_power(d, 1.0), 200 + seed), dtype)
+        Xd = torch.from_numpy(X).to(DEV)
+        if dtype == "bf16":
+            Xd = Xd.to(torch.bfloat16)
+        singles.append(ops.factor_refresh(Xd, 32, 16, 4, seed))
+        U = torch.empty((d, 32), device=DEV)
+        lam = torch.empty((32,), device=DEV)
+        rho = torch.empty((1,), device=DEV)
+        ws = torch.empty((ops.refresh_workspace_size(N, d, 32, 16),), device=DEV, dtype=torch.uint8)
+        st = torch.zeros((1,), device=DEV, dtype=torch.int32)
+        items.append((Xd, U, lam, rho, ws, st, seed, None))
+    jobs = ops.make_refresh_jobs(items)
+    ops.factor_refresh_many(jobs, len(items), 32, 16, 4)
+    torch.cuda.synchronize()
+    for (Xd, U, lam, rho, ws, st, seed, _), single in zip(items, singles):
+        assert torch.equal(U, single[0]) and torch.equal(lam, single[1]) and torch.equal(rho, single[2])
+        assert int(st.item()) == int(single[3].item())
