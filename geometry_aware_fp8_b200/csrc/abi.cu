@@ -60,7 +60,7 @@ gift_status check_codec_args(const void* G, int gdt, int64_t d_out, int64_t d_in
 // Whitened bf16 layers with rank 32 go to the tensor-core kernels when they
 // are built in; everything else runs on the CUDA-core kernels.
 inline bool use_tc(int dt, int rank, int64_t d_in) {
-  return dt == GIFT_BF16 && rank > 0 && tc_codec_available() && d_in <= 8192;
+  return dt == GIFT_BF16 && rank == GIFT_MAX_RANK && tc_codec_available() && d_in <= 8192;
 }
 
 }  // namespace

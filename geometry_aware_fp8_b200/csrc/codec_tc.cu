@@ -58,6 +58,7 @@ constexpr int kMaxPanels = 1536;
 
 struct alignas(64) EncJob {
   CUtensorMap tmG;  // bf16 [d_out][d_in], box [128][64], 128-byte swizzle
+  CUtensorMap tmU;  // fp32 U [d_in][32], box [128][32], 128-byte swizzle
   const float* U;
   const float* lambda;
   const float* rho;
@@ -150,23 +151,19 @@ GIFT_DEV void split_bf16(float x, float& hi, float& lo) {
   lo = x - hi;
 }
 
-// Row j of U (d_in x rank fp32) into registers, zero-padded to 32 values.
-GIFT_DEV void load_u_row(const float* __restrict__ U, int rank, int j, float (&u)[32]) {
-  const float* src = U + (int64_t)j * rank;
-  if (rank == 32) {
+// Row t of the U tile: TMA has placed U[j0 + t][0..31] there as fp32 (one
+// 128-byte swizzled row); it is replaced in place by its bf16 split
+// [hi 0..31 | lo 0..31], the same 128 bytes in the same swizzle.
+GIFT_DEV void convert_u_row_inplace(uint32_t tile, int t) {
+  float u[32];
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      float4 v = __ldg(reinterpret_cast<const float4*>(src) + q);
-      u[4 * q] = v.x; u[4 * q + 1] = v.y; u[4 * q + 2] = v.z; u[4 * q + 3] = v.w;
-    }
-  } else {
-#pragma unroll
-    for (int k = 0; k < 32; ++k) u[k] = k < rank ? __ldg(src + k) : 0.0f;
+  for (int q = 0; q < 8; ++q) {
+    const uint4 v = ld_shared_v4(tile + sw128(t, q));
+    u[4 * q] = __uint_as_float(v.x);
+    u[4 * q + 1] = __uint_as_float(v.y);
+    u[4 * q + 2] = __uint_as_float(v.z);
+    u[4 * q + 3] = __uint_as_float(v.w);
   }
-}
-
-// Row t of the swizzled [128][hi 32 | lo 32] bf16 U tile from its fp32 values.
-GIFT_DEV void store_u_row(const float (&u)[32], uint32_t tile, int t) {
   uint32_t hi[16], lo[16];
 #pragma unroll
   for (int k = 0; k < 16; ++k) {
@@ -190,9 +187,10 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
   const uint32_t sbase = smem_u32(smem);
   const uint32_t pc_tile = sbase + kStages * kStageBytes;
   uint64_t* bars = (uint64_t*)(smem + kStages * kStageBytes + kPcBytes);
-  uint64_t* full = bars;                  // [kStages] count 2: TMA tx + converter
+  uint64_t* full = bars;                  // [kStages] count 1: converter (stage ready for the MMA)
   uint64_t* empty = bars + kStages;       // [kStages] count 1
-  uint64_t* p_full = bars + 2 * kStages;  // count 1 (MMA commit)
+  uint64_t* tfull = bars + 2 * kStages;   // [kStages] count 1 + tx: TMA (G and fp32 U)
+  uint64_t* p_full = bars + 3 * kStages;  // count 1 (MMA commit)
   uint64_t* pc_full = p_full + 1;         // count 128 (epilogue)
   uint64_t* w_full = p_full + 2;          // [2] count 1
   uint64_t* w_empty = p_full + 4;         // [2] count 128
@@ -205,8 +203,9 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
   if (threadIdx.x == 0) {
     failed = 0;
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full[s], 2);
+      mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
+      mbar_init(&tfull[s], 1);
     }
     mbar_init(p_full, 1);
     mbar_init(pc_full, 128);
@@ -240,39 +239,30 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
         const EncJob& J = p.jobs[st.job()];
         const uint64_t pol = st.pass == 0 ? keep : drop;
         const uint32_t dst = sbase + s * kStageBytes;
-        mbar_arrive_expect_tx(&full[s], kGBytes);
-        tma_load_2d_hint(dst, &J.tmG, &full[s], st.chunk() * kChunk, st.panel() * kPanel, pol);
-        tma_load_2d_hint(dst + kGHalf, &J.tmG, &full[s], st.chunk() * kChunk + 64, st.panel() * kPanel, pol);
+        mbar_arrive_expect_tx(&tfull[s], kGBytes + kUBytes);
+        tma_load_2d_hint(dst, &J.tmG, &tfull[s], st.chunk() * kChunk, st.panel() * kPanel, pol);
+        tma_load_2d_hint(dst + kGHalf, &J.tmG, &tfull[s], st.chunk() * kChunk + 64, st.panel() * kPanel, pol);
+        tma_load_2d_hint(dst + kGBytes, &J.tmU, &tfull[s], 0, st.chunk() * kChunk, keep);
       }
     }
   } else if (warp >= 4 && warp < 8) {
-    // ---------------- converters: U rows -> bf16 hi/lo tile, one row each ----------------
-    // The next step's U row is loaded before waiting for this step's stage.
+    // ---------------- converters: fp32 U rows -> bf16 hi/lo, in place, one row each ----------------
     // Exit decisions are voted at a named barrier so all 128 threads leave
     // at the same step.
     const int t = threadIdx.x - 128;
     uint32_t step = 0;
-    Steps<EncParams> st(p, beg, end);
-    float u_next[32];
-    if (st.valid()) load_u_row(p.jobs[st.job()].U, p.jobs[st.job()].rank, st.chunk() * kChunk + t, u_next);
-    while (st.valid()) {
-      float u[32];
-#pragma unroll
-      for (int k = 0; k < 32; ++k) u[k] = u_next[k];
+    for (Steps<EncParams> st(p, beg, end); st.valid(); st.next(), ++step) {
       const int s = step % kStages;
       const uint32_t use = step / kStages;
-      st.next();
-      if (st.valid()) load_u_row(p.jobs[st.job()].U, p.jobs[st.job()].rank, st.chunk() * kChunk + t, u_next);
-      const bool ok = step < kStages || mbar_wait(&empty[s], (use - 1) & 1u, kWaitLimit);
+      const bool ok = mbar_wait(&tfull[s], use & 1u, kWaitLimit);
       if (named_sync_or(1, 128, !ok)) {
         failed = 1;
         break;
       }
-      store_u_row(u, sbase + s * kStageBytes + kGBytes, t);
+      convert_u_row_inplace(sbase + s * kStageBytes + kGBytes, t);
       fence_async_shared();
       named_sync(1, 128);
       if (t == 0) mbar_arrive(&full[s]);
-      ++step;
     }
   } else if (warp == 8) {
     // ---------------- MMA issuer ----------------
@@ -472,6 +462,7 @@ constexpr uint32_t kIdescD2 = umma_idesc_bf16(128, 64, 0, 1);
 
 struct alignas(64) DecJob {
   CUtensorMap tmC;  // uint8 codes [d_out][d_in], box [128][128], 128-byte swizzle
+  CUtensorMap tmU;  // fp32 U [d_in][32], box [128][32], 128-byte swizzle
   const float* U;
   const float* lambda;
   const float* rho;
@@ -550,38 +541,30 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
           break;
         }
         const DecJob& J = p.jobs[st.job()];
-        mbar_arrive_expect_tx(&cfull[s], kDCodes);
-        tma_load_2d_hint(sbase + s * kDStageBytes, &J.tmC, &cfull[s], st.chunk() * kChunk, st.panel() * kPanel,
+        const uint32_t dst = sbase + s * kDStageBytes;
+        mbar_arrive_expect_tx(&cfull[s], kDCodes + kUBytes);
+        tma_load_2d_hint(dst, &J.tmC, &cfull[s], st.chunk() * kChunk, st.panel() * kPanel,
                          st.pass == 0 ? keep : drop);
+        tma_load_2d_hint(dst + kDCodes + kDQ, &J.tmU, &cfull[s], 0, st.chunk() * kChunk, keep);
       }
     }
   } else if (warp >= 4 && warp < 8) {
-    // ---------------- converters: U tile, and in the first pass the bf16 codes ----------------
+    // ---------------- converters: U tile in place, and in the first pass the bf16 codes ----------------
     const int t = threadIdx.x - 128;
     uint32_t step = 0;
-    Steps<DecParams> st(p, beg, end);
-    float u_next[32];
-    if (st.valid()) load_u_row(p.jobs[st.job()].U, p.jobs[st.job()].rank, st.chunk() * kChunk + t, u_next);
-    while (st.valid()) {
-      float u[32];
-#pragma unroll
-      for (int k = 0; k < 32; ++k) u[k] = u_next[k];
+    for (Steps<DecParams> st(p, beg, end); st.valid(); st.next(), ++step) {
       const int s = step % kDStages;
       const uint32_t use = step / kDStages;
-      const int pass = st.pass;
-      st.next();
-      if (st.valid()) load_u_row(p.jobs[st.job()].U, p.jobs[st.job()].rank, st.chunk() * kChunk + t, u_next);
-      const bool ok = step < kDStages || mbar_wait(&empty[s], (use - 1) & 1u, kWaitLimit);
+      const bool ok = mbar_wait(&cfull[s], use & 1u, kWaitLimit);
       if (named_sync_or(1, 128, !ok)) {
         failed = 1;
         break;
       }
       const uint32_t c_tile = sbase + s * kDStageBytes;
       const uint32_t q_tile = c_tile + kDCodes;
-      store_u_row(u, q_tile + kDQ, t);
-      if (pass == 0) {
-        // the codes of row t: wait for the TMA, then widen to bf16
-        if (!mbar_wait(&cfull[s], use & 1u, kWaitLimit)) failed = 1;
+      convert_u_row_inplace(q_tile + kDQ, t);
+      if (st.pass == 0) {
+        // the codes of row t, widened to bf16
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
           const uint4 v = ld_shared_v4(c_tile + sw128(t, q));
@@ -601,7 +584,6 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
       fence_async_shared();
       named_sync(1, 128);
       if (t == 0) mbar_arrive(&full[s]);
-      ++step;
     }
   } else if (warp == 8) {
     // ---------------- MMA issuer ----------------
@@ -852,7 +834,8 @@ cudaError_t launch_whiten_encode_tc(const TcLayer* layers, int n, cudaStream_t s
       const TcLayer& L = layers[base + l];
       EncJob& J = P.jobs[l];
       if (!make_tmap_2d(&J.tmG, L.G, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)L.d_out, (uint64_t)L.d_in,
-                        kPanel, 64))
+                        kPanel, 64) ||
+          !make_tmap_2d(&J.tmU, L.U, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, (uint64_t)L.d_in, 32, kChunk, 32))
         return cudaErrorInvalidValue;
       J.U = L.U;
       J.lambda = L.lambda;
@@ -904,7 +887,8 @@ cudaError_t launch_whiten_decode_tc(const TcLayer* layers, int n, cudaStream_t s
       const TcLayer& L = layers[base + l];
       DecJob& J = P.jobs[l];
       if (!make_tmap_2d(&J.tmC, L.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)L.d_out, (uint64_t)L.d_in,
-                        kPanel, kChunk))
+                        kPanel, kChunk) ||
+          !make_tmap_2d(&J.tmU, L.U, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, (uint64_t)L.d_in, 32, kChunk, 32))
         return cudaErrorInvalidValue;
       J.U = L.U;
       J.lambda = L.lambda;
