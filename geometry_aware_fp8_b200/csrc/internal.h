@@ -64,14 +64,26 @@ struct RefreshPlan {
   int gram_parts;       // partial Gram blocks
   int syrk_splits;      // split-K partial sums of A
   int skinny_slices;    // k-slices of the A Q product
+  bool tc_skinny;       // iteration products on the tensor cores (needs the bf16 splits)
   // workspace carve-up (byte offsets from ws)
-  size_t off_A, off_Q, off_Y, off_T, off_gram, off_small, off_syrk, total;
+  size_t off_A, off_Q, off_Y, off_T, off_gram, off_small, off_syrk, off_Ah, off_Al, off_Qs, total;
 };
 // no_split: one token range for A and one k-slice for A Q (smallest workspace)
 void refresh_plan(int64_t N, int64_t d, int rank, int oversample, bool a_out_given, RefreshPlan* p,
                   bool no_split = false);
 cudaError_t launch_refresh(const RefreshPlan& p, const void* X, gift_dtype xdt, float* U, float* lambda,
                            float* rho, float* A_out, void* ws, uint32_t* dev_status, cudaStream_t s);
+// A Q on the tensor cores (bf16 hi/lo split operands), one k-slice per CTA row.
+constexpr int kSkinnyMaxBatch = 48;
+struct SkinnyTcJob {
+  const void* Ah;  // bf16 d x d
+  const void* Al;  // bf16 d x d
+  const void* Qs;  // bf16 d x 128: [Q_hi (64) | Q_lo (64)]
+  float* Yp;       // ns k-slices of d x m fp32
+  int d, ns, kslice;
+};
+cudaError_t launch_skinny_tc(const SkinnyTcJob* jobs, int n, int m, cudaStream_t s);
+
 // Many refreshes in one sequence of launches (same rank, oversample, iters).
 struct RefreshIO {
   const void* X;

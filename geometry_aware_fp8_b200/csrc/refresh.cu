@@ -35,6 +35,9 @@ constexpr int kJacobiMaxSweeps = 40;
 constexpr int kMaxBatch = 64;
 struct RefLayer {
   const float* A;   // d x d
+  __nv_bfloat16* Ah;  // bf16 hi / lo split of A (tensor-core products), or null
+  __nv_bfloat16* Al;
+  __nv_bfloat16* Qs;  // d x 128 bf16 [Q_hi | Q_lo] operand, or null
   float* buf[3];    // [0] Q (d x m), [1] Y (ns k-slices of d x m), [2] T (d x m)
   double* gram;     // parts x m x m fp64 partial Gram matrices
   double* Lf;       // Cholesky factor (m x m) + reciprocal diagonal (m)
@@ -161,6 +164,36 @@ __global__ void omega_kernel(const __grid_constant__ RefBatch b) {
   for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
     const uint64_t h = splitmix64(L.seed ^ (uint64_t)e);
     Y[e] = (h >> 63) ? -1.0f : 1.0f;
+  }
+  if (L.Qs) {  // split operand: +-1 is exact in bf16, lo parts and padding are 0
+    const int m = b.m;
+    const int64_t n2 = (int64_t)L.d * 128;
+    for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n2; e += (int64_t)gridDim.x * blockDim.x) {
+      const int64_t row = e >> 7;
+      const int c = (int)(e & 127);
+      float v = 0.0f;
+      if (c < m) v = (splitmix64(L.seed ^ (uint64_t)(row * m + c)) >> 63) ? -1.0f : 1.0f;
+      L.Qs[e] = __float2bfloat16_rn(v);
+    }
+  }
+}
+
+// Ah = bf16(A), Al = bf16(A - Ah), elementwise (the tensor-core operands).
+__global__ void split_a_kernel(const __grid_constant__ RefBatch b) {
+  const RefLayer& L = b.L[blockIdx.z];
+  if (!L.Ah) return;
+  const int64_t n4 = (int64_t)L.d * L.d / 4;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n4; e += (int64_t)gridDim.x * blockDim.x) {
+    const float4 a = __ldg(reinterpret_cast<const float4*>(L.A) + e);
+    const float v[4] = {a.x, a.y, a.z, a.w};
+    float h[4], l[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      h[i] = __bfloat162float(__float2bfloat16_rn(v[i]));
+      l[i] = v[i] - h[i];
+    }
+    reinterpret_cast<uint2*>(L.Ah)[e] = make_uint2(pack_bf16x2(h[0], h[1]), pack_bf16x2(h[2], h[3]));
+    reinterpret_cast<uint2*>(L.Al)[e] = make_uint2(pack_bf16x2(l[0], l[1]), pack_bf16x2(l[2], l[3]));
   }
 }
 
@@ -419,6 +452,15 @@ __global__ void __launch_bounds__(kRT) qr_apply_kernel(const __grid_constant__ R
     }
     if (lane < m) Qo[row * m + lane] = (float)q0;
     if (lane + 32 < m) Qo[row * m + lane + 32] = (float)q1;
+    if (dst == kBufQ && Lr.Qs) {  // bf16 [hi | lo] operand of the tensor-core product
+      const float f0 = (float)q0, f1 = (float)q1;
+      const float h0 = __bfloat162float(__float2bfloat16_rn(f0)), h1 = __bfloat162float(__float2bfloat16_rn(f1));
+      __nv_bfloat16* qs = Lr.Qs + row * 128;
+      qs[lane] = __float2bfloat16_rn(h0);
+      qs[lane + 32] = __float2bfloat16_rn(h1);
+      qs[64 + lane] = __float2bfloat16_rn(f0 - h0);
+      qs[96 + lane] = __float2bfloat16_rn(f1 - h1);
+    }
   }
 }
 
@@ -675,6 +717,16 @@ void refresh_plan(int64_t N, int64_t d, int rank, int oversample, bool a_out_giv
   off += align256(2 * 64 * 64 * sizeof(double));
   p->off_syrk = off;
   if (splits > 1) off += align256((size_t)splits * d * d * sizeof(float));
+  p->tc_skinny = !no_split;
+  p->off_Ah = p->off_Al = p->off_Qs = off;
+  if (p->tc_skinny) {
+    p->off_Ah = off;
+    off += align256((size_t)d * d * 2);
+    p->off_Al = off;
+    off += align256((size_t)d * d * 2);
+    p->off_Qs = off;
+    off += align256((size_t)d * 128 * 2);
+  }
   p->total = off;
 }
 
@@ -720,6 +772,9 @@ cudaError_t launch_refresh_batch(const RefreshPlan* plans, const RefreshIO* io, 
       L.gram = (double*)(w + p.off_gram);
       L.Lf = (double*)(w + p.off_small);
       L.Vs = L.Lf + 64 * 64 + 64;  // after m*m + m doubles (m <= 64)
+      L.Ah = p.tc_skinny ? (__nv_bfloat16*)(w + p.off_Ah) : nullptr;
+      L.Al = p.tc_skinny ? (__nv_bfloat16*)(w + p.off_Al) : nullptr;
+      L.Qs = p.tc_skinny ? (__nv_bfloat16*)(w + p.off_Qs) : nullptr;
       L.U = o.U;
       L.lambda = o.lambda;
       L.rho = o.rho;
@@ -735,7 +790,10 @@ cudaError_t launch_refresh_batch(const RefreshPlan* plans, const RefreshIO* io, 
     }
     const int64_t dm = (int64_t)dmax * m;
     const int ew_blocks = (int)((dm + kRT - 1) / kRT < 2 * kNumSMs ? (dm + kRT - 1) / kRT : 2 * kNumSMs);
-    const int qr_blocks = (dmax + 7) / 8 < 4 * kNumSMs ? (dmax + 7) / 8 : 4 * kNumSMs;
+    // qr_apply: each CTA loads the m x m factor once, so use just enough CTAs
+    // per layer to cover the SMs about twice over the whole batch
+    int qr_blocks = (2 * kNumSMs + cnt - 1) / cnt;
+    if (qr_blocks > (dmax + 7) / 8) qr_blocks = (dmax + 7) / 8;
     const dim3 g_ew(ew_blocks, 1, cnt), g_skinny(dmax / 64, nsmax, cnt), g_gram(pmax, 1, cnt), g_one(1, 1, cnt),
         g_qr(qr_blocks, 1, cnt);
     // one Cholesky-QR pass: dst = src R^{-1} with src^T src = R^T R
@@ -744,11 +802,34 @@ cudaError_t launch_refresh_batch(const RefreshPlan* plans, const RefreshIO* io, 
       chol_kernel<<<g_one, kST, kCholSmem, s>>>(B);
       qr_apply_kernel<<<g_qr, kRT, 0, s>>>(B, src, dst);
     };
-    // A Q into Y, k-slices folded into slice 0
-    auto skinny_product = [&]() {
-      skinny_kernel<<<g_skinny, kRT, 0, s>>>(B, kBufQ, kBufY);
-      if (nsmax > 1) fold_slices_kernel<<<g_ew, kRT, 0, s>>>(B, kBufY);
+    // A Q into Y, k-slices folded into slice 0: fp32 CUDA cores, or for the
+    // iteration products (tc) the tensor cores on the bf16 split operands
+    const bool tc = plans[base].tc_skinny;
+    int tc_tiles = 0;
+    for (int l = 0; l < cnt; ++l) tc_tiles += B.L[l].d / 128;
+    static thread_local SkinnyTcJob sk[kMaxBatch];
+    int tc_nsmax = 1;
+    for (int l = 0; l < cnt && tc; ++l) {
+      const RefLayer& L = B.L[l];
+      int ns = (2 * kNumSMs + tc_tiles - 1) / tc_tiles;
+      if (ns > L.ns) ns = L.ns;
+      if (ns > L.d / 256) ns = L.d / 256 > 0 ? L.d / 256 : 1;
+      sk[l] = SkinnyTcJob{L.Ah, L.Al, L.Qs, L.buf[kBufY], L.d, ns, (L.d / ns + 63) / 64 * 64};
+      tc_nsmax = ns > tc_nsmax ? ns : tc_nsmax;
+    }
+    auto skinny_product = [&](bool use_tc) {
+      if (use_tc) {
+        launch_skinny_tc(sk, cnt, m, s);
+        // fold the tensor-core k-slices (their count may differ from the CUDA-core one)
+        for (int l = 0; l < cnt; ++l) B.L[l].ns = sk[l].ns;
+        if (tc_nsmax > 1) fold_slices_kernel<<<g_ew, kRT, 0, s>>>(B, kBufY);
+        for (int l = 0; l < cnt; ++l) B.L[l].ns = plans[base + l].skinny_slices;
+      } else {
+        skinny_kernel<<<g_skinny, kRT, 0, s>>>(B, kBufQ, kBufY);
+        if (nsmax > 1) fold_slices_kernel<<<g_ew, kRT, 0, s>>>(B, kBufY);
+      }
     };
+    if (tc) split_a_kernel<<<dim3(2 * kNumSMs, 1, cnt), kRT, 0, s>>>(B);
     // R2: randomised subspace iteration.  span(A Omega) = span(A orth(Omega)),
     // so the +-1 start block (exact) is multiplied by A directly; with no
     // iterations it is orthonormalised for the Rayleigh-Ritz step instead.
@@ -758,12 +839,13 @@ cudaError_t launch_refresh_batch(const RefreshPlan* plans, const RefreshIO* io, 
       cholqr_pass(kBufT, kBufQ);
     }
     for (int it = 0; it < iters; ++it) {
-      skinny_product();
+      skinny_product(tc);
       cholqr_pass(kBufY, kBufT);  // Cholesky-QR2:
       cholqr_pass(kBufT, kBufQ);  // two passes
     }
-    // R3/R4: Rayleigh-Ritz, lambda, rho, U
-    skinny_product();
+    // R3/R4: Rayleigh-Ritz, lambda, rho, U (fp32 product: the Ritz values
+    // need the accuracy the bf16 split would not give)
+    skinny_product(false);
     gram_partial_kernel<<<g_gram, kRT, 0, s>>>(B, kBufQ, kBufY);
     rr_kernel<<<g_one, kST, kRRSmem, s>>>(B);
     form_u_kernel<<<g_ew, kRT, 0, s>>>(B);
