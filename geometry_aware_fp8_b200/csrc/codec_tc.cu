@@ -12,21 +12,26 @@
 // exact to ~2^-17 (G is exact in bf16, so E1 needs G.U_hi + G.U_lo; E2 needs
 // Pc_hi.U_hi + Pc_lo.U_hi + Pc_hi.U_lo).  Accumulation is fp32 in TMEM.
 //
-// Data flow (one persistent CTA per SM, 288 threads, warp-specialised):
-//   warp 4 lane 0   TMA loads of 128x128 G chunks (two 64-column SW128 boxes)
-//   warps 4-7       convert the matching 128 rows of U into one bf16 tile
+// Data flow (one persistent CTA per SM, 480 threads, warp-specialised):
+//   warp 13 lane 0  TMA loads of 128x128 G chunks (two 64-column SW128 boxes)
+//                   and of the matching 128 rows of U (fp32)
+//   warps 8-11      convert those U rows in place into one bf16 tile
 //                   [128 rows][hi 32 | lo 32] with the 128-byte swizzle; the
 //                   tile is the MN-major B operand of E1 and the K-major B
 //                   operand of E2
-//   warp 8          TMEM allocation; one thread issues every MMA
-//   warps 0-3       epilogue, thread = row: forms the bf16 hi/lo tile of P o c
-//                   (the A operand of E2), then per chunk reads W from TMEM and
-//                   G from shared memory, finds the block maximum and stores
-//                   128 codes (8 x 16-byte stores) and one scale.
-// E1 streams G forward from HBM; E2 walks the same chunks backwards so the
-// most recently loaded ones are re-read while still in L2.  Panels of all
-// layers of one launch are assigned to CTAs on the host by longest-first
-// greedy scheduling (a panel costs d_in/128 chunks).
+//   warp 12         TMEM allocation; one thread issues every MMA
+//   warps 0-7       epilogue, two threads per row (TMEM lane quarter warp % 4,
+//                   column half warp / 4): form the bf16 hi/lo tile of P o c
+//                   (the A operand of E2), then per chunk read W from TMEM and
+//                   G from shared memory, find the block maximum (the halves
+//                   exchange theirs through shared memory), write the 128
+//                   codes of the row into shared memory and one scale
+//   warp 14 lane 0  TMA store of each chunk's codes; frees the stage
+// A CTA's panels are processed in blocks that interleave the second pass of
+// one panel (E2, epilogue-bound, its chunks re-read from L2 in reverse order)
+// with the first pass of the next (E1, an HBM stream).  Panels of all layers
+// of one launch are assigned to CTAs on the host by longest-first greedy
+// scheduling (a panel costs d_in/128 chunks).
 #include <algorithm>
 #include <queue>
 #include <vector>
@@ -47,7 +52,7 @@ constexpr int kUBytes = kChunk * 128;          // 16 KB: [128 rows][64 bf16]
 constexpr int kStageBytes = kGBytes + kUBytes;
 constexpr int kPcBytes = kPanel * 128;         // 16 KB: [128 rows][64 bf16]
 constexpr int kSmemBytes = kStages * kStageBytes + kPcBytes + 1024 + 512;
-constexpr int kThreads = 320;
+constexpr int kThreads = 480;  // 8 epilogue + 4 converter + MMA + TMA load + TMA store warps
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColW0 = 0, kColW1 = 128, kColP = 256;
 constexpr uint32_t kIdescE1 = umma_idesc_bf16(128, 64, 0, 1);   // A K-major, B MN-major
@@ -59,6 +64,7 @@ constexpr int kMaxPanels = 1536;
 struct alignas(64) EncJob {
   CUtensorMap tmG;  // bf16 [d_out][d_in], box [128][64], 128-byte swizzle
   CUtensorMap tmU;  // fp32 U [d_in][32], box [128][32], 128-byte swizzle
+  CUtensorMap tmC;  // uint8 codes [d_out][d_in], box [128][128], 128-byte swizzle (stores)
   const float* U;
   const float* lambda;
   const float* rho;
@@ -72,6 +78,7 @@ struct EncParams {
   uint16_t sched_off[kNumSMs + 1];  // CTA b runs sched_ids[sched_off[b] .. sched_off[b+1])
   uint16_t sched_ids[kMaxPanels];   // job << 8 | panel
 };
+static_assert(sizeof(EncParams) <= 32760, "kernel parameter space");
 
 // 16-byte chunk q of row r of a [rows][128 B] tile with the 128-byte swizzle
 GIFT_DEV uint32_t sw128(uint32_t r, uint32_t q) { return r * 128u + ((q ^ (r & 7u)) << 4); }
@@ -98,26 +105,62 @@ GIFT_DEV void tma_load_2d_hint(uint32_t dst, const void* tmap, uint64_t* bar, in
       : "memory");
 }
 
-// Walks the (panel, pass, chunk) steps of one CTA in the order every role
-// uses: for each scheduled panel, the first pass over chunks 0..nc-1, then
-// the second pass over nc-1..0.
+// 2-D tiled TMA store shared -> global (bulk-group completion).  Rows and
+// columns outside the tensor are not written.
+GIFT_DEV void tma_store_2d_hint(const void* tmap, uint32_t src, int x, int y, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group.L2::cache_hint"
+      " [%0, {%2, %3}], [%1], %4;" ::"l"(tmap),
+      "r"(src), "r"(x), "r"(y), "l"(policy)
+      : "memory");
+}
+GIFT_DEV void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until at most N committed store groups still read shared memory.
+template <int N>
+GIFT_DEV void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+// Wait until every committed store group has completed.
+GIFT_DEV void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// Walks the steps of one CTA in the order every role uses.  A CTA's panels
+// p_0 .. p_{n-1} are visited in blocks: block 0 is the first pass of p_0
+// (chunks 0 .. nc-1); block k >= 1 is the second pass of p_{k-1} (chunks
+// nc-1 .. 0) interleaved step by step with the first pass of p_k, so that the
+// HBM stream of one panel overlaps the epilogue work of the previous one.
 template <class P>
 struct Steps {
   const P& p;
-  int it, end, pass, i, nc;
-  GIFT_DEV Steps(const P& p_, int beg, int end_) : p(p_), it(beg), end(end_), pass(0), i(0), nc(0) {
-    if (it < end) nc = p.jobs[job()].d_in / kChunk;
+  int beg, end, k;
+  int n1, n2, i1, i2;  // first- and second-pass steps of block k, and how many are done
+  int pass;            // pass of the current step
+  GIFT_DEV Steps(const P& p_, int b, int e) : p(p_), beg(b), end(e), k(0) { setup(); }
+  GIFT_DEV int nc_of(int it) const { return p.jobs[p.sched_ids[it] >> 8].d_in / kChunk; }
+  GIFT_DEV void setup() {
+    i1 = i2 = 0;
+    n1 = beg + k < end ? nc_of(beg + k) : 0;
+    n2 = k >= 1 && beg + k - 1 < end ? nc_of(beg + k - 1) : 0;
+    pick();
   }
-  GIFT_DEV bool valid() const { return it < end; }
-  GIFT_DEV int job() const { return p.sched_ids[it] >> 8; }
-  GIFT_DEV int panel() const { return p.sched_ids[it] & 255; }
-  GIFT_DEV int chunk() const { return pass == 0 ? i : nc - 1 - i; }
+  GIFT_DEV void pick() { pass = (i2 < n2 && (i1 >= n1 || i2 <= i1)) ? 1 : 0; }
+  GIFT_DEV bool valid() const { return n1 + n2 > 0; }
+  GIFT_DEV int slot() const { return pass ? beg + k - 1 : beg + k; }
+  GIFT_DEV int job() const { return p.sched_ids[slot()] >> 8; }
+  GIFT_DEV int panel() const { return p.sched_ids[slot()] & 255; }
+  GIFT_DEV int nc() const { return pass ? n2 : n1; }
+  GIFT_DEV int chunk() const { return pass ? n2 - 1 - i2 : i1; }
+  GIFT_DEV bool block_start() const { return i1 + i2 == 0; }
   GIFT_DEV void next() {
-    if (++i < nc) return;
-    i = 0;
-    if (++pass < 2) return;
-    pass = 0;
-    if (++it < end) nc = p.jobs[job()].d_in / kChunk;
+    if (pass)
+      ++i2;
+    else
+      ++i1;
+    if (i1 + i2 == n1 + n2) {
+      ++k;
+      setup();
+    } else {
+      pick();
+    }
   }
 };
 
@@ -188,12 +231,13 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
   const uint32_t pc_tile = sbase + kStages * kStageBytes;
   uint64_t* bars = (uint64_t*)(smem + kStages * kStageBytes + kPcBytes);
   uint64_t* full = bars;                  // [kStages] count 1: converter (stage ready for the MMA)
-  uint64_t* empty = bars + kStages;       // [kStages] count 1
+  uint64_t* empty = bars + kStages;       // [kStages] count 1: MMA commit (E1) or code store (E2)
   uint64_t* tfull = bars + 2 * kStages;   // [kStages] count 1 + tx: TMA (G and fp32 U)
-  uint64_t* p_full = bars + 3 * kStages;  // count 1 (MMA commit)
-  uint64_t* pc_full = p_full + 1;         // count 128 (epilogue)
+  uint64_t* cready = bars + 3 * kStages;  // [kStages] count 256: codes of an E2 step in shared memory
+  uint64_t* p_full = bars + 4 * kStages;  // count 1 (MMA commit)
+  uint64_t* pc_full = p_full + 1;         // count 256 (epilogue)
   uint64_t* w_full = p_full + 2;          // [2] count 1
-  uint64_t* w_empty = p_full + 4;         // [2] count 128
+  uint64_t* w_empty = p_full + 4;         // [2] count 256
   uint32_t* tmem_slot = (uint32_t*)(p_full + 6);
   __shared__ int failed;  // any role gave up (reported at exit)
 
@@ -206,16 +250,17 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
       mbar_init(&tfull[s], 1);
+      mbar_init(&cready[s], 256);
     }
     mbar_init(p_full, 1);
-    mbar_init(pc_full, 128);
+    mbar_init(pc_full, 256);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&w_full[b], 1);
-      mbar_init(&w_empty[b], 128);
+      mbar_init(&w_empty[b], 256);
     }
     fence_mbar_init();
   }
-  if (warp == 8) {
+  if (warp == 12) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
@@ -224,8 +269,8 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
 
-  if (warp == 9) {
-    // ---------------- TMA producer: G chunks, running ahead of the ring ----------------
+  if (warp == 13) {
+    // ---------------- TMA producer: G chunks and U rows, running ahead of the ring ----------------
     if (lane == 0) {
       const uint64_t keep = policy_evict_last(), drop = policy_evict_first();
       uint32_t step = 0;
@@ -245,11 +290,32 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
         tma_load_2d_hint(dst + kGBytes, &J.tmU, &tfull[s], 0, st.chunk() * kChunk, keep);
       }
     }
-  } else if (warp >= 4 && warp < 8) {
+  } else if (warp == 14) {
+    // ---------------- code stores: one TMA store per E2 step, then the stage is free ----------------
+    if (lane == 0) {
+      const uint64_t drop = policy_evict_first();
+      uint32_t step = 0, par = 0;  // par: bit s = phase parity of cready[s]
+      for (Steps<EncParams> st(p, beg, end); st.valid() && !failed; st.next(), ++step) {
+        if (st.pass == 0) continue;
+        const int s = step % kStages;
+        if (!mbar_wait(&cready[s], (par >> s) & 1u, kWaitLimit)) {
+          failed = 1;
+          break;
+        }
+        par ^= 1u << s;
+        const EncJob& J = p.jobs[st.job()];
+        tma_store_2d_hint(&J.tmC, sbase + s * kStageBytes + kGBytes, st.chunk() * kChunk, st.panel() * kPanel, drop);
+        bulk_commit();
+        bulk_wait_read<0>();
+        mbar_arrive(&empty[s]);
+      }
+      bulk_wait_all();
+    }
+  } else if (warp >= 8 && warp < 12) {
     // ---------------- converters: fp32 U rows -> bf16 hi/lo, in place, one row each ----------------
     // Exit decisions are voted at a named barrier so all 128 threads leave
     // at the same step.
-    const int t = threadIdx.x - 128;
+    const int t = threadIdx.x - 256;
     uint32_t step = 0;
     for (Steps<EncParams> st(p, beg, end); st.valid(); st.next(), ++step) {
       const int s = step % kStages;
@@ -264,19 +330,21 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
       named_sync(1, 128);
       if (t == 0) mbar_arrive(&full[s]);
     }
-  } else if (warp == 8) {
+  } else if (warp == 12) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
-      uint32_t step = 0, e2 = 0, np = 0;
-      for (int it = beg; it < end && !failed; ++it, ++np) {
-        const EncJob& J = p.jobs[p.sched_ids[it] >> 8];
-        const int nc = J.d_in / kChunk;
-        // E1: P2[128 x 64] = G . [U_hi | U_lo]
-        for (int c = 0; c < nc; ++c, ++step) {
-          const int s = step % kStages;
-          if (!mbar_wait(&full[s], (step / kStages) & 1u, kWaitLimit)) { failed = 1; break; }
-          tc_fence_after();
-          const uint32_t g_tile = sbase + s * kStageBytes, u_tile = g_tile + kGBytes;
+      uint32_t step = 0, e2 = 0;
+      for (Steps<EncParams> st(p, beg, end); st.valid() && !failed; st.next(), ++step) {
+        const int s = step % kStages;
+        // block k >= 1 starts with the second pass of p_{k-1}: its P o c must be
+        // in shared memory, and P in TMEM has been read (it is reused for p_k)
+        if (st.block_start() && st.k >= 1 && !mbar_wait(pc_full, (st.k - 1) & 1u, kWaitLimit)) { failed = 1; break; }
+        if (!mbar_wait(&full[s], (step / kStages) & 1u, kWaitLimit)) { failed = 1; break; }
+        tc_fence_after();
+        const uint32_t g_tile = sbase + s * kStageBytes, u_tile = g_tile + kGBytes;
+        if (st.pass == 0) {
+          // E1: P2[128 x 64] += G_c . [U_hi | U_lo]_c
+          const int c = st.chunk();
 #pragma unroll
           for (int h = 0; h < 2; ++h)
 #pragma unroll
@@ -286,18 +354,12 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
               umma_bf16(tbase + kColP, ad, bd, kIdescE1, (c | h | kk) ? 1u : 0u);
             }
           umma_commit(&empty[s]);
-        }
-        umma_commit(p_full);
-        if (failed || !mbar_wait(pc_full, np & 1u, kWaitLimit)) { failed = 1; break; }
-        tc_fence_after();
-        // E2: W[128 x 128] = Pc_hi U_hi^T + Pc_lo U_hi^T + Pc_hi U_lo^T
-        for (int i = 0; i < nc; ++i, ++step, ++e2) {
-          const int s = step % kStages;
+          if (c == st.nc() - 1) umma_commit(p_full);
+        } else {
+          // E2: W[128 x 128] = Pc_hi U_hi^T + Pc_lo U_hi^T + Pc_hi U_lo^T
           const int b = e2 & 1;
-          if (!mbar_wait(&full[s], (step / kStages) & 1u, kWaitLimit)) { failed = 1; break; }
           if (e2 >= 2 && !mbar_wait(&w_empty[b], ((e2 >> 1) - 1) & 1u, kWaitLimit)) { failed = 1; break; }
           tc_fence_after();
-          const uint32_t u_tile = sbase + s * kStageBytes + kGBytes;
           const uint32_t d = tbase + (b ? kColW1 : kColW0);
           const int ak[6] = {0, 16, 32, 48, 0, 16};   // Pc: hi = k 0..31, lo = k 32..63
           const int bk[6] = {0, 16, 0, 16, 32, 48};   // U : hi = k 0..31, lo = k 32..63
@@ -308,134 +370,131 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
             umma_bf16(d, ad, bd, kIdescE2, q ? 1u : 0u);
           }
           umma_commit(&w_full[b]);
+          ++e2;
         }
       }
     }
   } else {
-    // ---------------- epilogue: warps 0-3, thread = row ----------------
-    const int r = threadIdx.x;                 // 0..127
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-    uint32_t step = 0, e2 = 0, np = 0;
-    bool stop = false;  // group vote: set for all 128 threads at the same barrier
-    for (int it = beg; it < end && !stop; ++it, ++np) {
-      const int jb = p.sched_ids[it] >> 8, panel = p.sched_ids[it] & 255;
-      const EncJob& J = p.jobs[jb];
-      const int nc = J.d_in / kChunk;
-      // transform coefficients of this layer (fp64, rounded once)
-      float cf[32];
-      const double rho = (double)__ldg(J.rho);
-      const double a64 = 1.0 / sqrt(rho);
-      const float a = (float)a64;
+    // ---------------- epilogue: warps 0-7 ----------------
+    // Thread (r, h): row r = 32 (warp % 4) + lane of the panel (its TMEM
+    // lane), columns 64 h .. 64 h + 63 of every 128-column chunk (h = warp / 4,
+    // the G box it reads).  The two halves of a row exchange their partial
+    // block maxima through shared memory.  The codes of a chunk are written
+    // into the stage's U tile, which the E2 MMA no longer needs once W is in
+    // TMEM, for the store warp.
+    __shared__ float amax_x[2][128];
+    const int h = warp >> 2;
+    const int r = (warp & 3) * 32 + lane;
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    uint32_t step = 0, e2 = 0;
+    float a = 0.0f;
+    bool stop = false;  // group vote: set for all 256 threads at the same barrier
+    for (Steps<EncParams> st(p, beg, end); st.valid() && !stop; st.next(), ++step) {
+      if (st.pass == 0) continue;  // first-pass steps are the MMA's alone
+      const EncJob& J = p.jobs[st.job()];
+      const int panel = st.panel();
+      if (st.i2 == 0) {
+        // P o c of this panel for k = 16 h .. 16 h + 15, split into the bf16 A operand of E2
+        const double rho = (double)__ldg(J.rho);
+        const double a64 = 1.0 / sqrt(rho);
+        a = (float)a64;
+        float cf[16];
 #pragma unroll
-      for (int k = 0; k < 32; ++k)
-        cf[k] = k < J.rank ? (float)(1.0 / sqrt((double)__ldg(J.lambda + k) + rho) - a64) : 0.0f;
-      // P o c, split into the bf16 A operand of E2
-      stop = named_sync_or(2, 128, !mbar_wait(p_full, np & 1u, kWaitLimit));
-      if (stop) {
-        failed = 1;
-        break;
-      }
-      tc_fence_after();
-      uint32_t pr[64];
-      tmem_ld32(tbase + lane_off + kColP, pr);
-      tmem_ld32(tbase + lane_off + kColP + 32, pr + 32);
-      tmem_wait_ld();
-      uint32_t hi[16], lo[16];
-#pragma unroll
-      for (int k = 0; k < 16; ++k) {
-        const float v0 = (__uint_as_float(pr[2 * k]) + __uint_as_float(pr[32 + 2 * k])) * cf[2 * k];
-        const float v1 = (__uint_as_float(pr[2 * k + 1]) + __uint_as_float(pr[33 + 2 * k])) * cf[2 * k + 1];
-        float h0, l0, h1, l1;
-        split_bf16(v0, h0, l0);
-        split_bf16(v1, h1, l1);
-        hi[k] = pack_bf16x2(h0, h1);
-        lo[k] = pack_bf16x2(l0, l1);
-      }
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-        st_shared_v4(pc_tile + sw128(r, q), hi[4 * q], hi[4 * q + 1], hi[4 * q + 2], hi[4 * q + 3]);
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-        st_shared_v4(pc_tile + sw128(r, 4 + q), lo[4 * q], lo[4 * q + 1], lo[4 * q + 2], lo[4 * q + 3]);
-      fence_async_shared();
-      tc_fence_before();
-      mbar_arrive(pc_full);
-      step += nc;  // the E1 steps
-      const int64_t row = (int64_t)panel * kPanel + r;
-      const bool live = row < J.d_out;
-      for (int i = 0; i < nc; ++i, ++step, ++e2) {
-        const int c = nc - 1 - i;
-        const int s = step % kStages;
-        const int b = e2 & 1;
-        stop = named_sync_or(2, 128, !mbar_wait(&w_full[b], (e2 >> 1) & 1u, kWaitLimit));
+        for (int k = 0; k < 16; ++k) {
+          const int kk = 16 * h + k;
+          cf[k] = kk < J.rank ? (float)(1.0 / sqrt((double)__ldg(J.lambda + kk) + rho) - a64) : 0.0f;
+        }
+        stop = named_sync_or(2, 256, !mbar_wait(p_full, (st.k - 1) & 1u, kWaitLimit));
         if (stop) {
           failed = 1;
           break;
         }
         tc_fence_after();
-        const uint32_t wcol = tbase + lane_off + (b ? kColW1 : kColW0);
-        const uint32_t g_tile = sbase + s * kStageBytes;
-        // pass 1: block maximum of w = a g + acc
-        float amax = 0.0f;
+        uint32_t ph[16], pl[16];
+        tmem_ld16(tbase + lane_off + kColP + 16 * h, ph);
+        tmem_ld16(tbase + lane_off + kColP + 32 + 16 * h, pl);
+        tmem_wait_ld();
+        uint32_t hi[8], lo[8];
 #pragma unroll
-        for (int g4 = 0; g4 < 4; ++g4) {
-          uint32_t acc[32];
-          tmem_ld32(wcol + g4 * 32, acc);
-          tmem_wait_ld();
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int qq = g4 * 4 + q;                       // 16-byte chunk of the 256-byte row
-            const uint4 gv = ld_shared_v4(g_tile + (qq >> 3) * kGHalf + sw128(r, qq & 7));
-            const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float w0 = fmaf(a, bf16lo(gw[e]), __uint_as_float(acc[q * 8 + 2 * e]));
-              const float w1 = fmaf(a, bf16hi(gw[e]), __uint_as_float(acc[q * 8 + 2 * e + 1]));
-              amax = fmaxf(amax, fmaxf(fabsf(w0), fabsf(w1)));
-            }
-          }
+        for (int k = 0; k < 8; ++k) {
+          const float v0 = (__uint_as_float(ph[2 * k]) + __uint_as_float(pl[2 * k])) * cf[2 * k];
+          const float v1 = (__uint_as_float(ph[2 * k + 1]) + __uint_as_float(pl[2 * k + 1])) * cf[2 * k + 1];
+          float h0, l0, h1, l1;
+          split_bf16(v0, h0, l0);
+          split_bf16(v1, h1, l1);
+          hi[k] = pack_bf16x2(h0, h1);
+          lo[k] = pack_bf16x2(l0, l1);
         }
-        const float inv = e4m3_inv_scale(amax);
-        // pass 2: codes
-        uint8_t* dst = J.codes + row * J.d_in + c * kChunk;
-#pragma unroll
-        for (int g4 = 0; g4 < 4; ++g4) {
-          uint32_t acc[32];
-          tmem_ld32(wcol + g4 * 32, acc);
-          tmem_wait_ld();
-          uint32_t cw[8];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int qq = g4 * 4 + q;
-            const uint4 gv = ld_shared_v4(g_tile + (qq >> 3) * kGHalf + sw128(r, qq & 7));
-            const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const float w0 = fmaf(a, bf16lo(gw[2 * e]), __uint_as_float(acc[q * 8 + 4 * e]));
-              const float w1 = fmaf(a, bf16hi(gw[2 * e]), __uint_as_float(acc[q * 8 + 4 * e + 1]));
-              const float w2 = fmaf(a, bf16lo(gw[2 * e + 1]), __uint_as_float(acc[q * 8 + 4 * e + 2]));
-              const float w3 = fmaf(a, bf16hi(gw[2 * e + 1]), __uint_as_float(acc[q * 8 + 4 * e + 3]));
-              const uint32_t c01 = f32x2_to_e4m3x2(__fmul_rn(w0, inv), __fmul_rn(w1, inv));
-              const uint32_t c23 = f32x2_to_e4m3x2(__fmul_rn(w2, inv), __fmul_rn(w3, inv));
-              cw[q * 2 + e] = inv > 0.0f ? (c01 | (c23 << 16)) : 0u;
-            }
-          }
-          if (live) {
-            __stcs(reinterpret_cast<uint4*>(dst + g4 * 32), make_uint4(cw[0], cw[1], cw[2], cw[3]));
-            __stcs(reinterpret_cast<uint4*>(dst + g4 * 32 + 16), make_uint4(cw[4], cw[5], cw[6], cw[7]));
-          }
-        }
-        if (live) J.scales[row * (J.d_in / kChunk) + c] = e4m3_scale(amax, inv);
+        st_shared_v4(pc_tile + sw128(r, 2 * h), hi[0], hi[1], hi[2], hi[3]);
+        st_shared_v4(pc_tile + sw128(r, 2 * h + 1), hi[4], hi[5], hi[6], hi[7]);
+        st_shared_v4(pc_tile + sw128(r, 4 + 2 * h), lo[0], lo[1], lo[2], lo[3]);
+        st_shared_v4(pc_tile + sw128(r, 5 + 2 * h), lo[4], lo[5], lo[6], lo[7]);
+        fence_async_shared();
         tc_fence_before();
-        mbar_arrive(&w_empty[b]);
-        named_sync(2, 128);
-        if (r == 0) mbar_arrive(&empty[s]);
+        mbar_arrive(pc_full);
       }
+      const int c = st.chunk();
+      const int s = step % kStages;
+      const int b = e2 & 1;
+      const int64_t row = (int64_t)panel * kPanel + r;
+      const bool live = row < J.d_out;
+      const bool ok = mbar_wait(&w_full[b], (e2 >> 1) & 1u, kWaitLimit) &&
+                      mbar_wait(&tfull[s], (step / kStages) & 1u, kWaitLimit);
+      stop = named_sync_or(2, 256, !ok);
+      if (stop) {
+        failed = 1;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t wcol = tbase + lane_off + (b ? kColW1 : kColW0) + 64 * h;
+      const uint32_t g_box = sbase + s * kStageBytes + h * kGHalf;  // this half's 64 columns
+      // w = a g + acc for the 64 columns, and their maximum
+      float w[64];
+      float amax = 0.0f;
+#pragma unroll
+      for (int g2 = 0; g2 < 2; ++g2) {
+        uint32_t acc[32];
+        tmem_ld32(wcol + g2 * 32, acc);
+        tmem_wait_ld();
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint4 gv = ld_shared_v4(g_box + sw128(r, g2 * 4 + q));
+          const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int k = g2 * 32 + q * 8 + 2 * e;
+            w[k] = fmaf(a, bf16lo(gw[e]), __uint_as_float(acc[q * 8 + 2 * e]));
+            w[k + 1] = fmaf(a, bf16hi(gw[e]), __uint_as_float(acc[q * 8 + 2 * e + 1]));
+            amax = fmaxf(amax, fmaxf(fabsf(w[k]), fabsf(w[k + 1])));
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&w_empty[b]);
+      amax_x[h][r] = amax;
+      named_sync(2, 256);
+      amax = fmaxf(amax_x[0][r], amax_x[1][r]);
+      const float inv = e4m3_inv_scale(amax);
+      uint32_t cw[16];
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+        const uint32_t c01 = f32x2_to_e4m3x2(__fmul_rn(w[4 * q], inv), __fmul_rn(w[4 * q + 1], inv));
+        const uint32_t c23 = f32x2_to_e4m3x2(__fmul_rn(w[4 * q + 2], inv), __fmul_rn(w[4 * q + 3], inv));
+        cw[q] = inv > 0.0f ? (c01 | (c23 << 16)) : 0u;
+      }
+      const uint32_t c_tile = sbase + s * kStageBytes + kGBytes;  // [128][128 B], 128-byte swizzle
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        st_shared_v4(c_tile + sw128(r, 4 * h + q), cw[4 * q], cw[4 * q + 1], cw[4 * q + 2], cw[4 * q + 3]);
+      if (live && h == 0) J.scales[row * (J.d_in / kChunk) + c] = e4m3_scale(amax, inv);
+      fence_async_shared();
+      mbar_arrive(&cready[s]);
+      ++e2;
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 8) tmem_dealloc(tbase, kTmemCols);
+  if (warp == 12) tmem_dealloc(tbase, kTmemCols);
   if (threadIdx.x == 0 && failed && err) atomicOr(err, GIFT_DEV_TIMEOUT);
 }
 
@@ -463,11 +522,11 @@ constexpr uint32_t kIdescD2 = umma_idesc_bf16(128, 64, 0, 1);
 struct alignas(64) DecJob {
   CUtensorMap tmC;  // uint8 codes [d_out][d_in], box [128][128], 128-byte swizzle
   CUtensorMap tmU;  // fp32 U [d_in][32], box [128][32], 128-byte swizzle
+  CUtensorMap tmO;  // bf16 G_hat [d_out][d_in], box [128][64], 128-byte swizzle (stores)
   const float* U;
   const float* lambda;
   const float* rho;
   const float* scales;
-  __nv_bfloat16* out;
   int d_out, d_in, rank, pad;
 };
 
@@ -476,6 +535,7 @@ struct DecParams {
   uint16_t sched_off[kNumSMs + 1];
   uint16_t sched_ids[kMaxPanels];
 };
+static_assert(sizeof(DecParams) <= 32760, "kernel parameter space");
 
 // E4M3 pair -> bf16 pair (exact: every E4M3 value is a bf16 value)
 GIFT_DEV uint32_t e4m3x2_to_bf16x2(uint16_t v) {
@@ -492,12 +552,13 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
   uint64_t* bars = (uint64_t*)(smem + kDStages * kDStageBytes + kPcBytes);
   uint64_t* full = bars;                   // [kDStages] count 1: converter (U tile, bf16 codes)
   uint64_t* cfull = bars + kDStages;       // [kDStages] count 1 + tx: codes TMA
-  uint64_t* empty = bars + 2 * kDStages;   // [kDStages] count 1
-  uint64_t* t_full = bars + 3 * kDStages;  // [2] count 1
-  uint64_t* t_empty = t_full + 2;          // [2] count 128
-  uint64_t* pc_full = t_full + 4;          // count 128
+  uint64_t* empty = bars + 2 * kDStages;   // [kDStages] count 1: MMA commit (D2) or output store (D3)
+  uint64_t* oready = bars + 3 * kDStages;  // [kDStages] count 256: output tile of a D3 step in shared memory
+  uint64_t* t_full = bars + 4 * kDStages;  // [2] count 1
+  uint64_t* t_empty = t_full + 2;          // [2] count 256
+  uint64_t* pc_full = t_full + 4;          // count 256
   uint64_t* w_full = t_full + 5;           // [2] count 1
-  uint64_t* w_empty = t_full + 7;          // [2] count 128
+  uint64_t* w_empty = t_full + 7;          // [2] count 256
   uint32_t* tmem_slot = (uint32_t*)(t_full + 9);
   __shared__ int failed;
 
@@ -509,17 +570,18 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
       mbar_init(&full[s], 1);
       mbar_init(&cfull[s], 1);
       mbar_init(&empty[s], 1);
+      mbar_init(&oready[s], 256);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&t_full[b], 1);
-      mbar_init(&t_empty[b], 128);
+      mbar_init(&t_empty[b], 256);
       mbar_init(&w_full[b], 1);
-      mbar_init(&w_empty[b], 128);
+      mbar_init(&w_empty[b], 256);
     }
-    mbar_init(pc_full, 128);
+    mbar_init(pc_full, 256);
     fence_mbar_init();
   }
-  if (warp == 8) {
+  if (warp == 12) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
@@ -528,8 +590,8 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
 
-  if (warp == 9) {
-    // ---------------- TMA producer: codes chunks, running ahead of the ring ----------------
+  if (warp == 13) {
+    // ---------------- TMA producer: codes chunks and U rows, running ahead of the ring ----------------
     if (lane == 0) {
       const uint64_t keep = policy_evict_last(), drop = policy_evict_first();
       uint32_t step = 0;
@@ -548,9 +610,32 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
         tma_load_2d_hint(dst + kDCodes + kDQ, &J.tmU, &cfull[s], 0, st.chunk() * kChunk, keep);
       }
     }
-  } else if (warp >= 4 && warp < 8) {
+  } else if (warp == 14) {
+    // ---------------- output stores: two TMA stores per D3 step, then the stage is free ----------------
+    if (lane == 0) {
+      const uint64_t drop = policy_evict_first();
+      uint32_t step = 0, par = 0;  // par: bit s = phase parity of oready[s]
+      for (Steps<DecParams> st(p, beg, end); st.valid() && !failed; st.next(), ++step) {
+        if (st.pass == 0) continue;
+        const int s = step % kDStages;
+        if (!mbar_wait(&oready[s], (par >> s) & 1u, kWaitLimit)) {
+          failed = 1;
+          break;
+        }
+        par ^= 1u << s;
+        const DecJob& J = p.jobs[st.job()];
+        const uint32_t o_tile = sbase + s * kDStageBytes + kDCodes;
+        tma_store_2d_hint(&J.tmO, o_tile, st.chunk() * kChunk, st.panel() * kPanel, drop);
+        tma_store_2d_hint(&J.tmO, o_tile + kGHalf, st.chunk() * kChunk + 64, st.panel() * kPanel, drop);
+        bulk_commit();
+        bulk_wait_read<0>();
+        mbar_arrive(&empty[s]);
+      }
+      bulk_wait_all();
+    }
+  } else if (warp >= 8 && warp < 12) {
     // ---------------- converters: U tile in place, and in the first pass the bf16 codes ----------------
-    const int t = threadIdx.x - 128;
+    const int t = threadIdx.x - 256;
     uint32_t step = 0;
     for (Steps<DecParams> st(p, beg, end); st.valid(); st.next(), ++step) {
       const int s = step % kDStages;
@@ -585,21 +670,21 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
       named_sync(1, 128);
       if (t == 0) mbar_arrive(&full[s]);
     }
-  } else if (warp == 8) {
+  } else if (warp == 12) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
-      uint32_t step = 0, e2 = 0, d2 = 0, np = 0;
-      for (int it = beg; it < end && !failed; ++it, ++np) {
-        const DecJob& J = p.jobs[p.sched_ids[it] >> 8];
-        const int nc = J.d_in / kChunk;
-        // D2: T_c[128 x 64] = q_c . [U_hi | U_lo]
-        for (int c = 0; c < nc; ++c, ++step, ++d2) {
-          const int s = step % kDStages;
+      uint32_t step = 0, e2 = 0, d2 = 0;
+      for (Steps<DecParams> st(p, beg, end); st.valid() && !failed; st.next(), ++step) {
+        const int s = step % kDStages;
+        // block k >= 1 starts with D3 of p_{k-1}, which needs its P o c
+        if (st.block_start() && st.k >= 1 && !mbar_wait(pc_full, (st.k - 1) & 1u, kWaitLimit)) { failed = 1; break; }
+        if (!mbar_wait(&full[s], (step / kDStages) & 1u, kWaitLimit)) { failed = 1; break; }
+        const uint32_t q_tile = sbase + s * kDStageBytes + kDCodes, u_tile = q_tile + kDQ;
+        if (st.pass == 0) {
+          // D2: T_c[128 x 64] = q_c . [U_hi | U_lo]
           const int b = d2 & 1;
-          if (!mbar_wait(&full[s], (step / kDStages) & 1u, kWaitLimit)) { failed = 1; break; }
           if (d2 >= 2 && !mbar_wait(&t_empty[b], ((d2 >> 1) - 1) & 1u, kWaitLimit)) { failed = 1; break; }
           tc_fence_after();
-          const uint32_t q_tile = sbase + s * kDStageBytes + kDCodes, u_tile = q_tile + kDQ;
           const uint32_t d = tbase + (b ? kColT1 : kColT0);
 #pragma unroll
           for (int h = 0; h < 2; ++h)
@@ -611,17 +696,12 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
             }
           umma_commit(&empty[s]);
           umma_commit(&t_full[b]);
-        }
-        if (failed || !mbar_wait(pc_full, np & 1u, kWaitLimit)) { failed = 1; break; }
-        tc_fence_after();
-        // D3: W[128 x 128] = Pc . U^T (three split products)
-        for (int i = 0; i < nc; ++i, ++step, ++e2) {
-          const int s = step % kDStages;
+          ++d2;
+        } else {
+          // D3: W[128 x 128] = Pc . U^T (three split products)
           const int b = e2 & 1;
-          if (!mbar_wait(&full[s], (step / kDStages) & 1u, kWaitLimit)) { failed = 1; break; }
           if (e2 >= 2 && !mbar_wait(&w_empty[b], ((e2 >> 1) - 1) & 1u, kWaitLimit)) { failed = 1; break; }
           tc_fence_after();
-          const uint32_t u_tile = sbase + s * kDStageBytes + kDCodes + kDQ;
           const uint32_t d = tbase + (b ? kColW1 : kColW0);
           const int ak[6] = {0, 16, 32, 48, 0, 16};
           const int bk[6] = {0, 16, 0, 16, 32, 48};
@@ -632,133 +712,135 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
             umma_bf16(d, ad, bd, kIdescE2, q ? 1u : 0u);
           }
           umma_commit(&w_full[b]);
+          ++e2;
         }
       }
     }
   } else {
-    // ---------------- epilogue: warps 0-3, thread = row ----------------
-    const int r = threadIdx.x;
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-    uint32_t step = 0, e2 = 0, d2 = 0, np = 0;
+    // ---------------- epilogue: warps 0-7 ----------------
+    // Thread (r, h): row r = 32 (warp % 4) + lane (its TMEM lane); in D2 the
+    // coefficients k = 16 h .. 16 h + 15, in D3 the columns 64 h .. 64 h + 63
+    // of every 128-column chunk (h = warp / 4).  P of the panel in its first
+    // pass stays in registers until the block that starts its second pass;
+    // D3 writes its bf16 tile into the stage's codes-as-bf16 region (free in
+    // the second pass) for the store warp.
+    const int h = warp >> 2;
+    const int r = (warp & 3) * 32 + lane;
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    uint32_t step = 0, e2 = 0, d2 = 0;
+    float P[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) P[k] = 0.0f;
+    float a = 0.0f;
     bool stop = false;
-    for (int it = beg; it < end && !stop; ++it, ++np) {
-      const int jb = p.sched_ids[it] >> 8, panel = p.sched_ids[it] & 255;
-      const DecJob& J = p.jobs[jb];
-      const int nc = J.d_in / kChunk;
-      const int64_t row = (int64_t)panel * kPanel + r;
+    for (Steps<DecParams> st(p, beg, end); st.valid() && !stop; st.next(), ++step) {
+      const int s = step % kDStages;
+      const DecJob& J = p.jobs[st.job()];
+      const int nc = st.nc(), c = st.chunk();
+      const int64_t row = (int64_t)st.panel() * kPanel + r;
       const bool live = row < J.d_out;
-      const float* srow = J.scales + (live ? row : 0) * nc;
-      float cf[32];
-      const double rho = (double)__ldg(J.rho);
-      const double a64 = sqrt(rho);
-      const float a = (float)a64;
+      const float sc = live ? __ldg(J.scales + row * nc + c) : 0.0f;
+      if (st.block_start() && st.k >= 1) {
+        // P of p_{k-1} is complete: P o c -> bf16 hi/lo A operand of D3
+        // (this half's 16 of the 32 columns of each part)
+        const double rho = (double)__ldg(J.rho);
+        const double a64 = sqrt(rho);
+        a = (float)a64;
+        uint32_t hi[8], lo[8];
 #pragma unroll
-      for (int k = 0; k < 32; ++k)
-        cf[k] = k < J.rank ? (float)(sqrt((double)__ldg(J.lambda + k) + rho) - a64) : 0.0f;
-      // D2 epilogue: P += s_c (T_hi + T_lo)
-      float P[32];
+        for (int k = 0; k < 8; ++k) {
+          const int k0 = 16 * h + 2 * k;
+          const float c0 = k0 < J.rank ? (float)(sqrt((double)__ldg(J.lambda + k0) + rho) - a64) : 0.0f;
+          const float c1 = k0 + 1 < J.rank ? (float)(sqrt((double)__ldg(J.lambda + k0 + 1) + rho) - a64) : 0.0f;
+          float h0, l0, h1, l1;
+          split_bf16(P[2 * k] * c0, h0, l0);
+          split_bf16(P[2 * k + 1] * c1, h1, l1);
+          hi[k] = pack_bf16x2(h0, h1);
+          lo[k] = pack_bf16x2(l0, l1);
+        }
+        st_shared_v4(pc_tile + sw128(r, 2 * h), hi[0], hi[1], hi[2], hi[3]);
+        st_shared_v4(pc_tile + sw128(r, 2 * h + 1), hi[4], hi[5], hi[6], hi[7]);
+        st_shared_v4(pc_tile + sw128(r, 4 + 2 * h), lo[0], lo[1], lo[2], lo[3]);
+        st_shared_v4(pc_tile + sw128(r, 5 + 2 * h), lo[4], lo[5], lo[6], lo[7]);
+        fence_async_shared();
+        mbar_arrive(pc_full);
+      }
+      if (st.pass == 0) {
+        // D2 epilogue: P += s_c (T_hi + T_lo) for this half's 16 coefficients
+        if (c == 0) {
 #pragma unroll
-      for (int k = 0; k < 32; ++k) P[k] = 0.0f;
-      float sc_next = live ? __ldg(srow) : 0.0f;  // scale of the next chunk, loaded one chunk ahead
-      for (int c = 0; c < nc; ++c, ++step, ++d2) {
-        const float sc = sc_next;
-        if (live && c + 1 < nc) sc_next = __ldg(srow + c + 1);
+          for (int k = 0; k < 16; ++k) P[k] = 0.0f;
+        }
         const int b = d2 & 1;
-        stop = named_sync_or(2, 128, !mbar_wait(&t_full[b], (d2 >> 1) & 1u, kWaitLimit));
+        stop = named_sync_or(2, 256, !mbar_wait(&t_full[b], (d2 >> 1) & 1u, kWaitLimit));
         if (stop) {
           failed = 1;
           break;
         }
         tc_fence_after();
-        uint32_t tr[64];
-        const uint32_t tcol = tbase + lane_off + (b ? kColT1 : kColT0);
-        tmem_ld32(tcol, tr);
-        tmem_ld32(tcol + 32, tr + 32);
+        uint32_t th[16], tl[16];
+        const uint32_t tcol = tbase + lane_off + (b ? kColT1 : kColT0) + 16 * h;
+        tmem_ld16(tcol, th);
+        tmem_ld16(tcol + 32, tl);
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(&t_empty[b]);
 #pragma unroll
-        for (int k = 0; k < 32; ++k) P[k] = fmaf(sc, __uint_as_float(tr[k]) + __uint_as_float(tr[32 + k]), P[k]);
-      }
-      if (stop) break;
-      // P o c -> bf16 hi/lo A operand of D3
-      uint32_t hi[16], lo[16];
-#pragma unroll
-      for (int k = 0; k < 16; ++k) {
-        float h0, l0, h1, l1;
-        split_bf16(P[2 * k] * cf[2 * k], h0, l0);
-        split_bf16(P[2 * k + 1] * cf[2 * k + 1], h1, l1);
-        hi[k] = pack_bf16x2(h0, h1);
-        lo[k] = pack_bf16x2(l0, l1);
-      }
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-        st_shared_v4(pc_tile + sw128(r, q), hi[4 * q], hi[4 * q + 1], hi[4 * q + 2], hi[4 * q + 3]);
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-        st_shared_v4(pc_tile + sw128(r, 4 + q), lo[4 * q], lo[4 * q + 1], lo[4 * q + 2], lo[4 * q + 3]);
-      fence_async_shared();
-      mbar_arrive(pc_full);
-      // D3 epilogue: G_hat = a s q + acc
-      sc_next = live ? __ldg(srow + nc - 1) : 0.0f;
-      for (int i = 0; i < nc; ++i, ++step, ++e2) {
-        const int c = nc - 1 - i;
-        const float sc3 = sc_next;
-        if (live && c > 0) sc_next = __ldg(srow + c - 1);
-        const int s = step % kDStages;
+        for (int k = 0; k < 16; ++k) P[k] = fmaf(sc, __uint_as_float(th[k]) + __uint_as_float(tl[k]), P[k]);
+        ++d2;
+      } else {
+        // D3 epilogue: G_hat = a s q + acc
         const int b = e2 & 1;
         const bool ok = mbar_wait(&w_full[b], (e2 >> 1) & 1u, kWaitLimit) &&
                         mbar_wait(&cfull[s], (step / kDStages) & 1u, kWaitLimit);
-        stop = named_sync_or(2, 128, !ok);
+        stop = named_sync_or(2, 256, !ok);
         if (stop) {
           failed = 1;
           break;
         }
         tc_fence_after();
-        const uint32_t wcol = tbase + lane_off + (b ? kColW1 : kColW0);
+        const uint32_t wcol = tbase + lane_off + (b ? kColW1 : kColW0) + 64 * h;
         const uint32_t c_tile = sbase + s * kDStageBytes;
-        const float as = a * sc3;
-        __nv_bfloat16* dst = J.out + row * J.d_in + c * kChunk;
+        const uint32_t o_tile = c_tile + kDCodes;  // two [128][64] bf16 boxes, 128-byte swizzle
+        const float as = a * sc;
 #pragma unroll
-        for (int g4 = 0; g4 < 4; ++g4) {
+        for (int g2 = 0; g2 < 2; ++g2) {
           uint32_t acc[32];
-          tmem_ld32(wcol + g4 * 32, acc);
+          tmem_ld32(wcol + g2 * 32, acc);
           tmem_wait_ld();
-          // codes 32*g4 .. 32*g4+31 of this row: two 16-byte chunks
+          // codes 64 h + 32 g2 .. + 31 of this row: two 16-byte chunks
           uint32_t o[16];
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const uint4 v = ld_shared_v4(c_tile + sw128(r, 2 * g4 + h));
+          for (int hh = 0; hh < 2; ++hh) {
+            const uint4 v = ld_shared_v4(c_tile + sw128(r, 4 * h + 2 * g2 + hh));
             const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const float2 f0 = e4m3x2_to_f32x2((uint16_t)(w[e] & 0xFFFFu));
               const float2 f1 = e4m3x2_to_f32x2((uint16_t)(w[e] >> 16));
-              const int k = h * 16 + e * 4;
-              o[h * 8 + 2 * e] = pack_bf16x2(fmaf(as, f0.x, __uint_as_float(acc[k])),
-                                             fmaf(as, f0.y, __uint_as_float(acc[k + 1])));
-              o[h * 8 + 2 * e + 1] = pack_bf16x2(fmaf(as, f1.x, __uint_as_float(acc[k + 2])),
-                                                 fmaf(as, f1.y, __uint_as_float(acc[k + 3])));
+              const int k = hh * 16 + e * 4;
+              o[hh * 8 + 2 * e] = pack_bf16x2(fmaf(as, f0.x, __uint_as_float(acc[k])),
+                                              fmaf(as, f0.y, __uint_as_float(acc[k + 1])));
+              o[hh * 8 + 2 * e + 1] = pack_bf16x2(fmaf(as, f1.x, __uint_as_float(acc[k + 2])),
+                                                  fmaf(as, f1.y, __uint_as_float(acc[k + 3])));
             }
           }
-          if (live) {
-            uint4* d4 = reinterpret_cast<uint4*>(dst + g4 * 32);
-            __stcs(d4 + 0, make_uint4(o[0], o[1], o[2], o[3]));
-            __stcs(d4 + 1, make_uint4(o[4], o[5], o[6], o[7]));
-            __stcs(d4 + 2, make_uint4(o[8], o[9], o[10], o[11]));
-            __stcs(d4 + 3, make_uint4(o[12], o[13], o[14], o[15]));
-          }
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            st_shared_v4(o_tile + h * kGHalf + sw128(r, 4 * g2 + q), o[4 * q], o[4 * q + 1], o[4 * q + 2],
+                         o[4 * q + 3]);
         }
         tc_fence_before();
         mbar_arrive(&w_empty[b]);
-        named_sync(2, 128);
-        if (r == 0) mbar_arrive(&empty[s]);
+        fence_async_shared();
+        mbar_arrive(&oready[s]);
+        ++e2;
       }
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 8) tmem_dealloc(tbase, kTmemCols);
+  if (warp == 12) tmem_dealloc(tbase, kTmemCols);
   if (threadIdx.x == 0 && failed && err) atomicOr(err, GIFT_DEV_TIMEOUT);
 }
 
@@ -835,7 +917,9 @@ cudaError_t launch_whiten_encode_tc(const TcLayer* layers, int n, cudaStream_t s
       EncJob& J = P.jobs[l];
       if (!make_tmap_2d(&J.tmG, L.G, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)L.d_out, (uint64_t)L.d_in,
                         kPanel, 64) ||
-          !make_tmap_2d(&J.tmU, L.U, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, (uint64_t)L.d_in, 32, kChunk, 32))
+          !make_tmap_2d(&J.tmU, L.U, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, (uint64_t)L.d_in, 32, kChunk, 32) ||
+          !make_tmap_2d(&J.tmC, L.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)L.d_out, (uint64_t)L.d_in,
+                        kPanel, kChunk))
         return cudaErrorInvalidValue;
       J.U = L.U;
       J.lambda = L.lambda;
@@ -888,13 +972,14 @@ cudaError_t launch_whiten_decode_tc(const TcLayer* layers, int n, cudaStream_t s
       DecJob& J = P.jobs[l];
       if (!make_tmap_2d(&J.tmC, L.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)L.d_out, (uint64_t)L.d_in,
                         kPanel, kChunk) ||
-          !make_tmap_2d(&J.tmU, L.U, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, (uint64_t)L.d_in, 32, kChunk, 32))
+          !make_tmap_2d(&J.tmU, L.U, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, (uint64_t)L.d_in, 32, kChunk, 32) ||
+          !make_tmap_2d(&J.tmO, L.G_hat, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)L.d_out, (uint64_t)L.d_in,
+                        kPanel, 64))
         return cudaErrorInvalidValue;
       J.U = L.U;
       J.lambda = L.lambda;
       J.rho = L.rho;
       J.scales = L.scales;
-      J.out = (__nv_bfloat16*)L.G_hat;
       J.d_out = L.d_out;
       J.d_in = L.d_in;
       J.rank = L.rank;
