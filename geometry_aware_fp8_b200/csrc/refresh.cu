@@ -337,8 +337,10 @@ constexpr int kST = 1024;  // threads of the single-CTA small-matrix kernels
 // k > j, by G[i][k] -= G[i][j] G[k][j] / G[j][j]; one barrier per column.
 // A pivot below kCholTol of the largest diagonal entry drops column j
 // (L[:, j] = e_j, flagged), so that column of Q comes out zero.
-// Output: Lout (m x m, row-major, lower part + diagonal), inv[j] = 1/L[j][j]
-// (0 for dropped columns).
+// Output: Lout = X (m x m, row-major, lower triangle), the inverse of L in
+// the sense of the forward substitution that qr_apply_kernel applies to every
+// row:  x_i = inv_i (e_i - sum_{k<i} L[i][k] x_k),  inv_i = 1/L[i][i] (0 for a
+// dropped column, whose row of X is then zero), followed by inv (m).
 __global__ void __launch_bounds__(kST) chol_kernel(const __grid_constant__ RefBatch bt) {
   const RefLayer& Lr = bt.L[blockIdx.z];
   const double* __restrict__ part = Lr.gram;
@@ -394,20 +396,34 @@ __global__ void __launch_bounds__(kST) chol_kernel(const __grid_constant__ RefBa
     }
     __syncthreads();
   }
-  // L[i][j] = G[i][j] / sqrt(piv_j) below the diagonal, sqrt(piv_j) on it
+  // L[i][j] = G[i][j] / sqrt(piv_j) below the diagonal (in place; the
+  // diagonal is not needed below: inv carries it)
+  __shared__ double inv[64];
+  if (threadIdx.x < m) inv[threadIdx.x] = piv[threadIdx.x] > 0.0 ? 1.0 / sqrt(piv[threadIdx.x]) : 0.0;
   for (int e = threadIdx.x; e < m * m; e += kST) {
     const int i = e / m, j = e % m;
     const double pj = piv[j];
-    double v = 0.0;
-    if (pj > 0.0) {
-      if (i == j) v = sqrt(pj);
-      else if (i > j) v = G[i * ld + j] / sqrt(pj);
-    } else if (i == j) {
-      v = 1.0;
-    }
-    Lout[e] = v;
+    if (i > j) G[i * ld + j] = pj > 0.0 ? G[i * ld + j] / sqrt(pj) : 0.0;
   }
-  if (threadIdx.x < m) Lout[m * m + threadIdx.x] = piv[threadIdx.x] > 0.0 ? 1.0 / sqrt(piv[threadIdx.x]) : 0.0;
+  // Z = unscaled rows of X, right-looking: Z starts as I; once row k is final
+  // (after step k-1), every row i > k takes Z[i] -= L[i][k] inv_k Z[k]
+  // (entries j <= k).  X[i] = inv_i Z[i].  One barrier per k.
+  double* Z = sm + 64 * ld;
+  for (int e = threadIdx.x; e < m * m; e += kST) Z[(e / m) * ld + e % m] = (e / m == e % m) ? 1.0 : 0.0;
+  __syncthreads();
+  for (int k = 0; k + 1 < m; ++k) {
+    const double ik = inv[k];
+    for (int e = threadIdx.x; e < (m - 1 - k) * (k + 1); e += kST) {
+      const int i = k + 1 + e / (k + 1), j = e % (k + 1);
+      Z[i * ld + j] -= G[i * ld + k] * ik * Z[k * ld + j];
+    }
+    __syncthreads();
+  }
+  for (int e = threadIdx.x; e < m * m; e += kST) {
+    const int i = e / m, j = e % m;
+    Lout[e] = j <= i ? inv[i] * Z[i * ld + j] : 0.0;
+  }
+  if (threadIdx.x < m) Lout[m * m + threadIdx.x] = inv[threadIdx.x];
   if (threadIdx.x == 0 && dev_status) {
     uint32_t f = 0;
     for (int j = 0; j < m; ++j)
@@ -417,49 +433,48 @@ __global__ void __launch_bounds__(kST) chol_kernel(const __grid_constant__ RefBa
   }
 }
 
-// Qo = Yi R^{-1} with R = L^T: for each row, the forward substitution
-// q_c = (y_c - sum_{k<c} q_k L[c][k]) / L[c][c] (fp64), q_c = 0 for dropped
-// columns.  One warp per row: lane l owns columns l and l+32, the owner of
-// column c finishes q_c and broadcasts it.
+// Qo = Yi R^{-1} with R = L^T, i.e. every row q = X y with X the
+// substitution inverse written by chol_kernel (fp64 products, fp32 out).
+// A CTA keeps X in shared memory and walks 32-row tiles of Yi; thread
+// (i, rg) computes column i of rows rg, rg + 4, ..., rg + 28 of the tile.
+// With dst == Q the bf16 [hi | lo] operand of the tensor-core product is
+// written too (columns m..63 zero).
 __global__ void __launch_bounds__(kRT) qr_apply_kernel(const __grid_constant__ RefBatch bt, int src, int dst) {
   const RefLayer& Lr = bt.L[blockIdx.z];
   const int d = Lr.d, m = bt.m;
   const float* __restrict__ Yi = Lr.buf[src];
-  const double* __restrict__ L = Lr.Lf;
+  const double* __restrict__ X = Lr.Lf;
   float* __restrict__ Qo = Lr.buf[dst];
-  __shared__ double Ls[64 * 65];
-  __shared__ double inv[64];
-  for (int e = threadIdx.x; e < m * m; e += kRT) Ls[(e / m) * 65 + e % m] = L[e];
-  if (threadIdx.x < m) inv[threadIdx.x] = L[m * m + threadIdx.x];
-  __syncthreads();
-  const int lane = threadIdx.x & 31;
-  for (int64_t row = (int64_t)blockIdx.x * (kRT / 32) + (threadIdx.x >> 5); row < d;
-       row += (int64_t)gridDim.x * (kRT / 32)) {
-    double acc0 = lane < m ? (double)Yi[row * m + lane] : 0.0;
-    double acc1 = lane + 32 < m ? (double)Yi[row * m + lane + 32] : 0.0;
-    double q0 = 0.0, q1 = 0.0;
-    for (int c = 0; c < m; ++c) {
-      double qc;
-      if (c < 32) {
-        qc = __shfl_sync(0xffffffffu, acc0 * inv[c], c);
-        if (lane == c) q0 = qc;
-      } else {
-        qc = __shfl_sync(0xffffffffu, acc1 * inv[c], c - 32);
-        if (lane == c - 32) q1 = qc;
+  __nv_bfloat16* __restrict__ Qs = dst == kBufQ ? Lr.Qs : nullptr;
+  __shared__ double Xs[64 * 65];
+  __shared__ float Ys[32 * 65];
+  if ((int64_t)blockIdx.x * 32 >= d) return;
+  for (int e = threadIdx.x; e < m * m; e += kRT) Xs[(e / m) * 65 + e % m] = X[e];
+  const int i = threadIdx.x & 63, rg = threadIdx.x >> 6;
+  for (int64_t t0 = (int64_t)blockIdx.x * 32; t0 < d; t0 += (int64_t)gridDim.x * 32) {
+    __syncthreads();
+    for (int e = threadIdx.x; e < 32 * m; e += kRT) Ys[(e / m) * 65 + e % m] = Yi[t0 * m + e];
+    __syncthreads();
+    double acc[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) acc[u] = 0.0;
+    if (i < m) {
+      for (int j = 0; j <= i; ++j) {
+        const double x = Xs[i * 65 + j];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) acc[u] = fma(x, (double)Ys[(rg + 4 * u) * 65 + j], acc[u]);
       }
-      if (lane > c) acc0 -= qc * Ls[lane * 65 + c];
-      if (lane + 32 > c && lane + 32 < m) acc1 -= qc * Ls[(lane + 32) * 65 + c];
     }
-    if (lane < m) Qo[row * m + lane] = (float)q0;
-    if (lane + 32 < m) Qo[row * m + lane + 32] = (float)q1;
-    if (dst == kBufQ && Lr.Qs) {  // bf16 [hi | lo] operand of the tensor-core product
-      const float f0 = (float)q0, f1 = (float)q1;
-      const float h0 = __bfloat162float(__float2bfloat16_rn(f0)), h1 = __bfloat162float(__float2bfloat16_rn(f1));
-      __nv_bfloat16* qs = Lr.Qs + row * 128;
-      qs[lane] = __float2bfloat16_rn(h0);
-      qs[lane + 32] = __float2bfloat16_rn(h1);
-      qs[64 + lane] = __float2bfloat16_rn(f0 - h0);
-      qs[96 + lane] = __float2bfloat16_rn(f1 - h1);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int64_t row = t0 + rg + 4 * u;
+      const float q = (float)acc[u];
+      if (i < m) Qo[row * m + i] = q;
+      if (Qs) {
+        const float hi = __bfloat162float(__float2bfloat16_rn(q));
+        Qs[row * 128 + i] = __float2bfloat16_rn(hi);
+        Qs[row * 128 + 64 + i] = __float2bfloat16_rn(q - hi);
+      }
     }
   }
 }
@@ -670,7 +685,7 @@ __global__ void form_u_kernel(const __grid_constant__ RefBatch bt) {
   }
 }
 
-constexpr size_t kCholSmem = 64 * 65 * sizeof(double);
+constexpr size_t kCholSmem = 2 * 64 * 65 * sizeof(double);
 constexpr size_t kRRSmem = 4 * 64 * 65 * sizeof(double);
 
 // k-slices of the skinny product: enough CTAs to cover the SMs twice
@@ -790,10 +805,8 @@ cudaError_t launch_refresh_batch(const RefreshPlan* plans, const RefreshIO* io, 
     }
     const int64_t dm = (int64_t)dmax * m;
     const int ew_blocks = (int)((dm + kRT - 1) / kRT < 2 * kNumSMs ? (dm + kRT - 1) / kRT : 2 * kNumSMs);
-    // qr_apply: each CTA loads the m x m factor once, so use just enough CTAs
-    // per layer to cover the SMs about twice over the whole batch
-    int qr_blocks = (2 * kNumSMs + cnt - 1) / cnt;
-    if (qr_blocks > (dmax + 7) / 8) qr_blocks = (dmax + 7) / 8;
+    // qr_apply: two 32-row tiles per CTA (the m x m factor is loaded once per CTA)
+    const int qr_blocks = (dmax / 32 + 1) / 2;
     const dim3 g_ew(ew_blocks, 1, cnt), g_skinny(dmax / 64, nsmax, cnt), g_gram(pmax, 1, cnt), g_one(1, 1, cnt),
         g_qr(qr_blocks, 1, cnt);
     // one Cholesky-QR pass: dst = src R^{-1} with src^T src = R^T R
