@@ -226,6 +226,33 @@ def step(ops, W, k, ev=None):
     rec(6)
 
 
+# DRAM traffic (read + write bytes per gradient element) of the whitened codec
+# launches from one ncu capture of the depth-8 stack (16 whitened layers); the
+# kernels' work grows in proportion to the elements, so the bench's launch is
+# that figure x its elements.  Valid only for the kernel source it was taken
+# on (sha256 of the file); otherwise the bench reports traffic as null.
+TRAFFIC = {
+    "encode_whitened": {"bytes_per_element": 222.925312e6 / 69206016,
+                        "profile": "profiles/whiten_encode_tc_stack8.md"},
+    "decode_whitened": {"bytes_per_element": 174.122752e6 / 69206016,
+                        "profile": "profiles/whiten_decode_tc_stack8.md"},
+}
+TRAFFIC_SOURCE = ("geometry_aware_fp8_b200/csrc/codec_tc.cu",
+                  "4edd617c87fff8f3d1bf0028a359453eade8269c207088792592e9952795f009")
+
+
+def traffic_for(phase, n_elements):
+    import hashlib
+    t = TRAFFIC.get(phase)
+    path = os.path.join(ROOT, TRAFFIC_SOURCE[0])
+    if t is None or not os.path.exists(path):
+        return None
+    with open(path, "rb") as f:
+        if hashlib.sha256(f.read()).hexdigest() != TRAFFIC_SOURCE[1]:
+            return None
+    return t["bytes_per_element"] * n_elements
+
+
 def phase_bytes(W):
     """Algorithmic bytes of each codec launch: encode reads G (2 B/element) and
     writes codes (1 B) + scales (4/128 B); decode the reverse; plus U per layer."""
@@ -347,7 +374,9 @@ def run_gpu(args):
     achieved = pb[dom] / (pm[dom] * 1e-3) / 1e9
     roofline = {"bound": "hbm", "kernel": f"{dom} (one grouped launch over its layers of the stack)",
                 "achieved": achieved, "peak": peak, "peak_source": peak_kind, "unit": "GB/s",
-                "frac": achieved / peak, "traffic": None}
+                "frac": achieved / peak,
+                "traffic": traffic_for(dom, W["n_wh"] if dom.endswith("whitened") else W["n_eu"]),
+                "traffic_unit": "bytes per launch (DRAM read + write, ncu, scaled from the depth-8 capture)"}
     codec_ms = sum(pm[n] for n in pb)
     ref_steps = [k for k in range(K) if k % K_REFRESH == 0]
     codec = {"phase_ms": pm,
