@@ -45,18 +45,21 @@ namespace {
 
 constexpr int kPanel = 128;                 // rows per panel = UMMA M
 constexpr int kChunk = 128;                 // columns per step = one scale block
-constexpr int kStages = 4;
+constexpr int kStages = 3;
 constexpr int kGBytes = kPanel * kChunk * 2;   // 32 KB: two [128][64] bf16 boxes
 constexpr int kGHalf = kGBytes / 2;
 constexpr int kUBytes = kChunk * 128;          // 16 KB: [128 rows][64 bf16]
 constexpr int kStageBytes = kGBytes + kUBytes;
 constexpr int kPcBytes = kPanel * 128;         // 16 KB: [128 rows][64 bf16]
-constexpr int kSmemBytes = kStages * kStageBytes + kPcBytes + 1024 + 512;
+constexpr int kCodesBytes = kPanel * kChunk;    // 16 KB: codes of one chunk
+constexpr int kIdBytes = 16 * 128;             // 2 KB: 16 x 16 bf16 identity, 128-byte rows
+constexpr int kSmemBytes = kStages * kStageBytes + kPcBytes + 2 * kCodesBytes + kIdBytes + 1024 + 512;
 constexpr int kThreads = 480;  // 8 epilogue + 4 converter + MMA + TMA load + TMA store warps
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColW0 = 0, kColW1 = 128, kColP = 256;
 constexpr uint32_t kIdescE1 = umma_idesc_bf16(128, 64, 0, 1);   // A K-major, B MN-major
 constexpr uint32_t kIdescE2 = umma_idesc_bf16(128, 128, 0, 0);  // both K-major
+constexpr uint32_t kIdescId = umma_idesc_bf16(128, 16, 0, 0);   // G . I16, both K-major
 constexpr uint32_t kWaitLimit = 1u << 22;
 constexpr int kMaxJobs = 48;
 constexpr int kMaxPanels = 1536;
@@ -229,16 +232,19 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const uint32_t sbase = smem_u32(smem);
   const uint32_t pc_tile = sbase + kStages * kStageBytes;
-  uint64_t* bars = (uint64_t*)(smem + kStages * kStageBytes + kPcBytes);
+  const uint32_t cbuf = pc_tile + kPcBytes;             // [2] codes tiles [128][128 B], 128-byte swizzle
+  const uint32_t id_tile = cbuf + 2 * kCodesBytes;      // 16 x 16 identity, K-major, 128-byte swizzle
+  uint64_t* bars = (uint64_t*)(smem + kStages * kStageBytes + kPcBytes + 2 * kCodesBytes + kIdBytes);
   uint64_t* full = bars;                  // [kStages] count 1: converter (stage ready for the MMA)
-  uint64_t* empty = bars + kStages;       // [kStages] count 1: MMA commit (E1) or code store (E2)
+  uint64_t* empty = bars + kStages;       // [kStages] count 1: MMA commit
   uint64_t* tfull = bars + 2 * kStages;   // [kStages] count 1 + tx: TMA (G and fp32 U)
-  uint64_t* cready = bars + 3 * kStages;  // [kStages] count 256: codes of an E2 step in shared memory
-  uint64_t* p_full = bars + 4 * kStages;  // count 1 (MMA commit)
+  uint64_t* p_full = bars + 3 * kStages;  // count 1 (MMA commit)
   uint64_t* pc_full = p_full + 1;         // count 256 (epilogue)
   uint64_t* w_full = p_full + 2;          // [2] count 1
   uint64_t* w_empty = p_full + 4;         // [2] count 256
-  uint32_t* tmem_slot = (uint32_t*)(p_full + 6);
+  uint64_t* cready = p_full + 6;          // [2] count 256: a codes tile is written
+  uint64_t* cfree = p_full + 8;           // [2] count 1: the store of a codes tile has read it
+  uint32_t* tmem_slot = (uint32_t*)(p_full + 10);
   __shared__ int failed;  // any role gave up (reported at exit)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -250,15 +256,28 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
       mbar_init(&tfull[s], 1);
-      mbar_init(&cready[s], 256);
     }
     mbar_init(p_full, 1);
     mbar_init(pc_full, 256);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&w_full[b], 1);
       mbar_init(&w_empty[b], 256);
+      mbar_init(&cready[b], 256);
+      mbar_init(&cfree[b], 1);
     }
     fence_mbar_init();
+  }
+  if (warp == 0) {
+    // identity I16 as a K-major B operand: row n holds e_n in its first 32 bytes
+    for (int n = lane; n < 16; n += 32) {
+#pragma unroll
+      for (int q = 0; q < 8; ++q) st_shared_v4(id_tile + sw128(n, q), 0u, 0u, 0u, 0u);
+      const uint32_t one = 0x3F80u << (16 * (n & 1));  // bf16 1.0 in the half of the word for column n
+      const uint32_t w4[4] = {(n & 7) >> 1 == 0 ? one : 0u, (n & 7) >> 1 == 1 ? one : 0u,
+                              (n & 7) >> 1 == 2 ? one : 0u, (n & 7) >> 1 == 3 ? one : 0u};
+      st_shared_v4(id_tile + sw128(n, n >> 3), w4[0], w4[1], w4[2], w4[3]);
+    }
+    fence_async_shared();
   }
   if (warp == 12) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -291,23 +310,23 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
       }
     }
   } else if (warp == 14) {
-    // ---------------- code stores: one TMA store per E2 step, then the stage is free ----------------
+    // ---------------- code stores: one TMA store per second-pass step ----------------
     if (lane == 0) {
       const uint64_t drop = policy_evict_first();
-      uint32_t step = 0, par = 0;  // par: bit s = phase parity of cready[s]
-      for (Steps<EncParams> st(p, beg, end); st.valid() && !failed; st.next(), ++step) {
+      uint32_t e2 = 0;
+      for (Steps<EncParams> st(p, beg, end); st.valid() && !failed; st.next()) {
         if (st.pass == 0) continue;
-        const int s = step % kStages;
-        if (!mbar_wait(&cready[s], (par >> s) & 1u, kWaitLimit)) {
+        const int cb = e2 & 1;
+        if (!mbar_wait(&cready[cb], (e2 >> 1) & 1u, kWaitLimit)) {
           failed = 1;
           break;
         }
-        par ^= 1u << s;
         const EncJob& J = p.jobs[st.job()];
-        tma_store_2d_hint(&J.tmC, sbase + s * kStageBytes + kGBytes, st.chunk() * kChunk, st.panel() * kPanel, drop);
+        tma_store_2d_hint(&J.tmC, cbuf + cb * kCodesBytes, st.chunk() * kChunk, st.panel() * kPanel, drop);
         bulk_commit();
         bulk_wait_read<0>();
-        mbar_arrive(&empty[s]);
+        mbar_arrive(&cfree[cb]);
+        ++e2;
       }
       bulk_wait_all();
     }
@@ -336,7 +355,7 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
       uint32_t step = 0, e2 = 0;
       for (Steps<EncParams> st(p, beg, end); st.valid() && !failed; st.next(), ++step) {
         const int s = step % kStages;
-        // block k >= 1 starts with the second pass of p_{k-1}: its P o c must be
+        // block k >= 1 starts with the second pass of p_{k-1}: its P o (c/a) must be
         // in shared memory, and P in TMEM has been read (it is reused for p_k)
         if (st.block_start() && st.k >= 1 && !mbar_wait(pc_full, (st.k - 1) & 1u, kWaitLimit)) { failed = 1; break; }
         if (!mbar_wait(&full[s], (step / kStages) & 1u, kWaitLimit)) { failed = 1; break; }
@@ -356,7 +375,8 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
           umma_commit(&empty[s]);
           if (c == st.nc() - 1) umma_commit(p_full);
         } else {
-          // E2: W[128 x 128] = Pc_hi U_hi^T + Pc_lo U_hi^T + Pc_hi U_lo^T
+          // E2: W/a [128 x 128] = Pc_hi U_hi^T + Pc_lo U_hi^T + Pc_hi U_lo^T + G . I
+          // (Pc already divided by a; G . I adds G exactly, 16 columns per MMA)
           const int b = e2 & 1;
           if (e2 >= 2 && !mbar_wait(&w_empty[b], ((e2 >> 1) - 1) & 1u, kWaitLimit)) { failed = 1; break; }
           tc_fence_after();
@@ -369,6 +389,13 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
             const uint64_t bd = umma_desc_sw128(u_tile + bk[q] * 2, 16, 1024);
             umma_bf16(d, ad, bd, kIdescE2, q ? 1u : 0u);
           }
+          const uint64_t idd = umma_desc_sw128(id_tile, 16, 1024);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const uint64_t ad = umma_desc_sw128(g_tile + (j >> 2) * kGHalf + (j & 3) * 32, 16, 1024);
+            umma_bf16(d + 16 * j, ad, idd, kIdescId, 1u);
+          }
+          umma_commit(&empty[s]);
           umma_commit(&w_full[b]);
           ++e2;
         }
@@ -377,32 +404,31 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
   } else {
     // ---------------- epilogue: warps 0-7 ----------------
     // Thread (r, h): row r = 32 (warp % 4) + lane of the panel (its TMEM
-    // lane), columns 64 h .. 64 h + 63 of every 128-column chunk (h = warp / 4,
-    // the G box it reads).  The two halves of a row exchange their partial
-    // block maxima through shared memory.  The codes of a chunk are written
-    // into the stage's U tile, which the E2 MMA no longer needs once W is in
-    // TMEM, for the store warp.
+    // lane), columns 64 h .. 64 h + 63 of every 128-column chunk (h = warp / 4).
+    // TMEM holds W' = W / a; the two halves of a row exchange their partial
+    // block maxima through shared memory and write their codes into one of two
+    // codes tiles for the store warp.
     __shared__ float amax_x[2][128];
     const int h = warp >> 2;
     const int r = (warp & 3) * 32 + lane;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    uint32_t step = 0, e2 = 0;
+    uint32_t e2 = 0;
     float a = 0.0f;
     bool stop = false;  // group vote: set for all 256 threads at the same barrier
-    for (Steps<EncParams> st(p, beg, end); st.valid() && !stop; st.next(), ++step) {
+    for (Steps<EncParams> st(p, beg, end); st.valid() && !stop; st.next()) {
       if (st.pass == 0) continue;  // first-pass steps are the MMA's alone
       const EncJob& J = p.jobs[st.job()];
       const int panel = st.panel();
       if (st.i2 == 0) {
-        // P o c of this panel for k = 16 h .. 16 h + 15, split into the bf16 A operand of E2
+        // P o (c / a) of this panel for k = 16 h .. 16 h + 15, split into the bf16
+        // A operand of E2:  c_k / a = (rho / (lambda_k + rho))^{1/2} - 1
         const double rho = (double)__ldg(J.rho);
-        const double a64 = 1.0 / sqrt(rho);
-        a = (float)a64;
+        a = (float)(1.0 / sqrt(rho));
         float cf[16];
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
           const int kk = 16 * h + k;
-          cf[k] = kk < J.rank ? (float)(1.0 / sqrt((double)__ldg(J.lambda + kk) + rho) - a64) : 0.0f;
+          cf[k] = kk < J.rank ? (float)(sqrt(rho / ((double)__ldg(J.lambda + kk) + rho)) - 1.0) : 0.0f;
         }
         stop = named_sync_or(2, 256, !mbar_wait(p_full, (st.k - 1) & 1u, kWaitLimit));
         if (stop) {
@@ -434,61 +460,60 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
         mbar_arrive(pc_full);
       }
       const int c = st.chunk();
-      const int s = step % kStages;
       const int b = e2 & 1;
       const int64_t row = (int64_t)panel * kPanel + r;
       const bool live = row < J.d_out;
-      const bool ok = mbar_wait(&w_full[b], (e2 >> 1) & 1u, kWaitLimit) &&
-                      mbar_wait(&tfull[s], (step / kStages) & 1u, kWaitLimit);
-      stop = named_sync_or(2, 256, !ok);
+      stop = named_sync_or(2, 256, !mbar_wait(&w_full[b], (e2 >> 1) & 1u, kWaitLimit));
       if (stop) {
         failed = 1;
         break;
       }
       tc_fence_after();
       const uint32_t wcol = tbase + lane_off + (b ? kColW1 : kColW0) + 64 * h;
-      const uint32_t g_box = sbase + s * kStageBytes + h * kGHalf;  // this half's 64 columns
-      // w = a g + acc for the 64 columns, and their maximum
-      float w[64];
-      float amax = 0.0f;
-#pragma unroll
-      for (int g2 = 0; g2 < 2; ++g2) {
-        uint32_t acc[32];
-        tmem_ld32(wcol + g2 * 32, acc);
-        tmem_wait_ld();
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const uint4 gv = ld_shared_v4(g_box + sw128(r, g2 * 4 + q));
-          const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int k = g2 * 32 + q * 8 + 2 * e;
-            w[k] = fmaf(a, bf16lo(gw[e]), __uint_as_float(acc[q * 8 + 2 * e]));
-            w[k + 1] = fmaf(a, bf16hi(gw[e]), __uint_as_float(acc[q * 8 + 2 * e + 1]));
-            amax = fmaxf(amax, fmaxf(fabsf(w[k]), fabsf(w[k + 1])));
-          }
-        }
-      }
+      uint32_t w[64];
+      tmem_ld32(wcol, w);
+      tmem_ld32(wcol + 32, w + 32);
+      tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(&w_empty[b]);
-      amax_x[h][r] = amax;
-      named_sync(2, 256);
-      amax = fmaxf(amax_x[0][r], amax_x[1][r]);
+      float m0 = 0.0f, m1 = 0.0f, m2 = 0.0f, m3 = 0.0f;
+#pragma unroll
+      for (int k = 0; k < 64; k += 4) {
+        m0 = fmaxf(m0, fabsf(__uint_as_float(w[k])));
+        m1 = fmaxf(m1, fabsf(__uint_as_float(w[k + 1])));
+        m2 = fmaxf(m2, fabsf(__uint_as_float(w[k + 2])));
+        m3 = fmaxf(m3, fabsf(__uint_as_float(w[k + 3])));
+      }
+      amax_x[h][r] = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+      // the codes tile is free once the store of its previous use has read it;
+      // this barrier also exchanges the halves' maxima
+      const int cb = e2 & 1;
+      const bool freed = e2 < 2 || mbar_wait(&cfree[cb], ((e2 >> 1) - 1) & 1u, kWaitLimit);
+      stop = named_sync_or(2, 256, !freed);
+      if (stop) {
+        failed = 1;
+        break;
+      }
+      // block maximum of W = a W' (rounded once), then the codes of W' x (a 448 / amax)
+      const float amax = __fmul_rn(a, fmaxf(amax_x[0][r], amax_x[1][r]));
       const float inv = e4m3_inv_scale(amax);
+      const float ai = __fmul_rn(a, inv);
       uint32_t cw[16];
 #pragma unroll
       for (int q = 0; q < 16; ++q) {
-        const uint32_t c01 = f32x2_to_e4m3x2(__fmul_rn(w[4 * q], inv), __fmul_rn(w[4 * q + 1], inv));
-        const uint32_t c23 = f32x2_to_e4m3x2(__fmul_rn(w[4 * q + 2], inv), __fmul_rn(w[4 * q + 3], inv));
+        const uint32_t c01 = f32x2_to_e4m3x2(__fmul_rn(__uint_as_float(w[4 * q]), ai),
+                                             __fmul_rn(__uint_as_float(w[4 * q + 1]), ai));
+        const uint32_t c23 = f32x2_to_e4m3x2(__fmul_rn(__uint_as_float(w[4 * q + 2]), ai),
+                                             __fmul_rn(__uint_as_float(w[4 * q + 3]), ai));
         cw[q] = inv > 0.0f ? (c01 | (c23 << 16)) : 0u;
       }
-      const uint32_t c_tile = sbase + s * kStageBytes + kGBytes;  // [128][128 B], 128-byte swizzle
+      if (live && h == 0) J.scales[row * (J.d_in / kChunk) + c] = e4m3_scale(amax, inv);
+      const uint32_t c_tile = cbuf + cb * kCodesBytes;
 #pragma unroll
       for (int q = 0; q < 4; ++q)
         st_shared_v4(c_tile + sw128(r, 4 * h + q), cw[4 * q], cw[4 * q + 1], cw[4 * q + 2], cw[4 * q + 3]);
-      if (live && h == 0) J.scales[row * (J.d_in / kChunk) + c] = e4m3_scale(amax, inv);
       fence_async_shared();
-      mbar_arrive(&cready[s]);
+      mbar_arrive(&cready[cb]);
       ++e2;
     }
   }
@@ -509,7 +534,7 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
 // Stage = codes tile (TMA, [128][128 B], 128-byte swizzle) + bf16 copy of the
 // codes (the D2 A operand, written by the converter warps) + U tile.
 // ===========================================================================
-constexpr int kDStages = 3;
+constexpr int kDStages = 3;  // decode ring
 constexpr int kDCodes = kPanel * kChunk;            // 16 KB
 constexpr int kDQ = kPanel * kChunk * 2;            // 32 KB: two [128][64] bf16 tiles
 constexpr int kDStageBytes = kDCodes + kDQ + kUBytes;
