@@ -57,6 +57,7 @@ def parse():
     ap.add_argument("--impl", default="gift", choices=["gift", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-nvfp4", action="store_true", help="skip the NVFP4 measurement on the 11008x4096 gradient")
     ap.add_argument("--depth", type=int, default=24, help="layers in the stack (24 = the full stand-in)")
     return ap.parse_args()
 
@@ -192,6 +193,57 @@ def build_workload(torch, ops, synth, dev, depth, seed):
                 n_wh=sum(L.d_out * L.d_in for L in wl), n_eu=sum(L.d_out * L.d_in for L in el),
                 packed_wh=ops.make_layers(wl), n_packed_wh=len(wl),
                 packed_eu=ops.make_layers(el), n_packed_eu=len(el))
+
+
+def nvfp4_measure(torch, ops, synth, dev, peak, reps=20):
+    """NVFP4 codec on one 11008 x 4096 bf16 gradient (an MLP projection of the
+    stand-in model's larger sibling), whitened with a rank-32 factor refreshed
+    from 8192 tokens, and the Euclidean NVFP4 codec on the same tensor.
+    Algorithmic bytes per element and direction: 2 + 0.5 + 1/16 = 2.5625."""
+    d_out, d_in = 11008, 4096
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(5005)
+    Q = torch.from_numpy(synth.haar_orthogonal(d_in, 5003).astype(np.float32)).to(dev)
+    G = synth.device_gradient(d_out, d_in, 1.0, Q, gen, torch.bfloat16)
+    sigma = torch.arange(1, d_in + 1, device=dev, dtype=torch.float32) ** -1.0
+    X = synth.device_activations(REFRESH_N, sigma, Q, gen, torch.bfloat16)
+    U, lam, rho, _ = ops.factor_refresh(X, RANK, OVERSAMPLE, ITERS, seed=5004)
+    del X
+    codes = torch.empty((d_out, d_in // 2), device=dev, dtype=torch.uint8)
+    sb = torch.empty((d_out, d_in // 16), device=dev, dtype=torch.uint8)
+    ts = torch.empty((1,), device=dev, dtype=torch.float32)
+    Gh = torch.empty_like(G)
+    flush = torch.empty((256 << 20,), device=dev, dtype=torch.uint8)  # > L2 between timed calls
+    err = torch.empty((3,), device=dev, dtype=torch.float64)
+    ews = torch.empty((ops.error_workspace_size(d_out, d_in),), device=dev, dtype=torch.uint8)
+
+    def timed(fn):
+        ts_ms = []
+        for i in range(reps + 3):
+            flush.zero_()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            if i >= 3:
+                ts_ms.append(a.elapsed_time(b))
+        return float(np.median(ts_ms))
+
+    out = {"workload": f"G {d_out}x{d_in} bf16, rank {RANK} factor from X {REFRESH_N}x{d_in}; "
+                       "median of 20 calls, L2 flushed between calls",
+           "bytes_per_element_each_way": 2.5625}
+    n = d_out * d_in
+    for name, args in (("whitened", (U, lam, rho)), ("euclid", (None, None, None))):
+        enc = timed(lambda: ops.encode_nvfp4(G, *args, codes=codes, block_scales=sb, tensor_scale=ts))
+        dec = timed(lambda: ops.decode_nvfp4(codes, sb, ts, *args, out=Gh))
+        ops.roundtrip_error(G, Gh, out=err, ws=ews)
+        gbs = 2 * n / ((enc + dec) * 1e-3) / 1e9
+        out[name] = {"encode_ms": enc, "decode_ms": dec, "gradient_gbs": gbs,
+                     "roofline_frac": 2 * 2.5625 * n / ((enc + dec) * 1e-3) / 1e9 / peak,
+                     "roundtrip_rel_error": float(err[0].item())}
+    return out
 
 
 def refresh_all(ops, W):
@@ -388,6 +440,7 @@ def run_gpu(args):
              "codec_roofline_frac": sum(pb.values()) / (codec_ms * 1e-3) / 1e9 / peak}
 
     launches, names = count_launches(torch, ops, W, K)
+    nvfp4 = nvfp4_measure(torch, ops, synth, dev, peak) if not args.no_nvfp4 else None
 
     # ---- end to end through host buffers: the same schedule, with every
     # step's gradients copied in from pinned host memory, the activations of
@@ -438,7 +491,7 @@ def run_gpu(args):
                            "gradient_bytes": g_bytes, "storage": "bf16 G / e4m3 codes / fp32 scales",
                            "l2": "inputs larger than L2 (1.06 GB of gradients streamed per step)",
                            "parallelism": f"replicas x{world}"},
-                "roofline": roofline, "codec": codec, "e2e": e2e, "cpu_baseline": cpu,
+                "roofline": roofline, "codec": codec, "nvfp4": nvfp4, "e2e": e2e, "cpu_baseline": cpu,
                 "gpu_launches": launches, "kernels": names, "clocks": clock_info}
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -255,4 +255,67 @@ gift_status gift_roundtrip_error(const void* G, const void* G_hat, gift_dtype dt
   return cuda_status(launch_roundtrip_error(G, G_hat, dt, d_out * d_in, out, ws, (cudaStream_t)stream));
 }
 
+// ---------------------------------------------------------------------------
+static gift_status check_nvfp4_args(const void* G, int gdt, int64_t d_out, int64_t d_in, const float* U,
+                                    const float* lambda, const float* rho, int rank, const void* codes,
+                                    const void* sb, const float* ts) {
+  if (!dtype_ok(gdt)) return GIFT_ERR_INVALID_ARG;
+  if (d_out < 0 || d_in <= 0) return GIFT_ERR_INVALID_ARG;
+  if (rank < 0 || rank > GIFT_MAX_RANK) return GIFT_ERR_SHAPE;
+  if (d_in % GIFT_NVFP4_BLOCK != 0 || (rank > 0 && d_in % GIFT_E4M3_BLOCK != 0)) return GIFT_ERR_SHAPE;
+  if (d_in > (1 << 20) || d_out > ((int64_t)1 << 31)) return GIFT_ERR_SHAPE;
+  if (rank > 0 && (rank != GIFT_MAX_RANK || gdt != GIFT_BF16 || d_in > 8192)) return GIFT_ERR_UNSUPPORTED;
+  if (d_out == 0) return GIFT_OK;  // empty gradient: nothing is read or written
+  if (!G || !codes || !sb || !ts) return GIFT_ERR_INVALID_ARG;
+  if (rank > 0 && (!U || !lambda || !rho)) return GIFT_ERR_INVALID_ARG;
+  if (!aligned16(G) || !aligned16(codes) || !aligned(sb, 8) || !aligned(ts, 4)) return GIFT_ERR_ALIGN;
+  if (rank > 0 && (!aligned16(U) || !aligned(lambda, 4) || !aligned(rho, 4))) return GIFT_ERR_ALIGN;
+  return GIFT_OK;
+}
+
+gift_status gift_encode_nvfp4(const void* G, gift_dtype gdt, int64_t d_out, int64_t d_in, const float* U,
+                              const float* lambda, const float* rho, int rank, uint8_t* codes,
+                              uint8_t* block_scales, float* tensor_scale, gift_stream_t stream) {
+  gift_status st = check_nvfp4_args(G, gdt, d_out, d_in, U, lambda, rho, rank, codes, block_scales, tensor_scale);
+  if (st != GIFT_OK || d_out == 0) return st;
+  if ((st = device_ok()) != GIFT_OK) return st;
+  if (rank > 0 && !tc_codec_available()) return GIFT_ERR_UNSUPPORTED;
+  cudaStream_t s = (cudaStream_t)stream;
+  // *tensor_scale first accumulates amax(W) as the bits of a non-negative float
+  if (cudaMemsetAsync(tensor_scale, 0, sizeof(float), s) != cudaSuccess) return GIFT_ERR_CUDA;
+  if (rank == 0) {
+    const int64_t nb = d_out * (d_in / GIFT_NVFP4_BLOCK);
+    if ((st = cuda_status(launch_nvfp4_amax(G, gdt, nb, tensor_scale, s))) != GIFT_OK) return st;
+    if ((st = cuda_status(launch_nvfp4_quant(G, gdt, nb, tensor_scale, codes, block_scales, s))) != GIFT_OK) return st;
+  } else {
+    TcLayer L{G, nullptr, codes, nullptr, U, lambda, rho, (int)d_out, (int)d_in, rank};
+    L.block_scales = block_scales;
+    L.tensor_scale = tensor_scale;
+    L.fmt = kFmtNvfp4Amax;
+    if ((st = cuda_status(launch_whiten_encode_tc(&L, 1, s))) != GIFT_OK) return st;
+    L.fmt = kFmtNvfp4;
+    if ((st = cuda_status(launch_whiten_encode_tc(&L, 1, s))) != GIFT_OK) return st;
+  }
+  return cuda_status(launch_nvfp4_finalize(tensor_scale, s));
+}
+
+gift_status gift_decode_nvfp4(const uint8_t* codes, const uint8_t* block_scales, const float* tensor_scale,
+                              int64_t d_out, int64_t d_in, const float* U, const float* lambda, const float* rho,
+                              int rank, void* G_hat, gift_dtype out_dt, gift_stream_t stream) {
+  gift_status st =
+      check_nvfp4_args(G_hat, out_dt, d_out, d_in, U, lambda, rho, rank, codes, block_scales, tensor_scale);
+  if (st != GIFT_OK || d_out == 0) return st;
+  if ((st = device_ok()) != GIFT_OK) return st;
+  if (rank > 0 && !tc_codec_available()) return GIFT_ERR_UNSUPPORTED;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (rank == 0)
+    return cuda_status(launch_nvfp4_decode(codes, block_scales, tensor_scale, d_out * (d_in / GIFT_NVFP4_BLOCK),
+                                           G_hat, out_dt, s));
+  TcLayer L{nullptr, G_hat, (uint8_t*)codes, nullptr, U, lambda, rho, (int)d_out, (int)d_in, rank};
+  L.block_scales = (uint8_t*)block_scales;
+  L.tensor_scale = (float*)tensor_scale;
+  L.fmt = kFmtNvfp4;
+  return cuda_status(launch_whiten_decode_tc(&L, 1, s));
+}
+
 }  // extern "C"

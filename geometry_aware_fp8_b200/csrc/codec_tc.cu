@@ -67,13 +67,15 @@ constexpr int kMaxPanels = 1536;
 struct alignas(64) EncJob {
   CUtensorMap tmG;  // bf16 [d_out][d_in], box [128][64], 128-byte swizzle
   CUtensorMap tmU;  // fp32 U [d_in][32], box [128][32], 128-byte swizzle
-  CUtensorMap tmC;  // uint8 codes [d_out][d_in], box [128][128], 128-byte swizzle (stores)
+  CUtensorMap tmC;  // uint8 codes [d_out][d_in], box [128][128], 128-byte swizzle (E4M3 stores)
   const float* U;
   const float* lambda;
   const float* rho;
-  uint8_t* codes;
-  float* scales;
-  int d_out, d_in, rank, pad;
+  uint8_t* codes;   // E4M3 [d_out][d_in], or NVFP4 [d_out][d_in/2]
+  float* scales;    // E4M3 fp32 [d_out][d_in/128]
+  uint8_t* sb;      // NVFP4 E4M3 block scales [d_out][d_in/16]
+  float* tscale;    // NVFP4 tensor scale (amax bits while encoding)
+  int d_out, d_in, rank, fmt;
 };
 
 struct EncParams {
@@ -226,6 +228,7 @@ GIFT_DEV void convert_u_row_inplace(uint32_t tile, int t) {
     st_shared_v4(tile + sw128(t, 4 + q), lo[4 * q], lo[4 * q + 1], lo[4 * q + 2], lo[4 * q + 3]);
 }
 
+template <int FMT>
 __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __grid_constant__ EncParams p,
                                                                      uint32_t* err) {
   extern __shared__ uint8_t smem_raw[];
@@ -322,9 +325,11 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
           break;
         }
         const EncJob& J = p.jobs[st.job()];
-        tma_store_2d_hint(&J.tmC, cbuf + cb * kCodesBytes, st.chunk() * kChunk, st.panel() * kPanel, drop);
-        bulk_commit();
-        bulk_wait_read<0>();
+        if (FMT == kFmtE4M3) {  // NVFP4 codes leave from the epilogue
+          tma_store_2d_hint(&J.tmC, cbuf + cb * kCodesBytes, st.chunk() * kChunk, st.panel() * kPanel, drop);
+          bulk_commit();
+          bulk_wait_read<0>();
+        }
         mbar_arrive(&cfree[cb]);
         ++e2;
       }
@@ -414,12 +419,15 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     uint32_t e2 = 0;
     float a = 0.0f;
+    float S_t = 0.0f;   // NVFP4 tensor scale (codes pass)
+    float pmax = 0.0f;  // NVFP4 amax pass: this thread's max |W'| over the panel
     bool stop = false;  // group vote: set for all 256 threads at the same barrier
     for (Steps<EncParams> st(p, beg, end); st.valid() && !stop; st.next()) {
       if (st.pass == 0) continue;  // first-pass steps are the MMA's alone
       const EncJob& J = p.jobs[st.job()];
       const int panel = st.panel();
       if (st.i2 == 0) {
+        if (FMT == kFmtNvfp4) S_t = nvfp4_tensor_scale(__uint_as_float(*reinterpret_cast<volatile uint32_t*>(J.tscale)));
         // P o (c / a) of this panel for k = 16 h .. 16 h + 15, split into the bf16
         // A operand of E2:  c_k / a = (rho / (lambda_k + rho))^{1/2} - 1
         const double rho = (double)__ldg(J.rho);
@@ -485,6 +493,32 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
         m3 = fmaxf(m3, fabsf(__uint_as_float(w[k + 3])));
       }
       amax_x[h][r] = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+      if (FMT == kFmtNvfp4Amax) {
+        // amax(W) = a max|W'| (rounded once); one atomic per warp at the panel's end
+        pmax = fmaxf(pmax, live ? amax_x[h][r] : 0.0f);
+        if (st.i2 == st.nc() - 1) {
+          const float wm = warp_max(pmax);
+          if (lane == 0 && wm > 0.0f) atomicMax(reinterpret_cast<uint32_t*>(J.tscale), __float_as_uint(__fmul_rn(a, wm)));
+          pmax = 0.0f;
+        }
+      } else if (FMT == kFmtNvfp4 && live) {
+        // four NVFP4 blocks of 16 from W = a W'
+        uint2 c4[4];
+        uint32_t sbw = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          float v[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[i] = __fmul_rn(a, __uint_as_float(w[16 * j + i]));
+          uint8_t sbj;
+          c4[j] = nvfp4_block16(v, S_t, &sbj);
+          sbw |= (uint32_t)sbj << (8 * j);
+        }
+        uint4* cd = reinterpret_cast<uint4*>(J.codes + row * (J.d_in / 2) + st.chunk() * 64 + 32 * h);
+        cd[0] = make_uint4(c4[0].x, c4[0].y, c4[1].x, c4[1].y);
+        cd[1] = make_uint4(c4[2].x, c4[2].y, c4[3].x, c4[3].y);
+        *reinterpret_cast<uint32_t*>(J.sb + row * (J.d_in / 16) + st.chunk() * 8 + 4 * h) = sbw;
+      }
       // the codes tile is free once the store of its previous use has read it;
       // this barrier also exchanges the halves' maxima
       const int cb = e2 & 1;
@@ -507,7 +541,7 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
                                              __fmul_rn(__uint_as_float(w[4 * q + 3]), ai));
         cw[q] = inv > 0.0f ? (c01 | (c23 << 16)) : 0u;
       }
-      if (live && h == 0) J.scales[row * (J.d_in / kChunk) + c] = e4m3_scale(amax, inv);
+      if (FMT == kFmtE4M3 && live && h == 0) J.scales[row * (J.d_in / kChunk) + c] = e4m3_scale(amax, inv);
       const uint32_t c_tile = cbuf + cb * kCodesBytes;
 #pragma unroll
       for (int q = 0; q < 4; ++q)
@@ -551,8 +585,11 @@ struct alignas(64) DecJob {
   const float* U;
   const float* lambda;
   const float* rho;
-  const float* scales;
-  int d_out, d_in, rank, pad;
+  const float* scales;    // E4M3 fp32 [d_out][d_in/128]
+  const uint8_t* codes;   // NVFP4 [d_out][d_in/2] (read directly; E4M3 codes arrive by TMA)
+  const uint8_t* sb;      // NVFP4 E4M3 block scales [d_out][d_in/16]
+  const float* tscale;    // NVFP4 tensor scale
+  int d_out, d_in, rank, fmt;
 };
 
 struct DecParams {
@@ -568,6 +605,7 @@ GIFT_DEV uint32_t e4m3x2_to_bf16x2(uint16_t v) {
   return pack_bf16x2(f.x, f.y);
 }
 
+template <int FMT>
 __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __grid_constant__ DecParams p,
                                                                      uint32_t* err) {
   extern __shared__ uint8_t smem_raw[];
@@ -629,9 +667,13 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
         }
         const DecJob& J = p.jobs[st.job()];
         const uint32_t dst = sbase + s * kDStageBytes;
-        mbar_arrive_expect_tx(&cfull[s], kDCodes + kUBytes);
-        tma_load_2d_hint(dst, &J.tmC, &cfull[s], st.chunk() * kChunk, st.panel() * kPanel,
-                         st.pass == 0 ? keep : drop);
+        if (FMT == kFmtE4M3) {
+          mbar_arrive_expect_tx(&cfull[s], kDCodes + kUBytes);
+          tma_load_2d_hint(dst, &J.tmC, &cfull[s], st.chunk() * kChunk, st.panel() * kPanel,
+                           st.pass == 0 ? keep : drop);
+        } else {
+          mbar_arrive_expect_tx(&cfull[s], kUBytes);  // NVFP4 codes are read by the converters
+        }
         tma_load_2d_hint(dst + kDCodes + kDQ, &J.tmU, &cfull[s], 0, st.chunk() * kChunk, keep);
       }
     }
@@ -673,7 +715,33 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
       const uint32_t c_tile = sbase + s * kDStageBytes;
       const uint32_t q_tile = c_tile + kDCodes;
       convert_u_row_inplace(q_tile + kDQ, t);
-      if (st.pass == 0) {
+      const DecJob& J = p.jobs[st.job()];
+      if (st.pass == 0 && FMT != kFmtE4M3) {
+        // NVFP4: row t's 128 codes (64 bytes) and 8 block scales from global,
+        // widened to bf16 value(code) x value(scale) (exact)
+        const int64_t row = (int64_t)st.panel() * kPanel + t;
+        uint4 cw[4] = {};
+        uint2 sw = make_uint2(0u, 0u);
+        if (row < J.d_out) {
+          const uint4* src = reinterpret_cast<const uint4*>(J.codes + row * (J.d_in / 2) + st.chunk() * 64);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) cw[q] = __ldg(src + q);
+          sw = __ldg(reinterpret_cast<const uint2*>(J.sb + row * (J.d_in / 16) + st.chunk() * 8));
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {  // block j = columns 16 j .. 16 j + 15
+          const uint4& c = cw[j >> 1];
+          const uint2 cb = (j & 1) ? make_uint2(c.z, c.w) : make_uint2(c.x, c.y);
+          float v[16];
+          nvfp4_block16_values(cb, (uint8_t)(((j < 4) ? sw.x : sw.y) >> (8 * (j & 3))), v);
+          uint32_t o[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) o[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+          const int c0 = 2 * j, c1 = 2 * j + 1;  // 16-byte chunks of the 256-byte bf16 row
+          st_shared_v4(q_tile + (c0 >> 3) * kGHalf + sw128(t, c0 & 7), o[0], o[1], o[2], o[3]);
+          st_shared_v4(q_tile + (c1 >> 3) * kGHalf + sw128(t, c1 & 7), o[4], o[5], o[6], o[7]);
+        }
+      } else if (st.pass == 0) {
         // the codes of row t, widened to bf16
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
@@ -764,7 +832,9 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
       const int nc = st.nc(), c = st.chunk();
       const int64_t row = (int64_t)st.panel() * kPanel + r;
       const bool live = row < J.d_out;
-      const float sc = live ? __ldg(J.scales + row * nc + c) : 0.0f;
+      // E4M3: the chunk's fp32 block scale; NVFP4: the tensor scale (the block
+      // scales are inside the widened values)
+      const float sc = !live ? 0.0f : (FMT == kFmtE4M3 ? __ldg(J.scales + row * nc + c) : __ldg(J.tscale));
       if (st.block_start() && st.k >= 1) {
         // P of p_{k-1} is complete: P o c -> bf16 hi/lo A operand of D3
         // (this half's 16 of the 32 columns of each part)
@@ -835,20 +905,37 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
           tmem_wait_ld();
           // codes 64 h + 32 g2 .. + 31 of this row: two 16-byte chunks
           uint32_t o[16];
+          if (FMT == kFmtE4M3) {
 #pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            const uint4 v = ld_shared_v4(c_tile + sw128(r, 4 * h + 2 * g2 + hh));
-            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+            for (int hh = 0; hh < 2; ++hh) {
+              const uint4 v = ld_shared_v4(c_tile + sw128(r, 4 * h + 2 * g2 + hh));
+              const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float2 f0 = e4m3x2_to_f32x2((uint16_t)(w[e] & 0xFFFFu));
-              const float2 f1 = e4m3x2_to_f32x2((uint16_t)(w[e] >> 16));
-              const int k = hh * 16 + e * 4;
-              o[hh * 8 + 2 * e] = pack_bf16x2(fmaf(as, f0.x, __uint_as_float(acc[k])),
-                                              fmaf(as, f0.y, __uint_as_float(acc[k + 1])));
-              o[hh * 8 + 2 * e + 1] = pack_bf16x2(fmaf(as, f1.x, __uint_as_float(acc[k + 2])),
-                                                  fmaf(as, f1.y, __uint_as_float(acc[k + 3])));
+              for (int e = 0; e < 4; ++e) {
+                const float2 f0 = e4m3x2_to_f32x2((uint16_t)(w[e] & 0xFFFFu));
+                const float2 f1 = e4m3x2_to_f32x2((uint16_t)(w[e] >> 16));
+                const int k = hh * 16 + e * 4;
+                o[hh * 8 + 2 * e] = pack_bf16x2(fmaf(as, f0.x, __uint_as_float(acc[k])),
+                                                fmaf(as, f0.y, __uint_as_float(acc[k + 1])));
+                o[hh * 8 + 2 * e + 1] = pack_bf16x2(fmaf(as, f1.x, __uint_as_float(acc[k + 2])),
+                                                    fmaf(as, f1.y, __uint_as_float(acc[k + 3])));
+              }
             }
+          } else {
+            // NVFP4: columns 64 h + 32 g2 .. + 31 are blocks 4 h + 2 g2 and the next
+            uint4 cq = make_uint4(0u, 0u, 0u, 0u);
+            uint32_t sq = 0;
+            if (live) {
+              cq = __ldg(reinterpret_cast<const uint4*>(J.codes + row * (J.d_in / 2) + c * 64 + 32 * h + 16 * g2));
+              sq = __ldg(reinterpret_cast<const uint16_t*>(J.sb + row * (J.d_in / 16) + c * 8 + 4 * h + 2 * g2));
+            }
+            float qv[32];
+            nvfp4_block16_values(make_uint2(cq.x, cq.y), (uint8_t)(sq & 0xFFu), qv);
+            nvfp4_block16_values(make_uint2(cq.z, cq.w), (uint8_t)(sq >> 8), qv + 16);
+#pragma unroll
+            for (int k = 0; k < 16; ++k)
+              o[k] = pack_bf16x2(fmaf(as, qv[2 * k], __uint_as_float(acc[2 * k])),
+                                 fmaf(as, qv[2 * k + 1], __uint_as_float(acc[2 * k + 1])));
           }
 #pragma unroll
           for (int q = 0; q < 4; ++q)
@@ -869,8 +956,49 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
   if (threadIdx.x == 0 && failed && err) atomicOr(err, GIFT_DEV_TIMEOUT);
 }
 
-unsigned long long g_dec_attr = 0;
-unsigned long long g_enc_attr = 0;
+unsigned long long g_dec_attr[3] = {0, 0, 0};
+unsigned long long g_enc_attr[3] = {0, 0, 0};
+
+// One launch runs layers of one format (its kernel instantiation).
+cudaError_t enc_launch(int fmt, int grid, const EncParams& P, cudaStream_t s) {
+  cudaError_t e;
+  switch (fmt) {
+    case kFmtE4M3:
+      if ((e = ensure_smem_attr(whiten_encode_tc_kernel<kFmtE4M3>, kSmemBytes, &g_enc_attr[0])) != cudaSuccess) return e;
+      whiten_encode_tc_kernel<kFmtE4M3><<<grid, kThreads, kSmemBytes, s>>>(P, nullptr);
+      break;
+    case kFmtNvfp4Amax:
+      if ((e = ensure_smem_attr(whiten_encode_tc_kernel<kFmtNvfp4Amax>, kSmemBytes, &g_enc_attr[1])) != cudaSuccess)
+        return e;
+      whiten_encode_tc_kernel<kFmtNvfp4Amax><<<grid, kThreads, kSmemBytes, s>>>(P, nullptr);
+      break;
+    case kFmtNvfp4:
+      if ((e = ensure_smem_attr(whiten_encode_tc_kernel<kFmtNvfp4>, kSmemBytes, &g_enc_attr[2])) != cudaSuccess) return e;
+      whiten_encode_tc_kernel<kFmtNvfp4><<<grid, kThreads, kSmemBytes, s>>>(P, nullptr);
+      break;
+    default:
+      return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t dec_launch(int fmt, int grid, const DecParams& P, cudaStream_t s) {
+  cudaError_t e;
+  switch (fmt) {
+    case kFmtE4M3:
+      if ((e = ensure_smem_attr(whiten_decode_tc_kernel<kFmtE4M3>, kDSmemBytes, &g_dec_attr[0])) != cudaSuccess) return e;
+      whiten_decode_tc_kernel<kFmtE4M3><<<grid, kThreads, kDSmemBytes, s>>>(P, nullptr);
+      break;
+    case kFmtNvfp4:
+      if ((e = ensure_smem_attr(whiten_decode_tc_kernel<kFmtNvfp4>, kDSmemBytes, &g_dec_attr[2])) != cudaSuccess)
+        return e;
+      whiten_decode_tc_kernel<kFmtNvfp4><<<grid, kThreads, kDSmemBytes, s>>>(P, nullptr);
+      break;
+    default:
+      return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
 
 // Longest-processing-time-first assignment of panels to CTAs.
 int schedule(const TcLayer* layers, int n, uint16_t* off, uint16_t* ids, int max_ids) {
@@ -910,12 +1038,11 @@ int schedule(const TcLayer* layers, int n, uint16_t* off, uint16_t* ids, int max
 bool tc_codec_available() { return tmap_encoder() != nullptr; }
 
 cudaError_t launch_whiten_encode_tc(const TcLayer* layers, int n, cudaStream_t s) {
-  cudaError_t e = ensure_smem_attr(whiten_encode_tc_kernel, kSmemBytes, &g_enc_attr);
-  if (e != cudaSuccess) return e;
+  cudaError_t e = cudaSuccess;
   for (int base = 0; base < n;) {
     // pack as many layers as fit one launch
     int cnt = 0, panels = 0;
-    while (base + cnt < n && cnt < kMaxJobs) {
+    while (base + cnt < n && cnt < kMaxJobs && layers[base + cnt].fmt == layers[base].fmt) {
       const int np = (layers[base + cnt].d_out + kPanel - 1) / kPanel;
       if (np > 256 || panels + np > kMaxPanels) break;
       panels += np;
@@ -929,8 +1056,13 @@ cudaError_t launch_whiten_encode_tc(const TcLayer* layers, int n, cudaStream_t s
         TcLayer part = L;
         part.d_out = std::min(rows, L.d_out - r0);
         part.G = (const __nv_bfloat16*)L.G + (int64_t)r0 * L.d_in;
-        part.codes = L.codes + (int64_t)r0 * L.d_in;
-        part.scales = L.scales + (int64_t)r0 * (L.d_in / kChunk);
+        if (L.fmt == kFmtE4M3) {
+          part.codes = L.codes + (int64_t)r0 * L.d_in;
+          part.scales = L.scales + (int64_t)r0 * (L.d_in / kChunk);
+        } else {
+          part.codes = L.codes + (int64_t)r0 * (L.d_in / 2);
+          part.block_scales = L.block_scales + (int64_t)r0 * (L.d_in / 16);
+        }
         if ((e = launch_whiten_encode_tc(&part, 1, s)) != cudaSuccess) return e;
       }
       ++base;
@@ -943,13 +1075,16 @@ cudaError_t launch_whiten_encode_tc(const TcLayer* layers, int n, cudaStream_t s
       if (!make_tmap_2d(&J.tmG, L.G, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)L.d_out, (uint64_t)L.d_in,
                         kPanel, 64) ||
           !make_tmap_2d(&J.tmU, L.U, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, (uint64_t)L.d_in, 32, kChunk, 32) ||
-          !make_tmap_2d(&J.tmC, L.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)L.d_out, (uint64_t)L.d_in,
-                        kPanel, kChunk))
+          (L.fmt == kFmtE4M3 && !make_tmap_2d(&J.tmC, L.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)L.d_out,
+                                              (uint64_t)L.d_in, kPanel, kChunk)))
         return cudaErrorInvalidValue;
       J.U = L.U;
       J.lambda = L.lambda;
       J.rho = L.rho;
       J.codes = L.codes;
+      J.sb = L.block_scales;
+      J.tscale = L.tensor_scale;
+      J.fmt = L.fmt;
       J.scales = L.scales;
       J.d_out = L.d_out;
       J.d_in = L.d_in;
@@ -957,8 +1092,7 @@ cudaError_t launch_whiten_encode_tc(const TcLayer* layers, int n, cudaStream_t s
     }
     const int grid = schedule(layers + base, cnt, P.sched_off, P.sched_ids, kMaxPanels);
     if (grid <= 0) return cudaErrorInvalidValue;
-    whiten_encode_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(P, nullptr);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = enc_launch(layers[base].fmt, grid, P, s)) != cudaSuccess) return e;
     base += cnt;
   }
   return cudaSuccess;
@@ -967,11 +1101,10 @@ cudaError_t launch_whiten_encode_tc(const TcLayer* layers, int n, cudaStream_t s
 
 
 cudaError_t launch_whiten_decode_tc(const TcLayer* layers, int n, cudaStream_t s) {
-  cudaError_t e = ensure_smem_attr(whiten_decode_tc_kernel, kDSmemBytes, &g_dec_attr);
-  if (e != cudaSuccess) return e;
+  cudaError_t e = cudaSuccess;
   for (int base = 0; base < n;) {
     int cnt = 0, panels = 0;
-    while (base + cnt < n && cnt < kMaxJobs) {
+    while (base + cnt < n && cnt < kMaxJobs && layers[base + cnt].fmt == layers[base].fmt) {
       const int np = (layers[base + cnt].d_out + kPanel - 1) / kPanel;
       if (np > 256 || panels + np > kMaxPanels) break;
       panels += np;
@@ -984,8 +1117,13 @@ cudaError_t launch_whiten_decode_tc(const TcLayer* layers, int n, cudaStream_t s
         TcLayer part = L;
         part.d_out = std::min(rows, L.d_out - r0);
         part.G_hat = (__nv_bfloat16*)L.G_hat + (int64_t)r0 * L.d_in;
-        part.codes = L.codes + (int64_t)r0 * L.d_in;
-        part.scales = L.scales + (int64_t)r0 * (L.d_in / kChunk);
+        if (L.fmt == kFmtE4M3) {
+          part.codes = L.codes + (int64_t)r0 * L.d_in;
+          part.scales = L.scales + (int64_t)r0 * (L.d_in / kChunk);
+        } else {
+          part.codes = L.codes + (int64_t)r0 * (L.d_in / 2);
+          part.block_scales = L.block_scales + (int64_t)r0 * (L.d_in / 16);
+        }
         if ((e = launch_whiten_decode_tc(&part, 1, s)) != cudaSuccess) return e;
       }
       ++base;
@@ -995,8 +1133,8 @@ cudaError_t launch_whiten_decode_tc(const TcLayer* layers, int n, cudaStream_t s
     for (int l = 0; l < cnt; ++l) {
       const TcLayer& L = layers[base + l];
       DecJob& J = P.jobs[l];
-      if (!make_tmap_2d(&J.tmC, L.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)L.d_out, (uint64_t)L.d_in,
-                        kPanel, kChunk) ||
+      if ((L.fmt == kFmtE4M3 && !make_tmap_2d(&J.tmC, L.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)L.d_out,
+                                              (uint64_t)L.d_in, kPanel, kChunk)) ||
           !make_tmap_2d(&J.tmU, L.U, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, (uint64_t)L.d_in, 32, kChunk, 32) ||
           !make_tmap_2d(&J.tmO, L.G_hat, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)L.d_out, (uint64_t)L.d_in,
                         kPanel, 64))
@@ -1005,14 +1143,17 @@ cudaError_t launch_whiten_decode_tc(const TcLayer* layers, int n, cudaStream_t s
       J.lambda = L.lambda;
       J.rho = L.rho;
       J.scales = L.scales;
+      J.codes = L.codes;
+      J.sb = L.block_scales;
+      J.tscale = L.tensor_scale;
+      J.fmt = L.fmt;
       J.d_out = L.d_out;
       J.d_in = L.d_in;
       J.rank = L.rank;
     }
     const int grid = schedule(layers + base, cnt, P.sched_off, P.sched_ids, kMaxPanels);
     if (grid <= 0) return cudaErrorInvalidValue;
-    whiten_decode_tc_kernel<<<grid, kThreads, kDSmemBytes, s>>>(P, nullptr);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = dec_launch(layers[base].fmt, grid, P, s)) != cudaSuccess) return e;
     base += cnt;
   }
   return cudaSuccess;

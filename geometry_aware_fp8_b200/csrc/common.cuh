@@ -75,6 +75,53 @@ GIFT_DEV float2 e2m1x2_to_f32x2(uint8_t v) {
 
 GIFT_DEV float e4m3_to_f32(uint8_t v) { return e4m3x2_to_f32x2((uint16_t)v).x; }
 
+// ---------------------------------------------------------------------------
+// NVFP4 block of 16 (abstract of the GIFT paper: NVFP4 as the second format),
+// decisions in fp32: tensor scale S_t = amax(W) / (6 * 448); the block's scale
+// code sb = E4M3(amax_b / fp32(6 S_t)) (IEEE division, RNE, saturating);
+// element codes E2M1(w * fp32(1 / fp32(value(sb) * S_t))).  A block whose
+// scale decodes to 0, or whose reciprocal overflows fp32, gets sb = 0 and all
+// codes 0.  Codes come back packed two per byte, element 2i in the low nibble.
+// ---------------------------------------------------------------------------
+constexpr float kNvfp4TensorDiv = 6.0f * 448.0f;
+
+GIFT_DEV float nvfp4_tensor_scale(float amax_t) { return __fdiv_rn(amax_t, kNvfp4TensorDiv); }
+
+GIFT_DEV uint2 nvfp4_block16(const float* w, float S_t, uint8_t* sb_out) {
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(w[i]));
+  const float denom = __fmul_rn(6.0f, S_t);
+  const float ratio = denom > 0.0f ? __fdiv_rn(amax, denom) : 0.0f;
+  uint8_t sb = (uint8_t)(f32x2_to_e4m3x2(ratio, 0.0f) & 0xFFu);
+  const float dq = __fmul_rn(e4m3_to_f32(sb), S_t);
+  const float inv = dq > 0.0f ? __frcp_rn(dq) : 0.0f;
+  const bool live = dq > 0.0f && !isinf(inv);
+  uint32_t c[2] = {0u, 0u};
+  if (live) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      c[i >> 2] |= (uint32_t)f32x2_to_e2m1x2(__fmul_rn(w[2 * i], inv), __fmul_rn(w[2 * i + 1], inv)) << (8 * (i & 3));
+  } else {
+    sb = 0;
+  }
+  *sb_out = sb;
+  return make_uint2(c[0], c[1]);
+}
+
+// The 16 values of an NVFP4 block divided by S_t: value(code) * value(sb), exact
+// (E2M1 x E4M3 has at most 6 significant bits).
+GIFT_DEV void nvfp4_block16_values(uint2 codes, uint8_t sb, float* v) {
+  const float s = e4m3_to_f32(sb);
+  const uint32_t c[2] = {codes.x, codes.y};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float2 f = e2m1x2_to_f32x2((uint8_t)(c[i >> 2] >> (8 * (i & 3))));
+    v[2 * i] = f.x * s;
+    v[2 * i + 1] = f.y * s;
+  }
+}
+
 // Reciprocal scale of one E4M3 block: 448/amax (IEEE fp32 division).  A block
 // whose amax is 0, or so small that 448/amax overflows fp32, is flushed:
 // the function returns 0, and the caller writes scale 0 and codes 0x00.

@@ -45,13 +45,29 @@ struct TcLayer {
   int d_out;
   int d_in;
   int rank;
+  // 0: E4M3 codes + fp32 scales per 128.  NVFP4 (codes two per byte, E4M3
+  // scales per 16 in block_scales, tensor scale in tensor_scale): encode pass 1
+  // folds amax(W) into tensor_scale's bits, encode pass 2 writes the codes,
+  // decode reads them.
+  int fmt = 0;
+  uint8_t* block_scales = nullptr;
+  float* tensor_scale = nullptr;
 };
+constexpr int kFmtE4M3 = 0, kFmtNvfp4Amax = 1, kFmtNvfp4 = 2;
 bool tc_codec_available();
 cudaError_t launch_whiten_encode_tc(const TcLayer* layers, int n, cudaStream_t s);
 cudaError_t launch_whiten_decode_tc(const TcLayer* layers, int n, cudaStream_t s);
 
 // ---- Round-trip error ----
 size_t error_ws_bytes(int64_t n_elems);
+// ---- NVFP4, Euclidean (M = I) ----
+cudaError_t launch_nvfp4_amax(const void* G, gift_dtype dt, int64_t n_blocks, float* tensor_scale, cudaStream_t s);
+cudaError_t launch_nvfp4_quant(const void* G, gift_dtype dt, int64_t n_blocks, const float* tensor_scale,
+                               uint8_t* codes, uint8_t* sb, cudaStream_t s);
+cudaError_t launch_nvfp4_finalize(float* tensor_scale, cudaStream_t s);
+cudaError_t launch_nvfp4_decode(const uint8_t* codes, const uint8_t* sb, const float* tensor_scale, int64_t n_blocks,
+                                void* out, gift_dtype dt, cudaStream_t s);
+
 cudaError_t launch_roundtrip_error(const void* G, const void* G_hat, gift_dtype dt, int64_t n_elems,
                                    double* out, void* ws, cudaStream_t s);
 

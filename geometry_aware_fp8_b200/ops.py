@@ -26,7 +26,7 @@ STATUS = {0: "GIFT_OK", 1: "GIFT_ERR_INVALID_ARG", 2: "GIFT_ERR_SHAPE", 3: "GIFT
 
 EXPORTED = ("gift_status_string", "gift_version", "gift_refresh_workspace_size", "gift_factor_refresh",
             "gift_factor_refresh_noalloc", "gift_factor_refresh_many", "gift_encode", "gift_decode", "gift_encode_many", "gift_decode_many",
-            "gift_error_workspace_size", "gift_roundtrip_error")
+            "gift_error_workspace_size", "gift_roundtrip_error", "gift_encode_nvfp4", "gift_decode_nvfp4")
 
 
 class GiftError(RuntimeError):
@@ -79,6 +79,8 @@ def lib() -> ctypes.CDLL:
         L.gift_decode_many.argtypes = [ctypes.POINTER(Layer), i32, vp]
         L.gift_error_workspace_size.argtypes = [i64, i64, ctypes.POINTER(sz)]
         L.gift_roundtrip_error.argtypes = [vp, vp, i32, i64, i64, vp, vp, sz, vp]
+        L.gift_encode_nvfp4.argtypes = [vp, i32, i64, i64, vp, vp, vp, i32, vp, vp, vp, vp]
+        L.gift_decode_nvfp4.argtypes = [vp, vp, vp, i64, i64, vp, vp, vp, i32, vp, i32, vp]
         for name in EXPORTED:
             if name not in ("gift_status_string", "gift_version"):
                 getattr(L, name).restype = i32
@@ -222,6 +224,45 @@ def decode(codes: torch.Tensor, scales: torch.Tensor, U=None, lam=None, rho=None
         out = torch.empty((d_out, d_in), device=codes.device, dtype=out_dtype)
     _check(lib().gift_decode(_ptr(codes), _ptr(scales), d_out, d_in, _ptr(U), _ptr(lam), _ptr(rho), rank,
                              _ptr(out), _dt(out), _stream(stream)), "gift_decode")
+    return out
+
+
+NVFP4_BLOCK = 16
+
+
+def encode_nvfp4(G: torch.Tensor, U=None, lam=None, rho=None, rank: Optional[int] = None,
+                 codes: Optional[torch.Tensor] = None, block_scales: Optional[torch.Tensor] = None,
+                 tensor_scale: Optional[torch.Tensor] = None, stream=None):
+    """(codes uint8 [d_out, d_in/2], block scales uint8 [d_out, d_in/16], tensor scale fp32 [1])."""
+    _cuda(G, U, lam, rho, codes, block_scales, tensor_scale)
+    d_out, d_in = G.shape
+    if rank is None:
+        rank = 0 if U is None else U.shape[1]
+    if codes is None:
+        codes = torch.empty((d_out, d_in // 2), device=G.device, dtype=torch.uint8)
+    if block_scales is None:
+        block_scales = torch.empty((d_out, max(d_in // NVFP4_BLOCK, 1)), device=G.device, dtype=torch.uint8)
+    if tensor_scale is None:
+        tensor_scale = torch.empty((1,), device=G.device, dtype=torch.float32)
+    _check(lib().gift_encode_nvfp4(_ptr(G), _dt(G), d_out, d_in, _ptr(U), _ptr(lam), _ptr(rho), rank,
+                                   _ptr(codes), _ptr(block_scales), _ptr(tensor_scale), _stream(stream)),
+           "gift_encode_nvfp4")
+    return codes, block_scales, tensor_scale
+
+
+def decode_nvfp4(codes: torch.Tensor, block_scales: torch.Tensor, tensor_scale: torch.Tensor, U=None, lam=None,
+                 rho=None, rank: Optional[int] = None, out_dtype=torch.bfloat16, out: Optional[torch.Tensor] = None,
+                 stream=None):
+    """G_hat [d_out, d_in] in out_dtype from NVFP4 codes."""
+    _cuda(codes, block_scales, tensor_scale, U, lam, rho, out)
+    d_out, d_in = codes.shape[0], codes.shape[1] * 2
+    if rank is None:
+        rank = 0 if U is None else U.shape[1]
+    if out is None:
+        out = torch.empty((d_out, d_in), device=codes.device, dtype=out_dtype)
+    _check(lib().gift_decode_nvfp4(_ptr(codes), _ptr(block_scales), _ptr(tensor_scale), d_out, d_in, _ptr(U),
+                                   _ptr(lam), _ptr(rho), rank, _ptr(out), _dt(out), _stream(stream)),
+           "gift_decode_nvfp4")
     return out
 
 

@@ -223,6 +223,40 @@ gift_status gift_roundtrip_error(const void* G, const void* G_hat, gift_dtype dt
                                  int64_t d_in, double* out, void* ws, size_t ws_bytes,
                                  gift_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * NVFP4 codec (abstract: NVFP4 is the second low-precision format the
+ * whitening is applied to).  The pages give no recipe; this library uses the
+ * two-level one of the NVFP4 format, decisions in fp32:
+ *
+ *   W = G (rank 0) or G M (rank 32);  S_t = amax(W) / (6 * 448);
+ *   per row and block b of 16 columns:  amax_b = max |W|,
+ *   block_scales[b] = E4M3_RNE_satfinite(amax_b / (6 S_t));
+ *   codes = E2M1_RNE_satfinite(W * (1 / (value(block_scales[b]) * S_t)))
+ *   (a block whose scale decodes to 0, or whose reciprocal overflows fp32,
+ *   gets scale code 0 and all-zero codes).
+ *
+ * codes: d_out x d_in/2 bytes, two E2M1 codes per byte, column 2i in the low
+ * nibble, 16-byte aligned.  block_scales: d_out x d_in/16 E4M3 bytes, 8-byte
+ * aligned.  tensor_scale: one fp32 in device memory, 4-byte aligned.
+ * Encode needs the tensor-wide maximum before any block is coded, so it
+ * makes two passes over W (the first folds amax(W) into *tensor_scale, the
+ * second writes the codes, then *tensor_scale becomes S_t); *tensor_scale
+ * holds intermediate values while the call's work runs.
+ * rank must be 0 (any dtype, d_in % 16 == 0) or 32 with bf16 G / G_hat and
+ * d_in % 128 == 0, d_in <= 8192 (tensor-core path); other ranks return
+ * GIFT_ERR_UNSUPPORTED.  G / G_hat and U 16-byte aligned.
+ * Decode: G_hat = W_hat (rank 0) or W_hat M^{-1} with
+ * W_hat = value(code) * value(block scale) * S_t.
+ * ------------------------------------------------------------------------ */
+gift_status gift_encode_nvfp4(const void* G, gift_dtype gdt, int64_t d_out, int64_t d_in, const float* U,
+                              const float* lambda, const float* rho, int rank, uint8_t* codes,
+                              uint8_t* block_scales, float* tensor_scale, gift_stream_t stream);
+
+gift_status gift_decode_nvfp4(const uint8_t* codes, const uint8_t* block_scales, const float* tensor_scale,
+                              int64_t d_out, int64_t d_in, const float* U, const float* lambda,
+                              const float* rho, int rank, void* G_hat, gift_dtype out_dt,
+                              gift_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

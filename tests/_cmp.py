@@ -10,6 +10,13 @@ Match criteria for the codec (written here once, used by every parity test):
   * G_hat (decoder fed the oracle's codes): fp32 output within 1e-3 of the
     oracle relative to the row's largest magnitude; bf16 output within one
     bf16 rounding (2^-8 relative) of the same reference plus that 1e-3.
+  * NVFP4, Euclidean: every decision is taken in fp32 on exact inputs, so the
+    tensor scale, block scales and codes are bit-exact (+0 / -0 the same).
+  * NVFP4, whitened: W comes from the tensor cores (different summation
+    order), so the tensor scale is within 1e-5 relative; block scale codes are
+    exact on >= 99.9 % of blocks and one E4M3 step away elsewhere; inside
+    blocks whose scale codes agree, E2M1 codes are exact on >= 99.9 % and one
+    step away elsewhere.
 """
 import numpy as np
 
@@ -55,3 +62,37 @@ def check_rows(got, want, rtol=GHAT_RTOL, bf16=False):
         tol = tol + 2.0 ** -8 * np.abs(want)
     bad = np.abs(got - want) > tol + 1e-30
     assert not bad.any(), f"{bad.sum()} elements off; worst {(np.abs(got - want) / np.maximum(rowmax, 1e-30)).max()}"
+
+
+def e2m1_position(codes):
+    c = np.asarray(codes, dtype=np.int64) & 0xF
+    mag = c & 0x7
+    return np.where(c & 0x8, -mag, mag)
+
+
+def unpack_nibbles(packed):
+    p = np.asarray(packed, dtype=np.uint8)
+    q = np.empty((p.shape[0], p.shape[1] * 2), dtype=np.uint8)
+    q[:, 0::2] = p & 0xF
+    q[:, 1::2] = p >> 4
+    return q
+
+
+def check_nvfp4(got, want, exact=False, frac=CODE_EXACT_FRAC, st_rtol=1e-5):
+    """got / want: (packed codes, block scale codes, tensor scale)."""
+    (gc, gs, gt), (wc, ws, wt) = got, want
+    gt, wt = float(np.asarray(gt).reshape(-1)[0]), float(wt)
+    qg, qw = e2m1_position(unpack_nibbles(gc)), e2m1_position(unpack_nibbles(wc))
+    sg, sw = e4m3_position(gs), e4m3_position(ws)
+    if exact:
+        assert gt == wt, (gt, wt)
+        assert np.array_equal(sg, sw), f"{(sg != sw).sum()} block scales differ"
+        assert np.array_equal(qg, qw), f"{(qg != qw).sum()} codes differ"
+        return
+    assert abs(gt - wt) <= st_rtol * abs(wt), (gt, wt)
+    ds = np.abs(sg - sw)
+    assert ds.max(initial=0) <= 1 and (ds == 0).mean() >= frac, f"block scales: {(ds != 0).sum()} differ"
+    same = np.repeat(ds == 0, 16, axis=1)
+    dq = np.abs(qg - qw)[same]
+    assert dq.max(initial=0) <= 1, f"max E2M1 code distance {dq.max()}"
+    assert (dq == 0).mean() >= frac if dq.size else True, f"code exact rate {(dq == 0).mean():.6f}"

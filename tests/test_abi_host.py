@@ -77,6 +77,30 @@ def test_decode_rejects_bad_arguments(L):
     assert L.gift_decode(A16, A16, 4, 128, None, None, None, 0, A_ODD, 1, s) == ALIGN
 
 
+def test_nvfp4_rejects_bad_arguments(L):
+    s = None
+    UNSUPPORTED = 6
+    enc, dec = L.gift_encode_nvfp4, L.gift_decode_nvfp4
+    # empty gradient: nothing is touched
+    assert enc(None, 1, 0, 128, None, None, None, 0, None, None, None, s) == OK
+    # null outputs
+    assert enc(A16, 1, 4, 128, None, None, None, 0, A16, A16, None, s) == INVALID
+    # Euclidean blocks of 16: d_in % 16; whitened: d_in % 128
+    assert enc(A16, 1, 4, 24, None, None, None, 0, A16, A16, A16, s) == SHAPE
+    assert enc(A16, 1, 4, 144, A16, A16, A16, 32, A16, A16, A16, s) == SHAPE
+    # whitened NVFP4 runs on the tensor cores only: rank 32, bf16
+    assert enc(A16, 1, 4, 128, A16, A16, A16, 7, A16, A16, A16, s) == UNSUPPORTED
+    assert enc(A16, 0, 4, 128, A16, A16, A16, 32, A16, A16, A16, s) == UNSUPPORTED
+    assert enc(A16, 1, 4, 128, A16, A16, A16, 33, A16, A16, A16, s) == SHAPE
+    # alignment: codes 16 B, block scales 8 B, tensor scale 4 B
+    assert enc(A16, 1, 4, 128, None, None, None, 0, A_ODD, A16, A16, s) == ALIGN
+    assert enc(A16, 1, 4, 128, None, None, None, 0, A16, A16 + 4, A16, s) == ALIGN
+    assert enc(A16, 1, 4, 128, None, None, None, 0, A16, A16, A16 + 2, s) == ALIGN
+    assert dec(A16, A16, A16, 4, 128, None, None, None, 0, None, 1, s) == INVALID
+    assert dec(A16, A16, A16, 4, 128, None, None, None, 0, A16, 5, s) == INVALID
+    assert dec(A16, A16, A16, 4, 128, A16, A16, A16, 32, A16, 0, s) == UNSUPPORTED
+
+
 def test_refresh_rejects_bad_arguments(L):
     s = None
     n = ctypes.c_size_t(0)
