@@ -124,8 +124,10 @@ __global__ void __launch_bounds__(256) euclid_decode_kernel(const uint8_t* __res
 }
 
 // Grouped form: many layers in one launch.  A block index b of the
-// concatenated layers is mapped to its layer by a search over the prefix
-// sums of the layers' block counts (kept in shared memory).
+// concatenated layers is mapped to its layer through the prefix sums of the
+// layers' block counts (kept in shared memory): the encoder searches once per
+// thread and then advances (each thread's block index only grows), the
+// decoder searches per block pair (measured faster for it).
 constexpr int kGroupMax = 64;
 
 struct EuclidGroup {
@@ -144,6 +146,11 @@ GIFT_DEV int find_layer(const int64_t* pre, int n, int64_t b) {
   }
   return lo;
 }
+// the layer of block b, given the layer of an earlier block of this thread
+GIFT_DEV int advance_layer(const int64_t* pre, int n, int l, int64_t b) {
+  while (l + 1 < n && b >= pre[l + 1]) ++l;
+  return l;
+}
 
 // Two blocks per thread group per iteration: both blocks' loads are issued
 // before either is used, doubling the bytes in flight per thread.
@@ -155,11 +162,13 @@ __global__ void __launch_bounds__(256) euclid_encode_group_kernel(const __grid_c
   const int sub = threadIdx.x & 7;
   const int64_t total = pre[g.n];
   const int64_t G = (int64_t)gridDim.x * (blockDim.x >> 3);
-  for (int64_t b0 = (int64_t)blockIdx.x * (blockDim.x >> 3) + (threadIdx.x >> 3); b0 < total; b0 += 2 * G) {
+  const int64_t first = (int64_t)blockIdx.x * (blockDim.x >> 3) + (threadIdx.x >> 3);
+  int l0 = first < total ? find_layer(pre, g.n, first) : 0, l1 = l0;
+  for (int64_t b0 = first; b0 < total; b0 += 2 * G) {
     const int64_t b1 = b0 + G;
     const bool has1 = b1 < total;
-    const int l0 = find_layer(pre, g.n, b0);
-    const int l1 = has1 ? find_layer(pre, g.n, b1) : l0;
+    l0 = advance_layer(pre, g.n, l0, b0);
+    l1 = has1 ? advance_layer(pre, g.n, l1 > l0 ? l1 : l0, b1) : l0;
     const int64_t e0 = (b0 - pre[l0]) * kBlock + sub * 16;
     const int64_t e1 = has1 ? (b1 - pre[l1]) * kBlock + sub * 16 : e0;
     float v0[16], v1[16];
@@ -265,6 +274,23 @@ cudaError_t launch_euclid_decode(const uint8_t* codes, const float* scales, int6
   return cudaGetLastError();
 }
 
+// Grid of a grouped launch: as many CTAs as stay resident (one wave), found once
+// per kernel with the occupancy calculator.
+// slot: one cached count per kernel (the kernels share one pointer type).
+template <typename K>
+int group_grid(K kernel, int slot, int64_t n_blocks) {
+  static int resident[4] = {0, 0, 0, 0};
+  if (resident[slot] == 0) {
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, 256, 0) != cudaSuccess || per_sm < 1) per_sm = 4;
+    resident[slot] = per_sm * kNumSMs;
+  }
+  const int res = resident[slot];
+  int64_t need = (n_blocks + 31) / 32;
+  if (need < 1) need = 1;
+  return (int)(need < res ? need : res);
+}
+
 cudaError_t launch_euclid_group(const EuclidLayer* layers, int n, gift_dtype dt, bool encode, cudaStream_t s) {
   for (int base = 0; base < n; base += kGroupMax) {
     const int cnt = n - base < kGroupMax ? n - base : kGroupMax;
@@ -281,13 +307,22 @@ cudaError_t launch_euclid_group(const EuclidLayer* layers, int n, gift_dtype dt,
     }
     g.prefix[cnt] = tot;
     if (tot == 0) continue;
-    const int grid = grid_for(tot);
     if (encode) {
-      if (dt == GIFT_BF16) euclid_encode_group_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(g);
-      else euclid_encode_group_kernel<float><<<grid, 256, 0, s>>>(g);
+      if (dt == GIFT_BF16) {
+        auto k = euclid_encode_group_kernel<__nv_bfloat16>;
+        k<<<group_grid(k, 0, tot), 256, 0, s>>>(g);
+      } else {
+        auto k = euclid_encode_group_kernel<float>;
+        k<<<group_grid(k, 1, tot), 256, 0, s>>>(g);
+      }
     } else {
-      if (dt == GIFT_BF16) euclid_decode_group_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(g);
-      else euclid_decode_group_kernel<float><<<grid, 256, 0, s>>>(g);
+      if (dt == GIFT_BF16) {
+        auto k = euclid_decode_group_kernel<__nv_bfloat16>;
+        k<<<group_grid(k, 2, tot), 256, 0, s>>>(g);
+      } else {
+        auto k = euclid_decode_group_kernel<float>;
+        k<<<group_grid(k, 3, tot), 256, 0, s>>>(g);
+      }
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
