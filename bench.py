@@ -52,7 +52,7 @@ HBM_FALLBACK = 6650.0
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=K_REFRESH)
+    ap.add_argument("--steps", type=int, default=10 * K_REFRESH)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="gift", choices=["gift", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
@@ -90,8 +90,12 @@ class ClockSampler:
             os.close(fd)
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=self.f, stderr=subprocess.DEVNULL)
+            # the timed region starts once the sampler has written its first sample
+            t_end = time.time() + 3.0
+            while time.time() < t_end and os.path.getsize(self.path) == 0:
+                time.sleep(0.01)
         except Exception:
             self.proc = None
 
@@ -284,13 +288,13 @@ def step(ops, W, k, ev=None):
 # that figure x its elements.  Valid only for the kernel source it was taken
 # on (sha256 of the file); otherwise the bench reports traffic as null.
 TRAFFIC = {
-    "encode_whitened": {"bytes_per_element": 222.925312e6 / 69206016,
+    "encode_whitened": {"bytes_per_element": (201.38752e6 + 21.316352e6) / 69206016,
                         "profile": "profiles/whiten_encode_tc_stack8.md"},
-    "decode_whitened": {"bytes_per_element": 174.122752e6 / 69206016,
+    "decode_whitened": {"bytes_per_element": (97.158656e6 + 83.8272e6) / 69206016,
                         "profile": "profiles/whiten_decode_tc_stack8.md"},
 }
 TRAFFIC_SOURCE = ("geometry_aware_fp8_b200/csrc/codec_tc.cu",
-                  "4edd617c87fff8f3d1bf0028a359453eade8269c207088792592e9952795f009")
+                  "ccb4961a553802a9b90fdf98a127d2507b45044a055a60ded6ec50481cde3093")
 
 
 def traffic_for(phase, n_elements):
