@@ -197,63 +197,85 @@ __global__ void split_a_kernel(const __grid_constant__ RefBatch b) {
   }
 }
 
-// Y = A Q (d x d times d x m, m <= 64).  64 x 64 output tiles (columns >= m
-// idle), 4 x 4 outputs per thread from float4 shared-memory loads; the k
-// range is split into `ns` slices written to Yp[slice] (fp32, fixed order);
-// consumers add the slices in index order.
-constexpr int kSkK = 32;
+// Y = A Q (d x d times d x m, m <= 64), fp32 on the CUDA cores.  128 x 64
+// output tiles (columns >= m idle), 8 x 4 outputs per thread; the k range of a
+// CTA is walked in steps of 16 through two shared-memory buffers, the next
+// step's A and Q values prefetched into registers while the current one is
+// used.  Each output is one fmaf chain in increasing k over its slice; the k
+// range is split into `ns` slices written to Yp[slice] (fixed order), which
+// consumers add in index order.
+constexpr int kSkK = 32;   // k-slice granularity
+constexpr int kSkStep = 16;
 
 __global__ void __launch_bounds__(kRT) skinny_kernel(const __grid_constant__ RefBatch b, int src, int dst) {
   const RefLayer& Lr = b.L[blockIdx.z];
   const int d = Lr.d, m = b.m, kslice = Lr.kslice;
-  if ((int)blockIdx.x >= d / 64 || (int)blockIdx.y >= Lr.ns) return;
+  if ((int)blockIdx.x >= d / 128 || (int)blockIdx.y >= Lr.ns) return;
   const float* __restrict__ A = Lr.A;
   const float* __restrict__ Q = Lr.buf[src];
   float* __restrict__ Yp = Lr.buf[dst];
-  __shared__ __align__(16) float As[kSkK][64 + 4];  // As[k][row]
-  __shared__ __align__(16) float Qs[kSkK][64];
-  const int row0 = blockIdx.x * 64;
+  __shared__ __align__(16) float As[2][kSkStep][128 + 4];  // As[k][row]
+  __shared__ __align__(16) float Qs[2][kSkStep][64];
+  const int row0 = blockIdx.x * 128;
   const int k_begin = blockIdx.y * kslice;
   const int k_end = min(d, k_begin + kslice);
-  const int ti = threadIdx.x >> 4, tj = threadIdx.x & 15;
-  float acc[4][4];
+  const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;  // rows 8 ty.., columns 4 tx..
+  // loaders: A rows (t & 127), k (t >> 7) * 8 .. + 7; Q row k = t >> 4, columns 4 (t & 15) ..
+  const int ar = threadIdx.x & 127, ak = (threadIdx.x >> 7) * 8;
+  const int qk = threadIdx.x >> 4, qc = (threadIdx.x & 15) * 4;
+  float acc[8][4];
 #pragma unroll
-  for (int a = 0; a < 4; ++a)
+  for (int a = 0; a < 8; ++a)
 #pragma unroll
-    for (int b = 0; b < 4; ++b) acc[a][b] = 0.0f;
-  const int lr = threadIdx.x & 63, lk = (threadIdx.x >> 6) * 8;  // A loader: row lr, k lk..lk+7
-  const int qk = threadIdx.x >> 3, qc = (threadIdx.x & 7) * 8;   // Q loader: k qk, cols qc..qc+7
-  for (int k0 = k_begin; k0 < k_end; k0 += kSkK) {
-    {
-      const float* src = A + (int64_t)(row0 + lr) * d + k0 + lk;
-      const float4 x = __ldg(reinterpret_cast<const float4*>(src));
-      const float4 y = __ldg(reinterpret_cast<const float4*>(src) + 1);
-      As[lk + 0][lr] = x.x; As[lk + 1][lr] = x.y; As[lk + 2][lr] = x.z; As[lk + 3][lr] = x.w;
-      As[lk + 4][lr] = y.x; As[lk + 5][lr] = y.y; As[lk + 6][lr] = y.z; As[lk + 7][lr] = y.w;
-      const float* qs = Q + (int64_t)(k0 + qk) * m;
+    for (int c = 0; c < 4; ++c) acc[a][c] = 0.0f;
+  float4 ra0, ra1, rq;
+  auto fetch = [&](int k0) {
+    const float4* src4 = reinterpret_cast<const float4*>(A + (int64_t)(row0 + ar) * d + k0 + ak);
+    ra0 = __ldg(src4);
+    ra1 = __ldg(src4 + 1);
+    const float* qrow = Q + (int64_t)(k0 + qk) * m;
+    rq.x = qc + 0 < m ? __ldg(qrow + qc + 0) : 0.0f;
+    rq.y = qc + 1 < m ? __ldg(qrow + qc + 1) : 0.0f;
+    rq.z = qc + 2 < m ? __ldg(qrow + qc + 2) : 0.0f;
+    rq.w = qc + 3 < m ? __ldg(qrow + qc + 3) : 0.0f;
+  };
+  auto stash = [&](int buf) {
+    As[buf][ak + 0][ar] = ra0.x; As[buf][ak + 1][ar] = ra0.y; As[buf][ak + 2][ar] = ra0.z; As[buf][ak + 3][ar] = ra0.w;
+    As[buf][ak + 4][ar] = ra1.x; As[buf][ak + 5][ar] = ra1.y; As[buf][ak + 6][ar] = ra1.z; As[buf][ak + 7][ar] = ra1.w;
+    *reinterpret_cast<float4*>(&Qs[buf][qk][qc]) = rq;
+  };
+  int buf = 0;
+  if (k_begin < k_end) {
+    fetch(k_begin);
+    stash(0);
+  }
+  __syncthreads();
+  for (int k0 = k_begin; k0 < k_end; k0 += kSkStep) {
+    const bool more = k0 + kSkStep < k_end;
+    if (more) fetch(k0 + kSkStep);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) Qs[qk][qc + e] = (qc + e < m) ? __ldg(qs + qc + e) : 0.0f;
+    for (int kk = 0; kk < kSkStep; ++kk) {
+      const float4 a0 = *reinterpret_cast<const float4*>(&As[buf][kk][ty * 8]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&As[buf][kk][ty * 8 + 4]);
+      const float4 q4 = *reinterpret_cast<const float4*>(&Qs[buf][kk][tx * 4]);
+      const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float qv[4] = {q4.x, q4.y, q4.z, q4.w};
+#pragma unroll
+      for (int a = 0; a < 8; ++a)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc[a][c] = fmaf(av[a], qv[c], acc[a][c]);
     }
+    if (more) stash(buf ^ 1);
     __syncthreads();
-#pragma unroll 8
-    for (int kk = 0; kk < kSkK; ++kk) {
-      const float4 a4 = *reinterpret_cast<const float4*>(&As[kk][ti * 4]);
-      const float4 q4 = *reinterpret_cast<const float4*>(&Qs[kk][tj * 4]);
-      const float av[4] = {a4.x, a4.y, a4.z, a4.w}, qv[4] = {q4.x, q4.y, q4.z, q4.w};
-#pragma unroll
-      for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int b = 0; b < 4; ++b) acc[a][b] = fmaf(av[a], qv[b], acc[a][b]);
-    }
-    __syncthreads();
+    buf ^= 1;
   }
   float* out = Yp + (int64_t)blockIdx.y * d * m;
 #pragma unroll
-  for (int a = 0; a < 4; ++a)
+  for (int a = 0; a < 8; ++a)
 #pragma unroll
-    for (int b = 0; b < 4; ++b) {
-      const int c = tj * 4 + b;
-      if (c < m) out[(int64_t)(row0 + ti * 4 + a) * m + c] = acc[a][b];
+    for (int c = 0; c < 4; ++c) {
+      const int col = tx * 4 + c;
+      if (col < m) out[(int64_t)(row0 + ty * 8 + a) * m + col] = acc[a][c];
     }
 }
 
@@ -690,7 +712,7 @@ constexpr size_t kRRSmem = 4 * 64 * 65 * sizeof(double);
 
 // k-slices of the skinny product: enough CTAs to cover the SMs twice
 inline int skinny_slices(int d) {
-  const int tiles = d / 64;
+  const int tiles = d / 128;
   int ns = (2 * kNumSMs + tiles - 1) / tiles;
   const int max_ns = d / (4 * kSkK);
   if (ns > max_ns) ns = max_ns;
@@ -807,7 +829,7 @@ cudaError_t launch_refresh_batch(const RefreshPlan* plans, const RefreshIO* io, 
     const int ew_blocks = (int)((dm + kRT - 1) / kRT < 2 * kNumSMs ? (dm + kRT - 1) / kRT : 2 * kNumSMs);
     // qr_apply: two 32-row tiles per CTA (the m x m factor is loaded once per CTA)
     const int qr_blocks = (dmax / 32 + 1) / 2;
-    const dim3 g_ew(ew_blocks, 1, cnt), g_skinny(dmax / 64, nsmax, cnt), g_gram(pmax, 1, cnt), g_one(1, 1, cnt),
+    const dim3 g_ew(ew_blocks, 1, cnt), g_skinny(dmax / 128, nsmax, cnt), g_gram(pmax, 1, cnt), g_one(1, 1, cnt),
         g_qr(qr_blocks, 1, cnt);
     // one Cholesky-QR pass: dst = src R^{-1} with src^T src = R^T R
     auto cholqr_pass = [&](int src, int dst) {
