@@ -228,6 +228,36 @@ GIFT_DEV void convert_u_row_inplace(uint32_t tile, int t) {
     st_shared_v4(tile + sw128(t, 4 + q), lo[4 * q], lo[4 * q + 1], lo[4 * q + 2], lo[4 * q + 3]);
 }
 
+// As convert_u_row_inplace, with f16 parts for the decoder's first pass:
+// [hi 0..31 | lo 0..31] with hi = f16(u) and lo = f16((u - hi) * 2^11) (the
+// product with lo is scaled back by 2^-11 in the epilogue).  f16 keeps 11
+// mantissa bits per part, and every E4M3 or NVFP4 value is exact in f16.
+constexpr float kF16LoScale = 2048.0f;
+GIFT_DEV void convert_u_row_inplace_f16(uint32_t tile, int t) {
+  float u[32];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const uint4 v = ld_shared_v4(tile + sw128(t, q));
+    u[4 * q] = __uint_as_float(v.x);
+    u[4 * q + 1] = __uint_as_float(v.y);
+    u[4 * q + 2] = __uint_as_float(v.z);
+    u[4 * q + 3] = __uint_as_float(v.w);
+  }
+  uint32_t hi[16], lo[16];
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    const float h0 = __half2float(__float2half_rn(u[2 * k]));
+    const float h1 = __half2float(__float2half_rn(u[2 * k + 1]));
+    hi[k] = pack_f16x2(h0, h1);
+    lo[k] = pack_f16x2((u[2 * k] - h0) * kF16LoScale, (u[2 * k + 1] - h1) * kF16LoScale);
+  }
+#pragma unroll
+  for (int q = 0; q < 4; ++q) st_shared_v4(tile + sw128(t, q), hi[4 * q], hi[4 * q + 1], hi[4 * q + 2], hi[4 * q + 3]);
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    st_shared_v4(tile + sw128(t, 4 + q), lo[4 * q], lo[4 * q + 1], lo[4 * q + 2], lo[4 * q + 3]);
+}
+
 template <int FMT>
 __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __grid_constant__ EncParams p,
                                                                      uint32_t* err) {
@@ -560,13 +590,15 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
 // ===========================================================================
 // Decode: G_hat = W_hat M^{-1},  W_hat = value(codes) * scale (per block),
 //   M^{-1} = a I + U diag(c) U^T,  a = rho^{1/2},  c_k = (lambda_k+rho)^{1/2} - a.
-//   D2  P = W_hat U = sum_c s_c (q_c U_c): the codes q are exact in bf16, so
-//       each chunk's product T_c = q_c [U_hi | U_lo] (M=128, N=64, K=128) is
-//       scaled by its block scale in the epilogue and summed in fp32.
-//   D3  G_hat = a W_hat + (P o c) U^T   (M=128, N=128 per chunk, K=32, split
-//       as in the encoder), bf16 output with round-to-nearest-even.
-// Stage = codes tile (TMA, [128][128 B], 128-byte swizzle) + bf16 copy of the
-// codes (the D2 A operand, written by the converter warps) + U tile.
+//   D2  P = W_hat U = sum_c s_c (q_c U_c): the codes q are exact in f16, so
+//       each chunk's product T_c = q_c [U_hi | U_lo 2^11] (f16 operands, M=128,
+//       N=64, K=128) is scaled by its block scale in the epilogue and summed in
+//       fp32 (f16 widening is one instruction per pair of codes).
+//   D3  G_hat = a W_hat + (P o c) U^T   (M=128, N=128 per chunk, K=32, bf16
+//       split as in the encoder), bf16 output with round-to-nearest-even.
+// Stage = codes tile (TMA, [128][128 B], 128-byte swizzle) + f16 copy of the
+// codes (the D2 A operand, written by the converter warps; the output tile of
+// D3) + U tile (split to f16 for D2, to bf16 for D3).
 // ===========================================================================
 constexpr int kDStages = 3;  // decode ring
 constexpr int kDCodes = kPanel * kChunk;            // 16 KB
@@ -576,7 +608,7 @@ constexpr int kDSmemBytes = kDStages * kDStageBytes + kPcBytes + 1024 + 512;
 static_assert(kDSmemBytes <= 232448, "decode shared memory");
 static_assert(kSmemBytes <= 232448, "encode shared memory");
 constexpr uint32_t kColT0 = 256, kColT1 = 320;
-constexpr uint32_t kIdescD2 = umma_idesc_bf16(128, 64, 0, 1);
+constexpr uint32_t kIdescD2 = umma_idesc_f16(128, 64, 0, 1);   // D2 runs on f16 operands
 
 struct alignas(64) DecJob {
   CUtensorMap tmC;  // uint8 codes [d_out][d_in], box [128][128], 128-byte swizzle
@@ -599,10 +631,11 @@ struct DecParams {
 };
 static_assert(sizeof(DecParams) <= 32760, "kernel parameter space");
 
-// E4M3 pair -> bf16 pair (exact: every E4M3 value is a bf16 value)
-GIFT_DEV uint32_t e4m3x2_to_bf16x2(uint16_t v) {
-  const float2 f = e4m3x2_to_f32x2(v);
-  return pack_bf16x2(f.x, f.y);
+// E4M3 pair -> f16 pair (exact: every E4M3 value is an f16 value), byte 0 in the low half
+GIFT_DEV uint32_t e4m3x2_to_f16x2(uint16_t v) {
+  uint32_t h;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(v));
+  return h;
 }
 
 template <int FMT>
@@ -714,11 +747,15 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
       }
       const uint32_t c_tile = sbase + s * kDStageBytes;
       const uint32_t q_tile = c_tile + kDCodes;
-      convert_u_row_inplace(q_tile + kDQ, t);
+      // D2 multiplies f16 codes by an f16 split of U, D3 the bf16 P' o c' by a bf16 split
+      if (st.pass == 0)
+        convert_u_row_inplace_f16(q_tile + kDQ, t);
+      else
+        convert_u_row_inplace(q_tile + kDQ, t);
       const DecJob& J = p.jobs[st.job()];
       if (st.pass == 0 && FMT != kFmtE4M3) {
         // NVFP4: row t's 128 codes (64 bytes) and 8 block scales from global,
-        // widened to bf16 value(code) x value(scale) (exact)
+        // widened to f16 value(code) x value(scale) (exact)
         const int64_t row = (int64_t)st.panel() * kPanel + t;
         uint4 cw[4] = {};
         uint2 sw = make_uint2(0u, 0u);
@@ -736,13 +773,13 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
           nvfp4_block16_values(cb, (uint8_t)(((j < 4) ? sw.x : sw.y) >> (8 * (j & 3))), v);
           uint32_t o[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) o[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
-          const int c0 = 2 * j, c1 = 2 * j + 1;  // 16-byte chunks of the 256-byte bf16 row
+          for (int i = 0; i < 8; ++i) o[i] = pack_f16x2(v[2 * i], v[2 * i + 1]);
+          const int c0 = 2 * j, c1 = 2 * j + 1;  // 16-byte chunks of the 256-byte f16 row
           st_shared_v4(q_tile + (c0 >> 3) * kGHalf + sw128(t, c0 & 7), o[0], o[1], o[2], o[3]);
           st_shared_v4(q_tile + (c1 >> 3) * kGHalf + sw128(t, c1 & 7), o[4], o[5], o[6], o[7]);
         }
       } else if (st.pass == 0) {
-        // the codes of row t, widened to bf16
+        // the codes of row t, widened to f16
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
           const uint4 v = ld_shared_v4(c_tile + sw128(t, q));
@@ -750,8 +787,8 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
           uint32_t o[8];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            o[2 * e] = e4m3x2_to_bf16x2((uint16_t)(w[e] & 0xFFFFu));
-            o[2 * e + 1] = e4m3x2_to_bf16x2((uint16_t)(w[e] >> 16));
+            o[2 * e] = e4m3x2_to_f16x2((uint16_t)(w[e] & 0xFFFFu));
+            o[2 * e + 1] = e4m3x2_to_f16x2((uint16_t)(w[e] >> 16));
           }
           // 16 codes -> 32 bytes of bf16 = chunks 2q, 2q+1 of the 256-byte row
           const int c0 = 2 * q, c1 = 2 * q + 1;
@@ -881,7 +918,8 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
         tc_fence_before();
         mbar_arrive(&t_empty[b]);
 #pragma unroll
-        for (int k = 0; k < 16; ++k) P[k] = fmaf(sc, __uint_as_float(th[k]) + __uint_as_float(tl[k]), P[k]);
+        for (int k = 0; k < 16; ++k)
+          P[k] = fmaf(sc, fmaf(__uint_as_float(tl[k]), 1.0f / kF16LoScale, __uint_as_float(th[k])), P[k]);
         ++d2;
       } else {
         // D3 epilogue: G_hat = a s q + acc

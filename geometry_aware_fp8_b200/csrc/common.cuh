@@ -38,6 +38,19 @@ GIFT_DEV uint32_t pack_bf16x2(float x0, float x1) {
   return r;
 }
 
+// two floats -> f16x2 with round-to-nearest-even, x0 in the low half
+GIFT_DEV uint32_t pack_f16x2(float x0, float x1) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(x1), "f"(x0));
+  return r;
+}
+
+// Instruction descriptor for kind::f16 with f16 A/B, fp32 D (see umma_idesc_bf16).
+__host__ __device__ constexpr uint32_t umma_idesc_f16(int M, int N, int a_mn, int b_mn) {
+  return (1u << 4) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) | ((uint32_t)(N >> 3) << 17) |
+         ((uint32_t)(M >> 4) << 24);
+}
+
 // ---------------------------------------------------------------------------
 // E4M3 through the hardware converters (round to nearest even, saturating to
 // +-448; the sign of zero follows the input).  The first operand of the PTX
