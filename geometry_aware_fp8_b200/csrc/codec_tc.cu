@@ -596,15 +596,18 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
 //       fp32 (f16 widening is one instruction per pair of codes).
 //   D3  G_hat = a W_hat + (P o c) U^T   (M=128, N=128 per chunk, K=32, bf16
 //       split as in the encoder), bf16 output with round-to-nearest-even.
-// Stage = codes tile (TMA, [128][128 B], 128-byte swizzle) + f16 copy of the
-// codes (the D2 A operand, written by the converter warps; the output tile of
-// D3) + U tile (split to f16 for D2, to bf16 for D3).
+// Stage (4-deep ring) = codes tile (TMA, [128][128 B], 128-byte swizzle) + U
+// tile (split to f16 for D2, to bf16 for D3).  Two scratch tiles, taken in
+// step order, hold a D2 step's f16 codes (the A operand, written by the
+// converter warps, free when the MMA completes) or a D3 step's bf16 output
+// (free once the TMA stores have read it).  A D3 stage is released as soon as
+// every epilogue thread has read its codes.
 // ===========================================================================
-constexpr int kDStages = 3;  // decode ring
+constexpr int kDStages = 4;                         // decode ring
 constexpr int kDCodes = kPanel * kChunk;            // 16 KB
-constexpr int kDQ = kPanel * kChunk * 2;            // 32 KB: two [128][64] bf16 tiles
-constexpr int kDStageBytes = kDCodes + kDQ + kUBytes;
-constexpr int kDSmemBytes = kDStages * kDStageBytes + kPcBytes + 1024 + 512;
+constexpr int kDStageBytes = kDCodes + kUBytes;     // codes + U
+constexpr int kDScratch = kPanel * kChunk * 2;      // 32 KB: two [128][64] 16-bit boxes
+constexpr int kDSmemBytes = kDStages * kDStageBytes + 2 * kDScratch + kPcBytes + 1024 + 512;
 static_assert(kDSmemBytes <= 232448, "decode shared memory");
 static_assert(kSmemBytes <= 232448, "encode shared memory");
 constexpr uint32_t kColT0 = 256, kColT1 = 320;
@@ -644,13 +647,15 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const uint32_t sbase = smem_u32(smem);
-  const uint32_t pc_tile = sbase + kDStages * kDStageBytes;
-  uint64_t* bars = (uint64_t*)(smem + kDStages * kDStageBytes + kPcBytes);
-  uint64_t* full = bars;                   // [kDStages] count 1: converter (U tile, bf16 codes)
-  uint64_t* cfull = bars + kDStages;       // [kDStages] count 1 + tx: codes TMA
-  uint64_t* empty = bars + 2 * kDStages;   // [kDStages] count 1: MMA commit (D2) or output store (D3)
-  uint64_t* oready = bars + 3 * kDStages;  // [kDStages] count 256: output tile of a D3 step in shared memory
-  uint64_t* t_full = bars + 4 * kDStages;  // [2] count 1
+  const uint32_t scr = sbase + kDStages * kDStageBytes;  // [2] scratch tiles: two [128][64] 16-bit boxes each
+  const uint32_t pc_tile = scr + 2 * kDScratch;
+  uint64_t* bars = (uint64_t*)(smem + kDStages * kDStageBytes + 2 * kDScratch + kPcBytes);
+  uint64_t* full = bars;                   // [kDStages] count 1: converter (U split; first pass: codes widened)
+  uint64_t* cfull = bars + kDStages;       // [kDStages] count 1 + tx: TMA (codes and U)
+  uint64_t* empty = bars + 2 * kDStages;   // [kDStages] count 1: MMA commit (D2) or store warp (D3)
+  uint64_t* sfree = bars + 3 * kDStages;   // [2] count 1: scratch tile free (MMA commit or store read)
+  uint64_t* oready = sfree + 2;            // [2] count 256: output tile written
+  uint64_t* t_full = oready + 2;           // [2] count 1
   uint64_t* t_empty = t_full + 2;          // [2] count 256
   uint64_t* pc_full = t_full + 4;          // count 256
   uint64_t* w_full = t_full + 5;           // [2] count 1
@@ -666,9 +671,10 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
       mbar_init(&full[s], 1);
       mbar_init(&cfull[s], 1);
       mbar_init(&empty[s], 1);
-      mbar_init(&oready[s], 256);
     }
     for (int b = 0; b < 2; ++b) {
+      mbar_init(&sfree[b], 1);
+      mbar_init(&oready[b], 256);
       mbar_init(&t_full[b], 1);
       mbar_init(&t_empty[b], 256);
       mbar_init(&w_full[b], 1);
@@ -705,53 +711,59 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
           tma_load_2d_hint(dst, &J.tmC, &cfull[s], st.chunk() * kChunk, st.panel() * kPanel,
                            st.pass == 0 ? keep : drop);
         } else {
-          mbar_arrive_expect_tx(&cfull[s], kUBytes);  // NVFP4 codes are read by the converters
+          mbar_arrive_expect_tx(&cfull[s], kUBytes);  // NVFP4 codes are read from global memory
         }
-        tma_load_2d_hint(dst + kDCodes + kDQ, &J.tmU, &cfull[s], 0, st.chunk() * kChunk, keep);
+        tma_load_2d_hint(dst + kDCodes, &J.tmU, &cfull[s], 0, st.chunk() * kChunk, keep);
       }
     }
   } else if (warp == 14) {
-    // ---------------- output stores: two TMA stores per D3 step, then the stage is free ----------------
+    // ---------------- output stores: a second-pass step's tile leaves by two TMA stores ----------------
+    // All epilogue threads have read the step's codes when its tile is ready,
+    // so the stage is released first, then the scratch tile once the stores
+    // have read it.
     if (lane == 0) {
       const uint64_t drop = policy_evict_first();
-      uint32_t step = 0, par = 0;  // par: bit s = phase parity of oready[s]
+      uint32_t step = 0, par = 0;  // par: bit j = phase parity of oready[j]
       for (Steps<DecParams> st(p, beg, end); st.valid() && !failed; st.next(), ++step) {
         if (st.pass == 0) continue;
-        const int s = step % kDStages;
-        if (!mbar_wait(&oready[s], (par >> s) & 1u, kWaitLimit)) {
+        const int s = step % kDStages, j = step & 1;
+        if (!mbar_wait(&oready[j], (par >> j) & 1u, kWaitLimit)) {
           failed = 1;
           break;
         }
-        par ^= 1u << s;
+        par ^= 1u << j;
+        mbar_arrive(&empty[s]);
         const DecJob& J = p.jobs[st.job()];
-        const uint32_t o_tile = sbase + s * kDStageBytes + kDCodes;
+        const uint32_t o_tile = scr + j * kDScratch;
         tma_store_2d_hint(&J.tmO, o_tile, st.chunk() * kChunk, st.panel() * kPanel, drop);
         tma_store_2d_hint(&J.tmO, o_tile + kGHalf, st.chunk() * kChunk + 64, st.panel() * kPanel, drop);
         bulk_commit();
         bulk_wait_read<0>();
-        mbar_arrive(&empty[s]);
+        mbar_arrive(&sfree[j]);
       }
       bulk_wait_all();
     }
   } else if (warp >= 8 && warp < 12) {
-    // ---------------- converters: U tile in place, and in the first pass the bf16 codes ----------------
+    // ---------------- converters: U split in place; first pass: codes widened into a scratch tile ----------------
     const int t = threadIdx.x - 256;
     uint32_t step = 0;
     for (Steps<DecParams> st(p, beg, end); st.valid(); st.next(), ++step) {
-      const int s = step % kDStages;
+      const int s = step % kDStages, j = step & 1;
       const uint32_t use = step / kDStages;
-      const bool ok = mbar_wait(&cfull[s], use & 1u, kWaitLimit);
+      bool ok = mbar_wait(&cfull[s], use & 1u, kWaitLimit);
+      if (st.pass == 0 && step >= 2) ok = ok && mbar_wait(&sfree[j], ((step >> 1) - 1) & 1u, kWaitLimit);
       if (named_sync_or(1, 128, !ok)) {
         failed = 1;
         break;
       }
       const uint32_t c_tile = sbase + s * kDStageBytes;
-      const uint32_t q_tile = c_tile + kDCodes;
+      const uint32_t u_tile = c_tile + kDCodes;
+      const uint32_t q_tile = scr + j * kDScratch;
       // D2 multiplies f16 codes by an f16 split of U, D3 the bf16 P' o c' by a bf16 split
       if (st.pass == 0)
-        convert_u_row_inplace_f16(q_tile + kDQ, t);
+        convert_u_row_inplace_f16(u_tile, t);
       else
-        convert_u_row_inplace(q_tile + kDQ, t);
+        convert_u_row_inplace(u_tile, t);
       const DecJob& J = p.jobs[st.job()];
       if (st.pass == 0 && FMT != kFmtE4M3) {
         // NVFP4: row t's 128 codes (64 bytes) and 8 block scales from global,
@@ -766,15 +778,15 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
           sw = __ldg(reinterpret_cast<const uint2*>(J.sb + row * (J.d_in / 16) + st.chunk() * 8));
         }
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {  // block j = columns 16 j .. 16 j + 15
-          const uint4& c = cw[j >> 1];
-          const uint2 cb = (j & 1) ? make_uint2(c.z, c.w) : make_uint2(c.x, c.y);
+        for (int b = 0; b < 8; ++b) {  // block b = columns 16 b .. 16 b + 15
+          const uint4& c = cw[b >> 1];
+          const uint2 cb = (b & 1) ? make_uint2(c.z, c.w) : make_uint2(c.x, c.y);
           float v[16];
-          nvfp4_block16_values(cb, (uint8_t)(((j < 4) ? sw.x : sw.y) >> (8 * (j & 3))), v);
+          nvfp4_block16_values(cb, (uint8_t)(((b < 4) ? sw.x : sw.y) >> (8 * (b & 3))), v);
           uint32_t o[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i) o[i] = pack_f16x2(v[2 * i], v[2 * i + 1]);
-          const int c0 = 2 * j, c1 = 2 * j + 1;  // 16-byte chunks of the 256-byte f16 row
+          const int c0 = 2 * b, c1 = 2 * b + 1;  // 16-byte chunks of the 256-byte f16 row
           st_shared_v4(q_tile + (c0 >> 3) * kGHalf + sw128(t, c0 & 7), o[0], o[1], o[2], o[3]);
           st_shared_v4(q_tile + (c1 >> 3) * kGHalf + sw128(t, c1 & 7), o[4], o[5], o[6], o[7]);
         }
@@ -790,7 +802,7 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
             o[2 * e] = e4m3x2_to_f16x2((uint16_t)(w[e] & 0xFFFFu));
             o[2 * e + 1] = e4m3x2_to_f16x2((uint16_t)(w[e] >> 16));
           }
-          // 16 codes -> 32 bytes of bf16 = chunks 2q, 2q+1 of the 256-byte row
+          // 16 codes -> 32 bytes of f16 = chunks 2q, 2q+1 of the 256-byte row
           const int c0 = 2 * q, c1 = 2 * q + 1;
           st_shared_v4(q_tile + (c0 >> 3) * kGHalf + sw128(t, c0 & 7), o[0], o[1], o[2], o[3]);
           st_shared_v4(q_tile + (c1 >> 3) * kGHalf + sw128(t, c1 & 7), o[4], o[5], o[6], o[7]);
@@ -805,16 +817,17 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
     if (lane == 0) {
       uint32_t step = 0, e2 = 0, d2 = 0;
       for (Steps<DecParams> st(p, beg, end); st.valid() && !failed; st.next(), ++step) {
-        const int s = step % kDStages;
+        const int s = step % kDStages, j = step & 1;
         // block k >= 1 starts with D3 of p_{k-1}, which needs its P o c
         if (st.block_start() && st.k >= 1 && !mbar_wait(pc_full, (st.k - 1) & 1u, kWaitLimit)) { failed = 1; break; }
         if (!mbar_wait(&full[s], (step / kDStages) & 1u, kWaitLimit)) { failed = 1; break; }
-        const uint32_t q_tile = sbase + s * kDStageBytes + kDCodes, u_tile = q_tile + kDQ;
+        const uint32_t u_tile = sbase + s * kDStageBytes + kDCodes;
         if (st.pass == 0) {
-          // D2: T_c[128 x 64] = q_c . [U_hi | U_lo]
+          // D2: T_c[128 x 64] = q_c . [U_hi | U_lo 2^11]   (f16)
           const int b = d2 & 1;
           if (d2 >= 2 && !mbar_wait(&t_empty[b], ((d2 >> 1) - 1) & 1u, kWaitLimit)) { failed = 1; break; }
           tc_fence_after();
+          const uint32_t q_tile = scr + j * kDScratch;
           const uint32_t d = tbase + (b ? kColT1 : kColT0);
 #pragma unroll
           for (int h = 0; h < 2; ++h)
@@ -825,10 +838,11 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
               umma_bf16(d, ad, bd, kIdescD2, (h | kk) ? 1u : 0u);
             }
           umma_commit(&empty[s]);
+          umma_commit(&sfree[j]);
           umma_commit(&t_full[b]);
           ++d2;
         } else {
-          // D3: W[128 x 128] = Pc . U^T (three split products)
+          // D3: W[128 x 128] = Pc . U^T (three split products, bf16)
           const int b = e2 & 1;
           if (e2 >= 2 && !mbar_wait(&w_empty[b], ((e2 >> 1) - 1) & 1u, kWaitLimit)) { failed = 1; break; }
           tc_fence_after();
@@ -852,8 +866,7 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
     // coefficients k = 16 h .. 16 h + 15, in D3 the columns 64 h .. 64 h + 63
     // of every 128-column chunk (h = warp / 4).  P of the panel in its first
     // pass stays in registers until the block that starts its second pass;
-    // D3 writes its bf16 tile into the stage's codes-as-bf16 region (free in
-    // the second pass) for the store warp.
+    // D3 writes its bf16 tile into the step's scratch tile for the store warp.
     const int h = warp >> 2;
     const int r = (warp & 3) * 32 + lane;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
@@ -864,7 +877,7 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
     float a = 0.0f;
     bool stop = false;
     for (Steps<DecParams> st(p, beg, end); st.valid() && !stop; st.next(), ++step) {
-      const int s = step % kDStages;
+      const int s = step % kDStages, j = step & 1;
       const DecJob& J = p.jobs[st.job()];
       const int nc = st.nc(), c = st.chunk();
       const int64_t row = (int64_t)st.panel() * kPanel + r;
@@ -898,7 +911,7 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
         mbar_arrive(pc_full);
       }
       if (st.pass == 0) {
-        // D2 epilogue: P += s_c (T_hi + T_lo) for this half's 16 coefficients
+        // D2 epilogue: P += s_c (T_hi + 2^-11 T_lo) for this half's 16 coefficients
         if (c == 0) {
 #pragma unroll
           for (int k = 0; k < 16; ++k) P[k] = 0.0f;
@@ -922,10 +935,11 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
           P[k] = fmaf(sc, fmaf(__uint_as_float(tl[k]), 1.0f / kF16LoScale, __uint_as_float(th[k])), P[k]);
         ++d2;
       } else {
-        // D3 epilogue: G_hat = a s q + acc
+        // D3 epilogue: G_hat = a s q + acc, into scratch tile j once its previous use is stored
         const int b = e2 & 1;
-        const bool ok = mbar_wait(&w_full[b], (e2 >> 1) & 1u, kWaitLimit) &&
-                        mbar_wait(&cfull[s], (step / kDStages) & 1u, kWaitLimit);
+        bool ok = mbar_wait(&w_full[b], (e2 >> 1) & 1u, kWaitLimit) &&
+                  mbar_wait(&cfull[s], (step / kDStages) & 1u, kWaitLimit);
+        if (step >= 2) ok = ok && mbar_wait(&sfree[j], ((step >> 1) - 1) & 1u, kWaitLimit);
         stop = named_sync_or(2, 256, !ok);
         if (stop) {
           failed = 1;
@@ -934,7 +948,7 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
         tc_fence_after();
         const uint32_t wcol = tbase + lane_off + (b ? kColW1 : kColW0) + 64 * h;
         const uint32_t c_tile = sbase + s * kDStageBytes;
-        const uint32_t o_tile = c_tile + kDCodes;  // two [128][64] bf16 boxes, 128-byte swizzle
+        const uint32_t o_tile = scr + j * kDScratch;  // two [128][64] bf16 boxes, 128-byte swizzle
         const float as = a * sc;
 #pragma unroll
         for (int g2 = 0; g2 < 2; ++g2) {
@@ -983,7 +997,7 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
         tc_fence_before();
         mbar_arrive(&w_empty[b]);
         fence_async_shared();
-        mbar_arrive(&oready[s]);
+        mbar_arrive(&oready[j]);
         ++e2;
       }
     }
