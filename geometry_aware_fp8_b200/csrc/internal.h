@@ -89,6 +89,20 @@ void refresh_plan(int64_t N, int64_t d, int rank, int oversample, bool a_out_giv
                   bool no_split = false);
 cudaError_t launch_refresh(const RefreshPlan& p, const void* X, gift_dtype xdt, float* U, float* lambda,
                            float* rho, float* A_out, void* ws, uint32_t* dev_status, cudaStream_t s);
+// ---- A = X^T X / N of many layers in one tensor-core launch (syrk_tc.cu) ----
+struct SyrkJob {
+  const void* X;
+  gift_dtype xdt;
+  int64_t N;
+  int d;
+  float* A;
+  uint32_t* err;
+};
+// Every job with bf16 X and d % 128 == 0 is computed (token range never split,
+// so a layer's A does not depend on what it is batched with) and gets
+// used[i] = true; the others are left to the caller.  n <= 64.
+cudaError_t launch_syrk_tc_batch(const SyrkJob* jobs, int n, cudaStream_t s, bool* used);
+
 // A Q on the tensor cores (bf16 hi/lo split operands), one k-slice per CTA row.
 constexpr int kSkinnyMaxBatch = 48;
 struct SkinnyTcJob {

@@ -781,16 +781,26 @@ cudaError_t launch_refresh_batch(const RefreshPlan* plans, const RefreshIO* io, 
     B.m = m;
     B.r = r;
     int dmax = 0, nsmax = 1, pmax = 1;
+    // R1: A = X^T X / N for every layer of the batch in one tensor-core launch
+    // (bf16 X); otherwise one launch per layer below
+    static thread_local SyrkJob sj[kMaxBatch];
+    for (int l = 0; l < cnt; ++l) {
+      const RefreshPlan& p = plans[base + l];
+      const RefreshIO& o = io[base + l];
+      sj[l] = SyrkJob{o.X, o.xdt, p.N, (int)p.d, o.A_out ? o.A_out : (float*)((char*)o.ws + p.off_A), o.dev_status};
+    }
+    static thread_local bool batched[kMaxBatch];
+    if ((e = launch_syrk_tc_batch(sj, cnt, s, batched)) != cudaSuccess) return e;
     for (int l = 0; l < cnt; ++l) {
       const RefreshPlan& p = plans[base + l];
       const RefreshIO& o = io[base + l];
       char* w = (char*)o.ws;
       const int d = (int)p.d;
       float* A = o.A_out ? o.A_out : (float*)(w + p.off_A);
-      // R1: A = X^T X / N (one launch per layer; each fills the GPU)
-      bool used_tc = false;
-      e = launch_syrk_tc(o.X, o.xdt, p.N, d, A, (float*)(w + p.off_syrk), p.syrk_splits, o.dev_status, s,
-                         &used_tc);
+      bool used_tc = batched[l];
+      if (!used_tc)
+        e = launch_syrk_tc(o.X, o.xdt, p.N, d, A, (float*)(w + p.off_syrk), p.syrk_splits, o.dev_status, s,
+                           &used_tc);
       if (e != cudaSuccess) return e;
       if (!used_tc) {
         const int nt = d / 64;

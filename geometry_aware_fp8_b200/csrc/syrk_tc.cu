@@ -10,7 +10,9 @@
 // dimension, streamed in 64-row chunks by TMA.  Both operands come straight
 // from X's rows: X[n][i] has i contiguous, so A-operand (M = i) and
 // B-operand (N = j) are MN-major 128-byte-swizzled tiles, one 64-column box
-// per 64 features.  One CTA per (tile, token split):
+// per 64 features.  One launch covers a batch of layers (the batched factor
+// refresh): the CTA index picks the layer, its tile and token split.  One CTA
+// per (layer, tile, token split):
 //   warp 8     TMA producer (4-stage ring, 48 KB per stage)
 //   warp 9     TMEM allocation and the single-thread MMA issue
 //   warps 0-7  epilogue: TMEM -> registers -> A (j >= i only, mirrored),
@@ -41,16 +43,24 @@ constexpr int THREADS = 320;
 constexpr uint32_t IDESC = umma_idesc_bf16(BM, BN, /*a MN-major*/ 1, /*b MN-major*/ 1);
 constexpr uint32_t kWaitLimit = 1u << 22;
 
-struct SyrkArgs {
+struct alignas(64) SyrkLayer {
+  CUtensorMap tmX;  // bf16 X [N][d], box [64 tokens][64 features], 128-byte swizzle
   int d;
+  int tile_begin;   // first tile of this layer in the launch
   int64_t N;
-  int splits;
   int64_t rows_per_split;
   float scale;
-  float* A;       // direct output (splits == 1)
-  float* part;    // splits x d x d raw partial sums (splits > 1)
-  uint32_t* err;  // optional device status word
+  float* A;         // direct output (splits == 1)
+  float* part;      // splits x d x d raw partial sums (splits > 1)
+  uint32_t* err;    // optional device status word
 };
+constexpr int kSyrkMaxBatch = 64;
+struct SyrkBatch {
+  SyrkLayer L[kSyrkMaxBatch];
+  int n;
+  int splits;
+};
+static_assert(sizeof(SyrkBatch) <= 32760, "kernel parameter space");
 
 __device__ void tile_of(int t, int d, int* I, int* J2) {
   const int nI = d / BM, nJ = (d + BN - 1) / BN;
@@ -63,7 +73,7 @@ __device__ void tile_of(int t, int d, int* I, int* J2) {
   *J2 = i / 2 + t;
 }
 
-__global__ void __launch_bounds__(THREADS, 1) syrk_tc_kernel(const __grid_constant__ CUtensorMap tmX, SyrkArgs a) {
+__global__ void __launch_bounds__(THREADS, 1) syrk_tc_kernel(const __grid_constant__ SyrkBatch p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint64_t* full = (uint64_t*)(smem + STAGES * STAGE_BYTES);
@@ -74,9 +84,14 @@ __global__ void __launch_bounds__(THREADS, 1) syrk_tc_kernel(const __grid_consta
   __shared__ int failed;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int split = blockIdx.x % a.splits;
+  const int split = blockIdx.x % p.splits;
+  const int tile = blockIdx.x / p.splits;
+  int l = 0;
+  while (l + 1 < p.n && tile >= p.L[l + 1].tile_begin) ++l;
+  const SyrkLayer& a = p.L[l];
+  const CUtensorMap& tmX = a.tmX;
   int I, J2;
-  tile_of(blockIdx.x / a.splits, a.d, &I, &J2);
+  tile_of(tile - a.tile_begin, a.d, &I, &J2);
   const int64_t n_begin = (int64_t)split * a.rows_per_split;
   int64_t n_end = n_begin + a.rows_per_split;
   if (n_end > a.N) n_end = a.N;
@@ -185,7 +200,7 @@ __global__ void __launch_bounds__(THREADS, 1) syrk_tc_kernel(const __grid_consta
         const int j = J2 * BN + wh * 128 + t;
         if (j < i || j >= a.d) continue;
         const float v = sum[t];
-        if (a.splits == 1) {
+        if (p.splits == 1) {
           a.A[(int64_t)i * a.d + j] = v * a.scale;
           if (j != i) a.A[(int64_t)j * a.d + i] = v * a.scale;
         } else {
@@ -215,27 +230,64 @@ cudaError_t launch_syrk_tc(const void* X, gift_dtype xdt, int64_t N, int d, floa
                            uint32_t* err, cudaStream_t s, bool* used) {
   *used = false;
   if (xdt != GIFT_BF16 || d % BM != 0) return cudaSuccess;
-  CUtensorMap tm;
-  if (!make_tmap_2d(&tm, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)N, (uint64_t)d, 64, 64))
+  static thread_local SyrkBatch P;
+  SyrkLayer& a = P.L[0];
+  if (!make_tmap_2d(&a.tmX, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)N, (uint64_t)d, 64, 64))
     return cudaSuccess;  // no driver entry point: the CUDA-core syrk runs instead
   cudaError_t e = ensure_smem_attr(syrk_tc_kernel, SMEM_BYTES, &g_attr_mask);
   if (e != cudaSuccess) return e;
-  SyrkArgs a;
+  P.n = 1;
+  P.splits = splits < 1 ? 1 : splits;
   a.d = d;
+  a.tile_begin = 0;
   a.N = N;
-  a.splits = splits < 1 ? 1 : splits;
-  a.rows_per_split = ((N + a.splits - 1) / a.splits + BK - 1) / BK * BK;
+  a.rows_per_split = ((N + P.splits - 1) / P.splits + BK - 1) / BK * BK;
   a.scale = (float)(1.0 / (double)N);
   a.A = A;
   a.part = part;
   a.err = err;
-  const int items = syrk_tc_tiles(d) * a.splits;
-  syrk_tc_kernel<<<items, THREADS, SMEM_BYTES, s>>>(tm, a);
+  const int items = syrk_tc_tiles(d) * P.splits;
+  syrk_tc_kernel<<<items, THREADS, SMEM_BYTES, s>>>(P);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  if (a.splits > 1) e = launch_syrk_reduce(part, a.splits, d, A, a.scale, s);
+  if (P.splits > 1) e = launch_syrk_reduce(part, P.splits, d, A, a.scale, s);
   *used = true;
   return e;
+}
+
+cudaError_t launch_syrk_tc_batch(const SyrkJob* jobs, int n, cudaStream_t s, bool* used) {
+  for (int l = 0; l < n; ++l) used[l] = false;
+  if (n <= 0 || n > kSyrkMaxBatch) return cudaSuccess;
+  static thread_local SyrkBatch P;
+  int tiles = 0, m = 0;
+  for (int l = 0; l < n; ++l) {
+    const SyrkJob& J = jobs[l];
+    if (J.xdt != GIFT_BF16 || J.d % BM != 0) continue;
+    SyrkLayer& a = P.L[m];
+    if (!make_tmap_2d(&a.tmX, J.X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)J.N, (uint64_t)J.d, 64, 64))
+      continue;  // no driver entry point: the CUDA-core syrk runs instead
+    a.d = J.d;
+    a.tile_begin = tiles;
+    a.N = J.N;
+    a.rows_per_split = (J.N + BK - 1) / BK * BK;
+    a.scale = (float)(1.0 / (double)J.N);
+    a.A = J.A;
+    a.part = nullptr;
+    a.err = J.err;
+    tiles += syrk_tc_tiles(J.d);
+    used[l] = true;
+    ++m;
+  }
+  if (m == 0) return cudaSuccess;
+  cudaError_t e = ensure_smem_attr(syrk_tc_kernel, SMEM_BYTES, &g_attr_mask);
+  if (e != cudaSuccess) {
+    for (int l = 0; l < n; ++l) used[l] = false;
+    return e;
+  }
+  P.n = m;
+  P.splits = 1;
+  syrk_tc_kernel<<<tiles, THREADS, SMEM_BYTES, s>>>(P);
+  return cudaGetLastError();
 }
 
 }  // namespace gift
