@@ -192,11 +192,15 @@ def build_workload(torch, ops, synth, dev, depth, seed):
     el = [L for L in layers if L.rank == 0]
     jobs = ops.make_refresh_jobs([(w["X"], w["layer"].U, w["layer"].lam, w["layer"].rho, w["ws"], w["st"],
                                    w["seed"], None) for w in whitened])
-    return dict(layers=layers, whitened=whitened, G_all=G_all, Gh_all=Gh_all, C_all=C_all, S_all=S_all,
+    W = dict(layers=layers, whitened=whitened, G_all=G_all, Gh_all=Gh_all, C_all=C_all, S_all=S_all,
                 n_el=n_el, ews=ews, err=err, jobs=jobs,
                 n_wh=sum(L.d_out * L.d_in for L in wl), n_eu=sum(L.d_out * L.d_in for L in el),
                 packed_wh=ops.make_layers(wl), n_packed_wh=len(wl),
                 packed_eu=ops.make_layers(el), n_packed_eu=len(el))
+    W["sets"] = [dict(packed_wh=W["packed_wh"], packed_eu=W["packed_eu"],
+                      err_pairs=[(w["layer"].G, w["layer"].G_hat) for w in whitened], G_all=G_all, Gh_all=Gh_all,
+                      err=err)]
+    return W
 
 
 def nvfp4_measure(torch, ops, synth, dev, peak, reps=20):
@@ -258,28 +262,49 @@ def refresh_all(ops, W):
 PHASES = ("refresh", "encode_euclid", "encode_whitened", "decode_euclid", "decode_whitened", "error")
 
 
-def step(ops, W, k, ev=None):
+def step(ops, W, k, ev=None, S=None):
     """Step k: on every K_REFRESH-th step the batched refresh of all whitened
     layers; then encode and decode all 96 gradients (each codec phase is one
     grouped launch) and the round-trip error of one whitened layer.
-    If `ev` (len(PHASES)+1 events) is given, phase boundaries are recorded."""
-    w = W["whitened"][k % len(W["whitened"])]
-    rec = (lambda i: ev[i].record()) if ev else (lambda i: None)
+    If `ev` (len(PHASES)+1 events) is given, phase boundaries are recorded.
+    S selects the G / G_hat buffer set (default: the workload's own)."""
+    S = S or W["sets"][0]
+    i = k % len(W["whitened"])
+    rec = (lambda j: ev[j].record()) if ev else (lambda j: None)
     rec(0)
     if k % K_REFRESH == 0:
         refresh_all(ops, W)
     rec(1)
-    ops.encode_many(W["packed_eu"], W["n_packed_eu"])
+    ops.encode_many(S["packed_eu"], W["n_packed_eu"])
     rec(2)
-    ops.encode_many(W["packed_wh"], W["n_packed_wh"])
+    ops.encode_many(S["packed_wh"], W["n_packed_wh"])
     rec(3)
-    ops.decode_many(W["packed_eu"], W["n_packed_eu"])
+    ops.decode_many(S["packed_eu"], W["n_packed_eu"])
     rec(4)
-    ops.decode_many(W["packed_wh"], W["n_packed_wh"])
+    ops.decode_many(S["packed_wh"], W["n_packed_wh"])
     rec(5)
-    L = w["layer"]
-    ops.roundtrip_error(L.G, L.G_hat, out=W["err"], ws=W["ews"])
+    G, Gh = S["err_pairs"][i]
+    ops.roundtrip_error(G, Gh, out=S["err"], ws=W["ews"])
     rec(6)
+
+
+def buffer_set(ops, W, G_all, Gh_all):
+    import torch
+    """Layer descriptors of the stack over other G / G_hat buffers (same offsets,
+    shared codes, scales and factors)."""
+    import copy
+    layers, off = [], 0
+    for L in W["layers"]:
+        n = L.d_out * L.d_in
+        M = copy.copy(L)
+        M.G = G_all[off:off + n].view(L.d_out, L.d_in)
+        M.G_hat = Gh_all[off:off + n].view(L.d_out, L.d_in)
+        layers.append(M)
+        off += n
+    wl = [L for L in layers if L.rank > 0]
+    el = [L for L in layers if L.rank == 0]
+    return dict(packed_wh=ops.make_layers(wl), packed_eu=ops.make_layers(el),
+                err_pairs=[(L.G, L.G_hat) for L in wl], G_all=G_all, Gh_all=Gh_all, err=torch.empty_like(W["err"]))
 
 
 # DRAM traffic (read + write bytes per gradient element) of the whitened codec
@@ -451,37 +476,76 @@ def run_gpu(args):
     # all whitened layers copied in on refresh steps, and G_hat copied back ----
     e2e = None
     if not args.no_e2e:
+        # Through host buffers: every step's gradients come in from pinned host
+        # memory (and all activations on refresh steps), G_hat and the error go
+        # back.  Copies in, compute and copies out run on three streams over two
+        # device buffer sets, so step k+1's upload and step k-1's download
+        # overlap step k (PCIe is full duplex); every byte still crosses inside
+        # the timed region.
         G_host = torch.empty((W["n_el"],), dtype=torch.bfloat16, pin_memory=True)
         G_host.copy_(W["G_all"].cpu())
         Gh_host = torch.empty_like(G_host, pin_memory=True)
         X_host = [w["X"].cpu().pin_memory() for w in W["whitened"]]
         err_host = torch.empty((3,), dtype=torch.float64, pin_memory=True)
         x_bytes = sum(x.numel() * 2 for x in X_host)
+        if len(W["sets"]) < 2:
+            W["sets"].append(buffer_set(ops, W, torch.empty_like(W["G_all"]), torch.empty_like(W["Gh_all"])))
+        comp = torch.cuda.current_stream()
+        s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+        E = torch.cuda.Event
 
-        def e2e_step(k):
-            W["G_all"].copy_(G_host, non_blocking=True)
-            if k % K_REFRESH == 0:
-                for w, xh in zip(W["whitened"], X_host):
-                    w["X"].copy_(xh, non_blocking=True)
-            step(ops, W, k)
-            Gh_host.copy_(W["Gh_all"], non_blocking=True)
-            err_host.copy_(W["err"], non_blocking=True)
+        def run_e2e(ks):
+            done = {}     # k -> event: step k's compute finished (its G buffer is free)
+            out_done = {} # k -> event: step k's download finished (its G_hat buffer is free)
+            last_ref = None
+            for k in ks:
+                S = W["sets"][k % 2]
+                with torch.cuda.stream(s_in):
+                    if k - 2 in done:
+                        s_in.wait_event(done[k - 2])
+                    S["G_all"].copy_(G_host, non_blocking=True)
+                    if k % K_REFRESH == 0:
+                        if last_ref is not None:
+                            s_in.wait_event(last_ref)
+                        for w, xh in zip(W["whitened"], X_host):
+                            w["X"].copy_(xh, non_blocking=True)
+                    ev_in = E()
+                    ev_in.record(s_in)
+                comp.wait_event(ev_in)
+                if k - 2 in out_done:
+                    comp.wait_event(out_done[k - 2])
+                step(ops, W, k, S=S)
+                ev_c = E()
+                ev_c.record(comp)
+                done[k] = ev_c
+                if k % K_REFRESH == 0:
+                    last_ref = ev_c
+                with torch.cuda.stream(s_out):
+                    s_out.wait_event(ev_c)
+                    Gh_host.copy_(S["Gh_all"], non_blocking=True)
+                    err_host.copy_(S["err"], non_blocking=True)
+                    ev_o = E()
+                    ev_o.record(s_out)
+                out_done[k] = ev_o
+            return ev_o
 
-        e2e_step(1)
+        run_e2e(range(1, 3))
         torch.cuda.synchronize()
         barrier()
-        a = torch.cuda.Event(enable_timing=True)
-        b = torch.cuda.Event(enable_timing=True)
-        a.record()
-        for k in range(K):
-            e2e_step(k)
-        b.record()
+        a = E(enable_timing=True)
+        b = E(enable_timing=True)
+        a.record(comp)
+        s_in.wait_event(a)
+        last = run_e2e(range(K))
+        comp.wait_event(last)
+        b.record(comp)
         torch.cuda.synchronize()
         ms_e = max_over_ranks(a.elapsed_time(b), dev)
         n_ref = (K + K_REFRESH - 1) // K_REFRESH
         e2e = {"value": job_value(world, g_bytes, ms_e / K), "unit": UNIT,
                "h2d_bytes_per_step": int(g_bytes + n_ref * x_bytes / K), "d2h_bytes_per_step": int(g_bytes + 24),
-               "ms_per_step": ms_e / K}
+               "ms_per_step": ms_e / K,
+               "pipeline": "uploads, compute and downloads on three streams over two G / G_hat buffer sets"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
