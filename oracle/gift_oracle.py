@@ -368,7 +368,7 @@ def decode_e4m3(codes, scales, U, lam, rho, block: int = BLOCK_E4M3) -> np.ndarr
 # NVFP4 codec: E2M1 elements, E4M3 scale per 16 elements, fp32 tensor scale.
 # ---------------------------------------------------------------------------
 
-def quantize_nvfp4(W, block: int = BLOCK_NVFP4):
+def quantize_nvfp4(W, block: int = BLOCK_NVFP4, S_t=None):
     """Two-level NVFP4 quantisation of W (d_out x d_in), decisions in fp32.
 
     S_t = amax(W) / (6*448); per block b: s_b = E4M3(amax_b / (6*S_t));
@@ -377,12 +377,16 @@ def quantize_nvfp4(W, block: int = BLOCK_NVFP4):
     and all-zero element codes.
     Returns (codes packed two per byte, low nibble = even column;
     block scale codes uint8 [d_out, d_in/16]; tensor scale float32).
+    S_t, if given, is the tensor scale of a larger tensor whose rows W are.
     """
     W32 = np.asarray(W, dtype=np.float64).astype(_F32)
     d_out, d_in = W32.shape
     nb = d_in // block
-    amax_t = _F32(np.max(np.abs(W32))) if W32.size else _F32(0)
-    S_t = _F32(amax_t / _F32(6.0 * E4M3_MAX))
+    if S_t is None:
+        amax_t = _F32(np.max(np.abs(W32))) if W32.size else _F32(0)
+        S_t = _F32(amax_t / _F32(6.0 * E4M3_MAX))
+    else:  # rows of a larger tensor: its tensor scale is given
+        S_t = _F32(S_t)
     Wb = W32.reshape(d_out, nb, block)
     amax_b = np.max(np.abs(Wb), axis=2).astype(_F32)
     denom = _F32(_F32(6.0) * S_t)
