@@ -313,13 +313,13 @@ def buffer_set(ops, W, G_all, Gh_all):
 # that figure x its elements.  Valid only for the kernel source it was taken
 # on (sha256 of the file); otherwise the bench reports traffic as null.
 TRAFFIC = {
-    "encode_whitened": {"bytes_per_element": (201.38752e6 + 21.316352e6) / 69206016,
+    "encode_whitened": {"bytes_per_element": (201.215488e6 + 16.024064e6) / 69206016,
                         "profile": "profiles/whiten_encode_tc_stack8.md"},
-    "decode_whitened": {"bytes_per_element": (97.158656e6 + 83.8272e6) / 69206016,
+    "decode_whitened": {"bytes_per_element": (96.011264e6 + 79.978752e6) / 69206016,
                         "profile": "profiles/whiten_decode_tc_stack8.md"},
 }
 TRAFFIC_SOURCE = ("geometry_aware_fp8_b200/csrc/codec_tc.cu",
-                  "ccb4961a553802a9b90fdf98a127d2507b45044a055a60ded6ec50481cde3093")
+                  "287244caaa9383d3b936df0397543ddbb4392dec3482f5effe111b726df53718")
 
 
 def traffic_for(phase, n_elements):
