@@ -319,7 +319,7 @@ TRAFFIC = {
                         "profile": "profiles/whiten_decode_tc_stack8.md"},
 }
 TRAFFIC_SOURCE = ("geometry_aware_fp8_b200/csrc/codec_tc.cu",
-                  "287244caaa9383d3b936df0397543ddbb4392dec3482f5effe111b726df53718")
+                  "44fde76b4ef781b5768caf9d113e9b615ee04744c0a23358f06ea4f9ca3a34f3")
 
 
 def traffic_for(phase, n_elements):

@@ -601,7 +601,10 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
 // step order, hold a D2 step's f16 codes (the A operand, written by the
 // converter warps, free when the MMA completes) or a D3 step's bf16 output
 // (free once the TMA stores have read it).  A D3 stage is released as soon as
-// every epilogue thread has read its codes.
+// every epilogue thread has read its codes.  That release order also keeps
+// the converter warps, which wait on a scratch tile only in D2 steps, within
+// one phase of the tile's barrier: were D3 stages released at MMA completion,
+// the converters could run two uses ahead and pass a parity wait early.
 // ===========================================================================
 constexpr int kDStages = 4;                         // decode ring
 constexpr int kDCodes = kPanel * kChunk;            // 16 KB
