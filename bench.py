@@ -58,6 +58,7 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-nvfp4", action="store_true", help="skip the NVFP4 measurement on the 11008x4096 gradient")
+    ap.add_argument("--no-layers", action="store_true", help="skip the single-layer codec measurements")
     ap.add_argument("--depth", type=int, default=24, help="layers in the stack (24 = the full stand-in)")
     return ap.parse_args()
 
@@ -251,6 +252,61 @@ def nvfp4_measure(torch, ops, synth, dev, peak, reps=20):
         out[name] = {"encode_ms": enc, "decode_ms": dec, "gradient_gbs": gbs,
                      "roofline_frac": 2 * 2.5625 * n / ((enc + dec) * 1e-3) / 1e9 / peak,
                      "roundtrip_rel_error": float(err[0].item())}
+    return out
+
+
+def layers_measure(torch, ops, synth, dev, peak, reps=20):
+    """The whitened E4M3 codec called on one layer at a time (gift_encode then
+    gift_decode, G_hat in G's dtype), for the single-layer shapes: 512 x 512
+    fp32 (factor from 2048 fp32 tokens, G exponent 0.8), the 4096 x 1536 bf16
+    MLP up-projection stand-in and the largest shape, 11008 x 4096 bf16 (both
+    from 8192 bf16 tokens, exponent 1.0). One layer has d_out / 128 panels, so
+    a single call fills at most that many of the 148 SMs.
+    Algorithmic bytes per element each way: bytes(G) + 1 + 4/128."""
+    flush = torch.empty((256 << 20,), device=dev, dtype=torch.uint8)  # > L2 between timed calls
+
+    def timed(fn):
+        ts_ms = []
+        for i in range(reps + 3):
+            flush.zero_()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            if i >= 3:
+                ts_ms.append(a.elapsed_time(b))
+        return float(np.median(ts_ms))
+
+    out = {"workload": "one layer per call, rank-32 factor refreshed once (untimed); "
+                       "median of 20 calls, L2 flushed between calls"}
+    specs = (("512x512_f32", 512, 512, torch.float32, 2048, 0.8, 6001),
+             ("4096x1536_bf16", 4096, 1536, torch.bfloat16, REFRESH_N, 1.0, 6002),
+             ("11008x4096_bf16", 11008, 4096, torch.bfloat16, REFRESH_N, 1.0, 6003))
+    for name, d_out, d_in, dt, n_tok, expo, seed in specs:
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(seed)
+        Q = torch.from_numpy(synth.haar_orthogonal(d_in, seed + 10).astype(np.float32)).to(dev)
+        G = synth.device_gradient(d_out, d_in, expo, Q, gen, dt)
+        sigma = torch.arange(1, d_in + 1, device=dev, dtype=torch.float32) ** -1.0
+        X = synth.device_activations(n_tok, sigma, Q, gen, dt)
+        U, lam, rho, _ = ops.factor_refresh(X, RANK, OVERSAMPLE, ITERS, seed=seed + 20)
+        del X
+        codes = torch.empty((d_out, d_in), device=dev, dtype=torch.uint8)
+        scales = torch.empty((d_out, d_in // 128), device=dev, dtype=torch.float32)
+        Gh = torch.empty_like(G)
+        enc = timed(lambda: ops.encode(G, U, lam, rho, codes=codes, scales=scales))
+        dec = timed(lambda: ops.decode(codes, scales, U, lam, rho, out=Gh))
+        n = d_out * d_in
+        gb = G.element_size()
+        t = (enc + dec) * 1e-3
+        out[name] = {"encode_ms": enc, "decode_ms": dec, "gradient_gbs": gb * n / t / 1e9,
+                     "elements_per_s": n / t, "panels": (d_out + 127) // 128,
+                     "roofline_frac": 2 * (gb + 1 + 4 / 128) * n / t / 1e9 / peak}
+        del G, Gh, codes, scales
+    del flush
+    torch.cuda.empty_cache()
     return out
 
 
@@ -470,6 +526,7 @@ def run_gpu(args):
 
     launches, names = count_launches(torch, ops, W, K)
     nvfp4 = nvfp4_measure(torch, ops, synth, dev, peak) if not args.no_nvfp4 else None
+    single = layers_measure(torch, ops, synth, dev, peak) if not args.no_layers else None
 
     # ---- end to end through host buffers: the same schedule, with every
     # step's gradients copied in from pinned host memory, the activations of
@@ -559,7 +616,7 @@ def run_gpu(args):
                            "gradient_bytes": g_bytes, "storage": "bf16 G / e4m3 codes / fp32 scales",
                            "l2": "inputs larger than L2 (1.06 GB of gradients streamed per step)",
                            "parallelism": f"replicas x{world}"},
-                "roofline": roofline, "codec": codec, "nvfp4": nvfp4, "e2e": e2e, "cpu_baseline": cpu,
+                "roofline": roofline, "codec": codec, "layers": single, "nvfp4": nvfp4, "e2e": e2e, "cpu_baseline": cpu,
                 "gpu_launches": launches, "kernels": names, "clocks": clock_info}
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -227,6 +227,25 @@ static gift_status run_many(const gift_layer* layers, int n, gift_stream_t strea
   return GIFT_OK;
 }
 
+gift_status gift_codec_split(const gift_layer* layers, int n, int encode, int* split) {
+  if (!split || n < 0 || (n > 0 && !layers)) return GIFT_ERR_INVALID_ARG;
+  std::vector<TcLayer> tc;
+  for (int i = 0; i < n; ++i) {
+    const gift_layer& L = layers[i];
+    if (L.d_in < GIFT_E4M3_BLOCK || L.d_in % GIFT_E4M3_BLOCK != 0 || L.d_out < 0) return GIFT_ERR_SHAPE;
+    if (L.d_out > 0 && L.rank > 0 && use_tc(L.dtype, L.rank, L.d_in))
+      tc.push_back(TcLayer{L.G, L.G_hat, L.codes, L.scales, L.U, L.lambda, L.rho, (int)L.d_out, (int)L.d_in, L.rank});
+  }
+  *split = 0;
+  if (tc.empty()) return GIFT_OK;
+  gift_status st = device_ok();
+  if (st != GIFT_OK) return st;
+  const int S = tc_codec_split(tc.data(), (int)tc.size(), encode != 0);
+  if (S < 1) return GIFT_ERR_SHAPE;
+  *split = S;
+  return GIFT_OK;
+}
+
 gift_status gift_encode_many(const gift_layer* layers, int n, gift_stream_t stream) {
   return run_many(layers, n, stream, true);
 }

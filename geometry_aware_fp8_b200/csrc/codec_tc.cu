@@ -53,7 +53,9 @@ constexpr int kStageBytes = kGBytes + kUBytes;
 constexpr int kPcBytes = kPanel * 128;         // 16 KB: [128 rows][64 bf16]
 constexpr int kCodesBytes = kPanel * kChunk;    // 16 KB: codes of one chunk
 constexpr int kIdBytes = 16 * 128;             // 2 KB: 16 x 16 bf16 identity, 128-byte rows
+constexpr int kXBytes = kPanel * 32 * 4;        // 16 KB: fp32 partial projections exchanged in a cluster
 constexpr int kSmemBytes = kStages * kStageBytes + kPcBytes + 2 * kCodesBytes + kIdBytes + 1024 + 512;
+constexpr int enc_smem(bool cluster) { return kSmemBytes + (cluster ? kXBytes : 0); }
 constexpr int kThreads = 480;  // 8 epilogue + 4 converter + MMA + TMA load + TMA store warps
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColW0 = 0, kColW1 = 128, kColP = 256;
@@ -80,8 +82,9 @@ struct alignas(64) EncJob {
 
 struct EncParams {
   EncJob jobs[kMaxJobs];
-  uint16_t sched_off[kNumSMs + 1];  // CTA b runs sched_ids[sched_off[b] .. sched_off[b+1])
+  uint16_t sched_off[kNumSMs + 1];  // cluster b runs sched_ids[sched_off[b] .. sched_off[b+1])
   uint16_t sched_ids[kMaxPanels];   // job << 8 | panel
+  int split;                        // CTAs per cluster, each taking 1 / split of every panel's chunks
 };
 static_assert(sizeof(EncParams) <= 32760, "kernel parameter space");
 
@@ -133,14 +136,20 @@ GIFT_DEV void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "
 // (chunks 0 .. nc-1); block k >= 1 is the second pass of p_{k-1} (chunks
 // nc-1 .. 0) interleaved step by step with the first pass of p_k, so that the
 // HBM stream of one panel overlaps the epilogue work of the previous one.
+//
+// With a cluster of S CTAs sharing a panel list, CTA rank q runs chunks
+// [q nc / S, (q + 1) nc / S) of every panel (nc = d_in / 128 >= S); the step
+// counts and the local index below are over that range.
 template <class P>
 struct Steps {
   const P& p;
-  int beg, end, k;
+  int beg, end, k, q, S;
   int n1, n2, i1, i2;  // first- and second-pass steps of block k, and how many are done
   int pass;            // pass of the current step
-  GIFT_DEV Steps(const P& p_, int b, int e) : p(p_), beg(b), end(e), k(0) { setup(); }
-  GIFT_DEV int nc_of(int it) const { return p.jobs[p.sched_ids[it] >> 8].d_in / kChunk; }
+  GIFT_DEV Steps(const P& p_, int b, int e, int q_, int s_) : p(p_), beg(b), end(e), k(0), q(q_), S(s_) { setup(); }
+  GIFT_DEV int ncg_of(int it) const { return p.jobs[p.sched_ids[it] >> 8].d_in / kChunk; }
+  GIFT_DEV int lo_of(int it) const { return (q * ncg_of(it)) / S; }
+  GIFT_DEV int nc_of(int it) const { return ((q + 1) * ncg_of(it)) / S - lo_of(it); }
   GIFT_DEV void setup() {
     i1 = i2 = 0;
     n1 = beg + k < end ? nc_of(beg + k) : 0;
@@ -152,8 +161,9 @@ struct Steps {
   GIFT_DEV int slot() const { return pass ? beg + k - 1 : beg + k; }
   GIFT_DEV int job() const { return p.sched_ids[slot()] >> 8; }
   GIFT_DEV int panel() const { return p.sched_ids[slot()] & 255; }
-  GIFT_DEV int nc() const { return pass ? n2 : n1; }
-  GIFT_DEV int chunk() const { return pass ? n2 - 1 - i2 : i1; }
+  GIFT_DEV int nc() const { return pass ? n2 : n1; }                 // this CTA's chunks of the panel
+  GIFT_DEV int lidx() const { return pass ? i2 : i1; }                // step index within them
+  GIFT_DEV int chunk() const { return lo_of(slot()) + (pass ? n2 - 1 - i2 : i1); }  // chunk of d_in
   GIFT_DEV bool block_start() const { return i1 + i2 == 0; }
   GIFT_DEV void next() {
     if (pass)
@@ -192,6 +202,91 @@ GIFT_DEV uint4 ld_shared_v4(uint32_t addr) {
   asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
   return v;
 }
+
+// ---- thread-block clusters: the CTAs that split one panel's chunks ----
+GIFT_DEV uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Every thread of every CTA of the cluster (kernel start, after the barrier
+// inits, and kernel end, so no CTA leaves while a peer may still touch its
+// shared memory).
+GIFT_DEV void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Address of the same shared-memory location in cluster CTA `rank`.
+GIFT_DEV uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+GIFT_DEV void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+GIFT_DEV float4 ld_cluster_v4(uint32_t cluster_addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(cluster_addr)
+               : "memory");
+  return v;
+}
+GIFT_DEV bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, uint32_t limit) {
+  for (uint32_t i = 0; i < limit; ++i) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    if (ok) return true;
+  }
+  return false;
+}
+
+// Sum over the S CTAs of a cluster of one epilogue thread's 16 partial
+// projections (row r, coefficients 16 h .. 16 h + 15), added in cluster-rank
+// order so that every CTA of the cluster ends with the same fp32 sums.
+// xbuf is this CTA's [128][32] fp32 exchange tile; xfull (count 256 (S-1))
+// completes when every peer thread has written its partial, xempty (count
+// 256 (S-1)) when every peer thread has read this CTA's.  nx counts the
+// exchanges so far.  Returns false if a wait ran out.
+GIFT_DEV bool cluster_sum16(float (&v)[16], uint32_t xbuf, uint64_t* xfull, uint64_t* xempty, uint32_t& nx, int S,
+                            int q, int r, int h) {
+  if (nx >= 1 && !mbar_wait_cluster(xempty, (nx - 1) & 1u, kWaitLimit)) return false;
+  const uint32_t my = xbuf + (uint32_t)r * 128u + (uint32_t)h * 64u;
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    st_shared_v4(my + 16 * i, __float_as_uint(v[4 * i]), __float_as_uint(v[4 * i + 1]), __float_as_uint(v[4 * i + 2]),
+                 __float_as_uint(v[4 * i + 3]));
+  for (int t = 0; t < S; ++t)
+    if (t != q) mbar_arrive_remote(mapa_shared(smem_u32(xfull), t));
+  if (!mbar_wait_cluster(xfull, nx & 1u, kWaitLimit)) return false;
+  float sum[16];
+#pragma unroll
+  for (int k = 0; k < 16; ++k) sum[k] = 0.0f;
+  for (int t = 0; t < S; ++t) {
+    const uint32_t src = mapa_shared(my, t);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float4 w = ld_cluster_v4(src + 16 * i);
+      sum[4 * i] += w.x;
+      sum[4 * i + 1] += w.y;
+      sum[4 * i + 2] += w.z;
+      sum[4 * i + 3] += w.w;
+    }
+  }
+  for (int t = 0; t < S; ++t)
+    if (t != q) mbar_arrive_remote(mapa_shared(smem_u32(xempty), t));
+#pragma unroll
+  for (int k = 0; k < 16; ++k) v[k] = sum[k];
+  ++nx;
+  return true;
+}
+
 
 // Split fp32 into bf16 hi (RNE) and bf16 lo = RNE(x - hi).
 GIFT_DEV void split_bf16(float x, float& hi, float& lo) {
@@ -258,7 +353,7 @@ GIFT_DEV void convert_u_row_inplace_f16(uint32_t tile, int t) {
     st_shared_v4(tile + sw128(t, 4 + q), lo[4 * q], lo[4 * q + 1], lo[4 * q + 2], lo[4 * q + 3]);
 }
 
-template <int FMT>
+template <int FMT, bool CLUSTER>
 __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __grid_constant__ EncParams p,
                                                                      uint32_t* err) {
   extern __shared__ uint8_t smem_raw[];
@@ -267,7 +362,9 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
   const uint32_t pc_tile = sbase + kStages * kStageBytes;
   const uint32_t cbuf = pc_tile + kPcBytes;             // [2] codes tiles [128][128 B], 128-byte swizzle
   const uint32_t id_tile = cbuf + 2 * kCodesBytes;      // 16 x 16 identity, K-major, 128-byte swizzle
-  uint64_t* bars = (uint64_t*)(smem + kStages * kStageBytes + kPcBytes + 2 * kCodesBytes + kIdBytes);
+  const uint32_t xbuf = id_tile + kIdBytes;             // [128][32] fp32 partial P (CLUSTER only)
+  uint64_t* bars = (uint64_t*)(smem + kStages * kStageBytes + kPcBytes + 2 * kCodesBytes + kIdBytes +
+                               (CLUSTER ? kXBytes : 0));
   uint64_t* full = bars;                  // [kStages] count 1: converter (stage ready for the MMA)
   uint64_t* empty = bars + kStages;       // [kStages] count 1: MMA commit
   uint64_t* tfull = bars + 2 * kStages;   // [kStages] count 1 + tx: TMA (G and fp32 U)
@@ -277,11 +374,15 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
   uint64_t* w_empty = p_full + 4;         // [2] count 256
   uint64_t* cready = p_full + 6;          // [2] count 256: a codes tile is written
   uint64_t* cfree = p_full + 8;           // [2] count 1: the store of a codes tile has read it
-  uint32_t* tmem_slot = (uint32_t*)(p_full + 10);
+  uint64_t* xfull = p_full + 10;          // count 256 (S-1): the peers' partials are written (clusters)
+  uint64_t* xempty = p_full + 11;         // count 256 (S-1): the peers have read this CTA's partial
+  uint32_t* tmem_slot = (uint32_t*)(p_full + 12);
   __shared__ int failed;  // any role gave up (reported at exit)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int beg = p.sched_off[blockIdx.x], end = p.sched_off[blockIdx.x + 1];
+  const int S = CLUSTER ? p.split : 1;  // without clusters, the split arithmetic folds away
+  const int q = CLUSTER ? (int)cluster_ctarank() : 0;
+  const int beg = p.sched_off[blockIdx.x / S], end = p.sched_off[blockIdx.x / S + 1];
 
   if (threadIdx.x == 0) {
     failed = 0;
@@ -297,6 +398,10 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
       mbar_init(&w_empty[b], 256);
       mbar_init(&cready[b], 256);
       mbar_init(&cfree[b], 1);
+    }
+    if (CLUSTER) {
+      mbar_init(xfull, 256 * (S - 1));
+      mbar_init(xempty, 256 * (S - 1));
     }
     fence_mbar_init();
   }
@@ -319,6 +424,7 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (CLUSTER) cluster_sync_all();  // the peers' barriers are initialised before any remote arrive
   const uint32_t tbase = *tmem_slot;
 
   if (warp == 13) {
@@ -326,7 +432,7 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
     if (lane == 0) {
       const uint64_t keep = policy_evict_last(), drop = policy_evict_first();
       uint32_t step = 0;
-      for (Steps<EncParams> st(p, beg, end); st.valid() && !failed; st.next(), ++step) {
+      for (Steps<EncParams> st(p, beg, end, q, S); st.valid() && !failed; st.next(), ++step) {
         const int s = step % kStages;
         const uint32_t use = step / kStages;
         if (step >= kStages && !mbar_wait(&empty[s], (use - 1) & 1u, kWaitLimit)) {
@@ -347,7 +453,7 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
     if (lane == 0) {
       const uint64_t drop = policy_evict_first();
       uint32_t e2 = 0;
-      for (Steps<EncParams> st(p, beg, end); st.valid() && !failed; st.next()) {
+      for (Steps<EncParams> st(p, beg, end, q, S); st.valid() && !failed; st.next()) {
         if (st.pass == 0) continue;
         const int cb = e2 & 1;
         if (!mbar_wait(&cready[cb], (e2 >> 1) & 1u, kWaitLimit)) {
@@ -371,7 +477,7 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
     // at the same step.
     const int t = threadIdx.x - 256;
     uint32_t step = 0;
-    for (Steps<EncParams> st(p, beg, end); st.valid(); st.next(), ++step) {
+    for (Steps<EncParams> st(p, beg, end, q, S); st.valid(); st.next(), ++step) {
       const int s = step % kStages;
       const uint32_t use = step / kStages;
       const bool ok = mbar_wait(&tfull[s], use & 1u, kWaitLimit);
@@ -388,7 +494,7 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       uint32_t step = 0, e2 = 0;
-      for (Steps<EncParams> st(p, beg, end); st.valid() && !failed; st.next(), ++step) {
+      for (Steps<EncParams> st(p, beg, end, q, S); st.valid() && !failed; st.next(), ++step) {
         const int s = step % kStages;
         // block k >= 1 starts with the second pass of p_{k-1}: its P o (c/a) must be
         // in shared memory, and P in TMEM has been read (it is reused for p_k)
@@ -397,8 +503,8 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
         tc_fence_after();
         const uint32_t g_tile = sbase + s * kStageBytes, u_tile = g_tile + kGBytes;
         if (st.pass == 0) {
-          // E1: P2[128 x 64] += G_c . [U_hi | U_lo]_c
-          const int c = st.chunk();
+          // E1: P2[128 x 64] += G_c . [U_hi | U_lo]_c over this CTA's chunks
+          const int c = st.lidx();
 #pragma unroll
           for (int h = 0; h < 2; ++h)
 #pragma unroll
@@ -447,12 +553,12 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
     const int h = warp >> 2;
     const int r = (warp & 3) * 32 + lane;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    uint32_t e2 = 0;
+    uint32_t e2 = 0, nx = 0;
     float a = 0.0f;
     float S_t = 0.0f;   // NVFP4 tensor scale (codes pass)
     float pmax = 0.0f;  // NVFP4 amax pass: this thread's max |W'| over the panel
     bool stop = false;  // group vote: set for all 256 threads at the same barrier
-    for (Steps<EncParams> st(p, beg, end); st.valid() && !stop; st.next()) {
+    for (Steps<EncParams> st(p, beg, end, q, S); st.valid() && !stop; st.next()) {
       if (st.pass == 0) continue;  // first-pass steps are the MMA's alone
       const EncJob& J = p.jobs[st.job()];
       const int panel = st.panel();
@@ -478,11 +584,22 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
         tmem_ld16(tbase + lane_off + kColP + 16 * h, ph);
         tmem_ld16(tbase + lane_off + kColP + 32 + 16 * h, pl);
         tmem_wait_ld();
+        float pv[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) pv[k] = __uint_as_float(ph[k]) + __uint_as_float(pl[k]);
+        if (CLUSTER) {
+          // this CTA's chunks gave a partial P: the cluster sums the partials
+          stop = named_sync_or(2, 256, !cluster_sum16(pv, xbuf, xfull, xempty, nx, S, q, r, h));
+          if (stop) {
+            failed = 1;
+            break;
+          }
+        }
         uint32_t hi[8], lo[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-          const float v0 = (__uint_as_float(ph[2 * k]) + __uint_as_float(pl[2 * k])) * cf[2 * k];
-          const float v1 = (__uint_as_float(ph[2 * k + 1]) + __uint_as_float(pl[2 * k + 1])) * cf[2 * k + 1];
+          const float v0 = pv[2 * k] * cf[2 * k];
+          const float v1 = pv[2 * k + 1] * cf[2 * k + 1];
           float h0, l0, h1, l1;
           split_bf16(v0, h0, l0);
           split_bf16(v1, h1, l1);
@@ -583,6 +700,7 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
   }
   tc_fence_before();
   __syncthreads();
+  if (CLUSTER) cluster_sync_all();
   if (warp == 12) tmem_dealloc(tbase, kTmemCols);
   if (threadIdx.x == 0 && failed && err) atomicOr(err, GIFT_DEV_TIMEOUT);
 }
@@ -611,8 +729,9 @@ constexpr int kDCodes = kPanel * kChunk;            // 16 KB
 constexpr int kDStageBytes = kDCodes + kUBytes;     // codes + U
 constexpr int kDScratch = kPanel * kChunk * 2;      // 32 KB: two [128][64] 16-bit boxes
 constexpr int kDSmemBytes = kDStages * kDStageBytes + 2 * kDScratch + kPcBytes + 1024 + 512;
-static_assert(kDSmemBytes <= 232448, "decode shared memory");
-static_assert(kSmemBytes <= 232448, "encode shared memory");
+constexpr int dec_smem(bool cluster) { return kDSmemBytes + (cluster ? kXBytes : 0); }
+static_assert(dec_smem(true) <= 232448, "decode shared memory");
+static_assert(enc_smem(true) <= 232448, "encode shared memory");
 constexpr uint32_t kColT0 = 256, kColT1 = 320;
 constexpr uint32_t kIdescD2 = umma_idesc_f16(128, 64, 0, 1);   // D2 runs on f16 operands
 
@@ -632,8 +751,9 @@ struct alignas(64) DecJob {
 
 struct DecParams {
   DecJob jobs[kMaxJobs];
-  uint16_t sched_off[kNumSMs + 1];
-  uint16_t sched_ids[kMaxPanels];
+  uint16_t sched_off[kNumSMs + 1];  // cluster b runs sched_ids[sched_off[b] .. sched_off[b+1])
+  uint16_t sched_ids[kMaxPanels];   // job << 8 | panel
+  int split;                        // CTAs per cluster, each taking 1 / split of every panel's chunks
 };
 static_assert(sizeof(DecParams) <= 32760, "kernel parameter space");
 
@@ -644,7 +764,7 @@ GIFT_DEV uint32_t e4m3x2_to_f16x2(uint16_t v) {
   return h;
 }
 
-template <int FMT>
+template <int FMT, bool CLUSTER>
 __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __grid_constant__ DecParams p,
                                                                      uint32_t* err) {
   extern __shared__ uint8_t smem_raw[];
@@ -652,7 +772,8 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
   const uint32_t sbase = smem_u32(smem);
   const uint32_t scr = sbase + kDStages * kDStageBytes;  // [2] scratch tiles: two [128][64] 16-bit boxes each
   const uint32_t pc_tile = scr + 2 * kDScratch;
-  uint64_t* bars = (uint64_t*)(smem + kDStages * kDStageBytes + 2 * kDScratch + kPcBytes);
+  const uint32_t xbuf = pc_tile + kPcBytes;  // [128][32] fp32 partial P (CLUSTER only)
+  uint64_t* bars = (uint64_t*)(smem + kDStages * kDStageBytes + 2 * kDScratch + kPcBytes + (CLUSTER ? kXBytes : 0));
   uint64_t* full = bars;                   // [kDStages] count 1: converter (U split; first pass: codes widened)
   uint64_t* cfull = bars + kDStages;       // [kDStages] count 1 + tx: TMA (codes and U)
   uint64_t* empty = bars + 2 * kDStages;   // [kDStages] count 1: MMA commit (D2) or store warp (D3)
@@ -663,11 +784,15 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
   uint64_t* pc_full = t_full + 4;          // count 256
   uint64_t* w_full = t_full + 5;           // [2] count 1
   uint64_t* w_empty = t_full + 7;          // [2] count 256
-  uint32_t* tmem_slot = (uint32_t*)(t_full + 9);
+  uint64_t* xfull = t_full + 9;            // count 256 (S-1): the peers' partials are written (clusters)
+  uint64_t* xempty = t_full + 10;          // count 256 (S-1): the peers have read this CTA's partial
+  uint32_t* tmem_slot = (uint32_t*)(t_full + 11);
   __shared__ int failed;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int beg = p.sched_off[blockIdx.x], end = p.sched_off[blockIdx.x + 1];
+  const int S = CLUSTER ? p.split : 1;  // without clusters, the split arithmetic folds away
+  const int q = CLUSTER ? (int)cluster_ctarank() : 0;
+  const int beg = p.sched_off[blockIdx.x / S], end = p.sched_off[blockIdx.x / S + 1];
   if (threadIdx.x == 0) {
     failed = 0;
     for (int s = 0; s < kDStages; ++s) {
@@ -684,6 +809,10 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
       mbar_init(&w_empty[b], 256);
     }
     mbar_init(pc_full, 256);
+    if (CLUSTER) {
+      mbar_init(xfull, 256 * (S - 1));
+      mbar_init(xempty, 256 * (S - 1));
+    }
     fence_mbar_init();
   }
   if (warp == 12) {
@@ -693,6 +822,7 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (CLUSTER) cluster_sync_all();  // the peers' barriers are initialised before any remote arrive
   const uint32_t tbase = *tmem_slot;
 
   if (warp == 13) {
@@ -700,7 +830,7 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
     if (lane == 0) {
       const uint64_t keep = policy_evict_last(), drop = policy_evict_first();
       uint32_t step = 0;
-      for (Steps<DecParams> st(p, beg, end); st.valid() && !failed; st.next(), ++step) {
+      for (Steps<DecParams> st(p, beg, end, q, S); st.valid() && !failed; st.next(), ++step) {
         const int s = step % kDStages;
         const uint32_t use = step / kDStages;
         if (step >= kDStages && !mbar_wait(&empty[s], (use - 1) & 1u, kWaitLimit)) {
@@ -727,7 +857,7 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
     if (lane == 0) {
       const uint64_t drop = policy_evict_first();
       uint32_t step = 0, par = 0;  // par: bit j = phase parity of oready[j]
-      for (Steps<DecParams> st(p, beg, end); st.valid() && !failed; st.next(), ++step) {
+      for (Steps<DecParams> st(p, beg, end, q, S); st.valid() && !failed; st.next(), ++step) {
         if (st.pass == 0) continue;
         const int s = step % kDStages, j = step & 1;
         if (!mbar_wait(&oready[j], (par >> j) & 1u, kWaitLimit)) {
@@ -750,7 +880,7 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
     // ---------------- converters: U split in place; first pass: codes widened into a scratch tile ----------------
     const int t = threadIdx.x - 256;
     uint32_t step = 0;
-    for (Steps<DecParams> st(p, beg, end); st.valid(); st.next(), ++step) {
+    for (Steps<DecParams> st(p, beg, end, q, S); st.valid(); st.next(), ++step) {
       const int s = step % kDStages, j = step & 1;
       const uint32_t use = step / kDStages;
       bool ok = mbar_wait(&cfull[s], use & 1u, kWaitLimit);
@@ -819,7 +949,7 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       uint32_t step = 0, e2 = 0, d2 = 0;
-      for (Steps<DecParams> st(p, beg, end); st.valid() && !failed; st.next(), ++step) {
+      for (Steps<DecParams> st(p, beg, end, q, S); st.valid() && !failed; st.next(), ++step) {
         const int s = step % kDStages, j = step & 1;
         // block k >= 1 starts with D3 of p_{k-1}, which needs its P o c
         if (st.block_start() && st.k >= 1 && !mbar_wait(pc_full, (st.k - 1) & 1u, kWaitLimit)) { failed = 1; break; }
@@ -873,24 +1003,32 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
     const int h = warp >> 2;
     const int r = (warp & 3) * 32 + lane;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    uint32_t step = 0, e2 = 0, d2 = 0;
+    uint32_t step = 0, e2 = 0, d2 = 0, nx = 0;
     float P[16];
 #pragma unroll
     for (int k = 0; k < 16; ++k) P[k] = 0.0f;
     float a = 0.0f;
     bool stop = false;
-    for (Steps<DecParams> st(p, beg, end); st.valid() && !stop; st.next(), ++step) {
+    for (Steps<DecParams> st(p, beg, end, q, S); st.valid() && !stop; st.next(), ++step) {
       const int s = step % kDStages, j = step & 1;
       const DecJob& J = p.jobs[st.job()];
-      const int nc = st.nc(), c = st.chunk();
+      const int nc = J.d_in / kChunk, c = st.chunk();
       const int64_t row = (int64_t)st.panel() * kPanel + r;
       const bool live = row < J.d_out;
       // E4M3: the chunk's fp32 block scale; NVFP4: the tensor scale (the block
       // scales are inside the widened values)
       const float sc = !live ? 0.0f : (FMT == kFmtE4M3 ? __ldg(J.scales + row * nc + c) : __ldg(J.tscale));
       if (st.block_start() && st.k >= 1) {
-        // P of p_{k-1} is complete: P o c -> bf16 hi/lo A operand of D3
+        // P of p_{k-1} is complete (in a cluster: this CTA's chunks of it,
+        // summed over the cluster here): P o c -> bf16 hi/lo A operand of D3
         // (this half's 16 of the 32 columns of each part)
+        if (CLUSTER) {
+          stop = named_sync_or(2, 256, !cluster_sum16(P, xbuf, xfull, xempty, nx, S, q, r, h));
+          if (stop) {
+            failed = 1;
+            break;
+          }
+        }
         const double rho = (double)__ldg(J.rho);
         const double a64 = sqrt(rho);
         a = (float)a64;
@@ -915,7 +1053,7 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
       }
       if (st.pass == 0) {
         // D2 epilogue: P += s_c (T_hi + 2^-11 T_lo) for this half's 16 coefficients
-        if (c == 0) {
+        if (st.lidx() == 0) {
 #pragma unroll
           for (int k = 0; k < 16; ++k) P[k] = 0.0f;
         }
@@ -1007,102 +1145,242 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
   }
   tc_fence_before();
   __syncthreads();
+  if (CLUSTER) cluster_sync_all();
   if (warp == 12) tmem_dealloc(tbase, kTmemCols);
   if (threadIdx.x == 0 && failed && err) atomicOr(err, GIFT_DEV_TIMEOUT);
 }
 
-unsigned long long g_dec_attr[3] = {0, 0, 0};
-unsigned long long g_enc_attr[3] = {0, 0, 0};
+unsigned long long g_dec_attr[3][2] = {};
+unsigned long long g_enc_attr[3][2] = {};
+
+// One launch of `grid` clusters of S CTAs (S = 1: a plain launch).
+template <class Prm>
+cudaError_t launch_clusters(void (*kern)(Prm, uint32_t*), int smem, unsigned long long* attr, int grid, int S,
+                            const Prm& P, cudaStream_t s) {
+  cudaError_t e = ensure_smem_attr(kern, smem, attr);
+  if (e != cudaSuccess) return e;
+  if (S == 1) {
+    kern<<<grid, kThreads, smem, s>>>(P, nullptr);
+    return cudaGetLastError();
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(grid * S));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = (size_t)smem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = (unsigned)S;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, P, (uint32_t*)nullptr);
+}
+
+// Clusters of S CTAs of this kernel that can be resident at once (0 if none).
+template <class Prm>
+int cluster_slots(void (*kern)(Prm, uint32_t*), int smem, unsigned long long* attr, int S, int* cache) {
+  int& c = cache[S >> 2];  // S = 2 -> [0], S = 4 -> [1]
+  if (c >= 0) return c;
+  if (ensure_smem_attr(kern, smem, attr) != cudaSuccess) return c = 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(S * kNumSMs));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = (size_t)smem;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = (unsigned)S;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    n = 0;
+  }
+  return c = std::min(n, kNumSMs);
+}
+
+int g_enc_slots[3][2] = {{-1, -1}, {-1, -1}, {-1, -1}};
+int g_dec_slots[3][2] = {{-1, -1}, {-1, -1}, {-1, -1}};
+
+int enc_slots(int fmt, int S) {
+  if (S == 1) return kNumSMs;
+  constexpr int m = enc_smem(true);
+  switch (fmt) {
+    case kFmtE4M3: return cluster_slots(whiten_encode_tc_kernel<kFmtE4M3, true>, m, &g_enc_attr[0][1], S, g_enc_slots[0]);
+    case kFmtNvfp4Amax:
+      return cluster_slots(whiten_encode_tc_kernel<kFmtNvfp4Amax, true>, m, &g_enc_attr[1][1], S, g_enc_slots[1]);
+    case kFmtNvfp4: return cluster_slots(whiten_encode_tc_kernel<kFmtNvfp4, true>, m, &g_enc_attr[2][1], S, g_enc_slots[2]);
+    default: return 0;
+  }
+}
+
+int dec_slots(int fmt, int S) {
+  if (S == 1) return kNumSMs;
+  constexpr int m = dec_smem(true);
+  switch (fmt) {
+    case kFmtE4M3: return cluster_slots(whiten_decode_tc_kernel<kFmtE4M3, true>, m, &g_dec_attr[0][1], S, g_dec_slots[0]);
+    case kFmtNvfp4: return cluster_slots(whiten_decode_tc_kernel<kFmtNvfp4, true>, m, &g_dec_attr[2][1], S, g_dec_slots[2]);
+    default: return 0;
+  }
+}
+
+template <int FMT>
+cudaError_t enc_launch_fmt(int grid, const EncParams& P, cudaStream_t s) {
+  const int f = FMT == kFmtE4M3 ? 0 : FMT == kFmtNvfp4Amax ? 1 : 2;
+  if (P.split > 1)
+    return launch_clusters(whiten_encode_tc_kernel<FMT, true>, enc_smem(true), &g_enc_attr[f][1], grid, P.split, P, s);
+  return launch_clusters(whiten_encode_tc_kernel<FMT, false>, enc_smem(false), &g_enc_attr[f][0], grid, 1, P, s);
+}
+
+template <int FMT>
+cudaError_t dec_launch_fmt(int grid, const DecParams& P, cudaStream_t s) {
+  const int f = FMT == kFmtE4M3 ? 0 : 2;
+  if (P.split > 1)
+    return launch_clusters(whiten_decode_tc_kernel<FMT, true>, dec_smem(true), &g_dec_attr[f][1], grid, P.split, P, s);
+  return launch_clusters(whiten_decode_tc_kernel<FMT, false>, dec_smem(false), &g_dec_attr[f][0], grid, 1, P, s);
+}
 
 // One launch runs layers of one format (its kernel instantiation).
 cudaError_t enc_launch(int fmt, int grid, const EncParams& P, cudaStream_t s) {
-  cudaError_t e;
   switch (fmt) {
-    case kFmtE4M3:
-      if ((e = ensure_smem_attr(whiten_encode_tc_kernel<kFmtE4M3>, kSmemBytes, &g_enc_attr[0])) != cudaSuccess) return e;
-      whiten_encode_tc_kernel<kFmtE4M3><<<grid, kThreads, kSmemBytes, s>>>(P, nullptr);
-      break;
-    case kFmtNvfp4Amax:
-      if ((e = ensure_smem_attr(whiten_encode_tc_kernel<kFmtNvfp4Amax>, kSmemBytes, &g_enc_attr[1])) != cudaSuccess)
-        return e;
-      whiten_encode_tc_kernel<kFmtNvfp4Amax><<<grid, kThreads, kSmemBytes, s>>>(P, nullptr);
-      break;
-    case kFmtNvfp4:
-      if ((e = ensure_smem_attr(whiten_encode_tc_kernel<kFmtNvfp4>, kSmemBytes, &g_enc_attr[2])) != cudaSuccess) return e;
-      whiten_encode_tc_kernel<kFmtNvfp4><<<grid, kThreads, kSmemBytes, s>>>(P, nullptr);
-      break;
-    default:
-      return cudaErrorInvalidValue;
+    case kFmtE4M3: return enc_launch_fmt<kFmtE4M3>(grid, P, s);
+    case kFmtNvfp4Amax: return enc_launch_fmt<kFmtNvfp4Amax>(grid, P, s);
+    case kFmtNvfp4: return enc_launch_fmt<kFmtNvfp4>(grid, P, s);
+    default: return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
 }
 
 cudaError_t dec_launch(int fmt, int grid, const DecParams& P, cudaStream_t s) {
-  cudaError_t e;
   switch (fmt) {
-    case kFmtE4M3:
-      if ((e = ensure_smem_attr(whiten_decode_tc_kernel<kFmtE4M3>, kDSmemBytes, &g_dec_attr[0])) != cudaSuccess) return e;
-      whiten_decode_tc_kernel<kFmtE4M3><<<grid, kThreads, kDSmemBytes, s>>>(P, nullptr);
-      break;
-    case kFmtNvfp4:
-      if ((e = ensure_smem_attr(whiten_decode_tc_kernel<kFmtNvfp4>, kDSmemBytes, &g_dec_attr[2])) != cudaSuccess)
-        return e;
-      whiten_decode_tc_kernel<kFmtNvfp4><<<grid, kThreads, kDSmemBytes, s>>>(P, nullptr);
-      break;
-    default:
-      return cudaErrorInvalidValue;
+    case kFmtE4M3: return dec_launch_fmt<kFmtE4M3>(grid, P, s);
+    case kFmtNvfp4: return dec_launch_fmt<kFmtNvfp4>(grid, P, s);
+    default: return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
 }
 
-// Longest-processing-time-first assignment of panels to CTAs.
-int schedule(const TcLayer* layers, int n, uint16_t* off, uint16_t* ids, int max_ids) {
-  struct Item {
-    int cost;
-    uint16_t id;
-  };
-  std::vector<Item> items;
+// Longest-processing-time-first assignment of panels to `slots` clusters of S
+// CTAs (S = 1: single CTAs).  A panel costs each CTA of its cluster at most
+// ceil(nc / S) steps per pass.  Returns the clusters used (or -1) and the
+// largest per-cluster cost in *makespan; off / ids are written only if given.
+int schedule(const TcLayer* layers, int n, uint16_t* off, uint16_t* ids, int max_ids, int slots, int S,
+             long* makespan) {
+  static thread_local std::vector<std::pair<int, uint16_t>> items;  // (cost, id), reused across calls
+  static thread_local std::vector<int> owner;
+  items.clear();
   for (int l = 0; l < n; ++l) {
     const int np = (layers[l].d_out + kPanel - 1) / kPanel;
-    for (int q = 0; q < np; ++q) items.push_back({layers[l].d_in / kChunk, (uint16_t)((l << 8) | q)});
+    const int nc = layers[l].d_in / kChunk;
+    for (int q = 0; q < np; ++q) items.push_back({(nc + S - 1) / S, (uint16_t)((l << 8) | q)});
   }
-  if ((int)items.size() > max_ids) return -1;
-  std::stable_sort(items.begin(), items.end(), [](const Item& x, const Item& y) { return x.cost > y.cost; });
-  const int grid = std::min<int>(kNumSMs, (int)items.size());
-  std::vector<std::vector<uint16_t>> per(grid);
+  if ((int)items.size() > max_ids || slots <= 0) return -1;
+  std::stable_sort(items.begin(), items.end(),
+                   [](const std::pair<int, uint16_t>& x, const std::pair<int, uint16_t>& y) { return x.first > y.first; });
+  const int grid = std::min<int>(slots, (int)items.size());
   using E = std::pair<long, int>;
   std::priority_queue<E, std::vector<E>, std::greater<E>> heap;
   for (int b = 0; b < grid; ++b) heap.push({0, b});
-  for (const Item& it : items) {
+  owner.resize(items.size());
+  long worst = 0;
+  for (size_t i = 0; i < items.size(); ++i) {
     E e = heap.top();
     heap.pop();
-    per[e.second].push_back(it.id);
-    heap.push({e.first + it.cost, e.second});
+    owner[i] = e.second;
+    worst = std::max(worst, e.first + items[i].first);
+    heap.push({e.first + items[i].first, e.second});
   }
-  int k = 0;
-  for (int b = 0; b < grid; ++b) {
-    off[b] = (uint16_t)k;
-    for (uint16_t id : per[b]) ids[k++] = id;
+  if (makespan) *makespan = worst;
+  if (off && ids) {
+    // cluster b's panels, in the longest-first order they were assigned
+    std::vector<int> cnt(grid + 1, 0);
+    for (int o : owner) ++cnt[o + 1];
+    for (int b = 0; b < grid; ++b) cnt[b + 1] += cnt[b];
+    for (int b = 0; b <= grid; ++b) off[b] = (uint16_t)cnt[b];
+    for (size_t i = 0; i < items.size(); ++i) ids[cnt[owner[i]]++] = items[i].second;
   }
-  off[grid] = (uint16_t)k;
   return grid;
+}
+
+// Cluster size for a launch.  A CTA that owns a panel runs 2 nc chunk steps
+// (both passes); with a cluster of S CTAs per panel it runs 2 ceil(nc / S),
+// plus a fixed cost of the cluster launch and the partial-P exchange that
+// measured, on B200, about as long as kSplitCost[S] chunk steps.  A split is
+// taken only when every cluster gets at most one panel (a second panel would
+// repeat the exchange and the pipeline refill) and it is at least a tenth
+// faster by that estimate; a launch of many panels keeps single CTAs.
+constexpr int kSplitCost2 = 6, kSplitCost4 = 15;
+
+template <class SlotFn>
+int plan(const TcLayer* layers, int n, uint16_t* off, uint16_t* ids, int max_ids, SlotFn slots_for, int* split) {
+  int min_nc = 1 << 30, max_nc = 0, panels = 0;
+  for (int l = 0; l < n; ++l) {
+    min_nc = std::min(min_nc, layers[l].d_in / kChunk);
+    max_nc = std::max(max_nc, layers[l].d_in / kChunk);
+    panels += (layers[l].d_out + kPanel - 1) / kPanel;
+  }
+  int best_s = 1;
+  if (panels < kNumSMs) {
+    const long est1 = 2L * max_nc;
+    long best = est1;
+    for (int S : {2, 4}) {
+      if (S > min_nc) break;
+      const int slots = slots_for(S);
+      if (slots <= 0 || panels > slots) continue;
+      const long est = 2L * ((max_nc + S - 1) / S) + (S == 2 ? kSplitCost2 : kSplitCost4);
+      if (10 * est < 9 * est1 && est < best) {
+        best = est;
+        best_s = S;
+      }
+    }
+  }
+  *split = best_s;
+  return schedule(layers, n, off, ids, max_ids, best_s == 1 ? kNumSMs : slots_for(best_s), best_s, nullptr);
 }
 
 }  // namespace
 
 bool tc_codec_available() { return tmap_encoder() != nullptr; }
 
+// Layers [0, cnt) of one launch: the same format, at most kMaxJobs layers and
+// kMaxPanels panels, each layer at most 256 panels (0: the first layer is
+// larger and is coded in parts of 256 panels).
+static int group_count(const TcLayer* layers, int n) {
+  int cnt = 0, panels = 0;
+  while (cnt < n && cnt < kMaxJobs && layers[cnt].fmt == layers[0].fmt) {
+    const int np = (layers[cnt].d_out + kPanel - 1) / kPanel;
+    if (np > 256 || panels + np > kMaxPanels) break;
+    panels += np;
+    ++cnt;
+  }
+  return cnt;
+}
+
+int tc_codec_split(const TcLayer* layers, int n, bool encode) {
+  if (n <= 0) return -1;
+  TcLayer part = layers[0];
+  const TcLayer* g = layers;
+  int cnt = group_count(layers, n);
+  if (cnt == 0) {
+    part.d_out = std::min(part.d_out, 256 * kPanel);
+    g = &part;
+    cnt = 1;
+  }
+  static thread_local uint16_t off[kNumSMs + 1], ids[kMaxPanels];
+  const int fmt = g[0].fmt;
+  int S = 1;
+  const int grid = encode ? plan(g, cnt, off, ids, kMaxPanels, [fmt](int k) { return enc_slots(fmt, k); }, &S)
+                          : plan(g, cnt, off, ids, kMaxPanels, [fmt](int k) { return dec_slots(fmt, k); }, &S);
+  return grid <= 0 ? -1 : S;
+}
+
 cudaError_t launch_whiten_encode_tc(const TcLayer* layers, int n, cudaStream_t s) {
   cudaError_t e = cudaSuccess;
   for (int base = 0; base < n;) {
     // pack as many layers as fit one launch
-    int cnt = 0, panels = 0;
-    while (base + cnt < n && cnt < kMaxJobs && layers[base + cnt].fmt == layers[base].fmt) {
-      const int np = (layers[base + cnt].d_out + kPanel - 1) / kPanel;
-      if (np > 256 || panels + np > kMaxPanels) break;
-      panels += np;
-      ++cnt;
-    }
+    const int cnt = group_count(layers + base, n - base);
     if (cnt == 0) {
       // a single layer with more than 256 panels: split it by rows
       const TcLayer& L = layers[base];
@@ -1145,9 +1423,11 @@ cudaError_t launch_whiten_encode_tc(const TcLayer* layers, int n, cudaStream_t s
       J.d_in = L.d_in;
       J.rank = L.rank;
     }
-    const int grid = schedule(layers + base, cnt, P.sched_off, P.sched_ids, kMaxPanels);
+    const int fmt = layers[base].fmt;
+    const int grid = plan(layers + base, cnt, P.sched_off, P.sched_ids, kMaxPanels,
+                          [fmt](int S) { return enc_slots(fmt, S); }, &P.split);
     if (grid <= 0) return cudaErrorInvalidValue;
-    if ((e = enc_launch(layers[base].fmt, grid, P, s)) != cudaSuccess) return e;
+    if ((e = enc_launch(fmt, grid, P, s)) != cudaSuccess) return e;
     base += cnt;
   }
   return cudaSuccess;
@@ -1158,13 +1438,7 @@ cudaError_t launch_whiten_encode_tc(const TcLayer* layers, int n, cudaStream_t s
 cudaError_t launch_whiten_decode_tc(const TcLayer* layers, int n, cudaStream_t s) {
   cudaError_t e = cudaSuccess;
   for (int base = 0; base < n;) {
-    int cnt = 0, panels = 0;
-    while (base + cnt < n && cnt < kMaxJobs && layers[base + cnt].fmt == layers[base].fmt) {
-      const int np = (layers[base + cnt].d_out + kPanel - 1) / kPanel;
-      if (np > 256 || panels + np > kMaxPanels) break;
-      panels += np;
-      ++cnt;
-    }
+    const int cnt = group_count(layers + base, n - base);
     if (cnt == 0) {
       const TcLayer& L = layers[base];
       const int rows = 256 * kPanel;
@@ -1206,9 +1480,11 @@ cudaError_t launch_whiten_decode_tc(const TcLayer* layers, int n, cudaStream_t s
       J.d_in = L.d_in;
       J.rank = L.rank;
     }
-    const int grid = schedule(layers + base, cnt, P.sched_off, P.sched_ids, kMaxPanels);
+    const int fmt = layers[base].fmt;
+    const int grid = plan(layers + base, cnt, P.sched_off, P.sched_ids, kMaxPanels,
+                          [fmt](int S) { return dec_slots(fmt, S); }, &P.split);
     if (grid <= 0) return cudaErrorInvalidValue;
-    if ((e = dec_launch(layers[base].fmt, grid, P, s)) != cudaSuccess) return e;
+    if ((e = dec_launch(fmt, grid, P, s)) != cudaSuccess) return e;
     base += cnt;
   }
   return cudaSuccess;

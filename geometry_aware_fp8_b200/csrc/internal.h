@@ -57,6 +57,10 @@ constexpr int kFmtE4M3 = 0, kFmtNvfp4Amax = 1, kFmtNvfp4 = 2;
 bool tc_codec_available();
 cudaError_t launch_whiten_encode_tc(const TcLayer* layers, int n, cudaStream_t s);
 cudaError_t launch_whiten_decode_tc(const TcLayer* layers, int n, cudaStream_t s);
+// Cluster size (1, 2 or 4) the tensor-core codec plans for the first launch
+// over these layers (-1 if they cannot be planned).  Host-side; queries the
+// device's cluster occupancy once per kernel.
+int tc_codec_split(const TcLayer* layers, int n, bool encode);
 
 // ---- Round-trip error ----
 size_t error_ws_bytes(int64_t n_elems);

@@ -26,7 +26,8 @@ STATUS = {0: "GIFT_OK", 1: "GIFT_ERR_INVALID_ARG", 2: "GIFT_ERR_SHAPE", 3: "GIFT
 
 EXPORTED = ("gift_status_string", "gift_version", "gift_refresh_workspace_size", "gift_factor_refresh",
             "gift_factor_refresh_noalloc", "gift_factor_refresh_many", "gift_encode", "gift_decode", "gift_encode_many", "gift_decode_many",
-            "gift_error_workspace_size", "gift_roundtrip_error", "gift_encode_nvfp4", "gift_decode_nvfp4")
+            "gift_error_workspace_size", "gift_roundtrip_error", "gift_encode_nvfp4", "gift_decode_nvfp4",
+            "gift_codec_split")
 
 
 class GiftError(RuntimeError):
@@ -77,6 +78,7 @@ def lib() -> ctypes.CDLL:
         L.gift_decode.argtypes = [vp, vp, i64, i64, vp, vp, vp, i32, vp, i32, vp]
         L.gift_encode_many.argtypes = [ctypes.POINTER(Layer), i32, vp]
         L.gift_decode_many.argtypes = [ctypes.POINTER(Layer), i32, vp]
+        L.gift_codec_split.argtypes = [ctypes.POINTER(Layer), i32, i32, ctypes.POINTER(i32)]
         L.gift_error_workspace_size.argtypes = [i64, i64, ctypes.POINTER(sz)]
         L.gift_roundtrip_error.argtypes = [vp, vp, i32, i64, i64, vp, vp, sz, vp]
         L.gift_encode_nvfp4.argtypes = [vp, i32, i64, i64, vp, vp, vp, i32, vp, vp, vp, vp]
@@ -297,6 +299,14 @@ def encode_many(packed, n: int, stream=None):
 
 def decode_many(packed, n: int, stream=None):
     _check(lib().gift_decode_many(packed, n, _stream(stream)), "gift_decode_many")
+
+
+def codec_split(packed, n: int, encode: bool = True) -> int:
+    """CTAs per 128-row panel (1, 2 or 4; 0 if no layer takes the tensor-core
+    path) that the whitened codec plans for its first launch over these layers."""
+    out = ctypes.c_int32(-1)
+    _check(lib().gift_codec_split(packed, n, 1 if encode else 0, ctypes.byref(out)), "gift_codec_split")
+    return out.value
 
 
 def error_workspace_size(d_out: int, d_in: int) -> int:

@@ -210,6 +210,24 @@ gift_status gift_encode_many(const gift_layer* layers /* host */, int n, gift_st
 gift_status gift_decode_many(const gift_layer* layers /* host */, int n, gift_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * Planning query (launches nothing, reads no pointer of `layers`): how the
+ * tensor-core whitened codec lays out its first launch over these layers.
+ * A 128-row panel is one CTA's work in the pages' per-layer round trip; when
+ * a launch holds too few panels to fill the GPU (a single layer, say), the
+ * codec gives each panel to a thread-block cluster of 2 or 4 CTAs that split
+ * its 128-column chunks and add their partial projections G U (decode: W_hat
+ * U) in cluster-rank order.  The pages have no counterpart: this is a layout
+ * decision of this implementation.
+ *   encode: nonzero for the encoder's plan, 0 for the decoder's.
+ *   *split (host): 1, 2 or 4, or 0 if no layer takes the tensor-core path
+ *   (bf16, rank 32, d_in <= 8192).
+ * Errors: GIFT_ERR_INVALID_ARG (null split, n < 0, null layers with n > 0),
+ * GIFT_ERR_SHAPE (d_in not a positive multiple of 128, d_out < 0),
+ * GIFT_ERR_CUDA (no usable device).
+ * ------------------------------------------------------------------------ */
+gift_status gift_codec_split(const gift_layer* layers /* host */, int n, int encode, int* split /* host */);
+
+/* ------------------------------------------------------------------------
  * One-step round-trip error (Tables I-II: relative reconstruction error of
  * the FP8 round trip against the full-precision gradient).
  *

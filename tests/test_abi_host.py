@@ -153,3 +153,17 @@ def test_product_path_has_no_oracle_import():
             if f.endswith((".py", ".cu", ".cuh", ".h")):
                 txt = open(os.path.join(dirpath, f)).read()
                 assert not pat.search(txt), f
+
+
+def test_codec_split_rejects_bad_arguments(L):
+    import torch
+    out = ctypes.c_int(-1)
+    eu = ops.make_layers([ops.LayerArgs(d_out=256, d_in=256, rank=0, dtype=torch.bfloat16)])
+    assert L.gift_codec_split(eu, 1, 1, None) == INVALID
+    assert L.gift_codec_split(None, 1, 1, ctypes.byref(out)) == INVALID
+    assert L.gift_codec_split(eu, -1, 1, ctypes.byref(out)) == INVALID
+    bad = ops.make_layers([ops.LayerArgs(d_out=256, d_in=200, rank=32, dtype=torch.bfloat16)])
+    assert L.gift_codec_split(bad, 1, 1, ctypes.byref(out)) == SHAPE
+    # no layer on the tensor-core path (Euclidean): nothing to plan, no device needed
+    assert L.gift_codec_split(eu, 1, 0, ctypes.byref(out)) == OK and out.value == 0
+    assert L.gift_codec_split(eu, 0, 1, ctypes.byref(out)) == OK and out.value == 0
