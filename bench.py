@@ -369,13 +369,13 @@ def buffer_set(ops, W, G_all, Gh_all):
 # that figure x its elements.  Valid only for the kernel source it was taken
 # on (sha256 of the file); otherwise the bench reports traffic as null.
 TRAFFIC = {
-    "encode_whitened": {"bytes_per_element": (201.215488e6 + 16.024064e6) / 69206016,
+    "encode_whitened": {"bytes_per_element": (201.796864e6 + 21.118976e6) / 69206016,
                         "profile": "profiles/whiten_encode_tc_stack8.md"},
-    "decode_whitened": {"bytes_per_element": (96.011264e6 + 79.978752e6) / 69206016,
+    "decode_whitened": {"bytes_per_element": (96.061952e6 + 80.016384e6) / 69206016,
                         "profile": "profiles/whiten_decode_tc_stack8.md"},
 }
 TRAFFIC_SOURCE = ("geometry_aware_fp8_b200/csrc/codec_tc.cu",
-                  "44fde76b4ef781b5768caf9d113e9b615ee04744c0a23358f06ea4f9ca3a34f3")
+                  "36ce1421959db85fb7c3903ecc5d458e5c8bba6e6485a7eac2bacff6df6aafc2")
 
 
 def traffic_for(phase, n_elements):

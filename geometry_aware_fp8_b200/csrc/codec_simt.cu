@@ -4,19 +4,22 @@
 // quantiser, G_hat = W_hat M^{-1} after it, with
 //   M^{-+1} = a I + U diag(c) U^T   (a = rho^{-+1/2},
 //                                    c_k = (lambda_k+rho)^{-+1/2} - a).
-// One warp owns one row of G; each lane holds four consecutive elements of
-// every 128-element block, so one warp step covers exactly one scale block.
-// Pass 1 forms P = g U (32 partial dot products per lane, then a butterfly
-// reduction); pass 2 forms w = a g + (P o c) U^T, the block maximum with
-// five shuffles, and the codes.  This kernel serves fp32 gradients and any
-// rank; the tensor-core kernel (codec_tc.cu) serves bf16 gradients.
+// One CTA owns one row of G; its warps take the row's 128-element scale
+// blocks in turn (warp w: blocks w, w + 8, ...), and each lane holds four
+// consecutive elements of a block.  Pass 1 forms each warp's share of
+// P = g U (32 partial dot products per lane), reduces it across the lanes
+// with a 31-shuffle transpose (lane k ends with coefficient k) and across the
+// warps in warp order through shared memory; pass 2 forms w = a g +
+// (P o c) U^T, the block maximum with five shuffles, and the codes.  This
+// kernel serves fp32 gradients and ranks other than 32; the tensor-core
+// kernel (codec_tc.cu) serves bf16 gradients at rank 32.
 #include "common.cuh"
 #include "internal.h"
 
 namespace gift {
 namespace {
 
-constexpr int kWarps = 8;
+constexpr int kWarps = 8;  // per CTA; one CTA per row
 
 template <typename T>
 GIFT_DEV void load4(const T* p, float (&v)[4]);
@@ -41,10 +44,60 @@ GIFT_DEV void store4<__nv_bfloat16>(__nv_bfloat16* p, const float (&v)[4]) {
   *reinterpret_cast<uint2*>(p) = make_uint2(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]));
 }
 
-// Butterfly sum of the 32 per-lane partial projections.
-GIFT_DEV void project_row_reduce(float (&P)[32]) {
+// Row j of U (rank values, zero beyond): 16-byte loads when the rows are
+// 16-byte aligned (U itself is: the C ABI checks it; rank % 4 == 0 keeps
+// every row so).
+GIFT_DEV void u_row(const float* __restrict__ U, int64_t j, int rank, bool vec, float (&u)[32]) {
+  const float* p = U + j * rank;
+  if (vec) {
 #pragma unroll
-  for (int k = 0; k < 32; ++k) P[k] = warp_sum(P[k]);
+    for (int q = 0; q < 8; ++q) {
+      if (4 * q < rank) {
+        const float4 f = __ldg(reinterpret_cast<const float4*>(p) + q);
+        u[4 * q] = f.x; u[4 * q + 1] = f.y; u[4 * q + 2] = f.z; u[4 * q + 3] = f.w;
+      } else {
+        u[4 * q] = u[4 * q + 1] = u[4 * q + 2] = u[4 * q + 3] = 0.0f;
+      }
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < 32; ++k) u[k] = k < rank ? __ldg(p + k) : 0.0f;
+  }
+}
+
+// Sum of v[k] over the 32 lanes, delivered to lane k: at each of five steps a
+// lane keeps the half of its values whose index bit matches its lane bit and
+// adds the partner's copy of that half (31 shuffles in all).
+GIFT_DEV float reduce_transpose32(float (&v)[32], int lane) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    const bool upper = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < o; ++i) {
+      const float send = upper ? v[i] : v[i + o];
+      const float keep = upper ? v[i + o] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+    }
+  }
+  return v[0];
+}
+
+// P (32 coefficients) of the row from each warp's per-lane partial sums: the
+// lanes by transpose, the warps in warp order; every thread returns with
+// pc[k] = P_k c_k.  `part` and `pc_s` are reused row after row.
+GIFT_DEV void row_projection(float (&P)[32], const float* c_s, float (*part)[32], float* pc_s, float (&pc)[32],
+                             int warp, int lane) {
+  part[warp][lane] = reduce_transpose32(P, lane);
+  __syncthreads();
+  if (warp == 0) {
+    float s = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) s += part[w][lane];
+    pc_s[lane] = s * c_s[lane];
+  }
+  __syncthreads();
+#pragma unroll
+  for (int k = 0; k < 32; ++k) pc[k] = pc_s[k];
 }
 
 template <typename T>
@@ -54,33 +107,34 @@ __global__ void __launch_bounds__(kWarps * 32) whiten_encode_simt_kernel(
     float* __restrict__ scales) {
   __shared__ float c_s[32];
   __shared__ float a_s;
+  __shared__ float part[kWarps][32];
+  __shared__ float pc_s[32];
   transform_coeffs(lambda, rho, rank, false, c_s, &a_s, threadIdx.x);
   __syncthreads();
   const float a = a_s;
-  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool vec = (rank & 3) == 0;
   const int64_t nb = d_in / kBlock;
-  for (int64_t row = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5); row < d_out;
-       row += (int64_t)gridDim.x * kWarps) {
+  for (int64_t row = blockIdx.x; row < d_out; row += gridDim.x) {
     const T* g = G + row * d_in;
     float P[32];
 #pragma unroll
     for (int k = 0; k < 32; ++k) P[k] = 0.0f;
-    for (int64_t b = 0; b < nb; ++b) {
+    for (int64_t b = warp; b < nb; b += kWarps) {
       const int64_t j0 = b * kBlock + lane * 4;
       float v[4];
       load4<T>(g + j0, v);
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const float* u = U + (j0 + e) * rank;
+        float u[32];
+        u_row(U, j0 + e, rank, vec, u);
 #pragma unroll
-        for (int k = 0; k < 32; ++k)
-          if (k < rank) P[k] = fmaf(v[e], __ldg(u + k), P[k]);
+        for (int k = 0; k < 32; ++k) P[k] = fmaf(v[e], u[k], P[k]);
       }
     }
-    project_row_reduce(P);
-#pragma unroll
-    for (int k = 0; k < 32; ++k) P[k] *= c_s[k];
-    for (int64_t b = 0; b < nb; ++b) {
+    float pc[32];
+    row_projection(P, c_s, part, pc_s, pc, warp, lane);
+    for (int64_t b = warp; b < nb; b += kWarps) {
       const int64_t j0 = b * kBlock + lane * 4;
       float v[4];
       load4<T>(g + j0, v);
@@ -88,11 +142,11 @@ __global__ void __launch_bounds__(kWarps * 32) whiten_encode_simt_kernel(
       float m = 0.0f;
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const float* u = U + (j0 + e) * rank;
+        float u[32];
+        u_row(U, j0 + e, rank, vec, u);
         float acc = 0.0f;
 #pragma unroll
-        for (int k = 0; k < 32; ++k)
-          if (k < rank) acc = fmaf(P[k], __ldg(u + k), acc);
+        for (int k = 0; k < 32; ++k) acc = fmaf(pc[k], u[k], acc);
         w[e] = fmaf(a, v[e], acc);
         m = fmaxf(m, fabsf(w[e]));
       }
@@ -117,47 +171,48 @@ __global__ void __launch_bounds__(kWarps * 32) whiten_decode_simt_kernel(
     T* __restrict__ out) {
   __shared__ float c_s[32];
   __shared__ float a_s;
+  __shared__ float part[kWarps][32];
+  __shared__ float pc_s[32];
   transform_coeffs(lambda, rho, rank, true, c_s, &a_s, threadIdx.x);
   __syncthreads();
   const float a = a_s;
-  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool vec = (rank & 3) == 0;
   const int64_t nb = d_in / kBlock;
-  for (int64_t row = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5); row < d_out;
-       row += (int64_t)gridDim.x * kWarps) {
+  for (int64_t row = blockIdx.x; row < d_out; row += gridDim.x) {
     float P[32];
 #pragma unroll
     for (int k = 0; k < 32; ++k) P[k] = 0.0f;
-    for (int64_t b = 0; b < nb; ++b) {
+    for (int64_t b = warp; b < nb; b += kWarps) {
       const int64_t j0 = b * kBlock + lane * 4;
       const uint32_t q = __ldg(reinterpret_cast<const uint32_t*>(codes + row * d_in + j0));
       const float s = __ldg(scales + row * nb + b);
       float2 lo = e4m3x2_to_f32x2((uint16_t)(q & 0xFFFF)), hi = e4m3x2_to_f32x2((uint16_t)(q >> 16));
-      float v[4] = {lo.x * s, lo.y * s, hi.x * s, hi.y * s};
+      const float v[4] = {lo.x * s, lo.y * s, hi.x * s, hi.y * s};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const float* u = U + (j0 + e) * rank;
+        float u[32];
+        u_row(U, j0 + e, rank, vec, u);
 #pragma unroll
-        for (int k = 0; k < 32; ++k)
-          if (k < rank) P[k] = fmaf(v[e], __ldg(u + k), P[k]);
+        for (int k = 0; k < 32; ++k) P[k] = fmaf(v[e], u[k], P[k]);
       }
     }
-    project_row_reduce(P);
-#pragma unroll
-    for (int k = 0; k < 32; ++k) P[k] *= c_s[k];
-    for (int64_t b = 0; b < nb; ++b) {
+    float pc[32];
+    row_projection(P, c_s, part, pc_s, pc, warp, lane);
+    for (int64_t b = warp; b < nb; b += kWarps) {
       const int64_t j0 = b * kBlock + lane * 4;
       const uint32_t q = __ldg(reinterpret_cast<const uint32_t*>(codes + row * d_in + j0));
       const float s = __ldg(scales + row * nb + b);
       float2 lo = e4m3x2_to_f32x2((uint16_t)(q & 0xFFFF)), hi = e4m3x2_to_f32x2((uint16_t)(q >> 16));
-      float v[4] = {lo.x * s, lo.y * s, hi.x * s, hi.y * s};
+      const float v[4] = {lo.x * s, lo.y * s, hi.x * s, hi.y * s};
       float o[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const float* u = U + (j0 + e) * rank;
+        float u[32];
+        u_row(U, j0 + e, rank, vec, u);
         float acc = 0.0f;
 #pragma unroll
-        for (int k = 0; k < 32; ++k)
-          if (k < rank) acc = fmaf(P[k], __ldg(u + k), acc);
+        for (int k = 0; k < 32; ++k) acc = fmaf(pc[k], u[k], acc);
         o[e] = fmaf(a, v[e], acc);
       }
       store4<T>(out + row * d_in + j0, o);
@@ -165,10 +220,11 @@ __global__ void __launch_bounds__(kWarps * 32) whiten_decode_simt_kernel(
   }
 }
 
+// One CTA per row, capped at a few waves of resident CTAs (rows are then
+// taken in a grid-stride loop).
 int grid_rows(int64_t d_out) {
-  int64_t need = (d_out + kWarps - 1) / kWarps;
-  int64_t cap = (int64_t)kNumSMs * 8;
-  return (int)(need < cap ? need : cap);
+  const int64_t cap = (int64_t)kNumSMs * 16;
+  return (int)(d_out < cap ? d_out : cap);
 }
 
 }  // namespace
