@@ -375,7 +375,7 @@ TRAFFIC = {
                         "profile": "profiles/whiten_decode_tc_stack8.md"},
 }
 TRAFFIC_SOURCE = ("geometry_aware_fp8_b200/csrc/codec_tc.cu",
-                  "36ce1421959db85fb7c3903ecc5d458e5c8bba6e6485a7eac2bacff6df6aafc2")
+                  "a125250a24fa765d34175b4edf167016c9cb2d44bef6f718aafcde2f7c51a943")
 
 
 def traffic_for(phase, n_elements):

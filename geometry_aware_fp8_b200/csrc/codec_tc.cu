@@ -21,17 +21,22 @@
 //                   operand of E2
 //   warp 12         TMEM allocation; one thread issues every MMA
 //   warps 0-7       epilogue, two threads per row (TMEM lane quarter warp % 4,
-//                   column half warp / 4): form the bf16 hi/lo tile of P o c
-//                   (the A operand of E2), then per chunk read W from TMEM and
-//                   G from shared memory, find the block maximum (the halves
-//                   exchange theirs through shared memory), write the 128
-//                   codes of the row into shared memory and one scale
-//   warp 14 lane 0  TMA store of each chunk's codes; frees the stage
-// A CTA's panels are processed in blocks that interleave the second pass of
-// one panel (E2, epilogue-bound, its chunks re-read from L2 in reverse order)
-// with the first pass of the next (E1, an HBM stream).  Panels of all layers
-// of one launch are assigned to CTAs on the host by longest-first greedy
-// scheduling (a panel costs d_in/128 chunks).
+//                   column half warp / 4): form the bf16 hi/lo tile of P o c / a
+//                   (the A operand of E2), then per chunk read W / a from TMEM
+//                   (G enters it through identity MMAs, so the epilogue reads
+//                   no G), find the block maximum (the halves exchange theirs
+//                   through shared memory), write the 128 codes of the row into
+//                   one of two codes tiles and one scale
+//   warp 14 lane 0  TMA store of each chunk's codes tile, then frees the tile
+// A stage is freed by the MMA's completion.  A CTA's panels are processed in
+// blocks that interleave the second pass of one panel (E2, epilogue-bound, its
+// chunks re-read from L2 in reverse order) with the first pass of the next
+// (E1, an HBM stream).  Panels of all layers of one launch are assigned on the
+// host by longest-first greedy scheduling (a panel costs d_in/128 chunks).
+// A launch with few panels runs the CLUSTER instantiation instead: 2 or 4
+// CTAs of a thread-block cluster share each panel's chunks and sum their
+// partial P through distributed shared memory (see cluster_sum16).  The
+// decoder below follows the same plan with its own stages.
 #include <algorithm>
 #include <queue>
 #include <vector>
