@@ -59,6 +59,7 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-nvfp4", action="store_true", help="skip the NVFP4 measurement on the 11008x4096 gradient")
     ap.add_argument("--no-layers", action="store_true", help="skip the single-layer codec measurements")
+    ap.add_argument("--no-staleness", action="store_true", help="skip the factor-staleness sweep")
     ap.add_argument("--depth", type=int, default=24, help="layers in the stack (24 = the full stand-in)")
     return ap.parse_args()
 
@@ -310,6 +311,31 @@ def layers_measure(torch, ops, synth, dev, peak, reps=20):
     return out
 
 
+def staleness_measure(torch, dev):
+    """The falsifier of the review page ("What would settle it"): the FP8
+    round-trip error of GIFT, with its factor refreshed every K steps, against
+    the Euclidean codec as a function of the steps since the last refresh, for
+    K in {10, 25, 50, 100} (referee report, section V.E / Algorithm 1).  One
+    1536 x 1536 bf16 layer (the stack's o-projection), 4096 tokens a step, 100
+    steps of activations whose basis turns by exp(theta S) a step (slow and
+    fast drift); errors in the Frobenius norm and in the coordinates whitened
+    by the step's fresh factor.  Every refresh, codec and error step runs in
+    the library (see geometry_aware_fp8_b200/staleness.py)."""
+    from geometry_aware_fp8_b200 import staleness as stl
+    T, Ks = 100, (10, 25, 50, 100)
+    out = {"workload": "1536x1536 bf16 layer, X 4096x1536 bf16 per step, 100 steps, "
+                       "Q_t = Q_0 exp(theta S)^t, G_t = Delta_t^T X_t / N; rank 32, E4M3 block 128",
+           "K": list(Ks)}
+    for theta in (0.002, 0.01):
+        step = stl.drifting_device(T, 4096, 1536, 1536, theta, 8000, dtype=torch.bfloat16, device=dev)
+        t0 = time.time()
+        res = stl.sweep(step, T, Ks, seed=8100)
+        summ = stl.summary(res, Ks)
+        summ["seconds"] = time.time() - t0
+        out[f"theta={theta}"] = summ
+    return out
+
+
 def refresh_all(ops, W):
     """Factor refresh of every whitened layer in one batched call."""
     ops.factor_refresh_many(W["jobs"], len(W["whitened"]), RANK, OVERSAMPLE, ITERS)
@@ -527,6 +553,7 @@ def run_gpu(args):
     launches, names = count_launches(torch, ops, W, K)
     nvfp4 = nvfp4_measure(torch, ops, synth, dev, peak) if not args.no_nvfp4 else None
     single = layers_measure(torch, ops, synth, dev, peak) if not args.no_layers else None
+    stale = staleness_measure(torch, dev) if not args.no_staleness else None
 
     # ---- end to end through host buffers: the same schedule, with every
     # step's gradients copied in from pinned host memory, the activations of
@@ -616,7 +643,7 @@ def run_gpu(args):
                            "gradient_bytes": g_bytes, "storage": "bf16 G / e4m3 codes / fp32 scales",
                            "l2": "inputs larger than L2 (1.06 GB of gradients streamed per step)",
                            "parallelism": f"replicas x{world}"},
-                "roofline": roofline, "codec": codec, "layers": single, "nvfp4": nvfp4, "e2e": e2e, "cpu_baseline": cpu,
+                "roofline": roofline, "codec": codec, "layers": single, "staleness": stale, "nvfp4": nvfp4, "e2e": e2e, "cpu_baseline": cpu,
                 "gpu_launches": launches, "kernels": names, "clocks": clock_info}
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -274,6 +274,32 @@ gift_status gift_roundtrip_error(const void* G, const void* G_hat, gift_dtype dt
   return cuda_status(launch_roundtrip_error(G, G_hat, dt, d_out * d_in, out, ws, (cudaStream_t)stream));
 }
 
+gift_status gift_whitened_error_workspace_size(int64_t d_out, int64_t d_in, size_t* bytes) {
+  if (!bytes || d_out < 1 || d_in < 1) return GIFT_ERR_INVALID_ARG;
+  if (d_in % GIFT_E4M3_BLOCK != 0) return GIFT_ERR_SHAPE;
+  *bytes = whitened_error_ws_bytes(d_out);
+  return GIFT_OK;
+}
+
+gift_status gift_whitened_error(const void* G, const void* G_hat, gift_dtype dt, int64_t d_out, int64_t d_in,
+                                const float* U, const float* lambda, const float* rho, int rank, double* out,
+                                void* ws, size_t ws_bytes, gift_stream_t stream) {
+  if (!G || !G_hat || !out) return GIFT_ERR_INVALID_ARG;
+  if (!dtype_ok(dt)) return GIFT_ERR_INVALID_ARG;
+  if (rank < 0 || rank > GIFT_MAX_RANK) return GIFT_ERR_SHAPE;
+  if (rank > 0 && (!U || !lambda || !rho)) return GIFT_ERR_INVALID_ARG;
+  size_t need = 0;
+  gift_status st = gift_whitened_error_workspace_size(d_out, d_in, &need);
+  if (st != GIFT_OK) return st;
+  if (rank > d_in) return GIFT_ERR_SHAPE;
+  if (!ws || ws_bytes < need) return GIFT_ERR_WORKSPACE;
+  if (!aligned16(G) || !aligned16(G_hat) || !aligned(out, 8) || !aligned16(ws)) return GIFT_ERR_ALIGN;
+  if (rank > 0 && (!aligned16(U) || !aligned(lambda, 4) || !aligned(rho, 4))) return GIFT_ERR_ALIGN;
+  if ((st = device_ok()) != GIFT_OK) return st;
+  return cuda_status(launch_whitened_error(G, G_hat, dt, d_out, d_in, U, lambda, rho, rank, out, ws,
+                                           (cudaStream_t)stream));
+}
+
 // ---------------------------------------------------------------------------
 static gift_status check_nvfp4_args(const void* G, int gdt, int64_t d_out, int64_t d_in, const float* U,
                                     const float* lambda, const float* rho, int rank, const void* codes,

@@ -74,6 +74,10 @@ cudaError_t launch_nvfp4_decode(const uint8_t* codes, const uint8_t* sb, const f
 
 cudaError_t launch_roundtrip_error(const void* G, const void* G_hat, gift_dtype dt, int64_t n_elems,
                                    double* out, void* ws, cudaStream_t s);
+size_t whitened_error_ws_bytes(int64_t d_out);
+cudaError_t launch_whitened_error(const void* G, const void* G_hat, gift_dtype dt, int64_t d_out, int64_t d_in,
+                                  const float* U, const float* lambda, const float* rho, int rank, double* out,
+                                  void* ws, cudaStream_t s);
 
 // ---- Factor refresh ----
 struct RefreshPlan {

@@ -27,7 +27,7 @@ STATUS = {0: "GIFT_OK", 1: "GIFT_ERR_INVALID_ARG", 2: "GIFT_ERR_SHAPE", 3: "GIFT
 EXPORTED = ("gift_status_string", "gift_version", "gift_refresh_workspace_size", "gift_factor_refresh",
             "gift_factor_refresh_noalloc", "gift_factor_refresh_many", "gift_encode", "gift_decode", "gift_encode_many", "gift_decode_many",
             "gift_error_workspace_size", "gift_roundtrip_error", "gift_encode_nvfp4", "gift_decode_nvfp4",
-            "gift_codec_split")
+            "gift_codec_split", "gift_whitened_error_workspace_size", "gift_whitened_error")
 
 
 class GiftError(RuntimeError):
@@ -81,6 +81,8 @@ def lib() -> ctypes.CDLL:
         L.gift_codec_split.argtypes = [ctypes.POINTER(Layer), i32, i32, ctypes.POINTER(i32)]
         L.gift_error_workspace_size.argtypes = [i64, i64, ctypes.POINTER(sz)]
         L.gift_roundtrip_error.argtypes = [vp, vp, i32, i64, i64, vp, vp, sz, vp]
+        L.gift_whitened_error_workspace_size.argtypes = [i64, i64, ctypes.POINTER(sz)]
+        L.gift_whitened_error.argtypes = [vp, vp, i32, i64, i64, vp, vp, vp, i32, vp, vp, sz, vp]
         L.gift_encode_nvfp4.argtypes = [vp, i32, i64, i64, vp, vp, vp, i32, vp, vp, vp, vp]
         L.gift_decode_nvfp4.argtypes = [vp, vp, vp, i64, i64, vp, vp, vp, i32, vp, i32, vp]
         for name in EXPORTED:
@@ -328,4 +330,29 @@ def roundtrip_error(G: torch.Tensor, G_hat: torch.Tensor, out: Optional[torch.Te
         ws = torch.empty((error_workspace_size(d_out, d_in),), device=G.device, dtype=torch.uint8)
     _check(lib().gift_roundtrip_error(_ptr(G), _ptr(G_hat), _dt(G), d_out, d_in, _ptr(out), _ptr(ws),
                                       ws.numel(), _stream(stream)), "gift_roundtrip_error")
+    return out
+
+
+def whitened_error_workspace_size(d_out: int, d_in: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().gift_whitened_error_workspace_size(d_out, d_in, ctypes.byref(n)),
+           "gift_whitened_error_workspace_size")
+    return n.value
+
+
+def whitened_error(G: torch.Tensor, G_hat: torch.Tensor, U=None, lam=None, rho=None,
+                   out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+                   stream=None) -> torch.Tensor:
+    """Device tensor [||(G_hat-G) M|| / ||G M||, ||(G_hat-G) M||^2, ||G M||^2] (fp64), M from (U, lam, rho)."""
+    _cuda(G, G_hat, U, lam, rho, out, ws)
+    if G.dtype != G_hat.dtype or G.shape != G_hat.shape:
+        raise ValueError("G and G_hat must match in shape and dtype")
+    d_out, d_in = G.shape
+    rank = 0 if U is None else U.shape[1]
+    if out is None:
+        out = torch.empty((3,), device=G.device, dtype=torch.float64)
+    if ws is None:
+        ws = torch.empty((whitened_error_workspace_size(d_out, d_in),), device=G.device, dtype=torch.uint8)
+    _check(lib().gift_whitened_error(_ptr(G), _ptr(G_hat), _dt(G), d_out, d_in, _ptr(U), _ptr(lam), _ptr(rho), rank,
+                                     _ptr(out), _ptr(ws), ws.numel(), _stream(stream)), "gift_whitened_error")
     return out

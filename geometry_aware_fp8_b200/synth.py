@@ -20,6 +20,11 @@ round-to-nearest-even cast to the storage dtype):
   layer configurations, whose anisotropy axes are not A's), or
   ``aligned=True`` for Z diag(j^-e) Q, whose principal axes coincide with
   the activations' principal axes.
+* drifting layer (the staleness sweep): the activation basis rotates slowly,
+  Q_t = Q_0 R^t with R = exp(theta S) and S = (B - B^T) / sqrt(2 d) for a
+  Gaussian B (skew-symmetric, spectral norm about 2), X_t = Z_t diag(sigma)
+  Q_t, and the gradient follows the activations as a linear layer's does,
+  G_t = Delta_t^T X_t / N with Delta_t iid N(0,1) of shape N x d_out.
 """
 from __future__ import annotations
 
@@ -66,6 +71,35 @@ def gradient(d_out: int, Q: np.ndarray, exponent: float, seed: int,
     # literal recipe multiplies by Q^T (axes on Q's columns), the aligned
     # variant by Q (axes shared with A).
     return (Z * D[None, :]) @ (Q if aligned else Q.T)
+
+
+def drift_generator(d: int, seed: int) -> np.ndarray:
+    """S = (B - B^T) / sqrt(2 d), B iid N(0,1): the generator of the drift."""
+    rng = np.random.default_rng(seed)
+    B = rng.standard_normal((d, d))
+    return (B - B.T) / np.sqrt(2.0 * d)
+
+
+def drift_rotation(d: int, theta: float, seed: int) -> np.ndarray:
+    """R = exp(theta S): the orthogonal one-step rotation of the activation basis."""
+    from scipy.linalg import expm
+    return expm(theta * drift_generator(d, seed))
+
+
+def drifting_layer(T: int, N: int, d_in: int, d_out: int, theta: float, seed: int, a: float = 1.0):
+    """T steps of (X_t, G_t) on the CPU (fp64): X_t = Z_t diag(i^-a) Q_0 R^t,
+    G_t = Delta_t^T X_t / N.  Step t draws from default_rng(seed + 1000 + t)."""
+    Q = haar_orthogonal(d_in, seed)
+    R = drift_rotation(d_in, theta, seed + 1)
+    sigma = column_power(d_in, a)
+    out = []
+    for t in range(T):
+        rng = np.random.default_rng(seed + 1000 + t)
+        X = (rng.standard_normal((N, d_in)) * sigma[None, :]) @ Q
+        D = rng.standard_normal((N, d_out))
+        out.append((X, D.T @ X / N))
+        Q = Q @ R
+    return out
 
 
 def to_storage(x: np.ndarray, dtype: str) -> np.ndarray:

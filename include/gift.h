@@ -242,6 +242,29 @@ gift_status gift_roundtrip_error(const void* G, const void* G_hat, gift_dtype dt
                                  gift_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * The same error in whitened coordinates (the geometry-aware norm in which
+ * the review page's "direction-dependent distortion" is measured):
+ *
+ *   out[0] = ||(G_hat - G) M||_F / ||G M||_F,  out[1] = ||(G_hat - G) M||_F^2,
+ *   out[2] = ||G M||_F^2,
+ *
+ * M = rho^{-1/2} I + U diag((lambda + rho)^{-1/2} - rho^{-1/2}) U^T from the
+ * factor (U, lambda, rho) given here (rank 0: M = I, the plain relative
+ * error).  fp32 products, fp64 sums in a fixed order (deterministic).
+ * G, G_hat: d_out x d_in, dtype dt, 16-byte aligned; U: d_in x rank fp32,
+ * 16-byte aligned; out: 3 doubles on the device; ws: device scratch of at
+ * least gift_whitened_error_workspace_size bytes, 16-byte aligned.
+ * Errors: GIFT_ERR_INVALID_ARG (null pointer, bad dtype), GIFT_ERR_SHAPE
+ * (d_in not a multiple of 128, rank outside 0..32 or above d_in),
+ * GIFT_ERR_WORKSPACE, GIFT_ERR_ALIGN, GIFT_ERR_CUDA.
+ * ------------------------------------------------------------------------ */
+gift_status gift_whitened_error_workspace_size(int64_t d_out, int64_t d_in, size_t* bytes /* host */);
+
+gift_status gift_whitened_error(const void* G, const void* G_hat, gift_dtype dt, int64_t d_out, int64_t d_in,
+                                const float* U, const float* lambda, const float* rho, int rank, double* out,
+                                void* ws, size_t ws_bytes, gift_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * NVFP4 codec (abstract: NVFP4 is the second low-precision format the
  * whitening is applied to).  The pages give no recipe; this library uses the
  * two-level one of the NVFP4 format, decisions in fp32:

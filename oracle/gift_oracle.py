@@ -446,3 +446,47 @@ def whitened_error(G, G_hat, M) -> float:
     D = (np.asarray(G_hat, dtype=np.float64) - G) @ M
     W = G @ M
     return float(np.sqrt(np.sum(D * D)) / np.sqrt(np.sum(W * W)))
+
+
+# ---------------------------------------------------------------------------
+# Staleness of the factor (review page, "What would settle it": the round-trip
+# error of GIFT against the Euclidean baseline as a function of the steps since
+# the last refresh of A; referee report on section V.E / Algorithm 1: refresh
+# intervals K in {10, 25, 50, 100}).
+# ---------------------------------------------------------------------------
+
+def staleness_sweep(steps, Ks, rank: int = 32, oversample: int = 16, iters: int = 4, seed: int = 0,
+                    ghat_bf16: bool = False):
+    """Per-step errors of the Euclidean codec and of GIFT with its factor
+    refreshed every K steps, for a sequence steps = [(X_t, G_t), ...].
+
+    The factor of step t is the refresh of A_t = X_t^T X_t / N with Rademacher
+    seed (seed + t); GIFT under interval K codes G_t with the factor of step
+    K floor(t / K).  Errors: the Frobenius round-trip error and the error in
+    the coordinates whitened by the fresh factor of step t (the geometry the
+    gradient has at that step).  G_hat is kept in fp64, or rounded to bf16 by
+    round-to-nearest-even (ghat_bf16) as a codec whose G is bf16 returns it.
+    Returns {"euclid": {"frob": [...], "white": [...]}, K: {"frob": [...],
+    "white": [...]}, ...}."""
+    fresh = []
+    for t, (X, _) in enumerate(steps):
+        U, lam, rho, _ = factor_refresh(input_factor(X), rank, oversample, iters, seed=seed + t)
+        fresh.append((U, lam, rho))
+    M_now = [transform_matrix(*f) for f in fresh]
+    empty = np.zeros((steps[0][1].shape[1], 0))
+    out_round = bf16_round if ghat_bf16 else (lambda x: x)
+    out = {"euclid": {"frob": [], "white": []}}
+    for t, (_, G) in enumerate(steps):
+        c, s = encode_e4m3(G, empty, np.zeros(0), 1.0)
+        Gh = out_round(decode_e4m3(c, s, empty, np.zeros(0), 1.0))
+        out["euclid"]["frob"].append(roundtrip_error(G, Gh))
+        out["euclid"]["white"].append(whitened_error(G, Gh, M_now[t]))
+    for K in Ks:
+        out[K] = {"frob": [], "white": []}
+        for t, (_, G) in enumerate(steps):
+            f = fresh[K * (t // K)]
+            c, s = encode_e4m3(G, *f)
+            Gh = out_round(decode_e4m3(c, s, *f))
+            out[K]["frob"].append(roundtrip_error(G, Gh))
+            out[K]["white"].append(whitened_error(G, Gh, M_now[t]))
+    return out
