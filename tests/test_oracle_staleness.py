@@ -1,8 +1,10 @@
 """CPU pins of the staleness sweep (review page, "What would settle it";
 referee report on section V.E / Algorithm 1: refresh intervals K): the drift
 model's rotation and the sweep's bookkeeping of which factor codes which step.
-The codec, refresh and error functions it calls are pinned elsewhere."""
+The codec and refresh functions it calls are pinned elsewhere; the error in
+whitened coordinates is pinned here by closed forms."""
 import numpy as np
+import pytest
 
 from oracle import gift_oracle as O
 from geometry_aware_fp8_b200 import synth
@@ -74,3 +76,24 @@ def test_bf16_output_rounds_g_hat_before_the_errors():
     _, G = steps[1]
     c, s = O.quantize_e4m3_blocks(G)
     assert res["euclid"]["frob"][1] == O.roundtrip_error(G, O.bf16_round(O.dequantize_e4m3_blocks(c, s)))
+
+
+def test_whitened_error_closed_forms():
+    d = 256
+    rng = np.random.default_rng(3)
+    G = rng.standard_normal((4, d))
+    # an error proportional to G is the same fraction in any coordinates
+    U = np.linalg.qr(rng.standard_normal((d, 32)))[0]
+    lam = np.sort(rng.uniform(1, 10, 32))[::-1]
+    M = O.transform_matrix(U, lam, 0.01)
+    assert O.whitened_error(G, 1.03 * G, M) == pytest.approx(0.03, rel=1e-12)
+    # M = I is the Frobenius round-trip error
+    Gh = G + 0.01 * rng.standard_normal(G.shape)
+    assert O.whitened_error(G, Gh, np.eye(d)) == pytest.approx(O.roundtrip_error(G, Gh), rel=1e-12)
+    # one row along e_1 (inside span U = {e_1}) and an error delta e_2 (outside it):
+    # ||(G_hat - G) M|| = delta rho^{-1/2}, ||G M|| = (lambda + rho)^{-1/2}
+    E = np.eye(d)
+    lam1, rho, delta = 4.0, 0.25, 1e-3
+    M1 = O.transform_matrix(E[:, :1], np.array([lam1]), rho)
+    got = O.whitened_error(E[:1], E[:1] + delta * E[1:2], M1)
+    assert got == pytest.approx(delta * np.sqrt((lam1 + rho) / rho), rel=1e-12)
