@@ -490,3 +490,66 @@ def staleness_sweep(steps, Ks, rank: int = 32, oversample: int = 16, iters: int 
             out[K]["frob"].append(roundtrip_error(G, Gh))
             out[K]["white"].append(whitened_error(G, Gh, M_now[t]))
     return out
+
+
+# ---------------------------------------------------------------------------
+# The variants GIFT is simplified from (review page, "What carries the
+# argument": full two-sided K-FAC whitening, then the input side alone, then
+# rank 32; section IV.A, Eq. (14) writes the input-side Cholesky form L_A^{-T},
+# which the referee report's minor comment 3 reads as (L_A^{-1})^T).  Oracle
+# only: the library codes the rank-r eigen transform.
+# ---------------------------------------------------------------------------
+
+def full_rank_transform(A, inverse: bool = False) -> np.ndarray:
+    """A^{-1/2} (inverse: A^{1/2}) by LAPACK eigh: the rank-r construction at
+    r = d_in, where the floor rho is empty (reading C3: rho := 0)."""
+    lam, V = np.linalg.eigh(np.asarray(A, dtype=np.float64))
+    p = 0.5 if inverse else -0.5
+    return (V * lam ** p) @ V.T
+
+
+def cholesky_transform(A, inverse: bool = False) -> np.ndarray:
+    """L^{-T} with A = L L^T (Eq. 14's L_A^{-T}); inverse: L^T.  W = G L^{-T}
+    has input-side covariance L^{-1} A L^{-T} = I."""
+    L = np.linalg.cholesky(np.asarray(A, dtype=np.float64))
+    if inverse:
+        return L.T
+    return np.linalg.inv(L).T
+
+
+def two_sided_encode_decode(G, A, B, block: int = BLOCK_E4M3):
+    """Full two-sided Cholesky whitening: W = L_B^{-1} G L_A^{-T}, per-block
+    E4M3, G_hat = L_B W_hat L_A^T (B = E[delta delta^T], the output-side
+    factor, d_out x d_out)."""
+    LB = np.linalg.cholesky(np.asarray(B, dtype=np.float64))
+    W = np.linalg.solve(LB, np.asarray(G, dtype=np.float64)) @ cholesky_transform(A)
+    c, s = quantize_e4m3_blocks(W, block)
+    return LB @ dequantize_e4m3_blocks(c, s, block) @ cholesky_transform(A, inverse=True)
+
+
+def transform_comparison(G, X, Delta, rank: int = 32, oversample: int = 16, iters: int = 4, seed: int = 0):
+    """Round-trip errors of the E4M3 codec under each coordinate choice, for a
+    layer with activations X (N x d_in), output-side errors Delta (N x d_out)
+    and gradient G (d_out x d_in): Euclidean, input-side rank-r (the codec's
+    transform), input-side full rank (A^{-1/2}), input-side Cholesky (L_A^{-T})
+    and two-sided Cholesky.  Each reports the Frobenius error and the error in
+    the coordinates whitened by the input-side A^{-1/2} (a Table I/II-style
+    comparison on synthetic data)."""
+    A = input_factor(X)
+    B = input_factor(Delta)
+    M_ref = full_rank_transform(A)
+    U, lam, rho, _ = factor_refresh(A, rank, oversample, iters, seed=seed)
+    out = {}
+
+    def record(name, Gh):
+        out[name] = {"frob": roundtrip_error(G, Gh), "white": whitened_error(G, Gh, M_ref)}
+
+    c, s = quantize_e4m3_blocks(G)
+    record("euclid", dequantize_e4m3_blocks(c, s))
+    c, s = encode_e4m3(G, U, lam, rho)
+    record(f"input_rank{rank}", decode_e4m3(c, s, U, lam, rho))
+    for name, fn in (("input_full", full_rank_transform), ("input_cholesky", cholesky_transform)):
+        c, s = quantize_e4m3_blocks(np.asarray(G, dtype=np.float64) @ fn(A))
+        record(name, dequantize_e4m3_blocks(c, s) @ fn(A, inverse=True))
+    record("two_sided_cholesky", two_sided_encode_decode(G, A, B))
+    return out
