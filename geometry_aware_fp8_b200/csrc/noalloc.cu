@@ -13,6 +13,9 @@
 // (sampled subspace, its image, a Cholesky-QR temporary, fp64 Gram partials
 // and the small factors) at 5,308,416 bytes.  A must be given by the caller as an output buffer,
 // and the token range is not split, so the whole scratch need is known.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <mutex>
 
 #include "common.cuh"
@@ -33,20 +36,48 @@ static __device__ __align__(256) unsigned char g_refresh_scratch[kNoAllocScratch
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 void* g_scratch_addr[kMaxDevices] = {};
+unsigned long long g_scratch_ctx[kMaxDevices] = {};  // id of the context the address belongs to
 
-// Device address of the scratch array on the current device; looked up once
-// per device with that device current.
+// Unique id of the calling thread's current context (0 if it cannot be read).
+// A device reset destroys the primary context and the module image with it;
+// the next context gets a new id, so a cached address is never reused across
+// a reset.
+unsigned long long current_context_id() {
+  static PFN_cuCtxGetCurrent_v4000 get_ctx = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_ctx = (PFN_cuCtxGetCurrent_v4000)p;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = (PFN_cuCtxGetId_v12000)p;
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_ctx || !get_id || get_ctx(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+// Device address of the scratch array on the current device.  It is looked
+// up with the device current on the first call, and again whenever the
+// device's context has changed since (after a cudaDeviceReset, say).
 cudaError_t scratch_address(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  const unsigned long long ctx = current_context_id();  // 0 before the runtime has made a context
   std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_scratch_addr[dev]) {
+  if (!g_scratch_addr[dev] || ctx == 0 || ctx != g_scratch_ctx[dev]) {
     void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_refresh_scratch);
+    e = cudaGetSymbolAddress(&p, g_refresh_scratch);  // makes the context if there is none yet
     if (e != cudaSuccess) return e;
     g_scratch_addr[dev] = p;
+    g_scratch_ctx[dev] = current_context_id();
   }
   *out = g_scratch_addr[dev];
   return cudaSuccess;

@@ -285,13 +285,23 @@ class LayerArgs:
     rho: Optional[torch.Tensor] = None
 
 
+def _dtype_code(dt: torch.dtype) -> int:
+    if dt == torch.bfloat16:
+        return GIFT_BF16
+    if dt == torch.float32:
+        return GIFT_F32
+    raise TypeError(f"unsupported gradient dtype {dt} (bf16 or fp32)")
+
+
 def make_layers(layers: Sequence[LayerArgs]):
     """Pack a list of LayerArgs into a ctypes gift_layer array (kept alive by the caller)."""
     arr = (Layer * max(len(layers), 1))()
     for i, L in enumerate(layers):
+        for t in (L.G, L.G_hat):
+            if t is not None and t.dtype != L.dtype:
+                raise TypeError(f"layer {i}: tensor dtype {t.dtype} differs from the layer's {L.dtype}")
         arr[i] = Layer(_ptr(L.G), _ptr(L.G_hat), _ptr(L.codes), _ptr(L.scales), _ptr(L.U), _ptr(L.lam),
-                       _ptr(L.rho), L.d_out, L.d_in, L.rank,
-                       GIFT_BF16 if L.dtype == torch.bfloat16 else GIFT_F32)
+                       _ptr(L.rho), L.d_out, L.d_in, L.rank, _dtype_code(L.dtype))
     return arr
 
 

@@ -150,6 +150,9 @@ gift_status gift_factor_refresh_many(const gift_refresh_job* jobs /* host */, in
  * gift_factor_refresh would.
  * Set-up: the first call on each device looks up the array's device address
  * with that device current; make that first call before any stream capture.
+ * The address is looked up again when the device's context is no longer the
+ * one it was found in (after cudaDeviceReset, for example), so the library
+ * may be used across a device reset; such a call is again a first call.
  * Every call on a device shares the one array and leaves its contents
  * behind; no value in it needs to start at zero.  Calls whose executions
  * overlap on the GPU (different streams, or different host threads) race

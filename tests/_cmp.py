@@ -10,6 +10,9 @@ Match criteria for the codec (written here once, used by every parity test):
   * G_hat (decoder fed the oracle's codes): fp32 output within 1e-3 of the
     oracle relative to the row's largest magnitude; bf16 output within one
     bf16 rounding (2^-8 relative) of the same reference plus that 1e-3.
+    Each row also meets the criterion as a whole: its relative Frobenius
+    error ||got - want|| / ||want|| is at most 1e-3 (plus 2^-8 for bf16
+    output), so small elements cannot hide a large share of the error.
   * NVFP4, Euclidean: every decision is taken in fp32 on exact inputs, so the
     tensor scale, block scales and codes are bit-exact (+0 / -0 the same).
   * NVFP4, whitened: W comes from the tensor cores (different summation
@@ -62,6 +65,12 @@ def check_rows(got, want, rtol=GHAT_RTOL, bf16=False):
         tol = tol + 2.0 ** -8 * np.abs(want)
     bad = np.abs(got - want) > tol + 1e-30
     assert not bad.any(), f"{bad.sum()} elements off; worst {(np.abs(got - want) / np.maximum(rowmax, 1e-30)).max()}"
+    rn = np.linalg.norm(want, axis=1)
+    rel = np.linalg.norm(got - want, axis=1) / np.maximum(rn, 1e-300)
+    rel = np.where(rn == 0, np.linalg.norm(got, axis=1), rel)
+    lim = rtol + (2.0 ** -8 if bf16 else 0.0)
+    assert rel.max(initial=0) <= lim, f"row relative Frobenius error {rel.max()} > {lim}"
+    return float(rel.max(initial=0))
 
 
 def e2m1_position(codes):

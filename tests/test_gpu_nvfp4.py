@@ -93,3 +93,25 @@ def test_nvfp4_roundtrip_error_matches_oracle(rank):
     e_o = O.roundtrip_error(G64, want)
     e_g = O.roundtrip_error(G64, got.cpu().numpy())
     assert abs(e_g - e_o) <= 1e-3 * e_o, (e_g, e_o)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_nvfp4_euclidean_hand_derived_blocks(dtype):
+    """The hand-derived row of tests/golden/nvfp4_hand_blocks.txt (block scale
+    ratios between E4M3 values and on ties) through the GPU's Euclidean NVFP4
+    codec: tensor scale, block scale codes and element codes must be the
+    hand-derived ones (every value of the row except one in the flushed
+    block is exact in bf16, and that block stays flushed)."""
+    from _golden import nvfp4_hand_blocks
+    W, st, sb_want, q_want, _ = nvfp4_hand_blocks()
+    Gd = torch.from_numpy(np.repeat(W, 3, axis=0).astype(np.float32)).to(DEV).to(dtype)
+    codes, sb, ts = ops.encode_nvfp4(Gd)
+    torch.cuda.synchronize()
+    assert float(ts.item()) == st
+    from _cmp import unpack_nibbles
+    for r in range(3):
+        assert np.array_equal(sb[r].cpu().numpy(), sb_want)
+        assert np.array_equal(unpack_nibbles(codes[r:r + 1].cpu().numpy())[0], q_want)
+    out = ops.decode_nvfp4(codes, sb, ts, out_dtype=torch.float32)[0].cpu().numpy().astype(np.float64)
+    want = O.e2m1_decode(q_want) * np.repeat(O.e4m3_decode(sb_want), 16) * st
+    assert np.array_equal(out, want)

@@ -107,11 +107,8 @@ def test_stack_nvfp4_full_tensor_scale_and_rows():
     lam64 = lam.cpu().numpy().astype(np.float64)
     r = float(rho.item())
     G64 = G.float().cpu().numpy().astype(np.float64)
-    # W for the whole tensor through the rank-32 factor: a G + (G U o c) U^T
-    a = r ** -0.5
-    c = (lam64 + r) ** -0.5 - a
-    W = a * G64 + ((G64 @ U64) * c) @ U64.T
-    W32 = W.astype(np.float32)
+    # W = G M for the whole tensor, through the oracle's transform
+    W32 = O.whiten(G64, U64, lam64, r).astype(np.float32)
     S_t = np.float32(np.max(np.abs(W32)) / np.float32(6.0 * 448.0))
     rows = _rows(d_out)
     want_c, want_s, _ = O.quantize_nvfp4(W32[rows], S_t=S_t)

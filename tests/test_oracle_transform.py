@@ -186,3 +186,24 @@ def test_block_too_small_for_the_fp32_reciprocal_is_flushed():
     codes, scales = O.quantize_e4m3_blocks(W)
     assert scales[0, 0] == 0 and np.all(codes[0, :128] == 0)
     assert scales[0, 1] == np.float32(1e-30) / np.float32(448) and codes[0, 130] == 0x7E
+
+
+def test_nvfp4_hand_derived_blocks_between_and_on_scale_ties():
+    """Six blocks whose scale ratios amax_b / (6 S_t) fall between E4M3 values
+    or exactly on ties (tests/golden/nvfp4_hand_blocks.txt): the block scale
+    codes, the element codes and the dequantised values of the oracle must be
+    the hand-derived ones."""
+    from _golden import nvfp4_hand_blocks
+    W, st, sb_want, q_want, _ = nvfp4_hand_blocks()
+    packed, sb, St = O.quantize_nvfp4(W)
+    assert St == np.float32(st)
+    assert np.array_equal(sb[0], sb_want), (sb[0], sb_want)
+    q = np.empty(96, dtype=np.uint8)
+    q[0::2] = packed[0] & 0xF
+    q[1::2] = packed[0] >> 4
+    assert np.array_equal(q, q_want), np.nonzero(q != q_want)
+    back = O.dequantize_nvfp4(packed, sb, St)[0]
+    want = O.e2m1_decode(q_want) * np.repeat(O.e4m3_decode(sb_want), 16) * st
+    assert np.array_equal(back, want)
+    # the scale of the 8.25 block is 8 (not 9), of the 8.5 tie 8, of the 15.5 tie 16
+    assert list(O.e4m3_decode(sb_want[1:5])) == [8.0, 8.0, 16.0, 12.0]

@@ -6,7 +6,9 @@ not call cudaMalloc in that step).  It must return what gift_factor_refresh
 returns, within the refresh tolerances: top-32 eigenvalues within 1e-4
 relative, rho within the fp32-accumulation bound of its numerator, A within
 1e-5 of max|A|, and the transform within 1e-2 in relative Frobenius norm.
-Two calls in a row check that the shared scratch array is reused cleanly.
+Two calls in a row check that the shared scratch array is reused cleanly,
+and every call must leave its device status word at zero.  One case is also
+compared with the CPU oracle directly, under the same criteria.
 This file is collected last on purpose.
 """
 import numpy as np
@@ -27,6 +29,7 @@ def _rho_tol(rho, trace, N, d, r):
 def _compare(ref, got, A_ref, A_got, N):
     U0, l0, r0, _ = [t.cpu().numpy().astype(np.float64) for t in ref]
     U1, l1, r1, s1 = [t.cpu().numpy().astype(np.float64) for t in got]
+    assert int(s1[0]) == 0, f"device status {int(s1[0]):#x}"
     A0 = A_ref.cpu().numpy().astype(np.float64)
     A1 = A_got.cpu().numpy().astype(np.float64)
     d, r = U0.shape
@@ -59,6 +62,33 @@ def test_noalloc_refresh_matches_regular_refresh_twice(N, d, dtype, rank, over):
         else:
             for a, b in zip(first, got[:3]):
                 assert torch.equal(a, b)
+
+
+def test_noalloc_refresh_matches_oracle():
+    """One case against the CPU oracle directly (config 1's shape: X 2048 x
+    512 fp32, sigma_i = i^-1): A, the top-32 eigenvalues, rho, the floor bit,
+    U's orthonormality, the Ritz property and the transform, under the
+    criteria of the regular refresh's parity tests."""
+    d, N = 512, 2048
+    Q = synth.haar_orthogonal(d, 1003)
+    X = synth.activations(N, Q, synth.column_power(d, 1.0), 1001).astype(np.float32)
+    Xd = torch.from_numpy(X).to(DEV)
+    A_got = torch.empty((d, d), device=DEV, dtype=torch.float32)
+    U, lam, rho, st = ops.factor_refresh_noalloc(Xd, A_got, 32, 16, 4, 1004)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    A = O.input_factor(X)
+    Uo, lo, ro, fo = O.factor_refresh(A, 32, 16, 4, seed=1004)
+    Ag = A_got.cpu().numpy().astype(np.float64)
+    Ug, lg, rg = U.cpu().numpy().astype(np.float64), lam.cpu().numpy().astype(np.float64), float(rho.item())
+    assert np.max(np.abs(Ag - A)) <= 1e-5 * np.max(np.abs(A))
+    assert np.allclose(lg, lo, rtol=1e-4, atol=0)
+    assert abs(rg - ro) <= _rho_tol(ro, np.trace(A), N, d, 32), (rg, ro)
+    assert fo == 0
+    assert np.max(np.abs(Ug.T @ Ug - np.eye(32))) < 1e-5
+    assert np.max(np.abs(Ug.T @ A @ Ug - np.diag(lg))) < 1e-4 * lg[0]
+    Mg, Mo = O.transform_matrix(Ug, lg, rg), O.transform_matrix(Uo, lo, ro)
+    assert np.linalg.norm(Mg - Mo) / np.linalg.norm(Mo) < 1e-2
 
 
 def test_noalloc_refresh_rejects_what_it_cannot_hold():
