@@ -151,40 +151,49 @@ gift_status gift_factor_refresh_many(const gift_refresh_job* jobs, int n, int ra
 // ---------------------------------------------------------------------------
 gift_status gift_encode(const void* G, gift_dtype gdt, int64_t d_out, int64_t d_in, const float* U,
                         const float* lambda, const float* rho, int rank, uint8_t* codes, float* scales,
-                        gift_stream_t stream) {
+                        uint32_t* dev_status, gift_stream_t stream) {
   gift_status st = check_codec_args(G, gdt, d_out, d_in, U, lambda, rho, rank, codes, scales);
   if (st != GIFT_OK) return st;
-  if (d_out == 0) return GIFT_OK;
-  if ((st = device_ok()) != GIFT_OK) return st;
-  cudaStream_t s = (cudaStream_t)stream;
-  if (rank == 0) return cuda_status(launch_euclid_encode(G, gdt, d_out * (d_in / GIFT_E4M3_BLOCK), codes, scales, s));
-  if (use_tc(gdt, rank, d_in)) {
-    TcLayer L{G, nullptr, codes, scales, U, lambda, rho, (int)d_out, (int)d_in, rank};
-    return cuda_status(launch_whiten_encode_tc(&L, 1, s));
-  }
-  return cuda_status(launch_whiten_encode_simt(G, gdt, d_out, d_in, U, lambda, rho, rank, codes, scales, s));
-}
-
-gift_status gift_decode(const uint8_t* codes, const float* scales, int64_t d_out, int64_t d_in, const float* U,
-                        const float* lambda, const float* rho, int rank, void* G_hat, gift_dtype out_dt,
-                        gift_stream_t stream) {
-  gift_status st = check_codec_args(G_hat, out_dt, d_out, d_in, U, lambda, rho, rank, codes, scales);
-  if (st != GIFT_OK) return st;
+  if (dev_status && !aligned(dev_status, 4)) return GIFT_ERR_ALIGN;
   if (d_out == 0) return GIFT_OK;
   if ((st = device_ok()) != GIFT_OK) return st;
   cudaStream_t s = (cudaStream_t)stream;
   if (rank == 0)
-    return cuda_status(launch_euclid_decode(codes, scales, d_out * (d_in / GIFT_E4M3_BLOCK), G_hat, out_dt, s));
+    return cuda_status(
+        launch_euclid_encode(G, gdt, d_out * (d_in / GIFT_E4M3_BLOCK), codes, scales, dev_status, s));
+  if (use_tc(gdt, rank, d_in)) {
+    TcLayer L{G, nullptr, codes, scales, U, lambda, rho, (int)d_out, (int)d_in, rank};
+    return cuda_status(launch_whiten_encode_tc(&L, 1, dev_status, s));
+  }
+  return cuda_status(
+      launch_whiten_encode_simt(G, gdt, d_out, d_in, U, lambda, rho, rank, codes, scales, dev_status, s));
+}
+
+gift_status gift_decode(const uint8_t* codes, const float* scales, int64_t d_out, int64_t d_in, const float* U,
+                        const float* lambda, const float* rho, int rank, void* G_hat, gift_dtype out_dt,
+                        uint32_t* dev_status, gift_stream_t stream) {
+  gift_status st = check_codec_args(G_hat, out_dt, d_out, d_in, U, lambda, rho, rank, codes, scales);
+  if (st != GIFT_OK) return st;
+  if (dev_status && !aligned(dev_status, 4)) return GIFT_ERR_ALIGN;
+  if (d_out == 0) return GIFT_OK;
+  if ((st = device_ok()) != GIFT_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (rank == 0)
+    return cuda_status(
+        launch_euclid_decode(codes, scales, d_out * (d_in / GIFT_E4M3_BLOCK), G_hat, out_dt, dev_status, s));
   if (use_tc(out_dt, rank, d_in)) {
     TcLayer L{nullptr, G_hat, (uint8_t*)codes, (float*)scales, U, lambda, rho, (int)d_out, (int)d_in, rank};
-    return cuda_status(launch_whiten_decode_tc(&L, 1, s));
+    return cuda_status(launch_whiten_decode_tc(&L, 1, dev_status, s));
   }
-  return cuda_status(launch_whiten_decode_simt(codes, scales, d_out, d_in, U, lambda, rho, rank, G_hat, out_dt, s));
+  return cuda_status(
+      launch_whiten_decode_simt(codes, scales, d_out, d_in, U, lambda, rho, rank, G_hat, out_dt, dev_status, s));
 }
 
 // ---------------------------------------------------------------------------
-static gift_status run_many(const gift_layer* layers, int n, gift_stream_t stream, bool encode) {
+static gift_status run_many(const gift_layer* layers, int n, uint32_t* dev_status, gift_stream_t stream,
+                            bool encode) {
   if (n < 0 || (n > 0 && !layers)) return GIFT_ERR_INVALID_ARG;
+  if (dev_status && !aligned(dev_status, 4)) return GIFT_ERR_ALIGN;
   for (int i = 0; i < n; ++i) {
     const gift_layer& L = layers[i];
     const void* g = encode ? L.G : (const void*)L.G_hat;
@@ -209,19 +218,19 @@ static gift_status run_many(const gift_layer* layers, int n, gift_stream_t strea
       tc.push_back(TcLayer{L.G, L.G_hat, L.codes, L.scales, L.U, L.lambda, L.rho, (int)L.d_out, (int)L.d_in, L.rank});
     } else {
       e = encode ? launch_whiten_encode_simt(L.G, (gift_dtype)L.dtype, L.d_out, L.d_in, L.U, L.lambda, L.rho, L.rank,
-                                             L.codes, L.scales, s)
+                                             L.codes, L.scales, dev_status, s)
                  : launch_whiten_decode_simt(L.codes, L.scales, L.d_out, L.d_in, L.U, L.lambda, L.rho, L.rank,
-                                             L.G_hat, (gift_dtype)L.dtype, s);
+                                             L.G_hat, (gift_dtype)L.dtype, dev_status, s);
     }
     if (e != cudaSuccess) return GIFT_ERR_CUDA;
   }
   for (int dt = 0; dt < 2; ++dt)
     if (!eu[dt].empty() &&
-        launch_euclid_group(eu[dt].data(), (int)eu[dt].size(), (gift_dtype)dt, encode, s) != cudaSuccess)
+        launch_euclid_group(eu[dt].data(), (int)eu[dt].size(), (gift_dtype)dt, encode, dev_status, s) != cudaSuccess)
       return GIFT_ERR_CUDA;
   if (!tc.empty()) {
-    cudaError_t e = encode ? launch_whiten_encode_tc(tc.data(), (int)tc.size(), s)
-                           : launch_whiten_decode_tc(tc.data(), (int)tc.size(), s);
+    cudaError_t e = encode ? launch_whiten_encode_tc(tc.data(), (int)tc.size(), dev_status, s)
+                           : launch_whiten_decode_tc(tc.data(), (int)tc.size(), dev_status, s);
     if (e != cudaSuccess) return GIFT_ERR_CUDA;
   }
   return GIFT_OK;
@@ -246,11 +255,28 @@ gift_status gift_codec_split(const gift_layer* layers, int n, int encode, int* s
   return GIFT_OK;
 }
 
-gift_status gift_encode_many(const gift_layer* layers, int n, gift_stream_t stream) {
-  return run_many(layers, n, stream, true);
+gift_status gift_encode_many(const gift_layer* layers, int n, uint32_t* dev_status, gift_stream_t stream) {
+  return run_many(layers, n, dev_status, stream, true);
 }
-gift_status gift_decode_many(const gift_layer* layers, int n, gift_stream_t stream) {
-  return run_many(layers, n, stream, false);
+gift_status gift_decode_many(const gift_layer* layers, int n, uint32_t* dev_status, gift_stream_t stream) {
+  return run_many(layers, n, dev_status, stream, false);
+}
+
+gift_status gift_codec_stall_test(const gift_layer* layer, int encode, uint32_t stall_polls, uint32_t* dev_status,
+                                  gift_stream_t stream) {
+  if (!layer || !dev_status || stall_polls == 0) return GIFT_ERR_INVALID_ARG;
+  const gift_layer& L = *layer;
+  const void* g = encode ? L.G : (const void*)L.G_hat;
+  gift_status st = check_codec_args(g, L.dtype, L.d_out, L.d_in, L.U, L.lambda, L.rho, L.rank, L.codes, L.scales);
+  if (st != GIFT_OK) return st;
+  if (!aligned(dev_status, 4)) return GIFT_ERR_ALIGN;
+  if (L.d_out == 0 || L.rank == 0) return GIFT_ERR_INVALID_ARG;
+  if ((st = device_ok()) != GIFT_OK) return st;
+  if (!use_tc(L.dtype, L.rank, L.d_in)) return GIFT_ERR_UNSUPPORTED;
+  TcLayer T{L.G, L.G_hat, L.codes, L.scales, L.U, L.lambda, L.rho, (int)L.d_out, (int)L.d_in, L.rank};
+  cudaStream_t s = (cudaStream_t)stream;
+  return cuda_status(encode ? launch_whiten_encode_tc(&T, 1, dev_status, s, stall_polls)
+                            : launch_whiten_decode_tc(&T, 1, dev_status, s, stall_polls));
 }
 
 // ---------------------------------------------------------------------------
@@ -320,9 +346,11 @@ static gift_status check_nvfp4_args(const void* G, int gdt, int64_t d_out, int64
 
 gift_status gift_encode_nvfp4(const void* G, gift_dtype gdt, int64_t d_out, int64_t d_in, const float* U,
                               const float* lambda, const float* rho, int rank, uint8_t* codes,
-                              uint8_t* block_scales, float* tensor_scale, gift_stream_t stream) {
+                              uint8_t* block_scales, float* tensor_scale, uint32_t* dev_status, gift_stream_t stream) {
   gift_status st = check_nvfp4_args(G, gdt, d_out, d_in, U, lambda, rho, rank, codes, block_scales, tensor_scale);
-  if (st != GIFT_OK || d_out == 0) return st;
+  if (st != GIFT_OK) return st;
+  if (dev_status && !aligned(dev_status, 4)) return GIFT_ERR_ALIGN;
+  if (d_out == 0) return GIFT_OK;
   if ((st = device_ok()) != GIFT_OK) return st;
   if (rank > 0 && !tc_codec_available()) return GIFT_ERR_UNSUPPORTED;
   cudaStream_t s = (cudaStream_t)stream;
@@ -337,30 +365,33 @@ gift_status gift_encode_nvfp4(const void* G, gift_dtype gdt, int64_t d_out, int6
     L.block_scales = block_scales;
     L.tensor_scale = tensor_scale;
     L.fmt = kFmtNvfp4Amax;
-    if ((st = cuda_status(launch_whiten_encode_tc(&L, 1, s))) != GIFT_OK) return st;
+    if ((st = cuda_status(launch_whiten_encode_tc(&L, 1, dev_status, s))) != GIFT_OK) return st;
     L.fmt = kFmtNvfp4;
-    if ((st = cuda_status(launch_whiten_encode_tc(&L, 1, s))) != GIFT_OK) return st;
+    if ((st = cuda_status(launch_whiten_encode_tc(&L, 1, dev_status, s))) != GIFT_OK) return st;
   }
-  return cuda_status(launch_nvfp4_finalize(tensor_scale, s));
+  return cuda_status(launch_nvfp4_finalize(tensor_scale, dev_status, s));
 }
 
 gift_status gift_decode_nvfp4(const uint8_t* codes, const uint8_t* block_scales, const float* tensor_scale,
                               int64_t d_out, int64_t d_in, const float* U, const float* lambda, const float* rho,
-                              int rank, void* G_hat, gift_dtype out_dt, gift_stream_t stream) {
+                              int rank, void* G_hat, gift_dtype out_dt, uint32_t* dev_status,
+                              gift_stream_t stream) {
   gift_status st =
       check_nvfp4_args(G_hat, out_dt, d_out, d_in, U, lambda, rho, rank, codes, block_scales, tensor_scale);
-  if (st != GIFT_OK || d_out == 0) return st;
+  if (st != GIFT_OK) return st;
+  if (dev_status && !aligned(dev_status, 4)) return GIFT_ERR_ALIGN;
+  if (d_out == 0) return GIFT_OK;
   if ((st = device_ok()) != GIFT_OK) return st;
   if (rank > 0 && !tc_codec_available()) return GIFT_ERR_UNSUPPORTED;
   cudaStream_t s = (cudaStream_t)stream;
   if (rank == 0)
     return cuda_status(launch_nvfp4_decode(codes, block_scales, tensor_scale, d_out * (d_in / GIFT_NVFP4_BLOCK),
-                                           G_hat, out_dt, s));
+                                           G_hat, out_dt, dev_status, s));
   TcLayer L{nullptr, G_hat, (uint8_t*)codes, nullptr, U, lambda, rho, (int)d_out, (int)d_in, rank};
   L.block_scales = (uint8_t*)block_scales;
   L.tensor_scale = (float*)tensor_scale;
   L.fmt = kFmtNvfp4;
-  return cuda_status(launch_whiten_decode_tc(&L, 1, s));
+  return cuda_status(launch_whiten_decode_tc(&L, 1, dev_status, s));
 }
 
 }  // extern "C"

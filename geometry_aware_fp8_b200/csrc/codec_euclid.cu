@@ -77,8 +77,10 @@ GIFT_DEV uint4 quantize16(const float (&v)[16], float inv) {
 
 template <typename T>
 __global__ void __launch_bounds__(256) euclid_encode_kernel(const T* __restrict__ G, uint8_t* __restrict__ codes,
-                                                            float* __restrict__ scales, int64_t n_blocks) {
+                                                            float* __restrict__ scales, int64_t n_blocks,
+                                                            uint32_t* err) {
   const int sub = threadIdx.x & 7;
+  bool bad = false;
   const int64_t groups_per_grid = (int64_t)gridDim.x * (blockDim.x >> 3);
   for (int64_t b = (int64_t)blockIdx.x * (blockDim.x >> 3) + (threadIdx.x >> 3); b < n_blocks;
        b += groups_per_grid) {
@@ -87,27 +89,31 @@ __global__ void __launch_bounds__(256) euclid_encode_kernel(const T* __restrict_
     Vec16<T>::load(G + e0, v);
     float m = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[i]));
-    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+    for (int i = 0; i < 16; ++i) m = fmax_nan(m, fabsf(v[i]));
+    m = fmax_nan(m, __shfl_xor_sync(0xffffffffu, m, 1));
+    m = fmax_nan(m, __shfl_xor_sync(0xffffffffu, m, 2));
+    m = fmax_nan(m, __shfl_xor_sync(0xffffffffu, m, 4));
+    bad |= not_finite(m);
     const float inv = e4m3_inv_scale(m);
     __stcs(reinterpret_cast<uint4*>(codes + e0), quantize16(v, inv));
     if (sub == 0) scales[b] = e4m3_scale(m, inv);
   }
+  report_bits(err, bad, GIFT_DEV_NONFINITE);
 }
 
 template <typename T>
 __global__ void __launch_bounds__(256) euclid_decode_kernel(const uint8_t* __restrict__ codes,
                                                             const float* __restrict__ scales, T* __restrict__ out,
-                                                            int64_t n_blocks) {
+                                                            int64_t n_blocks, uint32_t* err) {
   const int sub = threadIdx.x & 7;
+  bool bad = false;
   const int64_t groups_per_grid = (int64_t)gridDim.x * (blockDim.x >> 3);
   for (int64_t b = (int64_t)blockIdx.x * (blockDim.x >> 3) + (threadIdx.x >> 3); b < n_blocks;
        b += groups_per_grid) {
     const int64_t e0 = b * kBlock + sub * 16;
     const uint4 q = __ldcs(reinterpret_cast<const uint4*>(codes + e0));
     const float s = __ldg(scales + b);
+    bad |= not_finite(s);
     uint32_t w[4] = {q.x, q.y, q.z, q.w};
     float v[16];
 #pragma unroll
@@ -121,6 +127,7 @@ __global__ void __launch_bounds__(256) euclid_decode_kernel(const uint8_t* __res
     }
     Vec16<T>::store(out + e0, v);
   }
+  report_bits(err, bad, GIFT_DEV_NONFINITE);
 }
 
 // Grouped form: many layers in one launch.  A block index b of the
@@ -136,6 +143,7 @@ struct EuclidGroup {
   float* scales[kGroupMax];
   int64_t prefix[kGroupMax + 1];  // prefix[i] = first block of layer i
   int n;
+  uint32_t* err;                  // device status word (nullable)
 };
 
 GIFT_DEV int find_layer(const int64_t* pre, int n, int64_t b) {
@@ -164,6 +172,7 @@ __global__ void __launch_bounds__(256) euclid_encode_group_kernel(const __grid_c
   const int64_t G = (int64_t)gridDim.x * (blockDim.x >> 3);
   const int64_t first = (int64_t)blockIdx.x * (blockDim.x >> 3) + (threadIdx.x >> 3);
   int l0 = first < total ? find_layer(pre, g.n, first) : 0, l1 = l0;
+  bool bad = false;
   for (int64_t b0 = first; b0 < total; b0 += 2 * G) {
     const int64_t b1 = b0 + G;
     const bool has1 = b1 < total;
@@ -177,14 +186,15 @@ __global__ void __launch_bounds__(256) euclid_encode_group_kernel(const __grid_c
     float m0 = 0.0f, m1 = 0.0f;
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-      m0 = fmaxf(m0, fabsf(v0[i]));
-      m1 = fmaxf(m1, fabsf(v1[i]));
+      m0 = fmax_nan(m0, fabsf(v0[i]));
+      m1 = fmax_nan(m1, fabsf(v1[i]));
     }
 #pragma unroll
     for (int o = 1; o < 8; o <<= 1) {
-      m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, o));
-      m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, o));
+      m0 = fmax_nan(m0, __shfl_xor_sync(0xffffffffu, m0, o));
+      m1 = fmax_nan(m1, __shfl_xor_sync(0xffffffffu, m1, o));
     }
+    bad |= not_finite(m0) || (has1 && not_finite(m1));
     const float i0 = e4m3_inv_scale(m0);
     __stcs(reinterpret_cast<uint4*>((uint8_t*)g.dst[l0] + e0), quantize16(v0, i0));
     if (sub == 0) g.scales[l0][b0 - pre[l0]] = e4m3_scale(m0, i0);
@@ -194,6 +204,7 @@ __global__ void __launch_bounds__(256) euclid_encode_group_kernel(const __grid_c
       if (sub == 0) g.scales[l1][b1 - pre[l1]] = e4m3_scale(m1, i1);
     }
   }
+  report_bits(g.err, bad, GIFT_DEV_NONFINITE);
 }
 
 GIFT_DEV void dequant16(uint4 q, float s, float (&v)[16]) {
@@ -217,6 +228,7 @@ __global__ void __launch_bounds__(256) euclid_decode_group_kernel(const __grid_c
   const int sub = threadIdx.x & 7;
   const int64_t total = pre[g.n];
   const int64_t G = (int64_t)gridDim.x * (blockDim.x >> 3);
+  bool bad = false;
   for (int64_t b0 = (int64_t)blockIdx.x * (blockDim.x >> 3) + (threadIdx.x >> 3); b0 < total; b0 += 2 * G) {
     const int64_t b1 = b0 + G;
     const bool has1 = b1 < total;
@@ -232,6 +244,7 @@ __global__ void __launch_bounds__(256) euclid_decode_group_kernel(const __grid_c
       q1 = __ldcs(reinterpret_cast<const uint4*>((const uint8_t*)g.src[l1] + e1));
       s1 = __ldg(g.scales[l1] + lb1);
     }
+    bad |= not_finite(s0) || not_finite(s1);
     float v[16];
     dequant16(q0, s0, v);
     Vec16<T>::store((T*)g.dst[l0] + e0, v);
@@ -240,6 +253,7 @@ __global__ void __launch_bounds__(256) euclid_decode_group_kernel(const __grid_c
       Vec16<T>::store((T*)g.dst[l1] + e1, v);
     }
   }
+  report_bits(g.err, bad, GIFT_DEV_NONFINITE);
 }
 
 inline int grid_for(int64_t n_blocks) {
@@ -253,24 +267,24 @@ inline int grid_for(int64_t n_blocks) {
 }  // namespace
 
 cudaError_t launch_euclid_encode(const void* G, gift_dtype dt, int64_t n_blocks, uint8_t* codes, float* scales,
-                                 cudaStream_t s) {
+                                 uint32_t* err, cudaStream_t s) {
   if (n_blocks == 0) return cudaSuccess;
   const int grid = grid_for(n_blocks);
   if (dt == GIFT_BF16)
-    euclid_encode_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>((const __nv_bfloat16*)G, codes, scales, n_blocks);
+    euclid_encode_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>((const __nv_bfloat16*)G, codes, scales, n_blocks, err);
   else
-    euclid_encode_kernel<float><<<grid, 256, 0, s>>>((const float*)G, codes, scales, n_blocks);
+    euclid_encode_kernel<float><<<grid, 256, 0, s>>>((const float*)G, codes, scales, n_blocks, err);
   return cudaGetLastError();
 }
 
 cudaError_t launch_euclid_decode(const uint8_t* codes, const float* scales, int64_t n_blocks, void* G_hat,
-                                 gift_dtype dt, cudaStream_t s) {
+                                 gift_dtype dt, uint32_t* err, cudaStream_t s) {
   if (n_blocks == 0) return cudaSuccess;
   const int grid = grid_for(n_blocks);
   if (dt == GIFT_BF16)
-    euclid_decode_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(codes, scales, (__nv_bfloat16*)G_hat, n_blocks);
+    euclid_decode_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(codes, scales, (__nv_bfloat16*)G_hat, n_blocks, err);
   else
-    euclid_decode_kernel<float><<<grid, 256, 0, s>>>(codes, scales, (float*)G_hat, n_blocks);
+    euclid_decode_kernel<float><<<grid, 256, 0, s>>>(codes, scales, (float*)G_hat, n_blocks, err);
   return cudaGetLastError();
 }
 
@@ -291,11 +305,13 @@ int group_grid(K kernel, int slot, int64_t n_blocks) {
   return (int)(need < res ? need : res);
 }
 
-cudaError_t launch_euclid_group(const EuclidLayer* layers, int n, gift_dtype dt, bool encode, cudaStream_t s) {
+cudaError_t launch_euclid_group(const EuclidLayer* layers, int n, gift_dtype dt, bool encode, uint32_t* err,
+                               cudaStream_t s) {
   for (int base = 0; base < n; base += kGroupMax) {
     const int cnt = n - base < kGroupMax ? n - base : kGroupMax;
     EuclidGroup g;
     g.n = cnt;
+    g.err = err;
     int64_t tot = 0;
     for (int i = 0; i < cnt; ++i) {
       const EuclidLayer& L = layers[base + i];

@@ -44,7 +44,7 @@ template <typename T>
 __global__ void __launch_bounds__(kWarps * 32) whiten_encode_simt_kernel(
     const T* __restrict__ G, int64_t d_out, int64_t d_in, const float* __restrict__ U,
     const float* __restrict__ lambda, const float* __restrict__ rho, int rank, uint8_t* __restrict__ codes,
-    float* __restrict__ scales) {
+    float* __restrict__ scales, uint32_t* err) {
   __shared__ float c_s[32];
   __shared__ float a_s;
   __shared__ float part[kWarps][32];
@@ -55,6 +55,7 @@ __global__ void __launch_bounds__(kWarps * 32) whiten_encode_simt_kernel(
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool vec = (rank & 3) == 0;
   const int64_t nb = d_in / kBlock;
+  bool bad = false;
   for (int64_t row = blockIdx.x; row < d_out; row += gridDim.x) {
     const T* g = G + row * d_in;
     float P[32];
@@ -88,9 +89,11 @@ __global__ void __launch_bounds__(kWarps * 32) whiten_encode_simt_kernel(
 #pragma unroll
         for (int k = 0; k < 32; ++k) acc = fmaf(pc[k], u[k], acc);
         w[e] = fmaf(a, v[e], acc);
-        m = fmaxf(m, fabsf(w[e]));
+        m = fmax_nan(m, fabsf(w[e]));
       }
-      m = warp_max(m);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = fmax_nan(m, __shfl_xor_sync(0xffffffffu, m, o));
+      bad |= not_finite(m);
       uint32_t q = 0u;
       const float inv = e4m3_inv_scale(m);
       if (inv > 0.0f) {
@@ -102,13 +105,14 @@ __global__ void __launch_bounds__(kWarps * 32) whiten_encode_simt_kernel(
       if (lane == 0) scales[row * nb + b] = e4m3_scale(m, inv);
     }
   }
+  report_bits(err, bad, GIFT_DEV_NONFINITE);
 }
 
 template <typename T>
 __global__ void __launch_bounds__(kWarps * 32) whiten_decode_simt_kernel(
     const uint8_t* __restrict__ codes, const float* __restrict__ scales, int64_t d_out, int64_t d_in,
     const float* __restrict__ U, const float* __restrict__ lambda, const float* __restrict__ rho, int rank,
-    T* __restrict__ out) {
+    T* __restrict__ out, uint32_t* err) {
   __shared__ float c_s[32];
   __shared__ float a_s;
   __shared__ float part[kWarps][32];
@@ -119,6 +123,7 @@ __global__ void __launch_bounds__(kWarps * 32) whiten_decode_simt_kernel(
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool vec = (rank & 3) == 0;
   const int64_t nb = d_in / kBlock;
+  bool bad = false;
   for (int64_t row = blockIdx.x; row < d_out; row += gridDim.x) {
     float P[32];
 #pragma unroll
@@ -143,6 +148,7 @@ __global__ void __launch_bounds__(kWarps * 32) whiten_decode_simt_kernel(
       const int64_t j0 = b * kBlock + lane * 4;
       const uint32_t q = __ldg(reinterpret_cast<const uint32_t*>(codes + row * d_in + j0));
       const float s = __ldg(scales + row * nb + b);
+      bad |= not_finite(s);
       float2 lo = e4m3x2_to_f32x2((uint16_t)(q & 0xFFFF)), hi = e4m3x2_to_f32x2((uint16_t)(q >> 16));
       const float v[4] = {lo.x * s, lo.y * s, hi.x * s, hi.y * s};
       float o[4];
@@ -158,6 +164,7 @@ __global__ void __launch_bounds__(kWarps * 32) whiten_decode_simt_kernel(
       store4<T>(out + row * d_in + j0, o);
     }
   }
+  report_bits(err, bad, GIFT_DEV_NONFINITE);
 }
 
 // One CTA per row, capped at a few waves of resident CTAs (rows are then
@@ -171,27 +178,27 @@ int grid_rows(int64_t d_out) {
 
 cudaError_t launch_whiten_encode_simt(const void* G, gift_dtype dt, int64_t d_out, int64_t d_in, const float* U,
                                       const float* lambda, const float* rho, int rank, uint8_t* codes,
-                                      float* scales, cudaStream_t s) {
+                                      float* scales, uint32_t* err, cudaStream_t s) {
   const int grid = grid_rows(d_out);
   if (dt == GIFT_BF16)
     whiten_encode_simt_kernel<__nv_bfloat16><<<grid, kWarps * 32, 0, s>>>(
-        (const __nv_bfloat16*)G, d_out, d_in, U, lambda, rho, rank, codes, scales);
+        (const __nv_bfloat16*)G, d_out, d_in, U, lambda, rho, rank, codes, scales, err);
   else
     whiten_encode_simt_kernel<float><<<grid, kWarps * 32, 0, s>>>((const float*)G, d_out, d_in, U, lambda, rho,
-                                                                   rank, codes, scales);
+                                                                   rank, codes, scales, err);
   return cudaGetLastError();
 }
 
 cudaError_t launch_whiten_decode_simt(const uint8_t* codes, const float* scales, int64_t d_out, int64_t d_in,
                                       const float* U, const float* lambda, const float* rho, int rank,
-                                      void* G_hat, gift_dtype dt, cudaStream_t s) {
+                                      void* G_hat, gift_dtype dt, uint32_t* err, cudaStream_t s) {
   const int grid = grid_rows(d_out);
   if (dt == GIFT_BF16)
     whiten_decode_simt_kernel<__nv_bfloat16><<<grid, kWarps * 32, 0, s>>>(codes, scales, d_out, d_in, U, lambda,
-                                                                          rho, rank, (__nv_bfloat16*)G_hat);
+                                                                          rho, rank, (__nv_bfloat16*)G_hat, err);
   else
     whiten_decode_simt_kernel<float><<<grid, kWarps * 32, 0, s>>>(codes, scales, d_out, d_in, U, lambda, rho,
-                                                                  rank, (float*)G_hat);
+                                                                  rank, (float*)G_hat, err);
   return cudaGetLastError();
 }
 

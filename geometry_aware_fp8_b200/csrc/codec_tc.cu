@@ -68,6 +68,17 @@ constexpr uint32_t kIdescE1 = umma_idesc_bf16(128, 64, 0, 1);   // A K-major, B 
 constexpr uint32_t kIdescE2 = umma_idesc_bf16(128, 128, 0, 0);  // both K-major
 constexpr uint32_t kIdescId = umma_idesc_bf16(128, 16, 0, 0);   // G . I16, both K-major
 constexpr uint32_t kWaitLimit = 1u << 22;
+#ifndef GIFT_ENC_PREFETCH
+#define GIFT_ENC_PREFETCH 0
+#endif
+#ifndef GIFT_DEC_PREFETCH
+#define GIFT_DEC_PREFETCH 0
+#endif
+#ifndef GIFT_PF_PASS2
+#define GIFT_PF_PASS2 1
+#endif
+constexpr int kEncPrefetch = GIFT_ENC_PREFETCH;  // steps of G the producer prefetches into L2 ahead of its loads
+constexpr int kDecPrefetch = GIFT_DEC_PREFETCH;
 constexpr int kMaxJobs = 48;
 constexpr int kMaxPanels = 1536;
 
@@ -90,6 +101,7 @@ struct EncParams {
   uint16_t sched_off[kNumSMs + 1];  // cluster b runs sched_ids[sched_off[b] .. sched_off[b+1])
   uint16_t sched_ids[kMaxPanels];   // job << 8 | panel
   int split;                        // CTAs per cluster, each taking 1 / split of every panel's chunks
+  uint32_t stall_polls;             // test hook (0 = off): see stall_check
 };
 static_assert(sizeof(EncParams) <= 32760, "kernel parameter space");
 
@@ -126,6 +138,13 @@ GIFT_DEV void tma_store_2d_hint(const void* tmap, uint32_t src, int x, int y, ui
       " [%0, {%2, %3}], [%1], %4;" ::"l"(tmap),
       "r"(src), "r"(x), "r"(y), "l"(policy)
       : "memory");
+}
+// 2-D tiled TMA prefetch global -> L2 (no shared-memory destination, no
+// completion to wait for): brings a box the ring will load later into L2.
+GIFT_DEV void tma_prefetch_2d(const void* tmap, int x, int y, uint64_t policy) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile.L2::cache_hint [%0, {%1, %2}], %3;" ::"l"(tmap),
+               "r"(x), "r"(y), "l"(policy)
+               : "memory");
 }
 GIFT_DEV void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Wait until at most N committed store groups still read shared memory.
@@ -197,6 +216,15 @@ GIFT_DEV bool named_sync_or(int id, int n, bool v) {
       : "r"(id), "r"(n), "r"((uint32_t)v)
       : "memory");
   return r != 0;
+}
+
+// Test hook of the failure path (stall_polls > 0): before any load or MMA is
+// issued, thread 0 waits at most stall_polls polls on `bar`, a barrier that
+// nothing arrives at; the wait runs out and sets *failed.  The caller then
+// syncs the CTA and every role skips its work, so the kernel returns with
+// nothing in flight and reports GIFT_DEV_TIMEOUT.
+GIFT_DEV void stall_check(uint32_t stall_polls, uint64_t* bar, int* failed) {
+  if (stall_polls && threadIdx.x == 0 && !mbar_wait(bar, 0u, stall_polls)) *failed = 1;
 }
 
 GIFT_DEV void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
@@ -381,8 +409,10 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
   uint64_t* cfree = p_full + 8;           // [2] count 1: the store of a codes tile has read it
   uint64_t* xfull = p_full + 10;          // count 256 (S-1): the peers' partials are written (clusters)
   uint64_t* xempty = p_full + 11;         // count 256 (S-1): the peers have read this CTA's partial
-  uint32_t* tmem_slot = (uint32_t*)(p_full + 12);
+  uint64_t* stall = p_full + 12;          // count 1, never arrived at (test hook)
+  uint32_t* tmem_slot = (uint32_t*)(p_full + 13);
   __shared__ int failed;  // any role gave up (reported at exit)
+  __shared__ int nonfin;  // a block maximum was not finite (reported at exit)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int S = CLUSTER ? p.split : 1;  // without clusters, the split arithmetic folds away
@@ -391,6 +421,7 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
 
   if (threadIdx.x == 0) {
     failed = 0;
+    nonfin = 0;
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
@@ -398,6 +429,7 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
     }
     mbar_init(p_full, 1);
     mbar_init(pc_full, 256);
+    mbar_init(stall, 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&w_full[b], 1);
       mbar_init(&w_empty[b], 256);
@@ -431,18 +463,36 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
   tc_fence_after();
   if (CLUSTER) cluster_sync_all();  // the peers' barriers are initialised before any remote arrive
   const uint32_t tbase = *tmem_slot;
+  stall_check(p.stall_polls, stall, &failed);
+  __syncthreads();
+  const bool skip = failed != 0;  // the same for every thread: read after the barrier
 
-  if (warp == 13) {
+  if (skip) {
+    // the test hook's wait ran out: nothing was issued, nothing to do
+  } else if (warp == 13) {
     // ---------------- TMA producer: G chunks and U rows, running ahead of the ring ----------------
     if (lane == 0) {
       const uint64_t keep = policy_evict_last(), drop = policy_evict_first();
       uint32_t step = 0;
+      Steps<EncParams> ahead(p, beg, end, q, S);
+      auto prefetch = [&](const Steps<EncParams>& a) {
+        if (a.pass == 0 || GIFT_PF_PASS2) {
+          const EncJob& J = p.jobs[a.job()];
+          tma_prefetch_2d(&J.tmG, a.chunk() * kChunk, a.panel() * kPanel, a.pass == 0 ? keep : drop);
+          tma_prefetch_2d(&J.tmG, a.chunk() * kChunk + 64, a.panel() * kPanel, a.pass == 0 ? keep : drop);
+        }
+      };
+      for (int i = 0; i < kEncPrefetch && ahead.valid(); ++i, ahead.next()) prefetch(ahead);
       for (Steps<EncParams> st(p, beg, end, q, S); st.valid() && !failed; st.next(), ++step) {
         const int s = step % kStages;
         const uint32_t use = step / kStages;
         if (step >= kStages && !mbar_wait(&empty[s], (use - 1) & 1u, kWaitLimit)) {
           failed = 1;
           break;
+        }
+        if (kEncPrefetch > 0 && ahead.valid()) {
+          prefetch(ahead);
+          ahead.next();
         }
         const EncJob& J = p.jobs[st.job()];
         const uint64_t pol = st.pass == 0 ? keep : drop;
@@ -639,12 +689,12 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
       float m0 = 0.0f, m1 = 0.0f, m2 = 0.0f, m3 = 0.0f;
 #pragma unroll
       for (int k = 0; k < 64; k += 4) {
-        m0 = fmaxf(m0, fabsf(__uint_as_float(w[k])));
-        m1 = fmaxf(m1, fabsf(__uint_as_float(w[k + 1])));
-        m2 = fmaxf(m2, fabsf(__uint_as_float(w[k + 2])));
-        m3 = fmaxf(m3, fabsf(__uint_as_float(w[k + 3])));
+        m0 = fmax_nan(m0, fabsf(__uint_as_float(w[k])));
+        m1 = fmax_nan(m1, fabsf(__uint_as_float(w[k + 1])));
+        m2 = fmax_nan(m2, fabsf(__uint_as_float(w[k + 2])));
+        m3 = fmax_nan(m3, fabsf(__uint_as_float(w[k + 3])));
       }
-      amax_x[h][r] = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+      amax_x[h][r] = fmax_nan(fmax_nan(m0, m1), fmax_nan(m2, m3));
       if (FMT == kFmtNvfp4Amax) {
         // amax(W) = a max|W'| (rounded once); one atomic per warp at the panel's end
         pmax = fmaxf(pmax, live ? amax_x[h][r] : 0.0f);
@@ -681,7 +731,8 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
         break;
       }
       // block maximum of W = a W' (rounded once), then the codes of W' x (a 448 / amax)
-      const float amax = __fmul_rn(a, fmaxf(amax_x[0][r], amax_x[1][r]));
+      const float amax = __fmul_rn(a, fmax_nan(amax_x[0][r], amax_x[1][r]));
+      if (live && h == 0 && not_finite(amax)) nonfin = 1;
       const float inv = e4m3_inv_scale(amax);
       const float ai = __fmul_rn(a, inv);
       uint32_t cw[16];
@@ -707,7 +758,8 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
   __syncthreads();
   if (CLUSTER) cluster_sync_all();
   if (warp == 12) tmem_dealloc(tbase, kTmemCols);
-  if (threadIdx.x == 0 && failed && err) atomicOr(err, GIFT_DEV_TIMEOUT);
+  if (threadIdx.x == 0 && err && (failed || nonfin))
+    atomicOr(err, (failed ? GIFT_DEV_TIMEOUT : 0u) | (nonfin ? GIFT_DEV_NONFINITE : 0u));
 }
 
 // ===========================================================================
@@ -759,6 +811,7 @@ struct DecParams {
   uint16_t sched_off[kNumSMs + 1];  // cluster b runs sched_ids[sched_off[b] .. sched_off[b+1])
   uint16_t sched_ids[kMaxPanels];   // job << 8 | panel
   int split;                        // CTAs per cluster, each taking 1 / split of every panel's chunks
+  uint32_t stall_polls;             // test hook (0 = off): see stall_check
 };
 static_assert(sizeof(DecParams) <= 32760, "kernel parameter space");
 
@@ -791,8 +844,10 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
   uint64_t* w_empty = t_full + 7;          // [2] count 256
   uint64_t* xfull = t_full + 9;            // count 256 (S-1): the peers' partials are written (clusters)
   uint64_t* xempty = t_full + 10;          // count 256 (S-1): the peers have read this CTA's partial
-  uint32_t* tmem_slot = (uint32_t*)(t_full + 11);
+  uint64_t* stall = t_full + 11;           // count 1, never arrived at (test hook)
+  uint32_t* tmem_slot = (uint32_t*)(t_full + 12);
   __shared__ int failed;
+  __shared__ int nonfin;  // a block scale was not finite (reported at exit)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int S = CLUSTER ? p.split : 1;  // without clusters, the split arithmetic folds away
@@ -800,6 +855,8 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
   const int beg = p.sched_off[blockIdx.x / S], end = p.sched_off[blockIdx.x / S + 1];
   if (threadIdx.x == 0) {
     failed = 0;
+    nonfin = 0;
+    mbar_init(stall, 1);
     for (int s = 0; s < kDStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&cfull[s], 1);
@@ -829,18 +886,33 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
   tc_fence_after();
   if (CLUSTER) cluster_sync_all();  // the peers' barriers are initialised before any remote arrive
   const uint32_t tbase = *tmem_slot;
+  stall_check(p.stall_polls, stall, &failed);
+  __syncthreads();
+  const bool skip = failed != 0;  // the same for every thread: read after the barrier
 
-  if (warp == 13) {
+  if (skip) {
+    // the test hook's wait ran out: nothing was issued, nothing to do
+  } else if (warp == 13) {
     // ---------------- TMA producer: codes chunks and U rows, running ahead of the ring ----------------
     if (lane == 0) {
       const uint64_t keep = policy_evict_last(), drop = policy_evict_first();
       uint32_t step = 0;
+      Steps<DecParams> ahead(p, beg, end, q, S);
+      auto prefetch = [&](const Steps<DecParams>& a) {
+        if (FMT == kFmtE4M3 && (a.pass == 0 || GIFT_PF_PASS2))
+          tma_prefetch_2d(&p.jobs[a.job()].tmC, a.chunk() * kChunk, a.panel() * kPanel, a.pass == 0 ? keep : drop);
+      };
+      for (int i = 0; i < kDecPrefetch && ahead.valid(); ++i, ahead.next()) prefetch(ahead);
       for (Steps<DecParams> st(p, beg, end, q, S); st.valid() && !failed; st.next(), ++step) {
         const int s = step % kDStages;
         const uint32_t use = step / kDStages;
         if (step >= kDStages && !mbar_wait(&empty[s], (use - 1) & 1u, kWaitLimit)) {
           failed = 1;
           break;
+        }
+        if (kDecPrefetch > 0 && ahead.valid()) {
+          prefetch(ahead);
+          ahead.next();
         }
         const DecJob& J = p.jobs[st.job()];
         const uint32_t dst = sbase + s * kDStageBytes;
@@ -1023,6 +1095,7 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
       // E4M3: the chunk's fp32 block scale; NVFP4: the tensor scale (the block
       // scales are inside the widened values)
       const float sc = !live ? 0.0f : (FMT == kFmtE4M3 ? __ldg(J.scales + row * nc + c) : __ldg(J.tscale));
+      if (not_finite(sc)) nonfin = 1;
       if (st.block_start() && st.k >= 1) {
         // P of p_{k-1} is complete (in a cluster: this CTA's chunks of it,
         // summed over the cluster here): P o c -> bf16 hi/lo A operand of D3
@@ -1152,7 +1225,8 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
   __syncthreads();
   if (CLUSTER) cluster_sync_all();
   if (warp == 12) tmem_dealloc(tbase, kTmemCols);
-  if (threadIdx.x == 0 && failed && err) atomicOr(err, GIFT_DEV_TIMEOUT);
+  if (threadIdx.x == 0 && err && (failed || nonfin))
+    atomicOr(err, (failed ? GIFT_DEV_TIMEOUT : 0u) | (nonfin ? GIFT_DEV_NONFINITE : 0u));
 }
 
 unsigned long long g_dec_attr[3][2] = {};
@@ -1161,11 +1235,11 @@ unsigned long long g_enc_attr[3][2] = {};
 // One launch of `grid` clusters of S CTAs (S = 1: a plain launch).
 template <class Prm>
 cudaError_t launch_clusters(void (*kern)(Prm, uint32_t*), int smem, unsigned long long* attr, int grid, int S,
-                            const Prm& P, cudaStream_t s) {
+                            const Prm& P, uint32_t* err, cudaStream_t s) {
   cudaError_t e = ensure_smem_attr(kern, smem, attr);
   if (e != cudaSuccess) return e;
   if (S == 1) {
-    kern<<<grid, kThreads, smem, s>>>(P, nullptr);
+    kern<<<grid, kThreads, smem, s>>>(P, err);
     return cudaGetLastError();
   }
   cudaLaunchConfig_t cfg = {};
@@ -1180,7 +1254,7 @@ cudaError_t launch_clusters(void (*kern)(Prm, uint32_t*), int smem, unsigned lon
   at[0].val.clusterDim.z = 1;
   cfg.attrs = at;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, P, (uint32_t*)nullptr);
+  return cudaLaunchKernelEx(&cfg, kern, P, err);
 }
 
 // Clusters of S CTAs of this kernel that can be resident at once (0 if none).
@@ -1234,35 +1308,37 @@ int dec_slots(int fmt, int S) {
 }
 
 template <int FMT>
-cudaError_t enc_launch_fmt(int grid, const EncParams& P, cudaStream_t s) {
+cudaError_t enc_launch_fmt(int grid, const EncParams& P, uint32_t* err, cudaStream_t s) {
   const int f = FMT == kFmtE4M3 ? 0 : FMT == kFmtNvfp4Amax ? 1 : 2;
   if (P.split > 1)
-    return launch_clusters(whiten_encode_tc_kernel<FMT, true>, enc_smem(true), &g_enc_attr[f][1], grid, P.split, P, s);
-  return launch_clusters(whiten_encode_tc_kernel<FMT, false>, enc_smem(false), &g_enc_attr[f][0], grid, 1, P, s);
+    return launch_clusters(whiten_encode_tc_kernel<FMT, true>, enc_smem(true), &g_enc_attr[f][1], grid, P.split, P,
+                           err, s);
+  return launch_clusters(whiten_encode_tc_kernel<FMT, false>, enc_smem(false), &g_enc_attr[f][0], grid, 1, P, err, s);
 }
 
 template <int FMT>
-cudaError_t dec_launch_fmt(int grid, const DecParams& P, cudaStream_t s) {
+cudaError_t dec_launch_fmt(int grid, const DecParams& P, uint32_t* err, cudaStream_t s) {
   const int f = FMT == kFmtE4M3 ? 0 : 2;
   if (P.split > 1)
-    return launch_clusters(whiten_decode_tc_kernel<FMT, true>, dec_smem(true), &g_dec_attr[f][1], grid, P.split, P, s);
-  return launch_clusters(whiten_decode_tc_kernel<FMT, false>, dec_smem(false), &g_dec_attr[f][0], grid, 1, P, s);
+    return launch_clusters(whiten_decode_tc_kernel<FMT, true>, dec_smem(true), &g_dec_attr[f][1], grid, P.split, P,
+                           err, s);
+  return launch_clusters(whiten_decode_tc_kernel<FMT, false>, dec_smem(false), &g_dec_attr[f][0], grid, 1, P, err, s);
 }
 
 // One launch runs layers of one format (its kernel instantiation).
-cudaError_t enc_launch(int fmt, int grid, const EncParams& P, cudaStream_t s) {
+cudaError_t enc_launch(int fmt, int grid, const EncParams& P, uint32_t* err, cudaStream_t s) {
   switch (fmt) {
-    case kFmtE4M3: return enc_launch_fmt<kFmtE4M3>(grid, P, s);
-    case kFmtNvfp4Amax: return enc_launch_fmt<kFmtNvfp4Amax>(grid, P, s);
-    case kFmtNvfp4: return enc_launch_fmt<kFmtNvfp4>(grid, P, s);
+    case kFmtE4M3: return enc_launch_fmt<kFmtE4M3>(grid, P, err, s);
+    case kFmtNvfp4Amax: return enc_launch_fmt<kFmtNvfp4Amax>(grid, P, err, s);
+    case kFmtNvfp4: return enc_launch_fmt<kFmtNvfp4>(grid, P, err, s);
     default: return cudaErrorInvalidValue;
   }
 }
 
-cudaError_t dec_launch(int fmt, int grid, const DecParams& P, cudaStream_t s) {
+cudaError_t dec_launch(int fmt, int grid, const DecParams& P, uint32_t* err, cudaStream_t s) {
   switch (fmt) {
-    case kFmtE4M3: return dec_launch_fmt<kFmtE4M3>(grid, P, s);
-    case kFmtNvfp4: return dec_launch_fmt<kFmtNvfp4>(grid, P, s);
+    case kFmtE4M3: return dec_launch_fmt<kFmtE4M3>(grid, P, err, s);
+    case kFmtNvfp4: return dec_launch_fmt<kFmtNvfp4>(grid, P, err, s);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -1381,7 +1457,8 @@ int tc_codec_split(const TcLayer* layers, int n, bool encode) {
   return grid <= 0 ? -1 : S;
 }
 
-cudaError_t launch_whiten_encode_tc(const TcLayer* layers, int n, cudaStream_t s) {
+cudaError_t launch_whiten_encode_tc(const TcLayer* layers, int n, uint32_t* err, cudaStream_t s,
+                                    uint32_t stall_polls) {
   cudaError_t e = cudaSuccess;
   for (int base = 0; base < n;) {
     // pack as many layers as fit one launch
@@ -1401,7 +1478,7 @@ cudaError_t launch_whiten_encode_tc(const TcLayer* layers, int n, cudaStream_t s
           part.codes = L.codes + (int64_t)r0 * (L.d_in / 2);
           part.block_scales = L.block_scales + (int64_t)r0 * (L.d_in / 16);
         }
-        if ((e = launch_whiten_encode_tc(&part, 1, s)) != cudaSuccess) return e;
+        if ((e = launch_whiten_encode_tc(&part, 1, err, s, stall_polls)) != cudaSuccess) return e;
       }
       ++base;
       continue;
@@ -1432,7 +1509,8 @@ cudaError_t launch_whiten_encode_tc(const TcLayer* layers, int n, cudaStream_t s
     const int grid = plan(layers + base, cnt, P.sched_off, P.sched_ids, kMaxPanels,
                           [fmt](int S) { return enc_slots(fmt, S); }, &P.split);
     if (grid <= 0) return cudaErrorInvalidValue;
-    if ((e = enc_launch(fmt, grid, P, s)) != cudaSuccess) return e;
+    P.stall_polls = stall_polls;
+    if ((e = enc_launch(fmt, grid, P, err, s)) != cudaSuccess) return e;
     base += cnt;
   }
   return cudaSuccess;
@@ -1440,7 +1518,8 @@ cudaError_t launch_whiten_encode_tc(const TcLayer* layers, int n, cudaStream_t s
 
 
 
-cudaError_t launch_whiten_decode_tc(const TcLayer* layers, int n, cudaStream_t s) {
+cudaError_t launch_whiten_decode_tc(const TcLayer* layers, int n, uint32_t* err, cudaStream_t s,
+                                    uint32_t stall_polls) {
   cudaError_t e = cudaSuccess;
   for (int base = 0; base < n;) {
     const int cnt = group_count(layers + base, n - base);
@@ -1458,7 +1537,7 @@ cudaError_t launch_whiten_decode_tc(const TcLayer* layers, int n, cudaStream_t s
           part.codes = L.codes + (int64_t)r0 * (L.d_in / 2);
           part.block_scales = L.block_scales + (int64_t)r0 * (L.d_in / 16);
         }
-        if ((e = launch_whiten_decode_tc(&part, 1, s)) != cudaSuccess) return e;
+        if ((e = launch_whiten_decode_tc(&part, 1, err, s, stall_polls)) != cudaSuccess) return e;
       }
       ++base;
       continue;
@@ -1489,7 +1568,8 @@ cudaError_t launch_whiten_decode_tc(const TcLayer* layers, int n, cudaStream_t s
     const int grid = plan(layers + base, cnt, P.sched_off, P.sched_ids, kMaxPanels,
                           [fmt](int S) { return dec_slots(fmt, S); }, &P.split);
     if (grid <= 0) return cudaErrorInvalidValue;
-    if ((e = dec_launch(fmt, grid, P, s)) != cudaSuccess) return e;
+    P.stall_polls = stall_polls;
+    if ((e = dec_launch(fmt, grid, P, err, s)) != cudaSuccess) return e;
     base += cnt;
   }
   return cudaSuccess;

@@ -146,6 +146,25 @@ GIFT_DEV float e4m3_inv_scale(float amax) {
 GIFT_DEV float e4m3_scale(float amax, float inv) { return inv > 0.0f ? __fdiv_rn(amax, kE4M3Max) : 0.0f; }
 
 // ---------------------------------------------------------------------------
+// Non-finite inputs.  Block maxima are taken with max.NaN, which returns NaN
+// when either operand is NaN (fmaxf would drop it), so a block holding a NaN
+// or an infinity has a non-finite maximum; such a block is coded as a
+// flushed block (scale 0, codes 0x00) and GIFT_DEV_NONFINITE is reported.
+// ---------------------------------------------------------------------------
+GIFT_DEV float fmax_nan(float a, float b) {
+  float r;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
+}
+GIFT_DEV bool not_finite(float x) { return !(fabsf(x) <= 3.402823466e38f); }
+
+// OR `bits` into *err once per warp for the lanes whose `bad` is set (every
+// lane of the warp must call it).
+GIFT_DEV void report_bits(uint32_t* err, bool bad, uint32_t bits) {
+  if (__any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0 && err) atomicOr(err, bits);
+}
+
+// ---------------------------------------------------------------------------
 // Warp reductions
 // ---------------------------------------------------------------------------
 GIFT_DEV float warp_max(float v) {

@@ -11,10 +11,11 @@
 namespace gift {
 
 // ---- Euclidean per-block E4M3 codec (rank 0): flat arrays of n_blocks*128 ----
+// `err` (nullable, device): the caller's status word; kernels OR GIFT_DEV_* bits into it.
 cudaError_t launch_euclid_encode(const void* G, gift_dtype dt, int64_t n_blocks, uint8_t* codes,
-                                 float* scales, cudaStream_t s);
+                                 float* scales, uint32_t* err, cudaStream_t s);
 cudaError_t launch_euclid_decode(const uint8_t* codes, const float* scales, int64_t n_blocks, void* G_hat,
-                                 gift_dtype dt, cudaStream_t s);
+                                 gift_dtype dt, uint32_t* err, cudaStream_t s);
 
 // Grouped Euclidean codec: one launch for many rank-0 layers of one dtype.
 struct EuclidLayer {
@@ -23,15 +24,16 @@ struct EuclidLayer {
   float* scales;
   int64_t n_blocks;  // d_out * d_in / 128
 };
-cudaError_t launch_euclid_group(const EuclidLayer* layers, int n, gift_dtype dt, bool encode, cudaStream_t s);
+cudaError_t launch_euclid_group(const EuclidLayer* layers, int n, gift_dtype dt, bool encode, uint32_t* err,
+                               cudaStream_t s);
 
 // ---- Whitened codec on CUDA cores (any rank <= 32, fp32 or bf16) ----
 cudaError_t launch_whiten_encode_simt(const void* G, gift_dtype dt, int64_t d_out, int64_t d_in, const float* U,
                                       const float* lambda, const float* rho, int rank, uint8_t* codes,
-                                      float* scales, cudaStream_t s);
+                                      float* scales, uint32_t* err, cudaStream_t s);
 cudaError_t launch_whiten_decode_simt(const uint8_t* codes, const float* scales, int64_t d_out, int64_t d_in,
                                       const float* U, const float* lambda, const float* rho, int rank,
-                                      void* G_hat, gift_dtype dt, cudaStream_t s);
+                                      void* G_hat, gift_dtype dt, uint32_t* err, cudaStream_t s);
 
 // ---- Whitened codec on the tensor cores (bf16 G, tcgen05 + TMA) ----
 struct TcLayer {
@@ -55,8 +57,13 @@ struct TcLayer {
 };
 constexpr int kFmtE4M3 = 0, kFmtNvfp4Amax = 1, kFmtNvfp4 = 2;
 bool tc_codec_available();
-cudaError_t launch_whiten_encode_tc(const TcLayer* layers, int n, cudaStream_t s);
-cudaError_t launch_whiten_decode_tc(const TcLayer* layers, int n, cudaStream_t s);
+// stall_polls > 0 is a test hook: before any work, one thread of every CTA
+// waits at most that many polls on a barrier nothing arrives at, gives up,
+// and the CTA skips its work and reports GIFT_DEV_TIMEOUT.
+cudaError_t launch_whiten_encode_tc(const TcLayer* layers, int n, uint32_t* err, cudaStream_t s,
+                                    uint32_t stall_polls = 0);
+cudaError_t launch_whiten_decode_tc(const TcLayer* layers, int n, uint32_t* err, cudaStream_t s,
+                                    uint32_t stall_polls = 0);
 // Cluster size (1, 2 or 4) the tensor-core codec plans for the first launch
 // over these layers (-1 if they cannot be planned).  Host-side; queries the
 // device's cluster occupancy once per kernel.
@@ -68,9 +75,9 @@ size_t error_ws_bytes(int64_t n_elems);
 cudaError_t launch_nvfp4_amax(const void* G, gift_dtype dt, int64_t n_blocks, float* tensor_scale, cudaStream_t s);
 cudaError_t launch_nvfp4_quant(const void* G, gift_dtype dt, int64_t n_blocks, const float* tensor_scale,
                                uint8_t* codes, uint8_t* sb, cudaStream_t s);
-cudaError_t launch_nvfp4_finalize(float* tensor_scale, cudaStream_t s);
+cudaError_t launch_nvfp4_finalize(float* tensor_scale, uint32_t* err, cudaStream_t s);
 cudaError_t launch_nvfp4_decode(const uint8_t* codes, const uint8_t* sb, const float* tensor_scale, int64_t n_blocks,
-                                void* out, gift_dtype dt, cudaStream_t s);
+                                void* out, gift_dtype dt, uint32_t* err, cudaStream_t s);
 
 cudaError_t launch_roundtrip_error(const void* G, const void* G_hat, gift_dtype dt, int64_t n_elems,
                                    double* out, void* ws, cudaStream_t s);

@@ -60,10 +60,12 @@ __global__ void __launch_bounds__(kThreads) nvfp4_amax_kernel(const T* __restric
     float v[16];
     load16(G + b * 16, v);
 #pragma unroll
-    for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[i]));
+    for (int i = 0; i < 16; ++i) m = fmax_nan(m, fabsf(v[i]));
   }
-  m = warp_max(m);
-  if ((threadIdx.x & 31) == 0 && m > 0.0f) atomicMax(amax_bits, __float_as_uint(m));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmax_nan(m, __shfl_xor_sync(0xffffffffu, m, o));
+  // a NaN maximum has the largest bit pattern of all, so it survives the max
+  if ((threadIdx.x & 31) == 0 && (m > 0.0f || m != m)) atomicMax(amax_bits, __float_as_uint(m));
 }
 
 template <typename T>
@@ -81,18 +83,20 @@ __global__ void __launch_bounds__(kThreads) nvfp4_quant_kernel(const T* __restri
   }
 }
 
-// amax bits -> S_t, in place (one thread)
-__global__ void nvfp4_finalize_kernel(float* tensor_scale) {
+// amax bits -> S_t, in place (one thread); a non-finite amax(W) is reported
+__global__ void nvfp4_finalize_kernel(float* tensor_scale, uint32_t* err) {
   const float amax = __uint_as_float(*reinterpret_cast<const uint32_t*>(tensor_scale));
   *tensor_scale = nvfp4_tensor_scale(amax);
+  if (err && not_finite(amax)) atomicOr(err, GIFT_DEV_NONFINITE);
 }
 
 template <typename T>
 __global__ void __launch_bounds__(kThreads) nvfp4_decode_kernel(const uint2* __restrict__ codes,
                                                                 const uint8_t* __restrict__ sb,
                                                                 const float* __restrict__ tensor_scale,
-                                                                int64_t n_blocks, T* __restrict__ out) {
+                                                                int64_t n_blocks, T* __restrict__ out, uint32_t* err) {
   const float S_t = __ldg(tensor_scale);
+  if (blockIdx.x == 0 && threadIdx.x == 0 && err && not_finite(S_t)) atomicOr(err, GIFT_DEV_NONFINITE);
   for (int64_t b = (int64_t)blockIdx.x * kThreads + threadIdx.x; b < n_blocks; b += (int64_t)gridDim.x * kThreads) {
     float v[16];
     nvfp4_block16_values(__ldcs(codes + b), sb[b], v);
@@ -131,18 +135,19 @@ cudaError_t launch_nvfp4_quant(const void* G, gift_dtype dt, int64_t n_blocks, c
   return cudaGetLastError();
 }
 
-cudaError_t launch_nvfp4_finalize(float* tensor_scale, cudaStream_t s) {
-  nvfp4_finalize_kernel<<<1, 1, 0, s>>>(tensor_scale);
+cudaError_t launch_nvfp4_finalize(float* tensor_scale, uint32_t* err, cudaStream_t s) {
+  nvfp4_finalize_kernel<<<1, 1, 0, s>>>(tensor_scale, err);
   return cudaGetLastError();
 }
 
 cudaError_t launch_nvfp4_decode(const uint8_t* codes, const uint8_t* sb, const float* tensor_scale, int64_t n_blocks,
-                                void* out, gift_dtype dt, cudaStream_t s) {
+                                void* out, gift_dtype dt, uint32_t* err, cudaStream_t s) {
   const int g = grid_for(n_blocks);
   if (dt == GIFT_BF16)
-    nvfp4_decode_kernel<<<g, kThreads, 0, s>>>((const uint2*)codes, sb, tensor_scale, n_blocks, (__nv_bfloat16*)out);
+    nvfp4_decode_kernel<<<g, kThreads, 0, s>>>((const uint2*)codes, sb, tensor_scale, n_blocks, (__nv_bfloat16*)out,
+                                               err);
   else
-    nvfp4_decode_kernel<<<g, kThreads, 0, s>>>((const uint2*)codes, sb, tensor_scale, n_blocks, (float*)out);
+    nvfp4_decode_kernel<<<g, kThreads, 0, s>>>((const uint2*)codes, sb, tensor_scale, n_blocks, (float*)out, err);
   return cudaGetLastError();
 }
 

@@ -20,14 +20,15 @@ LIB_PATH = os.path.join(_HERE, "libgift.so")
 
 GIFT_F32, GIFT_BF16 = 0, 1
 E4M3_BLOCK = 128
-DEV_RHO_FLOORED, DEV_RANK_DEFICIENT, DEV_NONFINITE = 0x1, 0x2, 0x4
+DEV_RHO_FLOORED, DEV_RANK_DEFICIENT, DEV_NONFINITE, DEV_TIMEOUT = 0x1, 0x2, 0x4, 0x8
 STATUS = {0: "GIFT_OK", 1: "GIFT_ERR_INVALID_ARG", 2: "GIFT_ERR_SHAPE", 3: "GIFT_ERR_ALIGN",
           4: "GIFT_ERR_WORKSPACE", 5: "GIFT_ERR_CUDA", 6: "GIFT_ERR_UNSUPPORTED"}
 
 EXPORTED = ("gift_status_string", "gift_version", "gift_refresh_workspace_size", "gift_factor_refresh",
             "gift_factor_refresh_noalloc", "gift_factor_refresh_many", "gift_encode", "gift_decode", "gift_encode_many", "gift_decode_many",
             "gift_error_workspace_size", "gift_roundtrip_error", "gift_encode_nvfp4", "gift_decode_nvfp4",
-            "gift_codec_split", "gift_whitened_error_workspace_size", "gift_whitened_error")
+            "gift_codec_split", "gift_whitened_error_workspace_size", "gift_whitened_error",
+            "gift_codec_stall_test")
 
 
 class GiftError(RuntimeError):
@@ -74,17 +75,18 @@ def lib() -> ctypes.CDLL:
         L.gift_factor_refresh_noalloc.argtypes = [vp, i32, i64, i64, i32, i32, i32, ctypes.c_uint64, vp, vp, vp,
                                                   vp, vp, vp]
         L.gift_factor_refresh_many.argtypes = [ctypes.POINTER(RefreshJob), i32, i32, i32, i32, vp]
-        L.gift_encode.argtypes = [vp, i32, i64, i64, vp, vp, vp, i32, vp, vp, vp]
-        L.gift_decode.argtypes = [vp, vp, i64, i64, vp, vp, vp, i32, vp, i32, vp]
-        L.gift_encode_many.argtypes = [ctypes.POINTER(Layer), i32, vp]
-        L.gift_decode_many.argtypes = [ctypes.POINTER(Layer), i32, vp]
+        L.gift_encode.argtypes = [vp, i32, i64, i64, vp, vp, vp, i32, vp, vp, vp, vp]
+        L.gift_decode.argtypes = [vp, vp, i64, i64, vp, vp, vp, i32, vp, i32, vp, vp]
+        L.gift_encode_many.argtypes = [ctypes.POINTER(Layer), i32, vp, vp]
+        L.gift_decode_many.argtypes = [ctypes.POINTER(Layer), i32, vp, vp]
+        L.gift_codec_stall_test.argtypes = [ctypes.POINTER(Layer), i32, ctypes.c_uint32, vp, vp]
         L.gift_codec_split.argtypes = [ctypes.POINTER(Layer), i32, i32, ctypes.POINTER(i32)]
         L.gift_error_workspace_size.argtypes = [i64, i64, ctypes.POINTER(sz)]
         L.gift_roundtrip_error.argtypes = [vp, vp, i32, i64, i64, vp, vp, sz, vp]
         L.gift_whitened_error_workspace_size.argtypes = [i64, i64, ctypes.POINTER(sz)]
         L.gift_whitened_error.argtypes = [vp, vp, i32, i64, i64, vp, vp, vp, i32, vp, vp, sz, vp]
-        L.gift_encode_nvfp4.argtypes = [vp, i32, i64, i64, vp, vp, vp, i32, vp, vp, vp, vp]
-        L.gift_decode_nvfp4.argtypes = [vp, vp, vp, i64, i64, vp, vp, vp, i32, vp, i32, vp]
+        L.gift_encode_nvfp4.argtypes = [vp, i32, i64, i64, vp, vp, vp, i32, vp, vp, vp, vp, vp]
+        L.gift_decode_nvfp4.argtypes = [vp, vp, vp, i64, i64, vp, vp, vp, i32, vp, i32, vp, vp]
         for name in EXPORTED:
             if name not in ("gift_status_string", "gift_version"):
                 getattr(L, name).restype = i32
@@ -202,9 +204,11 @@ def factor_refresh_many(jobs, n: int, rank: int = 32, oversample: int = 16, iter
 
 
 def encode(G: torch.Tensor, U=None, lam=None, rho=None, rank: Optional[int] = None,
-           codes: Optional[torch.Tensor] = None, scales: Optional[torch.Tensor] = None, stream=None):
-    """(codes uint8 [d_out, d_in], scales fp32 [d_out, d_in/128]); rank 0 / U None = Euclidean."""
-    _cuda(G, U, lam, rho, codes, scales)
+           codes: Optional[torch.Tensor] = None, scales: Optional[torch.Tensor] = None, stream=None,
+           dev_status: Optional[torch.Tensor] = None):
+    """(codes uint8 [d_out, d_in], scales fp32 [d_out, d_in/128]); rank 0 / U None = Euclidean.
+    dev_status: optional int32 device word the call ORs GIFT_DEV_* bits into."""
+    _cuda(G, U, lam, rho, codes, scales, dev_status)
     d_out, d_in = G.shape
     if rank is None:
         rank = 0 if U is None else U.shape[1]
@@ -213,21 +217,22 @@ def encode(G: torch.Tensor, U=None, lam=None, rho=None, rank: Optional[int] = No
     if scales is None:
         scales = torch.empty((d_out, max(d_in // E4M3_BLOCK, 1)), device=G.device, dtype=torch.float32)
     _check(lib().gift_encode(_ptr(G), _dt(G), d_out, d_in, _ptr(U), _ptr(lam), _ptr(rho), rank,
-                             _ptr(codes), _ptr(scales), _stream(stream)), "gift_encode")
+                             _ptr(codes), _ptr(scales), _ptr(dev_status), _stream(stream)), "gift_encode")
     return codes, scales
 
 
 def decode(codes: torch.Tensor, scales: torch.Tensor, U=None, lam=None, rho=None, rank: Optional[int] = None,
-           out_dtype=torch.bfloat16, out: Optional[torch.Tensor] = None, stream=None):
+           out_dtype=torch.bfloat16, out: Optional[torch.Tensor] = None, stream=None,
+           dev_status: Optional[torch.Tensor] = None):
     """G_hat [d_out, d_in] in out_dtype (bf16 or fp32)."""
-    _cuda(codes, scales, U, lam, rho, out)
+    _cuda(codes, scales, U, lam, rho, out, dev_status)
     d_out, d_in = codes.shape
     if rank is None:
         rank = 0 if U is None else U.shape[1]
     if out is None:
         out = torch.empty((d_out, d_in), device=codes.device, dtype=out_dtype)
     _check(lib().gift_decode(_ptr(codes), _ptr(scales), d_out, d_in, _ptr(U), _ptr(lam), _ptr(rho), rank,
-                             _ptr(out), _dt(out), _stream(stream)), "gift_decode")
+                             _ptr(out), _dt(out), _ptr(dev_status), _stream(stream)), "gift_decode")
     return out
 
 
@@ -236,9 +241,10 @@ NVFP4_BLOCK = 16
 
 def encode_nvfp4(G: torch.Tensor, U=None, lam=None, rho=None, rank: Optional[int] = None,
                  codes: Optional[torch.Tensor] = None, block_scales: Optional[torch.Tensor] = None,
-                 tensor_scale: Optional[torch.Tensor] = None, stream=None):
+                 tensor_scale: Optional[torch.Tensor] = None, stream=None,
+                 dev_status: Optional[torch.Tensor] = None):
     """(codes uint8 [d_out, d_in/2], block scales uint8 [d_out, d_in/16], tensor scale fp32 [1])."""
-    _cuda(G, U, lam, rho, codes, block_scales, tensor_scale)
+    _cuda(G, U, lam, rho, codes, block_scales, tensor_scale, dev_status)
     d_out, d_in = G.shape
     if rank is None:
         rank = 0 if U is None else U.shape[1]
@@ -249,23 +255,25 @@ def encode_nvfp4(G: torch.Tensor, U=None, lam=None, rho=None, rank: Optional[int
     if tensor_scale is None:
         tensor_scale = torch.empty((1,), device=G.device, dtype=torch.float32)
     _check(lib().gift_encode_nvfp4(_ptr(G), _dt(G), d_out, d_in, _ptr(U), _ptr(lam), _ptr(rho), rank,
-                                   _ptr(codes), _ptr(block_scales), _ptr(tensor_scale), _stream(stream)),
+                                   _ptr(codes), _ptr(block_scales), _ptr(tensor_scale), _ptr(dev_status),
+                                   _stream(stream)),
            "gift_encode_nvfp4")
     return codes, block_scales, tensor_scale
 
 
 def decode_nvfp4(codes: torch.Tensor, block_scales: torch.Tensor, tensor_scale: torch.Tensor, U=None, lam=None,
                  rho=None, rank: Optional[int] = None, out_dtype=torch.bfloat16, out: Optional[torch.Tensor] = None,
-                 stream=None):
+                 stream=None, dev_status: Optional[torch.Tensor] = None):
     """G_hat [d_out, d_in] in out_dtype from NVFP4 codes."""
-    _cuda(codes, block_scales, tensor_scale, U, lam, rho, out)
+    _cuda(codes, block_scales, tensor_scale, U, lam, rho, out, dev_status)
     d_out, d_in = codes.shape[0], codes.shape[1] * 2
     if rank is None:
         rank = 0 if U is None else U.shape[1]
     if out is None:
         out = torch.empty((d_out, d_in), device=codes.device, dtype=out_dtype)
     _check(lib().gift_decode_nvfp4(_ptr(codes), _ptr(block_scales), _ptr(tensor_scale), d_out, d_in, _ptr(U),
-                                   _ptr(lam), _ptr(rho), rank, _ptr(out), _dt(out), _stream(stream)),
+                                   _ptr(lam), _ptr(rho), rank, _ptr(out), _dt(out), _ptr(dev_status),
+                                   _stream(stream)),
            "gift_decode_nvfp4")
     return out
 
@@ -305,12 +313,24 @@ def make_layers(layers: Sequence[LayerArgs]):
     return arr
 
 
-def encode_many(packed, n: int, stream=None):
-    _check(lib().gift_encode_many(packed, n, _stream(stream)), "gift_encode_many")
+def encode_many(packed, n: int, stream=None, dev_status: Optional[torch.Tensor] = None):
+    _cuda(dev_status)
+    _check(lib().gift_encode_many(packed, n, _ptr(dev_status), _stream(stream)), "gift_encode_many")
 
 
-def decode_many(packed, n: int, stream=None):
-    _check(lib().gift_decode_many(packed, n, _stream(stream)), "gift_decode_many")
+def decode_many(packed, n: int, stream=None, dev_status: Optional[torch.Tensor] = None):
+    _cuda(dev_status)
+    _check(lib().gift_decode_many(packed, n, _ptr(dev_status), _stream(stream)), "gift_decode_many")
+
+
+def codec_stall_test(layer: LayerArgs, encode: bool, stall_polls: int, dev_status: torch.Tensor, stream=None):
+    """Test hook (gift_codec_stall_test): the tensor-core codec kernel on this
+    layer gives up a bounded wait on a barrier nothing arrives at before any
+    work, skips the layer and ORs GIFT_DEV_TIMEOUT into dev_status."""
+    _cuda(dev_status)
+    arr = make_layers([layer])
+    _check(lib().gift_codec_stall_test(arr, 1 if encode else 0, stall_polls, _ptr(dev_status), _stream(stream)),
+           "gift_codec_stall_test")
 
 
 def codec_split(packed, n: int, encode: bool = True) -> int:

@@ -62,11 +62,19 @@ typedef enum {
 
 typedef enum { GIFT_F32 = 0, GIFT_BF16 = 1 } gift_dtype;
 
-/* Bits OR-ed into *dev_status by the factor refresh. */
+/* Bits OR-ed into the caller's *dev_status word (device memory, 4-byte
+ * aligned; the caller zeroes it, calls only OR bits in).
+ *   refresh: RHO_FLOORED, RANK_DEFICIENT, NONFINITE (A, lambda or rho),
+ *            TIMEOUT (tensor-core syrk);
+ *   encode:  NONFINITE (a block maximum of W, or the NVFP4 tensor maximum,
+ *            is NaN or infinite: that block is coded as flushed, scale 0 and
+ *            codes 0), TIMEOUT (tensor-core whitened encoder);
+ *   decode:  NONFINITE (a block scale, or the NVFP4 tensor scale, is NaN or
+ *            infinite), TIMEOUT (tensor-core whitened decoder). */
 #define GIFT_DEV_RHO_FLOORED 0x1u    /* rho <= 2^-24 lambda_1: floored to that value */
 #define GIFT_DEV_RANK_DEFICIENT 0x2u /* a Cholesky-QR pivot vanished: the sampled
                                         subspace has lower rank; that column is zeroed */
-#define GIFT_DEV_NONFINITE 0x4u      /* a non-finite value reached A, lambda or rho */
+#define GIFT_DEV_NONFINITE 0x4u      /* a non-finite value reached the call's arithmetic */
 #define GIFT_DEV_TIMEOUT 0x8u        /* a pipeline wait inside a kernel gave up after its
                                         iteration bound; the outputs of that call are undefined */
 
@@ -173,20 +181,22 @@ gift_status gift_factor_refresh_noalloc(const void* X, gift_dtype xdt, int64_t N
  * G: d_out x d_in (GIFT_BF16 or GIFT_F32).  codes: d_out x d_in bytes.
  * scales: d_out x (d_in/128) fp32.  U/lambda/rho as produced by the refresh
  * (rho > 0 and finite); 0 <= rank <= 32.  d_in % 128 == 0, d_out >= 1.
+ * dev_status (nullable): GIFT_DEV_NONFINITE, GIFT_DEV_TIMEOUT.
  * ------------------------------------------------------------------------ */
 gift_status gift_encode(const void* G, gift_dtype gdt, int64_t d_out, int64_t d_in, const float* U,
                         const float* lambda, const float* rho, int rank, uint8_t* codes,
-                        float* scales, gift_stream_t stream);
+                        float* scales, uint32_t* dev_status, gift_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * Decode ("applies the inverse transform afterward").
  *
  *   W_hat = E4M3_value(codes) * scales (per block);  G_hat = W_hat M^{-1},
  *   written as out_dt (bf16 by round-to-nearest-even, or fp32).
+ * dev_status (nullable): GIFT_DEV_NONFINITE, GIFT_DEV_TIMEOUT.
  * ------------------------------------------------------------------------ */
 gift_status gift_decode(const uint8_t* codes, const float* scales, int64_t d_out, int64_t d_in,
                         const float* U, const float* lambda, const float* rho, int rank,
-                        void* G_hat, gift_dtype out_dt, gift_stream_t stream);
+                        void* G_hat, gift_dtype out_dt, uint32_t* dev_status, gift_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * Grouped encode / decode over many layers in as few launches as possible
@@ -209,8 +219,28 @@ typedef struct {
   int32_t dtype;       /* gift_dtype of G and G_hat */
 } gift_layer;
 
-gift_status gift_encode_many(const gift_layer* layers /* host */, int n, gift_stream_t stream);
-gift_status gift_decode_many(const gift_layer* layers /* host */, int n, gift_stream_t stream);
+/* dev_status (nullable): one word for the whole call, bits as for gift_encode
+ * / gift_decode; a TIMEOUT leaves the outputs of every layer undefined. */
+gift_status gift_encode_many(const gift_layer* layers /* host */, int n, uint32_t* dev_status,
+                             gift_stream_t stream);
+gift_status gift_decode_many(const gift_layer* layers /* host */, int n, uint32_t* dev_status,
+                             gift_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Test hook of the codec's failure path (the pages have no counterpart).
+ * Launches the tensor-core whitened encoder (encode != 0) or decoder on one
+ * layer (bf16, rank 32, d_in <= 8192) with one extra wait before any work:
+ * one thread of every CTA waits at most stall_polls polls on a barrier that
+ * nothing arrives at, the wait runs out, every CTA skips the layer's work
+ * and returns, and GIFT_DEV_TIMEOUT is OR-ed into *dev_status.  Nothing is
+ * loaded, computed or written and the context stays usable, so a test can
+ * check that a bounded wait that gives up is reported to the caller.
+ * Errors: GIFT_ERR_INVALID_ARG (null layer or dev_status, stall_polls == 0,
+ * empty layer, rank 0), the argument checks of gift_encode / gift_decode,
+ * GIFT_ERR_UNSUPPORTED (the layer does not take the tensor-core path).
+ * ------------------------------------------------------------------------ */
+gift_status gift_codec_stall_test(const gift_layer* layer /* host */, int encode, uint32_t stall_polls,
+                                  uint32_t* dev_status, gift_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * Planning query (launches nothing, reads no pointer of `layers`): how the
@@ -291,15 +321,18 @@ gift_status gift_whitened_error(const void* G, const void* G_hat, gift_dtype dt,
  * GIFT_ERR_UNSUPPORTED.  G / G_hat and U 16-byte aligned.
  * Decode: G_hat = W_hat (rank 0) or W_hat M^{-1} with
  * W_hat = value(code) * value(block scale) * S_t.
+ * dev_status (nullable): GIFT_DEV_NONFINITE (amax(W) or S_t not finite),
+ * GIFT_DEV_TIMEOUT (tensor-core path).
  * ------------------------------------------------------------------------ */
 gift_status gift_encode_nvfp4(const void* G, gift_dtype gdt, int64_t d_out, int64_t d_in, const float* U,
                               const float* lambda, const float* rho, int rank, uint8_t* codes,
-                              uint8_t* block_scales, float* tensor_scale, gift_stream_t stream);
+                              uint8_t* block_scales, float* tensor_scale, uint32_t* dev_status,
+                              gift_stream_t stream);
 
 gift_status gift_decode_nvfp4(const uint8_t* codes, const uint8_t* block_scales, const float* tensor_scale,
                               int64_t d_out, int64_t d_in, const float* U, const float* lambda,
                               const float* rho, int rank, void* G_hat, gift_dtype out_dt,
-                              gift_stream_t stream);
+                              uint32_t* dev_status, gift_stream_t stream);
 
 #ifdef __cplusplus
 }

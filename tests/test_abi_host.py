@@ -52,29 +52,42 @@ def test_version_and_status_strings(L):
 def test_encode_rejects_bad_arguments(L):
     s = None
     # null pointers (an empty gradient, d_out == 0, may pass nulls)
-    assert L.gift_encode(None, 1, 4, 128, None, None, None, 0, A16, A16, s) == INVALID
-    assert L.gift_encode(None, 1, 0, 128, None, None, None, 0, None, None, s) == OK
+    assert L.gift_encode(None, 1, 4, 128, None, None, None, 0, A16, A16, None, s) == INVALID
+    assert L.gift_encode(None, 1, 0, 128, None, None, None, 0, None, None, None, s) == OK
     # bad dtype
-    assert L.gift_encode(A16, 7, 4, 128, None, None, None, 0, A16, A16, s) == INVALID
+    assert L.gift_encode(A16, 7, 4, 128, None, None, None, 0, A16, A16, None, s) == INVALID
     # d_in not a multiple of 128
-    assert L.gift_encode(A16, 1, 4, 100, None, None, None, 0, A16, A16, s) == SHAPE
+    assert L.gift_encode(A16, 1, 4, 100, None, None, None, 0, A16, A16, None, s) == SHAPE
     # rank above 32
-    assert L.gift_encode(A16, 1, 4, 128, A16, A16, A16, 33, A16, A16, s) == SHAPE
+    assert L.gift_encode(A16, 1, 4, 128, A16, A16, A16, 33, A16, A16, None, s) == SHAPE
     # whitened without factors
-    assert L.gift_encode(A16, 1, 4, 128, None, None, None, 32, A16, A16, s) == INVALID
+    assert L.gift_encode(A16, 1, 4, 128, None, None, None, 32, A16, A16, None, s) == INVALID
     # misaligned gradient / codes
-    assert L.gift_encode(A_ODD, 1, 4, 128, None, None, None, 0, A16, A16, s) == ALIGN
-    assert L.gift_encode(A16, 1, 4, 128, None, None, None, 0, A_ODD, A16, s) == ALIGN
+    assert L.gift_encode(A_ODD, 1, 4, 128, None, None, None, 0, A16, A16, None, s) == ALIGN
+    assert L.gift_encode(A16, 1, 4, 128, None, None, None, 0, A_ODD, A16, None, s) == ALIGN
     # negative sizes
-    assert L.gift_encode(A16, 1, -1, 128, None, None, None, 0, A16, A16, s) == INVALID
+    assert L.gift_encode(A16, 1, -1, 128, None, None, None, 0, A16, A16, None, s) == INVALID
+
+
+def test_codec_status_word_alignment_and_stall_hook_arguments(L):
+    s = None
+    assert L.gift_encode(A16, 1, 4, 128, None, None, None, 0, A16, A16, A16 + 2, s) == ALIGN
+    assert L.gift_decode(A16, A16, 4, 128, None, None, None, 0, A16, 1, A16 + 1, s) == ALIGN
+    import torch
+    arr = ops.make_layers([ops.LayerArgs(d_out=256, d_in=256, rank=32, dtype=torch.bfloat16)])
+    assert L.gift_encode_many(arr, 1, A16 + 2, None) == ALIGN
+    assert L.gift_codec_stall_test(None, 1, 100, A16, s) == INVALID
+    assert L.gift_codec_stall_test(arr, 1, 0, A16, s) == INVALID      # stall_polls must be positive
+    assert L.gift_codec_stall_test(arr, 1, 100, None, s) == INVALID   # the status word is required
+    assert L.gift_codec_stall_test(arr, 1, 100, A16, s) == INVALID    # layer without tensors
 
 
 def test_decode_rejects_bad_arguments(L):
     s = None
-    assert L.gift_decode(None, A16, 4, 128, None, None, None, 0, A16, 1, s) == INVALID
-    assert L.gift_decode(A16, A16, 4, 256 + 64, None, None, None, 0, A16, 1, s) == SHAPE
-    assert L.gift_decode(A16, A16, 4, 128, None, None, None, 0, A16, 3, s) == INVALID
-    assert L.gift_decode(A16, A16, 4, 128, None, None, None, 0, A_ODD, 1, s) == ALIGN
+    assert L.gift_decode(None, A16, 4, 128, None, None, None, 0, A16, 1, None, s) == INVALID
+    assert L.gift_decode(A16, A16, 4, 256 + 64, None, None, None, 0, A16, 1, None, s) == SHAPE
+    assert L.gift_decode(A16, A16, 4, 128, None, None, None, 0, A16, 3, None, s) == INVALID
+    assert L.gift_decode(A16, A16, 4, 128, None, None, None, 0, A_ODD, 1, None, s) == ALIGN
 
 
 def test_nvfp4_rejects_bad_arguments(L):
@@ -82,23 +95,23 @@ def test_nvfp4_rejects_bad_arguments(L):
     UNSUPPORTED = 6
     enc, dec = L.gift_encode_nvfp4, L.gift_decode_nvfp4
     # empty gradient: nothing is touched
-    assert enc(None, 1, 0, 128, None, None, None, 0, None, None, None, s) == OK
+    assert enc(None, 1, 0, 128, None, None, None, 0, None, None, None, None, s) == OK
     # null outputs
-    assert enc(A16, 1, 4, 128, None, None, None, 0, A16, A16, None, s) == INVALID
+    assert enc(A16, 1, 4, 128, None, None, None, 0, A16, A16, None, None, s) == INVALID
     # Euclidean blocks of 16: d_in % 16; whitened: d_in % 128
-    assert enc(A16, 1, 4, 24, None, None, None, 0, A16, A16, A16, s) == SHAPE
-    assert enc(A16, 1, 4, 144, A16, A16, A16, 32, A16, A16, A16, s) == SHAPE
+    assert enc(A16, 1, 4, 24, None, None, None, 0, A16, A16, A16, None, s) == SHAPE
+    assert enc(A16, 1, 4, 144, A16, A16, A16, 32, A16, A16, A16, None, s) == SHAPE
     # whitened NVFP4 runs on the tensor cores only: rank 32, bf16
-    assert enc(A16, 1, 4, 128, A16, A16, A16, 7, A16, A16, A16, s) == UNSUPPORTED
-    assert enc(A16, 0, 4, 128, A16, A16, A16, 32, A16, A16, A16, s) == UNSUPPORTED
-    assert enc(A16, 1, 4, 128, A16, A16, A16, 33, A16, A16, A16, s) == SHAPE
+    assert enc(A16, 1, 4, 128, A16, A16, A16, 7, A16, A16, A16, None, s) == UNSUPPORTED
+    assert enc(A16, 0, 4, 128, A16, A16, A16, 32, A16, A16, A16, None, s) == UNSUPPORTED
+    assert enc(A16, 1, 4, 128, A16, A16, A16, 33, A16, A16, A16, None, s) == SHAPE
     # alignment: codes 16 B, block scales 8 B, tensor scale 4 B
-    assert enc(A16, 1, 4, 128, None, None, None, 0, A_ODD, A16, A16, s) == ALIGN
-    assert enc(A16, 1, 4, 128, None, None, None, 0, A16, A16 + 4, A16, s) == ALIGN
-    assert enc(A16, 1, 4, 128, None, None, None, 0, A16, A16, A16 + 2, s) == ALIGN
-    assert dec(A16, A16, A16, 4, 128, None, None, None, 0, None, 1, s) == INVALID
-    assert dec(A16, A16, A16, 4, 128, None, None, None, 0, A16, 5, s) == INVALID
-    assert dec(A16, A16, A16, 4, 128, A16, A16, A16, 32, A16, 0, s) == UNSUPPORTED
+    assert enc(A16, 1, 4, 128, None, None, None, 0, A_ODD, A16, A16, None, s) == ALIGN
+    assert enc(A16, 1, 4, 128, None, None, None, 0, A16, A16 + 4, A16, None, s) == ALIGN
+    assert enc(A16, 1, 4, 128, None, None, None, 0, A16, A16, A16 + 2, None, s) == ALIGN
+    assert dec(A16, A16, A16, 4, 128, None, None, None, 0, None, 1, None, s) == INVALID
+    assert dec(A16, A16, A16, 4, 128, None, None, None, 0, A16, 5, None, s) == INVALID
+    assert dec(A16, A16, A16, 4, 128, A16, A16, A16, 32, A16, 0, None, s) == UNSUPPORTED
 
 
 def test_refresh_rejects_bad_arguments(L):
@@ -140,9 +153,9 @@ def test_many_rejects_a_bad_layer_before_launching(L):
     good = ops.Layer(A16, A16, A16, A16, None, None, None, 8, 256, 0, 1)
     bad = ops.Layer(A16, A16, A16, A16, None, None, None, 8, 200, 0, 1)
     arr = (ops.Layer * 2)(good, bad)
-    assert L.gift_encode_many(arr, 2, None) == SHAPE
-    assert L.gift_encode_many(None, 3, None) == INVALID
-    assert L.gift_encode_many(arr, 0, None) == OK
+    assert L.gift_encode_many(arr, 2, None, None) == SHAPE
+    assert L.gift_encode_many(None, 3, None, None) == INVALID
+    assert L.gift_encode_many(arr, 0, None, None) == OK
 
 
 def test_product_path_has_no_oracle_import():
