@@ -394,4 +394,79 @@ gift_status gift_decode_nvfp4(const uint8_t* codes, const uint8_t* block_scales,
   return cuda_status(launch_whiten_decode_tc(&L, 1, dev_status, s));
 }
 
+// ---------------------------------------------------------------------------
+static gift_status check_dense_d(int64_t d) {
+  if (d < GIFT_E4M3_BLOCK || d % GIFT_E4M3_BLOCK != 0 || d > 8192) return GIFT_ERR_SHAPE;
+  return GIFT_OK;
+}
+
+gift_status gift_dense_factor_workspace_size(int64_t d, int kind, size_t* bytes) {
+  if (!bytes || (kind != GIFT_DENSE_CHOLESKY && kind != GIFT_DENSE_INVSQRT)) return GIFT_ERR_INVALID_ARG;
+  gift_status st = check_dense_d(d);
+  if (st != GIFT_OK) return st;
+  *bytes = dense_factor_ws_bytes(d, kind);
+  return GIFT_OK;
+}
+
+gift_status gift_dense_factor(const float* A, int64_t d, int kind, float* M, float* M_inv, uint16_t* M_split,
+                              uint16_t* M_inv_split, void* ws, size_t ws_bytes, uint32_t* dev_status,
+                              gift_stream_t stream) {
+  if (!A || !M || !M_inv || !M_split || !M_inv_split) return GIFT_ERR_INVALID_ARG;
+  size_t need = 0;
+  gift_status st = gift_dense_factor_workspace_size(d, kind, &need);
+  if (st != GIFT_OK) return st;
+  if (!ws || ws_bytes < need) return GIFT_ERR_WORKSPACE;
+  if (!aligned16(A) || !aligned16(M) || !aligned16(M_inv) || !aligned16(M_split) || !aligned16(M_inv_split) ||
+      !aligned16(ws) || (dev_status && !aligned(dev_status, 4)))
+    return GIFT_ERR_ALIGN;
+  if ((st = device_ok()) != GIFT_OK) return st;
+  return cuda_status(launch_dense_factor(A, (int)d, kind, M, M_inv, M_split, M_inv_split, ws, dev_status,
+                                         (cudaStream_t)stream));
+}
+
+gift_status gift_dense_split(const float* M, int64_t d, uint16_t* M_split, gift_stream_t stream) {
+  if (!M || !M_split) return GIFT_ERR_INVALID_ARG;
+  gift_status st = check_dense_d(d);
+  if (st != GIFT_OK) return st;
+  if (!aligned16(M) || !aligned16(M_split)) return GIFT_ERR_ALIGN;
+  if ((st = device_ok()) != GIFT_OK) return st;
+  return cuda_status(launch_dense_split(M, (int)d, M_split, (cudaStream_t)stream));
+}
+
+gift_status gift_dense_encode(const void* G, int64_t d_out, int64_t d_in, const uint16_t* M_split,
+                              int upper_triangular, uint8_t* codes, float* scales, uint32_t* dev_status,
+                              gift_stream_t stream) {
+  if (d_out < 0) return GIFT_ERR_INVALID_ARG;
+  gift_status st = check_dense_d(d_in);
+  if (st != GIFT_OK) return st;
+  if (d_out > ((int64_t)1 << 24)) return GIFT_ERR_SHAPE;
+  if (d_out == 0) return GIFT_OK;
+  if (!G || !M_split || !codes || !scales) return GIFT_ERR_INVALID_ARG;
+  if (!aligned16(G) || !aligned16(M_split) || !aligned16(codes) || !aligned16(scales) ||
+      (dev_status && !aligned(dev_status, 4)))
+    return GIFT_ERR_ALIGN;
+  if ((st = device_ok()) != GIFT_OK) return st;
+  if (!tc_codec_available()) return GIFT_ERR_UNSUPPORTED;
+  return cuda_status(launch_dense_encode(G, (int)d_out, (int)d_in, M_split, upper_triangular != 0, codes, scales,
+                                         dev_status, (cudaStream_t)stream));
+}
+
+gift_status gift_dense_decode(const uint8_t* codes, const float* scales, int64_t d_out, int64_t d_in,
+                              const uint16_t* M_inv_split, int upper_triangular, void* G_hat, gift_dtype out_dt,
+                              uint32_t* dev_status, gift_stream_t stream) {
+  if (d_out < 0 || !dtype_ok(out_dt)) return GIFT_ERR_INVALID_ARG;
+  gift_status st = check_dense_d(d_in);
+  if (st != GIFT_OK) return st;
+  if (d_out > ((int64_t)1 << 24)) return GIFT_ERR_SHAPE;
+  if (d_out == 0) return GIFT_OK;
+  if (!codes || !scales || !M_inv_split || !G_hat) return GIFT_ERR_INVALID_ARG;
+  if (!aligned16(codes) || !aligned16(scales) || !aligned16(M_inv_split) || !aligned16(G_hat) ||
+      (dev_status && !aligned(dev_status, 4)))
+    return GIFT_ERR_ALIGN;
+  if ((st = device_ok()) != GIFT_OK) return st;
+  if (!tc_codec_available()) return GIFT_ERR_UNSUPPORTED;
+  return cuda_status(launch_dense_decode(codes, scales, (int)d_out, (int)d_in, M_inv_split, upper_triangular != 0,
+                                         G_hat, out_dt, dev_status, (cudaStream_t)stream));
+}
+
 }  // extern "C"

@@ -28,7 +28,9 @@ EXPORTED = ("gift_status_string", "gift_version", "gift_refresh_workspace_size",
             "gift_factor_refresh_noalloc", "gift_factor_refresh_many", "gift_encode", "gift_decode", "gift_encode_many", "gift_decode_many",
             "gift_error_workspace_size", "gift_roundtrip_error", "gift_encode_nvfp4", "gift_decode_nvfp4",
             "gift_codec_split", "gift_whitened_error_workspace_size", "gift_whitened_error",
-            "gift_codec_stall_test")
+            "gift_codec_stall_test", "gift_dense_factor_workspace_size", "gift_dense_factor", "gift_dense_split",
+            "gift_dense_encode", "gift_dense_decode")
+DENSE_CHOLESKY, DENSE_INVSQRT = 1, 2
 
 
 class GiftError(RuntimeError):
@@ -87,6 +89,11 @@ def lib() -> ctypes.CDLL:
         L.gift_whitened_error.argtypes = [vp, vp, i32, i64, i64, vp, vp, vp, i32, vp, vp, sz, vp]
         L.gift_encode_nvfp4.argtypes = [vp, i32, i64, i64, vp, vp, vp, i32, vp, vp, vp, vp, vp]
         L.gift_decode_nvfp4.argtypes = [vp, vp, vp, i64, i64, vp, vp, vp, i32, vp, i32, vp, vp]
+        L.gift_dense_factor_workspace_size.argtypes = [i64, i32, ctypes.POINTER(sz)]
+        L.gift_dense_factor.argtypes = [vp, i64, i32, vp, vp, vp, vp, vp, sz, vp, vp]
+        L.gift_dense_split.argtypes = [vp, i64, vp, vp]
+        L.gift_dense_encode.argtypes = [vp, i64, i64, vp, i32, vp, vp, vp, vp]
+        L.gift_dense_decode.argtypes = [vp, vp, i64, i64, vp, i32, vp, i32, vp, vp]
         for name in EXPORTED:
             if name not in ("gift_status_string", "gift_version"):
                 getattr(L, name).restype = i32
@@ -385,4 +392,70 @@ def whitened_error(G: torch.Tensor, G_hat: torch.Tensor, U=None, lam=None, rho=N
         ws = torch.empty((whitened_error_workspace_size(d_out, d_in),), device=G.device, dtype=torch.uint8)
     _check(lib().gift_whitened_error(_ptr(G), _ptr(G_hat), _dt(G), d_out, d_in, _ptr(U), _ptr(lam), _ptr(rho), rank,
                                      _ptr(out), _ptr(ws), ws.numel(), _stream(stream)), "gift_whitened_error")
+    return out
+
+
+# ---------------------------------------------------------------------------
+# Dense input-side transforms (full-rank A^{-1/2} and Cholesky L^{-T} variants)
+# ---------------------------------------------------------------------------
+def dense_factor_workspace_size(d: int, kind: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().gift_dense_factor_workspace_size(d, kind, ctypes.byref(n)), "gift_dense_factor_workspace_size")
+    return n.value
+
+
+def dense_factor(A: torch.Tensor, kind: int, ws: Optional[torch.Tensor] = None,
+                 dev_status: Optional[torch.Tensor] = None, stream=None):
+    """(M, M_inv, M_split, M_inv_split, dev_status) of gift_dense_factor for A (d x d fp32)."""
+    _cuda(A, ws, dev_status)
+    d = A.shape[0]
+    dev = A.device
+    M = torch.empty((d, d), device=dev, dtype=torch.float32)
+    Mi = torch.empty_like(M)
+    Ms = torch.empty((2, d, d), device=dev, dtype=torch.int16)
+    Mis = torch.empty_like(Ms)
+    if ws is None:
+        ws = torch.empty((dense_factor_workspace_size(d, kind),), device=dev, dtype=torch.uint8)
+    if dev_status is None:
+        dev_status = torch.zeros((1,), device=dev, dtype=torch.int32)
+    _check(lib().gift_dense_factor(_ptr(A), d, kind, _ptr(M), _ptr(Mi), _ptr(Ms), _ptr(Mis), _ptr(ws), ws.numel(),
+                                   _ptr(dev_status), _stream(stream)), "gift_dense_factor")
+    return M, Mi, Ms, Mis, dev_status
+
+
+def dense_split(M: torch.Tensor, stream=None) -> torch.Tensor:
+    """bf16 pair [hi ; lo] (2 x d x d, stored as int16) of an fp32 d x d transform."""
+    _cuda(M)
+    d = M.shape[0]
+    out = torch.empty((2, d, d), device=M.device, dtype=torch.int16)
+    _check(lib().gift_dense_split(_ptr(M), d, _ptr(out), _stream(stream)), "gift_dense_split")
+    return out
+
+
+def dense_encode(G: torch.Tensor, M_split: torch.Tensor, upper: bool = False, codes=None, scales=None,
+                 dev_status: Optional[torch.Tensor] = None, stream=None):
+    """(codes, scales) of W = G M (G bf16, M given as its bf16 pair)."""
+    _cuda(G, M_split, codes, scales, dev_status)
+    if G.dtype != torch.bfloat16:
+        raise TypeError("gift_dense_encode takes bf16 gradients")
+    d_out, d_in = G.shape
+    if codes is None:
+        codes = torch.empty((d_out, d_in), device=G.device, dtype=torch.uint8)
+    if scales is None:
+        scales = torch.empty((d_out, max(d_in // E4M3_BLOCK, 1)), device=G.device, dtype=torch.float32)
+    _check(lib().gift_dense_encode(_ptr(G), d_out, d_in, _ptr(M_split), int(upper), _ptr(codes), _ptr(scales),
+                                   _ptr(dev_status), _stream(stream)), "gift_dense_encode")
+    return codes, scales
+
+
+def dense_decode(codes: torch.Tensor, scales: torch.Tensor, M_inv_split: torch.Tensor, upper: bool = False,
+                 out_dtype=torch.bfloat16, out: Optional[torch.Tensor] = None,
+                 dev_status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """G_hat = W_hat M_inv (M_inv given as its bf16 pair)."""
+    _cuda(codes, scales, M_inv_split, out, dev_status)
+    d_out, d_in = codes.shape
+    if out is None:
+        out = torch.empty((d_out, d_in), device=codes.device, dtype=out_dtype)
+    _check(lib().gift_dense_decode(_ptr(codes), _ptr(scales), d_out, d_in, _ptr(M_inv_split), int(upper), _ptr(out),
+                                   _dt(out), _ptr(dev_status), _stream(stream)), "gift_dense_decode")
     return out

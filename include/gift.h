@@ -334,6 +334,62 @@ gift_status gift_decode_nvfp4(const uint8_t* codes, const uint8_t* block_scales,
                               const float* rho, int rank, void* G_hat, gift_dtype out_dt,
                               uint32_t* dev_status, gift_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * Dense input-side transforms: the variants GIFT is simplified from (review
+ * page, "What carries the argument": full two-sided K-FAC whitening, then
+ * the input side alone at full rank (Fig. 2 caption), then rank 32; section
+ * IV.A, Eq. (14) writes the input side with the Cholesky factor L_A^{-T}).
+ *
+ * gift_dense_factor: from A (d x d fp32, symmetric positive definite, e.g.
+ * A_out of gift_factor_refresh), in fp64:
+ *   GIFT_DENSE_CHOLESKY: A = L L^T, M = L^{-T}, M_inv = L^T (both upper
+ *                        triangular; W = G M has input-side covariance I);
+ *   GIFT_DENSE_INVSQRT:  M = A^{-1/2}, M_inv = A^{1/2} (coupled Newton-Schulz
+ *                        iteration, at most 60 steps; the rank-r construction
+ *                        of gift_encode at r = d_in).
+ * Outputs (device, d x d, row-major): M, M_inv in fp32; M_split, M_inv_split
+ * as bf16 pairs [hi (d x d) ; lo (d x d)] with x ~ hi + lo, the operands of
+ * gift_dense_encode / gift_dense_decode.  d % 128 == 0, 128 <= d <= 8192.
+ * ws: device scratch of gift_dense_factor_workspace_size bytes, 16-byte
+ * aligned.  dev_status (nullable): GIFT_DEV_RANK_DEFICIENT (a non-positive
+ * Cholesky pivot, replaced by a tiny one), GIFT_DEV_NONFINITE.
+ * Errors: GIFT_ERR_INVALID_ARG (null pointer, bad kind), GIFT_ERR_SHAPE,
+ * GIFT_ERR_WORKSPACE, GIFT_ERR_ALIGN, GIFT_ERR_CUDA.
+ * ------------------------------------------------------------------------ */
+#define GIFT_DENSE_CHOLESKY 1
+#define GIFT_DENSE_INVSQRT 2
+
+gift_status gift_dense_factor_workspace_size(int64_t d, int kind, size_t* bytes /* host */);
+
+gift_status gift_dense_factor(const float* A, int64_t d, int kind, float* M, float* M_inv, uint16_t* M_split,
+                              uint16_t* M_inv_split, void* ws, size_t ws_bytes, uint32_t* dev_status,
+                              gift_stream_t stream);
+
+/* fp32 d x d matrix -> its bf16 pair [hi ; lo] (for a transform made elsewhere). */
+gift_status gift_dense_split(const float* M, int64_t d, uint16_t* M_split, gift_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * E4M3 codec under a dense transform (tensor cores, bf16 gradients):
+ *   encode  W = G M; per row and block of 128 columns, scales = amax/448 and
+ *           codes = E4M3_RNE_satfinite(W * (448/amax)) as in gift_encode;
+ *   decode  G_hat = W_hat M_inv, W_hat = value(codes) * scale per block,
+ *           written as out_dt (bf16 by round-to-nearest-even, or fp32).
+ * G: d_out x d_in bf16.  M_split / M_inv_split: [hi ; lo] bf16 pairs of
+ * d_in x d_in.  upper_triangular != 0 declares M (M_inv) upper triangular
+ * (the Cholesky form), so products skip its zero blocks.  d_in % 128 == 0,
+ * 128 <= d_in <= 8192, d_out >= 0.  All pointers 16-byte aligned except
+ * dev_status (4).  dev_status (nullable): GIFT_DEV_NONFINITE,
+ * GIFT_DEV_TIMEOUT.  Errors: GIFT_ERR_INVALID_ARG, GIFT_ERR_SHAPE,
+ * GIFT_ERR_ALIGN, GIFT_ERR_CUDA.
+ * ------------------------------------------------------------------------ */
+gift_status gift_dense_encode(const void* G, int64_t d_out, int64_t d_in, const uint16_t* M_split,
+                              int upper_triangular, uint8_t* codes, float* scales, uint32_t* dev_status,
+                              gift_stream_t stream);
+
+gift_status gift_dense_decode(const uint8_t* codes, const float* scales, int64_t d_out, int64_t d_in,
+                              const uint16_t* M_inv_split, int upper_triangular, void* G_hat, gift_dtype out_dt,
+                              uint32_t* dev_status, gift_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

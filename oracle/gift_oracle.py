@@ -517,6 +517,17 @@ def cholesky_transform(A, inverse: bool = False) -> np.ndarray:
     return np.linalg.inv(L).T
 
 
+def encode_dense(G, M, block: int = BLOCK_E4M3):
+    """Per-block E4M3 of W = G M for a dense d_in x d_in transform M (the
+    full-rank or Cholesky variant): (codes, scales) as encode_e4m3."""
+    return quantize_e4m3_blocks(np.asarray(G, dtype=np.float64) @ np.asarray(M, dtype=np.float64), block)
+
+
+def decode_dense(codes, scales, M_inv, block: int = BLOCK_E4M3) -> np.ndarray:
+    """G_hat = W_hat M^{-1} for a dense transform (fp64)."""
+    return dequantize_e4m3_blocks(codes, scales, block) @ np.asarray(M_inv, dtype=np.float64)
+
+
 def two_sided_encode_decode(G, A, B, block: int = BLOCK_E4M3):
     """Full two-sided Cholesky whitening: W = L_B^{-1} G L_A^{-T}, per-block
     E4M3, G_hat = L_B W_hat L_A^T (B = E[delta delta^T], the output-side

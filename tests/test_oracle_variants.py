@@ -79,3 +79,28 @@ def test_input_side_captures_the_two_sided_benefit_on_realistic_structure():
     assert inp < 1.05 * two
     assert inp < 0.1 * res["euclid"]["white"]
     assert res["input_rank32"]["white"] < 0.2 * res["euclid"]["white"]
+
+
+def test_dense_codec_reduces_to_the_euclidean_codec_and_to_rank_r_at_full_rank():
+    """encode_dense / decode_dense (the codec under a dense transform): with
+    M = I it is the Euclidean per-block codec exactly; with M = A^{-1/2} it is
+    the rank-r codec at r = d_in (rho := 0) up to the rounding of two fp64
+    evaluations of the same matrix; and with the Cholesky transform the
+    round trip stays within the E4M3 error of W, mapped back by M^{-1}."""
+    X, _, G = _layer(d_in=256, d_out=64)
+    c0, s0 = O.encode_dense(G, np.eye(256))
+    c1, s1 = O.quantize_e4m3_blocks(G)
+    assert np.array_equal(c0, c1) and np.array_equal(s0, s1)
+    assert np.array_equal(O.decode_dense(c0, s0, np.eye(256)), O.dequantize_e4m3_blocks(c1, s1))
+    A = O.input_factor(X)
+    lam, V = np.linalg.eigh(A)
+    cf, sf = O.encode_dense(G, O.full_rank_transform(A))
+    cr, sr = O.encode_e4m3(G, V[:, ::-1], lam[::-1], 0.0)
+    assert (cf == cr).mean() >= 0.999
+    assert np.allclose(sf, sr, rtol=1e-6)
+    M, Mi = O.cholesky_transform(A), O.cholesky_transform(A, inverse=True)
+    c, s = O.encode_dense(G, M)
+    W = G @ M
+    Wh = O.dequantize_e4m3_blocks(c, s)
+    assert np.allclose(O.decode_dense(c, s, Mi), Wh @ Mi)
+    assert np.linalg.norm(Wh - W) <= 2.0 ** -4 * np.linalg.norm(W)
