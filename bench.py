@@ -299,7 +299,8 @@ def layers_measure(torch, ops, synth, dev, peak, reps=20):
         return float(np.median(ts_ms))
 
     out = {"workload": "one layer per call, rank-32 factor refreshed once (untimed); "
-                       "median of 20 calls, L2 flushed between calls"}
+                       "median of 20 calls, L2 flushed between calls; graph_replay: the same two calls "
+                       "captured in CUDA graphs and replayed (no host work per call)"}
     specs = (("512x512_f32", 512, 512, torch.float32, 2048, 0.8, 6001),
              ("4096x1536_bf16", 4096, 1536, torch.bfloat16, REFRESH_N, 1.0, 6002),
              ("11008x4096_bf16", 11008, 4096, torch.bfloat16, REFRESH_N, 1.0, 6003))
@@ -317,13 +318,25 @@ def layers_measure(torch, ops, synth, dev, peak, reps=20):
         Gh = torch.empty_like(G)
         enc = timed(lambda: ops.encode(G, U, lam, rho, codes=codes, scales=scales))
         dec = timed(lambda: ops.decode(codes, scales, U, lam, rho, out=Gh))
+        # the same calls captured once in CUDA graphs and replayed: kernel time
+        # without the binding's host work
+        side = torch.cuda.Stream()
+        ge, gd = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(ge, stream=side):
+            ops.encode(G, U, lam, rho, codes=codes, scales=scales)
+        with torch.cuda.graph(gd, stream=side):
+            ops.decode(codes, scales, U, lam, rho, out=Gh)
+        enc_g, dec_g = timed(ge.replay), timed(gd.replay)
         n = d_out * d_in
         gb = G.element_size()
         t = (enc + dec) * 1e-3
+        tg = (enc_g + dec_g) * 1e-3
         out[name] = {"encode_ms": enc, "decode_ms": dec, "gradient_gbs": gb * n / t / 1e9,
                      "elements_per_s": n / t, "panels": (d_out + 127) // 128,
-                     "roofline_frac": 2 * (gb + 1 + 4 / 128) * n / t / 1e9 / peak}
-        del G, Gh, codes, scales
+                     "roofline_frac": 2 * (gb + 1 + 4 / 128) * n / t / 1e9 / peak,
+                     "graph_replay": {"encode_ms": enc_g, "decode_ms": dec_g, "gradient_gbs": gb * n / tg / 1e9,
+                                      "roofline_frac": 2 * (gb + 1 + 4 / 128) * n / tg / 1e9 / peak}}
+        del G, Gh, codes, scales, ge, gd
     del flush
     torch.cuda.empty_cache()
     return out

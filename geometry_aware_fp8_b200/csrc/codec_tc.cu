@@ -1394,6 +1394,12 @@ int schedule(const TcLayer* layers, int n, uint16_t* off, uint16_t* ids, int max
 // faster by that estimate; a launch of many panels keeps single CTAs.
 constexpr int kSplitCost2 = 6, kSplitCost4 = 15;
 
+#ifndef GIFT_FORCE_SPLIT_DIN
+#define GIFT_FORCE_SPLIT_DIN 0
+#endif
+#ifndef GIFT_FORCE_SPLIT
+#define GIFT_FORCE_SPLIT 2
+#endif
 template <class SlotFn>
 int plan(const TcLayer* layers, int n, uint16_t* off, uint16_t* ids, int max_ids, SlotFn slots_for, int* split) {
   int min_nc = 1 << 30, max_nc = 0, panels = 0;
@@ -1401,6 +1407,10 @@ int plan(const TcLayer* layers, int n, uint16_t* off, uint16_t* ids, int max_ids
     min_nc = std::min(min_nc, layers[l].d_in / kChunk);
     max_nc = std::max(max_nc, layers[l].d_in / kChunk);
     panels += (layers[l].d_out + kPanel - 1) / kPanel;
+  }
+  if (GIFT_FORCE_SPLIT_DIN > 0 && min_nc * kChunk >= GIFT_FORCE_SPLIT_DIN && slots_for(GIFT_FORCE_SPLIT) > 0) {
+    *split = GIFT_FORCE_SPLIT;
+    return schedule(layers, n, off, ids, max_ids, slots_for(GIFT_FORCE_SPLIT), GIFT_FORCE_SPLIT, nullptr);
   }
   int best_s = 1;
   if (panels < kNumSMs) {
@@ -1428,9 +1438,11 @@ bool tc_codec_available() { return tmap_encoder() != nullptr; }
 // Layers [0, cnt) of one launch: the same format, at most kMaxJobs layers and
 // kMaxPanels panels, each layer at most 256 panels (0: the first layer is
 // larger and is coded in parts of 256 panels).
+static bool split_class(const TcLayer& L) { return GIFT_FORCE_SPLIT_DIN > 0 && L.d_in >= GIFT_FORCE_SPLIT_DIN; }
 static int group_count(const TcLayer* layers, int n) {
   int cnt = 0, panels = 0;
-  while (cnt < n && cnt < kMaxJobs && layers[cnt].fmt == layers[0].fmt) {
+  while (cnt < n && cnt < kMaxJobs && layers[cnt].fmt == layers[0].fmt &&
+         split_class(layers[cnt]) == split_class(layers[0])) {
     const int np = (layers[cnt].d_out + kPanel - 1) / kPanel;
     if (np > 256 || panels + np > kMaxPanels) break;
     panels += np;
@@ -1460,6 +1472,12 @@ int tc_codec_split(const TcLayer* layers, int n, bool encode) {
 cudaError_t launch_whiten_encode_tc(const TcLayer* layers, int n, uint32_t* err, cudaStream_t s,
                                     uint32_t stall_polls) {
   cudaError_t e = cudaSuccess;
+  std::vector<TcLayer> sorted;
+  if (GIFT_FORCE_SPLIT_DIN > 0 && n > 1) {
+    sorted.assign(layers, layers + n);
+    std::stable_partition(sorted.begin(), sorted.end(), [](const TcLayer& L) { return !split_class(L); });
+    layers = sorted.data();
+  }
   for (int base = 0; base < n;) {
     // pack as many layers as fit one launch
     const int cnt = group_count(layers + base, n - base);
@@ -1521,6 +1539,12 @@ cudaError_t launch_whiten_encode_tc(const TcLayer* layers, int n, uint32_t* err,
 cudaError_t launch_whiten_decode_tc(const TcLayer* layers, int n, uint32_t* err, cudaStream_t s,
                                     uint32_t stall_polls) {
   cudaError_t e = cudaSuccess;
+  std::vector<TcLayer> sorted;
+  if (GIFT_FORCE_SPLIT_DIN > 0 && n > 1) {
+    sorted.assign(layers, layers + n);
+    std::stable_partition(sorted.begin(), sorted.end(), [](const TcLayer& L) { return !split_class(L); });
+    layers = sorted.data();
+  }
   for (int base = 0; base < n;) {
     const int cnt = group_count(layers + base, n - base);
     if (cnt == 0) {
