@@ -395,6 +395,23 @@ gift_status gift_decode_nvfp4(const uint8_t* codes, const uint8_t* block_scales,
 }
 
 // ---------------------------------------------------------------------------
+gift_status gift_decode_sum(const uint8_t* const* codes, const float* const* scales, int n_parts, int64_t d_out,
+                            int64_t d_in, const float* U, const float* lambda, const float* rho, int rank,
+                            float alpha, void* G_hat, gift_dtype out_dt, uint32_t* dev_status, gift_stream_t stream) {
+  if (!codes || !scales || n_parts < 1 || n_parts > kDecodeSumMaxParts) return GIFT_ERR_INVALID_ARG;
+  for (int r = 0; r < n_parts; ++r) {
+    gift_status st = check_codec_args(G_hat, out_dt, d_out, d_in, U, lambda, rho, rank, codes[r], scales[r]);
+    if (st != GIFT_OK) return st;
+  }
+  if (dev_status && !aligned(dev_status, 4)) return GIFT_ERR_ALIGN;
+  if (d_out == 0) return GIFT_OK;
+  gift_status st = device_ok();
+  if (st != GIFT_OK) return st;
+  return cuda_status(launch_decode_sum(codes, scales, n_parts, d_out, d_in, U, lambda, rho, rank, alpha, G_hat, out_dt,
+                                       dev_status, (cudaStream_t)stream));
+}
+
+// ---------------------------------------------------------------------------
 static gift_status check_dense_d(int64_t d) {
   if (d < GIFT_E4M3_BLOCK || d % GIFT_E4M3_BLOCK != 0 || d > 8192) return GIFT_ERR_SHAPE;
   return GIFT_OK;

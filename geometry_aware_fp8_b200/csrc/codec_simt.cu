@@ -167,6 +167,93 @@ __global__ void __launch_bounds__(kWarps * 32) whiten_decode_simt_kernel(
   report_bits(err, bad, GIFT_DEV_NONFINITE);
 }
 
+// Decode-and-sum of the codes of several data-parallel ranks (the per-rank
+// gradients g^(r) of Eq. (1) on the review page): every rank codes its own
+// gradient with the shared factor, the codes and scales are all-gathered, and
+// each rank forms alpha sum_r T^{-1}(W_hat_r) = alpha T^{-1}(sum_r W_hat_r)
+// (T is linear, so the inverse transform is applied once, to the sum).
+// Same row layout as the decoder above; W_hat is summed over the parts in
+// part order in fp32.
+constexpr int kMaxParts = 64;
+struct SumParts {
+  const uint8_t* codes[kMaxParts];
+  const float* scales[kMaxParts];
+  int n;
+};
+
+GIFT_DEV void load_sum4(const SumParts& sp, int64_t row, int64_t d_in, int64_t nb, int64_t b, int64_t j0,
+                        float (&v)[4], bool& bad) {
+  v[0] = v[1] = v[2] = v[3] = 0.0f;
+  for (int r = 0; r < sp.n; ++r) {
+    const uint32_t q = __ldg(reinterpret_cast<const uint32_t*>(sp.codes[r] + row * d_in + j0));
+    const float s = __ldg(sp.scales[r] + row * nb + b);
+    bad |= not_finite(s);
+    const float2 lo = e4m3x2_to_f32x2((uint16_t)(q & 0xFFFF)), hi = e4m3x2_to_f32x2((uint16_t)(q >> 16));
+    v[0] = fmaf(lo.x, s, v[0]);
+    v[1] = fmaf(lo.y, s, v[1]);
+    v[2] = fmaf(hi.x, s, v[2]);
+    v[3] = fmaf(hi.y, s, v[3]);
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kWarps * 32) whiten_decode_sum_simt_kernel(
+    const __grid_constant__ SumParts sp, int64_t d_out, int64_t d_in, const float* __restrict__ U,
+    const float* __restrict__ lambda, const float* __restrict__ rho, int rank, float alpha, T* __restrict__ out,
+    uint32_t* err) {
+  __shared__ float c_s[32];
+  __shared__ float a_s;
+  __shared__ float part[kWarps][32];
+  __shared__ float pc_s[32];
+  transform_coeffs(lambda, rho, rank, true, c_s, &a_s, threadIdx.x);
+  __syncthreads();
+  const float a = a_s;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool vec = (rank & 3) == 0;
+  const int64_t nb = d_in / kBlock;
+  bool bad = false;
+  for (int64_t row = blockIdx.x; row < d_out; row += gridDim.x) {
+    float P[32];
+#pragma unroll
+    for (int k = 0; k < 32; ++k) P[k] = 0.0f;
+    if (rank > 0) {
+      for (int64_t b = warp; b < nb; b += kWarps) {
+        const int64_t j0 = b * kBlock + lane * 4;
+        float v[4];
+        load_sum4(sp, row, d_in, nb, b, j0, v, bad);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          float u[32];
+          u_row(U, j0 + e, rank, vec, u);
+#pragma unroll
+          for (int k = 0; k < 32; ++k) P[k] = fmaf(v[e], u[k], P[k]);
+        }
+      }
+    }
+    float pc[32];
+    row_projection(P, c_s, part, pc_s, pc, warp, lane);
+    for (int64_t b = warp; b < nb; b += kWarps) {
+      const int64_t j0 = b * kBlock + lane * 4;
+      float v[4];
+      load_sum4(sp, row, d_in, nb, b, j0, v, bad);
+      float o[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        float acc = 0.0f;
+        if (rank > 0) {
+          float u[32];
+          u_row(U, j0 + e, rank, vec, u);
+#pragma unroll
+          for (int k = 0; k < 32; ++k) acc = fmaf(pc[k], u[k], acc);
+        }
+        o[e] = alpha * fmaf(a, v[e], acc);
+      }
+      store4<T>(out + row * d_in + j0, o);
+    }
+  }
+  report_bits(err, bad, GIFT_DEV_NONFINITE);
+}
+
 // One CTA per row, capped at a few waves of resident CTAs (rows are then
 // taken in a grid-stride loop).
 int grid_rows(int64_t d_out) {
@@ -199,6 +286,26 @@ cudaError_t launch_whiten_decode_simt(const uint8_t* codes, const float* scales,
   else
     whiten_decode_simt_kernel<float><<<grid, kWarps * 32, 0, s>>>(codes, scales, d_out, d_in, U, lambda, rho,
                                                                   rank, (float*)G_hat, err);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decode_sum(const uint8_t* const* codes, const float* const* scales, int n_parts, int64_t d_out,
+                              int64_t d_in, const float* U, const float* lambda, const float* rho, int rank,
+                              float alpha, void* G_hat, gift_dtype dt, uint32_t* err, cudaStream_t s) {
+  if (n_parts > kMaxParts) return cudaErrorInvalidValue;
+  SumParts sp;
+  sp.n = n_parts;
+  for (int r = 0; r < n_parts; ++r) {
+    sp.codes[r] = codes[r];
+    sp.scales[r] = scales[r];
+  }
+  const int grid = grid_rows(d_out);
+  if (dt == GIFT_BF16)
+    whiten_decode_sum_simt_kernel<__nv_bfloat16><<<grid, kWarps * 32, 0, s>>>(sp, d_out, d_in, U, lambda, rho, rank,
+                                                                              alpha, (__nv_bfloat16*)G_hat, err);
+  else
+    whiten_decode_sum_simt_kernel<float><<<grid, kWarps * 32, 0, s>>>(sp, d_out, d_in, U, lambda, rho, rank, alpha,
+                                                                      (float*)G_hat, err);
   return cudaGetLastError();
 }
 

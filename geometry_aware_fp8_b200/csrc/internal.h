@@ -35,6 +35,12 @@ cudaError_t launch_whiten_decode_simt(const uint8_t* codes, const float* scales,
                                       const float* U, const float* lambda, const float* rho, int rank,
                                       void* G_hat, gift_dtype dt, uint32_t* err, cudaStream_t s);
 
+// Decode-and-sum of n_parts code sets (data-parallel ranks), CUDA cores.
+constexpr int kDecodeSumMaxParts = 64;
+cudaError_t launch_decode_sum(const uint8_t* const* codes, const float* const* scales, int n_parts, int64_t d_out,
+                              int64_t d_in, const float* U, const float* lambda, const float* rho, int rank,
+                              float alpha, void* G_hat, gift_dtype dt, uint32_t* err, cudaStream_t s);
+
 // ---- Whitened codec on the tensor cores (bf16 G, tcgen05 + TMA) ----
 struct TcLayer {
   const void* G;      // bf16 d_out x d_in (encode input)

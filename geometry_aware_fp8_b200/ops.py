@@ -29,7 +29,7 @@ EXPORTED = ("gift_status_string", "gift_version", "gift_refresh_workspace_size",
             "gift_error_workspace_size", "gift_roundtrip_error", "gift_encode_nvfp4", "gift_decode_nvfp4",
             "gift_codec_split", "gift_whitened_error_workspace_size", "gift_whitened_error",
             "gift_codec_stall_test", "gift_dense_factor_workspace_size", "gift_dense_factor", "gift_dense_split",
-            "gift_dense_encode", "gift_dense_decode")
+            "gift_dense_encode", "gift_dense_decode", "gift_decode_sum")
 DENSE_CHOLESKY, DENSE_INVSQRT = 1, 2
 
 
@@ -89,6 +89,8 @@ def lib() -> ctypes.CDLL:
         L.gift_whitened_error.argtypes = [vp, vp, i32, i64, i64, vp, vp, vp, i32, vp, vp, sz, vp]
         L.gift_encode_nvfp4.argtypes = [vp, i32, i64, i64, vp, vp, vp, i32, vp, vp, vp, vp, vp]
         L.gift_decode_nvfp4.argtypes = [vp, vp, vp, i64, i64, vp, vp, vp, i32, vp, i32, vp, vp]
+        L.gift_decode_sum.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(vp), i32, i64, i64, vp, vp, vp, i32,
+                                      ctypes.c_float, vp, i32, vp, vp]
         L.gift_dense_factor_workspace_size.argtypes = [i64, i32, ctypes.POINTER(sz)]
         L.gift_dense_factor.argtypes = [vp, i64, i32, vp, vp, vp, vp, vp, sz, vp, vp]
         L.gift_dense_split.argtypes = [vp, i64, vp, vp]
@@ -328,6 +330,26 @@ def encode_many(packed, n: int, stream=None, dev_status: Optional[torch.Tensor] 
 def decode_many(packed, n: int, stream=None, dev_status: Optional[torch.Tensor] = None):
     _cuda(dev_status)
     _check(lib().gift_decode_many(packed, n, _ptr(dev_status), _stream(stream)), "gift_decode_many")
+
+
+def decode_sum(codes: Sequence[torch.Tensor], scales: Sequence[torch.Tensor], U=None, lam=None, rho=None,
+               rank: Optional[int] = None, alpha: float = 1.0, out_dtype=torch.float32,
+               out: Optional[torch.Tensor] = None, dev_status: Optional[torch.Tensor] = None, stream=None):
+    """alpha * sum_r decode(codes[r], scales[r]) through one inverse transform (gift_decode_sum)."""
+    n = len(codes)
+    if n != len(scales) or n < 1:
+        raise ValueError("codes and scales must be equally long, non-empty lists")
+    _cuda(*codes, *scales, U, lam, rho, out, dev_status)
+    d_out, d_in = codes[0].shape
+    if rank is None:
+        rank = 0 if U is None else U.shape[1]
+    if out is None:
+        out = torch.empty((d_out, d_in), device=codes[0].device, dtype=out_dtype)
+    cp = (ctypes.c_void_p * n)(*[c.data_ptr() for c in codes])
+    sp = (ctypes.c_void_p * n)(*[x.data_ptr() for x in scales])
+    _check(lib().gift_decode_sum(cp, sp, n, d_out, d_in, _ptr(U), _ptr(lam), _ptr(rho), rank, float(alpha), _ptr(out),
+                                 _dt(out), _ptr(dev_status), _stream(stream)), "gift_decode_sum")
+    return out
 
 
 def codec_stall_test(layer: LayerArgs, encode: bool, stall_polls: int, dev_status: torch.Tensor, stream=None):

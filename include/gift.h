@@ -227,6 +227,28 @@ gift_status gift_decode_many(const gift_layer* layers /* host */, int n, uint32_
                              gift_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * Decode-and-sum for data-parallel training (review page, referee report on
+ * section II.A, Eq. (1): the per-rank gradients g^(r); abstract: the
+ * communication collective is left unchanged).  Every rank codes its own
+ * gradient with the shared factor (gift_encode), the codes and scales of
+ * all ranks are all-gathered by the caller's collective, and each rank forms
+ *
+ *   G_hat = alpha * sum_r W_hat_r M^{-1}  =  alpha * (sum_r W_hat_r) M^{-1}
+ *
+ * (M^{-1} is linear, so it is applied once, to the fp32 sum of the
+ * dequantised parts, added in part order).  alpha = 1 gives the sum,
+ * 1 / n_parts the mean.  codes / scales: HOST arrays of n_parts DEVICE
+ * pointers, each laid out as gift_decode's codes and scales; 1 <= n_parts
+ * <= 64.  Other arguments, layouts and alignment as for gift_decode (rank 0:
+ * the Euclidean codec, M = I).  Runs on the CUDA cores.
+ * dev_status (nullable): GIFT_DEV_NONFINITE (a non-finite scale).
+ * ------------------------------------------------------------------------ */
+gift_status gift_decode_sum(const uint8_t* const* codes /* host */, const float* const* scales /* host */,
+                            int n_parts, int64_t d_out, int64_t d_in, const float* U, const float* lambda,
+                            const float* rho, int rank, float alpha, void* G_hat, gift_dtype out_dt,
+                            uint32_t* dev_status, gift_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * Test hook of the codec's failure path (the pages have no counterpart).
  * Launches the tensor-core whitened encoder (encode != 0) or decoder on one
  * layer (bf16, rank 32, d_in <= 8192) with one extra wait before any work:
