@@ -473,6 +473,13 @@ def profile_kernels(torch, fn):
     return out
 
 
+def kernel_short_name(name):
+    """'void gift::(anonymous namespace)::syrk_tc_kernel<...>(...)' -> 'syrk_tc_kernel'."""
+    import re
+    m = re.search(r"([A-Za-z_][A-Za-z0-9_]*)(<[^()]*>)?\(", name)
+    return m.group(1) if m else name
+
+
 def count_launches(torch, ops, W, K, n_refresh):
     """libgift kernels launched inside the two timed regions (K codec steps,
     n_refresh batched refreshes), counted with the CUDA profiler on one
@@ -592,7 +599,7 @@ def config4_refresh_measure(torch, ops, synth, dev, bf16_peak, reps=5):
            "syrk_ms": syrk, "syrk_tflops": flops / (syrk * 1e-3) / 1e12 if syrk else None,
            "syrk_frac_of_bf16_peak": flops / (syrk * 1e-3) / 1e12 / bf16_peak if syrk else None,
            "syrk_share": syrk / tot if tot else None,
-           "kernels_ms": {k.split("(")[0].split("::")[-1]: round(t, 4) for k, (_, t) in kern.items()},
+           "kernels_ms": {kernel_short_name(k): round(t, 4) for k, (_, t) in kern.items()},
            "lambda_1": float(lam[0].item()), "rho": float(rho.item()), "dev_status": int(st.item())}
     del X, A, ws
     torch.cuda.empty_cache()
