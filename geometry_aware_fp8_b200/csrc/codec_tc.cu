@@ -327,19 +327,9 @@ GIFT_DEV void split_bf16(float x, float& hi, float& lo) {
   lo = x - hi;
 }
 
-// Row t of the U tile: TMA has placed U[j0 + t][0..31] there as fp32 (one
-// 128-byte swizzled row); it is replaced in place by its bf16 split
-// [hi 0..31 | lo 0..31], the same 128 bytes in the same swizzle.
-GIFT_DEV void convert_u_row_inplace(uint32_t tile, int t) {
-  float u[32];
-#pragma unroll
-  for (int q = 0; q < 8; ++q) {
-    const uint4 v = ld_shared_v4(tile + sw128(t, q));
-    u[4 * q] = __uint_as_float(v.x);
-    u[4 * q + 1] = __uint_as_float(v.y);
-    u[4 * q + 2] = __uint_as_float(v.z);
-    u[4 * q + 3] = __uint_as_float(v.w);
-  }
+// bf16 split [hi 0..31 | lo 0..31] of a U row into row t of a [128][128 B]
+// tile with the 128-byte swizzle.
+GIFT_DEV void store_u_split_bf16(uint32_t tile, int t, const float (&u)[32]) {
   uint32_t hi[16], lo[16];
 #pragma unroll
   for (int k = 0; k < 16; ++k) {
@@ -356,21 +346,12 @@ GIFT_DEV void convert_u_row_inplace(uint32_t tile, int t) {
     st_shared_v4(tile + sw128(t, 4 + q), lo[4 * q], lo[4 * q + 1], lo[4 * q + 2], lo[4 * q + 3]);
 }
 
-// As convert_u_row_inplace, with f16 parts for the decoder's first pass:
+// As store_u_split_bf16, with f16 parts for the decoder's first pass:
 // [hi 0..31 | lo 0..31] with hi = f16(u) and lo = f16((u - hi) * 2^11) (the
 // product with lo is scaled back by 2^-11 in the epilogue).  f16 keeps 11
 // mantissa bits per part, and every E4M3 or NVFP4 value is exact in f16.
 constexpr float kF16LoScale = 2048.0f;
-GIFT_DEV void convert_u_row_inplace_f16(uint32_t tile, int t) {
-  float u[32];
-#pragma unroll
-  for (int q = 0; q < 8; ++q) {
-    const uint4 v = ld_shared_v4(tile + sw128(t, q));
-    u[4 * q] = __uint_as_float(v.x);
-    u[4 * q + 1] = __uint_as_float(v.y);
-    u[4 * q + 2] = __uint_as_float(v.z);
-    u[4 * q + 3] = __uint_as_float(v.w);
-  }
+GIFT_DEV void store_u_split_f16(uint32_t tile, int t, const float (&u)[32]) {
   uint32_t hi[16], lo[16];
 #pragma unroll
   for (int k = 0; k < 16; ++k) {
@@ -385,6 +366,36 @@ GIFT_DEV void convert_u_row_inplace_f16(uint32_t tile, int t) {
   for (int q = 0; q < 4; ++q)
     st_shared_v4(tile + sw128(t, 4 + q), lo[4 * q], lo[4 * q + 1], lo[4 * q + 2], lo[4 * q + 3]);
 }
+
+// Row t of a U tile that TMA placed in shared memory as fp32 (one 128-byte
+// swizzled row), or row `row` of U read from global memory (L2-resident).
+GIFT_DEV void u_row_from_tile(uint32_t tile, int t, float (&u)[32]) {
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const uint4 v = ld_shared_v4(tile + sw128(t, q));
+    u[4 * q] = __uint_as_float(v.x);
+    u[4 * q + 1] = __uint_as_float(v.y);
+    u[4 * q + 2] = __uint_as_float(v.z);
+    u[4 * q + 3] = __uint_as_float(v.w);
+  }
+}
+GIFT_DEV void u_row_from_global(const float* U, int64_t row, float (&u)[32]) {
+  const float4* p = reinterpret_cast<const float4*>(U + row * 32);
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const float4 v = __ldg(p + q);
+    u[4 * q] = v.x;
+    u[4 * q + 1] = v.y;
+    u[4 * q + 2] = v.z;
+    u[4 * q + 3] = v.w;
+  }
+}
+#ifndef GIFT_U_LSU
+#define GIFT_U_LSU 0
+#endif
+// U rows reach the converters by TMA with the stage (0) or by 16-byte loads
+// from global memory (1), which keeps them off the TMA path.
+constexpr bool kULsu = GIFT_U_LSU != 0;
 
 template <int FMT, bool CLUSTER>
 __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __grid_constant__ EncParams p,
@@ -497,10 +508,10 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
         const EncJob& J = p.jobs[st.job()];
         const uint64_t pol = st.pass == 0 ? keep : drop;
         const uint32_t dst = sbase + s * kStageBytes;
-        mbar_arrive_expect_tx(&tfull[s], kGBytes + kUBytes);
+        mbar_arrive_expect_tx(&tfull[s], kULsu ? kGBytes : kGBytes + kUBytes);
         tma_load_2d_hint(dst, &J.tmG, &tfull[s], st.chunk() * kChunk, st.panel() * kPanel, pol);
         tma_load_2d_hint(dst + kGHalf, &J.tmG, &tfull[s], st.chunk() * kChunk + 64, st.panel() * kPanel, pol);
-        tma_load_2d_hint(dst + kGBytes, &J.tmU, &tfull[s], 0, st.chunk() * kChunk, keep);
+        if (!kULsu) tma_load_2d_hint(dst + kGBytes, &J.tmU, &tfull[s], 0, st.chunk() * kChunk, keep);
       }
     }
   } else if (warp == 14) {
@@ -535,12 +546,16 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
     for (Steps<EncParams> st(p, beg, end, q, S); st.valid(); st.next(), ++step) {
       const int s = step % kStages;
       const uint32_t use = step / kStages;
+      float u[32];
+      if (kULsu) u_row_from_global(p.jobs[st.job()].U, (int64_t)st.chunk() * kChunk + t, u);  // before the wait
       const bool ok = mbar_wait(&tfull[s], use & 1u, kWaitLimit);
       if (named_sync_or(1, 128, !ok)) {
         failed = 1;
         break;
       }
-      convert_u_row_inplace(sbase + s * kStageBytes + kGBytes, t);
+      const uint32_t u_tile = sbase + s * kStageBytes + kGBytes;
+      if (!kULsu) u_row_from_tile(u_tile, t, u);
+      store_u_split_bf16(u_tile, t, u);
       fence_async_shared();
       named_sync(1, 128);
       if (t == 0) mbar_arrive(&full[s]);
@@ -916,14 +931,15 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
         }
         const DecJob& J = p.jobs[st.job()];
         const uint32_t dst = sbase + s * kDStageBytes;
+        const uint32_t ub = kULsu ? 0u : (uint32_t)kUBytes;
         if (FMT == kFmtE4M3) {
-          mbar_arrive_expect_tx(&cfull[s], kDCodes + kUBytes);
+          mbar_arrive_expect_tx(&cfull[s], kDCodes + ub);
           tma_load_2d_hint(dst, &J.tmC, &cfull[s], st.chunk() * kChunk, st.panel() * kPanel,
                            st.pass == 0 ? keep : drop);
         } else {
-          mbar_arrive_expect_tx(&cfull[s], kUBytes);  // NVFP4 codes are read from global memory
+          mbar_arrive_expect_tx(&cfull[s], ub);  // NVFP4 codes are read from global memory
         }
-        tma_load_2d_hint(dst + kDCodes, &J.tmU, &cfull[s], 0, st.chunk() * kChunk, keep);
+        if (!kULsu) tma_load_2d_hint(dst + kDCodes, &J.tmU, &cfull[s], 0, st.chunk() * kChunk, keep);
       }
     }
   } else if (warp == 14) {
@@ -960,6 +976,8 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
     for (Steps<DecParams> st(p, beg, end, q, S); st.valid(); st.next(), ++step) {
       const int s = step % kDStages, j = step & 1;
       const uint32_t use = step / kDStages;
+      float u[32];
+      if (kULsu) u_row_from_global(p.jobs[st.job()].U, (int64_t)st.chunk() * kChunk + t, u);  // before the wait
       bool ok = mbar_wait(&cfull[s], use & 1u, kWaitLimit);
       if (st.pass == 0 && step >= 2) ok = ok && mbar_wait(&sfree[j], ((step >> 1) - 1) & 1u, kWaitLimit);
       if (named_sync_or(1, 128, !ok)) {
@@ -970,10 +988,11 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
       const uint32_t u_tile = c_tile + kDCodes;
       const uint32_t q_tile = scr + j * kDScratch;
       // D2 multiplies f16 codes by an f16 split of U, D3 the bf16 P' o c' by a bf16 split
+      if (!kULsu) u_row_from_tile(u_tile, t, u);
       if (st.pass == 0)
-        convert_u_row_inplace_f16(u_tile, t);
+        store_u_split_f16(u_tile, t, u);
       else
-        convert_u_row_inplace(u_tile, t);
+        store_u_split_bf16(u_tile, t, u);
       const DecJob& J = p.jobs[st.job()];
       if (st.pass == 0 && FMT != kFmtE4M3) {
         // NVFP4: row t's 128 codes (64 bytes) and 8 block scales from global,
