@@ -396,6 +396,17 @@ GIFT_DEV void u_row_from_global(const float* U, int64_t row, float (&u)[32]) {
 // U rows reach the converters by TMA with the stage (0) or by 16-byte loads
 // from global memory (1), which keeps them off the TMA path.
 constexpr bool kULsu = GIFT_U_LSU != 0;
+#ifndef GIFT_OUT_LSU
+#define GIFT_OUT_LSU 0
+#endif
+// Output tiles (encoder codes, decoder G_hat) leave by TMA stores (0) or by
+// coalesced 16-byte stores of the epilogue threads (1).
+constexpr bool kOutLsu = GIFT_OUT_LSU != 0;
+
+GIFT_DEV void st_global_v4_cs(void* p, uint4 v) {
+  asm volatile("st.global.cs.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
 
 template <int FMT, bool CLUSTER>
 __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __grid_constant__ EncParams p,
@@ -527,7 +538,7 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
           break;
         }
         const EncJob& J = p.jobs[st.job()];
-        if (FMT == kFmtE4M3) {  // NVFP4 codes leave from the epilogue
+        if (FMT == kFmtE4M3 && !kOutLsu) {  // otherwise the epilogue has stored the tile
           tma_store_2d_hint(&J.tmC, cbuf + cb * kCodesBytes, st.chunk() * kChunk, st.panel() * kPanel, drop);
           bulk_commit();
           bulk_wait_read<0>();
@@ -764,7 +775,20 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
 #pragma unroll
       for (int q = 0; q < 4; ++q)
         st_shared_v4(c_tile + sw128(r, 4 * h + q), cw[4 * q], cw[4 * q + 1], cw[4 * q + 2], cw[4 * q + 3]);
-      fence_async_shared();
+      if (kOutLsu && FMT == kFmtE4M3) {
+        // the tile's 1024 16-byte chunks, two rows of 128 B per warp instruction
+        named_sync(2, 256);
+        const int tid = threadIdx.x;  // 0..255
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int e = i * 256 + tid, rr = e >> 3, cq = e & 7;
+          const int64_t grow = (int64_t)panel * kPanel + rr;
+          const uint4 v = ld_shared_v4(c_tile + sw128(rr, cq));
+          if (grow < J.d_out) st_global_v4_cs(J.codes + grow * J.d_in + c * kChunk + cq * 16, v);
+        }
+      } else {
+        fence_async_shared();
+      }
       mbar_arrive(&cready[cb]);
       ++e2;
     }
@@ -818,6 +842,7 @@ struct alignas(64) DecJob {
   const uint8_t* codes;   // NVFP4 [d_out][d_in/2] (read directly; E4M3 codes arrive by TMA)
   const uint8_t* sb;      // NVFP4 E4M3 block scales [d_out][d_in/16]
   const float* tscale;    // NVFP4 tensor scale
+  void* G_hat;            // bf16 [d_out][d_in] (stores by the epilogue; TMA stores use tmO)
   int d_out, d_in, rank, fmt;
 };
 
@@ -852,7 +877,8 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
   uint64_t* empty = bars + 2 * kDStages;   // [kDStages] count 1: MMA commit (D2) or store warp (D3)
   uint64_t* sfree = bars + 3 * kDStages;   // [2] count 1: scratch tile free (MMA commit or store read)
   uint64_t* oready = sfree + 2;            // [2] count 256: output tile written
-  uint64_t* t_full = oready + 2;           // [2] count 1
+  uint64_t* ostored = oready + 2;          // [2] count 256: output tile copied out by the epilogue
+  uint64_t* t_full = ostored + 2;          // [2] count 1
   uint64_t* t_empty = t_full + 2;          // [2] count 256
   uint64_t* pc_full = t_full + 4;          // count 256
   uint64_t* w_full = t_full + 5;           // [2] count 1
@@ -880,6 +906,7 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sfree[b], 1);
       mbar_init(&oready[b], 256);
+      mbar_init(&ostored[b], 256);
       mbar_init(&t_full[b], 1);
       mbar_init(&t_empty[b], 256);
       mbar_init(&w_full[b], 1);
@@ -957,14 +984,22 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
           failed = 1;
           break;
         }
-        par ^= 1u << j;
         mbar_arrive(&empty[s]);
-        const DecJob& J = p.jobs[st.job()];
-        const uint32_t o_tile = scr + j * kDScratch;
-        tma_store_2d_hint(&J.tmO, o_tile, st.chunk() * kChunk, st.panel() * kPanel, drop);
-        tma_store_2d_hint(&J.tmO, o_tile + kGHalf, st.chunk() * kChunk + 64, st.panel() * kPanel, drop);
-        bulk_commit();
-        bulk_wait_read<0>();
+        if (kOutLsu) {
+          // the epilogue copies the tile out itself; the tile is free once it has
+          if (!mbar_wait(&ostored[j], (par >> j) & 1u, kWaitLimit)) {
+            failed = 1;
+            break;
+          }
+        } else {
+          const DecJob& J = p.jobs[st.job()];
+          const uint32_t o_tile = scr + j * kDScratch;
+          tma_store_2d_hint(&J.tmO, o_tile, st.chunk() * kChunk, st.panel() * kPanel, drop);
+          tma_store_2d_hint(&J.tmO, o_tile + kGHalf, st.chunk() * kChunk + 64, st.panel() * kPanel, drop);
+          bulk_commit();
+          bulk_wait_read<0>();
+        }
+        par ^= 1u << j;
         mbar_arrive(&sfree[j]);
       }
       bulk_wait_all();
@@ -1236,6 +1271,20 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
         mbar_arrive(&w_empty[b]);
         fence_async_shared();
         mbar_arrive(&oready[j]);
+        if (kOutLsu) {
+          // the tile's 2048 16-byte chunks, two rows of 256 B per warp instruction
+          named_sync(2, 256);
+          const int tid = threadIdx.x;  // 0..255
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int e = i * 256 + tid, rr = e >> 4, cq = e & 15;
+            const int64_t grow = (int64_t)st.panel() * kPanel + rr;
+            const uint4 v = ld_shared_v4(o_tile + (cq >> 3) * kGHalf + sw128(rr, cq & 7));
+            if (grow < J.d_out)
+              st_global_v4_cs(reinterpret_cast<__nv_bfloat16*>(J.G_hat) + grow * J.d_in + c * kChunk + cq * 8, v);
+          }
+          mbar_arrive(&ostored[j]);
+        }
         ++e2;
       }
     }
@@ -1602,6 +1651,7 @@ cudaError_t launch_whiten_decode_tc(const TcLayer* layers, int n, uint32_t* err,
       J.codes = L.codes;
       J.sb = L.block_scales;
       J.tscale = L.tensor_scale;
+      J.G_hat = L.G_hat;
       J.fmt = L.fmt;
       J.d_out = L.d_out;
       J.d_in = L.d_in;
