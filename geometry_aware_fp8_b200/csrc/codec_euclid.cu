@@ -82,17 +82,27 @@ __global__ void __launch_bounds__(256) euclid_encode_kernel(const T* __restrict_
   const int sub = threadIdx.x & 7;
   bool bad = false;
   const int64_t groups_per_grid = (int64_t)gridDim.x * (blockDim.x >> 3);
-  for (int64_t b = (int64_t)blockIdx.x * (blockDim.x >> 3) + (threadIdx.x >> 3); b < n_blocks;
-       b += groups_per_grid) {
+  // the loop bound is the warp's first block, so all 32 lanes take every
+  // iteration together and meet at the shuffles; lanes past the end idle
+  for (int64_t base = (int64_t)blockIdx.x * (blockDim.x >> 3) + ((threadIdx.x >> 5) << 2); base < n_blocks;
+       base += groups_per_grid) {
+    const int64_t b = base + ((threadIdx.x & 31) >> 3);
+    const bool act = b < n_blocks;
     const int64_t e0 = b * kBlock + sub * 16;
     float v[16];
-    Vec16<T>::load(G + e0, v);
+    if (act) {
+      Vec16<T>::load(G + e0, v);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) v[i] = 0.0f;
+    }
     float m = 0.0f;
 #pragma unroll
     for (int i = 0; i < 16; ++i) m = fmax_nan(m, fabsf(v[i]));
     m = fmax_nan(m, __shfl_xor_sync(0xffffffffu, m, 1));
     m = fmax_nan(m, __shfl_xor_sync(0xffffffffu, m, 2));
     m = fmax_nan(m, __shfl_xor_sync(0xffffffffu, m, 4));
+    if (!act) continue;
     bad |= not_finite(m);
     const float inv = e4m3_inv_scale(m);
     __stcs(reinterpret_cast<uint4*>(codes + e0), quantize16(v, inv));
@@ -170,18 +180,26 @@ __global__ void __launch_bounds__(256) euclid_encode_group_kernel(const __grid_c
   const int sub = threadIdx.x & 7;
   const int64_t total = pre[g.n];
   const int64_t G = (int64_t)gridDim.x * (blockDim.x >> 3);
-  const int64_t first = (int64_t)blockIdx.x * (blockDim.x >> 3) + (threadIdx.x >> 3);
+  // per warp: blocks base .. base + 3 (the loop bound is the warp's first
+  // block, so all 32 lanes take every iteration together and meet at the
+  // shuffles; lanes past the end idle)
+  const int64_t wfirst = (int64_t)blockIdx.x * (blockDim.x >> 3) + ((threadIdx.x >> 5) << 2);
+  const int64_t first = wfirst + ((threadIdx.x & 31) >> 3);
   int l0 = first < total ? find_layer(pre, g.n, first) : 0, l1 = l0;
   bool bad = false;
-  for (int64_t b0 = first; b0 < total; b0 += 2 * G) {
+  for (int64_t base = wfirst; base < total; base += 2 * G) {
+    const int64_t b0 = base + ((threadIdx.x & 31) >> 3);
     const int64_t b1 = b0 + G;
+    const bool has0 = b0 < total;
     const bool has1 = b1 < total;
-    l0 = advance_layer(pre, g.n, l0, b0);
+    if (has0) l0 = advance_layer(pre, g.n, l0, b0);
     l1 = has1 ? advance_layer(pre, g.n, l1 > l0 ? l1 : l0, b1) : l0;
-    const int64_t e0 = (b0 - pre[l0]) * kBlock + sub * 16;
+    const int64_t e0 = has0 ? (b0 - pre[l0]) * kBlock + sub * 16 : 0;
     const int64_t e1 = has1 ? (b1 - pre[l1]) * kBlock + sub * 16 : e0;
     float v0[16], v1[16];
-    Vec16<T>::load((const T*)g.src[l0] + e0, v0);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v0[i] = v1[i] = 0.0f;
+    if (has0) Vec16<T>::load((const T*)g.src[l0] + e0, v0);
     if (has1) Vec16<T>::load((const T*)g.src[l1] + e1, v1);
     float m0 = 0.0f, m1 = 0.0f;
 #pragma unroll
@@ -194,6 +212,7 @@ __global__ void __launch_bounds__(256) euclid_encode_group_kernel(const __grid_c
       m0 = fmax_nan(m0, __shfl_xor_sync(0xffffffffu, m0, o));
       m1 = fmax_nan(m1, __shfl_xor_sync(0xffffffffu, m1, o));
     }
+    if (!has0) continue;  // after the shuffles; has1 implies has0
     bad |= not_finite(m0) || (has1 && not_finite(m1));
     const float i0 = e4m3_inv_scale(m0);
     __stcs(reinterpret_cast<uint4*>((uint8_t*)g.dst[l0] + e0), quantize16(v0, i0));

@@ -158,10 +158,10 @@ GIFT_DEV float fmax_nan(float a, float b) {
 }
 GIFT_DEV bool not_finite(float x) { return !(fabsf(x) <= 3.402823466e38f); }
 
-// OR `bits` into *err once per warp for the lanes whose `bad` is set (every
-// lane of the warp must call it).
+// OR `bits` into *err from every thread whose `bad` is set.  Not a warp
+// collective: callers may have lanes that already left their loops.
 GIFT_DEV void report_bits(uint32_t* err, bool bad, uint32_t bits) {
-  if (__any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0 && err) atomicOr(err, bits);
+  if (bad && err) atomicOr(err, bits);
 }
 
 // ---------------------------------------------------------------------------
