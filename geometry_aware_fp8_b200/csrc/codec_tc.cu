@@ -59,11 +59,24 @@ constexpr int kPcBytes = kPanel * 128;         // 16 KB: [128 rows][64 bf16]
 constexpr int kCodesBytes = kPanel * kChunk;    // 16 KB: codes of one chunk
 constexpr int kIdBytes = 16 * 128;             // 2 KB: 16 x 16 bf16 identity, 128-byte rows
 constexpr int kXBytes = kPanel * 32 * 4;        // 16 KB: fp32 partial projections exchanged in a cluster
-constexpr int kSmemBytes = kStages * kStageBytes + kPcBytes + 2 * kCodesBytes + kIdBytes + 1024 + 512;
+#ifndef GIFT_W_BUFS
+#define GIFT_W_BUFS 2
+#endif
+#ifndef GIFT_C_BUFS
+#define GIFT_C_BUFS 2
+#endif
+// TMEM accumulators of W for the second pass (2 or 3; the third sits at
+// columns 384..511, after P (encoder) or the decoder's T buffers) and codes
+// tiles of the encoder (2 or 3).
+constexpr int kWBufs = GIFT_W_BUFS, kCBufs = GIFT_C_BUFS;
+static_assert(kWBufs == 2 || kWBufs == 3, "W buffers");
+static_assert(kCBufs == 2 || kCBufs == 3, "codes tiles");
+constexpr int kSmemBytes = kStages * kStageBytes + kPcBytes + kCBufs * kCodesBytes + kIdBytes + 1024 + 512;
 constexpr int enc_smem(bool cluster) { return kSmemBytes + (cluster ? kXBytes : 0); }
 constexpr int kThreads = 480;  // 8 epilogue + 4 converter + MMA + TMA load + TMA store warps
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColW0 = 0, kColW1 = 128, kColP = 256;
+GIFT_DEV uint32_t w_col(int b) { return b == 0 ? 0u : b == 1 ? 128u : 384u; }
 constexpr uint32_t kIdescE1 = umma_idesc_bf16(128, 64, 0, 1);   // A K-major, B MN-major
 constexpr uint32_t kIdescE2 = umma_idesc_bf16(128, 128, 0, 0);  // both K-major
 constexpr uint32_t kIdescId = umma_idesc_bf16(128, 16, 0, 0);   // G . I16, both K-major
@@ -416,23 +429,23 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
   const uint32_t sbase = smem_u32(smem);
   const uint32_t pc_tile = sbase + kStages * kStageBytes;
   const uint32_t cbuf = pc_tile + kPcBytes;             // [2] codes tiles [128][128 B], 128-byte swizzle
-  const uint32_t id_tile = cbuf + 2 * kCodesBytes;      // 16 x 16 identity, K-major, 128-byte swizzle
+  const uint32_t id_tile = cbuf + kCBufs * kCodesBytes;  // 16 x 16 identity, K-major, 128-byte swizzle
   const uint32_t xbuf = id_tile + kIdBytes;             // [128][32] fp32 partial P (CLUSTER only)
-  uint64_t* bars = (uint64_t*)(smem + kStages * kStageBytes + kPcBytes + 2 * kCodesBytes + kIdBytes +
+  uint64_t* bars = (uint64_t*)(smem + kStages * kStageBytes + kPcBytes + kCBufs * kCodesBytes + kIdBytes +
                                (CLUSTER ? kXBytes : 0));
   uint64_t* full = bars;                  // [kStages] count 1: converter (stage ready for the MMA)
   uint64_t* empty = bars + kStages;       // [kStages] count 1: MMA commit
   uint64_t* tfull = bars + 2 * kStages;   // [kStages] count 1 + tx: TMA (G and fp32 U)
   uint64_t* p_full = bars + 3 * kStages;  // count 1 (MMA commit)
   uint64_t* pc_full = p_full + 1;         // count 256 (epilogue)
-  uint64_t* w_full = p_full + 2;          // [2] count 1
-  uint64_t* w_empty = p_full + 4;         // [2] count 256
-  uint64_t* cready = p_full + 6;          // [2] count 256: a codes tile is written
-  uint64_t* cfree = p_full + 8;           // [2] count 1: the store of a codes tile has read it
-  uint64_t* xfull = p_full + 10;          // count 256 (S-1): the peers' partials are written (clusters)
-  uint64_t* xempty = p_full + 11;         // count 256 (S-1): the peers have read this CTA's partial
-  uint64_t* stall = p_full + 12;          // count 1, never arrived at (test hook)
-  uint32_t* tmem_slot = (uint32_t*)(p_full + 13);
+  uint64_t* w_full = p_full + 2;          // [kWBufs] count 1
+  uint64_t* w_empty = p_full + 5;         // [kWBufs] count 256
+  uint64_t* cready = p_full + 8;          // [kCBufs] count 256: a codes tile is written
+  uint64_t* cfree = p_full + 11;          // [kCBufs] count 1: the store of a codes tile has read it
+  uint64_t* xfull = p_full + 14;          // count 256 (S-1): the peers' partials are written (clusters)
+  uint64_t* xempty = p_full + 15;         // count 256 (S-1): the peers have read this CTA's partial
+  uint64_t* stall = p_full + 16;          // count 1, never arrived at (test hook)
+  uint32_t* tmem_slot = (uint32_t*)(p_full + 17);
   __shared__ int failed;  // any role gave up (reported at exit)
   __shared__ int nonfin;  // a block maximum was not finite (reported at exit)
 
@@ -452,7 +465,7 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
     mbar_init(p_full, 1);
     mbar_init(pc_full, 256);
     mbar_init(stall, 1);
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < 3; ++b) {
       mbar_init(&w_full[b], 1);
       mbar_init(&w_empty[b], 256);
       mbar_init(&cready[b], 256);
@@ -532,8 +545,8 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
       uint32_t e2 = 0;
       for (Steps<EncParams> st(p, beg, end, q, S); st.valid() && !failed; st.next()) {
         if (st.pass == 0) continue;
-        const int cb = e2 & 1;
-        if (!mbar_wait(&cready[cb], (e2 >> 1) & 1u, kWaitLimit)) {
+        const int cb = (int)(e2 % kCBufs);
+        if (!mbar_wait(&cready[cb], (e2 / kCBufs) & 1u, kWaitLimit)) {
           failed = 1;
           break;
         }
@@ -599,10 +612,10 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
         } else {
           // E2: W/a [128 x 128] = Pc_hi U_hi^T + Pc_lo U_hi^T + Pc_hi U_lo^T + G . I
           // (Pc already divided by a; G . I adds G exactly, 16 columns per MMA)
-          const int b = e2 & 1;
-          if (e2 >= 2 && !mbar_wait(&w_empty[b], ((e2 >> 1) - 1) & 1u, kWaitLimit)) { failed = 1; break; }
+          const int b = (int)(e2 % kWBufs);
+          if (e2 >= kWBufs && !mbar_wait(&w_empty[b], ((e2 / kWBufs) - 1) & 1u, kWaitLimit)) { failed = 1; break; }
           tc_fence_after();
-          const uint32_t d = tbase + (b ? kColW1 : kColW0);
+          const uint32_t d = tbase + w_col(b);
           const int ak[6] = {0, 16, 32, 48, 0, 16};   // Pc: hi = k 0..31, lo = k 32..63
           const int bk[6] = {0, 16, 0, 16, 32, 48};   // U : hi = k 0..31, lo = k 32..63
 #pragma unroll
@@ -696,16 +709,16 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
         mbar_arrive(pc_full);
       }
       const int c = st.chunk();
-      const int b = e2 & 1;
+      const int b = (int)(e2 % kWBufs);
       const int64_t row = (int64_t)panel * kPanel + r;
       const bool live = row < J.d_out;
-      stop = named_sync_or(2, 256, !mbar_wait(&w_full[b], (e2 >> 1) & 1u, kWaitLimit));
+      stop = named_sync_or(2, 256, !mbar_wait(&w_full[b], (e2 / kWBufs) & 1u, kWaitLimit));
       if (stop) {
         failed = 1;
         break;
       }
       tc_fence_after();
-      const uint32_t wcol = tbase + lane_off + (b ? kColW1 : kColW0) + 64 * h;
+      const uint32_t wcol = tbase + lane_off + w_col(b) + 64 * h;
       uint32_t w[64];
       tmem_ld32(wcol, w);
       tmem_ld32(wcol + 32, w + 32);
@@ -749,8 +762,8 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
       }
       // the codes tile is free once the store of its previous use has read it;
       // this barrier also exchanges the halves' maxima
-      const int cb = e2 & 1;
-      const bool freed = e2 < 2 || mbar_wait(&cfree[cb], ((e2 >> 1) - 1) & 1u, kWaitLimit);
+      const int cb = (int)(e2 % kCBufs);
+      const bool freed = e2 < (uint32_t)kCBufs || mbar_wait(&cfree[cb], ((e2 / kCBufs) - 1) & 1u, kWaitLimit);
       stop = named_sync_or(2, 256, !freed);
       if (stop) {
         failed = 1;
@@ -881,12 +894,12 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
   uint64_t* t_full = ostored + 2;          // [2] count 1
   uint64_t* t_empty = t_full + 2;          // [2] count 256
   uint64_t* pc_full = t_full + 4;          // count 256
-  uint64_t* w_full = t_full + 5;           // [2] count 1
-  uint64_t* w_empty = t_full + 7;          // [2] count 256
-  uint64_t* xfull = t_full + 9;            // count 256 (S-1): the peers' partials are written (clusters)
-  uint64_t* xempty = t_full + 10;          // count 256 (S-1): the peers have read this CTA's partial
-  uint64_t* stall = t_full + 11;           // count 1, never arrived at (test hook)
-  uint32_t* tmem_slot = (uint32_t*)(t_full + 12);
+  uint64_t* w_full = t_full + 5;           // [kWBufs] count 1
+  uint64_t* w_empty = t_full + 8;          // [kWBufs] count 256
+  uint64_t* xfull = t_full + 11;           // count 256 (S-1): the peers' partials are written (clusters)
+  uint64_t* xempty = t_full + 12;          // count 256 (S-1): the peers have read this CTA's partial
+  uint64_t* stall = t_full + 13;           // count 1, never arrived at (test hook)
+  uint32_t* tmem_slot = (uint32_t*)(t_full + 14);
   __shared__ int failed;
   __shared__ int nonfin;  // a block scale was not finite (reported at exit)
 
@@ -909,6 +922,8 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
       mbar_init(&ostored[b], 256);
       mbar_init(&t_full[b], 1);
       mbar_init(&t_empty[b], 256);
+    }
+    for (int b = 0; b < 3; ++b) {
       mbar_init(&w_full[b], 1);
       mbar_init(&w_empty[b], 256);
     }
@@ -1107,10 +1122,10 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
           ++d2;
         } else {
           // D3: W[128 x 128] = Pc . U^T (three split products, bf16)
-          const int b = e2 & 1;
-          if (e2 >= 2 && !mbar_wait(&w_empty[b], ((e2 >> 1) - 1) & 1u, kWaitLimit)) { failed = 1; break; }
+          const int b = (int)(e2 % kWBufs);
+          if (e2 >= kWBufs && !mbar_wait(&w_empty[b], ((e2 / kWBufs) - 1) & 1u, kWaitLimit)) { failed = 1; break; }
           tc_fence_after();
-          const uint32_t d = tbase + (b ? kColW1 : kColW0);
+          const uint32_t d = tbase + w_col(b);
           const int ak[6] = {0, 16, 32, 48, 0, 16};
           const int bk[6] = {0, 16, 0, 16, 32, 48};
 #pragma unroll
@@ -1209,8 +1224,8 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
         ++d2;
       } else {
         // D3 epilogue: G_hat = a s q + acc, into scratch tile j once its previous use is stored
-        const int b = e2 & 1;
-        bool ok = mbar_wait(&w_full[b], (e2 >> 1) & 1u, kWaitLimit) &&
+        const int b = (int)(e2 % kWBufs);
+        bool ok = mbar_wait(&w_full[b], (e2 / kWBufs) & 1u, kWaitLimit) &&
                   mbar_wait(&cfull[s], (step / kDStages) & 1u, kWaitLimit);
         if (step >= 2) ok = ok && mbar_wait(&sfree[j], ((step >> 1) - 1) & 1u, kWaitLimit);
         stop = named_sync_or(2, 256, !ok);
@@ -1219,7 +1234,7 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
           break;
         }
         tc_fence_after();
-        const uint32_t wcol = tbase + lane_off + (b ? kColW1 : kColW0) + 64 * h;
+        const uint32_t wcol = tbase + lane_off + w_col(b) + 64 * h;
         const uint32_t c_tile = sbase + s * kDStageBytes;
         const uint32_t o_tile = scr + j * kDScratch;  // two [128][64] bf16 boxes, 128-byte swizzle
         const float as = a * sc;

@@ -73,8 +73,8 @@ def test_dense_factor_matches_oracle(kind, d):
 def test_dense_codec_matches_oracle_given_the_same_transform(kind, d_in, d_out):
     A32, G = _layer(d_in, d_out, 4 * d_in, 600 + d_in)
     A64 = A32.astype(np.float64)
-    M32 = _oracle_M(A64, kind).astype(np.float32)
-    Mi32 = _oracle_M(A64, kind, inverse=True).astype(np.float32)
+    M32 = np.ascontiguousarray(_oracle_M(A64, kind), dtype=np.float32)
+    Mi32 = np.ascontiguousarray(_oracle_M(A64, kind, inverse=True), dtype=np.float32)
     Ms = ops.dense_split(torch.from_numpy(M32).to(DEV))
     Mis = ops.dense_split(torch.from_numpy(Mi32).to(DEV))
     Gd = torch.from_numpy(G).to(DEV).to(torch.bfloat16)
