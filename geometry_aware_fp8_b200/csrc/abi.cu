@@ -441,13 +441,13 @@ gift_status gift_dense_factor(const float* A, int64_t d, int kind, float* M, flo
                                          (cudaStream_t)stream));
 }
 
-gift_status gift_dense_split(const float* M, int64_t d, uint16_t* M_split, gift_stream_t stream) {
-  if (!M || !M_split) return GIFT_ERR_INVALID_ARG;
+gift_status gift_dense_split(const float* M, int64_t d, int parts, uint16_t* M_split, gift_stream_t stream) {
+  if (!M || !M_split || (parts != 2 && parts != 3)) return GIFT_ERR_INVALID_ARG;
   gift_status st = check_dense_d(d);
   if (st != GIFT_OK) return st;
   if (!aligned16(M) || !aligned16(M_split)) return GIFT_ERR_ALIGN;
   if ((st = device_ok()) != GIFT_OK) return st;
-  return cuda_status(launch_dense_split(M, (int)d, M_split, (cudaStream_t)stream));
+  return cuda_status(launch_dense_split(M, (int)d, parts, M_split, (cudaStream_t)stream));
 }
 
 gift_status gift_dense_encode(const void* G, int64_t d_out, int64_t d_in, const uint16_t* M_split,

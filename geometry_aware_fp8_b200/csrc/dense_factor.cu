@@ -4,8 +4,9 @@
 // From A = X^T X / N (d x d, fp32), all arithmetic in fp64:
 //   Cholesky:     A = L L^T,  M = L^{-T},   M^{-1} = L^T       (upper triangular)
 //   full rank:    M = A^{-1/2},             M^{-1} = A^{1/2}   (symmetric)
-// Outputs M and M^{-1} in fp32 and as bf16 hi/lo pairs (the operands of the
-// dense tensor-core codec, dense_tc.cu).
+// Outputs M and M^{-1} in fp32, M as three bf16 parts (hi, mid, lo) and
+// M^{-1} as a bf16 hi/lo pair: the operands of the dense tensor-core codec
+// (dense_tc.cu).
 //
 // Cholesky is blocked by 64: per block column p, one CTA factors the diagonal
 // block and inverts its factor (fp64, shared memory), the blocks below are
@@ -322,13 +323,24 @@ __global__ void __launch_bounds__(kFT) trinv_row_kernel(const double* __restrict
     for (int y = 0; y < 4; ++y) X[(int64_t)(i * kNB + tr + 16 * x) * d + j * kNB + tc + 16 * y] = -out[x][y];
 }
 
-// ---- outputs: fp32 and the bf16 hi/lo pair of a d x d matrix ----
+// bf16 parts of x: parts = 2 (hi, lo) or 3 (hi, mid, lo), each the bf16
+// rounding of what the earlier parts leave; written at split[t * n + i].
+GIFT_DEV void write_bf16_parts(float x, int parts, uint16_t* __restrict__ split, int64_t n, int64_t i) {
+  float rest = x;
+  for (int t = 0; t < parts; ++t) {
+    const __nv_bfloat16 b = __float2bfloat16_rn(rest);
+    split[t * n + i] = __bfloat16_as_ushort(b);
+    rest -= __bfloat162float(b);
+  }
+}
+
+// ---- outputs: fp32 and the bf16 parts of a d x d matrix ----
 // mode 0: out[r][c] = s * S[r][c];  mode 1: out[r][c] = s * S[c][r] for r <= c, else 0
 // (the transpose of a lower-triangular source).  32 x 32 tiles through shared memory.
 __global__ void __launch_bounds__(256) dense_out_kernel(const double* __restrict__ S, int d, int mode,
                                                         const double* __restrict__ scale, int scale_pow,
                                                         float* __restrict__ out, uint16_t* __restrict__ split,
-                                                        uint32_t* err) {
+                                                        int parts, uint32_t* err) {
   __shared__ double T[32][33];
   const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
@@ -349,21 +361,15 @@ __global__ void __launch_bounds__(256) dense_out_kernel(const double* __restrict
     const float f = (float)v;
     bad |= not_finite(f);
     out[(int64_t)r * d + c] = f;
-    const float hi = __bfloat162float(__float2bfloat16_rn(f));
-    split[(int64_t)r * d + c] = __bfloat16_as_ushort(__float2bfloat16_rn(hi));
-    split[(int64_t)d * d + (int64_t)r * d + c] = __bfloat16_as_ushort(__float2bfloat16_rn(f - hi));
+    write_bf16_parts(f, parts, split, (int64_t)d * d, (int64_t)r * d + c);
   }
   report_bits(err, bad, GIFT_DEV_NONFINITE);
 }
 
-// fp32 M -> bf16 hi/lo pair (for a transform made elsewhere)
-__global__ void dense_split_kernel(const float* __restrict__ M, int64_t n, uint16_t* __restrict__ split) {
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
-    const float f = M[i];
-    const float hi = __bfloat162float(__float2bfloat16_rn(f));
-    split[i] = __bfloat16_as_ushort(__float2bfloat16_rn(hi));
-    split[n + i] = __bfloat16_as_ushort(__float2bfloat16_rn(f - hi));
-  }
+// fp32 M -> its bf16 parts (for a transform made elsewhere)
+__global__ void dense_split_kernel(const float* __restrict__ M, int64_t n, int parts, uint16_t* __restrict__ split) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+    write_bf16_parts(M[i], parts, split, n, i);
 }
 
 constexpr int kPartBlocks = 256;
@@ -405,8 +411,8 @@ cudaError_t launch_dense_factor(const float* A, int d, int kind, float* M, float
     }
     for (int i = 0; i < nb; ++i) trinv_row_kernel<<<i + 1, kFT, kBlockSmem, s>>>(A64, X, d, i, Dinv);
     // M = (L^{-1})^T, M^{-1} = L^T
-    dense_out_kernel<<<og, 256, 0, s>>>(X, d, 1, nullptr, 0, M, M_split, err);
-    dense_out_kernel<<<og, 256, 0, s>>>(A64, d, 1, nullptr, 0, M_inv, M_inv_split, err);
+    dense_out_kernel<<<og, 256, 0, s>>>(X, d, 1, nullptr, 0, M, M_split, 3, err);
+    dense_out_kernel<<<og, 256, 0, s>>>(A64, d, 1, nullptr, 0, M_inv, M_inv_split, 2, err);
     return cudaGetLastError();
   }
   double* Y = A64 + n;
@@ -435,13 +441,13 @@ cudaError_t launch_dense_factor(const float* A, int d, int kind, float* M, float
     Z = z;
   }
   // M = Z c^{-1/2} = A^{-1/2},  M^{-1} = Y c^{1/2} = A^{1/2}
-  dense_out_kernel<<<og, 256, 0, s>>>(Z, d, 0, cval, -1, M, M_split, err);
-  dense_out_kernel<<<og, 256, 0, s>>>(Y, d, 0, cval, +1, M_inv, M_inv_split, err);
+  dense_out_kernel<<<og, 256, 0, s>>>(Z, d, 0, cval, -1, M, M_split, 3, err);
+  dense_out_kernel<<<og, 256, 0, s>>>(Y, d, 0, cval, +1, M_inv, M_inv_split, 2, err);
   return cudaGetLastError();
 }
 
-cudaError_t launch_dense_split(const float* M, int d, uint16_t* split, cudaStream_t s) {
-  dense_split_kernel<<<kNumSMs * 8, 256, 0, s>>>(M, (int64_t)d * d, split);
+cudaError_t launch_dense_split(const float* M, int d, int parts, uint16_t* split, cudaStream_t s) {
+  dense_split_kernel<<<kNumSMs * 8, 256, 0, s>>>(M, (int64_t)d * d, parts, split);
   return cudaGetLastError();
 }
 

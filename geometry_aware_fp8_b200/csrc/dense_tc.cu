@@ -10,12 +10,15 @@
 //   decode  G_hat = W_hat M^{-1},  W_hat = value(codes) * scale (per block)
 // with M = L^{-T} (Cholesky) or A^{-1/2} (full rank); dense_factor.cu makes
 // them.  Both products are dense GEMMs, so both kernels are tensor-core
-// bound.  M and M^{-1} arrive as bf16 hi/lo pairs (M ~ M_hi + M_lo, each
-// product exact to ~2^-17; G is exact in bf16), accumulated in fp32 TMEM.
+// bound.  G is exact in bf16.  M arrives as three bf16 parts (M ~ M_hi +
+// M_mid + M_lo, ~2^-24 relative): the entries of a whitening transform are
+// large next to W = G M (the sum cancels), so the encoder needs M to fp32
+// accuracy for its codes; M^{-1} arrives as a hi/lo pair (~2^-17), enough for
+// G_hat.  Accumulation is fp32 in TMEM.
 //
 // Encode: one CTA per 128 x 128 tile of W (one E4M3 block per row), K = d_in
-// streamed in 64-column steps by TMA: G [128][64] (K-major) and M_hi, M_lo
-// [64][128] (MN-major, two 64-column boxes each), 4-stage ring.  Warp 4 issues
+// streamed in 64-column steps by TMA: G [128][64] (K-major) and the three
+// parts of M [64][128] (MN-major, two 64-column boxes each), 3-stage ring.  Warp 4 issues
 // TMA, warp 5 the MMAs (M=128, N=128, K=16), warps 0-3 own one row each: the
 // row's 128 accumulators are its whole block, so the block maximum, the scale
 // and the codes need no exchange.
@@ -39,16 +42,15 @@ constexpr uint32_t kWaitLimit = 1u << 22;
 constexpr uint32_t kIdesc = umma_idesc_bf16(128, 128, 0, 1);  // A K-major, B MN-major
 
 // ---------------------------------------------------------------- encode
-constexpr int kEStages = 4;
+constexpr int kEStages = 3;
 constexpr int kEA = 128 * 64 * 2;        // G box [128 rows][64 k], 16 KB
 constexpr int kEBox = 64 * 64 * 2;       // M box [64 k][64 n], 8 KB
-constexpr int kEStage = kEA + 4 * kEBox; // G + M_hi (2 boxes) + M_lo (2 boxes) = 48 KB
+constexpr int kEStage = kEA + 6 * kEBox; // G + three parts of M (2 boxes each) = 64 KB
 constexpr int kESmem = kEStages * kEStage + 1024 + 256;
 
 struct alignas(64) DenseEnc {
   CUtensorMap tmG;   // bf16 [d_out][d_in], box [128][64]
-  CUtensorMap tmMh;  // bf16 [d_in][d_in], box [64][64]
-  CUtensorMap tmMl;
+  CUtensorMap tmM[3];  // bf16 [d_in][d_in] hi, mid, lo; box [64][64]
   uint8_t* codes;
   float* scales;
   int d_out, d_in, upper;
@@ -98,10 +100,11 @@ __global__ void __launch_bounds__(192, 1) dense_encode_tc_kernel(const __grid_co
         uint8_t* st = smem + s * kEStage;
         mbar_arrive_expect_tx(&full[s], kEStage);
         tma_load_2d(st, &p.tmG, &full[s], k * 64, row0);
-        tma_load_2d(st + kEA, &p.tmMh, &full[s], n0, k * 64);
-        tma_load_2d(st + kEA + kEBox, &p.tmMh, &full[s], n0 + 64, k * 64);
-        tma_load_2d(st + kEA + 2 * kEBox, &p.tmMl, &full[s], n0, k * 64);
-        tma_load_2d(st + kEA + 3 * kEBox, &p.tmMl, &full[s], n0 + 64, k * 64);
+#pragma unroll
+        for (int t = 0; t < 3; ++t) {
+          tma_load_2d(st + kEA + 2 * t * kEBox, &p.tmM[t], &full[s], n0, k * 64);
+          tma_load_2d(st + kEA + (2 * t + 1) * kEBox, &p.tmM[t], &full[s], n0 + 64, k * 64);
+        }
       }
     }
   } else if (warp == 5) {
@@ -114,13 +117,15 @@ __global__ void __launch_bounds__(192, 1) dense_encode_tc_kernel(const __grid_co
           break;
         }
         tc_fence_after();
-        const uint32_t a = sbase + s * kEStage, bh = a + kEA, bl = bh + 2 * kEBox;
+        const uint32_t a = sbase + s * kEStage, b0 = a + kEA;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
           // B: 16 k-rows of 128 B, the two 64-column halves one box apart
           const uint64_t ad = umma_desc_sw128(a + kk * 32, 16, 1024);
-          umma_bf16(tbase, ad, umma_desc_sw128(bh + kk * 2048, kEBox, 1024), kIdesc, (k | kk) ? 1u : 0u);
-          umma_bf16(tbase, ad, umma_desc_sw128(bl + kk * 2048, kEBox, 1024), kIdesc, 1u);
+#pragma unroll
+          for (int t = 0; t < 3; ++t)
+            umma_bf16(tbase, ad, umma_desc_sw128(b0 + 2 * t * kEBox + kk * 2048, kEBox, 1024), kIdesc,
+                      (k | kk | t) ? 1u : 0u);
         }
         umma_commit(&empty[s]);
       }
@@ -405,12 +410,12 @@ unsigned long long g_enc_attr = 0, g_dec_attr = 0;
 cudaError_t launch_dense_encode(const void* G, int d_out, int d_in, const uint16_t* M_split, bool upper,
                                 uint8_t* codes, float* scales, uint32_t* err, cudaStream_t s) {
   static thread_local DenseEnc P;
-  const uint16_t* Mh = M_split;
-  const uint16_t* Ml = M_split + (int64_t)d_in * d_in;
-  if (!make_tmap_2d(&P.tmG, G, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)d_out, (uint64_t)d_in, 128, 64) ||
-      !make_tmap_2d(&P.tmMh, Mh, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)d_in, (uint64_t)d_in, 64, 64) ||
-      !make_tmap_2d(&P.tmMl, Ml, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)d_in, (uint64_t)d_in, 64, 64))
+  if (!make_tmap_2d(&P.tmG, G, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)d_out, (uint64_t)d_in, 128, 64))
     return cudaErrorInvalidValue;
+  for (int t = 0; t < 3; ++t)
+    if (!make_tmap_2d(&P.tmM[t], M_split + (int64_t)t * d_in * d_in, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                      (uint64_t)d_in, (uint64_t)d_in, 64, 64))
+      return cudaErrorInvalidValue;
   P.codes = codes;
   P.scales = scales;
   P.d_out = d_out;

@@ -96,7 +96,7 @@ cudaError_t launch_whitened_error(const void* G, const void* G_hat, gift_dtype d
 size_t dense_factor_ws_bytes(int64_t d, int kind);
 cudaError_t launch_dense_factor(const float* A, int d, int kind, float* M, float* M_inv, uint16_t* M_split,
                                 uint16_t* M_inv_split, void* ws, uint32_t* err, cudaStream_t s);
-cudaError_t launch_dense_split(const float* M, int d, uint16_t* split, cudaStream_t s);
+cudaError_t launch_dense_split(const float* M, int d, int parts, uint16_t* split, cudaStream_t s);
 cudaError_t launch_dense_encode(const void* G, int d_out, int d_in, const uint16_t* M_split, bool upper,
                                 uint8_t* codes, float* scales, uint32_t* err, cudaStream_t s);
 cudaError_t launch_dense_decode(const uint8_t* codes, const float* scales, int d_out, int d_in,

@@ -93,7 +93,7 @@ def lib() -> ctypes.CDLL:
                                       ctypes.c_float, vp, i32, vp, vp]
         L.gift_dense_factor_workspace_size.argtypes = [i64, i32, ctypes.POINTER(sz)]
         L.gift_dense_factor.argtypes = [vp, i64, i32, vp, vp, vp, vp, vp, sz, vp, vp]
-        L.gift_dense_split.argtypes = [vp, i64, vp, vp]
+        L.gift_dense_split.argtypes = [vp, i64, i32, vp, vp]
         L.gift_dense_encode.argtypes = [vp, i64, i64, vp, i32, vp, vp, vp, vp]
         L.gift_dense_decode.argtypes = [vp, vp, i64, i64, vp, i32, vp, i32, vp, vp]
         for name in EXPORTED:
@@ -428,14 +428,15 @@ def dense_factor_workspace_size(d: int, kind: int) -> int:
 
 def dense_factor(A: torch.Tensor, kind: int, ws: Optional[torch.Tensor] = None,
                  dev_status: Optional[torch.Tensor] = None, stream=None):
-    """(M, M_inv, M_split, M_inv_split, dev_status) of gift_dense_factor for A (d x d fp32)."""
+    """(M, M_inv, M_split (3 bf16 parts), M_inv_split (2 parts), dev_status) of
+    gift_dense_factor for A (d x d fp32); the parts are stored as int16."""
     _cuda(A, ws, dev_status)
     d = A.shape[0]
     dev = A.device
     M = torch.empty((d, d), device=dev, dtype=torch.float32)
     Mi = torch.empty_like(M)
-    Ms = torch.empty((2, d, d), device=dev, dtype=torch.int16)
-    Mis = torch.empty_like(Ms)
+    Ms = torch.empty((3, d, d), device=dev, dtype=torch.int16)
+    Mis = torch.empty((2, d, d), device=dev, dtype=torch.int16)
     if ws is None:
         ws = torch.empty((dense_factor_workspace_size(d, kind),), device=dev, dtype=torch.uint8)
     if dev_status is None:
@@ -445,18 +446,19 @@ def dense_factor(A: torch.Tensor, kind: int, ws: Optional[torch.Tensor] = None,
     return M, Mi, Ms, Mis, dev_status
 
 
-def dense_split(M: torch.Tensor, stream=None) -> torch.Tensor:
-    """bf16 pair [hi ; lo] (2 x d x d, stored as int16) of an fp32 d x d transform."""
+def dense_split(M: torch.Tensor, parts: int = 3, stream=None) -> torch.Tensor:
+    """bf16 parts (parts x d x d, stored as int16) of an fp32 d x d transform:
+    3 for the encoder's M, 2 for the decoder's M^{-1}."""
     _cuda(M)
     d = M.shape[0]
-    out = torch.empty((2, d, d), device=M.device, dtype=torch.int16)
-    _check(lib().gift_dense_split(_ptr(M), d, _ptr(out), _stream(stream)), "gift_dense_split")
+    out = torch.empty((parts, d, d), device=M.device, dtype=torch.int16)
+    _check(lib().gift_dense_split(_ptr(M), d, parts, _ptr(out), _stream(stream)), "gift_dense_split")
     return out
 
 
 def dense_encode(G: torch.Tensor, M_split: torch.Tensor, upper: bool = False, codes=None, scales=None,
                  dev_status: Optional[torch.Tensor] = None, stream=None):
-    """(codes, scales) of W = G M (G bf16, M given as its bf16 pair)."""
+    """(codes, scales) of W = G M (G bf16, M given as its three bf16 parts)."""
     _cuda(G, M_split, codes, scales, dev_status)
     if G.dtype != torch.bfloat16:
         raise TypeError("gift_dense_encode takes bf16 gradients")

@@ -369,9 +369,12 @@ gift_status gift_decode_nvfp4(const uint8_t* codes, const uint8_t* block_scales,
  *   GIFT_DENSE_INVSQRT:  M = A^{-1/2}, M_inv = A^{1/2} (coupled Newton-Schulz
  *                        iteration, at most 60 steps; the rank-r construction
  *                        of gift_encode at r = d_in).
- * Outputs (device, d x d, row-major): M, M_inv in fp32; M_split, M_inv_split
- * as bf16 pairs [hi (d x d) ; lo (d x d)] with x ~ hi + lo, the operands of
- * gift_dense_encode / gift_dense_decode.  d % 128 == 0, 128 <= d <= 8192.
+ * Outputs (device, d x d, row-major): M, M_inv in fp32; M_split as three bf16
+ * parts [hi ; mid ; lo] (3 x d x d, x ~ hi + mid + lo, each part the bf16
+ * rounding of what the earlier ones leave) and M_inv_split as a bf16 pair
+ * [hi ; lo] (2 x d x d): the operands of gift_dense_encode / gift_dense_decode.
+ * (The entries of a whitening transform are large next to W = G M, whose sum
+ * cancels, so the encoder takes M to fp32 accuracy; G_hat needs less.)  d % 128 == 0, 128 <= d <= 8192.
  * ws: device scratch of gift_dense_factor_workspace_size bytes, 16-byte
  * aligned.  dev_status (nullable): GIFT_DEV_RANK_DEFICIENT (a non-positive
  * Cholesky pivot, replaced by a tiny one), GIFT_DEV_NONFINITE.
@@ -387,8 +390,9 @@ gift_status gift_dense_factor(const float* A, int64_t d, int kind, float* M, flo
                               uint16_t* M_inv_split, void* ws, size_t ws_bytes, uint32_t* dev_status,
                               gift_stream_t stream);
 
-/* fp32 d x d matrix -> its bf16 pair [hi ; lo] (for a transform made elsewhere). */
-gift_status gift_dense_split(const float* M, int64_t d, uint16_t* M_split, gift_stream_t stream);
+/* fp32 d x d matrix -> its `parts` bf16 parts (2: [hi ; lo], 3: [hi ; mid ;
+ * lo]) as gift_dense_factor writes them, for a transform made elsewhere. */
+gift_status gift_dense_split(const float* M, int64_t d, int parts, uint16_t* M_split, gift_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * E4M3 codec under a dense transform (tensor cores, bf16 gradients):
@@ -396,8 +400,8 @@ gift_status gift_dense_split(const float* M, int64_t d, uint16_t* M_split, gift_
  *           codes = E4M3_RNE_satfinite(W * (448/amax)) as in gift_encode;
  *   decode  G_hat = W_hat M_inv, W_hat = value(codes) * scale per block,
  *           written as out_dt (bf16 by round-to-nearest-even, or fp32).
- * G: d_out x d_in bf16.  M_split / M_inv_split: [hi ; lo] bf16 pairs of
- * d_in x d_in.  upper_triangular != 0 declares M (M_inv) upper triangular
+ * G: d_out x d_in bf16.  M_split: the three bf16 parts [hi ; mid ; lo] of M,
+ * M_inv_split: the bf16 pair [hi ; lo] of M^{-1}, each part d_in x d_in.  upper_triangular != 0 declares M (M_inv) upper triangular
  * (the Cholesky form), so products skip its zero blocks.  d_in % 128 == 0,
  * 128 <= d_in <= 8192, d_out >= 0.  All pointers 16-byte aligned except
  * dev_status (4).  dev_status (nullable): GIFT_DEV_NONFINITE,
