@@ -88,14 +88,10 @@ __global__ void __launch_bounds__(256) euclid_encode_kernel(const T* __restrict_
        base += groups_per_grid) {
     const int64_t b = base + ((threadIdx.x & 31) >> 3);
     const bool act = b < n_blocks;
-    const int64_t e0 = b * kBlock + sub * 16;
+    // lanes past the end load (and discard) the warp's first block: no branch before the shuffles
+    const int64_t e0 = (act ? b : base) * kBlock + sub * 16;
     float v[16];
-    if (act) {
-      Vec16<T>::load(G + e0, v);
-    } else {
-#pragma unroll
-      for (int i = 0; i < 16; ++i) v[i] = 0.0f;
-    }
+    Vec16<T>::load(G + e0, v);
     float m = 0.0f;
 #pragma unroll
     for (int i = 0; i < 16; ++i) m = fmax_nan(m, fabsf(v[i]));
@@ -188,19 +184,19 @@ __global__ void __launch_bounds__(256) euclid_encode_group_kernel(const __grid_c
   int l0 = first < total ? find_layer(pre, g.n, first) : 0, l1 = l0;
   bool bad = false;
   for (int64_t base = wfirst; base < total; base += 2 * G) {
-    const int64_t b0 = base + ((threadIdx.x & 31) >> 3);
+    const bool has0 = base + ((threadIdx.x & 31) >> 3) < total;
+    // lanes past the end work on the warp's first block and discard it: no
+    // branch before the shuffles
+    const int64_t b0 = has0 ? base + ((threadIdx.x & 31) >> 3) : base;
     const int64_t b1 = b0 + G;
-    const bool has0 = b0 < total;
-    const bool has1 = b1 < total;
-    if (has0) l0 = advance_layer(pre, g.n, l0, b0);
+    const bool has1 = has0 && b1 < total;
+    l0 = advance_layer(pre, g.n, l0, b0);
     l1 = has1 ? advance_layer(pre, g.n, l1 > l0 ? l1 : l0, b1) : l0;
-    const int64_t e0 = has0 ? (b0 - pre[l0]) * kBlock + sub * 16 : 0;
+    const int64_t e0 = (b0 - pre[l0]) * kBlock + sub * 16;
     const int64_t e1 = has1 ? (b1 - pre[l1]) * kBlock + sub * 16 : e0;
     float v0[16], v1[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) v0[i] = v1[i] = 0.0f;
-    if (has0) Vec16<T>::load((const T*)g.src[l0] + e0, v0);
-    if (has1) Vec16<T>::load((const T*)g.src[l1] + e1, v1);
+    Vec16<T>::load((const T*)g.src[l0] + e0, v0);
+    Vec16<T>::load((const T*)g.src[l1] + e1, v1);
     float m0 = 0.0f, m1 = 0.0f;
 #pragma unroll
     for (int i = 0; i < 16; ++i) {

@@ -129,8 +129,6 @@ struct SyrkJob {
   int d;
   float* A;
   uint32_t* err;
-  void* Ah = nullptr;  // optional bf16 hi / lo split of A, written beside it
-  void* Al = nullptr;
 };
 // Every job with bf16 X and d % 128 == 0 is computed (token range never split,
 // so a layer's A does not depend on what it is batched with) and gets

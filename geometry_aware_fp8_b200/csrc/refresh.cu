@@ -37,7 +37,6 @@ struct RefLayer {
   const float* A;   // d x d
   __nv_bfloat16* Ah;  // bf16 hi / lo split of A (tensor-core products), or null
   __nv_bfloat16* Al;
-  int split_done;     // the split was written by the tensor-core syrk
   __nv_bfloat16* Qs;  // d x 128 bf16 [Q_hi | Q_lo] operand, or null
   float* buf[3];    // [0] Q (d x m), [1] Y (ns k-slices of d x m), [2] T (d x m)
   double* gram;     // parts x m x m fp64 partial Gram matrices
@@ -179,12 +178,10 @@ __global__ void omega_kernel(const __grid_constant__ RefBatch b) {
   }
 }
 
-// Ah = bf16(A), Al = bf16(A - Ah), elementwise (the tensor-core operands),
-// for the layers whose A did not come from the tensor-core syrk (which writes
-// the split beside A).
+// Ah = bf16(A), Al = bf16(A - Ah), elementwise (the tensor-core operands).
 __global__ void split_a_kernel(const __grid_constant__ RefBatch b) {
   const RefLayer& L = b.L[blockIdx.z];
-  if (!L.Ah || L.split_done) return;
+  if (!L.Ah) return;
   const int64_t n4 = (int64_t)L.d * L.d / 4;
   for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n4; e += (int64_t)gridDim.x * blockDim.x) {
     const float4 a = __ldg(reinterpret_cast<const float4*>(L.A) + e);
@@ -791,10 +788,6 @@ cudaError_t launch_refresh_batch(const RefreshPlan* plans, const RefreshIO* io, 
       const RefreshPlan& p = plans[base + l];
       const RefreshIO& o = io[base + l];
       sj[l] = SyrkJob{o.X, o.xdt, p.N, (int)p.d, o.A_out ? o.A_out : (float*)((char*)o.ws + p.off_A), o.dev_status};
-      if (p.tc_skinny) {
-        sj[l].Ah = (char*)o.ws + p.off_Ah;
-        sj[l].Al = (char*)o.ws + p.off_Al;
-      }
     }
     static thread_local bool batched[kMaxBatch];
     if ((e = launch_syrk_tc_batch(sj, cnt, s, batched)) != cudaSuccess) return e;
@@ -828,7 +821,6 @@ cudaError_t launch_refresh_batch(const RefreshPlan* plans, const RefreshIO* io, 
       L.Vs = L.Lf + 64 * 64 + 64;  // after m*m + m doubles (m <= 64)
       L.Ah = p.tc_skinny ? (__nv_bfloat16*)(w + p.off_Ah) : nullptr;
       L.Al = p.tc_skinny ? (__nv_bfloat16*)(w + p.off_Al) : nullptr;
-      L.split_done = batched[l] && p.tc_skinny ? 1 : 0;
       L.Qs = p.tc_skinny ? (__nv_bfloat16*)(w + p.off_Qs) : nullptr;
       L.U = o.U;
       L.lambda = o.lambda;

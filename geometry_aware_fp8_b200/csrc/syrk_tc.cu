@@ -53,8 +53,6 @@ struct alignas(64) SyrkLayer {
   float* A;         // direct output (splits == 1)
   float* part;      // splits x d x d raw partial sums (splits > 1)
   uint32_t* err;    // optional device status word
-  __nv_bfloat16* Ah;  // optional bf16 hi / lo split of A (splits == 1), written beside A
-  __nv_bfloat16* Al;
 };
 constexpr int kSyrkMaxBatch = 64;
 struct SyrkBatch {
@@ -203,19 +201,8 @@ __global__ void __launch_bounds__(THREADS, 1) syrk_tc_kernel(const __grid_consta
         if (j < i || j >= a.d) continue;
         const float v = sum[t];
         if (p.splits == 1) {
-          const float av = v * a.scale;
-          a.A[(int64_t)i * a.d + j] = av;
-          if (j != i) a.A[(int64_t)j * a.d + i] = av;
-          if (a.Ah) {  // the tensor-core operands of the subspace products
-            const __nv_bfloat16 h = __float2bfloat16_rn(av);
-            const __nv_bfloat16 l = __float2bfloat16_rn(av - __bfloat162float(h));
-            a.Ah[(int64_t)i * a.d + j] = h;
-            a.Al[(int64_t)i * a.d + j] = l;
-            if (j != i) {
-              a.Ah[(int64_t)j * a.d + i] = h;
-              a.Al[(int64_t)j * a.d + i] = l;
-            }
-          }
+          a.A[(int64_t)i * a.d + j] = v * a.scale;
+          if (j != i) a.A[(int64_t)j * a.d + i] = v * a.scale;
         } else {
           a.part[(int64_t)split * a.d * a.d + (int64_t)i * a.d + j] = v;
         }
@@ -259,7 +246,6 @@ cudaError_t launch_syrk_tc(const void* X, gift_dtype xdt, int64_t N, int d, floa
   a.A = A;
   a.part = part;
   a.err = err;
-  a.Ah = a.Al = nullptr;
   const int items = syrk_tc_tiles(d) * P.splits;
   syrk_tc_kernel<<<items, THREADS, SMEM_BYTES, s>>>(P);
   e = cudaGetLastError();
@@ -288,8 +274,6 @@ cudaError_t launch_syrk_tc_batch(const SyrkJob* jobs, int n, cudaStream_t s, boo
     a.A = J.A;
     a.part = nullptr;
     a.err = J.err;
-    a.Ah = (__nv_bfloat16*)J.Ah;
-    a.Al = (__nv_bfloat16*)J.Al;
     tiles += syrk_tc_tiles(J.d);
     used[l] = true;
     ++m;

@@ -7,10 +7,12 @@ Criteria:
     within 1e-5 of the oracle's in relative Frobenius norm; the sum of M's
     three bf16 parts within 2^-24 of M per element, of M^{-1}'s two parts
     within 2^-16 (relative to the largest entry);
-  * codec, given the same fp32 M: codes, scales and G_hat under the criteria
-    of _cmp.py (codes exact on >= 99.9 % and one step apart elsewhere, scales
-    within 1e-3, G_hat within 1e-3 of the row maximum with the decoder fed
-    the oracle's codes);
+  * codec, given the same fp32 M: codes and scales within the bound that the
+    fp32 evaluation of W = G M allows (_cmp.check_codes_within_bound: the
+    entries of a whitening transform are large next to W, whose sum cancels,
+    so the rank-32 codec's 99.9 % exact-code criterion does not transfer),
+    at least 99 % of codes exact; G_hat within 1e-3 of the row maximum with
+    the decoder fed the oracle's codes (the criterion of _cmp.check_rows);
   * round trip on the GPU's own factor: the relative Frobenius error within
     1 % of the oracle's.
 """
@@ -21,7 +23,7 @@ import torch
 from oracle import gift_oracle as O
 from geometry_aware_fp8_b200 import ops, synth
 
-from _cmp import check_codes, check_rows, check_scales
+from _cmp import check_codes_within_bound, check_rows
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
@@ -63,7 +65,7 @@ def test_dense_factor_matches_oracle(kind, d):
     print(f"{kind} d={d}: M rel err {e:.2e}, M_inv rel err {ei:.2e}")
     assert e <= 1e-5 and ei <= 1e-5
     for full, parts, tol in ((M, Ms, 2.0 ** -24), (Mi, Mis, 2.0 ** -16)):
-        pv = parts.view(torch.bfloat16).cpu().numpy().astype(np.float64)
+        pv = parts.view(torch.bfloat16).float().cpu().numpy().astype(np.float64)
         back = pv.sum(axis=0)
         f = full.cpu().numpy().astype(np.float64)
         assert np.max(np.abs(back - f)) <= tol * np.max(np.abs(f))
@@ -82,12 +84,14 @@ def test_dense_codec_matches_oracle_given_the_same_transform(kind, d_in, d_out):
     upper = kind == "cholesky"
     st = torch.zeros((1,), device=DEV, dtype=torch.int32)
     codes, scales = ops.dense_encode(Gd, Ms, upper, dev_status=st)
-    c_o, s_o = O.encode_dense(G, M32.astype(np.float64))
-    rate = check_codes(codes.cpu().numpy(), c_o)
-    check_scales(scales.cpu().numpy(), s_o)
-    if upper:  # the full K loop over the zero blocks gives the same codes
+    G64, M64 = G.astype(np.float64), M32.astype(np.float64)
+    c_o, s_o = O.encode_dense(G64, M64)
+    W = G64 @ M64
+    E = (d_in + 1) * 2.0 ** -24 * (np.abs(G64) @ np.abs(M64))
+    rate = check_codes_within_bound(codes.cpu().numpy(), scales.cpu().numpy(), W, E, want_codes=c_o)
+    if upper:  # the full K loop over the zero blocks meets the same bound
         c2, s2 = ops.dense_encode(Gd, Ms, False)
-        check_codes(c2.cpu().numpy(), c_o)
+        check_codes_within_bound(c2.cpu().numpy(), s2.cpu().numpy(), W, E, want_codes=c_o)
     want = O.decode_dense(c_o, s_o, Mi32.astype(np.float64))
     cd, sd = torch.from_numpy(c_o).to(DEV), torch.from_numpy(s_o).to(DEV)
     for dt in (torch.bfloat16, torch.float32):
