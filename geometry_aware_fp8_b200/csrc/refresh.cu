@@ -293,10 +293,11 @@ __global__ void fold_slices_kernel(const __grid_constant__ RefBatch b, int which
   }
 }
 
-// part[p] = Ya[rows of p]^T Yb[rows of p] (m x m, fp64), 64 rows per part
-// staged in shared memory; thread (ti, tj) of a 16 x 16 grid owns the 4 x 4
-// block of entries (4 ti.., 4 tj..).
-constexpr int kGramRows = 64;
+// part[p] = Ya[rows of p]^T Yb[rows of p] (m x m, fp64), 256 rows per part
+// staged in shared memory 64 rows at a time; thread (ti, tj) of a 16 x 16 grid
+// owns the 4 x 4 block of entries (4 ti.., 4 tj..).  Parts of 256 rows keep
+// the partials few (d / 256), so the one-CTA consumers sum little.
+constexpr int kGramRows = 256;
 
 __global__ void __launch_bounds__(kRT) gram_partial_kernel(const __grid_constant__ RefBatch bt, int wa, int wb) {
   const RefLayer& Lr = bt.L[blockIdx.z];
@@ -308,31 +309,33 @@ __global__ void __launch_bounds__(kRT) gram_partial_kernel(const __grid_constant
   __shared__ __align__(16) float Sa[64][64];
   __shared__ __align__(16) float Sb[64][64];
   const int p = blockIdx.x;
-  const int r0 = p * kGramRows;
-  const int rows = min(kGramRows, d - r0);
   const int ti = threadIdx.x >> 4, tj = threadIdx.x & 15;
-  for (int e = threadIdx.x; e < 64 * 64; e += kRT) {
-    const int rr = e >> 6, c = e & 63;
-    const bool in = rr < rows && c < m;
-    Sa[rr][c] = in ? Ya[(int64_t)(r0 + rr) * m + c] : 0.0f;
-    Sb[rr][c] = in ? Yb[(int64_t)(r0 + rr) * m + c] : 0.0f;
-  }
-  __syncthreads();
   double acc[4][4];
 #pragma unroll
   for (int a = 0; a < 4; ++a)
 #pragma unroll
     for (int b = 0; b < 4; ++b) acc[a][b] = 0.0;
+  for (int r0 = p * kGramRows; r0 < min(d, (p + 1) * kGramRows); r0 += 64) {
+    const int rows = min(64, d - r0);
+    __syncthreads();
+    for (int e = threadIdx.x; e < 64 * 64; e += kRT) {
+      const int rr = e >> 6, c = e & 63;
+      const bool in = rr < rows && c < m;
+      Sa[rr][c] = in ? Ya[(int64_t)(r0 + rr) * m + c] : 0.0f;
+      Sb[rr][c] = in ? Yb[(int64_t)(r0 + rr) * m + c] : 0.0f;
+    }
+    __syncthreads();
 #pragma unroll 4
-  for (int rr = 0; rr < 64; ++rr) {
-    const float4 va = *reinterpret_cast<const float4*>(&Sa[rr][ti * 4]);
-    const float4 vb = *reinterpret_cast<const float4*>(&Sb[rr][tj * 4]);
-    const double a4[4] = {va.x, va.y, va.z, va.w};
-    const double b4[4] = {vb.x, vb.y, vb.z, vb.w};
+    for (int rr = 0; rr < 64; ++rr) {
+      const float4 va = *reinterpret_cast<const float4*>(&Sa[rr][ti * 4]);
+      const float4 vb = *reinterpret_cast<const float4*>(&Sb[rr][tj * 4]);
+      const double a4[4] = {va.x, va.y, va.z, va.w};
+      const double b4[4] = {vb.x, vb.y, vb.z, vb.w};
 #pragma unroll
-    for (int a = 0; a < 4; ++a)
+      for (int a = 0; a < 4; ++a)
 #pragma unroll
-      for (int b = 0; b < 4; ++b) acc[a][b] = fma(a4[a], b4[b], acc[a][b]);
+        for (int b = 0; b < 4; ++b) acc[a][b] = fma(a4[a], b4[b], acc[a][b]);
+    }
   }
   const int mm = m * m;
 #pragma unroll
@@ -548,6 +551,26 @@ __global__ void __launch_bounds__(kST) rr_kernel(const __grid_constant__ RefBatc
   const int mp = m + (m & 1);  // even count for the round-robin tournament
   const int npairs = mp / 2;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // the tournament's pairs, round by round (p < q; q == m marks the dummy
+  // partner of an odd m), and this thread's fixed work items: 2 x 2 block
+  // (ba, bb) of B and up to two (row k, pair b) items of V
+  __shared__ unsigned char tab_p[63][32], tab_q[63][32];
+  for (int e = threadIdx.x; e < (mp - 1) * npairs; e += kST) {
+    const int round = e / npairs, a = e % npairs;
+    auto pos = [&](int k) { return k == 0 ? 0 : 1 + (k - 1 + round) % (mp - 1); };
+    int p = pos(a), q = pos(mp - 1 - a);
+    if (p > q) {
+      const int t = p;
+      p = q;
+      q = t;
+    }
+    tab_p[round][a] = (unsigned char)p;
+    tab_q[round][a] = (unsigned char)q;
+  }
+  const int nb = npairs * npairs, nv = m * npairs;
+  const int ba = threadIdx.x / npairs, bb = threadIdx.x % npairs;
+  const int v0 = threadIdx.x, v1 = threadIdx.x + kST;
+  const int vk0 = v0 / npairs, vb0 = v0 % npairs, vk1 = v1 / npairs, vb1 = v1 % npairs;
   for (int sweep = 0; sweep < kJacobiMaxSweeps; ++sweep) {
     // convergence: off(B)^2 <= tol^2 ||B||_F^2
     double off = 0.0, tot = 0.0;
@@ -580,13 +603,7 @@ __global__ void __launch_bounds__(kST) rr_kernel(const __grid_constant__ RefBatc
     for (int round = 0; round < mp - 1; ++round) {
       if (threadIdx.x < npairs) {
         const int a = threadIdx.x;
-        auto pos = [&](int k) { return k == 0 ? 0 : 1 + (k - 1 + round) % (mp - 1); };
-        int p = pos(a), q = pos(mp - 1 - a);
-        if (p > q) {
-          const int t = p;
-          p = q;
-          q = t;
-        }
+        const int p = tab_p[round][a], q = tab_q[round][a];
         double c = 1.0, s = 0.0;
         if (q < m) {
           const double bpq = B[p * ld + q];
@@ -602,41 +619,42 @@ __global__ void __launch_bounds__(kST) rr_kernel(const __grid_constant__ RefBatc
           }
         }
         pp[a] = p;
-        pq[a] = q;  // q == m marks the dummy partner of an odd m
+        pq[a] = q;
         pc[a] = c;
         ps[a] = s;
       }
       __syncthreads();
       // new row/column p = c p - s q, q = s p + c q
-      const int nb = npairs * npairs;
-      for (int w = threadIdx.x; w < nb + m * npairs; w += kST) {
-        if (w < nb) {
-          const int a = w / npairs, b = w % npairs;
-          const int pa = pp[a], qa = pq[a], pb = pp[b], qb = pq[b];
-          const double ca = pc[a], sa = ps[a], cb = pc[b], sb = ps[b];
-          const bool ha = qa < m, hb = qb < m;
-          const double b00 = B[pa * ld + pb];
-          const double b01 = hb ? B[pa * ld + qb] : 0.0;
-          const double b10 = ha ? B[qa * ld + pb] : 0.0;
-          const double b11 = (ha && hb) ? B[qa * ld + qb] : 0.0;
-          const double r00 = ca * b00 - sa * b10, r01 = ca * b01 - sa * b11;
-          const double r10 = sa * b00 + ca * b10, r11 = sa * b01 + ca * b11;
-          Bn[pa * ld + pb] = cb * r00 - sb * r01;
-          if (hb) Bn[pa * ld + qb] = sb * r00 + cb * r01;
-          if (ha) Bn[qa * ld + pb] = cb * r10 - sb * r11;
-          if (ha && hb) Bn[qa * ld + qb] = sb * r10 + cb * r11;
+      if (threadIdx.x < nb) {
+        const int a = ba, b = bb;
+        const int pa = pp[a], qa = pq[a], pb = pp[b], qb = pq[b];
+        const double ca = pc[a], sa = ps[a], cb = pc[b], sb = ps[b];
+        const bool ha = qa < m, hb = qb < m;
+        const double b00 = B[pa * ld + pb];
+        const double b01 = hb ? B[pa * ld + qb] : 0.0;
+        const double b10 = ha ? B[qa * ld + pb] : 0.0;
+        const double b11 = (ha && hb) ? B[qa * ld + qb] : 0.0;
+        const double r00 = ca * b00 - sa * b10, r01 = ca * b01 - sa * b11;
+        const double r10 = sa * b00 + ca * b10, r11 = sa * b01 + ca * b11;
+        Bn[pa * ld + pb] = cb * r00 - sb * r01;
+        if (hb) Bn[pa * ld + qb] = sb * r00 + cb * r01;
+        if (ha) Bn[qa * ld + pb] = cb * r10 - sb * r11;
+        if (ha && hb) Bn[qa * ld + qb] = sb * r10 + cb * r11;
+      }
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int w = u ? v1 : v0;
+        if (w >= nv) continue;
+        const int k = u ? vk1 : vk0, b = u ? vb1 : vb0;
+        const int pb = pp[b], qb = pq[b];
+        const double cb = pc[b], sb = ps[b];
+        const double vp = V[k * ld + pb];
+        if (qb < m) {
+          const double vq = V[k * ld + qb];
+          Vn[k * ld + pb] = cb * vp - sb * vq;
+          Vn[k * ld + qb] = sb * vp + cb * vq;
         } else {
-          const int k = (w - nb) / npairs, b = (w - nb) % npairs;
-          const int pb = pp[b], qb = pq[b];
-          const double cb = pc[b], sb = ps[b];
-          const double v0 = V[k * ld + pb];
-          if (qb < m) {
-            const double v1 = V[k * ld + qb];
-            Vn[k * ld + pb] = cb * v0 - sb * v1;
-            Vn[k * ld + qb] = sb * v0 + cb * v1;
-          } else {
-            Vn[k * ld + pb] = v0;
-          }
+          Vn[k * ld + pb] = vp;
         }
       }
       __syncthreads();
