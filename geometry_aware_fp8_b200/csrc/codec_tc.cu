@@ -59,39 +59,19 @@ constexpr int kPcBytes = kPanel * 128;         // 16 KB: [128 rows][64 bf16]
 constexpr int kCodesBytes = kPanel * kChunk;    // 16 KB: codes of one chunk
 constexpr int kIdBytes = 16 * 128;             // 2 KB: 16 x 16 bf16 identity, 128-byte rows
 constexpr int kXBytes = kPanel * 32 * 4;        // 16 KB: fp32 partial projections exchanged in a cluster
-#ifndef GIFT_W_BUFS
-#define GIFT_W_BUFS 2
-#endif
-#ifndef GIFT_C_BUFS
-#define GIFT_C_BUFS 2
-#endif
-// TMEM accumulators of W for the second pass (2 or 3; the third sits at
-// columns 384..511, after P (encoder) or the decoder's T buffers) and codes
-// tiles of the encoder (2 or 3).
-constexpr int kWBufs = GIFT_W_BUFS, kCBufs = GIFT_C_BUFS;
-static_assert(kWBufs == 2 || kWBufs == 3, "W buffers");
-static_assert(kCBufs == 2 || kCBufs == 3, "codes tiles");
+// TMEM accumulators of W for the second pass (columns 0..255) and codes
+// tiles of the encoder.  A third of either measured no faster on B200.
+constexpr int kWBufs = 2, kCBufs = 2;
 constexpr int kSmemBytes = kStages * kStageBytes + kPcBytes + kCBufs * kCodesBytes + kIdBytes + 1024 + 512;
 constexpr int enc_smem(bool cluster) { return kSmemBytes + (cluster ? kXBytes : 0); }
 constexpr int kThreads = 480;  // 8 epilogue + 4 converter + MMA + TMA load + TMA store warps
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColW0 = 0, kColW1 = 128, kColP = 256;
-GIFT_DEV uint32_t w_col(int b) { return b == 0 ? 0u : b == 1 ? 128u : 384u; }
+constexpr uint32_t kColP = 256;
+GIFT_DEV uint32_t w_col(int b) { return 128u * (uint32_t)b; }
 constexpr uint32_t kIdescE1 = umma_idesc_bf16(128, 64, 0, 1);   // A K-major, B MN-major
 constexpr uint32_t kIdescE2 = umma_idesc_bf16(128, 128, 0, 0);  // both K-major
 constexpr uint32_t kIdescId = umma_idesc_bf16(128, 16, 0, 0);   // G . I16, both K-major
 constexpr uint32_t kWaitLimit = 1u << 22;
-#ifndef GIFT_ENC_PREFETCH
-#define GIFT_ENC_PREFETCH 0
-#endif
-#ifndef GIFT_DEC_PREFETCH
-#define GIFT_DEC_PREFETCH 0
-#endif
-#ifndef GIFT_PF_PASS2
-#define GIFT_PF_PASS2 1
-#endif
-constexpr int kEncPrefetch = GIFT_ENC_PREFETCH;  // steps of G the producer prefetches into L2 ahead of its loads
-constexpr int kDecPrefetch = GIFT_DEC_PREFETCH;
 constexpr int kMaxJobs = 48;
 constexpr int kMaxPanels = 1536;
 
@@ -151,13 +131,6 @@ GIFT_DEV void tma_store_2d_hint(const void* tmap, uint32_t src, int x, int y, ui
       " [%0, {%2, %3}], [%1], %4;" ::"l"(tmap),
       "r"(src), "r"(x), "r"(y), "l"(policy)
       : "memory");
-}
-// 2-D tiled TMA prefetch global -> L2 (no shared-memory destination, no
-// completion to wait for): brings a box the ring will load later into L2.
-GIFT_DEV void tma_prefetch_2d(const void* tmap, int x, int y, uint64_t policy) {
-  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile.L2::cache_hint [%0, {%1, %2}], %3;" ::"l"(tmap),
-               "r"(x), "r"(y), "l"(policy)
-               : "memory");
 }
 GIFT_DEV void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Wait until at most N committed store groups still read shared memory.
@@ -392,35 +365,6 @@ GIFT_DEV void u_row_from_tile(uint32_t tile, int t, float (&u)[32]) {
     u[4 * q + 3] = __uint_as_float(v.w);
   }
 }
-GIFT_DEV void u_row_from_global(const float* U, int64_t row, float (&u)[32]) {
-  const float4* p = reinterpret_cast<const float4*>(U + row * 32);
-#pragma unroll
-  for (int q = 0; q < 8; ++q) {
-    const float4 v = __ldg(p + q);
-    u[4 * q] = v.x;
-    u[4 * q + 1] = v.y;
-    u[4 * q + 2] = v.z;
-    u[4 * q + 3] = v.w;
-  }
-}
-#ifndef GIFT_U_LSU
-#define GIFT_U_LSU 0
-#endif
-// U rows reach the converters by TMA with the stage (0) or by 16-byte loads
-// from global memory (1), which keeps them off the TMA path.
-constexpr bool kULsu = GIFT_U_LSU != 0;
-#ifndef GIFT_OUT_LSU
-#define GIFT_OUT_LSU 0
-#endif
-// Output tiles (encoder codes, decoder G_hat) leave by TMA stores (0) or by
-// coalesced 16-byte stores of the epilogue threads (1).
-constexpr bool kOutLsu = GIFT_OUT_LSU != 0;
-
-GIFT_DEV void st_global_v4_cs(void* p, uint4 v) {
-  asm volatile("st.global.cs.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
-               : "memory");
-}
-
 template <int FMT, bool CLUSTER>
 __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __grid_constant__ EncParams p,
                                                                      uint32_t* err) {
@@ -509,15 +453,6 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
     if (lane == 0) {
       const uint64_t keep = policy_evict_last(), drop = policy_evict_first();
       uint32_t step = 0;
-      Steps<EncParams> ahead(p, beg, end, q, S);
-      auto prefetch = [&](const Steps<EncParams>& a) {
-        if (a.pass == 0 || GIFT_PF_PASS2) {
-          const EncJob& J = p.jobs[a.job()];
-          tma_prefetch_2d(&J.tmG, a.chunk() * kChunk, a.panel() * kPanel, a.pass == 0 ? keep : drop);
-          tma_prefetch_2d(&J.tmG, a.chunk() * kChunk + 64, a.panel() * kPanel, a.pass == 0 ? keep : drop);
-        }
-      };
-      for (int i = 0; i < kEncPrefetch && ahead.valid(); ++i, ahead.next()) prefetch(ahead);
       for (Steps<EncParams> st(p, beg, end, q, S); st.valid() && !failed; st.next(), ++step) {
         const int s = step % kStages;
         const uint32_t use = step / kStages;
@@ -525,17 +460,13 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
           failed = 1;
           break;
         }
-        if (kEncPrefetch > 0 && ahead.valid()) {
-          prefetch(ahead);
-          ahead.next();
-        }
         const EncJob& J = p.jobs[st.job()];
         const uint64_t pol = st.pass == 0 ? keep : drop;
         const uint32_t dst = sbase + s * kStageBytes;
-        mbar_arrive_expect_tx(&tfull[s], kULsu ? kGBytes : kGBytes + kUBytes);
+        mbar_arrive_expect_tx(&tfull[s], kGBytes + kUBytes);
         tma_load_2d_hint(dst, &J.tmG, &tfull[s], st.chunk() * kChunk, st.panel() * kPanel, pol);
         tma_load_2d_hint(dst + kGHalf, &J.tmG, &tfull[s], st.chunk() * kChunk + 64, st.panel() * kPanel, pol);
-        if (!kULsu) tma_load_2d_hint(dst + kGBytes, &J.tmU, &tfull[s], 0, st.chunk() * kChunk, keep);
+        tma_load_2d_hint(dst + kGBytes, &J.tmU, &tfull[s], 0, st.chunk() * kChunk, keep);
       }
     }
   } else if (warp == 14) {
@@ -551,7 +482,7 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
           break;
         }
         const EncJob& J = p.jobs[st.job()];
-        if (FMT == kFmtE4M3 && !kOutLsu) {  // otherwise the epilogue has stored the tile
+        if (FMT == kFmtE4M3) {  // NVFP4 codes were stored by the epilogue
           tma_store_2d_hint(&J.tmC, cbuf + cb * kCodesBytes, st.chunk() * kChunk, st.panel() * kPanel, drop);
           bulk_commit();
           bulk_wait_read<0>();
@@ -571,14 +502,13 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
       const int s = step % kStages;
       const uint32_t use = step / kStages;
       float u[32];
-      if (kULsu) u_row_from_global(p.jobs[st.job()].U, (int64_t)st.chunk() * kChunk + t, u);  // before the wait
       const bool ok = mbar_wait(&tfull[s], use & 1u, kWaitLimit);
       if (named_sync_or(1, 128, !ok)) {
         failed = 1;
         break;
       }
       const uint32_t u_tile = sbase + s * kStageBytes + kGBytes;
-      if (!kULsu) u_row_from_tile(u_tile, t, u);
+      u_row_from_tile(u_tile, t, u);
       store_u_split_bf16(u_tile, t, u);
       fence_async_shared();
       named_sync(1, 128);
@@ -788,20 +718,7 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
 #pragma unroll
       for (int q = 0; q < 4; ++q)
         st_shared_v4(c_tile + sw128(r, 4 * h + q), cw[4 * q], cw[4 * q + 1], cw[4 * q + 2], cw[4 * q + 3]);
-      if (kOutLsu && FMT == kFmtE4M3) {
-        // the tile's 1024 16-byte chunks, two rows of 128 B per warp instruction
-        named_sync(2, 256);
-        const int tid = threadIdx.x;  // 0..255
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int e = i * 256 + tid, rr = e >> 3, cq = e & 7;
-          const int64_t grow = (int64_t)panel * kPanel + rr;
-          const uint4 v = ld_shared_v4(c_tile + sw128(rr, cq));
-          if (grow < J.d_out) st_global_v4_cs(J.codes + grow * J.d_in + c * kChunk + cq * 16, v);
-        }
-      } else {
-        fence_async_shared();
-      }
+      fence_async_shared();
       mbar_arrive(&cready[cb]);
       ++e2;
     }
@@ -855,7 +772,6 @@ struct alignas(64) DecJob {
   const uint8_t* codes;   // NVFP4 [d_out][d_in/2] (read directly; E4M3 codes arrive by TMA)
   const uint8_t* sb;      // NVFP4 E4M3 block scales [d_out][d_in/16]
   const float* tscale;    // NVFP4 tensor scale
-  void* G_hat;            // bf16 [d_out][d_in] (stores by the epilogue; TMA stores use tmO)
   int d_out, d_in, rank, fmt;
 };
 
@@ -890,8 +806,7 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
   uint64_t* empty = bars + 2 * kDStages;   // [kDStages] count 1: MMA commit (D2) or store warp (D3)
   uint64_t* sfree = bars + 3 * kDStages;   // [2] count 1: scratch tile free (MMA commit or store read)
   uint64_t* oready = sfree + 2;            // [2] count 256: output tile written
-  uint64_t* ostored = oready + 2;          // [2] count 256: output tile copied out by the epilogue
-  uint64_t* t_full = ostored + 2;          // [2] count 1
+  uint64_t* t_full = oready + 2;           // [2] count 1
   uint64_t* t_empty = t_full + 2;          // [2] count 256
   uint64_t* pc_full = t_full + 4;          // count 256
   uint64_t* w_full = t_full + 5;           // [kWBufs] count 1
@@ -919,7 +834,6 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sfree[b], 1);
       mbar_init(&oready[b], 256);
-      mbar_init(&ostored[b], 256);
       mbar_init(&t_full[b], 1);
       mbar_init(&t_empty[b], 256);
     }
@@ -954,12 +868,6 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
     if (lane == 0) {
       const uint64_t keep = policy_evict_last(), drop = policy_evict_first();
       uint32_t step = 0;
-      Steps<DecParams> ahead(p, beg, end, q, S);
-      auto prefetch = [&](const Steps<DecParams>& a) {
-        if (FMT == kFmtE4M3 && (a.pass == 0 || GIFT_PF_PASS2))
-          tma_prefetch_2d(&p.jobs[a.job()].tmC, a.chunk() * kChunk, a.panel() * kPanel, a.pass == 0 ? keep : drop);
-      };
-      for (int i = 0; i < kDecPrefetch && ahead.valid(); ++i, ahead.next()) prefetch(ahead);
       for (Steps<DecParams> st(p, beg, end, q, S); st.valid() && !failed; st.next(), ++step) {
         const int s = step % kDStages;
         const uint32_t use = step / kDStages;
@@ -967,13 +875,9 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
           failed = 1;
           break;
         }
-        if (kDecPrefetch > 0 && ahead.valid()) {
-          prefetch(ahead);
-          ahead.next();
-        }
         const DecJob& J = p.jobs[st.job()];
         const uint32_t dst = sbase + s * kDStageBytes;
-        const uint32_t ub = kULsu ? 0u : (uint32_t)kUBytes;
+        const uint32_t ub = (uint32_t)kUBytes;
         if (FMT == kFmtE4M3) {
           mbar_arrive_expect_tx(&cfull[s], kDCodes + ub);
           tma_load_2d_hint(dst, &J.tmC, &cfull[s], st.chunk() * kChunk, st.panel() * kPanel,
@@ -981,7 +885,7 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
         } else {
           mbar_arrive_expect_tx(&cfull[s], ub);  // NVFP4 codes are read from global memory
         }
-        if (!kULsu) tma_load_2d_hint(dst + kDCodes, &J.tmU, &cfull[s], 0, st.chunk() * kChunk, keep);
+        tma_load_2d_hint(dst + kDCodes, &J.tmU, &cfull[s], 0, st.chunk() * kChunk, keep);
       }
     }
   } else if (warp == 14) {
@@ -1000,20 +904,12 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
           break;
         }
         mbar_arrive(&empty[s]);
-        if (kOutLsu) {
-          // the epilogue copies the tile out itself; the tile is free once it has
-          if (!mbar_wait(&ostored[j], (par >> j) & 1u, kWaitLimit)) {
-            failed = 1;
-            break;
-          }
-        } else {
-          const DecJob& J = p.jobs[st.job()];
-          const uint32_t o_tile = scr + j * kDScratch;
-          tma_store_2d_hint(&J.tmO, o_tile, st.chunk() * kChunk, st.panel() * kPanel, drop);
-          tma_store_2d_hint(&J.tmO, o_tile + kGHalf, st.chunk() * kChunk + 64, st.panel() * kPanel, drop);
-          bulk_commit();
-          bulk_wait_read<0>();
-        }
+        const DecJob& J = p.jobs[st.job()];
+        const uint32_t o_tile = scr + j * kDScratch;
+        tma_store_2d_hint(&J.tmO, o_tile, st.chunk() * kChunk, st.panel() * kPanel, drop);
+        tma_store_2d_hint(&J.tmO, o_tile + kGHalf, st.chunk() * kChunk + 64, st.panel() * kPanel, drop);
+        bulk_commit();
+        bulk_wait_read<0>();
         par ^= 1u << j;
         mbar_arrive(&sfree[j]);
       }
@@ -1027,7 +923,6 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
       const int s = step % kDStages, j = step & 1;
       const uint32_t use = step / kDStages;
       float u[32];
-      if (kULsu) u_row_from_global(p.jobs[st.job()].U, (int64_t)st.chunk() * kChunk + t, u);  // before the wait
       bool ok = mbar_wait(&cfull[s], use & 1u, kWaitLimit);
       if (st.pass == 0 && step >= 2) ok = ok && mbar_wait(&sfree[j], ((step >> 1) - 1) & 1u, kWaitLimit);
       if (named_sync_or(1, 128, !ok)) {
@@ -1038,7 +933,7 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
       const uint32_t u_tile = c_tile + kDCodes;
       const uint32_t q_tile = scr + j * kDScratch;
       // D2 multiplies f16 codes by an f16 split of U, D3 the bf16 P' o c' by a bf16 split
-      if (!kULsu) u_row_from_tile(u_tile, t, u);
+      u_row_from_tile(u_tile, t, u);
       if (st.pass == 0)
         store_u_split_f16(u_tile, t, u);
       else
@@ -1286,20 +1181,6 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
         mbar_arrive(&w_empty[b]);
         fence_async_shared();
         mbar_arrive(&oready[j]);
-        if (kOutLsu) {
-          // the tile's 2048 16-byte chunks, two rows of 256 B per warp instruction
-          named_sync(2, 256);
-          const int tid = threadIdx.x;  // 0..255
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int e = i * 256 + tid, rr = e >> 4, cq = e & 15;
-            const int64_t grow = (int64_t)st.panel() * kPanel + rr;
-            const uint4 v = ld_shared_v4(o_tile + (cq >> 3) * kGHalf + sw128(rr, cq & 7));
-            if (grow < J.d_out)
-              st_global_v4_cs(reinterpret_cast<__nv_bfloat16*>(J.G_hat) + grow * J.d_in + c * kChunk + cq * 8, v);
-          }
-          mbar_arrive(&ostored[j]);
-        }
         ++e2;
       }
     }
@@ -1477,12 +1358,6 @@ int schedule(const TcLayer* layers, int n, uint16_t* off, uint16_t* ids, int max
 // faster by that estimate; a launch of many panels keeps single CTAs.
 constexpr int kSplitCost2 = 6, kSplitCost4 = 15;
 
-#ifndef GIFT_FORCE_SPLIT_DIN
-#define GIFT_FORCE_SPLIT_DIN 0
-#endif
-#ifndef GIFT_FORCE_SPLIT
-#define GIFT_FORCE_SPLIT 2
-#endif
 template <class SlotFn>
 int plan(const TcLayer* layers, int n, uint16_t* off, uint16_t* ids, int max_ids, SlotFn slots_for, int* split) {
   int min_nc = 1 << 30, max_nc = 0, panels = 0;
@@ -1490,10 +1365,6 @@ int plan(const TcLayer* layers, int n, uint16_t* off, uint16_t* ids, int max_ids
     min_nc = std::min(min_nc, layers[l].d_in / kChunk);
     max_nc = std::max(max_nc, layers[l].d_in / kChunk);
     panels += (layers[l].d_out + kPanel - 1) / kPanel;
-  }
-  if (GIFT_FORCE_SPLIT_DIN > 0 && min_nc * kChunk >= GIFT_FORCE_SPLIT_DIN && slots_for(GIFT_FORCE_SPLIT) > 0) {
-    *split = GIFT_FORCE_SPLIT;
-    return schedule(layers, n, off, ids, max_ids, slots_for(GIFT_FORCE_SPLIT), GIFT_FORCE_SPLIT, nullptr);
   }
   int best_s = 1;
   if (panels < kNumSMs) {
@@ -1521,11 +1392,9 @@ bool tc_codec_available() { return tmap_encoder() != nullptr; }
 // Layers [0, cnt) of one launch: the same format, at most kMaxJobs layers and
 // kMaxPanels panels, each layer at most 256 panels (0: the first layer is
 // larger and is coded in parts of 256 panels).
-static bool split_class(const TcLayer& L) { return GIFT_FORCE_SPLIT_DIN > 0 && L.d_in >= GIFT_FORCE_SPLIT_DIN; }
 static int group_count(const TcLayer* layers, int n) {
   int cnt = 0, panels = 0;
-  while (cnt < n && cnt < kMaxJobs && layers[cnt].fmt == layers[0].fmt &&
-         split_class(layers[cnt]) == split_class(layers[0])) {
+  while (cnt < n && cnt < kMaxJobs && layers[cnt].fmt == layers[0].fmt) {
     const int np = (layers[cnt].d_out + kPanel - 1) / kPanel;
     if (np > 256 || panels + np > kMaxPanels) break;
     panels += np;
@@ -1555,12 +1424,6 @@ int tc_codec_split(const TcLayer* layers, int n, bool encode) {
 cudaError_t launch_whiten_encode_tc(const TcLayer* layers, int n, uint32_t* err, cudaStream_t s,
                                     uint32_t stall_polls) {
   cudaError_t e = cudaSuccess;
-  std::vector<TcLayer> sorted;
-  if (GIFT_FORCE_SPLIT_DIN > 0 && n > 1) {
-    sorted.assign(layers, layers + n);
-    std::stable_partition(sorted.begin(), sorted.end(), [](const TcLayer& L) { return !split_class(L); });
-    layers = sorted.data();
-  }
   for (int base = 0; base < n;) {
     // pack as many layers as fit one launch
     const int cnt = group_count(layers + base, n - base);
@@ -1622,12 +1485,6 @@ cudaError_t launch_whiten_encode_tc(const TcLayer* layers, int n, uint32_t* err,
 cudaError_t launch_whiten_decode_tc(const TcLayer* layers, int n, uint32_t* err, cudaStream_t s,
                                     uint32_t stall_polls) {
   cudaError_t e = cudaSuccess;
-  std::vector<TcLayer> sorted;
-  if (GIFT_FORCE_SPLIT_DIN > 0 && n > 1) {
-    sorted.assign(layers, layers + n);
-    std::stable_partition(sorted.begin(), sorted.end(), [](const TcLayer& L) { return !split_class(L); });
-    layers = sorted.data();
-  }
   for (int base = 0; base < n;) {
     const int cnt = group_count(layers + base, n - base);
     if (cnt == 0) {
@@ -1666,7 +1523,6 @@ cudaError_t launch_whiten_decode_tc(const TcLayer* layers, int n, uint32_t* err,
       J.codes = L.codes;
       J.sb = L.block_scales;
       J.tscale = L.tensor_scale;
-      J.G_hat = L.G_hat;
       J.fmt = L.fmt;
       J.d_out = L.d_out;
       J.d_in = L.d_in;
