@@ -418,17 +418,26 @@ def buffer_set(ops, W, G_all, Gh_all):
                 err_pairs=[(L.G, L.G_hat) for L in wl], G_all=G_all, Gh_all=Gh_all, err=torch.empty_like(W["err"]))
 
 
-# DRAM traffic of the whitened codec launches from one ncu capture of the
-# depth-8 stack (16 whitened layers; profiles/ names the command): read and
-# write bytes per gradient element.  The kernels' work grows in proportion to
-# the elements, so the bench's launch is that figure x its elements.  Lines
-# still dirty in L2 when a kernel ends are written back during later kernels
-# and are not in its write count, so the read excess (read bytes over the
-# algorithmic read bytes) is the figure that shows wasted traffic.  Valid
-# only for the kernel source it was taken on (sha256 of the file); otherwise
-# the bench reports traffic as null.
-TRAFFIC = {}
-TRAFFIC_SOURCE = ("geometry_aware_fp8_b200/csrc/codec_tc.cu", "")
+# Memory traffic of the whitened codec launches from one ncu capture of the
+# depth-8 stack (16 whitened layers; profiles/ names the command), per
+# gradient element: DRAM read bytes, and the bytes the kernel wrote into L2
+# (L2 write sectors from the SMs x 32 B).  Every written line reaches DRAM,
+# but lines still dirty in L2 when a kernel ends are written back during
+# later kernels, so the kernel's own DRAM write counter sees only part of
+# them; the L2 write-in is the full write traffic (sector-granular: the
+# encoder's 4-byte scale stores count as whole 32-byte sectors there, an upper
+# bound that L2 merges before DRAM).  The kernels' work grows in
+# proportion to the elements, so the bench's launch is that figure x its
+# elements.  Valid only for the kernel source it was taken on (sha256 of the
+# file); otherwise the bench reports traffic as null.
+TRAFFIC = {
+    "decode_whitened": {"read_per_element": 1.342563, "l2_write_per_element": 2.000000,
+                        "dram_write_per_element": 1.156631, "profile": "profiles/whiten_decode_tc_stack8.md"},
+    "encode_whitened": {"read_per_element": 2.896140, "l2_write_per_element": 1.250000,
+                        "dram_write_per_element": 0.227620, "profile": "profiles/whiten_encode_tc_stack8.md"},
+}
+TRAFFIC_SOURCE = ("geometry_aware_fp8_b200/csrc/codec_tc.cu",
+                  "94743d17f861350e6c2dd80a5d21fefd16f856c9657ac62cf13bb4dd0a97126e")
 
 
 def traffic_for(phase, n_elements, alg_read, alg_write):
@@ -440,9 +449,10 @@ def traffic_for(phase, n_elements, alg_read, alg_write):
     with open(path, "rb") as f:
         if hashlib.sha256(f.read()).hexdigest() != TRAFFIC_SOURCE[1]:
             return None
-    rd, wr = t["read_per_element"] * n_elements, t["write_per_element"] * n_elements
+    rd, wr = t["read_per_element"] * n_elements, t["l2_write_per_element"] * n_elements
     return {"bytes": rd + wr, "read_bytes": rd, "write_bytes": wr, "read_excess": rd / alg_read,
-            "write_fraction_seen": wr / alg_write, "profile": t["profile"]}
+            "write_excess": wr / alg_write,
+            "dram_write_during_kernel_bytes": t["dram_write_per_element"] * n_elements, "profile": t["profile"]}
 
 
 def phase_bytes(W):

@@ -315,16 +315,33 @@ __global__ void __launch_bounds__(kRT) gram_partial_kernel(const __grid_constant
   for (int a = 0; a < 4; ++a)
 #pragma unroll
     for (int b = 0; b < 4; ++b) acc[a][b] = 0.0;
-  for (int r0 = p * kGramRows; r0 < min(d, (p + 1) * kGramRows); r0 += 64) {
+  // A thread's 16 entries of each 64 x 64 tile, loaded into registers all at
+  // once (one memory latency per tile), the next tile's while this one is
+  // multiplied.
+  static_assert(kRT * 16 == 64 * 64, "tile entries per thread");
+  float ra[16], rb[16];
+  auto fetch = [&](int r0) {
     const int rows = min(64, d - r0);
-    __syncthreads();
-    for (int e = threadIdx.x; e < 64 * 64; e += kRT) {
-      const int rr = e >> 6, c = e & 63;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const int e = threadIdx.x + k * kRT, rr = e >> 6, c = e & 63;
       const bool in = rr < rows && c < m;
-      Sa[rr][c] = in ? Ya[(int64_t)(r0 + rr) * m + c] : 0.0f;
-      Sb[rr][c] = in ? Yb[(int64_t)(r0 + rr) * m + c] : 0.0f;
+      ra[k] = in ? __ldg(Ya + (int64_t)(r0 + rr) * m + c) : 0.0f;
+      rb[k] = in ? __ldg(Yb + (int64_t)(r0 + rr) * m + c) : 0.0f;
+    }
+  };
+  const int rbeg = p * kGramRows, rend = min(d, rbeg + kGramRows);
+  if (rbeg < rend) fetch(rbeg);
+  for (int r0 = rbeg; r0 < rend; r0 += 64) {
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const int e = threadIdx.x + k * kRT;
+      Sa[e >> 6][e & 63] = ra[k];
+      Sb[e >> 6][e & 63] = rb[k];
     }
     __syncthreads();
+    if (r0 + 64 < rend) fetch(r0 + 64);
 #pragma unroll 4
     for (int rr = 0; rr < 64; ++rr) {
       const float4 va = *reinterpret_cast<const float4*>(&Sa[rr][ti * 4]);
@@ -604,18 +621,26 @@ __global__ void __launch_bounds__(kST) rr_kernel(const __grid_constant__ RefBatc
       if (threadIdx.x < npairs) {
         const int a = threadIdx.x;
         const int p = tab_p[round][a], q = tab_q[round][a];
+        // The rotation's tangent t only has to shrink B[p][q]: it is taken
+        // in fp32 from the fp64 entries (a factor ~1e-7 of B[p][q] remains,
+        // removed by the next sweep), so the fp64 divisions and square root
+        // leave the round's critical path.  The rotation itself, c = (1 +
+        // t^2)^{-1/2} and s = t c, is fp64, so B and V stay exact
+        // orthogonal transforms to fp64 rounding.
         double c = 1.0, s = 0.0;
         if (q < m) {
-          const double bpq = B[p * ld + q];
-          if (bpq != 0.0) {
-            const double theta = (B[q * ld + q] - B[p * ld + p]) / (2.0 * bpq);
-            double t;
-            if (fabs(theta) > 1e150)
-              t = 0.5 / theta;
+          const float bpq = (float)B[p * ld + q];
+          const float dqp = (float)(B[q * ld + q] - B[p * ld + p]);
+          if (bpq != 0.0f) {
+            const float theta = dqp / (2.0f * bpq);
+            float t;
+            if (fabsf(theta) > 1e18f)
+              t = 0.5f / theta;
             else
-              t = copysign(1.0, theta) / (fabs(theta) + sqrt(theta * theta + 1.0));
-            c = rsqrt(t * t + 1.0);
-            s = t * c;
+              t = copysignf(1.0f, theta) / (fabsf(theta) + sqrtf(fmaf(theta, theta, 1.0f)));
+            const double td = (double)t;
+            c = rsqrt(fma(td, td, 1.0));
+            s = td * c;
           }
         }
         pp[a] = p;
