@@ -3,58 +3,86 @@
 // selective deployment leaves unwhitened (section V.C, Fig. 4).
 //
 // Pure streaming work, bound by HBM: 2 (bf16) or 4 (fp32) bytes in, 1 byte
-// plus 4/128 bytes out per element.  Eight threads own one 128-element block
-// (16 elements each, 16-byte vector loads and one 16-byte code store), the
-// block maximum is three xor-shuffles, and the grid is a multiple of the SM
-// count that strides over all blocks.
+// plus 4/128 bytes out per element.  Eight threads own one 128-element block,
+// 16 elements each, the block maximum is three xor-shuffles, and the grid is a
+// multiple of the SM count that strides over all blocks.  A thread's elements
+// are pieces of 16 bytes of the gradient (8 bf16 or 4 fp32) spaced by the
+// eight threads' pieces, so each warp-wide 16-byte load or store of G or
+// G_hat covers whole 32-byte sectors (a thread owning 16 consecutive bf16
+// values would write every sector in two halves, from two instructions).
 #include "common.cuh"
 #include "internal.h"
 
 namespace gift {
 namespace {
 
+// The 16 elements of thread `sub` in a 128-element block: kPieces pieces of
+// kPiece elements (16 bytes of T); piece k starts at element
+// kPiece sub + 8 kPiece k, and holds v[kPiece k .. kPiece (k + 1) - 1].
+// The codes of those elements (1 byte each) sit at the same offsets.
 template <typename T>
-struct Vec16;  // 16 consecutive elements loaded with 16-byte loads
+struct Vec16;
 
 template <>
 struct Vec16<__nv_bfloat16> {
-  static GIFT_DEV void load(const __nv_bfloat16* p, float (&v)[16]) {
-    const uint4* q = reinterpret_cast<const uint4*>(p);
-    uint4 a = __ldcs(q), b = __ldcs(q + 1);
-    uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+  static constexpr int kPiece = 8;
+  static GIFT_DEV void load(const __nv_bfloat16* blk, int sub, float (&v)[16]) {
+    const uint4 a = __ldcs(reinterpret_cast<const uint4*>(blk + 8 * sub));
+    const uint4 b = __ldcs(reinterpret_cast<const uint4*>(blk + 64 + 8 * sub));
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       v[2 * i] = bf16lo(w[i]);
       v[2 * i + 1] = bf16hi(w[i]);
     }
   }
-  static GIFT_DEV void store(__nv_bfloat16* p, const float (&v)[16]) {
+  static GIFT_DEV void store(__nv_bfloat16* blk, int sub, const float (&v)[16]) {
     uint32_t w[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) w[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
-    uint4* q = reinterpret_cast<uint4*>(p);
-    __stcs(q, make_uint4(w[0], w[1], w[2], w[3]));
-    __stcs(q + 1, make_uint4(w[4], w[5], w[6], w[7]));
+    __stcs(reinterpret_cast<uint4*>(blk + 8 * sub), make_uint4(w[0], w[1], w[2], w[3]));
+    __stcs(reinterpret_cast<uint4*>(blk + 64 + 8 * sub), make_uint4(w[4], w[5], w[6], w[7]));
+  }
+  // codes word i (4 codes) holds v[4 i .. 4 i + 3]
+  static GIFT_DEV void store_codes(uint8_t* blk, int sub, uint4 q) {
+    __stcs(reinterpret_cast<uint2*>(blk + 8 * sub), make_uint2(q.x, q.y));
+    __stcs(reinterpret_cast<uint2*>(blk + 64 + 8 * sub), make_uint2(q.z, q.w));
+  }
+  static GIFT_DEV uint4 load_codes(const uint8_t* blk, int sub) {
+    const uint2 a = __ldcs(reinterpret_cast<const uint2*>(blk + 8 * sub));
+    const uint2 b = __ldcs(reinterpret_cast<const uint2*>(blk + 64 + 8 * sub));
+    return make_uint4(a.x, a.y, b.x, b.y);
   }
 };
 
 template <>
 struct Vec16<float> {
-  static GIFT_DEV void load(const float* p, float (&v)[16]) {
-    const float4* q = reinterpret_cast<const float4*>(p);
+  static constexpr int kPiece = 4;
+  static GIFT_DEV void load(const float* blk, int sub, float (&v)[16]) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      float4 f = __ldcs(q + i);
-      v[4 * i] = f.x;
-      v[4 * i + 1] = f.y;
-      v[4 * i + 2] = f.z;
-      v[4 * i + 3] = f.w;
+    for (int k = 0; k < 4; ++k) {
+      const float4 f = __ldcs(reinterpret_cast<const float4*>(blk + 4 * sub + 32 * k));
+      v[4 * k] = f.x;
+      v[4 * k + 1] = f.y;
+      v[4 * k + 2] = f.z;
+      v[4 * k + 3] = f.w;
     }
   }
-  static GIFT_DEV void store(float* p, const float (&v)[16]) {
-    float4* q = reinterpret_cast<float4*>(p);
+  static GIFT_DEV void store(float* blk, int sub, const float (&v)[16]) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) __stcs(q + i, make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]));
+    for (int k = 0; k < 4; ++k)
+      __stcs(reinterpret_cast<float4*>(blk + 4 * sub + 32 * k), make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]));
+  }
+  static GIFT_DEV void store_codes(uint8_t* blk, int sub, uint4 q) {
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) __stcs(reinterpret_cast<unsigned int*>(blk + 4 * sub + 32 * k), w[k]);
+  }
+  static GIFT_DEV uint4 load_codes(const uint8_t* blk, int sub) {
+    uint32_t w[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) w[k] = __ldcs(reinterpret_cast<const unsigned int*>(blk + 4 * sub + 32 * k));
+    return make_uint4(w[0], w[1], w[2], w[3]);
   }
 };
 
@@ -75,6 +103,20 @@ GIFT_DEV uint4 quantize16(const float (&v)[16], float inv) {
   return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
+// Dequantise the 16 codes of a thread (word i = codes of v[4 i .. 4 i + 3]).
+GIFT_DEV void dequant16(uint4 q, float s, float (&v)[16]) {
+  const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 a = e4m3x2_to_f32x2((uint16_t)(w[i] & 0xFFFF));
+    const float2 c = e4m3x2_to_f32x2((uint16_t)(w[i] >> 16));
+    v[4 * i] = a.x * s;
+    v[4 * i + 1] = a.y * s;
+    v[4 * i + 2] = c.x * s;
+    v[4 * i + 3] = c.y * s;
+  }
+}
+
 template <typename T>
 __global__ void __launch_bounds__(256) euclid_encode_kernel(const T* __restrict__ G, uint8_t* __restrict__ codes,
                                                             float* __restrict__ scales, int64_t n_blocks,
@@ -89,9 +131,9 @@ __global__ void __launch_bounds__(256) euclid_encode_kernel(const T* __restrict_
     const int64_t b = base + ((threadIdx.x & 31) >> 3);
     const bool act = b < n_blocks;
     // lanes past the end load (and discard) the warp's first block: no branch before the shuffles
-    const int64_t e0 = (act ? b : base) * kBlock + sub * 16;
+    const int64_t e0 = (act ? b : base) * kBlock;  // the block's first element
     float v[16];
-    Vec16<T>::load(G + e0, v);
+    Vec16<T>::load(G + e0, sub, v);
     float m = 0.0f;
 #pragma unroll
     for (int i = 0; i < 16; ++i) m = fmax_nan(m, fabsf(v[i]));
@@ -101,7 +143,7 @@ __global__ void __launch_bounds__(256) euclid_encode_kernel(const T* __restrict_
     if (!act) continue;
     bad |= not_finite(m);
     const float inv = e4m3_inv_scale(m);
-    __stcs(reinterpret_cast<uint4*>(codes + e0), quantize16(v, inv));
+    Vec16<T>::store_codes(codes + e0, sub, quantize16(v, inv));
     if (sub == 0) scales[b] = e4m3_scale(m, inv);
   }
   report_bits(err, bad, GIFT_DEV_NONFINITE);
@@ -116,22 +158,13 @@ __global__ void __launch_bounds__(256) euclid_decode_kernel(const uint8_t* __res
   const int64_t groups_per_grid = (int64_t)gridDim.x * (blockDim.x >> 3);
   for (int64_t b = (int64_t)blockIdx.x * (blockDim.x >> 3) + (threadIdx.x >> 3); b < n_blocks;
        b += groups_per_grid) {
-    const int64_t e0 = b * kBlock + sub * 16;
-    const uint4 q = __ldcs(reinterpret_cast<const uint4*>(codes + e0));
+    const int64_t e0 = b * kBlock;  // the block's first element
+    const uint4 q = Vec16<T>::load_codes(codes + e0, sub);
     const float s = __ldg(scales + b);
     bad |= not_finite(s);
-    uint32_t w[4] = {q.x, q.y, q.z, q.w};
     float v[16];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      float2 a = e4m3x2_to_f32x2((uint16_t)(w[i] & 0xFFFF));
-      float2 c = e4m3x2_to_f32x2((uint16_t)(w[i] >> 16));
-      v[4 * i] = a.x * s;
-      v[4 * i + 1] = a.y * s;
-      v[4 * i + 2] = c.x * s;
-      v[4 * i + 3] = c.y * s;
-    }
-    Vec16<T>::store(out + e0, v);
+    dequant16(q, s, v);
+    Vec16<T>::store(out + e0, sub, v);
   }
   report_bits(err, bad, GIFT_DEV_NONFINITE);
 }
@@ -192,11 +225,11 @@ __global__ void __launch_bounds__(256) euclid_encode_group_kernel(const __grid_c
     const bool has1 = has0 && b1 < total;
     l0 = advance_layer(pre, g.n, l0, b0);
     l1 = has1 ? advance_layer(pre, g.n, l1 > l0 ? l1 : l0, b1) : l0;
-    const int64_t e0 = (b0 - pre[l0]) * kBlock + sub * 16;
-    const int64_t e1 = has1 ? (b1 - pre[l1]) * kBlock + sub * 16 : e0;
+    const int64_t e0 = (b0 - pre[l0]) * kBlock;  // the blocks' first elements
+    const int64_t e1 = has1 ? (b1 - pre[l1]) * kBlock : e0;
     float v0[16], v1[16];
-    Vec16<T>::load((const T*)g.src[l0] + e0, v0);
-    Vec16<T>::load((const T*)g.src[l1] + e1, v1);
+    Vec16<T>::load((const T*)g.src[l0] + e0, sub, v0);
+    Vec16<T>::load((const T*)g.src[l1] + e1, sub, v1);
     float m0 = 0.0f, m1 = 0.0f;
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
@@ -211,29 +244,17 @@ __global__ void __launch_bounds__(256) euclid_encode_group_kernel(const __grid_c
     if (!has0) continue;  // after the shuffles; has1 implies has0
     bad |= not_finite(m0) || (has1 && not_finite(m1));
     const float i0 = e4m3_inv_scale(m0);
-    __stcs(reinterpret_cast<uint4*>((uint8_t*)g.dst[l0] + e0), quantize16(v0, i0));
+    Vec16<T>::store_codes((uint8_t*)g.dst[l0] + e0, sub, quantize16(v0, i0));
     if (sub == 0) g.scales[l0][b0 - pre[l0]] = e4m3_scale(m0, i0);
     if (has1) {
       const float i1 = e4m3_inv_scale(m1);
-      __stcs(reinterpret_cast<uint4*>((uint8_t*)g.dst[l1] + e1), quantize16(v1, i1));
+      Vec16<T>::store_codes((uint8_t*)g.dst[l1] + e1, sub, quantize16(v1, i1));
       if (sub == 0) g.scales[l1][b1 - pre[l1]] = e4m3_scale(m1, i1);
     }
   }
   report_bits(g.err, bad, GIFT_DEV_NONFINITE);
 }
 
-GIFT_DEV void dequant16(uint4 q, float s, float (&v)[16]) {
-  const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float2 a = e4m3x2_to_f32x2((uint16_t)(w[i] & 0xFFFF));
-    const float2 c = e4m3x2_to_f32x2((uint16_t)(w[i] >> 16));
-    v[4 * i] = a.x * s;
-    v[4 * i + 1] = a.y * s;
-    v[4 * i + 2] = c.x * s;
-    v[4 * i + 3] = c.y * s;
-  }
-}
 
 template <typename T>
 __global__ void __launch_bounds__(256) euclid_decode_group_kernel(const __grid_constant__ EuclidGroup g) {
@@ -250,22 +271,22 @@ __global__ void __launch_bounds__(256) euclid_decode_group_kernel(const __grid_c
     const int l0 = find_layer(pre, g.n, b0);
     const int l1 = has1 ? find_layer(pre, g.n, b1) : l0;
     const int64_t lb0 = b0 - pre[l0], lb1 = has1 ? b1 - pre[l1] : lb0;
-    const int64_t e0 = lb0 * kBlock + sub * 16, e1 = lb1 * kBlock + sub * 16;
-    const uint4 q0 = __ldcs(reinterpret_cast<const uint4*>((const uint8_t*)g.src[l0] + e0));
+    const int64_t e0 = lb0 * kBlock, e1 = lb1 * kBlock;  // the blocks' first elements
+    const uint4 q0 = Vec16<T>::load_codes((const uint8_t*)g.src[l0] + e0, sub);
     const float s0 = __ldg(g.scales[l0] + lb0);
     uint4 q1 = make_uint4(0, 0, 0, 0);
     float s1 = 0.0f;
     if (has1) {
-      q1 = __ldcs(reinterpret_cast<const uint4*>((const uint8_t*)g.src[l1] + e1));
+      q1 = Vec16<T>::load_codes((const uint8_t*)g.src[l1] + e1, sub);
       s1 = __ldg(g.scales[l1] + lb1);
     }
     bad |= not_finite(s0) || not_finite(s1);
     float v[16];
     dequant16(q0, s0, v);
-    Vec16<T>::store((T*)g.dst[l0] + e0, v);
+    Vec16<T>::store((T*)g.dst[l0] + e0, sub, v);
     if (has1) {
       dequant16(q1, s1, v);
-      Vec16<T>::store((T*)g.dst[l1] + e1, v);
+      Vec16<T>::store((T*)g.dst[l1] + e1, sub, v);
     }
   }
   report_bits(g.err, bad, GIFT_DEV_NONFINITE);
