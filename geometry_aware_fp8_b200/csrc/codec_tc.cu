@@ -1050,16 +1050,26 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
     for (int k = 0; k < 16; ++k) P[k] = 0.0f;
     float a = 0.0f;
     bool stop = false;
+    // E4M3: the chunk's fp32 block scale of this thread's row; NVFP4: the
+    // tensor scale (the block scales are inside the widened values).  Loaded
+    // one step ahead, so its memory latency overlaps the step before.
+    auto scale_of = [&](const Steps<DecParams>& t) -> float {
+      const DecJob& Jt = p.jobs[t.job()];
+      const int64_t rw = (int64_t)t.panel() * kPanel + r;
+      if (rw >= Jt.d_out) return 0.0f;
+      return FMT == kFmtE4M3 ? __ldg(Jt.scales + rw * (Jt.d_in / kChunk) + t.chunk()) : __ldg(Jt.tscale);
+    };
+    Steps<DecParams> ahead(p, beg, end, q, S);
+    float sc_next = ahead.valid() ? scale_of(ahead) : 0.0f;
     for (Steps<DecParams> st(p, beg, end, q, S); st.valid() && !stop; st.next(), ++step) {
       const int s = step % kDStages, j = step & 1;
       const DecJob& J = p.jobs[st.job()];
-      const int nc = J.d_in / kChunk, c = st.chunk();
+      const int c = st.chunk();
       const int64_t row = (int64_t)st.panel() * kPanel + r;
       const bool live = row < J.d_out;
-      // E4M3: the chunk's fp32 block scale; NVFP4: the tensor scale (the block
-      // scales are inside the widened values)
-      const float sc = !live ? 0.0f : (FMT == kFmtE4M3 ? __ldg(J.scales + row * nc + c) : __ldg(J.tscale));
-      if (not_finite(sc)) nonfin = 1;
+      const float sc = sc_next;
+      ahead.next();
+      sc_next = ahead.valid() ? scale_of(ahead) : 0.0f;
       if (st.block_start() && st.k >= 1) {
         // P of p_{k-1} is complete (in a cluster: this CTA's chunks of it,
         // summed over the cluster here): P o c -> bf16 hi/lo A operand of D3
@@ -1116,6 +1126,7 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
 #pragma unroll
         for (int k = 0; k < 16; ++k)
           P[k] = fmaf(sc, fmaf(__uint_as_float(tl[k]), 1.0f / kF16LoScale, __uint_as_float(th[k])), P[k]);
+        if (not_finite(sc)) nonfin = 1;
         ++d2;
       } else {
         // D3 epilogue: G_hat = a s q + acc, into scratch tile j once its previous use is stored
@@ -1133,6 +1144,7 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
         const uint32_t c_tile = sbase + s * kDStageBytes;
         const uint32_t o_tile = scr + j * kDScratch;  // two [128][64] bf16 boxes, 128-byte swizzle
         const float as = a * sc;
+        if (not_finite(sc)) nonfin = 1;
 #pragma unroll
         for (int g2 = 0; g2 < 2; ++g2) {
           uint32_t acc[32];
