@@ -200,6 +200,7 @@ def build_workload(torch, ops, synth, dev, depth, seed):
             L.U = torch.empty((d_in, RANK), device=dev, dtype=torch.float32)
             L.lam = torch.empty((RANK,), device=dev, dtype=torch.float32)
             L.rho = torch.empty((1,), device=dev, dtype=torch.float32)
+            L.U_split = torch.empty((2, d_in, 64), device=dev, dtype=torch.int16)
             ws = torch.empty((ops.refresh_workspace_size(REFRESH_N, d_in, RANK, OVERSAMPLE),), device=dev,
                              dtype=torch.uint8)
             st = torch.zeros((1,), device=dev, dtype=torch.int32)
@@ -368,8 +369,12 @@ def staleness_measure(torch, dev):
 
 
 def refresh_all(ops, W):
-    """Factor refresh of every whitened layer in one batched call."""
+    """Factor refresh of every whitened layer in one batched call, then the U
+    split the tensor-core codec loads (gift_split_u, one small launch a layer)."""
     ops.factor_refresh_many(W["jobs"], len(W["whitened"]), RANK, OVERSAMPLE, ITERS)
+    for w in W["whitened"]:
+        L = w["layer"]
+        ops.split_u(L.U, out=L.U_split)
 
 
 PHASES = ("encode_euclid", "encode_whitened", "decode_euclid", "decode_whitened", "error")
@@ -508,8 +513,8 @@ def config2_batch_measure(torch, ops, synth, dev, peak, reps=20, batch=24):
     """Config 2 (the MLP up-projection stand-in, d_in 1536, d_out 4096, bf16,
     exponent 1.0) as a batch of `batch` distinct gradients of that layer, each
     with its own rank-32 factor refreshed from 8192 bf16 tokens (one batched
-    refresh, untimed), coded by one grouped whitened encode and one grouped
-    decode.  The batch (302 MB of G) is larger than L2, and L2 is flushed
+    refresh and its U splits, untimed), coded by one grouped whitened encode
+    and one grouped decode.  The batch (302 MB of G) is larger than L2, and L2 is flushed
     between timed repetitions."""
     d_out, d_in = 4096, 1536
     gen = torch.Generator(device=dev)
@@ -531,6 +536,8 @@ def config2_batch_measure(torch, ops, synth, dev, peak, reps=20, batch=24):
         layers.append(L)
     jobs = ops.make_refresh_jobs(items)
     ops.factor_refresh_many(jobs, batch, RANK, OVERSAMPLE, ITERS)
+    for L in layers:
+        L.U_split = ops.split_u(L.U)
     torch.cuda.synchronize()
     del items, jobs
     packed = ops.make_layers(layers)

@@ -199,6 +199,7 @@ static gift_status run_many(const gift_layer* layers, int n, uint32_t* dev_statu
     const void* g = encode ? L.G : (const void*)L.G_hat;
     gift_status st = check_codec_args(g, L.dtype, L.d_out, L.d_in, L.U, L.lambda, L.rho, L.rank, L.codes, L.scales);
     if (st != GIFT_OK) return st;
+    if (L.U_split && !aligned16(L.U_split)) return GIFT_ERR_ALIGN;
   }
   if (n == 0) return GIFT_OK;
   gift_status st = device_ok();
@@ -216,6 +217,7 @@ static gift_status run_many(const gift_layer* layers, int n, uint32_t* dev_statu
                                    : EuclidLayer{L.codes, L.G_hat, L.scales, nb});
     } else if (use_tc(L.dtype, L.rank, L.d_in)) {
       tc.push_back(TcLayer{L.G, L.G_hat, L.codes, L.scales, L.U, L.lambda, L.rho, (int)L.d_out, (int)L.d_in, L.rank});
+      tc.back().U_split = L.U_split;
     } else {
       e = encode ? launch_whiten_encode_simt(L.G, (gift_dtype)L.dtype, L.d_out, L.d_in, L.U, L.lambda, L.rho, L.rank,
                                              L.codes, L.scales, dev_status, s)
@@ -242,8 +244,10 @@ gift_status gift_codec_split(const gift_layer* layers, int n, int encode, int* s
   for (int i = 0; i < n; ++i) {
     const gift_layer& L = layers[i];
     if (L.d_in < GIFT_E4M3_BLOCK || L.d_in % GIFT_E4M3_BLOCK != 0 || L.d_out < 0) return GIFT_ERR_SHAPE;
-    if (L.d_out > 0 && L.rank > 0 && use_tc(L.dtype, L.rank, L.d_in))
+    if (L.d_out > 0 && L.rank > 0 && use_tc(L.dtype, L.rank, L.d_in)) {
       tc.push_back(TcLayer{L.G, L.G_hat, L.codes, L.scales, L.U, L.lambda, L.rho, (int)L.d_out, (int)L.d_in, L.rank});
+      tc.back().U_split = L.U_split;
+    }
   }
   *split = 0;
   if (tc.empty()) return GIFT_OK;
@@ -253,6 +257,14 @@ gift_status gift_codec_split(const gift_layer* layers, int n, int encode, int* s
   if (S < 1) return GIFT_ERR_SHAPE;
   *split = S;
   return GIFT_OK;
+}
+
+gift_status gift_split_u(const float* U, int64_t d_in, int rank, uint16_t* U_split, gift_stream_t stream) {
+  if (!U || !U_split || rank != 32 || d_in < 1) return GIFT_ERR_INVALID_ARG;
+  if (!aligned16(U) || !aligned16(U_split)) return GIFT_ERR_ALIGN;
+  gift_status st = device_ok();
+  if (st != GIFT_OK) return st;
+  return cuda_status(launch_split_u(U, d_in, U_split, (cudaStream_t)stream));
 }
 
 gift_status gift_encode_many(const gift_layer* layers, int n, uint32_t* dev_status, gift_stream_t stream) {
@@ -273,7 +285,9 @@ gift_status gift_codec_stall_test(const gift_layer* layer, int encode, uint32_t 
   if (L.d_out == 0 || L.rank == 0) return GIFT_ERR_INVALID_ARG;
   if ((st = device_ok()) != GIFT_OK) return st;
   if (!use_tc(L.dtype, L.rank, L.d_in)) return GIFT_ERR_UNSUPPORTED;
+  if (L.U_split && !aligned16(L.U_split)) return GIFT_ERR_ALIGN;
   TcLayer T{L.G, L.G_hat, L.codes, L.scales, L.U, L.lambda, L.rho, (int)L.d_out, (int)L.d_in, L.rank};
+  T.U_split = L.U_split;
   cudaStream_t s = (cudaStream_t)stream;
   return cuda_status(encode ? launch_whiten_encode_tc(&T, 1, dev_status, s, stall_polls)
                             : launch_whiten_decode_tc(&T, 1, dev_status, s, stall_polls));

@@ -95,6 +95,7 @@ struct EncParams {
   uint16_t sched_ids[kMaxPanels];   // job << 8 | panel
   int split;                        // CTAs per cluster, each taking 1 / split of every panel's chunks
   uint32_t stall_polls;             // test hook (0 = off): see stall_check
+  int presplit;                     // 1: tmU maps the caller's U split (no conversion in the kernel)
 };
 static_assert(sizeof(EncParams) <= 32760, "kernel parameter space");
 
@@ -466,6 +467,7 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
         mbar_arrive_expect_tx(&tfull[s], kGBytes + kUBytes);
         tma_load_2d_hint(dst, &J.tmG, &tfull[s], st.chunk() * kChunk, st.panel() * kPanel, pol);
         tma_load_2d_hint(dst + kGHalf, &J.tmG, &tfull[s], st.chunk() * kChunk + 64, st.panel() * kPanel, pol);
+        // U: fp32 rows (split by the converters), or the caller's bf16 [hi | lo] rows
         tma_load_2d_hint(dst + kGBytes, &J.tmU, &tfull[s], 0, st.chunk() * kChunk, keep);
       }
     }
@@ -498,7 +500,8 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
     // at the same step.
     const int t = threadIdx.x - 256;
     uint32_t step = 0;
-    for (Steps<EncParams> st(p, beg, end, q, S); st.valid(); st.next(), ++step) {
+    // with a pre-split U the stages are ready as TMA lands them: nothing to do
+    for (Steps<EncParams> st(p, beg, end, q, S); st.valid() && !p.presplit; st.next(), ++step) {
       const int s = step % kStages;
       const uint32_t use = step / kStages;
       float u[32];
@@ -523,7 +526,7 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
         // block k >= 1 starts with the second pass of p_{k-1}: its P o (c/a) must be
         // in shared memory, and P in TMEM has been read (it is reused for p_k)
         if (st.block_start() && st.k >= 1 && !mbar_wait(pc_full, (st.k - 1) & 1u, kWaitLimit)) { failed = 1; break; }
-        if (!mbar_wait(&full[s], (step / kStages) & 1u, kWaitLimit)) { failed = 1; break; }
+        if (!mbar_wait(p.presplit ? &tfull[s] : &full[s], (step / kStages) & 1u, kWaitLimit)) { failed = 1; break; }
         tc_fence_after();
         const uint32_t g_tile = sbase + s * kStageBytes, u_tile = g_tile + kGBytes;
         if (st.pass == 0) {
@@ -781,6 +784,7 @@ struct DecParams {
   uint16_t sched_ids[kMaxPanels];   // job << 8 | panel
   int split;                        // CTAs per cluster, each taking 1 / split of every panel's chunks
   uint32_t stall_polls;             // test hook (0 = off): see stall_check
+  int presplit;                     // 1: tmU maps the caller's U split (no conversion in the kernel)
 };
 static_assert(sizeof(DecParams) <= 32760, "kernel parameter space");
 
@@ -885,14 +889,23 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
         } else {
           mbar_arrive_expect_tx(&cfull[s], ub);  // NVFP4 codes are read from global memory
         }
-        tma_load_2d_hint(dst + kDCodes, &J.tmU, &cfull[s], 0, st.chunk() * kChunk, keep);
+        // U: fp32 rows (split by the converters), or the caller's split, whose rows
+        // d_in .. 2 d_in - 1 hold the f16 parts for D2 and rows 0 .. d_in - 1 the
+        // bf16 parts for D3
+        const int urow = (p.presplit && st.pass == 0 ? J.d_in : 0) + st.chunk() * kChunk;
+        tma_load_2d_hint(dst + kDCodes, &J.tmU, &cfull[s], 0, urow, keep);
       }
     }
   } else if (warp == 14) {
     // ---------------- output stores: a second-pass step's tile leaves by two TMA stores ----------------
-    // All epilogue threads have read the step's codes when its tile is ready,
-    // so the stage is released first, then the scratch tile once the stores
-    // have read it.
+    // The epilogue has read the step's codes from its stage when the tile is
+    // ready; the stage and the scratch tile are released once the stores
+    // have read the tile.  Releasing the stage only then keeps the protocol
+    // safe: the converters, which wait for a scratch tile only in first-pass
+    // steps, cannot reach a step whose tile still has an earlier second-pass
+    // use unstored (with the stage released at the tile's readiness, a CPU
+    // simulation of the protocol found schedules of mixed panel lengths where
+    // their parity wait on the tile passed two phases early).
     if (lane == 0) {
       const uint64_t drop = policy_evict_first();
       uint32_t step = 0, par = 0;  // par: bit j = phase parity of oready[j]
@@ -903,7 +916,6 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
           failed = 1;
           break;
         }
-        mbar_arrive(&empty[s]);
         const DecJob& J = p.jobs[st.job()];
         const uint32_t o_tile = scr + j * kDScratch;
         tma_store_2d_hint(&J.tmO, o_tile, st.chunk() * kChunk, st.panel() * kPanel, drop);
@@ -911,12 +923,16 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
         bulk_commit();
         bulk_wait_read<0>();
         par ^= 1u << j;
+        mbar_arrive(&empty[s]);
         mbar_arrive(&sfree[j]);
       }
       bulk_wait_all();
     }
   } else if (warp >= 8 && warp < 12) {
     // ---------------- converters: U split in place; first pass: codes widened into a scratch tile ----------------
+    // With a pre-split U, first-pass stages need only the codes widened and
+    // second-pass stages nothing; the converters still take every stage in
+    // turn, so their waits on the stages never fall a phase behind the ring.
     const int t = threadIdx.x - 256;
     uint32_t step = 0;
     for (Steps<DecParams> st(p, beg, end, q, S); st.valid(); st.next(), ++step) {
@@ -933,11 +949,13 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
       const uint32_t u_tile = c_tile + kDCodes;
       const uint32_t q_tile = scr + j * kDScratch;
       // D2 multiplies f16 codes by an f16 split of U, D3 the bf16 P' o c' by a bf16 split
-      u_row_from_tile(u_tile, t, u);
-      if (st.pass == 0)
-        store_u_split_f16(u_tile, t, u);
-      else
-        store_u_split_bf16(u_tile, t, u);
+      if (!p.presplit) {
+        u_row_from_tile(u_tile, t, u);
+        if (st.pass == 0)
+          store_u_split_f16(u_tile, t, u);
+        else
+          store_u_split_bf16(u_tile, t, u);
+      }
       const DecJob& J = p.jobs[st.job()];
       if (st.pass == 0 && FMT != kFmtE4M3) {
         // NVFP4: row t's 128 codes (64 bytes) and 8 block scales from global,
@@ -1401,12 +1419,69 @@ int plan(const TcLayer* layers, int n, uint16_t* off, uint16_t* ids, int max_ids
 
 bool tc_codec_available() { return tmap_encoder() != nullptr; }
 
+namespace {
+// One thread per U row: the same parts the converter warps form in shared
+// memory (store_u_split_bf16 / store_u_split_f16), written to global memory.
+__global__ void __launch_bounds__(128) split_u_kernel(const float* __restrict__ U, int64_t d_in,
+                                                      uint16_t* __restrict__ out) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= d_in) return;
+  const float4* src = reinterpret_cast<const float4*>(U + i * 32);
+  float u[32];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const float4 v = __ldg(src + q);
+    u[4 * q] = v.x;
+    u[4 * q + 1] = v.y;
+    u[4 * q + 2] = v.z;
+    u[4 * q + 3] = v.w;
+  }
+  uint32_t bh[16], bl[16], fh[16], fl[16];
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    float h0, l0, h1, l1;
+    split_bf16(u[2 * k], h0, l0);
+    split_bf16(u[2 * k + 1], h1, l1);
+    bh[k] = pack_bf16x2(h0, h1);
+    bl[k] = pack_bf16x2(l0, l1);
+    const float g0 = __half2float(__float2half_rn(u[2 * k]));
+    const float g1 = __half2float(__float2half_rn(u[2 * k + 1]));
+    fh[k] = pack_f16x2(g0, g1);
+    fl[k] = pack_f16x2((u[2 * k] - g0) * kF16LoScale, (u[2 * k + 1] - g1) * kF16LoScale);
+  }
+  uint4* b = reinterpret_cast<uint4*>(out + i * 64);
+  uint4* f = reinterpret_cast<uint4*>(out + (d_in + i) * 64);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    b[q] = make_uint4(bh[4 * q], bh[4 * q + 1], bh[4 * q + 2], bh[4 * q + 3]);
+    b[4 + q] = make_uint4(bl[4 * q], bl[4 * q + 1], bl[4 * q + 2], bl[4 * q + 3]);
+    f[q] = make_uint4(fh[4 * q], fh[4 * q + 1], fh[4 * q + 2], fh[4 * q + 3]);
+    f[4 + q] = make_uint4(fl[4 * q], fl[4 * q + 1], fl[4 * q + 2], fl[4 * q + 3]);
+  }
+}
+}  // namespace
+
+cudaError_t launch_split_u(const float* U, int64_t d_in, uint16_t* U_split, cudaStream_t s) {
+  if (d_in <= 0) return cudaSuccess;
+  split_u_kernel<<<(unsigned)((d_in + 127) / 128), 128, 0, s>>>(U, d_in, U_split);
+  return cudaGetLastError();
+}
+
 // Layers [0, cnt) of one launch: the same format, at most kMaxJobs layers and
 // kMaxPanels panels, each layer at most 256 panels (0: the first layer is
 // larger and is coded in parts of 256 panels).
+// Tensor map of a layer's U tiles: fp32 [d_in][32] (split in the kernel), or
+// the pre-split [2 d_in][64] 16-bit rows; both give 128-byte rows in 128-row boxes.
+static bool make_u_tmap(CUtensorMap* m, const TcLayer& L) {
+  if (L.U_split)
+    return make_tmap_2d(m, L.U_split, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, 2 * (uint64_t)L.d_in, 64, kChunk, 64);
+  return make_tmap_2d(m, L.U, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, (uint64_t)L.d_in, 32, kChunk, 32);
+}
+
 static int group_count(const TcLayer* layers, int n) {
   int cnt = 0, panels = 0;
-  while (cnt < n && cnt < kMaxJobs && layers[cnt].fmt == layers[0].fmt) {
+  while (cnt < n && cnt < kMaxJobs && layers[cnt].fmt == layers[0].fmt &&
+         (layers[cnt].U_split != nullptr) == (layers[0].U_split != nullptr)) {
     const int np = (layers[cnt].d_out + kPanel - 1) / kPanel;
     if (np > 256 || panels + np > kMaxPanels) break;
     panels += np;
@@ -1465,7 +1540,7 @@ cudaError_t launch_whiten_encode_tc(const TcLayer* layers, int n, uint32_t* err,
       EncJob& J = P.jobs[l];
       if (!make_tmap_2d(&J.tmG, L.G, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)L.d_out, (uint64_t)L.d_in,
                         kPanel, 64) ||
-          !make_tmap_2d(&J.tmU, L.U, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, (uint64_t)L.d_in, 32, kChunk, 32) ||
+          !make_u_tmap(&J.tmU, L) ||
           (L.fmt == kFmtE4M3 && !make_tmap_2d(&J.tmC, L.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)L.d_out,
                                               (uint64_t)L.d_in, kPanel, kChunk)))
         return cudaErrorInvalidValue;
@@ -1486,6 +1561,7 @@ cudaError_t launch_whiten_encode_tc(const TcLayer* layers, int n, uint32_t* err,
                           [fmt](int S) { return enc_slots(fmt, S); }, &P.split);
     if (grid <= 0) return cudaErrorInvalidValue;
     P.stall_polls = stall_polls;
+    P.presplit = layers[base].U_split != nullptr;
     if ((e = enc_launch(fmt, grid, P, err, s)) != cudaSuccess) return e;
     base += cnt;
   }
@@ -1524,7 +1600,7 @@ cudaError_t launch_whiten_decode_tc(const TcLayer* layers, int n, uint32_t* err,
       DecJob& J = P.jobs[l];
       if ((L.fmt == kFmtE4M3 && !make_tmap_2d(&J.tmC, L.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)L.d_out,
                                               (uint64_t)L.d_in, kPanel, kChunk)) ||
-          !make_tmap_2d(&J.tmU, L.U, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, (uint64_t)L.d_in, 32, kChunk, 32) ||
+          !make_u_tmap(&J.tmU, L) ||
           !make_tmap_2d(&J.tmO, L.G_hat, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)L.d_out, (uint64_t)L.d_in,
                         kPanel, 64))
         return cudaErrorInvalidValue;
@@ -1545,6 +1621,7 @@ cudaError_t launch_whiten_decode_tc(const TcLayer* layers, int n, uint32_t* err,
                           [fmt](int S) { return dec_slots(fmt, S); }, &P.split);
     if (grid <= 0) return cudaErrorInvalidValue;
     P.stall_polls = stall_polls;
+    P.presplit = layers[base].U_split != nullptr;
     if ((e = dec_launch(fmt, grid, P, err, s)) != cudaSuccess) return e;
     base += cnt;
   }

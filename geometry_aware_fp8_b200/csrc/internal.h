@@ -60,12 +60,19 @@ struct TcLayer {
   int fmt = 0;
   uint8_t* block_scales = nullptr;
   float* tensor_scale = nullptr;
+  // Optional U split by gift_split_u ([2][d_in][64] 16-bit: bf16 [hi | lo]
+  // rows, then f16 [hi | 2^11 lo] rows): the kernels then load it as it is
+  // instead of splitting U themselves.  Layers with and without it go to
+  // separate launches.
+  const uint16_t* U_split = nullptr;
 };
 constexpr int kFmtE4M3 = 0, kFmtNvfp4Amax = 1, kFmtNvfp4 = 2;
 bool tc_codec_available();
 // stall_polls > 0 is a test hook: before any work, one thread of every CTA
 // waits at most that many polls on a barrier nothing arrives at, gives up,
 // and the CTA skips its work and reports GIFT_DEV_TIMEOUT.
+// U (d_in x 32 fp32) -> the [2][d_in][64] split the tensor-core codec loads (see TcLayer::U_split).
+cudaError_t launch_split_u(const float* U, int64_t d_in, uint16_t* U_split, cudaStream_t s);
 cudaError_t launch_whiten_encode_tc(const TcLayer* layers, int n, uint32_t* err, cudaStream_t s,
                                     uint32_t stall_polls = 0);
 cudaError_t launch_whiten_decode_tc(const TcLayer* layers, int n, uint32_t* err, cudaStream_t s,

@@ -29,7 +29,7 @@ EXPORTED = ("gift_status_string", "gift_version", "gift_refresh_workspace_size",
             "gift_error_workspace_size", "gift_roundtrip_error", "gift_encode_nvfp4", "gift_decode_nvfp4",
             "gift_codec_split", "gift_whitened_error_workspace_size", "gift_whitened_error",
             "gift_codec_stall_test", "gift_dense_factor_workspace_size", "gift_dense_factor", "gift_dense_split",
-            "gift_dense_encode", "gift_dense_decode", "gift_decode_sum")
+            "gift_dense_encode", "gift_dense_decode", "gift_decode_sum", "gift_split_u")
 DENSE_CHOLESKY, DENSE_INVSQRT = 1, 2
 
 
@@ -53,7 +53,7 @@ class Layer(ctypes.Structure):
     _fields_ = [("G", ctypes.c_void_p), ("G_hat", ctypes.c_void_p), ("codes", ctypes.c_void_p),
                 ("scales", ctypes.c_void_p), ("U", ctypes.c_void_p), ("lambda_", ctypes.c_void_p),
                 ("rho", ctypes.c_void_p), ("d_out", ctypes.c_int64), ("d_in", ctypes.c_int64),
-                ("rank", ctypes.c_int32), ("dtype", ctypes.c_int32)]
+                ("rank", ctypes.c_int32), ("dtype", ctypes.c_int32), ("U_split", ctypes.c_void_p)]
 
 
 _lib = None
@@ -80,6 +80,7 @@ def lib() -> ctypes.CDLL:
         L.gift_encode.argtypes = [vp, i32, i64, i64, vp, vp, vp, i32, vp, vp, vp, vp]
         L.gift_decode.argtypes = [vp, vp, i64, i64, vp, vp, vp, i32, vp, i32, vp, vp]
         L.gift_encode_many.argtypes = [ctypes.POINTER(Layer), i32, vp, vp]
+        L.gift_split_u.argtypes = [vp, i64, i32, vp, vp]
         L.gift_decode_many.argtypes = [ctypes.POINTER(Layer), i32, vp, vp]
         L.gift_codec_stall_test.argtypes = [ctypes.POINTER(Layer), i32, ctypes.c_uint32, vp, vp]
         L.gift_codec_split.argtypes = [ctypes.POINTER(Layer), i32, i32, ctypes.POINTER(i32)]
@@ -300,6 +301,7 @@ class LayerArgs:
     U: Optional[torch.Tensor] = None
     lam: Optional[torch.Tensor] = None
     rho: Optional[torch.Tensor] = None
+    U_split: Optional[torch.Tensor] = None  # split_u(U), or None: the kernels split U themselves
 
 
 def _dtype_code(dt: torch.dtype) -> int:
@@ -318,8 +320,18 @@ def make_layers(layers: Sequence[LayerArgs]):
             if t is not None and t.dtype != L.dtype:
                 raise TypeError(f"layer {i}: tensor dtype {t.dtype} differs from the layer's {L.dtype}")
         arr[i] = Layer(_ptr(L.G), _ptr(L.G_hat), _ptr(L.codes), _ptr(L.scales), _ptr(L.U), _ptr(L.lam),
-                       _ptr(L.rho), L.d_out, L.d_in, L.rank, _dtype_code(L.dtype))
+                       _ptr(L.rho), L.d_out, L.d_in, L.rank, _dtype_code(L.dtype), _ptr(L.U_split))
     return arr
+
+
+def split_u(U: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """The (2, d_in, 64) int16 U split that LayerArgs.U_split takes (gift_split_u)."""
+    _cuda(U, out)
+    d_in, rank = U.shape
+    if out is None:
+        out = torch.empty((2, d_in, 64), device=U.device, dtype=torch.int16)
+    _check(lib().gift_split_u(_ptr(U), d_in, rank, _ptr(out), _stream(stream)), "gift_split_u")
+    return out
 
 
 def encode_many(packed, n: int, stream=None, dev_status: Optional[torch.Tensor] = None):

@@ -217,7 +217,25 @@ typedef struct {
   int64_t d_in;
   int32_t rank;        /* 0 (Euclidean) or 1..32 */
   int32_t dtype;       /* gift_dtype of G and G_hat */
+  /* Optional (NULL: unused): U split once by gift_split_u after the factor
+   * refresh.  The tensor-core codec (bf16, rank 32, d_in % 128 == 0) then
+   * loads it as it is instead of splitting U in every launch; the results are
+   * bit-identical either way.  Must be the split of this layer's current U.
+   * Ignored by the other paths (which read U). */
+  const uint16_t* U_split;
 } gift_layer;
+
+/* ------------------------------------------------------------------------
+ * U split for the tensor-core codec (an implementation format, not part of
+ * the method): U_split = [2][d_in][64] 16-bit words, device, 16-byte
+ * aligned, caller-owned.  Row i of part 0 is [bf16(U_i) | bf16(U_i -
+ * bf16(U_i))] (32 + 32 values, round to nearest even), row i of part 1 is
+ * [f16(U_i) | f16((U_i - f16(U_i)) 2^11)].  U: d_in x 32 fp32, device,
+ * 16-byte aligned.  rank must be 32.  Asynchronous on `stream`.
+ * Errors: GIFT_ERR_INVALID_ARG (null pointer, rank != 32, d_in < 1),
+ * GIFT_ERR_ALIGN, GIFT_ERR_CUDA.
+ * ------------------------------------------------------------------------ */
+gift_status gift_split_u(const float* U, int64_t d_in, int rank, uint16_t* U_split, gift_stream_t stream);
 
 /* dev_status (nullable): one word for the whole call, bits as for gift_encode
  * / gift_decode; a TIMEOUT leaves the outputs of every layer undefined. */

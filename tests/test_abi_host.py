@@ -180,3 +180,18 @@ def test_codec_split_rejects_bad_arguments(L):
     # no layer on the tensor-core path (Euclidean): nothing to plan, no device needed
     assert L.gift_codec_split(eu, 1, 0, ctypes.byref(out)) == OK and out.value == 0
     assert L.gift_codec_split(eu, 0, 1, ctypes.byref(out)) == OK and out.value == 0
+
+
+def test_split_u_and_layer_split_arguments(L):
+    s = None
+    assert L.gift_split_u(None, 128, 32, A16, s) == INVALID
+    assert L.gift_split_u(A16, 128, 32, None, s) == INVALID
+    assert L.gift_split_u(A16, 128, 16, A16, s) == INVALID    # the split serves the rank-32 codec only
+    assert L.gift_split_u(A16, 0, 32, A16, s) == INVALID
+    assert L.gift_split_u(A_ODD, 128, 32, A16, s) == ALIGN
+    assert L.gift_split_u(A16, 128, 32, A_ODD, s) == ALIGN
+    # a grouped layer whose U split is misaligned is rejected before any launch
+    arr = (ops.Layer * 1)()
+    arr[0] = ops.Layer(A16, A16, A16, A16, A16, A16, A16, 256, 256, 32, 1, A_ODD)
+    assert L.gift_encode_many(arr, 1, None, None) == ALIGN
+    assert L.gift_decode_many(arr, 1, None, None) == ALIGN

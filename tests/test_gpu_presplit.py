@@ -1,0 +1,93 @@
+"""The tensor-core codec with a pre-split U (gift_split_u + gift_layer.U_split),
+through the C ABI on the GPU.
+
+The split is an implementation format, so it is checked against its
+definition (round-to-nearest-even bf16 and f16 parts, computed here with plain
+PyTorch casts), and the codec with it must give bit-identical codes, scales
+and G_hat to the same grouped call without it (whose parity with the oracle
+the other codec tests establish); one layer is also compared with the oracle
+directly.  Layers span ragged panels, both codec launch shapes (many panels,
+and few panels, where CTAs share a panel in a cluster) and a Euclidean layer
+in the same group.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import gift_oracle as O
+from geometry_aware_fp8_b200 import ops
+
+from _cmp import check_codes, check_scales
+from test_gpu_codec import _factor, _g, _to_dev
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+
+def test_split_u_matches_its_definition():
+    _, U, _, _ = _factor(512, 71)
+    Ud = torch.from_numpy(U).to(DEV)
+    S = ops.split_u(Ud)
+    torch.cuda.synchronize()
+    bh = Ud.to(torch.bfloat16)
+    bl = (Ud - bh.float()).to(torch.bfloat16)
+    fh = Ud.to(torch.float16)
+    fl = ((Ud - fh.float()) * 2048.0).to(torch.float16)
+    want0 = torch.cat([bh.view(torch.int16), bl.view(torch.int16)], dim=1)
+    want1 = torch.cat([fh.view(torch.int16), fl.view(torch.int16)], dim=1)
+    assert torch.equal(S[0], want0)
+    assert torch.equal(S[1], want1)
+
+
+def _layers(shapes, seed):
+    out = []
+    for i, (d_out, d_in, rank) in enumerate(shapes):
+        if rank:
+            Q, U, lam, rho = _factor(d_in, seed + 10 * i)
+            G, Gd = _g(d_out, Q, seed + 10 * i + 1, "bf16")
+            Ud, lamd, rhod = _to_dev(U, lam, np.array([rho], dtype=np.float32))
+            fac = (U, lam, rho)
+        else:
+            from geometry_aware_fp8_b200 import synth
+            G, Gd = _g(d_out, synth.haar_orthogonal(d_in, seed + 10 * i), seed + 10 * i + 1, "bf16")
+            Ud = lamd = rhod = None
+            fac = None
+        out.append((G, Gd, Ud, lamd, rhod, fac))
+    return out
+
+
+def _args(d_out, d_in, rank, Gd, Ud, lamd, rhod, presplit):
+    return ops.LayerArgs(d_out=d_out, d_in=d_in, rank=rank, dtype=torch.bfloat16, G=Gd,
+                         G_hat=torch.empty_like(Gd),
+                         codes=torch.empty((d_out, d_in), device=DEV, dtype=torch.uint8),
+                         scales=torch.empty((d_out, d_in // 128), device=DEV, dtype=torch.float32),
+                         U=Ud, lam=lamd, rho=rhod,
+                         U_split=ops.split_u(Ud) if (presplit and rank) else None)
+
+
+@pytest.mark.parametrize("shapes", [
+    [(300, 1536, 32), (129, 512, 32), (1536, 4096, 32), (200, 1536, 0)],  # many panels: one CTA each
+    [(4096, 1536, 32)],                                                   # few panels: a cluster per panel
+])
+def test_grouped_codec_with_presplit_u_is_bit_identical(shapes):
+    data = _layers(shapes, 300)
+    runs = {}
+    for presplit in (False, True):
+        args = [_args(d_out, d_in, rank, Gd, Ud, lamd, rhod, presplit)
+                for (d_out, d_in, rank), (_, Gd, Ud, lamd, rhod, _) in zip(shapes, data)]
+        packed = ops.make_layers(args)
+        st = torch.zeros((1,), device=DEV, dtype=torch.int32)
+        ops.encode_many(packed, len(args), dev_status=st)
+        ops.decode_many(packed, len(args), dev_status=st)
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        runs[presplit] = args
+    for a, b in zip(runs[False], runs[True]):
+        assert torch.equal(a.codes, b.codes)
+        assert torch.equal(a.scales, b.scales)
+        assert torch.equal(a.G_hat.view(torch.int16), b.G_hat.view(torch.int16))
+    # and one whitened layer against the oracle directly
+    (d_out, d_in, rank), (G, _, _, _, _, (U, lam, rho)) = shapes[0], data[0]
+    c_o, s_o = O.encode_e4m3(G.astype(np.float64), U.astype(np.float64), lam.astype(np.float64), float(rho))
+    check_codes(runs[True][0].codes.cpu().numpy(), c_o)
+    check_scales(runs[True][0].scales.cpu().numpy(), s_o)
