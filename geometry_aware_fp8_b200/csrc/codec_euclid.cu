@@ -26,16 +26,22 @@ struct Vec16;
 template <>
 struct Vec16<__nv_bfloat16> {
   static constexpr int kPiece = 8;
-  static GIFT_DEV void load(const __nv_bfloat16* blk, int sub, float (&v)[16]) {
-    const uint4 a = __ldcs(reinterpret_cast<const uint4*>(blk + 8 * sub));
-    const uint4 b = __ldcs(reinterpret_cast<const uint4*>(blk + 64 + 8 * sub));
-    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+  struct Raw {
+    uint4 a, b;
+  };
+  static GIFT_DEV Raw load_raw(const __nv_bfloat16* blk, int sub) {
+    return Raw{__ldcs(reinterpret_cast<const uint4*>(blk + 8 * sub)),
+               __ldcs(reinterpret_cast<const uint4*>(blk + 64 + 8 * sub))};
+  }
+  static GIFT_DEV void unpack(const Raw& r, float (&v)[16]) {
+    const uint32_t w[8] = {r.a.x, r.a.y, r.a.z, r.a.w, r.b.x, r.b.y, r.b.z, r.b.w};
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       v[2 * i] = bf16lo(w[i]);
       v[2 * i + 1] = bf16hi(w[i]);
     }
   }
+  static GIFT_DEV void load(const __nv_bfloat16* blk, int sub, float (&v)[16]) { unpack(load_raw(blk, sub), v); }
   static GIFT_DEV void store(__nv_bfloat16* blk, int sub, const float (&v)[16]) {
     uint32_t w[8];
 #pragma unroll
@@ -58,16 +64,25 @@ struct Vec16<__nv_bfloat16> {
 template <>
 struct Vec16<float> {
   static constexpr int kPiece = 4;
-  static GIFT_DEV void load(const float* blk, int sub, float (&v)[16]) {
+  struct Raw {
+    float4 f[4];
+  };
+  static GIFT_DEV Raw load_raw(const float* blk, int sub) {
+    Raw r;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) r.f[k] = __ldcs(reinterpret_cast<const float4*>(blk + 4 * sub + 32 * k));
+    return r;
+  }
+  static GIFT_DEV void unpack(const Raw& r, float (&v)[16]) {
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      const float4 f = __ldcs(reinterpret_cast<const float4*>(blk + 4 * sub + 32 * k));
-      v[4 * k] = f.x;
-      v[4 * k + 1] = f.y;
-      v[4 * k + 2] = f.z;
-      v[4 * k + 3] = f.w;
+      v[4 * k] = r.f[k].x;
+      v[4 * k + 1] = r.f[k].y;
+      v[4 * k + 2] = r.f[k].z;
+      v[4 * k + 3] = r.f[k].w;
     }
   }
+  static GIFT_DEV void load(const float* blk, int sub, float (&v)[16]) { unpack(load_raw(blk, sub), v); }
   static GIFT_DEV void store(float* blk, int sub, const float (&v)[16]) {
 #pragma unroll
     for (int k = 0; k < 4; ++k)
@@ -172,8 +187,8 @@ __global__ void __launch_bounds__(256) euclid_decode_kernel(const uint8_t* __res
 // Grouped form: many layers in one launch.  A block index b of the
 // concatenated layers is mapped to its layer through the prefix sums of the
 // layers' block counts (kept in shared memory): the encoder searches once per
-// thread and then advances (each thread's block index only grows), the
-// decoder searches per block pair (measured faster for it).
+// thread and stream and then advances (each stream's block index only grows),
+// the decoder searches per block.
 constexpr int kGroupMax = 64;
 
 struct EuclidGroup {
@@ -199,8 +214,11 @@ GIFT_DEV int advance_layer(const int64_t* pre, int n, int l, int64_t b) {
   return l;
 }
 
-// Two blocks per thread group per iteration: both blocks' loads are issued
-// before either is used, doubling the bytes in flight per thread.
+// kEncU blocks per thread group per iteration: every block's loads are issued
+// (as raw 16-byte words) before any is used, so each thread keeps kEncU x 32
+// bytes (bf16) in flight.  Stream u of a thread group takes blocks
+// first + u G, first + (u + kEncU) G, ... and keeps its own layer cursor.
+constexpr int kEncU = 4;
 template <typename T>
 __global__ void __launch_bounds__(256) euclid_encode_group_kernel(const __grid_constant__ EuclidGroup g) {
   __shared__ int64_t pre[kGroupMax + 1];
@@ -214,47 +232,50 @@ __global__ void __launch_bounds__(256) euclid_encode_group_kernel(const __grid_c
   // shuffles; lanes past the end idle)
   const int64_t wfirst = (int64_t)blockIdx.x * (blockDim.x >> 3) + ((threadIdx.x >> 5) << 2);
   const int64_t first = wfirst + ((threadIdx.x & 31) >> 3);
-  int l0 = first < total ? find_layer(pre, g.n, first) : 0, l1 = l0;
+  int lc[kEncU];
+#pragma unroll
+  for (int u = 0; u < kEncU; ++u) lc[u] = first + u * G < total ? find_layer(pre, g.n, first + u * G) : 0;
   bool bad = false;
-  for (int64_t base = wfirst; base < total; base += 2 * G) {
+  for (int64_t base = wfirst; base < total; base += kEncU * G) {
     const bool has0 = base + ((threadIdx.x & 31) >> 3) < total;
     // lanes past the end work on the warp's first block and discard it: no
     // branch before the shuffles
     const int64_t b0 = has0 ? base + ((threadIdx.x & 31) >> 3) : base;
-    const int64_t b1 = b0 + G;
-    const bool has1 = has0 && b1 < total;
-    l0 = advance_layer(pre, g.n, l0, b0);
-    l1 = has1 ? advance_layer(pre, g.n, l1 > l0 ? l1 : l0, b1) : l0;
-    const int64_t e0 = (b0 - pre[l0]) * kBlock;  // the blocks' first elements
-    const int64_t e1 = has1 ? (b1 - pre[l1]) * kBlock : e0;
-    float v0[16], v1[16];
-    Vec16<T>::load((const T*)g.src[l0] + e0, sub, v0);
-    Vec16<T>::load((const T*)g.src[l1] + e1, sub, v1);
-    float m0 = 0.0f, m1 = 0.0f;
+    int64_t e[kEncU];
+    bool has[kEncU];
+    typename Vec16<T>::Raw raw[kEncU];
+    // stream 0 follows b0 even on idle lanes (b0 only grows), so its cursor
+    // always names the layer of a block that exists
+    lc[0] = advance_layer(pre, g.n, lc[0], b0);
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      m0 = fmax_nan(m0, fabsf(v0[i]));
-      m1 = fmax_nan(m1, fabsf(v1[i]));
+    for (int u = 0; u < kEncU; ++u) {
+      const int64_t b = b0 + u * G;
+      has[u] = has0 && b < total;
+      if (u > 0 && has[u]) lc[u] = advance_layer(pre, g.n, lc[u], b);
+      // a stream past the end loads (and discards) stream 0's block
+      const int l = has[u] ? lc[u] : lc[0];
+      e[u] = ((has[u] ? b : b0) - pre[l]) * kBlock;  // the block's first element
+      raw[u] = Vec16<T>::load_raw((const T*)g.src[l] + e[u], sub);
     }
 #pragma unroll
-    for (int o = 1; o < 8; o <<= 1) {
-      m0 = fmax_nan(m0, __shfl_xor_sync(0xffffffffu, m0, o));
-      m1 = fmax_nan(m1, __shfl_xor_sync(0xffffffffu, m1, o));
-    }
-    if (!has0) continue;  // after the shuffles; has1 implies has0
-    bad |= not_finite(m0) || (has1 && not_finite(m1));
-    const float i0 = e4m3_inv_scale(m0);
-    Vec16<T>::store_codes((uint8_t*)g.dst[l0] + e0, sub, quantize16(v0, i0));
-    if (sub == 0) g.scales[l0][b0 - pre[l0]] = e4m3_scale(m0, i0);
-    if (has1) {
-      const float i1 = e4m3_inv_scale(m1);
-      Vec16<T>::store_codes((uint8_t*)g.dst[l1] + e1, sub, quantize16(v1, i1));
-      if (sub == 0) g.scales[l1][b1 - pre[l1]] = e4m3_scale(m1, i1);
+    for (int u = 0; u < kEncU; ++u) {
+      float v[16];
+      Vec16<T>::unpack(raw[u], v);
+      float m = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) m = fmax_nan(m, fabsf(v[i]));
+#pragma unroll
+      for (int o = 1; o < 8; o <<= 1) m = fmax_nan(m, __shfl_xor_sync(0xffffffffu, m, o));
+      if (!has[u]) continue;  // after the shuffles
+      const int l = lc[u];
+      bad |= not_finite(m);
+      const float inv = e4m3_inv_scale(m);
+      Vec16<T>::store_codes((uint8_t*)g.dst[l] + e[u], sub, quantize16(v, inv));
+      if (sub == 0) g.scales[l][e[u] / kBlock] = e4m3_scale(m, inv);
     }
   }
   report_bits(g.err, bad, GIFT_DEV_NONFINITE);
 }
-
 
 template <typename T>
 __global__ void __launch_bounds__(256) euclid_decode_group_kernel(const __grid_constant__ EuclidGroup g) {
@@ -265,28 +286,34 @@ __global__ void __launch_bounds__(256) euclid_decode_group_kernel(const __grid_c
   const int64_t total = pre[g.n];
   const int64_t G = (int64_t)gridDim.x * (blockDim.x >> 3);
   bool bad = false;
-  for (int64_t b0 = (int64_t)blockIdx.x * (blockDim.x >> 3) + (threadIdx.x >> 3); b0 < total; b0 += 2 * G) {
-    const int64_t b1 = b0 + G;
-    const bool has1 = b1 < total;
-    const int l0 = find_layer(pre, g.n, b0);
-    const int l1 = has1 ? find_layer(pre, g.n, b1) : l0;
-    const int64_t lb0 = b0 - pre[l0], lb1 = has1 ? b1 - pre[l1] : lb0;
-    const int64_t e0 = lb0 * kBlock, e1 = lb1 * kBlock;  // the blocks' first elements
-    const uint4 q0 = Vec16<T>::load_codes((const uint8_t*)g.src[l0] + e0, sub);
-    const float s0 = __ldg(g.scales[l0] + lb0);
-    uint4 q1 = make_uint4(0, 0, 0, 0);
-    float s1 = 0.0f;
-    if (has1) {
-      q1 = Vec16<T>::load_codes((const uint8_t*)g.src[l1] + e1, sub);
-      s1 = __ldg(g.scales[l1] + lb1);
+  // kDecU blocks per thread group per iteration, all loads issued first
+  constexpr int kDecU = 4;
+  for (int64_t b0 = (int64_t)blockIdx.x * (blockDim.x >> 3) + (threadIdx.x >> 3); b0 < total; b0 += kDecU * G) {
+    uint4 qv[kDecU];
+    float sv[kDecU];
+    int lv[kDecU];
+    int64_t lbv[kDecU];
+#pragma unroll
+    for (int u = 0; u < kDecU; ++u) {
+      const int64_t b = b0 + u * G;
+      qv[u] = make_uint4(0, 0, 0, 0);
+      sv[u] = 0.0f;
+      lv[u] = 0;
+      lbv[u] = 0;
+      if (b < total) {
+        lv[u] = find_layer(pre, g.n, b);
+        lbv[u] = b - pre[lv[u]];
+        qv[u] = Vec16<T>::load_codes((const uint8_t*)g.src[lv[u]] + lbv[u] * kBlock, sub);
+        sv[u] = __ldg(g.scales[lv[u]] + lbv[u]);
+      }
     }
-    bad |= not_finite(s0) || not_finite(s1);
-    float v[16];
-    dequant16(q0, s0, v);
-    Vec16<T>::store((T*)g.dst[l0] + e0, sub, v);
-    if (has1) {
-      dequant16(q1, s1, v);
-      Vec16<T>::store((T*)g.dst[l1] + e1, sub, v);
+#pragma unroll
+    for (int u = 0; u < kDecU; ++u) {
+      if (b0 + u * G >= total) continue;
+      bad |= not_finite(sv[u]);
+      float v[16];
+      dequant16(qv[u], sv[u], v);
+      Vec16<T>::store((T*)g.dst[lv[u]] + lbv[u] * kBlock, sub, v);
     }
   }
   report_bits(g.err, bad, GIFT_DEV_NONFINITE);
