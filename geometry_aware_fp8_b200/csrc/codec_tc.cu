@@ -66,7 +66,8 @@ constexpr int kSmemBytes = kStages * kStageBytes + kPcBytes + kCBufs * kCodesByt
 constexpr int enc_smem(bool cluster) { return kSmemBytes + (cluster ? kXBytes : 0); }
 constexpr int kThreads = 480;  // 8 epilogue + 4 converter + MMA + TMA load + TMA store warps
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColP = 256;
+constexpr uint32_t kColP = 256;  // two 64-column slots of P: panel parity
+constexpr int kLead = 3;         // first-pass steps that open a block (see Steps)
 GIFT_DEV uint32_t w_col(int b) { return 128u * (uint32_t)b; }
 constexpr uint32_t kIdescE1 = umma_idesc_bf16(128, 64, 0, 1);   // A K-major, B MN-major
 constexpr uint32_t kIdescE2 = umma_idesc_bf16(128, 128, 0, 0);  // both K-major
@@ -147,6 +148,10 @@ GIFT_DEV void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "
 // (chunks 0 .. nc-1); block k >= 1 is the second pass of p_{k-1} (chunks
 // nc-1 .. 0) interleaved step by step with the first pass of p_k, so that the
 // HBM stream of one panel overlaps the epilogue work of the previous one.
+// Each block opens with kLead first-pass steps: the second pass of p_{k-1}
+// needs P o c of p_{k-1}, which the epilogue forms only once the first pass
+// of p_{k-1} has completed, and the MMA issues p_k's first steps meanwhile
+// (the encoder keeps P in two TMEM slots, by panel parity).
 //
 // With a cluster of S CTAs sharing a panel list, CTA rank q runs chunks
 // [q nc / S, (q + 1) nc / S) of every panel (nc = d_in / 128 >= S); the step
@@ -167,7 +172,7 @@ struct Steps {
     n2 = k >= 1 && beg + k - 1 < end ? nc_of(beg + k - 1) : 0;
     pick();
   }
-  GIFT_DEV void pick() { pass = (i2 < n2 && (i1 >= n1 || i2 <= i1)) ? 1 : 0; }
+  GIFT_DEV void pick() { pass = (i2 < n2 && (i1 >= n1 || i1 >= i2 + kLead)) ? 1 : 0; }
   GIFT_DEV bool valid() const { return n1 + n2 > 0; }
   GIFT_DEV int slot() const { return pass ? beg + k - 1 : beg + k; }
   GIFT_DEV int job() const { return p.sched_ids[slot()] >> 8; }
@@ -366,6 +371,17 @@ GIFT_DEV void u_row_from_tile(uint32_t tile, int t, float (&u)[32]) {
     u[4 * q + 3] = __uint_as_float(v.w);
   }
 }
+// The transform's coefficients of the layer of schedule entry `it`, written by
+// one warp into a shared-memory slot of 33 floats: c_k / a = (rho / (lambda_k +
+// rho))^{1/2} - 1 for k < rank (0 beyond), then a = rho^{-1/2}.  Formed once per
+// panel, a block ahead of their use, off the path of the MMA's wait for P o c.
+GIFT_DEV void enc_coefs(const EncParams& p, int it, float* slot, int lane) {
+  const EncJob& J = p.jobs[p.sched_ids[it] >> 8];
+  const double rho = (double)__ldg(J.rho);
+  slot[lane] = lane < J.rank ? (float)(sqrt(rho / ((double)__ldg(J.lambda + lane) + rho)) - 1.0) : 0.0f;
+  if (lane == 0) slot[32] = (float)(1.0 / sqrt(rho));
+}
+
 template <int FMT, bool CLUSTER>
 __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __grid_constant__ EncParams p,
                                                                      uint32_t* err) {
@@ -381,7 +397,7 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
   uint64_t* full = bars;                  // [kStages] count 1: converter (stage ready for the MMA)
   uint64_t* empty = bars + kStages;       // [kStages] count 1: MMA commit
   uint64_t* tfull = bars + 2 * kStages;   // [kStages] count 1 + tx: TMA (G and fp32 U)
-  uint64_t* p_full = bars + 3 * kStages;  // count 1 (MMA commit)
+  uint64_t* p_full = bars + 3 * kStages;  // [2: p_full, p_full + 17] count 1 (MMA commit): P of a panel, by parity
   uint64_t* pc_full = p_full + 1;         // count 256 (epilogue)
   uint64_t* w_full = p_full + 2;          // [kWBufs] count 1
   uint64_t* w_empty = p_full + 5;         // [kWBufs] count 256
@@ -390,7 +406,7 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
   uint64_t* xfull = p_full + 14;          // count 256 (S-1): the peers' partials are written (clusters)
   uint64_t* xempty = p_full + 15;         // count 256 (S-1): the peers have read this CTA's partial
   uint64_t* stall = p_full + 16;          // count 1, never arrived at (test hook)
-  uint32_t* tmem_slot = (uint32_t*)(p_full + 17);
+  uint32_t* tmem_slot = (uint32_t*)(p_full + 18);
   __shared__ int failed;  // any role gave up (reported at exit)
   __shared__ int nonfin;  // a block maximum was not finite (reported at exit)
 
@@ -408,6 +424,7 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
       mbar_init(&tfull[s], 1);
     }
     mbar_init(p_full, 1);
+    mbar_init(p_full + 17, 1);
     mbar_init(pc_full, 256);
     mbar_init(stall, 1);
     for (int b = 0; b < 3; ++b) {
@@ -523,9 +540,10 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
       uint32_t step = 0, e2 = 0;
       for (Steps<EncParams> st(p, beg, end, q, S); st.valid() && !failed; st.next(), ++step) {
         const int s = step % kStages;
-        // block k >= 1 starts with the second pass of p_{k-1}: its P o (c/a) must be
-        // in shared memory, and P in TMEM has been read (it is reused for p_k)
-        if (st.block_start() && st.k >= 1 && !mbar_wait(pc_full, (st.k - 1) & 1u, kWaitLimit)) { failed = 1; break; }
+        // the second pass of p_{k-1} needs its P o (c/a) in shared memory; that
+        // also means P of p_{k-1} has been read from its TMEM slot, which the
+        // first pass of p_{k+1} reuses
+        if (st.pass == 1 && st.i2 == 0 && !mbar_wait(pc_full, (st.k - 1) & 1u, kWaitLimit)) { failed = 1; break; }
         if (!mbar_wait(p.presplit ? &tfull[s] : &full[s], (step / kStages) & 1u, kWaitLimit)) { failed = 1; break; }
         tc_fence_after();
         const uint32_t g_tile = sbase + s * kStageBytes, u_tile = g_tile + kGBytes;
@@ -538,10 +556,12 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
             for (int kk = 0; kk < 4; ++kk) {
               const uint64_t ad = umma_desc_sw128(g_tile + h * kGHalf + kk * 32, 16, 1024);
               const uint64_t bd = umma_desc_sw128(u_tile + (h * 64 + kk * 16) * 128, 16, 1024);
-              umma_bf16(tbase + kColP, ad, bd, kIdescE1, (c | h | kk) ? 1u : 0u);
+              umma_bf16(tbase + kColP + 64u * (st.k & 1), ad, bd, kIdescE1, (c | h | kk) ? 1u : 0u);
             }
           umma_commit(&empty[s]);
-          if (c == st.nc() - 1) umma_commit(p_full);
+          // one barrier per panel parity: the first pass of p_{k+1} may complete
+          // before the epilogue has waited for p_k's
+          if (c == st.nc() - 1) umma_commit((st.k & 1) ? p_full + 17 : p_full);
         } else {
           // E2: W/a [128 x 128] = Pc_hi U_hi^T + Pc_lo U_hi^T + Pc_hi U_lo^T + G . I
           // (Pc already divided by a; G . I adds G exactly, 16 columns per MMA)
@@ -577,9 +597,11 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
     // block maxima through shared memory and write their codes into one of two
     // codes tiles for the store warp.
     __shared__ float amax_x[2][128];
+    __shared__ float coefs[2][33];  // by panel parity: see enc_coefs
     const int h = warp >> 2;
     const int r = (warp & 3) * 32 + lane;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    if (warp == 0 && beg < end) enc_coefs(p, beg, coefs[0], lane);  // p_0 (read after a barrier)
     uint32_t e2 = 0, nx = 0;
     float a = 0.0f;
     float S_t = 0.0f;   // NVFP4 tensor scale (codes pass)
@@ -592,24 +614,23 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
       if (st.i2 == 0) {
         if (FMT == kFmtNvfp4) S_t = nvfp4_tensor_scale(__uint_as_float(*reinterpret_cast<volatile uint32_t*>(J.tscale)));
         // P o (c / a) of this panel for k = 16 h .. 16 h + 15, split into the bf16
-        // A operand of E2:  c_k / a = (rho / (lambda_k + rho))^{1/2} - 1
-        const double rho = (double)__ldg(J.rho);
-        a = (float)(1.0 / sqrt(rho));
-        float cf[16];
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          const int kk = 16 * h + k;
-          cf[k] = kk < J.rank ? (float)(sqrt(rho / ((double)__ldg(J.lambda + kk) + rho)) - 1.0) : 0.0f;
-        }
-        stop = named_sync_or(2, 256, !mbar_wait(p_full, (st.k - 1) & 1u, kWaitLimit));
+        // A operand of E2 (coefficients from the panel's slot, formed a block ago)
+        stop = named_sync_or(2, 256, !mbar_wait(((st.k - 1) & 1) ? p_full + 17 : p_full, ((st.k - 1) >> 1) & 1u,
+                                                kWaitLimit));
         if (stop) {
           failed = 1;
           break;
         }
+        const float* cs = coefs[(st.k - 1) & 1];
+        a = cs[32];
+        float cf[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) cf[k] = cs[16 * h + k];
         tc_fence_after();
         uint32_t ph[16], pl[16];
-        tmem_ld16(tbase + lane_off + kColP + 16 * h, ph);
-        tmem_ld16(tbase + lane_off + kColP + 32 + 16 * h, pl);
+        const uint32_t pcol = kColP + 64u * ((st.k - 1) & 1);  // P of p_{k-1}
+        tmem_ld16(tbase + lane_off + pcol + 16 * h, ph);
+        tmem_ld16(tbase + lane_off + pcol + 32 + 16 * h, pl);
         tmem_wait_ld();
         float pv[16];
 #pragma unroll
@@ -640,6 +661,8 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
         fence_async_shared();
         tc_fence_before();
         mbar_arrive(pc_full);
+        // the next panel's coefficients (its slot was last read a block ago)
+        if (warp == 0 && beg + st.k < end) enc_coefs(p, beg + st.k, coefs[st.k & 1], lane);
       }
       const int c = st.chunk();
       const int b = (int)(e2 % kWBufs);
@@ -793,6 +816,16 @@ GIFT_DEV uint32_t e4m3x2_to_f16x2(uint16_t v) {
   uint32_t h;
   asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(v));
   return h;
+}
+
+// As enc_coefs, for the inverse: c'_k = (lambda_k + rho)^{1/2} - rho^{1/2} for
+// k < rank (0 beyond), then a = rho^{1/2}.
+GIFT_DEV void dec_coefs(const DecParams& p, int it, float* slot, int lane) {
+  const DecJob& J = p.jobs[p.sched_ids[it] >> 8];
+  const double rho = (double)__ldg(J.rho);
+  const double a64 = sqrt(rho);
+  slot[lane] = lane < J.rank ? (float)(sqrt((double)__ldg(J.lambda + lane) + rho) - a64) : 0.0f;
+  if (lane == 0) slot[32] = (float)a64;
 }
 
 template <int FMT, bool CLUSTER>
@@ -1010,8 +1043,8 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
       uint32_t step = 0, e2 = 0, d2 = 0;
       for (Steps<DecParams> st(p, beg, end, q, S); st.valid() && !failed; st.next(), ++step) {
         const int s = step % kDStages, j = step & 1;
-        // block k >= 1 starts with D3 of p_{k-1}, which needs its P o c
-        if (st.block_start() && st.k >= 1 && !mbar_wait(pc_full, (st.k - 1) & 1u, kWaitLimit)) { failed = 1; break; }
+        // D3 of p_{k-1} needs its P o c, which the epilogue forms at the block's start
+        if (st.pass == 1 && st.i2 == 0 && !mbar_wait(pc_full, (st.k - 1) & 1u, kWaitLimit)) { failed = 1; break; }
         if (!mbar_wait(&full[s], (step / kDStages) & 1u, kWaitLimit)) { failed = 1; break; }
         const uint32_t u_tile = sbase + s * kDStageBytes + kDCodes;
         if (st.pass == 0) {
@@ -1062,6 +1095,8 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
     const int h = warp >> 2;
     const int r = (warp & 3) * 32 + lane;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    __shared__ float coefs[2][33];  // by panel parity: see dec_coefs
+    if (warp == 0 && beg < end) dec_coefs(p, beg, coefs[0], lane);  // p_0 (read after barriers)
     uint32_t step = 0, e2 = 0, d2 = 0, nx = 0;
     float P[16];
 #pragma unroll
@@ -1099,15 +1134,13 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
             break;
           }
         }
-        const double rho = (double)__ldg(J.rho);
-        const double a64 = sqrt(rho);
-        a = (float)a64;
+        // coefficients of p_{k-1} from its slot (formed a block ago)
+        const float* cs = coefs[(st.k - 1) & 1];
+        a = cs[32];
         uint32_t hi[8], lo[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-          const int k0 = 16 * h + 2 * k;
-          const float c0 = k0 < J.rank ? (float)(sqrt((double)__ldg(J.lambda + k0) + rho) - a64) : 0.0f;
-          const float c1 = k0 + 1 < J.rank ? (float)(sqrt((double)__ldg(J.lambda + k0 + 1) + rho) - a64) : 0.0f;
+          const float c0 = cs[16 * h + 2 * k], c1 = cs[16 * h + 2 * k + 1];
           float h0, l0, h1, l1;
           split_bf16(P[2 * k] * c0, h0, l0);
           split_bf16(P[2 * k + 1] * c1, h1, l1);
@@ -1120,6 +1153,8 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
         st_shared_v4(pc_tile + sw128(r, 5 + 2 * h), lo[4], lo[5], lo[6], lo[7]);
         fence_async_shared();
         mbar_arrive(pc_full);
+        // the next panel's coefficients (its slot was last read a block ago)
+        if (warp == 0 && beg + st.k < end) dec_coefs(p, beg + st.k, coefs[st.k & 1], lane);
       }
       if (st.pass == 0) {
         // D2 epilogue: P += s_c (T_hi + 2^-11 T_lo) for this half's 16 coefficients

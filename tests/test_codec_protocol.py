@@ -43,10 +43,14 @@ class Bar:
             self.pending, self.done = 0, self.done + 1
 
 
-def steps_of(ncs):
-    """(pass, block k, block start, index within the pass) of every step of a
-    CTA that owns panels with ncs chunks, in the kernels' interleaved order:
-    block k runs the first pass of panel k and the second pass of panel k-1."""
+LEAD = 3  # first-pass steps that open a block (kLead in codec_tc.cu)
+
+
+def steps_of(ncs, lead=LEAD):
+    """(pass, block k, block start, index within the pass, steps of the pass)
+    of every step of a CTA that owns panels with ncs chunks, in the kernels'
+    interleaved order: block k runs the first pass of panel k and the second
+    pass of panel k-1, opening with `lead` first-pass steps."""
     out, k = [], 0
     while True:
         n1 = ncs[k] if k < len(ncs) else 0
@@ -55,7 +59,7 @@ def steps_of(ncs):
             return out
         i1 = i2 = 0
         while i1 + i2 < n1 + n2:
-            second = i2 < n2 and (i1 >= n1 or i2 <= i1)
+            second = i2 < n2 and (i1 >= n1 or i1 >= i2 + lead)
             out.append((1 if second else 0, k, i1 + i2 == 0, i2 if second else i1, n2 if second else n1))
             if second:
                 i2 += 1
@@ -150,7 +154,7 @@ def decoder(ncs, rng, release_at_readiness=False, presplit=False, n_stages=4):
         e2 = d2 = 0
         for x, (ps, k, bs, i, n) in enumerate(seq):
             s, j = x % n_stages, x & 1
-            if bs and k >= 1:
+            if ps == 1 and i == 0:
                 yield from sim.wait("pcfull", k - 1)
             yield from sim.wait(f"full{s}", x // n_stages)
             if ps == 0:
@@ -260,12 +264,13 @@ def encoder(ncs, rng, presplit=False, n_stages=3):
     for j in range(2):
         for b in ("wfull", "wempty", "cready", "cfree"):
             sim.bar(f"{b}{j}")
-    sim.bar("pfull")
+    sim.bar("pfull0")
+    sim.bar("pfull1")
     sim.bar("pcfull")
     B = sim.B
     stage, stage_rd = [None] * n_stages, [0] * n_stages
     ctile = [None] * 2
-    P = {"panel": None}
+    P = [None, None]  # the panel whose P each TMEM slot holds (or is being written)
 
     def producer():
         for x in range(N):
@@ -296,14 +301,14 @@ def encoder(ncs, rng, presplit=False, n_stages=3):
         e2 = 0
         for x, (ps, k, bs, i, n) in enumerate(seq):
             s = x % n_stages
-            if bs and k >= 1:
+            if ps == 1 and i == 0:
                 yield from sim.wait("pcfull", k - 1)
             yield from sim.wait(f"{'tfull' if presplit else 'full'}{s}", x // n_stages)
             stage_rd[s] += 1
             if ps == 0:
                 last = i == n - 1
                 if i == 0:
-                    P["panel"] = k  # E1 of panel k starts overwriting P
+                    P[k & 1] = k  # E1 of panel k starts overwriting its slot
 
                 def done(x=x, s=s, last=last, k=k):
                     if stage[s] != x:
@@ -311,7 +316,7 @@ def encoder(ncs, rng, presplit=False, n_stages=3):
                     stage_rd[s] -= 1
                     B[f"empty{s}"].arrive()
                     if last:
-                        B["pfull"].arrive()
+                        B[f"pfull{k & 1}"].arrive()
                 sim.later(done)
             else:
                 b = e2 & 1
@@ -334,9 +339,9 @@ def encoder(ncs, rng, presplit=False, n_stages=3):
             if ps == 0:
                 continue
             if i == 0:
-                yield from sim.wait("pfull", k - 1)
-                if P["panel"] != k - 1:
-                    raise Fail(f"the epilogue read P of panel {P['panel']} for panel {k - 1}")
+                yield from sim.wait(f"pfull{(k - 1) & 1}", (k - 1) >> 1)
+                if P[(k - 1) & 1] != k - 1:
+                    raise Fail(f"the epilogue read P of panel {P[(k - 1) & 1]} for panel {k - 1}")
                 yield
                 B["pcfull"].arrive()
             b, cb = e2 & 1, e2 & 1
