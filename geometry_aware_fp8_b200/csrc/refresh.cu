@@ -197,17 +197,19 @@ __global__ void split_a_kernel(const __grid_constant__ RefBatch b) {
   }
 }
 
-// Y = A Q (d x d times d x m, m <= 64), fp32 on the CUDA cores.  128 x 64
-// output tiles (columns >= m idle), 8 x 4 outputs per thread; the k range of a
-// CTA is walked in steps of 16 through two shared-memory buffers, the next
-// step's A and Q values prefetched into registers while the current one is
-// used.  Each output is one fmaf chain in increasing k over its slice; the k
-// range is split into `ns` slices written to Yp[slice] (fixed order), which
-// consumers add in index order.
+// Y = A Q (d x d times d x m, m <= 64), fp32 on the CUDA cores.  128 x 16 CW
+// output tiles (CW = 3 for m <= 48, else 4; columns >= m idle), 8 x CW outputs
+// per thread; the k range of a CTA is walked in steps of 16 through two
+// shared-memory buffers, the next step's A and Q values prefetched into
+// registers while the current one is used.  Each output is one fmaf chain in
+// increasing k over its slice; the k range is split into `ns` slices written
+// to Yp[slice] (fixed order), which consumers add in index order.
 constexpr int kSkK = 32;   // k-slice granularity
 constexpr int kSkStep = 16;
 
+template <int CW>
 __global__ void __launch_bounds__(kRT) skinny_kernel(const __grid_constant__ RefBatch b, int src, int dst) {
+  constexpr int NC = 16 * CW;  // tile columns
   const RefLayer& Lr = b.L[blockIdx.z];
   const int d = Lr.d, m = b.m, kslice = Lr.kslice;
   if ((int)blockIdx.x >= d / 128 || (int)blockIdx.y >= Lr.ns) return;
@@ -215,34 +217,37 @@ __global__ void __launch_bounds__(kRT) skinny_kernel(const __grid_constant__ Ref
   const float* __restrict__ Q = Lr.buf[src];
   float* __restrict__ Yp = Lr.buf[dst];
   __shared__ __align__(16) float As[2][kSkStep][128 + 4];  // As[k][row]
-  __shared__ __align__(16) float Qs[2][kSkStep][64];
+  __shared__ __align__(16) float Qs[2][kSkStep][NC];
   const int row0 = blockIdx.x * 128;
   const int k_begin = blockIdx.y * kslice;
   const int k_end = min(d, k_begin + kslice);
-  const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;  // rows 8 ty.., columns 4 tx..
-  // loaders: A rows (t & 127), k (t >> 7) * 8 .. + 7; Q row k = t >> 4, columns 4 (t & 15) ..
+  const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;  // rows 8 ty.., columns CW tx..
+  // loaders: A rows (t & 127), k (t >> 7) * 8 .. + 7; Q row k = t / (NC / 4), columns 4 (t % (NC / 4)) ..
   const int ar = threadIdx.x & 127, ak = (threadIdx.x >> 7) * 8;
-  const int qk = threadIdx.x >> 4, qc = (threadIdx.x & 15) * 4;
-  float acc[8][4];
+  const bool qld = threadIdx.x < kSkStep * NC / 4;
+  const int qk = threadIdx.x / (NC / 4), qc = (threadIdx.x % (NC / 4)) * 4;
+  float acc[8][CW];
 #pragma unroll
   for (int a = 0; a < 8; ++a)
 #pragma unroll
-    for (int c = 0; c < 4; ++c) acc[a][c] = 0.0f;
+    for (int c = 0; c < CW; ++c) acc[a][c] = 0.0f;
   float4 ra0, ra1, rq;
   auto fetch = [&](int k0) {
     const float4* src4 = reinterpret_cast<const float4*>(A + (int64_t)(row0 + ar) * d + k0 + ak);
     ra0 = __ldg(src4);
     ra1 = __ldg(src4 + 1);
-    const float* qrow = Q + (int64_t)(k0 + qk) * m;
-    rq.x = qc + 0 < m ? __ldg(qrow + qc + 0) : 0.0f;
-    rq.y = qc + 1 < m ? __ldg(qrow + qc + 1) : 0.0f;
-    rq.z = qc + 2 < m ? __ldg(qrow + qc + 2) : 0.0f;
-    rq.w = qc + 3 < m ? __ldg(qrow + qc + 3) : 0.0f;
+    if (qld) {
+      const float* qrow = Q + (int64_t)(k0 + qk) * m;
+      rq.x = qc + 0 < m ? __ldg(qrow + qc + 0) : 0.0f;
+      rq.y = qc + 1 < m ? __ldg(qrow + qc + 1) : 0.0f;
+      rq.z = qc + 2 < m ? __ldg(qrow + qc + 2) : 0.0f;
+      rq.w = qc + 3 < m ? __ldg(qrow + qc + 3) : 0.0f;
+    }
   };
   auto stash = [&](int buf) {
     As[buf][ak + 0][ar] = ra0.x; As[buf][ak + 1][ar] = ra0.y; As[buf][ak + 2][ar] = ra0.z; As[buf][ak + 3][ar] = ra0.w;
     As[buf][ak + 4][ar] = ra1.x; As[buf][ak + 5][ar] = ra1.y; As[buf][ak + 6][ar] = ra1.z; As[buf][ak + 7][ar] = ra1.w;
-    *reinterpret_cast<float4*>(&Qs[buf][qk][qc]) = rq;
+    if (qld) *reinterpret_cast<float4*>(&Qs[buf][qk][qc]) = rq;
   };
   int buf = 0;
   if (k_begin < k_end) {
@@ -257,13 +262,22 @@ __global__ void __launch_bounds__(kRT) skinny_kernel(const __grid_constant__ Ref
     for (int kk = 0; kk < kSkStep; ++kk) {
       const float4 a0 = *reinterpret_cast<const float4*>(&As[buf][kk][ty * 8]);
       const float4 a1 = *reinterpret_cast<const float4*>(&As[buf][kk][ty * 8 + 4]);
-      const float4 q4 = *reinterpret_cast<const float4*>(&Qs[buf][kk][tx * 4]);
       const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-      const float qv[4] = {q4.x, q4.y, q4.z, q4.w};
+      float qv[CW];
+      if constexpr (CW == 4) {
+        const float4 q4 = *reinterpret_cast<const float4*>(&Qs[buf][kk][tx * 4]);
+        qv[0] = q4.x;
+        qv[1] = q4.y;
+        qv[2] = q4.z;
+        qv[3] = q4.w;
+      } else {
+#pragma unroll
+        for (int c = 0; c < CW; ++c) qv[c] = Qs[buf][kk][tx * CW + c];
+      }
 #pragma unroll
       for (int a = 0; a < 8; ++a)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) acc[a][c] = fmaf(av[a], qv[c], acc[a][c]);
+        for (int c = 0; c < CW; ++c) acc[a][c] = fmaf(av[a], qv[c], acc[a][c]);
     }
     if (more) stash(buf ^ 1);
     __syncthreads();
@@ -273,8 +287,8 @@ __global__ void __launch_bounds__(kRT) skinny_kernel(const __grid_constant__ Ref
 #pragma unroll
   for (int a = 0; a < 8; ++a)
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const int col = tx * 4 + c;
+    for (int c = 0; c < CW; ++c) {
+      const int col = tx * CW + c;
       if (col < m) out[(int64_t)(row0 + ty * 8 + a) * m + col] = acc[a][c];
     }
 }
@@ -481,6 +495,10 @@ __global__ void __launch_bounds__(kST) chol_kernel(const __grid_constant__ RefBa
 // (i, rg) computes column i of rows rg, rg + 4, ..., rg + 28 of the tile.
 // With dst == Q the bf16 [hi | lo] operand of the tensor-core product is
 // written too (columns m..63 zero).
+// fp64 shared memory of qr_apply_kernel: the m x m factor and one 32-row tile of
+// Y, both as doubles (Y converted once per element, not once per product)
+constexpr size_t kQrSmem = (64 * 65 + 32 * 65) * sizeof(double);
+
 __global__ void __launch_bounds__(kRT) qr_apply_kernel(const __grid_constant__ RefBatch bt, int src, int dst) {
   const RefLayer& Lr = bt.L[blockIdx.z];
   const int d = Lr.d, m = bt.m;
@@ -488,14 +506,15 @@ __global__ void __launch_bounds__(kRT) qr_apply_kernel(const __grid_constant__ R
   const double* __restrict__ X = Lr.Lf;
   float* __restrict__ Qo = Lr.buf[dst];
   __nv_bfloat16* __restrict__ Qs = dst == kBufQ ? Lr.Qs : nullptr;
-  __shared__ double Xs[64 * 65];
-  __shared__ float Ys[32 * 65];
+  extern __shared__ double qsm[];
+  double* Xs = qsm;            // [64][65]
+  double* Yd = qsm + 64 * 65;  // [32][65]
   if ((int64_t)blockIdx.x * 32 >= d) return;
   for (int e = threadIdx.x; e < m * m; e += kRT) Xs[(e / m) * 65 + e % m] = X[e];
   const int i = threadIdx.x & 63, rg = threadIdx.x >> 6;
   for (int64_t t0 = (int64_t)blockIdx.x * 32; t0 < d; t0 += (int64_t)gridDim.x * 32) {
     __syncthreads();
-    for (int e = threadIdx.x; e < 32 * m; e += kRT) Ys[(e / m) * 65 + e % m] = Yi[t0 * m + e];
+    for (int e = threadIdx.x; e < 32 * m; e += kRT) Yd[(e / m) * 65 + e % m] = (double)Yi[t0 * m + e];
     __syncthreads();
     double acc[8];
 #pragma unroll
@@ -504,7 +523,7 @@ __global__ void __launch_bounds__(kRT) qr_apply_kernel(const __grid_constant__ R
       for (int j = 0; j <= i; ++j) {
         const double x = Xs[i * 65 + j];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) acc[u] = fma(x, (double)Ys[(rg + 4 * u) * 65 + j], acc[u]);
+        for (int u = 0; u < 8; ++u) acc[u] = fma(x, Yd[(rg + 4 * u) * 65 + j], acc[u]);
       }
     }
 #pragma unroll
@@ -811,10 +830,11 @@ void refresh_plan(int64_t N, int64_t d, int rank, int oversample, bool a_out_giv
 }
 
 cudaError_t launch_refresh_batch(const RefreshPlan* plans, const RefreshIO* io, int n, cudaStream_t s) {
-  static unsigned long long chol_attr = 0, rr_attr = 0;
+  static unsigned long long chol_attr = 0, rr_attr = 0, qr_attr = 0;
   cudaError_t e = ensure_smem_attr(chol_kernel, (int)kCholSmem, &chol_attr);
   if (e != cudaSuccess) return e;
   if ((e = ensure_smem_attr(rr_kernel, (int)kRRSmem, &rr_attr)) != cudaSuccess) return e;
+  if ((e = ensure_smem_attr(qr_apply_kernel, (int)kQrSmem, &qr_attr)) != cudaSuccess) return e;
   if (n <= 0) return cudaSuccess;
   const int m = plans[0].m, r = plans[0].rank, iters = plans[0].iters;
   for (int base = 0; base < n; base += kMaxBatch) {
@@ -888,7 +908,7 @@ cudaError_t launch_refresh_batch(const RefreshPlan* plans, const RefreshIO* io, 
     auto cholqr_pass = [&](int src, int dst) {
       gram_partial_kernel<<<g_gram, kRT, 0, s>>>(B, src, src);
       chol_kernel<<<g_one, kST, kCholSmem, s>>>(B);
-      qr_apply_kernel<<<g_qr, kRT, 0, s>>>(B, src, dst);
+      qr_apply_kernel<<<g_qr, kRT, kQrSmem, s>>>(B, src, dst);
     };
     // A Q into Y, k-slices folded into slice 0: fp32 CUDA cores, or for the
     // iteration products (tc) the tensor cores on the bf16 split operands
@@ -913,7 +933,10 @@ cudaError_t launch_refresh_batch(const RefreshPlan* plans, const RefreshIO* io, 
         if (tc_nsmax > 1) fold_slices_kernel<<<g_ew, kRT, 0, s>>>(B, kBufY);
         for (int l = 0; l < cnt; ++l) B.L[l].ns = plans[base + l].skinny_slices;
       } else {
-        skinny_kernel<<<g_skinny, kRT, 0, s>>>(B, kBufQ, kBufY);
+        if (m <= 48)
+          skinny_kernel<3><<<g_skinny, kRT, 0, s>>>(B, kBufQ, kBufY);
+        else
+          skinny_kernel<4><<<g_skinny, kRT, 0, s>>>(B, kBufQ, kBufY);
         if (nsmax > 1) fold_slices_kernel<<<g_ew, kRT, 0, s>>>(B, kBufY);
       }
     };
