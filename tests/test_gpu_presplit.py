@@ -17,7 +17,7 @@ import torch
 from oracle import gift_oracle as O
 from geometry_aware_fp8_b200 import ops
 
-from _cmp import check_codes, check_scales
+from _cmp import check_codes, check_rows, check_scales
 from test_gpu_codec import _factor, _g, _to_dev
 
 pytestmark = pytest.mark.gpu
@@ -86,8 +86,13 @@ def test_grouped_codec_with_presplit_u_is_bit_identical(shapes):
         assert torch.equal(a.codes, b.codes)
         assert torch.equal(a.scales, b.scales)
         assert torch.equal(a.G_hat.view(torch.int16), b.G_hat.view(torch.int16))
-    # and one whitened layer against the oracle directly
+    # and one whitened layer against the oracle directly, both directions
     (d_out, d_in, rank), (G, _, _, _, _, (U, lam, rho)) = shapes[0], data[0]
-    c_o, s_o = O.encode_e4m3(G.astype(np.float64), U.astype(np.float64), lam.astype(np.float64), float(rho))
-    check_codes(runs[True][0].codes.cpu().numpy(), c_o)
-    check_scales(runs[True][0].scales.cpu().numpy(), s_o)
+    U64, lam64 = U.astype(np.float64), lam.astype(np.float64)
+    c_o, s_o = O.encode_e4m3(G.astype(np.float64), U64, lam64, float(rho))
+    codes = runs[True][0].codes.cpu().numpy()
+    scales = runs[True][0].scales.cpu().numpy()
+    check_codes(codes, c_o)
+    check_scales(scales, s_o)
+    want = O.decode_e4m3(codes, scales, U64, lam64, float(rho))
+    check_rows(runs[True][0].G_hat.float().cpu().numpy(), want, bf16=True)
