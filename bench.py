@@ -436,13 +436,13 @@ def buffer_set(ops, W, G_all, Gh_all):
 # elements.  Valid only for the kernel source it was taken on (sha256 of the
 # file); otherwise the bench reports traffic as null.
 TRAFFIC = {
-    "decode_whitened": {"read_per_element": 1.490519, "l2_write_per_element": 2.000000,
-                        "dram_write_per_element": 1.145404, "profile": "profiles/whiten_decode_tc_stack8.md"},
-    "encode_whitened": {"read_per_element": 2.908292, "l2_write_per_element": 1.250000,
-                        "dram_write_per_element": 0.317571, "profile": "profiles/whiten_encode_tc_stack8.md"},
+    "decode_whitened": {"read_per_element": 1.447617, "l2_write_per_element": 2.000000,
+                        "dram_write_per_element": 1.145445, "profile": "profiles/whiten_decode_tc_stack8.md"},
+    "encode_whitened": {"read_per_element": 2.936679, "l2_write_per_element": 1.250000,
+                        "dram_write_per_element": 0.229733, "profile": "profiles/whiten_encode_tc_stack8.md"},
 }
 TRAFFIC_SOURCE = ("geometry_aware_fp8_b200/csrc/codec_tc.cu",
-                  "58dd7b7eb2cc9759872399244891ace3e6ae0c512523c1577496a1e3fd8cb782")
+                  "dff908fb504a3cd582883528dae5bcb63e835993d8a3652d1952aa8f8d615f4e")
 
 
 def traffic_for(phase, n_elements, alg_read, alg_write):
