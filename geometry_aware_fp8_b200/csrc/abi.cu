@@ -80,7 +80,7 @@ const char* gift_status_string(gift_status s) {
   return "GIFT_ERR_UNKNOWN";
 }
 
-int gift_version(void) { return 100; }
+int gift_version(void) { return GIFT_VERSION; }
 
 // ---------------------------------------------------------------------------
 gift_status gift_refresh_workspace_size(int64_t N, int64_t d_in, int rank, int oversample, int a_out_given,

@@ -85,7 +85,11 @@ typedef enum { GIFT_F32 = 0, GIFT_BF16 = 1 } gift_dtype;
 
 const char* gift_status_string(gift_status s);
 
-/* Library version, e.g. 100 for 0.1.0. */
+/* Library version, e.g. 200 for 0.2.0.  GIFT_VERSION is the version this
+ * header describes; a caller can compare it with gift_version() at run time
+ * (0.2.0: dev_status on every codec call, gift_layer.U_split, gift_split_u,
+ * the dense-transform and decode-and-sum calls). */
+#define GIFT_VERSION 200
 int gift_version(void);
 
 /* ------------------------------------------------------------------------
