@@ -1049,7 +1049,9 @@ def run_reference(args):
               f"{K_REFRESH} steps; {wall:.1f} s")
     cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample, "cpu_model": cpu_model(),
            "refresh_s_per_group": t_ref / steps, "codec_s_per_group": t_codec / steps}
-    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": 0, "steps": steps,
+    # n_gpus: the N this arm was launched for (it runs on rank 0's host cores)
+    n_launch = int(os.environ.get("WORLD_SIZE", str(args.gpus)))
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": n_launch, "steps": steps,
             "warmup": warm, "ms_per_step": (t_codec + t_ref / K_REFRESH) / steps * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": WORKLOAD, "sample": sample},
