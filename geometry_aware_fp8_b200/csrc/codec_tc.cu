@@ -766,25 +766,27 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_encode_tc_kernel(const __g
 //       fp32 (f16 widening is one instruction per pair of codes).
 //   D3  G_hat = a W_hat + (P o c) U^T   (M=128, N=128 per chunk, K=32, bf16
 //       split as in the encoder), bf16 output with round-to-nearest-even.
-// Stage (4-deep ring) = codes tile (TMA, [128][128 B], 128-byte swizzle) + U
-// tile (split to f16 for D2, to bf16 for D3).  Two scratch tiles, taken in
-// step order, hold a D2 step's f16 codes (the A operand, written by the
-// converter warps, free when the MMA completes) or a D3 step's bf16 output
-// (free once the TMA stores have read it).  A D3 stage is released as soon as
-// every epilogue thread has read its codes.  That release order also keeps
-// the converter warps, which wait on a scratch tile only in D2 steps, within
-// one phase of the tile's barrier: were D3 stages released at MMA completion,
-// the converters could run two uses ahead and pass a parity wait early.
+// Stage (ring of kDStages) = codes tile (TMA, [128][128 B], 128-byte swizzle)
+// + U tile (split to f16 for D2, to bf16 for D3).  D2's A operand, the step's
+// codes widened to f16, lives in TMEM: the converter warps write it with
+// tcgen05.st into one of two 64-column tiles (row r in lane r), freed when
+// the MMA that read it completes.  D3's bf16 output goes through kDOut
+// shared-memory tiles, written by the epilogue and freed once the TMA stores
+// have read them.  A first-pass stage is released by the D2 commit; a
+// second-pass stage as soon as every epilogue thread holds its codes in
+// registers (D3, which reads the stage's U, has completed by then).
 // ===========================================================================
 constexpr int kDStages = 4;                         // decode ring
+constexpr int kDOut = 2;                            // output tiles
 constexpr int kDCodes = kPanel * kChunk;            // 16 KB
 constexpr int kDStageBytes = kDCodes + kUBytes;     // codes + U
-constexpr int kDScratch = kPanel * kChunk * 2;      // 32 KB: two [128][64] 16-bit boxes
-constexpr int kDSmemBytes = kDStages * kDStageBytes + 2 * kDScratch + kPcBytes + 1024 + 512;
+constexpr int kDOutBytes = kPanel * kChunk * 2;     // 32 KB: two [128][64] bf16 boxes
+constexpr int kDSmemBytes = kDStages * kDStageBytes + kDOut * kDOutBytes + kPcBytes + 1024 + 512;
 constexpr int dec_smem(bool cluster) { return kDSmemBytes + (cluster ? kXBytes : 0); }
 static_assert(dec_smem(true) <= 232448, "decode shared memory");
 static_assert(enc_smem(true) <= 232448, "encode shared memory");
-constexpr uint32_t kColT0 = 256, kColT1 = 320;
+constexpr uint32_t kColT0 = 256, kColT1 = 320;  // D2 accumulators (D3's are w_col(0), w_col(1))
+constexpr uint32_t kColA = 384;                 // two 64-column D2 A tiles: 128 f16 codes per lane
 constexpr uint32_t kIdescD2 = umma_idesc_f16(128, 64, 0, 1);   // D2 runs on f16 operands
 
 struct alignas(64) DecJob {
@@ -834,15 +836,16 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const uint32_t sbase = smem_u32(smem);
-  const uint32_t scr = sbase + kDStages * kDStageBytes;  // [2] scratch tiles: two [128][64] 16-bit boxes each
-  const uint32_t pc_tile = scr + 2 * kDScratch;
+  const uint32_t otile = sbase + kDStages * kDStageBytes;  // [kDOut] output tiles: two [128][64] bf16 boxes each
+  const uint32_t pc_tile = otile + kDOut * kDOutBytes;
   const uint32_t xbuf = pc_tile + kPcBytes;  // [128][32] fp32 partial P (CLUSTER only)
-  uint64_t* bars = (uint64_t*)(smem + kDStages * kDStageBytes + 2 * kDScratch + kPcBytes + (CLUSTER ? kXBytes : 0));
-  uint64_t* full = bars;                   // [kDStages] count 1: converter (U split; first pass: codes widened)
+  uint64_t* bars = (uint64_t*)(smem + kDStages * kDStageBytes + kDOut * kDOutBytes + kPcBytes + (CLUSTER ? kXBytes : 0));
+  uint64_t* full = bars;                   // [kDStages] count 1: converter (U split; first pass: A tile written)
   uint64_t* cfull = bars + kDStages;       // [kDStages] count 1 + tx: TMA (codes and U)
-  uint64_t* empty = bars + 2 * kDStages;   // [kDStages] count 1: MMA commit (D2) or store warp (D3)
-  uint64_t* sfree = bars + 3 * kDStages;   // [2] count 1: scratch tile free (MMA commit or store read)
-  uint64_t* oready = sfree + 2;            // [2] count 256: output tile written
+  uint64_t* empty = bars + 2 * kDStages;   // [kDStages] count 1: MMA commit (D2) or epilogue (D3, codes read)
+  uint64_t* afree = bars + 3 * kDStages;   // [2] count 1: TMEM A tile free (MMA commit)
+  uint64_t* ofree = afree + 2;             // [kDOut <= 2] count 1: output tile stored (store warp)
+  uint64_t* oready = ofree + 2;            // [kDOut <= 2] count 256: output tile written
   uint64_t* t_full = oready + 2;           // [2] count 1
   uint64_t* t_empty = t_full + 2;          // [2] count 256
   uint64_t* pc_full = t_full + 4;          // count 256
@@ -869,10 +872,13 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&sfree[b], 1);
-      mbar_init(&oready[b], 256);
+      mbar_init(&afree[b], 1);
       mbar_init(&t_full[b], 1);
       mbar_init(&t_empty[b], 256);
+    }
+    for (int o = 0; o < kDOut; ++o) {
+      mbar_init(&ofree[o], 1);
+      mbar_init(&oready[o], 256);
     }
     for (int b = 0; b < 3; ++b) {
       mbar_init(&w_full[b], 1);
@@ -931,56 +937,51 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
     }
   } else if (warp == 14) {
     // ---------------- output stores: a second-pass step's tile leaves by two TMA stores ----------------
-    // The epilogue has read the step's codes from its stage when the tile is
-    // ready; the stage and the scratch tile are released once the stores
-    // have read the tile.  Releasing the stage only then keeps the protocol
-    // safe: the converters, which wait for a scratch tile only in first-pass
-    // steps, cannot reach a step whose tile still has an earlier second-pass
-    // use unstored (with the stage released at the tile's readiness, a CPU
-    // simulation of the protocol found schedules of mixed panel lengths where
-    // their parity wait on the tile passed two phases early).
     if (lane == 0) {
       const uint64_t drop = policy_evict_first();
-      uint32_t step = 0, par = 0;  // par: bit j = phase parity of oready[j]
-      for (Steps<DecParams> st(p, beg, end, q, S); st.valid() && !failed; st.next(), ++step) {
+      uint32_t e2 = 0;  // second-pass steps so far
+      for (Steps<DecParams> st(p, beg, end, q, S); st.valid() && !failed; st.next()) {
         if (st.pass == 0) continue;
-        const int s = step % kDStages, j = step & 1;
-        if (!mbar_wait(&oready[j], (par >> j) & 1u, kWaitLimit)) {
+        const int o = (int)(e2 % kDOut);
+        if (!mbar_wait(&oready[o], (e2 / kDOut) & 1u, kWaitLimit)) {
           failed = 1;
           break;
         }
         const DecJob& J = p.jobs[st.job()];
-        const uint32_t o_tile = scr + j * kDScratch;
+        const uint32_t o_tile = otile + o * kDOutBytes;
         tma_store_2d_hint(&J.tmO, o_tile, st.chunk() * kChunk, st.panel() * kPanel, drop);
         tma_store_2d_hint(&J.tmO, o_tile + kGHalf, st.chunk() * kChunk + 64, st.panel() * kPanel, drop);
         bulk_commit();
         bulk_wait_read<0>();
-        par ^= 1u << j;
-        mbar_arrive(&empty[s]);
-        mbar_arrive(&sfree[j]);
+        mbar_arrive(&ofree[o]);
+        ++e2;
       }
       bulk_wait_all();
     }
   } else if (warp >= 8 && warp < 12) {
-    // ---------------- converters: U split in place; first pass: codes widened into a scratch tile ----------------
+    // ---------------- converters: U split in place; first pass: codes widened into a TMEM A tile ----------------
     // With a pre-split U, first-pass stages need only the codes widened and
     // second-pass stages nothing; the converters still take every stage in
-    // turn, so their waits on the stages never fall a phase behind the ring.
-    const int t = threadIdx.x - 256;
-    uint32_t step = 0;
+    // turn, so their waits on the stages never fall a phase behind the ring
+    // (a stage is reloaded only after the MMA has taken it, and the MMA
+    // takes it after the converters).
+    const int t = threadIdx.x - 256;  // row t = TMEM lane t (warps 8-11 own lane quarters 0-3)
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    uint32_t step = 0, d2 = 0;
     for (Steps<DecParams> st(p, beg, end, q, S); st.valid(); st.next(), ++step) {
-      const int s = step % kDStages, j = step & 1;
+      const int s = step % kDStages, a = d2 & 1;
       const uint32_t use = step / kDStages;
       float u[32];
       bool ok = mbar_wait(&cfull[s], use & 1u, kWaitLimit);
-      if (st.pass == 0 && step >= 2) ok = ok && mbar_wait(&sfree[j], ((step >> 1) - 1) & 1u, kWaitLimit);
+      if (st.pass == 0 && d2 >= 2) ok = ok && mbar_wait(&afree[a], ((d2 >> 1) - 1) & 1u, kWaitLimit);
       if (named_sync_or(1, 128, !ok)) {
         failed = 1;
         break;
       }
+      tc_fence_after();  // the MMA that read A tile a has completed
       const uint32_t c_tile = sbase + s * kDStageBytes;
       const uint32_t u_tile = c_tile + kDCodes;
-      const uint32_t q_tile = scr + j * kDScratch;
+      const uint32_t a_tile = tbase + lane_off + kColA + 64u * (uint32_t)a;  // columns: f16 pairs of row t
       // D2 multiplies f16 codes by an f16 split of U, D3 the bf16 P' o c' by a bf16 split
       if (!p.presplit) {
         u_row_from_tile(u_tile, t, u);
@@ -1011,9 +1012,7 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
           uint32_t o[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i) o[i] = pack_f16x2(v[2 * i], v[2 * i + 1]);
-          const int c0 = 2 * b, c1 = 2 * b + 1;  // 16-byte chunks of the 256-byte f16 row
-          st_shared_v4(q_tile + (c0 >> 3) * kGHalf + sw128(t, c0 & 7), o[0], o[1], o[2], o[3]);
-          st_shared_v4(q_tile + (c1 >> 3) * kGHalf + sw128(t, c1 & 7), o[4], o[5], o[6], o[7]);
+          tmem_st8(a_tile + 8u * b, o);  // columns 16 b .. 16 b + 15 of the chunk
         }
       } else if (st.pass == 0) {
         // the codes of row t, widened to f16
@@ -1027,13 +1026,15 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
             o[2 * e] = e4m3x2_to_f16x2((uint16_t)(w[e] & 0xFFFFu));
             o[2 * e + 1] = e4m3x2_to_f16x2((uint16_t)(w[e] >> 16));
           }
-          // 16 codes -> 32 bytes of f16 = chunks 2q, 2q+1 of the 256-byte row
-          const int c0 = 2 * q, c1 = 2 * q + 1;
-          st_shared_v4(q_tile + (c0 >> 3) * kGHalf + sw128(t, c0 & 7), o[0], o[1], o[2], o[3]);
-          st_shared_v4(q_tile + (c1 >> 3) * kGHalf + sw128(t, c1 & 7), o[4], o[5], o[6], o[7]);
+          tmem_st8(a_tile + 8u * q, o);  // codes 16 q .. 16 q + 15 = TMEM columns 8 q .. 8 q + 7
         }
       }
-      fence_async_shared();
+      if (st.pass == 0) {
+        tmem_wait_st();
+        ++d2;
+      }
+      tc_fence_before();
+      fence_async_shared();  // the in-place U split, for the MMA
       named_sync(1, 128);
       if (t == 0) mbar_arrive(&full[s]);
     }
@@ -1042,7 +1043,7 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
     if (lane == 0) {
       uint32_t step = 0, e2 = 0, d2 = 0;
       for (Steps<DecParams> st(p, beg, end, q, S); st.valid() && !failed; st.next(), ++step) {
-        const int s = step % kDStages, j = step & 1;
+        const int s = step % kDStages;
         // D3 of p_{k-1} needs its P o c, which the epilogue forms at the block's start
         if (st.pass == 1 && st.i2 == 0 && !mbar_wait(pc_full, (st.k - 1) & 1u, kWaitLimit)) { failed = 1; break; }
         if (!mbar_wait(&full[s], (step / kDStages) & 1u, kWaitLimit)) { failed = 1; break; }
@@ -1052,18 +1053,15 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
           const int b = d2 & 1;
           if (d2 >= 2 && !mbar_wait(&t_empty[b], ((d2 >> 1) - 1) & 1u, kWaitLimit)) { failed = 1; break; }
           tc_fence_after();
-          const uint32_t q_tile = scr + j * kDScratch;
+          const uint32_t a_tile = tbase + kColA + 64u * (uint32_t)b;  // the converters' A tile d2 & 1
           const uint32_t d = tbase + (b ? kColT1 : kColT0);
 #pragma unroll
-          for (int h = 0; h < 2; ++h)
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t ad = umma_desc_sw128(q_tile + h * kGHalf + kk * 32, 16, 1024);
-              const uint64_t bd = umma_desc_sw128(u_tile + (h * 64 + kk * 16) * 128, 16, 1024);
-              umma_bf16(d, ad, bd, kIdescD2, (h | kk) ? 1u : 0u);
-            }
+          for (int kc = 0; kc < 8; ++kc) {  // K = 16 kc .. 16 kc + 15: A columns 8 kc .., U rows 16 kc ..
+            const uint64_t bd = umma_desc_sw128(u_tile + kc * 16 * 128, 16, 1024);
+            umma_f16_tmem_a(d, a_tile + 8u * kc, bd, kIdescD2, kc ? 1u : 0u);
+          }
           umma_commit(&empty[s]);
-          umma_commit(&sfree[j]);
+          umma_commit(&afree[b]);
           umma_commit(&t_full[b]);
           ++d2;
         } else {
@@ -1091,7 +1089,7 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
     // coefficients k = 16 h .. 16 h + 15, in D3 the columns 64 h .. 64 h + 63
     // of every 128-column chunk (h = warp / 4).  P of the panel in its first
     // pass stays in registers until the block that starts its second pass;
-    // D3 writes its bf16 tile into the step's scratch tile for the store warp.
+    // D3 writes its bf16 tile into an output tile for the store warp.
     const int h = warp >> 2;
     const int r = (warp & 3) * 32 + lane;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
@@ -1115,7 +1113,7 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
     Steps<DecParams> ahead(p, beg, end, q, S);
     float sc_next = ahead.valid() ? scale_of(ahead) : 0.0f;
     for (Steps<DecParams> st(p, beg, end, q, S); st.valid() && !stop; st.next(), ++step) {
-      const int s = step % kDStages, j = step & 1;
+      const int s = step % kDStages;
       const DecJob& J = p.jobs[st.job()];
       const int c = st.chunk();
       const int64_t row = (int64_t)st.panel() * kPanel + r;
@@ -1182,20 +1180,27 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
         if (not_finite(sc)) nonfin = 1;
         ++d2;
       } else {
-        // D3 epilogue: G_hat = a s q + acc, into scratch tile j once its previous use is stored
-        const int b = (int)(e2 % kWBufs);
+        // D3 epilogue: G_hat = a s q + acc, into output tile o once its previous use is stored.
+        // The stage is released as soon as every thread holds its 64 codes.
+        const int b = (int)(e2 % kWBufs), o = (int)(e2 % kDOut);
         bool ok = mbar_wait(&w_full[b], (e2 / kWBufs) & 1u, kWaitLimit) &&
                   mbar_wait(&cfull[s], (step / kDStages) & 1u, kWaitLimit);
-        if (step >= 2) ok = ok && mbar_wait(&sfree[j], ((step >> 1) - 1) & 1u, kWaitLimit);
+        if (e2 >= kDOut) ok = ok && mbar_wait(&ofree[o], ((e2 / kDOut) - 1) & 1u, kWaitLimit);
+        const uint32_t c_tile = sbase + s * kDStageBytes;
+        uint4 cv[4];  // E4M3: codes 64 h + 16 i .. + 15 of this row (in bounds whatever the waits gave)
+        if (FMT == kFmtE4M3) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) cv[i] = ld_shared_v4(c_tile + sw128(r, 4 * h + i));
+        }
         stop = named_sync_or(2, 256, !ok);
         if (stop) {
           failed = 1;
           break;
         }
+        if (threadIdx.x == 0) mbar_arrive(&empty[s]);
         tc_fence_after();
         const uint32_t wcol = tbase + lane_off + w_col(b) + 64 * h;
-        const uint32_t c_tile = sbase + s * kDStageBytes;
-        const uint32_t o_tile = scr + j * kDScratch;  // two [128][64] bf16 boxes, 128-byte swizzle
+        const uint32_t o_tile = otile + o * kDOutBytes;  // two [128][64] bf16 boxes, 128-byte swizzle
         const float as = a * sc;
         if (not_finite(sc)) nonfin = 1;
 #pragma unroll
@@ -1208,7 +1213,7 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
           if (FMT == kFmtE4M3) {
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
-              const uint4 v = ld_shared_v4(c_tile + sw128(r, 4 * h + 2 * g2 + hh));
+              const uint4 v = cv[2 * g2 + hh];
               const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
@@ -1245,7 +1250,7 @@ __global__ void __launch_bounds__(kThreads, 1) whiten_decode_tc_kernel(const __g
         tc_fence_before();
         mbar_arrive(&w_empty[b]);
         fence_async_shared();
-        mbar_arrive(&oready[j]);
+        mbar_arrive(&oready[o]);
         ++e2;
       }
     }

@@ -105,21 +105,29 @@ class Sim:
                 del alive[pick]
 
 
-def decoder(ncs, rng, release_at_readiness=False, presplit=False, n_stages=4):
-    """The decoder: D2 (first pass) and D3 (second pass), four stages, two
-    scratch tiles taken as j = step & 1, two TMEM buffers per kind."""
+def decoder(ncs, rng, n_stages=4, n_out=2, release_at_mma=False):
+    """The decoder: D2 (first pass) and D3 (second pass).  The converters widen
+    a first-pass step's codes into one of two TMEM A tiles (their own, freed by
+    the MMA commit); the epilogue writes a second-pass step's output into one of
+    `n_out` shared-memory tiles (freed once the TMA stores have read them) and
+    releases the step's stage as soon as it has read the codes."""
     seq, sim = steps_of(ncs), Sim(rng)
     N = len(seq)
     for s in range(n_stages):
         for b in ("full", "cfull", "empty"):
             sim.bar(f"{b}{s}")
     for j in range(2):
-        for b in ("sfree", "oready", "tfull", "tempty", "wfull", "wempty"):
+        for b in ("afree", "tfull", "tempty", "wfull", "wempty"):
             sim.bar(f"{b}{j}")
+    for o in range(n_out):
+        sim.bar(f"ofree{o}")
+        sim.bar(f"oready{o}")
     sim.bar("pcfull")
     B = sim.B
     stage, stage_rd = [None] * n_stages, [0] * n_stages
-    tile, tile_rd = [None] * 2, [0] * 2
+    atile, atile_rd = [None] * 2, [0] * 2
+    otile, otile_rd = [None] * n_out, [0] * n_out
+    pc, pc_rd = [None], [0]
 
     def producer():
         for x in range(N):
@@ -136,42 +144,48 @@ def decoder(ncs, rng, release_at_readiness=False, presplit=False, n_stages=4):
             yield
 
     def converters():
+        d2 = 0
         for x, (ps, k, bs, i, n) in enumerate(seq):
-            s, j = x % n_stages, x & 1
+            s = x % n_stages
             yield from sim.wait(f"cfull{s}", x // n_stages)
-            if ps == 0 and x >= 2:
-                yield from sim.wait(f"sfree{j}", (x >> 1) - 1)
             if stage[s] != x:
-                raise Fail(f"converters read stage {s} holding step {stage[s]} at step {x}")
+                raise Fail(f"converters took stage {s} holding step {stage[s]} at step {x}")
             if ps == 0:
-                if tile_rd[j]:
-                    raise Fail(f"converters overwrote tile {j} while it was read")
-                tile[j] = ("wide", x)
+                a = d2 & 1
+                if d2 >= 2:
+                    yield from sim.wait(f"afree{a}", (d2 >> 1) - 1)
+                stage_rd[s] += 1
+                yield
+                stage_rd[s] -= 1
+                if atile_rd[a]:
+                    raise Fail(f"converters overwrote A tile {a} while the MMA read it")
+                atile[a] = x
+                d2 += 1
             yield
             B[f"full{s}"].arrive()
 
     def mma():
         e2 = d2 = 0
         for x, (ps, k, bs, i, n) in enumerate(seq):
-            s, j = x % n_stages, x & 1
+            s = x % n_stages
             if ps == 1 and i == 0:
                 yield from sim.wait("pcfull", k - 1)
             yield from sim.wait(f"full{s}", x // n_stages)
             if ps == 0:
-                b = d2 & 1
+                b = a = d2 & 1
                 if d2 >= 2:
                     yield from sim.wait(f"tempty{b}", (d2 >> 1) - 1)
-                if tile[j] != ("wide", x):
-                    raise Fail(f"D2 read tile {j} holding {tile[j]} at step {x}")
+                if atile[a] != x:
+                    raise Fail(f"D2 read A tile {a} holding {atile[a]} at step {x}")
                 stage_rd[s] += 1
-                tile_rd[j] += 1
+                atile_rd[a] += 1
 
-                def done(x=x, s=s, j=j, b=b):
-                    if stage[s] != x or tile[j] != ("wide", x):
+                def done(x=x, s=s, a=a, b=b):
+                    if stage[s] != x or atile[a] != x:
                         raise Fail("a D2 operand changed under the MMA")
                     stage_rd[s] -= 1
-                    tile_rd[j] -= 1
-                    for name in (f"empty{s}", f"sfree{j}", f"tfull{b}"):
+                    atile_rd[a] -= 1
+                    for name in (f"empty{s}", f"afree{a}", f"tfull{b}"):
                         B[name].arrive()
                 sim.later(done)
                 d2 += 1
@@ -179,13 +193,19 @@ def decoder(ncs, rng, release_at_readiness=False, presplit=False, n_stages=4):
                 b = e2 & 1
                 if e2 >= 2:
                     yield from sim.wait(f"wempty{b}", (e2 >> 1) - 1)
+                if pc[0] != k - 1:
+                    raise Fail(f"D3 of panel {k - 1} read P o c of panel {pc[0]}")
                 stage_rd[s] += 1
+                pc_rd[0] += 1
 
-                def done(x=x, s=s, b=b):
-                    if stage[s] != x:
+                def done(x=x, s=s, b=b, k=k):
+                    if stage[s] != x or pc[0] != k - 1:
                         raise Fail("a D3 operand changed under the MMA")
                     stage_rd[s] -= 1
+                    pc_rd[0] -= 1
                     B[f"wfull{b}"].arrive()
+                    if release_at_mma:
+                        B[f"empty{s}"].arrive()
                 sim.later(done)
                 e2 += 1
             yield
@@ -193,8 +213,11 @@ def decoder(ncs, rng, release_at_readiness=False, presplit=False, n_stages=4):
     def epilogue():
         e2 = d2 = 0
         for x, (ps, k, bs, i, n) in enumerate(seq):
-            s, j = x % n_stages, x & 1
+            s = x % n_stages
             if bs and k >= 1:
+                if pc_rd[0]:
+                    raise Fail("the epilogue overwrote P o c while D3 read it")
+                pc[0] = k - 1
                 B["pcfull"].arrive()
             if ps == 0:
                 b = d2 & 1
@@ -203,51 +226,50 @@ def decoder(ncs, rng, release_at_readiness=False, presplit=False, n_stages=4):
                 B[f"tempty{b}"].arrive()
                 d2 += 1
                 continue
-            b = e2 & 1
+            b, o = e2 & 1, e2 % n_out
             yield from sim.wait(f"wfull{b}", e2 >> 1)
             yield from sim.wait(f"cfull{s}", x // n_stages)
-            if x >= 2:
-                yield from sim.wait(f"sfree{j}", (x >> 1) - 1)
+            if e2 >= n_out:
+                yield from sim.wait(f"ofree{o}", e2 // n_out - 1)
             if stage[s] != x:
                 raise Fail(f"the epilogue read codes of step {stage[s]} at step {x}")
             stage_rd[s] += 1
             yield
+            if stage[s] != x:
+                raise Fail(f"the codes of step {x} changed while the epilogue read them")
             stage_rd[s] -= 1
-            if tile_rd[j]:
-                raise Fail(f"the epilogue overwrote tile {j} while it was read")
-            tile[j] = ("out", x)
+            if not release_at_mma:
+                B[f"empty{s}"].arrive()
+            yield
+            if otile_rd[o]:
+                raise Fail(f"the epilogue overwrote output tile {o} while it was stored")
+            otile[o] = x
             B[f"wempty{b}"].arrive()
-            B[f"oready{j}"].arrive()
+            B[f"oready{o}"].arrive()
             e2 += 1
 
     def store():
-        par = 0
+        e2 = 0
         for x, (ps, k, bs, i, n) in enumerate(seq):
             if ps == 0:
                 continue
-            s, j = x % n_stages, x & 1
-            b = B[f"oready{j}"]
-            while (b.done & 1) == ((par >> j) & 1):
-                yield
-            if release_at_readiness:
-                B[f"empty{s}"].arrive()
-            if tile[j] != ("out", x):
-                raise Fail(f"the store read tile {j} holding {tile[j]} at step {x}")
-            tile_rd[j] += 1
+            o = e2 % n_out
+            yield from sim.wait(f"oready{o}", e2 // n_out)
+            if otile[o] != x:
+                raise Fail(f"the store read output tile {o} holding {otile[o]} at step {x}")
+            otile_rd[o] += 1
             read = []
 
-            def rd(x=x, j=j):
-                if tile[j] != ("out", x):
+            def rd(x=x, o=o):
+                if otile[o] != x:
                     raise Fail("a tile changed under its store")
-                tile_rd[j] -= 1
+                otile_rd[o] -= 1
                 read.append(1)
             sim.later(rd)
             while not read:
                 yield
-            par ^= 1 << j
-            if not release_at_readiness:
-                B[f"empty{s}"].arrive()
-            B[f"sfree{j}"].arrive()
+            B[f"ofree{o}"].arrive()
+            e2 += 1
 
     sim.run({"producer": producer(), "converters": converters(), "mma": mma(), "epilogue": epilogue(),
              "store": store()})
@@ -382,10 +404,10 @@ def _schedules(seed, n):
         yield [rng.choice([1, 2, 3, 5, 12, 32]) for _ in range(rng.randint(1, 5))], rng
 
 
-@pytest.mark.parametrize("presplit", [False, True])
-def test_decoder_protocol_holds_on_random_schedules(presplit):
-    for ncs, rng in _schedules(11 + presplit, 150):
-        decoder(ncs, rng, presplit=presplit)
+@pytest.mark.parametrize("n_stages,n_out", [(4, 2), (5, 1)])
+def test_decoder_protocol_holds_on_random_schedules(n_stages, n_out):
+    for ncs, rng in _schedules(11 + n_stages, 150):
+        decoder(ncs, rng, n_stages=n_stages, n_out=n_out)
 
 
 @pytest.mark.parametrize("presplit", [False, True])
@@ -394,9 +416,10 @@ def test_encoder_protocol_holds_on_random_schedules(presplit):
         encoder(ncs, rng, presplit=presplit)
 
 
-def test_releasing_a_second_pass_stage_at_tile_readiness_is_caught():
-    """The earlier decoder released a second-pass stage as soon as its output
-    tile was ready; the model finds a schedule where that breaks."""
+def test_releasing_a_second_pass_stage_at_mma_completion_is_caught():
+    """A second-pass stage still holds the codes that the epilogue adds to the
+    product: released when the MMA completes, its next TMA load can overwrite
+    them before they are read.  The model finds such a schedule."""
     with pytest.raises(Fail):
         for ncs, rng in _schedules(3, 400):
-            decoder(ncs, rng, release_at_readiness=True)
+            decoder(ncs, rng, release_at_mma=True)
