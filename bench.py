@@ -436,13 +436,13 @@ def buffer_set(ops, W, G_all, Gh_all):
 # elements.  Valid only for the kernel source it was taken on (sha256 of the
 # file); otherwise the bench reports traffic as null.
 TRAFFIC = {
-    "decode_whitened": {"read_per_element": 1.447617, "l2_write_per_element": 2.000000,
-                        "dram_write_per_element": 1.145445, "profile": "profiles/whiten_decode_tc_stack8.md"},
-    "encode_whitened": {"read_per_element": 2.936679, "l2_write_per_element": 1.250000,
-                        "dram_write_per_element": 0.229733, "profile": "profiles/whiten_encode_tc_stack8.md"},
+    "decode_whitened": {"read_per_element": 1.482048, "l2_write_per_element": 2.006570,
+                        "dram_write_per_element": 1.148715, "profile": "profiles/whiten_decode_tc_stack8.md"},
+    "encode_whitened": {"read_per_element": 2.949004, "l2_write_per_element": 1.250000,
+                        "dram_write_per_element": 0.298965, "profile": "profiles/whiten_encode_tc_stack8.md"},
 }
 TRAFFIC_SOURCE = ("geometry_aware_fp8_b200/csrc/codec_tc.cu",
-                  "dff908fb504a3cd582883528dae5bcb63e835993d8a3652d1952aa8f8d615f4e")
+                  "4dd3db93aff24074a976fe973fc77adf86a1e11c3075d8f80168cac25f3a2a08")
 
 
 def traffic_for(phase, n_elements, alg_read, alg_write):
