@@ -10,16 +10,20 @@ completed phases differs from P in parity.  The checks:
 
   * every wait passes on the very phase it means (a pass two phases early or
     late is a silent error on the GPU);
-  * every reader of a stage or scratch tile sees the step's own data, and no
-    TMA load or writer overwrites data that is still being read;
+  * every reader of a stage or tile sees the step's own data, and no TMA load
+    or writer overwrites data that is still being read;
   * the run ends (no deadlock).
 
-The decoder's scratch tiles are shared by first-pass steps (widened codes,
-written by the converters) and second-pass steps (output, written by the
-epilogue).  Releasing a second-pass stage as soon as its output tile is ready
-let the converters, which wait for a tile only in first-pass steps, pass a
-tile's wait two phases early; the model finds such a schedule, and the
-kernel releases the stage after the tile's stores have read it instead.
+In the decoder, the converters write a first-pass step's widened codes into
+one of two TMEM A tiles, and the epilogue writes a second-pass step's output
+into shared-memory output tiles; each tile has one writer role and one
+reader role.  A second-pass stage is released by the epilogue once it has
+read the codes; the model catches a release at D3's completion instead,
+where the stage's next TMA load can overwrite codes not yet read.  (An
+earlier layout shared two scratch tiles between the converters and the
+epilogue; there the model found that releasing a second-pass stage as soon
+as its output tile was ready let the converters pass a tile's parity wait
+two phases early.)
 """
 import random
 
