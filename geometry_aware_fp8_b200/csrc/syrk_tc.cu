@@ -11,8 +11,10 @@
 // from X's rows: X[n][i] has i contiguous, so A-operand (M = i) and
 // B-operand (N = j) are MN-major 128-byte-swizzled tiles, one 64-column box
 // per 64 features.  One launch covers a batch of layers (the batched factor
-// refresh): the CTA index picks the layer, its tile and token split.  One CTA
-// per (layer, tile, token split):
+// refresh): a work item is (layer, tile, token split), and one persistent CTA
+// per SM takes every gridDim.x-th item, the load ring and the accumulators
+// running on from one item to the next so that a tile's stores overlap the
+// next tile's MMAs.  Roles:
 //   warp 8     TMA producer (4-stage ring, 48 KB per stage)
 //   warp 9     TMEM allocation and the single-thread MMA issue
 //   warps 0-7  epilogue: TMEM -> registers -> A (j >= i only, mirrored),
@@ -73,7 +75,31 @@ __device__ void tile_of(int t, int d, int* I, int* J2) {
   *J2 = i / 2 + t;
 }
 
-__global__ void __launch_bounds__(THREADS, 1) syrk_tc_kernel(const __grid_constant__ SyrkBatch p) {
+// Work item `it` of a launch: layer, tile (I, J2) and token range.
+struct Item {
+  int l, I, J2, split, nk;
+  int64_t n_begin;
+};
+__device__ Item item_of(const SyrkBatch& p, int it) {
+  Item w;
+  w.split = it % p.splits;
+  const int tile = it / p.splits;
+  int l = 0;
+  while (l + 1 < p.n && tile >= p.L[l + 1].tile_begin) ++l;
+  w.l = l;
+  const SyrkLayer& a = p.L[l];
+  tile_of(tile - a.tile_begin, a.d, &w.I, &w.J2);
+  w.n_begin = (int64_t)w.split * a.rows_per_split;
+  int64_t n_end = w.n_begin + a.rows_per_split;
+  if (n_end > a.N) n_end = a.N;
+  w.nk = n_end > w.n_begin ? (int)((n_end - w.n_begin + BK - 1) / BK) : 0;
+  return w;
+}
+
+// Persistent: CTA b takes items b, b + gridDim.x, ...  The ring's chunk
+// counter and the accumulation-block counter run on across items, so the
+// epilogue's stores of one tile overlap the MMAs of the next.
+__global__ void __launch_bounds__(THREADS, 1) syrk_tc_kernel(const __grid_constant__ SyrkBatch p, int items) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint64_t* full = (uint64_t*)(smem + STAGES * STAGE_BYTES);
@@ -82,23 +108,13 @@ __global__ void __launch_bounds__(THREADS, 1) syrk_tc_kernel(const __grid_consta
   uint64_t* acc_empty = acc_full + 2;    // [2] count 256
   uint32_t* tmem_slot = (uint32_t*)(acc_full + 4);
   __shared__ int failed;
+  __shared__ int failed_layer;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int split = blockIdx.x % p.splits;
-  const int tile = blockIdx.x / p.splits;
-  int l = 0;
-  while (l + 1 < p.n && tile >= p.L[l + 1].tile_begin) ++l;
-  const SyrkLayer& a = p.L[l];
-  const CUtensorMap& tmX = a.tmX;
-  int I, J2;
-  tile_of(tile - a.tile_begin, a.d, &I, &J2);
-  const int64_t n_begin = (int64_t)split * a.rows_per_split;
-  int64_t n_end = n_begin + a.rows_per_split;
-  if (n_end > a.N) n_end = a.N;
-  const int nk = n_end > n_begin ? (int)((n_end - n_begin + BK - 1) / BK) : 0;
 
   if (threadIdx.x == 0) {
     failed = 0;
+    failed_layer = 0;
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
@@ -120,91 +136,126 @@ __global__ void __launch_bounds__(THREADS, 1) syrk_tc_kernel(const __grid_consta
 
   if (warp == 8) {
     if (lane == 0) {
-      tma_prefetch_desc(&tmX);
-      for (int k = 0; k < nk; ++k) {
-        const int s = k % STAGES;
-        const uint32_t ph = (uint32_t)(k / STAGES) & 1u;
-        if (k >= STAGES && !mbar_wait(&empty[s], ph ^ 1u, kWaitLimit)) {
-          failed = 1;
-          break;
-        }
-        uint8_t* sa = smem + s * STAGE_BYTES;
-        uint8_t* sb = sa + A_BYTES;
-        const int y = (int)(n_begin + (int64_t)k * BK);
-        mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
-        tma_load_2d(sa, &tmX, &full[s], I * BM, y);
-        tma_load_2d(sa + BOX_BYTES, &tmX, &full[s], I * BM + 64, y);
+      uint32_t kg = 0;  // chunks loaded so far
+      for (int it = blockIdx.x; it < items && !failed; it += gridDim.x) {
+        const Item w = item_of(p, it);
+        const CUtensorMap& tmX = p.L[w.l].tmX;
+        tma_prefetch_desc(&tmX);
+        for (int k = 0; k < w.nk; ++k, ++kg) {
+          const int s = (int)(kg % STAGES);
+          if (kg >= STAGES && !mbar_wait(&empty[s], ((kg / STAGES) - 1) & 1u, kWaitLimit)) {
+            failed_layer = w.l;
+            failed = 1;
+            break;
+          }
+          uint8_t* sa = smem + s * STAGE_BYTES;
+          uint8_t* sb = sa + A_BYTES;
+          const int y = (int)(w.n_begin + (int64_t)k * BK);
+          mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
+          tma_load_2d(sa, &tmX, &full[s], w.I * BM, y);
+          tma_load_2d(sa + BOX_BYTES, &tmX, &full[s], w.I * BM + 64, y);
 #pragma unroll
-        for (int b = 0; b < 4; ++b) tma_load_2d(sb + b * BOX_BYTES, &tmX, &full[s], J2 * BN + b * 64, y);
+          for (int b = 0; b < 4; ++b) tma_load_2d(sb + b * BOX_BYTES, &tmX, &full[s], w.J2 * BN + b * 64, y);
+        }
       }
     }
   } else if (warp == 9) {
     if (lane == 0) {
-      for (int k = 0; k < nk; ++k) {
-        const int s = k % STAGES;
-        const uint32_t ph = (uint32_t)(k / STAGES) & 1u;
-        const int bk = k / KB, b = bk & 1;
-        if (!mbar_wait(&full[s], ph, kWaitLimit)) {
-          failed = 1;
-          break;
-        }
-        if (k % KB == 0 && bk >= 2 && !mbar_wait(&acc_empty[b], ((bk >> 1) - 1) & 1u, kWaitLimit)) {
-          failed = 1;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t a0 = smem_u32(smem + s * STAGE_BYTES);
-        const uint32_t b0 = a0 + A_BYTES;
+      uint32_t kg = 0, bg = 0;  // chunks and accumulation blocks consumed so far
+      for (int it = blockIdx.x; it < items && !failed; it += gridDim.x) {
+        const Item w = item_of(p, it);
+        for (int k = 0; k < w.nk; ++k, ++kg) {
+          const int s = (int)(kg % STAGES);
+          const uint32_t bgk = bg + (uint32_t)(k / KB);
+          const int b = (int)(bgk & 1u);
+          if (!mbar_wait(&full[s], (kg / STAGES) & 1u, kWaitLimit)) {
+            failed_layer = w.l;
+            failed = 1;
+            break;
+          }
+          if (k % KB == 0 && bgk >= 2 && !mbar_wait(&acc_empty[b], ((bgk >> 1) - 1) & 1u, kWaitLimit)) {
+            failed_layer = w.l;
+            failed = 1;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(smem + s * STAGE_BYTES);
+          const uint32_t b0 = a0 + A_BYTES;
 #pragma unroll
-        for (int kk = 0; kk < BK / 16; ++kk) {
-          // 16 tokens = 16 rows of 128 B; MN groups (64 features) one box apart
-          const uint64_t ad = umma_desc_sw128(a0 + kk * 2048, BOX_BYTES, 1024);
-          const uint64_t bd = umma_desc_sw128(b0 + kk * 2048, BOX_BYTES, 1024);
-          umma_bf16(tbase + b * BN, ad, bd, IDESC, (k % KB > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            // 16 tokens = 16 rows of 128 B; MN groups (64 features) one box apart
+            const uint64_t ad = umma_desc_sw128(a0 + kk * 2048, BOX_BYTES, 1024);
+            const uint64_t bd = umma_desc_sw128(b0 + kk * 2048, BOX_BYTES, 1024);
+            umma_bf16(tbase + b * BN, ad, bd, IDESC, (k % KB > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(&empty[s]);
+          if (k % KB == KB - 1 || k == w.nk - 1) umma_commit(&acc_full[b]);
         }
-        umma_commit(&empty[s]);
-        if (k % KB == KB - 1 || k == nk - 1) umma_commit(&acc_full[b]);
+        bg += (uint32_t)((w.nk + KB - 1) / KB);
       }
     }
   } else {
     // epilogue: warp w owns rows 32*(w%4).. (its TMEM lane quarter) and
     // columns 128*(w/4)..+128 of the tile; blocks are summed in registers
     const int wq = warp & 3, wh = warp >> 2;
-    float sum[128];
+    uint32_t bg = 0;
+    for (int it = blockIdx.x; it < items; it += gridDim.x) {
+      const Item w = item_of(p, it);
+      const SyrkLayer& a = p.L[w.l];
+      float sum[128];
 #pragma unroll
-    for (int t = 0; t < 128; ++t) sum[t] = 0.0f;
-    const int nblk = (nk + KB - 1) / KB;
-    const uint32_t trow = tbase + ((uint32_t)(wq * 32) << 16) + wh * 128;
-    for (int bk = 0; bk < nblk; ++bk) {
-      const int b = bk & 1;
-      if (!mbar_wait(&acc_full[b], (bk >> 1) & 1u, kWaitLimit)) {
-        failed = 1;
-        break;
+      for (int t = 0; t < 128; ++t) sum[t] = 0.0f;
+      const int nblk = (w.nk + KB - 1) / KB;
+      const uint32_t trow = tbase + ((uint32_t)(wq * 32) << 16) + wh * 128;
+      bool stop = false;
+      for (int bk = 0; bk < nblk; ++bk, ++bg) {
+        const int b = (int)(bg & 1u);
+        if (!mbar_wait(&acc_full[b], (bg >> 1) & 1u, kWaitLimit)) {
+          failed_layer = w.l;
+          failed = 1;
+          stop = true;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          uint32_t r[32];
+          tmem_ld32(trow + b * BN + g * 32, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int t = 0; t < 32; ++t) sum[g * 32 + t] += __uint_as_float(r[t]);
+        }
+        tc_fence_before();
+        mbar_arrive(&acc_empty[b]);
       }
-      tc_fence_after();
+      if (stop) break;
+      const int i = w.I * BM + wq * 32 + lane;
+      const int j0 = w.J2 * BN + wh * 128;
+      if (p.splits == 1) {
+        // row i, columns j0 .. j0 + 127 (j >= i, j < d): 16-byte stores where
+        // four columns are all kept; the mirror A[j][i] is coalesced over i
 #pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        uint32_t r[32];
-        tmem_ld32(trow + b * BN + g * 32, r);
-        tmem_wait_ld();
+        for (int t = 0; t < 128; t += 4) {
+          const int j = j0 + t;
+          if (j >= i && j + 3 < a.d) {
+            *reinterpret_cast<float4*>(a.A + (int64_t)i * a.d + j) =
+                make_float4(sum[t] * a.scale, sum[t + 1] * a.scale, sum[t + 2] * a.scale, sum[t + 3] * a.scale);
+          } else {
 #pragma unroll
-        for (int t = 0; t < 32; ++t) sum[g * 32 + t] += __uint_as_float(r[t]);
-      }
-      tc_fence_before();
-      mbar_arrive(&acc_empty[b]);
-    }
-    const int i = I * BM + wq * 32 + lane;
+            for (int u = 0; u < 4; ++u)
+              if (j + u >= i && j + u < a.d) a.A[(int64_t)i * a.d + j + u] = sum[t + u] * a.scale;
+          }
+        }
 #pragma unroll
-    for (int t = 0; t < 128; ++t) {
-      {
-        const int j = J2 * BN + wh * 128 + t;
-        if (j < i || j >= a.d) continue;
-        const float v = sum[t];
-        if (p.splits == 1) {
-          a.A[(int64_t)i * a.d + j] = v * a.scale;
-          if (j != i) a.A[(int64_t)j * a.d + i] = v * a.scale;
-        } else {
-          a.part[(int64_t)split * a.d * a.d + (int64_t)i * a.d + j] = v;
+        for (int t = 0; t < 128; ++t) {
+          const int j = j0 + t;
+          if (j > i && j < a.d) a.A[(int64_t)j * a.d + i] = sum[t] * a.scale;
+        }
+      } else {
+#pragma unroll
+        for (int t = 0; t < 128; ++t) {
+          const int j = j0 + t;
+          if (j >= i && j < a.d) a.part[(int64_t)w.split * a.d * a.d + (int64_t)i * a.d + j] = sum[t];
         }
       }
     }
@@ -212,7 +263,7 @@ __global__ void __launch_bounds__(THREADS, 1) syrk_tc_kernel(const __grid_consta
   tc_fence_before();
   __syncthreads();
   if (warp == 9) tmem_dealloc(tbase, TMEM_COLS);
-  if (threadIdx.x == 0 && failed && a.err) atomicOr(a.err, GIFT_DEV_TIMEOUT);
+  if (threadIdx.x == 0 && failed && p.L[failed_layer].err) atomicOr(p.L[failed_layer].err, GIFT_DEV_TIMEOUT);
 }
 
 unsigned long long g_attr_mask = 0;
@@ -247,7 +298,7 @@ cudaError_t launch_syrk_tc(const void* X, gift_dtype xdt, int64_t N, int d, floa
   a.part = part;
   a.err = err;
   const int items = syrk_tc_tiles(d) * P.splits;
-  syrk_tc_kernel<<<items, THREADS, SMEM_BYTES, s>>>(P);
+  syrk_tc_kernel<<<std::min(items, kNumSMs), THREADS, SMEM_BYTES, s>>>(P, items);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (P.splits > 1) e = launch_syrk_reduce(part, P.splits, d, A, a.scale, s);
@@ -286,7 +337,7 @@ cudaError_t launch_syrk_tc_batch(const SyrkJob* jobs, int n, cudaStream_t s, boo
   }
   P.n = m;
   P.splits = 1;
-  syrk_tc_kernel<<<tiles, THREADS, SMEM_BYTES, s>>>(P);
+  syrk_tc_kernel<<<std::min(tiles, kNumSMs), THREADS, SMEM_BYTES, s>>>(P, tiles);
   return cudaGetLastError();
 }
 
