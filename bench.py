@@ -370,11 +370,10 @@ def staleness_measure(torch, dev):
 
 def refresh_all(ops, W):
     """Factor refresh of every whitened layer in one batched call, then the U
-    split the tensor-core codec loads (gift_split_u, one small launch a layer)."""
+    split the tensor-core codec loads (gift_split_u_many: one launch for all
+    layers of the grouped codec's array)."""
     ops.factor_refresh_many(W["jobs"], len(W["whitened"]), RANK, OVERSAMPLE, ITERS)
-    for w in W["whitened"]:
-        L = w["layer"]
-        ops.split_u(L.U, out=L.U_split)
+    ops.split_u_many(W["packed_wh"], W["n_packed_wh"])
 
 
 PHASES = ("encode_euclid", "encode_whitened", "decode_euclid", "decode_whitened", "error")

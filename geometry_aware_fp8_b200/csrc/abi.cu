@@ -267,6 +267,26 @@ gift_status gift_split_u(const float* U, int64_t d_in, int rank, uint16_t* U_spl
   return cuda_status(launch_split_u(U, d_in, U_split, (cudaStream_t)stream));
 }
 
+gift_status gift_split_u_many(const gift_layer* layers, int n, gift_stream_t stream) {
+  if (n < 0 || (n > 0 && !layers)) return GIFT_ERR_INVALID_ARG;
+  std::vector<const float*> U;
+  std::vector<uint16_t*> out;
+  std::vector<int64_t> d;
+  for (int i = 0; i < n; ++i) {
+    const gift_layer& L = layers[i];
+    if (!L.U_split || L.rank != 32) continue;
+    if (!L.U || L.d_in < 1) return GIFT_ERR_INVALID_ARG;
+    if (!aligned16(L.U) || !aligned16(L.U_split)) return GIFT_ERR_ALIGN;
+    U.push_back(L.U);
+    out.push_back(const_cast<uint16_t*>(L.U_split));
+    d.push_back(L.d_in);
+  }
+  if (U.empty()) return GIFT_OK;
+  gift_status st = device_ok();
+  if (st != GIFT_OK) return st;
+  return cuda_status(launch_split_u_many(U.data(), out.data(), d.data(), (int)U.size(), (cudaStream_t)stream));
+}
+
 gift_status gift_encode_many(const gift_layer* layers, int n, uint32_t* dev_status, gift_stream_t stream) {
   return run_many(layers, n, dev_status, stream, true);
 }

@@ -73,6 +73,8 @@ bool tc_codec_available();
 // and the CTA skips its work and reports GIFT_DEV_TIMEOUT.
 // U (d_in x 32 fp32) -> the [2][d_in][64] split the tensor-core codec loads (see TcLayer::U_split).
 cudaError_t launch_split_u(const float* U, int64_t d_in, uint16_t* U_split, cudaStream_t s);
+cudaError_t launch_split_u_many(const float* const* U, uint16_t* const* U_split, const int64_t* d_in, int n,
+                                cudaStream_t s);
 cudaError_t launch_whiten_encode_tc(const TcLayer* layers, int n, uint32_t* err, cudaStream_t s,
                                     uint32_t stall_polls = 0);
 cudaError_t launch_whiten_decode_tc(const TcLayer* layers, int n, uint32_t* err, cudaStream_t s,

@@ -29,7 +29,8 @@ EXPORTED = ("gift_status_string", "gift_version", "gift_refresh_workspace_size",
             "gift_error_workspace_size", "gift_roundtrip_error", "gift_encode_nvfp4", "gift_decode_nvfp4",
             "gift_codec_split", "gift_whitened_error_workspace_size", "gift_whitened_error",
             "gift_codec_stall_test", "gift_dense_factor_workspace_size", "gift_dense_factor", "gift_dense_split",
-            "gift_dense_encode", "gift_dense_decode", "gift_decode_sum", "gift_split_u")
+            "gift_dense_encode", "gift_dense_decode", "gift_decode_sum", "gift_split_u",
+            "gift_split_u_many")
 DENSE_CHOLESKY, DENSE_INVSQRT = 1, 2
 
 
@@ -81,6 +82,7 @@ def lib() -> ctypes.CDLL:
         L.gift_decode.argtypes = [vp, vp, i64, i64, vp, vp, vp, i32, vp, i32, vp, vp]
         L.gift_encode_many.argtypes = [ctypes.POINTER(Layer), i32, vp, vp]
         L.gift_split_u.argtypes = [vp, i64, i32, vp, vp]
+        L.gift_split_u_many.argtypes = [ctypes.POINTER(Layer), i32, vp]
         L.gift_decode_many.argtypes = [ctypes.POINTER(Layer), i32, vp, vp]
         L.gift_codec_stall_test.argtypes = [ctypes.POINTER(Layer), i32, ctypes.c_uint32, vp, vp]
         L.gift_codec_split.argtypes = [ctypes.POINTER(Layer), i32, i32, ctypes.POINTER(i32)]
@@ -332,6 +334,12 @@ def split_u(U: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None) ->
         out = torch.empty((2, d_in, 64), device=U.device, dtype=torch.int16)
     _check(lib().gift_split_u(_ptr(U), d_in, rank, _ptr(out), _stream(stream)), "gift_split_u")
     return out
+
+
+def split_u_many(packed, n: int, stream=None):
+    """gift_split_u_many over a make_layers() array: every layer with a U_split
+    and rank 32 gets the split of its current U, in one launch."""
+    _check(lib().gift_split_u_many(packed, n, _stream(stream)), "gift_split_u_many")
 
 
 def encode_many(packed, n: int, stream=None, dev_status: Optional[torch.Tensor] = None):

@@ -88,8 +88,8 @@ const char* gift_status_string(gift_status s);
 /* Library version, e.g. 200 for 0.2.0.  GIFT_VERSION is the version this
  * header describes; a caller can compare it with gift_version() at run time
  * (0.2.0: dev_status on every codec call, gift_layer.U_split, gift_split_u,
- * the dense-transform and decode-and-sum calls). */
-#define GIFT_VERSION 200
+ * the dense-transform and decode-and-sum calls; 0.2.1: gift_split_u_many). */
+#define GIFT_VERSION 201
 int gift_version(void);
 
 /* ------------------------------------------------------------------------
@@ -240,6 +240,17 @@ typedef struct {
  * GIFT_ERR_ALIGN, GIFT_ERR_CUDA.
  * ------------------------------------------------------------------------ */
 gift_status gift_split_u(const float* U, int64_t d_in, int rank, uint16_t* U_split, gift_stream_t stream);
+
+/* The same split for every layer of `layers` whose U_split is non-NULL and
+ * rank is 32 (others are skipped), in one launch: after a batched factor
+ * refresh, one call refreshes the splits of a whole grouped codec's layer
+ * array.  Per layer the result is that of gift_split_u (bit-identical).
+ * layers: host array of n descriptors (read during the call only); U and
+ * U_split as for gift_split_u.  n == 0 is a no-op.
+ * Errors: GIFT_ERR_INVALID_ARG (layers NULL with n > 0, n < 0, a U_split
+ * layer with U NULL or d_in < 1), GIFT_ERR_ALIGN, GIFT_ERR_CUDA.  Nothing is
+ * launched when an argument check fails. */
+gift_status gift_split_u_many(const gift_layer* layers, int n, gift_stream_t stream);
 
 /* dev_status (nullable): one word for the whole call, bits as for gift_encode
  * / gift_decode; a TIMEOUT leaves the outputs of every layer undefined. */

@@ -65,6 +65,41 @@ def _args(d_out, d_in, rank, Gd, Ud, lamd, rhod, presplit):
                          U_split=ops.split_u(Ud) if (presplit and rank) else None)
 
 
+def test_split_u_many_matches_split_u_per_layer():
+    """gift_split_u_many writes, in one launch, each U_split layer's
+    gift_split_u result; layers without a U_split or with rank 0 are left
+    alone."""
+    layers, want = [], []
+    rng = np.random.default_rng(80)
+    for i, (d_out, d_in) in enumerate([(256, 512), (300, 1536), (128, 128), (256, 4096), (256, 640)]):
+        # any fp32 matrix will do for the split; columns of unit norm, as U's are
+        Ud = torch.from_numpy((rng.standard_normal((d_in, 32)) / np.sqrt(d_in)).astype(np.float32)).to(DEV)
+        keep = i != 2  # layer 2 carries no U_split
+        sp = torch.full((2, d_in, 64), 0x5A5A, device=DEV, dtype=torch.int16) if keep else None
+        layers.append(ops.LayerArgs(d_out=d_out, d_in=d_in, rank=32, dtype=torch.bfloat16, U=Ud, U_split=sp))
+        want.append(ops.split_u(Ud) if keep else None)
+    eu_split = torch.full((2, 256, 64), 0x1234, device=DEV, dtype=torch.int16)
+    layers.append(ops.LayerArgs(d_out=64, d_in=256, rank=0, dtype=torch.bfloat16, U_split=eu_split))
+    ops.split_u_many(ops.make_layers(layers), len(layers))
+    torch.cuda.synchronize()
+    for L, w in zip(layers, want):
+        if w is not None:
+            assert torch.equal(L.U_split, w)
+    assert bool((eu_split == 0x1234).all())
+
+
+def test_split_u_many_rejects_bad_arguments():
+    L = ops.lib()
+    assert L.gift_split_u_many(None, 0, None) == 0
+    assert L.gift_split_u_many(None, 1, None) == 1
+    U = torch.zeros((512, 32), device=DEV)
+    sp = torch.zeros((2 * 512 * 64 + 8,), device=DEV, dtype=torch.int16)
+    bad = ops.LayerArgs(d_out=128, d_in=512, rank=32, dtype=torch.bfloat16, U=U, lam=torch.zeros((32,), device=DEV),
+                        rho=torch.ones((1,), device=DEV), U_split=sp[1:])  # 2-byte offset: misaligned
+    assert L.gift_split_u_many(ops.make_layers([bad]), 1, None) == 3
+    assert int(sp[1:].abs().sum().item()) == 0  # nothing was launched
+
+
 @pytest.mark.parametrize("shapes", [
     [(300, 1536, 32), (129, 512, 32), (1536, 4096, 32), (200, 1536, 0)],  # many panels: one CTA each
     [(4096, 1536, 32)],                                                   # few panels: a cluster per panel
