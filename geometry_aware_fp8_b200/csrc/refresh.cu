@@ -313,32 +313,35 @@ __global__ void fold_slices_kernel(const __grid_constant__ RefBatch b, int which
 // the partials few (d / 256), so the one-CTA consumers sum little.
 constexpr int kGramRows = 256;
 
+template <int TM>  // outputs per thread and dimension: 16 TM >= m columns of the tile
 __global__ void __launch_bounds__(kRT) gram_partial_kernel(const __grid_constant__ RefBatch bt, int wa, int wb) {
+  constexpr int W = 16 * TM;        // tile columns (48 or 64)
+  constexpr int E = 64 * W / kRT;   // entries of a 64-row tile per thread
+  static_assert(E * kRT == 64 * W, "tile entries per thread");
   const RefLayer& Lr = bt.L[blockIdx.z];
   const int d = Lr.d, m = bt.m;
   if ((int)blockIdx.x >= Lr.parts) return;
   const float* __restrict__ Ya = Lr.buf[wa];
   const float* __restrict__ Yb = Lr.buf[wb];
   double* __restrict__ part = Lr.gram;
-  __shared__ __align__(16) float Sa[64][64];
-  __shared__ __align__(16) float Sb[64][64];
+  __shared__ __align__(16) float Sa[64][W];
+  __shared__ __align__(16) float Sb[64][W];
   const int p = blockIdx.x;
   const int ti = threadIdx.x >> 4, tj = threadIdx.x & 15;
-  double acc[4][4];
+  double acc[TM][TM];
 #pragma unroll
-  for (int a = 0; a < 4; ++a)
+  for (int a = 0; a < TM; ++a)
 #pragma unroll
-    for (int b = 0; b < 4; ++b) acc[a][b] = 0.0;
-  // A thread's 16 entries of each 64 x 64 tile, loaded into registers all at
+    for (int b = 0; b < TM; ++b) acc[a][b] = 0.0;
+  // A thread's E entries of each 64-row tile, loaded into registers all at
   // once (one memory latency per tile), the next tile's while this one is
   // multiplied.
-  static_assert(kRT * 16 == 64 * 64, "tile entries per thread");
-  float ra[16], rb[16];
+  float ra[E], rb[E];
   auto fetch = [&](int r0) {
     const int rows = min(64, d - r0);
 #pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      const int e = threadIdx.x + k * kRT, rr = e >> 6, c = e & 63;
+    for (int k = 0; k < E; ++k) {
+      const int e = threadIdx.x + k * kRT, rr = e / W, c = e % W;
       const bool in = rr < rows && c < m;
       ra[k] = in ? __ldg(Ya + (int64_t)(r0 + rr) * m + c) : 0.0f;
       rb[k] = in ? __ldg(Yb + (int64_t)(r0 + rr) * m + c) : 0.0f;
@@ -349,31 +352,40 @@ __global__ void __launch_bounds__(kRT) gram_partial_kernel(const __grid_constant
   for (int r0 = rbeg; r0 < rend; r0 += 64) {
     __syncthreads();
 #pragma unroll
-    for (int k = 0; k < 16; ++k) {
+    for (int k = 0; k < E; ++k) {
       const int e = threadIdx.x + k * kRT;
-      Sa[e >> 6][e & 63] = ra[k];
-      Sb[e >> 6][e & 63] = rb[k];
+      Sa[e / W][e % W] = ra[k];
+      Sb[e / W][e % W] = rb[k];
     }
     __syncthreads();
     if (r0 + 64 < rend) fetch(r0 + 64);
 #pragma unroll 4
     for (int rr = 0; rr < 64; ++rr) {
-      const float4 va = *reinterpret_cast<const float4*>(&Sa[rr][ti * 4]);
-      const float4 vb = *reinterpret_cast<const float4*>(&Sb[rr][tj * 4]);
-      const double a4[4] = {va.x, va.y, va.z, va.w};
-      const double b4[4] = {vb.x, vb.y, vb.z, vb.w};
+      double a4[TM], b4[TM];
+      if constexpr (TM == 4) {
+        const float4 va = *reinterpret_cast<const float4*>(&Sa[rr][ti * 4]);
+        const float4 vb = *reinterpret_cast<const float4*>(&Sb[rr][tj * 4]);
+        a4[0] = va.x; a4[1] = va.y; a4[2] = va.z; a4[3] = va.w;
+        b4[0] = vb.x; b4[1] = vb.y; b4[2] = vb.z; b4[3] = vb.w;
+      } else {
 #pragma unroll
-      for (int a = 0; a < 4; ++a)
+        for (int a = 0; a < TM; ++a) {
+          a4[a] = Sa[rr][ti * TM + a];
+          b4[a] = Sb[rr][tj * TM + a];
+        }
+      }
 #pragma unroll
-        for (int b = 0; b < 4; ++b) acc[a][b] = fma(a4[a], b4[b], acc[a][b]);
+      for (int a = 0; a < TM; ++a)
+#pragma unroll
+        for (int b = 0; b < TM; ++b) acc[a][b] = fma(a4[a], b4[b], acc[a][b]);
     }
   }
   const int mm = m * m;
 #pragma unroll
-  for (int a = 0; a < 4; ++a)
+  for (int a = 0; a < TM; ++a)
 #pragma unroll
-    for (int b = 0; b < 4; ++b) {
-      const int i = ti * 4 + a, j = tj * 4 + b;
+    for (int b = 0; b < TM; ++b) {
+      const int i = ti * TM + a, j = tj * TM + b;
       if (i < m && j < m) part[(int64_t)p * mm + i * m + j] = acc[a][b];
     }
 }
@@ -906,7 +918,10 @@ cudaError_t launch_refresh_batch(const RefreshPlan* plans, const RefreshIO* io, 
         g_qr(qr_blocks, 1, cnt);
     // one Cholesky-QR pass: dst = src R^{-1} with src^T src = R^T R
     auto cholqr_pass = [&](int src, int dst) {
-      gram_partial_kernel<<<g_gram, kRT, 0, s>>>(B, src, src);
+      if (m <= 48)
+        gram_partial_kernel<3><<<g_gram, kRT, 0, s>>>(B, src, src);
+      else
+        gram_partial_kernel<4><<<g_gram, kRT, 0, s>>>(B, src, src);
       chol_kernel<<<g_one, kST, kCholSmem, s>>>(B);
       qr_apply_kernel<<<g_qr, kRT, kQrSmem, s>>>(B, src, dst);
     };
@@ -957,7 +972,10 @@ cudaError_t launch_refresh_batch(const RefreshPlan* plans, const RefreshIO* io, 
     // R3/R4: Rayleigh-Ritz, lambda, rho, U (fp32 product: the Ritz values
     // need the accuracy the bf16 split would not give)
     skinny_product(false);
-    gram_partial_kernel<<<g_gram, kRT, 0, s>>>(B, kBufQ, kBufY);
+    if (m <= 48)
+      gram_partial_kernel<3><<<g_gram, kRT, 0, s>>>(B, kBufQ, kBufY);
+    else
+      gram_partial_kernel<4><<<g_gram, kRT, 0, s>>>(B, kBufQ, kBufY);
     rr_kernel<<<g_one, kST, kRRSmem, s>>>(B);
     form_u_kernel<<<g_ew, kRT, 0, s>>>(B);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
