@@ -964,10 +964,18 @@ cudaError_t launch_refresh_batch(const RefreshPlan* plans, const RefreshIO* io, 
       cholqr_pass(kBufQ, kBufT);
       cholqr_pass(kBufT, kBufQ);
     }
+    // Each iteration needs only an orthonormal basis of span(A Q): one
+    // Cholesky-QR pass (orthogonal to ~kappa^2 eps in fp64) until the last,
+    // whose basis feeds the Rayleigh-Ritz step and gets the second pass
+    // (Cholesky-QR2, orthogonal to working precision).
     for (int it = 0; it < iters; ++it) {
       skinny_product(tc);
-      cholqr_pass(kBufY, kBufT);  // Cholesky-QR2:
-      cholqr_pass(kBufT, kBufQ);  // two passes
+      if (it + 1 < iters) {
+        cholqr_pass(kBufY, kBufQ);
+      } else {
+        cholqr_pass(kBufY, kBufT);
+        cholqr_pass(kBufT, kBufQ);
+      }
     }
     // R3/R4: Rayleigh-Ritz, lambda, rho, U (fp32 product: the Ritz values
     // need the accuracy the bf16 split would not give)
