@@ -88,6 +88,21 @@ def test_split_u_many_matches_split_u_per_layer():
     assert bool((eu_split == 0x1234).all())
 
 
+def test_split_u_many_over_more_layers_than_one_launch_takes():
+    """520 layers (one launch takes at most 512): every split is that of
+    gift_split_u for its layer."""
+    rng = np.random.default_rng(81)
+    n = 520
+    U = torch.from_numpy((rng.standard_normal((n, 128, 32)) / np.sqrt(128)).astype(np.float32)).to(DEV)
+    S = torch.zeros((n, 2, 128, 64), device=DEV, dtype=torch.int16)
+    layers = [ops.LayerArgs(d_out=128, d_in=128, rank=32, dtype=torch.bfloat16, U=U[i], U_split=S[i]) for i in range(n)]
+    ops.split_u_many(ops.make_layers(layers), n)
+    torch.cuda.synchronize()
+    for i in (0, 1, 511, 512, 519):
+        assert torch.equal(S[i], ops.split_u(U[i]))
+    assert int((S == 0).all(dim=(1, 2, 3)).sum().item()) == 0  # every layer was written
+
+
 def test_split_u_many_rejects_bad_arguments():
     L = ops.lib()
     assert L.gift_split_u_many(None, 0, None) == 0
