@@ -197,19 +197,26 @@ __global__ void split_a_kernel(const __grid_constant__ RefBatch b) {
   }
 }
 
-// Y = A Q (d x d times d x m, m <= 64), fp32 on the CUDA cores.  128 x 16 CW
-// output tiles (CW = 3 for m <= 48, else 4; columns >= m idle), 8 x CW outputs
-// per thread; the k range of a CTA is walked in steps of 16 through two
-// shared-memory buffers, the next step's A and Q values prefetched into
-// registers while the current one is used.  Each output is one fmaf chain in
-// increasing k over its slice; the k range is split into `ns` slices written
-// to Yp[slice] (fixed order), which consumers add in index order.
+// Y = A Q (d x d times d x m, m <= 64), fp32 on the CUDA cores.  128 x 8 CW
+// output tiles (CW = 6 for m <= 48, else 8; columns >= m idle) on 128
+// threads, 8 x CW outputs per thread (two 16-byte A reads and CW / 2 8-byte Q
+// reads of shared memory per 8 CW fmaf: the kernel is bound by shared-memory
+// issue, not by the FMA pipe); the k range of a CTA is walked in steps of 16
+// through two shared-memory buffers, the next step's A and Q values
+// prefetched into registers while the current one is used.  Each output is
+// one fmaf chain in increasing k over its slice; the k range is split into
+// `ns` slices written to Yp[slice] (fixed order), which consumers add in
+// index order.
 constexpr int kSkK = 32;   // k-slice granularity
 constexpr int kSkStep = 16;
+constexpr int kSkThreads = 128;
 
 template <int CW>
-__global__ void __launch_bounds__(kRT) skinny_kernel(const __grid_constant__ RefBatch b, int src, int dst) {
-  constexpr int NC = 16 * CW;  // tile columns
+__global__ void __launch_bounds__(kSkThreads) skinny_kernel(const __grid_constant__ RefBatch b, int src, int dst) {
+  constexpr int NC = 8 * CW;                        // tile columns
+  constexpr int QPT = kSkStep * NC / kSkThreads;    // Q values a thread stages per step
+  static_assert(QPT * kSkThreads == kSkStep * NC, "Q staging");
+  static_assert(CW % 2 == 0, "8-byte Q reads");
   const RefLayer& Lr = b.L[blockIdx.z];
   const int d = Lr.d, m = b.m, kslice = Lr.kslice;
   if ((int)blockIdx.x >= d / 128 || (int)blockIdx.y >= Lr.ns) return;
@@ -221,33 +228,35 @@ __global__ void __launch_bounds__(kRT) skinny_kernel(const __grid_constant__ Ref
   const int row0 = blockIdx.x * 128;
   const int k_begin = blockIdx.y * kslice;
   const int k_end = min(d, k_begin + kslice);
-  const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;  // rows 8 ty.., columns CW tx..
-  // loaders: A rows (t & 127), k (t >> 7) * 8 .. + 7; Q row k = t / (NC / 4), columns 4 (t % (NC / 4)) ..
-  const int ar = threadIdx.x & 127, ak = (threadIdx.x >> 7) * 8;
-  const bool qld = threadIdx.x < kSkStep * NC / 4;
-  const int qk = threadIdx.x / (NC / 4), qc = (threadIdx.x % (NC / 4)) * 4;
+  const int ty = threadIdx.x >> 3, tx = threadIdx.x & 7;  // rows 8 ty.., columns CW tx..
+  // loaders: A row t, k 0 .. 15 of the step; Q row k = t / 8, columns QPT (t % 8) ..
+  const int ar = threadIdx.x;
+  const int qk = threadIdx.x >> 3, qc = (threadIdx.x & 7) * QPT;
   float acc[8][CW];
 #pragma unroll
   for (int a = 0; a < 8; ++a)
 #pragma unroll
     for (int c = 0; c < CW; ++c) acc[a][c] = 0.0f;
-  float4 ra0, ra1, rq;
+  float4 ra[4];
+  float rq[QPT];
   auto fetch = [&](int k0) {
-    const float4* src4 = reinterpret_cast<const float4*>(A + (int64_t)(row0 + ar) * d + k0 + ak);
-    ra0 = __ldg(src4);
-    ra1 = __ldg(src4 + 1);
-    if (qld) {
-      const float* qrow = Q + (int64_t)(k0 + qk) * m;
-      rq.x = qc + 0 < m ? __ldg(qrow + qc + 0) : 0.0f;
-      rq.y = qc + 1 < m ? __ldg(qrow + qc + 1) : 0.0f;
-      rq.z = qc + 2 < m ? __ldg(qrow + qc + 2) : 0.0f;
-      rq.w = qc + 3 < m ? __ldg(qrow + qc + 3) : 0.0f;
-    }
+    const float4* src4 = reinterpret_cast<const float4*>(A + (int64_t)(row0 + ar) * d + k0);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) ra[q] = __ldg(src4 + q);
+    const float* qrow = Q + (int64_t)(k0 + qk) * m;
+#pragma unroll
+    for (int c = 0; c < QPT; ++c) rq[c] = qc + c < m ? __ldg(qrow + qc + c) : 0.0f;
   };
   auto stash = [&](int buf) {
-    As[buf][ak + 0][ar] = ra0.x; As[buf][ak + 1][ar] = ra0.y; As[buf][ak + 2][ar] = ra0.z; As[buf][ak + 3][ar] = ra0.w;
-    As[buf][ak + 4][ar] = ra1.x; As[buf][ak + 5][ar] = ra1.y; As[buf][ak + 6][ar] = ra1.z; As[buf][ak + 7][ar] = ra1.w;
-    if (qld) *reinterpret_cast<float4*>(&Qs[buf][qk][qc]) = rq;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      As[buf][4 * q + 0][ar] = ra[q].x;
+      As[buf][4 * q + 1][ar] = ra[q].y;
+      As[buf][4 * q + 2][ar] = ra[q].z;
+      As[buf][4 * q + 3][ar] = ra[q].w;
+    }
+#pragma unroll
+    for (int c = 0; c < QPT; ++c) Qs[buf][qk][qc + c] = rq[c];
   };
   int buf = 0;
   if (k_begin < k_end) {
@@ -264,15 +273,11 @@ __global__ void __launch_bounds__(kRT) skinny_kernel(const __grid_constant__ Ref
       const float4 a1 = *reinterpret_cast<const float4*>(&As[buf][kk][ty * 8 + 4]);
       const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
       float qv[CW];
-      if constexpr (CW == 4) {
-        const float4 q4 = *reinterpret_cast<const float4*>(&Qs[buf][kk][tx * 4]);
-        qv[0] = q4.x;
-        qv[1] = q4.y;
-        qv[2] = q4.z;
-        qv[3] = q4.w;
-      } else {
 #pragma unroll
-        for (int c = 0; c < CW; ++c) qv[c] = Qs[buf][kk][tx * CW + c];
+      for (int c = 0; c < CW; c += 2) {
+        const float2 q2 = *reinterpret_cast<const float2*>(&Qs[buf][kk][tx * CW + c]);
+        qv[c] = q2.x;
+        qv[c + 1] = q2.y;
       }
 #pragma unroll
       for (int a = 0; a < 8; ++a)
@@ -949,9 +954,9 @@ cudaError_t launch_refresh_batch(const RefreshPlan* plans, const RefreshIO* io, 
         for (int l = 0; l < cnt; ++l) B.L[l].ns = plans[base + l].skinny_slices;
       } else {
         if (m <= 48)
-          skinny_kernel<3><<<g_skinny, kRT, 0, s>>>(B, kBufQ, kBufY);
+          skinny_kernel<6><<<g_skinny, kSkThreads, 0, s>>>(B, kBufQ, kBufY);
         else
-          skinny_kernel<4><<<g_skinny, kRT, 0, s>>>(B, kBufQ, kBufY);
+          skinny_kernel<8><<<g_skinny, kSkThreads, 0, s>>>(B, kBufQ, kBufY);
         if (nsmax > 1) fold_slices_kernel<<<g_ew, kRT, 0, s>>>(B, kBufY);
       }
     };
