@@ -727,13 +727,19 @@ __global__ void __launch_bounds__(kST) rr_kernel(const __grid_constant__ RefBatc
       Vn = t;
     }
   }
-  // sort eigenvalues descending (ties by index)
+  // sort eigenvalues descending (ties by index).  A NaN sorts as -inf, so the
+  // comparison is a total order and `order` is a permutation whatever B holds
+  // (a non-finite input gives NaN eigenvalues, reported as GIFT_DEV_NONFINITE;
+  // with NaN compared as is, every index took rank 0 and `order` kept stale
+  // shared-memory contents, which the gathers below then used as indices).
   if (threadIdx.x < m) {
     const int i = threadIdx.x;
-    const double ti = B[i * ld + i];
+    const double bi = B[i * ld + i];
+    const double ti = isnan(bi) ? -INFINITY : bi;
     int rank_i = 0;
     for (int j = 0; j < m; ++j) {
-      const double tj = B[j * ld + j];
+      const double bj = B[j * ld + j];
+      const double tj = isnan(bj) ? -INFINITY : bj;
       if (tj > ti || (tj == ti && j < i)) ++rank_i;
     }
     order[rank_i] = i;
